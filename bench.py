@@ -1,0 +1,435 @@
+"""Benchmark: causal attention forward + backward through libcattn's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {cattn,reference}]
+                    [--workload INDEX]
+
+One step = one pass of the whole hot path over one batch: attn_fwd (O, LSE)
+then attn_bwd (Delta preprocess, main backward, dQ convert) on the GPT-2
+124M attention layer (B=16, H=12, T=1024, D=64, bf16) unless --workload
+picks another of the five workloads.  Prints one JSON line on rank 0.
+
+Throughput uses the causal FLOP convention: forward = 2*B*H*T^2*D (half of
+the dense 4*B*H*T^2*D), backward = 2.5 x forward, step = 3.5 x forward.
+
+L2 (126 MB): every step's working set (about 280 MB at the headline
+workload) exceeds L2, and steps rotate over 3 input sets, so each step's
+inputs were last touched two steps (>500 MB of traffic) earlier.
+
+N > 1 (torchrun): the path does not shard inside one problem and needs no
+collective, so every rank runs its own full replica of the workload
+(weak scaling); NCCL is used only for the barrier and the max-over-ranks
+timing.
+
+--impl reference: the fp64 CPU oracle (the correctness reference; there is
+no other implementation to compare with) timed on the host cores over a
+bounded sample of heads of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from workloads import WORKLOADS, HEADLINE, seed_for, workload_inputs  # noqa: E402
+
+METRIC = "causal attn fwd+bwd TFLOP/s at GPT-2 124M shape; % of B200 BF16 peak"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+CSRC = os.path.join(ROOT, "causal_self_attention_flash_b200", "csrc")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+N_SETS = 3
+
+
+def fwd_flops(w) -> float:
+    return 2.0 * w.B * w.H * w.T * w.T * w.D
+
+
+def step_flops(w) -> float:
+    return 3.5 * fwd_flops(w)
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(CSRC)):
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(f.encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def kernel_algorithmic(w, name):
+    """(amount per launch, unit, bound) for a kernel of the step."""
+    bhtd = w.B * w.H * w.T * w.D
+    bht = w.B * w.H * w.T
+    tpad = (w.T + 127) // 128 * 128
+    if name == "fwd_kernel":
+        return fwd_flops(w), "flop", "tensor"
+    if name == "bwd_kernel":
+        return 2.5 * fwd_flops(w), "flop", "tensor"
+    if name == "bwd_pre_kernel":
+        # read O, dO (bf16), LSE; write Delta, LSE*log2e (padded); zero dQ acc
+        return 2 * bhtd * 2 + bht * 4 + 2 * w.B * w.H * tpad * 4 + bhtd * 4, "byte", "hbm"
+    if name == "dq_convert_kernel":
+        return bhtd * 4 + bhtd * 2, "byte", "hbm"
+    raise KeyError(name)
+
+
+class ClockSampler:
+    """NVML sampler of SM clock and throttle reasons during a region."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.ok = False
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # noqa: BLE001  (no NVML: clocks reported as unknown)
+            self.ok = False
+
+    def sample(self):
+        if not self.ok:
+            return
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for name, bit in self.REASONS.items():
+                if r & bit:
+                    self.reasons.add(name)
+        except Exception:  # noqa: BLE001
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            self.sample()
+            time.sleep(self.period)
+
+    def __enter__(self):
+        self.sample()
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        self.t.join()
+        self.sample()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        reasons = sorted(self.reasons - {"gpu_idle"})
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, x: float) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [i.get("num_threads") for i in info if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:  # noqa: BLE001
+        return 1
+
+
+def cpu_oracle_rate(w, index, budget_s=15.0, max_heads=None):
+    """Time the fp64 oracle (fwd + bwd) on whole heads of the workload until
+    about budget_s of CPU work; returns (TFLOP/s, heads, seconds)."""
+    import oracle
+    from workloads import as_f64, bf16_inputs, sample_heads
+    heads = sample_heads(w.BH, max_heads or w.BH, seed=seed_for(index) + 77)
+    per_head = step_flops(w) / w.BH
+    done, t_total = 0, 0.0
+    for f in heads:
+        b, h = divmod(f, w.H)
+        # draw this head's inputs on their own (the oracle sees the same
+        # distribution as the workload; values need not match the GPU's)
+        q, k, v, do = (as_f64(t) for t in bf16_inputs(1, 1, w.T, w.D, seed_for(index) * 1000 + f,
+                                                       w.qk_std))
+        t0 = time.perf_counter()
+        oracle.attention_forward(q, k, v, w.scale)
+        oracle.attention_backward(q, k, v, do, w.scale)
+        t_total += time.perf_counter() - t0
+        done += 1
+        if t_total >= budget_s:
+            break
+    return per_head * done / t_total / 1e12, done, t_total
+
+
+def run_reference(args, w, index, world, rank):
+    if rank != 0:
+        return
+    # one step = one bounded sample of heads; K steps after W warm-ups
+    per_step = max(1, min(w.BH, int(os.environ.get("CATTN_REF_HEADS", "4"))))
+    import oracle
+    from workloads import as_f64, bf16_inputs
+    heads = [bf16_inputs(1, 1, w.T, w.D, seed_for(index) * 1000 + i, w.qk_std)
+             for i in range(per_step)]
+    heads = [[as_f64(t) for t in hd] for hd in heads]
+
+    def step():
+        for q, k, v, do in heads:
+            oracle.attention_forward(q, k, v, w.scale)
+            oracle.attention_backward(q, k, v, do, w.scale)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    flops = step_flops(w) / w.BH * per_step * args.steps
+    value = flops / dt / 1e12
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "D": w.D,
+                   "parallelism": "replicas", "reference": "fp64 CPU oracle"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{per_step} of {w.BH} heads per step, fwd+bwd, fp64"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_cattn(args, w, index, world, rank, local):
+    import causal_self_attention_flash_b200 as cattn
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    q0, k0, v0, do0 = workload_inputs(index)
+    sets = []
+    for s in range(N_SETS):
+        # distinct buffers per set (same values: the work is identical)
+        qd, kd, vd, dod = (t.to(dev) for t in (q0, k0, v0, do0))
+        o = torch.empty_like(qd)
+        lse = torch.empty(w.B, w.H, w.T, dtype=torch.float32, device=dev)
+        dq, dk, dv = (torch.empty_like(qd) for _ in range(3))
+        ws = torch.empty(cattn.attn_bwd_workspace_bytes(w.B, w.H, w.T, w.D), dtype=torch.uint8,
+                         device=dev)
+        sets.append((qd, kd, vd, dod, o, lse, dq, dk, dv, ws))
+
+    def step(i):
+        qd, kd, vd, dod, o, lse, dq, dk, dv, ws = sets[i % N_SETS]
+        cattn.attn_fwd(qd, kd, vd, w.scale, o=o, lse=lse, stream=stream)
+        cattn.attn_bwd(qd, kd, vd, o, lse, dod, w.scale, dq=dq, dk=dk, dv=dv, workspace=ws,
+                       stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert cattn.cattn_get_device_status() == cattn.OK
+
+    # ---- timed region: exactly K steps
+    sampler = ClockSampler(local)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with sampler:
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = e0.elapsed_time(e1)
+    ms_max = max_over_ranks(world, ms)
+    status = cattn.cattn_get_device_status()
+    total_flops = step_flops(w) * args.steps * world
+    value = total_flops / (ms_max / 1e3) / 1e12
+
+    # ---- per-kernel device time (same K steps again, events per launch)
+    cattn.cattn_timing_enable(True)
+    cattn.cattn_timing_read()
+    for i in range(args.steps):
+        step(i)
+    torch.cuda.synchronize()
+    ktimes = cattn.cattn_timing_read()
+    cattn.cattn_timing_enable(False)
+    total_k = sum(t for t, _ in ktimes.values()) or 1.0
+    dom = max(ktimes, key=lambda n: ktimes[n][0])
+    amount, unit, bound = kernel_algorithmic(w, dom)
+    per_launch_ms = ktimes[dom][0] / max(ktimes[dom][1], 1)
+    peaks, peak_src = load_peaks()
+    if bound == "tensor":
+        achieved = amount / (per_launch_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops"]
+        r_unit = "TFLOP/s"
+    else:
+        achieved = amount / (per_launch_ms / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        r_unit = "GB/s"
+    traffic = None
+    try:
+        with open(TRAFFIC_FILE) as f:
+            tr = json.load(f)
+        ent = tr.get(dom, {})
+        if ent.get("source_hash") == source_hash() and ent.get("workload") == w.name:
+            traffic = ent.get("bytes_per_launch")
+    except (OSError, ValueError):
+        pass
+
+    # ---- end to end: pinned host buffers -> device -> fwd+bwd -> host
+    host_in = [t.pin_memory() for t in (q0, k0, v0, do0)]
+    host_out = [torch.empty(w.B, w.H, w.T, w.D, dtype=torch.bfloat16).pin_memory()
+                for _ in range(4)] + [torch.empty(w.B, w.H, w.T, dtype=torch.float32).pin_memory()]
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+    def e2e_step(i):
+        qd, kd, vd, dod, o, lse, dq, dk, dv, ws = sets[i % N_SETS]
+        for dst, src in zip((qd, kd, vd, dod), host_in):
+            dst.copy_(src, non_blocking=True)
+        step(i)
+        for dst, src in zip(host_out, (o, dq, dk, dv, lse)):
+            dst.copy_(src, non_blocking=True)
+
+    for i in range(min(args.warmup, 3)):
+        e2e_step(i)
+    barrier(world)
+    torch.cuda.synchronize()
+    e2 = torch.cuda.Event(enable_timing=True)
+    e3 = torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(world, e2.elapsed_time(e3))
+    e2e_value = total_flops / (e2e_ms / 1e3) / 1e12
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, nheads, secs = cpu_oracle_rate(w, index, budget_s=args.cpu_budget)
+        cpu = {"value": rate, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{nheads} of {w.BH} heads, fwd+bwd in fp64 ({secs:.1f} s)"}
+
+    if rank == 0:
+        clocks = sampler.summary()
+        pct = value / world / peaks["bf16_tflops"] * 100.0
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "D": w.D,
+                       "global_batch": w.B * world, "seq_len": w.T,
+                       "parallelism": f"replicas x{world}",
+                       "l2": f"{N_SETS} rotating input sets, step working set > L2"},
+            "pct_of_peak": pct,
+            "peak_source": f"{peak_src} bf16 {peaks['bf16_tflops']} TFLOP/s (burst)",
+            "fwd_tflops": fwd_flops(w) / (ktimes["fwd_kernel"][0] / max(ktimes["fwd_kernel"][1], 1)
+                                          / 1e3) / 1e12 if ktimes["fwd_kernel"][1] else None,
+            "kernels": {n: {"ms_per_launch": t / c if c else None, "launches": c,
+                            "share": t / total_k} for n, (t, c) in ktimes.items()},
+            "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak,
+                         "unit": r_unit, "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": peak_src,
+                         "algorithmic_per_launch": amount, "algorithmic_unit": unit},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks,
+            "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="cattn", choices=["cattn", "reference"])
+    ap.add_argument("--workload", type=int, default=HEADLINE)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, w, args.workload, int(os.environ.get("WORLD_SIZE", "1")), rank)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        run_cattn(args, w, args.workload, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

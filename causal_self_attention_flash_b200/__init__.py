@@ -1,0 +1,166 @@
+"""libcattn: fused causal multi-head self-attention for B200 (sm_100a).
+
+Python entry points with the same names as the C ABI (include/cattn.h).
+They take torch CUDA tensors, allocate outputs with torch when none are
+given, pass raw device pointers and the current CUDA stream to the library
+and raise CattnError on a non-zero status.  Nothing here computes: torch
+only provides device memory and streams.
+
+Layout: q, k, v, o, do, dq, dk, dv are bf16 (B, H, T, D) contiguous; lse
+and delta are fp32 (B, H, T).
+"""
+
+from __future__ import annotations
+
+import math
+
+import torch
+
+from ._binding import (ERR_CUDA, ERR_INVALID_ARG, ERR_TIMEOUT,
+                       ERR_UNSUPPORTED, LIB, LIB_PATH, OK, CattnError)
+
+__all__ = [
+    "attn_fwd", "attn_bwd", "attn_bwd_preprocess", "attn_bwd_workspace_bytes",
+    "cattn_get_device_status", "cattn_set_wait_timeout_us",
+    "cattn_selftest_wait_timeout", "cattn_status_string", "cattn_version",
+    "cattn_timing_enable", "cattn_timing_read", "KERNEL_NAMES",
+    "CausalAttention", "CattnError", "LIB", "LIB_PATH",
+    "OK", "ERR_INVALID_ARG", "ERR_UNSUPPORTED", "ERR_CUDA", "ERR_TIMEOUT",
+]
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(name, st):
+    if st != OK:
+        raise CattnError(name, st)
+
+
+def _shape(q):
+    if q.dim() != 4:
+        raise ValueError("expected a (B, H, T, D) tensor")
+    return tuple(int(x) for x in q.shape)
+
+
+def _want(t, like, dtype, shape):
+    if t is None:
+        return torch.empty(shape, dtype=dtype, device=like.device)
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"output must be contiguous {dtype} of shape {shape}")
+    return t
+
+
+def _inputs(*ts):
+    for t in ts:
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous bf16 CUDA tensors")
+
+
+def attn_fwd(q, k, v, scale=None, o=None, lse=None, stream=None):
+    """(o, lse) = causal attention of bf16 (B,H,T,D) q, k, v."""
+    _inputs(q, k, v)
+    B, H, T, D = _shape(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    o = _want(o, q, torch.bfloat16, (B, H, T, D))
+    lse = _want(lse, q, torch.float32, (B, H, T))
+    st = LIB.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), float(scale), B, H, T, D,
+                      o.data_ptr(), lse.data_ptr(), _stream(stream))
+    _check("attn_fwd", st)
+    return o, lse
+
+
+def attn_bwd_workspace_bytes(B, H, T, D):
+    return int(LIB.attn_bwd_workspace_bytes(B, H, T, D))
+
+
+def attn_bwd_preprocess(o, do, delta=None, stream=None):
+    """delta = rowsum(do * o), fp32 (B,H,T)."""
+    _inputs(o, do)
+    B, H, T, D = _shape(o)
+    delta = _want(delta, o, torch.float32, (B, H, T))
+    st = LIB.attn_bwd_preprocess(o.data_ptr(), do.data_ptr(), B, H, T, D, delta.data_ptr(),
+                                 _stream(stream))
+    _check("attn_bwd_preprocess", st)
+    return delta
+
+
+def attn_bwd(q, k, v, o, lse, do, scale=None, dq=None, dk=None, dv=None,
+             workspace=None, stream=None):
+    """(dq, dk, dv) of causal attention; workspace allocated with torch if
+    not given (a uint8 CUDA tensor of attn_bwd_workspace_bytes bytes)."""
+    _inputs(q, k, v, o, do)
+    B, H, T, D = _shape(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous fp32 (B, H, T)")
+    dq = _want(dq, q, torch.bfloat16, (B, H, T, D))
+    dk = _want(dk, q, torch.bfloat16, (B, H, T, D))
+    dv = _want(dv, q, torch.bfloat16, (B, H, T, D))
+    need = attn_bwd_workspace_bytes(B, H, T, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = LIB.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                      do.data_ptr(), float(scale), B, H, T, D, dq.data_ptr(), dk.data_ptr(),
+                      dv.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream))
+    _check("attn_bwd", st)
+    return dq, dk, dv
+
+
+def cattn_get_device_status(clear=False, stream=None):
+    return int(LIB.cattn_get_device_status(1 if clear else 0, _stream(stream)))
+
+
+def cattn_set_wait_timeout_us(us: int):
+    LIB.cattn_set_wait_timeout_us(int(us))
+
+
+def cattn_selftest_wait_timeout(timeout_us: int, stream=None):
+    return int(LIB.cattn_selftest_wait_timeout(int(timeout_us), _stream(stream)))
+
+
+KERNEL_NAMES = ("fwd_kernel", "bwd_pre_kernel", "bwd_kernel", "dq_convert_kernel")
+
+
+def cattn_timing_enable(enable: bool = True):
+    LIB.cattn_timing_enable(1 if enable else 0)
+
+
+def cattn_timing_read():
+    """{kernel name: (total ms, launches)} since the last read."""
+    import ctypes
+    n = len(KERNEL_NAMES)
+    ms = (ctypes.c_float * n)()
+    cnt = (ctypes.c_int * n)()
+    _check("cattn_timing_read", LIB.cattn_timing_read(ms, cnt, n))
+    return {KERNEL_NAMES[i]: (float(ms[i]), int(cnt[i])) for i in range(n)}
+
+
+def cattn_status_string(st: int) -> str:
+    return LIB.cattn_status_string(int(st)).decode()
+
+
+def cattn_version() -> int:
+    return int(LIB.cattn_version())
+
+
+class CausalAttention(torch.autograd.Function):
+    """autograd wrapper: forward = attn_fwd, backward = attn_bwd."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, scale=None):
+        o, lse = attn_fwd(q, k, v, scale)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.scale = scale
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv = attn_bwd(q, k, v, o, lse, do.contiguous(), ctx.scale)
+        return dq, dk, dv, None

@@ -1,0 +1,64 @@
+"""ctypes binding of libcattn's C ABI (declared in include/cattn.h).
+
+Argument marshalling only: every step of the computation runs in the
+library's CUDA kernels.  There is no fallback; if the shared library is
+missing, importing this module raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libcattn.so")
+
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_UNSUPPORTED = 2
+ERR_CUDA = 3
+ERR_TIMEOUT = 4
+
+STATUS_NAMES = {OK: "CATTN_OK", ERR_INVALID_ARG: "CATTN_ERR_INVALID_ARG",
+                ERR_UNSUPPORTED: "CATTN_ERR_UNSUPPORTED", ERR_CUDA: "CATTN_ERR_CUDA",
+                ERR_TIMEOUT: "CATTN_ERR_TIMEOUT"}
+
+# name -> (restype, argtypes), mirroring include/cattn.h
+_vp, _i, _f, _sz, _u32 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_float,
+                          ctypes.c_size_t, ctypes.c_uint32)
+SIGNATURES = {
+    "attn_fwd": (_i, [_vp, _vp, _vp, _f, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "attn_bwd_workspace_bytes": (_sz, [_i, _i, _i, _i]),
+    "attn_bwd_preprocess": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp]),
+    "attn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _f, _i, _i, _i, _i,
+                      _vp, _vp, _vp, _vp, _sz, _vp]),
+    "cattn_get_device_status": (_i, [_i, _vp]),
+    "cattn_set_wait_timeout_us": (None, [_u32]),
+    "cattn_selftest_wait_timeout": (_i, [_u32, _vp]),
+    "cattn_timing_enable": (None, [_i]),
+    "cattn_timing_read": (_i, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int), _i]),
+    "cattn_status_string": (ctypes.c_char_p, [_i]),
+    "cattn_version": (_i, []),
+}
+
+
+class CattnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(
+            f"libcattn.so not found at {path}; build it with "
+            "`python causal_self_attention_flash_b200/build.py`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+LIB = load()

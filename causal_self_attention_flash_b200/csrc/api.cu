@@ -1,0 +1,486 @@
+// C ABI of libcattn: argument checks, TMA tensor maps, launches.
+// The operations are declared and documented in include/cattn.h.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+#include <vector>
+
+#include "cattn.h"
+#include "bwd.cuh"
+#include "fwd.cuh"
+
+namespace cattn {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
+uint64_t g_timeout_ns = kDefaultTimeoutNs;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_mu;
+EncodeTiledFn g_encode = nullptr;
+int g_dev_ok[kMaxDevices];           // 0 unknown, 1 sm_100, -1 other
+unsigned g_attr_done[kMaxDevices];   // bit per kernel instance
+
+cattn_status init_encode() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode) return CATTN_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr) {
+    cudaGetLastError();
+    return CATTN_ERR_CUDA;
+  }
+  g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  return CATTN_OK;
+}
+
+cattn_status check_device(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return CATTN_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return CATTN_ERR_UNSUPPORTED;
+  if (g_dev_ok[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return CATTN_ERR_CUDA;
+    }
+    g_dev_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  if (g_dev_ok[dev] != 1) return CATTN_ERR_UNSUPPORTED;
+  *dev_out = dev;
+  return init_encode();
+}
+
+// Set the dynamic shared-memory limit of a kernel once per device.
+template <typename K>
+cattn_status ensure_smem(int dev, unsigned bit, K kernel, int bytes) {
+  if (g_attr_done[dev] & (1u << bit)) return CATTN_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return CATTN_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_attr_done[dev] |= 1u << bit;
+  return CATTN_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool d_supported(int D) { return D == 16 || D == 32 || D == 64 || D == 128; }
+
+// Common shape checks. Returns CATTN_OK, or INVALID_ARG / UNSUPPORTED.
+cattn_status check_shape(int B, int H, int T, int D) {
+  if (B < 0 || H < 0 || T < 0 || D < 0) return CATTN_ERR_INVALID_ARG;
+  if (!d_supported(D)) return CATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H > 0x7fffffffLL) return CATTN_ERR_INVALID_ARG;
+  if (T > (1 << 20)) return CATTN_ERR_INVALID_ARG;
+  return CATTN_OK;
+}
+
+bool empty_shape(int B, int H, int T) { return B == 0 || H == 0 || T == 0; }
+
+// 3-D tensor map over a contiguous (BH, T, D) tensor: x = d, y = t, z = head.
+cattn_status make_tmap(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int elem_bytes,
+                       int D, int T, long long BH, int box_x, int box_y) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(T),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * elem_bytes,
+                                 static_cast<cuuint64_t>(D) * T * elem_bytes};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_x), static_cast<cuuint32_t>(box_y), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const int row_bytes = box_x * elem_bytes;
+  CUtensorMapSwizzle sw = row_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                          : row_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                            : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUresult r = g_encode(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CATTN_OK : CATTN_ERR_CUDA;
+}
+
+cattn_status make_bf16_map(CUtensorMap* m, const void* ptr, int D, int T, long long BH) {
+  const int cb = D < 64 ? D : 64;
+  return make_tmap(m, ptr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, T, BH, cb, 128);
+}
+
+cattn_status launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? CATTN_OK : CATTN_ERR_CUDA;
+}
+
+int grid_for(size_t work_items, int per_block) {
+  size_t g = (work_items + per_block - 1) / per_block;
+  const size_t cap = 148 * 16;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return static_cast<int>(g);
+}
+
+// ------------------------------------------------------------ kernel timer
+// Optional CUDA-event timing of each launch, on the launching stream (a
+// benchmarking aid; off by default, and then it costs nothing).
+
+enum KernelId { K_FWD = 0, K_BWD_PRE = 1, K_BWD_MAIN = 2, K_DQ_CONVERT = 3, K_COUNT = 4 };
+
+bool g_timing = false;
+struct TimingRec {
+  cudaEvent_t a, b;
+  int kernel;
+};
+std::vector<TimingRec> g_recs;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return e;
+}
+
+struct LaunchTimer {
+  cudaEvent_t a = nullptr, b = nullptr;
+  cudaStream_t s;
+  int kernel;
+  LaunchTimer(int k, cudaStream_t st) : s(st), kernel(k) {
+    if (!g_timing) return;
+    std::lock_guard<std::mutex> lk(g_mu);
+    a = take_event();
+    b = take_event();
+    if (a) cudaEventRecord(a, s);
+  }
+  ~LaunchTimer() {
+    if (!g_timing || !a || !b) return;
+    cudaEventRecord(b, s);
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_recs.push_back({a, b, kernel});
+  }
+};
+
+// ------------------------------------------------------------------ forward
+
+template <int D>
+cattn_status fwd_impl(int dev, const void* q, const void* k, const void* v, float scale, int BH,
+                      int T, void* o, float* lse, cudaStream_t s) {
+  using C = FwdCfg<D>;
+  cattn_status st = ensure_smem(dev, 0 + (D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3),
+                                fwd_kernel<D>, C::SMEM_BYTES);
+  if (st != CATTN_OK) return st;
+  CUtensorMap mq, mk, mv, mo;
+  if ((st = make_bf16_map(&mq, q, D, T, BH)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mk, k, D, T, BH)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mv, v, D, T, BH)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mo, o, D, T, BH)) != CATTN_OK) return st;
+  FwdParams p;
+  p.lse = lse;
+  p.T = T;
+  p.n_qtiles = (T + 127) / 128;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_timeout_ns;
+  dim3 grid(BH, p.n_qtiles);
+  {
+    LaunchTimer t(K_FWD, s);
+    fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, p);
+  }
+  return launch_status();
+}
+
+// ----------------------------------------------------------------- backward
+
+struct WsLayout {
+  size_t dq_off, lse2_off, delta_off, total;
+  int T_pad;
+};
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+WsLayout ws_layout(long long BH, int T, int D) {
+  WsLayout L;
+  L.T_pad = (T + 127) / 128 * 128;
+  L.dq_off = 0;
+  L.lse2_off = round256(static_cast<size_t>(BH) * T * D * 4);
+  L.delta_off = L.lse2_off + round256(static_cast<size_t>(BH) * L.T_pad * 4);
+  L.total = L.delta_off + round256(static_cast<size_t>(BH) * L.T_pad * 4);
+  return L;
+}
+
+template <int D>
+cattn_status pre_impl(const void* o, const void* dout, const float* lse, float* delta,
+                      float* lse2, float4* zero, size_t zero_n4, long long BH, int T,
+                      int row_stride, cudaStream_t s) {
+  PreParams p;
+  p.o = static_cast<const __nv_bfloat16*>(o);
+  p.dout = static_cast<const __nv_bfloat16*>(dout);
+  p.lse = lse;
+  p.delta = delta;
+  p.lse2 = lse2;
+  p.zero = zero;
+  p.zero_n4 = zero_n4;
+  p.T = T;
+  p.row_stride = row_stride;
+  p.n_rows = BH * row_stride;
+  constexpr int rows_per_block = 256 / (D / 8);
+  const size_t work = static_cast<size_t>(p.n_rows);
+  {
+    LaunchTimer t(K_BWD_PRE, s);
+    bwd_pre_kernel<D><<<grid_for(work > zero_n4 / 64 ? work : zero_n4 / 64, rows_per_block), 256,
+                        0, s>>>(p);
+  }
+  return launch_status();
+}
+
+template <int D>
+cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, const void* o,
+                      const float* lse, const void* dout, float scale, int BH, int T, void* dq,
+                      void* dk, void* dv, void* ws, cudaStream_t s) {
+  using C = BwdCfg<D>;
+  cattn_status st = ensure_smem(dev, 4 + (D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3),
+                                bwd_kernel<D>, C::SMEM_BYTES);
+  if (st != CATTN_OK) return st;
+  const WsLayout L = ws_layout(BH, T, D);
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  float* dq_acc = reinterpret_cast<float*>(wb + L.dq_off);
+  float* lse2 = reinterpret_cast<float*>(wb + L.lse2_off);
+  float* delta = reinterpret_cast<float*>(wb + L.delta_off);
+  const size_t n_dq = static_cast<size_t>(BH) * T * D;
+
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv, mdq;
+  if ((st = make_bf16_map(&mq, q, D, T, BH)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mk, k, D, T, BH)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mv, v, D, T, BH)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mdo, dout, D, T, BH)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mdk, dk, D, T, BH)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mdv, dv, D, T, BH)) != CATTN_OK) return st;
+  if ((st = make_tmap(&mdq, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, T, BH, C::CBQ, 128)) !=
+      CATTN_OK)
+    return st;
+
+  st = pre_impl<D>(o, dout, lse, delta, lse2, reinterpret_cast<float4*>(dq_acc), n_dq / 4, BH, T,
+                   L.T_pad, s);
+  if (st != CATTN_OK) return st;
+
+  BwdParams p;
+  p.lse2 = lse2;
+  p.delta = delta;
+  p.T = T;
+  p.T_pad = L.T_pad;
+  p.n_tiles = L.T_pad / 128;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_timeout_ns;
+  dim3 grid(BH, p.n_tiles);
+  {
+    LaunchTimer t(K_BWD_MAIN, s);
+    bwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mdo, mdk, mdv, mdq, p);
+  }
+  if ((st = launch_status()) != CATTN_OK) return st;
+  {
+    LaunchTimer t(K_DQ_CONVERT, s);
+    dq_convert_kernel<<<grid_for(n_dq / 8, 256), 256, 0, s>>>(
+        reinterpret_cast<const float4*>(dq_acc), static_cast<uint4*>(dq), n_dq / 8, scale);
+  }
+  return launch_status();
+}
+
+// ---------------------------------------------------------- hang-guard test
+
+__global__ void selftest_wait_kernel(uint64_t timeout_ns) {
+  __shared__ __align__(8) uint64_t mbar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&mbar), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    WaitCtx w{timeout_ns, &abort_flag, 15u};
+    wait1(w, smem_u32(&mbar), 0, 1);  // nothing ever arrives
+  }
+  __syncthreads();
+}
+
+}  // namespace
+}  // namespace cattn
+
+using namespace cattn;
+
+extern "C" {
+
+cattn_status attn_fwd(const void* q, const void* k, const void* v, float scale, int B, int H,
+                      int T, int D, void* o, float* lse, void* stream) {
+  cattn_status st = check_shape(B, H, T, D);
+  if (st != CATTN_OK) return st;
+  if (!(scale > 0.f) || !isfinite(scale)) return CATTN_ERR_INVALID_ARG;
+  if (empty_shape(B, H, T)) return CATTN_OK;
+  if (!q || !k || !v || !o || !lse) return CATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return CATTN_ERR_INVALID_ARG;
+  int dev;
+  if ((st = check_device(&dev)) != CATTN_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  switch (D) {
+    case 16: return fwd_impl<16>(dev, q, k, v, scale, BH, T, o, lse, s);
+    case 32: return fwd_impl<32>(dev, q, k, v, scale, BH, T, o, lse, s);
+    case 64: return fwd_impl<64>(dev, q, k, v, scale, BH, T, o, lse, s);
+    case 128: return fwd_impl<128>(dev, q, k, v, scale, BH, T, o, lse, s);
+  }
+  return CATTN_ERR_UNSUPPORTED;
+}
+
+size_t attn_bwd_workspace_bytes(int B, int H, int T, int D) {
+  if (check_shape(B, H, T, D) != CATTN_OK) return 0;
+  if (empty_shape(B, H, T)) return 0;
+  return ws_layout(static_cast<long long>(B) * H, T, D).total;
+}
+
+cattn_status attn_bwd_preprocess(const void* o, const void* dout, int B, int H, int T, int D,
+                                 float* delta, void* stream) {
+  cattn_status st = check_shape(B, H, T, D);
+  if (st != CATTN_OK) return st;
+  if (empty_shape(B, H, T)) return CATTN_OK;
+  if (!o || !dout || !delta) return CATTN_ERR_INVALID_ARG;
+  if (!aligned(o, 16) || !aligned(dout, 16) || !aligned(delta, 4)) return CATTN_ERR_INVALID_ARG;
+  int dev;
+  if ((st = check_device(&dev)) != CATTN_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long BH = static_cast<long long>(B) * H;
+  switch (D) {
+    case 16: return pre_impl<16>(o, dout, nullptr, delta, nullptr, nullptr, 0, BH, T, T, s);
+    case 32: return pre_impl<32>(o, dout, nullptr, delta, nullptr, nullptr, 0, BH, T, T, s);
+    case 64: return pre_impl<64>(o, dout, nullptr, delta, nullptr, nullptr, 0, BH, T, T, s);
+    case 128: return pre_impl<128>(o, dout, nullptr, delta, nullptr, nullptr, 0, BH, T, T, s);
+  }
+  return CATTN_ERR_UNSUPPORTED;
+}
+
+cattn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                      const float* lse, const void* dout, float scale, int B, int H, int T, int D,
+                      void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  cattn_status st = check_shape(B, H, T, D);
+  if (st != CATTN_OK) return st;
+  if (!(scale > 0.f) || !isfinite(scale)) return CATTN_ERR_INVALID_ARG;
+  if (empty_shape(B, H, T)) return CATTN_OK;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
+    return CATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      !aligned(lse, 4) || !aligned(workspace, 256))
+    return CATTN_ERR_INVALID_ARG;
+  const int BH = B * H;
+  if (workspace_bytes < ws_layout(BH, T, D).total) return CATTN_ERR_INVALID_ARG;
+  int dev;
+  if ((st = check_device(&dev)) != CATTN_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (D) {
+    case 16: return bwd_impl<16>(dev, q, k, v, o, lse, dout, scale, BH, T, dq, dk, dv, workspace, s);
+    case 32: return bwd_impl<32>(dev, q, k, v, o, lse, dout, scale, BH, T, dq, dk, dv, workspace, s);
+    case 64: return bwd_impl<64>(dev, q, k, v, o, lse, dout, scale, BH, T, dq, dk, dv, workspace, s);
+    case 128:
+      return bwd_impl<128>(dev, q, k, v, o, lse, dout, scale, BH, T, dq, dk, dv, workspace, s);
+  }
+  return CATTN_ERR_UNSUPPORTED;
+}
+
+cattn_status cattn_get_device_status(int clear, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return CATTN_ERR_CUDA;
+  }
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) {
+    cudaGetLastError();
+    return CATTN_ERR_CUDA;
+  }
+  if (clear) {
+    const unsigned int z = 0;
+    if (cudaMemcpyToSymbol(g_status, &z, sizeof(z)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_status_where, &z, sizeof(z)) != cudaSuccess) {
+      cudaGetLastError();
+      return CATTN_ERR_CUDA;
+    }
+  }
+  return v == 0 ? CATTN_OK : static_cast<cattn_status>(v);
+}
+
+void cattn_set_wait_timeout_us(uint32_t us) {
+  g_timeout_ns = us == 0 ? kDefaultTimeoutNs : static_cast<uint64_t>(us) * 1000ull;
+}
+
+cattn_status cattn_selftest_wait_timeout(uint32_t timeout_us, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cattn_status st = cattn_get_device_status(1, stream);  // start from a clear word
+  if (st != CATTN_OK && st != CATTN_ERR_TIMEOUT) return st;
+  selftest_wait_kernel<<<1, 32, 0, s>>>(static_cast<uint64_t>(timeout_us) * 1000ull);
+  if (launch_status() != CATTN_OK) return CATTN_ERR_CUDA;
+  st = cattn_get_device_status(1, stream);
+  return st;
+}
+
+void cattn_timing_enable(int enable) { g_timing = enable != 0; }
+
+cattn_status cattn_timing_read(float* total_ms, int* launches, int n) {
+  if (!total_ms || !launches || n < 0) return CATTN_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    total_ms[i] = 0.f;
+    launches[i] = 0;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  cattn_status st = CATTN_OK;
+  for (const TimingRec& r : g_recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) {
+      cudaGetLastError();
+      st = CATTN_ERR_CUDA;
+    } else if (r.kernel < n) {
+      total_ms[r.kernel] += ms;
+      launches[r.kernel] += 1;
+    }
+    g_event_pool.push_back(r.a);
+    g_event_pool.push_back(r.b);
+  }
+  g_recs.clear();
+  return st;
+}
+
+const char* cattn_status_string(cattn_status s) {
+  switch (s) {
+    case CATTN_OK: return "ok";
+    case CATTN_ERR_INVALID_ARG: return "invalid argument";
+    case CATTN_ERR_UNSUPPORTED: return "unsupported (head size or device)";
+    case CATTN_ERR_CUDA: return "CUDA error";
+    case CATTN_ERR_TIMEOUT: return "kernel wait timed out";
+  }
+  return "unknown status";
+}
+
+int cattn_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,159 @@
+/*
+ * libcattn -- fused causal multi-head self-attention for NVIDIA B200 (sm_100a).
+ *
+ * What is computed.  For every batch b and head h independently
+ * ("nanoGPT: a real GPT in two 300-line files", section 2 "How the code
+ * works", CausalSelfAttention: one head per slice, attention on its own
+ * slice, heads glued back together):
+ *
+ *     S   = scale * Q K^T                  (T x T, never stored)
+ *     S_ij = -inf for j > i                ("fill the future with -inf";
+ *                                           "Causal" in "Words to know":
+ *                                           a position sees itself and
+ *                                           earlier positions only)
+ *     P   = softmax(S) row-wise
+ *     O   = P V
+ *     LSE_i = log(sum_{j<=i} exp(S_ij))    (natural log)
+ *
+ * "The 300-Line LLM Engine: Inside nanoGPT" ("Flat Architecture and Flash
+ * Attention") names not materialising that T x T matrix as the source of
+ * the model's speed; no call here ever writes an S- or P-sized buffer.
+ *
+ * Conventions common to every call:
+ *  - Q, K, V, O, dO, dQ, dK, dV are caller-owned DEVICE pointers to bf16
+ *    (__nv_bfloat16) tensors of shape (B, H, T, D), contiguous, row-major
+ *    (D fastest), 16-byte aligned.  LSE and Delta are caller-owned device
+ *    fp32 tensors of shape (B, H, T), contiguous, 4-byte aligned.
+ *  - T_q = T_k = T.  Causality is always on; there is no dropout and no
+ *    mask argument.  D must be 16, 32, 64 or 128; B, H, T >= 0 with
+ *    B*H <= 2^31-1 and T <= 2^20.  A shape with B*H*T == 0 is empty: the
+ *    call checks its other scalar arguments, launches nothing and returns
+ *    CATTN_OK (pointers may then be NULL).
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  All
+ *    work is asynchronous on that stream; a return of CATTN_OK means the
+ *    arguments were valid and every launch was accepted, nothing more.
+ *  - On any error return nothing has been launched and no output has
+ *    been touched.
+ *  - The library allocates no device memory for these calls and keeps no
+ *    per-call state.  Kernels whose internal waits exceed their poll limit
+ *    (a hang guard) record CATTN_ERR_TIMEOUT in a library-global device
+ *    status word and exit; read it with cattn_get_device_status().
+ */
+#ifndef CATTN_H
+#define CATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CATTN_API __attribute__((visibility("default")))
+#else
+#define CATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CATTN_OK = 0,
+  CATTN_ERR_INVALID_ARG = 1, /* null pointer, bad size, misalignment, small workspace */
+  CATTN_ERR_UNSUPPORTED = 2, /* head size D not instantiated; device not sm_100 */
+  CATTN_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+  CATTN_ERR_TIMEOUT = 4      /* a kernel's bounded wait ran out (device status) */
+} cattn_status;
+
+/* Forward pass: o = softmax(scale*q k^T + causal mask) v and its
+ * log-sum-exp.  Definition as above ("nanoGPT: a real GPT in two 300-line
+ * files", section 2, the written-out attention).
+ *   q, k, v : in,  bf16 (B,H,T,D)
+ *   scale   : softmax temperature, finite and > 0 (nanoGPT uses 1/sqrt(D))
+ *   o       : out, bf16 (B,H,T,D), round-to-nearest-even
+ *   lse     : out, fp32 (B,H,T), natural log
+ * Errors: CATTN_ERR_INVALID_ARG (null/misaligned pointer, negative or too
+ * large B, H, T, non-finite or non-positive scale), CATTN_ERR_UNSUPPORTED
+ * (D, or a device other than sm_100), CATTN_ERR_CUDA. */
+CATTN_API cattn_status attn_fwd(const void* q, const void* k, const void* v, float scale,
+                      int B, int H, int T, int D,
+                      void* o, float* lse, void* stream);
+
+/* Bytes of device workspace attn_bwd needs for this shape (0 on bad
+ * arguments).  The layout is internal: an fp32 dQ accumulator of
+ * B*H*T*D floats, fp32 Delta and scaled-LSE vectors of B*H*roundup(T,128)
+ * floats each,
+ * each part 256-byte aligned. */
+CATTN_API size_t attn_bwd_workspace_bytes(int B, int H, int T, int D);
+
+/* Backward preprocess on its own: delta_i = sum_d dout_id * o_id (fp32),
+ * the row term of the softmax Jacobian.  It follows from the definition
+ * above by the chain rule (the pages leave the gradient to autograd:
+ * "nanoGPT: a real GPT in two 300-line files", section 1, "Autograd does
+ * the calculus").
+ *   o, dout : in,  bf16 (B,H,T,D)
+ *   delta   : out, fp32 (B,H,T)
+ * Errors as attn_fwd. */
+CATTN_API cattn_status attn_bwd_preprocess(const void* o, const void* dout,
+                                 int B, int H, int T, int D,
+                                 float* delta, void* stream);
+
+/* Backward pass of a scalar loss L with dL/dO = dout:
+ *   dV = P^T dO;  dP = dO V^T;  Delta = rowsum(dO * O);
+ *   dS = P * (dP - Delta);  dQ = scale dS K;  dK = scale dS^T Q
+ * P is recomputed from q, k and lse per key tile (never stored).
+ *   q, k, v, o, dout : in, bf16 (B,H,T,D); o and lse as produced by attn_fwd
+ *   lse              : in, fp32 (B,H,T)
+ *   dq, dk, dv       : out, bf16 (B,H,T,D)
+ *   workspace        : caller-owned device scratch of at least
+ *                      attn_bwd_workspace_bytes(B,H,T,D) bytes, 256-byte
+ *                      aligned; overwritten; no contents needed on entry
+ * Calls that share a workspace must not overlap on the GPU.
+ * Errors as attn_fwd, plus CATTN_ERR_INVALID_ARG for a small or
+ * misaligned workspace. */
+CATTN_API cattn_status attn_bwd(const void* q, const void* k, const void* v,
+                      const void* o, const float* lse, const void* dout,
+                      float scale, int B, int H, int T, int D,
+                      void* dq, void* dk, void* dv,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Library-global device status word: CATTN_OK, or the first
+ * CATTN_ERR_TIMEOUT recorded by a kernel since the last clear.  Reads it
+ * synchronously (waits for all work on `stream`); clears it when `clear`
+ * is non-zero. */
+CATTN_API cattn_status cattn_get_device_status(int clear, void* stream);
+
+/* Time limit of every mbarrier wait inside the kernels (the hang guard), in
+ * microseconds.  0 restores the default of 2 s.  Process-global; affects
+ * launches made after the call.  A wait that runs out records
+ * CATTN_ERR_TIMEOUT in the device status word, and its CTA skips all later
+ * waits, drains the copies and MMAs it has in flight, frees its tensor
+ * memory and exits (outputs are then undefined). */
+CATTN_API void cattn_set_wait_timeout_us(uint32_t us);
+
+/* Self-test of the hang guard: clears the status word, launches one tiny
+ * kernel that waits on an mbarrier that nothing ever arrives on, with a
+ * limit of `timeout_us`, and returns the device status that kernel recorded
+ * (CATTN_ERR_TIMEOUT expected), clearing it again.  Faults nothing; the
+ * CUDA context stays usable.  Synchronises `stream`. */
+CATTN_API cattn_status cattn_selftest_wait_timeout(uint32_t timeout_us, void* stream);
+
+/* Kernel timer (benchmarking aid).  While enabled, every kernel this
+ * library launches is bracketed by two CUDA events recorded on its own
+ * launching stream.  cattn_timing_read() waits for the recorded events and
+ * returns, per kernel, the summed device time in ms and the launch count,
+ * then forgets them.  Kernel index: 0 forward, 1 backward preprocess,
+ * 2 backward main, 3 dQ convert.  n = length of both output arrays.  Not
+ * for use while a stream is being captured into a CUDA graph. */
+CATTN_API void cattn_timing_enable(int enable);
+CATTN_API cattn_status cattn_timing_read(float* total_ms, int* launches, int n);
+
+/* Human-readable name of a status code (static string). */
+CATTN_API const char* cattn_status_string(cattn_status s);
+
+/* Library version, major*10000 + minor*100 + patch. */
+CATTN_API int cattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CATTN_H */

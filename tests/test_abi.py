@@ -1,0 +1,151 @@
+"""CPU tests of the C ABI: the library loads, exports every function the
+header declares, and rejects bad arguments before touching any device.
+
+Only argument errors that the library detects before its first CUDA call
+are exercised here (no GPU on this host): every call below returns without
+launching anything and without dereferencing the (fake) pointers.
+"""
+
+import ctypes
+import math
+import os
+import re
+
+import pytest
+import torch  # noqa: F401  (loads the CUDA runtime libcattn links against)
+
+import causal_self_attention_flash_b200 as cattn
+from causal_self_attention_flash_b200 import _binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "cattn.h")
+
+ALIGNED = 0x10000  # fake, 16-byte aligned; never dereferenced by these calls
+
+
+def header_functions():
+    with open(HEADER) as f:
+        src = f.read()
+    return re.findall(r"^CATTN_API\s+[\w\s\*]+?\b(\w+)\s*\(", src, flags=re.M)
+
+
+def test_header_declares_the_north_star_calls():
+    names = header_functions()
+    for n in ("attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "attn_bwd_preprocess"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported():
+    lib = ctypes.CDLL(_binding.LIB_PATH)
+    names = header_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in _binding.SIGNATURES, n
+
+
+def test_version_and_strings():
+    assert cattn.cattn_version() == 100
+    assert cattn.cattn_status_string(0) == "ok"
+    assert "invalid" in cattn.cattn_status_string(1)
+    assert cattn.cattn_status_string(99) == "unknown status"
+
+
+def fwd(q=ALIGNED, k=ALIGNED, v=ALIGNED, scale=0.125, B=1, H=1, T=8, D=64,
+        o=ALIGNED, lse=ALIGNED):
+    return cattn.LIB.attn_fwd(q, k, v, scale, B, H, T, D, o, lse, None)
+
+
+def bwd(ptrs=None, scale=0.125, B=1, H=1, T=8, D=64, ws=ALIGNED, ws_bytes=1 << 30):
+    p = ptrs or [ALIGNED] * 9
+    return cattn.LIB.attn_bwd(p[0], p[1], p[2], p[3], p[4], p[5], scale, B, H, T, D,
+                              p[6], p[7], p[8], ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("D", [0, 8, 48, 96, 256])
+def test_unsupported_head_size(D):
+    assert fwd(D=D) == cattn.ERR_UNSUPPORTED
+    assert bwd(D=D) == cattn.ERR_UNSUPPORTED
+    assert cattn.attn_bwd_workspace_bytes(1, 1, 8, D) == 0
+
+
+@pytest.mark.parametrize("shape", [(-1, 1, 8), (1, -1, 8), (1, 1, -8), (1, 1, (1 << 20) + 1),
+                                   (1 << 16, 1 << 16, 8)])
+def test_bad_sizes(shape):
+    B, H, T = shape
+    assert fwd(B=B, H=H, T=T) == cattn.ERR_INVALID_ARG
+    assert bwd(B=B, H=H, T=T) == cattn.ERR_INVALID_ARG
+    assert cattn.attn_bwd_workspace_bytes(B, H, T, 64) == 0
+
+
+@pytest.mark.parametrize("scale", [0.0, -1.0, math.nan, math.inf])
+def test_bad_scale(scale):
+    assert fwd(scale=scale) == cattn.ERR_INVALID_ARG
+    assert bwd(scale=scale) == cattn.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("which", range(5))
+def test_null_pointer_fwd(which):
+    args = dict(q=ALIGNED, k=ALIGNED, v=ALIGNED, o=ALIGNED, lse=ALIGNED)
+    args[list(args)[which]] = None
+    assert fwd(**args) == cattn.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("which", range(9))
+def test_null_pointer_bwd(which):
+    p = [ALIGNED] * 9
+    p[which] = None
+    assert bwd(ptrs=p) == cattn.ERR_INVALID_ARG
+    assert bwd(ws=None) == cattn.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("which", range(4))
+def test_misaligned_fwd(which):
+    args = dict(q=ALIGNED, k=ALIGNED, v=ALIGNED, o=ALIGNED)
+    args[list(args)[which]] = ALIGNED + 8     # bf16 tensors need 16 bytes
+    assert fwd(**args) == cattn.ERR_INVALID_ARG
+    assert fwd(lse=ALIGNED + 2) == cattn.ERR_INVALID_ARG
+
+
+def test_misaligned_or_small_workspace():
+    assert bwd(ws=ALIGNED + 128) == cattn.ERR_INVALID_ARG
+    need = cattn.attn_bwd_workspace_bytes(1, 1, 8, 64)
+    assert bwd(ws_bytes=need - 1) == cattn.ERR_INVALID_ARG
+
+
+def test_empty_shapes_are_noops():
+    for B, H, T in ((0, 4, 8), (2, 0, 8), (2, 4, 0)):
+        assert fwd(q=None, k=None, v=None, o=None, lse=None, B=B, H=H, T=T) == cattn.OK
+        assert bwd(ptrs=[None] * 9, ws=None, ws_bytes=0, B=B, H=H, T=T) == cattn.OK
+        assert cattn.LIB.attn_bwd_preprocess(None, None, B, H, T, 64, None, None) == cattn.OK
+        assert cattn.attn_bwd_workspace_bytes(B, H, T, 64) == 0
+
+
+@pytest.mark.parametrize("B,H,T,D", [(1, 1, 1, 16), (16, 12, 1024, 64), (2, 16, 8192, 128),
+                                     (3, 5, 1000, 32)])
+def test_workspace_formula(B, H, T, D):
+    def r256(x):
+        return (x + 255) // 256 * 256
+    tpad = (T + 127) // 128 * 128
+    want = r256(B * H * T * D * 4) + 2 * r256(B * H * tpad * 4)
+    assert cattn.attn_bwd_workspace_bytes(B, H, T, D) == want
+
+
+def test_binding_refuses_cpu_tensors():
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        cattn.attn_fwd(q, q, q)
+    with pytest.raises(ValueError):
+        cattn.attn_fwd(q.float(), q.float(), q.float())
+
+
+def test_product_has_no_oracle_dependency():
+    """The product package never imports or names the oracle."""
+    pkg = os.path.dirname(cattn.__file__)
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                with open(os.path.join(dirpath, f)) as fh:
+                    src = fh.read()
+                assert "oracle" not in src, f
+                assert "workloads" not in src, f

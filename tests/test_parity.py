@@ -1,0 +1,209 @@
+"""GPU parity: libcattn (through its C ABI) against the fp64 oracle on the
+same seeded bf16 inputs, for the five workloads and for ragged/edge shapes.
+
+The oracle always receives the bf16-rounded inputs the GPU receives, so the
+difference measured is the kernels' own error.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity_util import check_bf16, check_lse, errors
+from workloads import (WORKLOADS, as_f64, bf16_inputs, draw_extra,
+                       sample_heads, seed_for, workload_inputs)
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gpu(lib, q, k, v, do, scale):
+    dev = torch.device("cuda:0")
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o, lse = lib.attn_fwd(qd, kd, vd, scale)
+    dq, dk, dv = lib.attn_bwd(qd, kd, vd, o, lse, dod, scale)
+    torch.cuda.synchronize()
+    assert lib.cattn_get_device_status() == lib.OK
+    return {n: as_f64(t) for n, t in
+            (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+
+
+def full_oracle(q, k, v, do, scale):
+    qn, kn, vn, don = (as_f64(t) for t in (q, k, v, do))
+    o, lse = oracle.attention_forward(qn, kn, vn, scale)
+    dq, dk, dv = oracle.attention_backward(qn, kn, vn, don, scale)
+    return dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv)
+
+
+def check_all(got, ref, report=None):
+    for n in ("o", "dq", "dk", "dv"):
+        ma, rl = check_bf16(n, got[n], ref[n])
+        if report is not None:
+            report[n] = (ma, rl)
+    ma = check_lse(got["lse"], ref["lse"])
+    if report is not None:
+        report["lse"] = ma
+
+
+@pytest.mark.parametrize("index", [0, 1, 2, 3])
+def test_workload_full_oracle(lib, index):
+    w = WORKLOADS[index]
+    q, k, v, do = workload_inputs(index)
+    got = run_gpu(lib, q, k, v, do, w.scale)
+    ref = full_oracle(q, k, v, do, w.scale)
+    rep = {}
+    check_all(got, ref, rep)
+    print(w.name, rep)
+
+
+def test_long_context_sampled_heads(lib):
+    """T = 8192, D = 128, logit std 4: two whole heads through the full
+    oracle (fwd + bwd), plus single rows of O/LSE on eight more heads."""
+    index = 4
+    w = WORKLOADS[index]
+    q, k, v, do = workload_inputs(index)
+    got = run_gpu(lib, q, k, v, do, w.scale)
+    heads = sample_heads(w.BH, 2, seed=seed_for(index))
+    qn, kn, vn, don = (as_f64(t) for t in (q, k, v, do))
+    ro, rl = oracle.attention_forward_heads(qn, kn, vn, w.scale, heads)
+    rq, rk, rv = oracle.attention_backward_heads(qn, kn, vn, don, w.scale, heads)
+    flat = {n: got[n].reshape(w.BH, w.T, -1) for n in ("o", "dq", "dk", "dv")}
+    flat["lse"] = got["lse"].reshape(w.BH, w.T)
+    rep = {}
+    for n, ref in (("o", ro), ("dq", rq), ("dk", rk), ("dv", rv)):
+        rep[n] = check_bf16(n, flat[n][heads], ref)
+    rep["lse"] = check_lse(flat["lse"][heads], rl)
+    print(w.name, heads, rep)
+    rows = [0, 1, 127, 128, 4095, 8191]
+    for f in sample_heads(w.BH, 8, seed=seed_for(index) + 1):
+        b, h = divmod(f, w.H)
+        o_rows, lse_rows = oracle.attention_rows(qn, kn, vn, w.scale, b, h, rows)
+        check_bf16("o rows", got["o"][b, h, rows], o_rows)
+        check_lse(got["lse"][b, h, rows], lse_rows)
+
+
+RAGGED_T = [1, 17, 63, 64, 65, 127, 128, 129, 255, 1000]
+
+
+@pytest.mark.parametrize("D", [16, 32, 64, 128])
+@pytest.mark.parametrize("T", RAGGED_T)
+def test_ragged_lengths(lib, T, D):
+    B, H = 2, 1
+    q, k, v, do = bf16_inputs(B, H, T, D, seed=7000 + 10 * T + D)
+    scale = 1.0 / math.sqrt(D)
+    check_all(run_gpu(lib, q, k, v, do, scale), full_oracle(q, k, v, do, scale))
+
+
+@pytest.mark.parametrize("scale", [0.02, 0.5])
+def test_other_scales_and_peaked_logits(lib, scale):
+    B, H, T, D = 1, 3, 300, 64
+    q, k, v, do = bf16_inputs(B, H, T, D, seed=91, qk_std=2.0)
+    check_all(run_gpu(lib, q, k, v, do, scale), full_oracle(q, k, v, do, scale))
+
+
+def test_preprocess_delta(lib):
+    """The Delta step on its own: synthetic O and dO (independent draws)."""
+    B, H, T, D = 3, 4, 333, 64
+    o = draw_extra((B, H, T, D), seed=501)
+    do = draw_extra((B, H, T, D), seed=502)
+    delta = lib.attn_bwd_preprocess(o.cuda(), do.cuda())
+    torch.cuda.synchronize()
+    ref = oracle.delta_from_o(as_f64(o), as_f64(do))
+    err = np.abs(as_f64(delta) - ref).max()
+    assert err <= 1e-4 * max(1.0, np.abs(ref).max()), err
+    for D2 in (16, 32, 128):
+        o2 = draw_extra((1, 2, 77, D2), seed=503 + D2)
+        do2 = draw_extra((1, 2, 77, D2), seed=504 + D2)
+        d2 = lib.attn_bwd_preprocess(o2.cuda(), do2.cuda())
+        ref2 = oracle.delta_from_o(as_f64(o2), as_f64(do2))
+        assert np.abs(as_f64(d2) - ref2).max() <= 1e-4 * max(1.0, np.abs(ref2).max())
+
+
+def test_outputs_stay_in_bounds(lib):
+    """Canary-padded outputs: every byte outside the tensors is untouched,
+    and a NaN-poisoned workspace does not leak into the results."""
+    B, H, T, D = 2, 3, 200, 64
+    q, k, v, do = bf16_inputs(B, H, T, D, seed=333)
+    scale = 1.0 / math.sqrt(D)
+    dev = torch.device("cuda:0")
+    n = B * H * T * D
+    pad = 4096
+    sentinel = torch.tensor(1234.0, dtype=torch.bfloat16)
+
+    def padded(numel, dtype):
+        buf = torch.full((numel + 2 * pad,), float(sentinel) if dtype == torch.bfloat16
+                         else -777.0, dtype=dtype, device=dev)
+        return buf, buf[pad:pad + numel]
+
+    ob, o = padded(n, torch.bfloat16)
+    lb, lse = padded(B * H * T, torch.float32)
+    outs = [padded(n, torch.bfloat16) for _ in range(3)]
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    lib.attn_fwd(qd, kd, vd, scale, o=o.view(B, H, T, D), lse=lse.view(B, H, T))
+    wsn = lib.attn_bwd_workspace_bytes(B, H, T, D)
+    ws = torch.full((wsn,), 0xFF, dtype=torch.uint8, device=dev)   # NaN floats
+    lib.attn_bwd(qd, kd, vd, o.view(B, H, T, D), lse.view(B, H, T), dod, scale,
+                 dq=outs[0][1].view(B, H, T, D), dk=outs[1][1].view(B, H, T, D),
+                 dv=outs[2][1].view(B, H, T, D), workspace=ws)
+    torch.cuda.synchronize()
+    for buf in [ob] + [b for b, _ in outs]:
+        assert (buf[:pad] == sentinel).all() and (buf[-pad:] == sentinel).all()
+    assert (lb[:pad] == -777.0).all() and (lb[-pad:] == -777.0).all()
+    got = dict(o=as_f64(o.view(B, H, T, D)), lse=as_f64(lse.view(B, H, T)),
+               dq=as_f64(outs[0][1].view(B, H, T, D)), dk=as_f64(outs[1][1].view(B, H, T, D)),
+               dv=as_f64(outs[2][1].view(B, H, T, D)))
+    check_all(got, full_oracle(q, k, v, do, scale))
+
+
+def test_forward_is_deterministic(lib):
+    q, k, v, _ = (t.cuda() for t in bf16_inputs(2, 4, 700, 64, seed=44))
+    o1, l1 = lib.attn_fwd(q, k, v)
+    o2, l2 = lib.attn_fwd(q, k, v)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_empty_sequence(lib):
+    q = torch.empty(2, 3, 0, 64, dtype=torch.bfloat16, device="cuda")
+    o, lse = lib.attn_fwd(q, q, q)
+    dq, dk, dv = lib.attn_bwd(q, q, q, o, lse, q)
+    assert o.shape == (2, 3, 0, 64) and dq.shape == (2, 3, 0, 64)
+
+
+def test_autograd_wrapper(lib):
+    B, H, T, D = 1, 2, 150, 64
+    q, k, v, do = bf16_inputs(B, H, T, D, seed=12)
+    qd, kd, vd = (t.cuda().requires_grad_(True) for t in (q, k, v))
+    out = lib.CausalAttention.apply(qd, kd, vd, None)
+    out.backward(do.cuda())
+    ref = full_oracle(q, k, v, do, 1.0 / math.sqrt(D))
+    check_bf16("o", as_f64(out), ref["o"])
+    check_bf16("dq", as_f64(qd.grad), ref["dq"])
+    check_bf16("dk", as_f64(kd.grad), ref["dk"])
+    check_bf16("dv", as_f64(vd.grad), ref["dv"])
+
+
+def test_hang_guard_times_out_cleanly(lib):
+    """A wait on a barrier nothing arrives on gives up after its limit,
+    records CATTN_ERR_TIMEOUT, and leaves the context usable."""
+    st = lib.cattn_selftest_wait_timeout(2000)
+    assert st == lib.ERR_TIMEOUT
+    assert lib.cattn_get_device_status() == lib.OK   # the self-test cleared it
+    q, k, v, do = bf16_inputs(1, 2, 130, 64, seed=5)
+    got = run_gpu(lib, q, k, v, do, 0.125)
+    check_all(got, full_oracle(q, k, v, do, 0.125))
+
+
+def test_errors_reported_on_device(lib):
+    q = torch.zeros(1, 1, 8, 48, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(lib.CattnError) as e:
+        lib.attn_fwd(q, q, q)
+    assert e.value.status == lib.ERR_UNSUPPORTED
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16, device="cuda")
+    o, lse = lib.attn_fwd(q, q, q)
+    with pytest.raises(lib.CattnError):
+        lib.attn_bwd(q, q, q, o, lse, q,
+                     workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
+    assert errors(as_f64(o), np.zeros((1, 1, 8, 64)))[0] == 0.0
