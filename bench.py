@@ -69,9 +69,19 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_hash() -> str:
+KERNEL_SOURCES = {
+    "fwd_kernel": ("fwd.cuh", "sm100.cuh"),
+    "bwd_kernel": ("bwd.cuh", "sm100.cuh"),
+    "bwd_pre_kernel": ("bwd.cuh", "sm100.cuh"),
+    "dq_convert_kernel": ("bwd.cuh", "sm100.cuh"),
+}
+
+
+def source_hash(kernel: str) -> str:
+    """Hash of the device sources a kernel is compiled from (its ncu traffic
+    figure is reported only while this matches the one stored with it)."""
     h = hashlib.sha256()
-    for f in sorted(os.listdir(CSRC)):
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(CSRC, f), "rb") as fh:
             h.update(f.encode())
             h.update(fh.read())
@@ -333,7 +343,7 @@ def run_cattn(args, w, index, world, rank, local):
         with open(TRAFFIC_FILE) as f:
             tr = json.load(f)
         ent = tr.get(dom, {})
-        if ent.get("source_hash") == source_hash() and ent.get("workload") == w.name:
+        if ent.get("source_hash") == source_hash(dom) and ent.get("workload") == w.name:
             traffic = ent.get("bytes_per_launch")
     except (OSError, ValueError):
         pass

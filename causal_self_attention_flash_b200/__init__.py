@@ -37,7 +37,7 @@ def _stream(stream):
 
 def _check(name, st):
     if st != OK:
-        raise CattnError(name, st)
+        raise CattnError(name, st, int(LIB.cattn_last_cuda_error()) if st == ERR_CUDA else 0)
 
 
 def _shape(q):

@@ -39,13 +39,16 @@ SIGNATURES = {
     "cattn_timing_read": (_i, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int), _i]),
     "cattn_status_string": (ctypes.c_char_p, [_i]),
     "cattn_version": (_i, []),
+    "cattn_last_cuda_error": (_i, []),
 }
 
 
 class CattnError(RuntimeError):
-    def __init__(self, fn: str, status: int):
+    def __init__(self, fn: str, status: int, cuda_error: int = 0):
         self.status = status
-        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+        self.cuda_error = cuda_error
+        extra = f" (CUDA error {cuda_error})" if status == ERR_CUDA else ""
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}{extra}")
 
 
 def load(path: str = LIB_PATH) -> ctypes.CDLL:

@@ -28,6 +28,12 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 
 std::mutex g_mu;
 EncodeTiledFn g_encode = nullptr;
+thread_local int g_last_cuda_error = 0;  // cudaError_t / CUresult of the last failure
+
+cattn_status cuda_fail(int code) {
+  g_last_cuda_error = code;
+  return CATTN_ERR_CUDA;
+}
 int g_dev_ok[kMaxDevices];           // 0 unknown, 1 sm_100, -1 other
 unsigned g_attr_done[kMaxDevices];   // bit per kernel instance
 
@@ -39,26 +45,30 @@ cattn_status init_encode() {
   if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
           cudaSuccess ||
       q != cudaDriverEntryPointSuccess || fn == nullptr) {
-    cudaGetLastError();
-    return CATTN_ERR_CUDA;
+    return cuda_fail(cudaGetLastError());
   }
   g_encode = reinterpret_cast<EncodeTiledFn>(fn);
   return CATTN_OK;
 }
 
+thread_local int g_bound_device = -1;  // device whose primary context this thread holds
+
 cattn_status check_device(int* dev_out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) {
-    cudaGetLastError();
-    return CATTN_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail(cudaGetLastError());
+  // A host thread that has made no runtime call yet (an autograd worker, a
+  // fresh std::thread) has no current context, and the driver's tensor-map
+  // encoder needs one: bind the device's primary context once per thread.
+  if (g_bound_device != dev) {
+    if (cudaSetDevice(dev) != cudaSuccess) return cuda_fail(cudaGetLastError());
+    g_bound_device = dev;
   }
   if (dev < 0 || dev >= kMaxDevices) return CATTN_ERR_UNSUPPORTED;
   if (g_dev_ok[dev] == 0) {
     int major = 0, minor = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
-      cudaGetLastError();
-      return CATTN_ERR_CUDA;
+      return cuda_fail(cudaGetLastError());
     }
     g_dev_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
   }
@@ -73,8 +83,7 @@ cattn_status ensure_smem(int dev, unsigned bit, K kernel, int bytes) {
   if (g_attr_done[dev] & (1u << bit)) return CATTN_OK;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
       cudaSuccess) {
-    cudaGetLastError();
-    return CATTN_ERR_CUDA;
+    return cuda_fail(cudaGetLastError());
   }
   std::lock_guard<std::mutex> lk(g_mu);
   g_attr_done[dev] |= 1u << bit;
@@ -113,7 +122,7 @@ cattn_status make_tmap(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, 
   CUresult r = g_encode(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? CATTN_OK : CATTN_ERR_CUDA;
+  return r == CUDA_SUCCESS ? CATTN_OK : cuda_fail(10000 + static_cast<int>(r));
 }
 
 cattn_status make_bf16_map(CUtensorMap* m, const void* ptr, int D, int T, long long BH) {
@@ -123,8 +132,13 @@ cattn_status make_bf16_map(CUtensorMap* m, const void* ptr, int D, int T, long l
 
 cattn_status launch_status() {
   cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? CATTN_OK : CATTN_ERR_CUDA;
+  return e == cudaSuccess ? CATTN_OK : cuda_fail(e);
 }
+
+// A non-sticky error left in this thread's runtime state by an earlier call
+// of the caller's (e.g. a not-ready query) must not be taken for a failure
+// of our launches: clear it before launching.
+void clear_stale_error() { (void)cudaGetLastError(); }
 
 int grid_for(size_t work_items, int per_block) {
   size_t g = (work_items + per_block - 1) / per_block;
@@ -187,6 +201,7 @@ template <int D>
 cattn_status fwd_impl(int dev, const void* q, const void* k, const void* v, float scale, int BH,
                       int T, void* o, float* lse, cudaStream_t s) {
   using C = FwdCfg<D>;
+  clear_stale_error();
   cattn_status st = ensure_smem(dev, 0 + (D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3),
                                 fwd_kernel<D>, C::SMEM_BYTES);
   if (st != CATTN_OK) return st;
@@ -232,6 +247,7 @@ template <int D>
 cattn_status pre_impl(const void* o, const void* dout, const float* lse, float* delta,
                       float* lse2, float4* zero, size_t zero_n4, long long BH, int T,
                       int row_stride, cudaStream_t s) {
+  clear_stale_error();
   PreParams p;
   p.o = static_cast<const __nv_bfloat16*>(o);
   p.dout = static_cast<const __nv_bfloat16*>(dout);
@@ -258,6 +274,7 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
                       const float* lse, const void* dout, float scale, int BH, int T, void* dq,
                       void* dk, void* dv, void* ws, cudaStream_t s) {
   using C = BwdCfg<D>;
+  clear_stale_error();
   cattn_status st = ensure_smem(dev, 4 + (D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3),
                                 bwd_kernel<D>, C::SMEM_BYTES);
   if (st != CATTN_OK) return st;
@@ -410,21 +427,15 @@ cattn_status attn_bwd(const void* q, const void* k, const void* v, const void* o
 
 cattn_status cattn_get_device_status(int clear, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaStreamSynchronize(s) != cudaSuccess) {
-    cudaGetLastError();
-    return CATTN_ERR_CUDA;
-  }
+  if (cudaStreamSynchronize(s) != cudaSuccess) return cuda_fail(cudaGetLastError());
   unsigned int v = 0;
-  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) {
-    cudaGetLastError();
-    return CATTN_ERR_CUDA;
-  }
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess)
+    return cuda_fail(cudaGetLastError());
   if (clear) {
     const unsigned int z = 0;
     if (cudaMemcpyToSymbol(g_status, &z, sizeof(z)) != cudaSuccess ||
         cudaMemcpyToSymbol(g_status_where, &z, sizeof(z)) != cudaSuccess) {
-      cudaGetLastError();
-      return CATTN_ERR_CUDA;
+      return cuda_fail(cudaGetLastError());
     }
   }
   return v == 0 ? CATTN_OK : static_cast<cattn_status>(v);
@@ -456,9 +467,9 @@ cattn_status cattn_timing_read(float* total_ms, int* launches, int n) {
   cattn_status st = CATTN_OK;
   for (const TimingRec& r : g_recs) {
     float ms = 0.f;
-    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) {
-      cudaGetLastError();
-      st = CATTN_ERR_CUDA;
+    if (cudaEventSynchronize(r.b) != cudaSuccess ||
+        cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) {
+      st = cuda_fail(cudaGetLastError());
     } else if (r.kernel < n) {
       total_ms[r.kernel] += ms;
       launches[r.kernel] += 1;
@@ -482,5 +493,7 @@ const char* cattn_status_string(cattn_status s) {
 }
 
 int cattn_version(void) { return 100; }
+
+int cattn_last_cuda_error(void) { return g_last_cuda_error; }
 
 }  // extern "C"

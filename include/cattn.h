@@ -149,6 +149,11 @@ CATTN_API cattn_status cattn_timing_read(float* total_ms, int* launches, int n);
 /* Human-readable name of a status code (static string). */
 CATTN_API const char* cattn_status_string(cattn_status s);
 
+/* Code of the CUDA failure behind the last CATTN_ERR_CUDA returned to this
+ * host thread: a cudaError_t, or 10000 + CUresult for a failed tensor-map
+ * encoding; 0 if none. */
+CATTN_API int cattn_last_cuda_error(void);
+
 /* Library version, major*10000 + minor*100 + patch. */
 CATTN_API int cattn_version(void);
 
