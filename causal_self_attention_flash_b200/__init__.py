@@ -20,7 +20,8 @@ from ._binding import (ERR_CUDA, ERR_INVALID_ARG, ERR_TIMEOUT,
                        ERR_UNSUPPORTED, LIB, LIB_PATH, OK, CattnError)
 
 __all__ = [
-    "attn_fwd", "attn_bwd", "attn_bwd_preprocess", "attn_bwd_workspace_bytes",
+    "attn_fwd", "attn_bwd", "attn_fwd_ex", "attn_bwd_ex", "attn_bwd_preprocess",
+    "attn_bwd_workspace_bytes",
     "cattn_get_device_status", "cattn_set_wait_timeout_us",
     "cattn_selftest_wait_timeout", "cattn_status_string", "cattn_version",
     "cattn_timing_enable", "cattn_timing_read", "KERNEL_NAMES",
@@ -60,6 +61,26 @@ def _inputs(*ts):
             raise ValueError("inputs must be contiguous bf16 CUDA tensors")
 
 
+def attn_fwd_ex(q, k, v, scale=None, o=None, lse=None, o_lo=None, want_o_lo=True,
+                stream=None):
+    """(o, lse, o_lo) = causal attention of bf16 (B,H,T,D) q, k, v, with the
+    bf16 rounding residual o_lo = bf16(O - o) of the output (None if not
+    wanted)."""
+    _inputs(q, k, v)
+    B, H, T, D = _shape(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    o = _want(o, q, torch.bfloat16, (B, H, T, D))
+    lse = _want(lse, q, torch.float32, (B, H, T))
+    if want_o_lo:
+        o_lo = _want(o_lo, q, torch.bfloat16, (B, H, T, D))
+    st = LIB.attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), float(scale), B, H, T, D,
+                         o.data_ptr(), lse.data_ptr(),
+                         o_lo.data_ptr() if o_lo is not None else None, _stream(stream))
+    _check("attn_fwd_ex", st)
+    return o, lse, o_lo
+
+
 def attn_fwd(q, k, v, scale=None, o=None, lse=None, stream=None):
     """(o, lse) = causal attention of bf16 (B,H,T,D) q, k, v."""
     _inputs(q, k, v)
@@ -90,9 +111,10 @@ def attn_bwd_preprocess(o, do, delta=None, stream=None):
 
 
 def attn_bwd(q, k, v, o, lse, do, scale=None, dq=None, dk=None, dv=None,
-             workspace=None, stream=None):
+             workspace=None, stream=None, o_lo=None):
     """(dq, dk, dv) of causal attention; workspace allocated with torch if
-    not given (a uint8 CUDA tensor of attn_bwd_workspace_bytes bytes)."""
+    not given (a uint8 CUDA tensor of attn_bwd_workspace_bytes bytes).
+    With the forward's o_lo (attn_fwd_ex) this calls attn_bwd_ex."""
     _inputs(q, k, v, o, do)
     B, H, T, D = _shape(q)
     if scale is None:
@@ -105,11 +127,23 @@ def attn_bwd(q, k, v, o, lse, do, scale=None, dq=None, dk=None, dv=None,
     need = attn_bwd_workspace_bytes(B, H, T, D)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    st = LIB.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                      do.data_ptr(), float(scale), B, H, T, D, dq.data_ptr(), dk.data_ptr(),
-                      dv.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream))
-    _check("attn_bwd", st)
+    if o_lo is None:
+        st = LIB.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                          lse.data_ptr(), do.data_ptr(), float(scale), B, H, T, D,
+                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                          workspace.numel(), _stream(stream))
+        _check("attn_bwd", st)
+    else:
+        _inputs(o_lo)
+        st = LIB.attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                             o_lo.data_ptr(), lse.data_ptr(), do.data_ptr(), float(scale),
+                             B, H, T, D, dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                             workspace.data_ptr(), workspace.numel(), _stream(stream))
+        _check("attn_bwd_ex", st)
     return dq, dk, dv
+
+
+attn_bwd_ex = attn_bwd
 
 
 def cattn_get_device_status(clear=False, stream=None):
@@ -154,13 +188,13 @@ class CausalAttention(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, q, k, v, scale=None):
-        o, lse = attn_fwd(q, k, v, scale)
-        ctx.save_for_backward(q, k, v, o, lse)
+        o, lse, o_lo = attn_fwd_ex(q, k, v, scale)
+        ctx.save_for_backward(q, k, v, o, lse, o_lo)
         ctx.scale = scale
         return o
 
     @staticmethod
     def backward(ctx, do):
-        q, k, v, o, lse = ctx.saved_tensors
-        dq, dk, dv = attn_bwd(q, k, v, o, lse, do.contiguous(), ctx.scale)
+        q, k, v, o, lse, o_lo = ctx.saved_tensors
+        dq, dk, dv = attn_bwd(q, k, v, o, lse, do.contiguous(), ctx.scale, o_lo=o_lo)
         return dq, dk, dv, None

@@ -28,10 +28,13 @@ _vp, _i, _f, _sz, _u32 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_float,
                           ctypes.c_size_t, ctypes.c_uint32)
 SIGNATURES = {
     "attn_fwd": (_i, [_vp, _vp, _vp, _f, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "attn_fwd_ex": (_i, [_vp, _vp, _vp, _f, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "attn_bwd_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "attn_bwd_preprocess": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp]),
     "attn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _f, _i, _i, _i, _i,
                       _vp, _vp, _vp, _vp, _sz, _vp]),
+    "attn_bwd_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _f, _i, _i, _i, _i,
+                         _vp, _vp, _vp, _vp, _sz, _vp]),
     "cattn_get_device_status": (_i, [_i, _vp]),
     "cattn_set_wait_timeout_us": (None, [_u32]),
     "cattn_selftest_wait_timeout": (_i, [_u32, _vp]),

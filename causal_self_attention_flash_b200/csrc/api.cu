@@ -199,19 +199,22 @@ struct LaunchTimer {
 
 template <int D>
 cattn_status fwd_impl(int dev, const void* q, const void* k, const void* v, float scale, int BH,
-                      int T, void* o, float* lse, cudaStream_t s) {
+                      int T, void* o, float* lse, void* o_lo, cudaStream_t s) {
   using C = FwdCfg<D>;
   clear_stale_error();
   cattn_status st = ensure_smem(dev, 0 + (D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3),
                                 fwd_kernel<D>, C::SMEM_BYTES);
   if (st != CATTN_OK) return st;
-  CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mq, mk, mv, mo, molo;
   if ((st = make_bf16_map(&mq, q, D, T, BH)) != CATTN_OK) return st;
   if ((st = make_bf16_map(&mk, k, D, T, BH)) != CATTN_OK) return st;
   if ((st = make_bf16_map(&mv, v, D, T, BH)) != CATTN_OK) return st;
   if ((st = make_bf16_map(&mo, o, D, T, BH)) != CATTN_OK) return st;
+  // without O_lo the kernel never touches this map; it reuses O's
+  if ((st = make_bf16_map(&molo, o_lo ? o_lo : o, D, T, BH)) != CATTN_OK) return st;
   FwdParams p;
   p.lse = lse;
+  p.write_o_lo = o_lo != nullptr;
   p.T = T;
   p.n_qtiles = (T + 127) / 128;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -219,7 +222,7 @@ cattn_status fwd_impl(int dev, const void* q, const void* k, const void* v, floa
   dim3 grid(BH, p.n_qtiles);
   {
     LaunchTimer t(K_FWD, s);
-    fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, p);
+    fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, molo, p);
   }
   return launch_status();
 }
@@ -244,12 +247,13 @@ WsLayout ws_layout(long long BH, int T, int D) {
 }
 
 template <int D>
-cattn_status pre_impl(const void* o, const void* dout, const float* lse, float* delta,
-                      float* lse2, float4* zero, size_t zero_n4, long long BH, int T,
-                      int row_stride, cudaStream_t s) {
+cattn_status pre_impl(const void* o, const void* o_lo, const void* dout, const float* lse,
+                      float* delta, float* lse2, float4* zero, size_t zero_n4, long long BH,
+                      int T, int row_stride, cudaStream_t s) {
   clear_stale_error();
   PreParams p;
   p.o = static_cast<const __nv_bfloat16*>(o);
+  p.o_lo = static_cast<const __nv_bfloat16*>(o_lo);
   p.dout = static_cast<const __nv_bfloat16*>(dout);
   p.lse = lse;
   p.delta = delta;
@@ -271,8 +275,8 @@ cattn_status pre_impl(const void* o, const void* dout, const float* lse, float* 
 
 template <int D>
 cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, const void* o,
-                      const float* lse, const void* dout, float scale, int BH, int T, void* dq,
-                      void* dk, void* dv, void* ws, cudaStream_t s) {
+                      const void* o_lo, const float* lse, const void* dout, float scale, int BH,
+                      int T, void* dq, void* dk, void* dv, void* ws, cudaStream_t s) {
   using C = BwdCfg<D>;
   clear_stale_error();
   cattn_status st = ensure_smem(dev, 4 + (D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3),
@@ -296,7 +300,7 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
       CATTN_OK)
     return st;
 
-  st = pre_impl<D>(o, dout, lse, delta, lse2, reinterpret_cast<float4*>(dq_acc), n_dq / 4, BH, T,
+  st = pre_impl<D>(o, o_lo, dout, lse, delta, lse2, reinterpret_cast<float4*>(dq_acc), n_dq / 4, BH, T,
                    L.T_pad, s);
   if (st != CATTN_OK) return st;
 
@@ -348,26 +352,32 @@ using namespace cattn;
 
 extern "C" {
 
-cattn_status attn_fwd(const void* q, const void* k, const void* v, float scale, int B, int H,
-                      int T, int D, void* o, float* lse, void* stream) {
+cattn_status attn_fwd_ex(const void* q, const void* k, const void* v, float scale, int B, int H,
+                         int T, int D, void* o, float* lse, void* o_lo, void* stream) {
   cattn_status st = check_shape(B, H, T, D);
   if (st != CATTN_OK) return st;
   if (!(scale > 0.f) || !isfinite(scale)) return CATTN_ERR_INVALID_ARG;
   if (empty_shape(B, H, T)) return CATTN_OK;
   if (!q || !k || !v || !o || !lse) return CATTN_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4) || !aligned(o_lo, 16))
     return CATTN_ERR_INVALID_ARG;
   int dev;
   if ((st = check_device(&dev)) != CATTN_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int BH = B * H;
   switch (D) {
-    case 16: return fwd_impl<16>(dev, q, k, v, scale, BH, T, o, lse, s);
-    case 32: return fwd_impl<32>(dev, q, k, v, scale, BH, T, o, lse, s);
-    case 64: return fwd_impl<64>(dev, q, k, v, scale, BH, T, o, lse, s);
-    case 128: return fwd_impl<128>(dev, q, k, v, scale, BH, T, o, lse, s);
+    case 16: return fwd_impl<16>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s);
+    case 32: return fwd_impl<32>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s);
+    case 64: return fwd_impl<64>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s);
+    case 128: return fwd_impl<128>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s);
   }
   return CATTN_ERR_UNSUPPORTED;
+}
+
+cattn_status attn_fwd(const void* q, const void* k, const void* v, float scale, int B, int H,
+                      int T, int D, void* o, float* lse, void* stream) {
+  return attn_fwd_ex(q, k, v, scale, B, H, T, D, o, lse, nullptr, stream);
 }
 
 size_t attn_bwd_workspace_bytes(int B, int H, int T, int D) {
@@ -388,18 +398,18 @@ cattn_status attn_bwd_preprocess(const void* o, const void* dout, int B, int H, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const long long BH = static_cast<long long>(B) * H;
   switch (D) {
-    case 16: return pre_impl<16>(o, dout, nullptr, delta, nullptr, nullptr, 0, BH, T, T, s);
-    case 32: return pre_impl<32>(o, dout, nullptr, delta, nullptr, nullptr, 0, BH, T, T, s);
-    case 64: return pre_impl<64>(o, dout, nullptr, delta, nullptr, nullptr, 0, BH, T, T, s);
-    case 128: return pre_impl<128>(o, dout, nullptr, delta, nullptr, nullptr, 0, BH, T, T, s);
+    case 16: return pre_impl<16>(o, nullptr, dout, nullptr, delta, nullptr, nullptr, 0, BH, T, T, s);
+    case 32: return pre_impl<32>(o, nullptr, dout, nullptr, delta, nullptr, nullptr, 0, BH, T, T, s);
+    case 64: return pre_impl<64>(o, nullptr, dout, nullptr, delta, nullptr, nullptr, 0, BH, T, T, s);
+    case 128: return pre_impl<128>(o, nullptr, dout, nullptr, delta, nullptr, nullptr, 0, BH, T, T, s);
   }
   return CATTN_ERR_UNSUPPORTED;
 }
 
-cattn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
-                      const float* lse, const void* dout, float scale, int B, int H, int T, int D,
-                      void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
-                      void* stream) {
+cattn_status attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
+                         const void* o_lo, const float* lse, const void* dout, float scale, int B,
+                         int H, int T, int D, void* dq, void* dk, void* dv, void* workspace,
+                         size_t workspace_bytes, void* stream) {
   cattn_status st = check_shape(B, H, T, D);
   if (st != CATTN_OK) return st;
   if (!(scale > 0.f) || !isfinite(scale)) return CATTN_ERR_INVALID_ARG;
@@ -408,7 +418,7 @@ cattn_status attn_bwd(const void* q, const void* k, const void* v, const void* o
     return CATTN_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
       !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
-      !aligned(lse, 4) || !aligned(workspace, 256))
+      !aligned(lse, 4) || !aligned(workspace, 256) || !aligned(o_lo, 16))
     return CATTN_ERR_INVALID_ARG;
   const int BH = B * H;
   if (workspace_bytes < ws_layout(BH, T, D).total) return CATTN_ERR_INVALID_ARG;
@@ -416,13 +426,25 @@ cattn_status attn_bwd(const void* q, const void* k, const void* v, const void* o
   if ((st = check_device(&dev)) != CATTN_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (D) {
-    case 16: return bwd_impl<16>(dev, q, k, v, o, lse, dout, scale, BH, T, dq, dk, dv, workspace, s);
-    case 32: return bwd_impl<32>(dev, q, k, v, o, lse, dout, scale, BH, T, dq, dk, dv, workspace, s);
-    case 64: return bwd_impl<64>(dev, q, k, v, o, lse, dout, scale, BH, T, dq, dk, dv, workspace, s);
+    case 16:
+      return bwd_impl<16>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, workspace, s);
+    case 32:
+      return bwd_impl<32>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, workspace, s);
+    case 64:
+      return bwd_impl<64>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, workspace, s);
     case 128:
-      return bwd_impl<128>(dev, q, k, v, o, lse, dout, scale, BH, T, dq, dk, dv, workspace, s);
+      return bwd_impl<128>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, workspace,
+                           s);
   }
   return CATTN_ERR_UNSUPPORTED;
+}
+
+cattn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                      const float* lse, const void* dout, float scale, int B, int H, int T, int D,
+                      void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  return attn_bwd_ex(q, k, v, o, nullptr, lse, dout, scale, B, H, T, D, dq, dk, dv, workspace,
+                     workspace_bytes, stream);
 }
 
 cattn_status cattn_get_device_status(int clear, void* stream) {

@@ -10,7 +10,9 @@
 // no T x T matrix is ever stored.
 //
 // Three kernels:
-//   bwd_pre_kernel   Delta = rowsum(dO * O) with 16-byte loads, LSE * log2(e)
+//   bwd_pre_kernel   Delta = rowsum(dO * O) with 16-byte loads (O + O_lo when
+//                    the forward's bf16 residual O_lo = O - bf16(O) is given,
+//                    which makes Delta exact to fp32 rounding), LSE * log2(e)
 //                    into a tile-padded vector, and zeroing of the fp32 dQ
 //                    accumulator.
 //   bwd_kernel       one CTA per (head, 128-key tile); loops over the query
@@ -18,6 +20,10 @@
 //                    TMEM and adding each dQ tile into the fp32 accumulator
 //                    with a TMA reduce-add.
 //   dq_convert_kernel dQ = bf16(scale * accumulator).
+//
+// Precision: P and dS enter the gradient MMAs as a bf16 hi/lo pair
+// (x = hi + lo to ~16 bits), so dV, dK and dQ carry fp32-level error instead
+// of bf16's 2^-9; the only bf16 rounding left is that of the outputs.
 #pragma once
 
 #include "sm100.cuh"
@@ -30,6 +36,7 @@ namespace cattn {
 
 struct PreParams {
   const __nv_bfloat16* o;
+  const __nv_bfloat16* o_lo;  // may be null
   const __nv_bfloat16* dout;
   const float* lse;      // may be null (no lse2 output)
   float* delta;          // (BH, row_stride)
@@ -67,14 +74,18 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
       const size_t off = (static_cast<size_t>(bh) * p.T + t) * D + sub * 8;
       const uint4 a = *reinterpret_cast<const uint4*>(p.o + off);
       const uint4 b = *reinterpret_cast<const uint4*>(p.dout + off);
+      uint4 c = make_uint4(0u, 0u, 0u, 0u);
+      if (p.o_lo != nullptr) c = *reinterpret_cast<const uint4*>(p.o_lo + off);
       const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
       const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+      const __nv_bfloat162* c2 = reinterpret_cast<const __nv_bfloat162*>(&c);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 fa = __bfloat1622float2(a2[e]);
         const float2 fb = __bfloat1622float2(b2[e]);
-        acc = fmaf(fa.x, fb.x, acc);
-        acc = fmaf(fa.y, fb.y, acc);
+        const float2 fc = __bfloat1622float2(c2[e]);
+        acc = fmaf(fa.x + fc.x, fb.x, acc);
+        acc = fmaf(fa.y + fc.y, fb.y, acc);
       }
     }
 #pragma unroll
@@ -116,6 +127,31 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float4* __restric
 // ---------------------------------------------------------------------------
 // Main backward kernel
 // ---------------------------------------------------------------------------
+//
+// One CTA per (head, 128-key tile j).  For each query tile i >= j:
+//   S^T  = K_j Q_i^T               (TMEM, fp32; lane = key)
+//   P^T  = exp2(S^T*scale*log2e - LSE2_i); masked on the diagonal tile;
+//          written back over S^T as bf16 hi/lo pairs
+//   dP^T = V_j dO_i^T              (TMEM, fp32)
+//   dS^T = P^T * (dP^T - Delta_i); written back over dP^T as hi/lo pairs,
+//          and (as dS) to shared memory for the dQ MMA
+//   dV  += P^T_hi dO_i + P^T_lo dO_i        (A from TMEM)
+//   dK  += dS^T_hi Q_i + dS^T_lo Q_i        (A from TMEM)
+//   dQ_i = dS_hi K_j + dS_lo K_j            (A from shared, MN-major),
+//          drained to shared memory and added into the fp32 accumulator
+//          with a TMA reduce-add.
+//
+// Warp roles (320 threads):
+//   warps 0-7  compute: warp w serves TMEM lanes 32*(w%4).. (key rows) and
+//              query columns 64*(w/4) .. +64 of the tile; they also drain
+//              dQ and write dK, dV at the end.
+//   warp 8     TMA producer: K_j, V_j once; Q_i with the LSE2 and Delta
+//              vectors through a 2-stage ring (freed after dK(i), which
+//              follows every read of them), dO_i through a 2-stage
+//              (D <= 64) or 1-stage ring (freed after dV(i)).
+//   warp 9     MMA issuer and TMEM owner.  Order per iteration:
+//              dV(i), S(i+1), dK(i), dQ(i), dP(i+1) -- so S(i+1) runs while
+//              dS(i) is computed and dK/dQ(i), dP(i+1) while P(i+1) is.
 
 struct BwdParams {
   const float* lse2;   // (BH, T_pad) LSE * log2(e); +inf on padding rows
@@ -135,27 +171,29 @@ struct BwdCfg {
   static constexpr int NCB = D / CB;
   static constexpr int BLOCK_BYTES = 128 * RB;
   static constexpr int TILE_BYTES = 128 * D * 2;
-  static constexpr int ST = D <= 64 ? 2 : 1;        // Q/dO ring depth
+  static constexpr int QST = 2;                     // Q ring depth
+  static constexpr int DOST = D <= 64 ? 2 : 1;      // dO ring depth
   static constexpr uint32_t SW = swizzle_code(RB);
-  // fp32 dQ staging: blocks of [128 rows][CBQ floats], swizzled by row bytes
+  // fp32 dQ staging (in the dS buffers): blocks of [128 rows][CBQ floats]
   static constexpr int CBQ = D < 32 ? D : 32;
   static constexpr int RBQ = CBQ * 4;
-  static constexpr int QCHUNK = D < 64 ? D : 64;    // dQ columns staged at a time
-  static constexpr int QCHUNK_BYTES = 128 * QCHUNK * 4;
   // shared memory map
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE_BYTES;
   static constexpr int OFF_Q = OFF_V + TILE_BYTES;
-  static constexpr int OFF_DO = OFF_Q + ST * TILE_BYTES;
-  static constexpr int OFF_PT = OFF_DO + ST * TILE_BYTES;   // [2][128 keys][64 queries] bf16
-  static constexpr int OFF_DST = OFF_PT + 32768;            // same layout, dS^T
-  static constexpr int OFF_DQ = OFF_DST + 32768;
-  static constexpr int OFF_LSE = OFF_DQ + QCHUNK_BYTES;     // [ST][128] fp32
-  static constexpr int OFF_DELTA = OFF_LSE + ST * 512;
-  static constexpr int OFF_BAR = OFF_DELTA + ST * 512;
+  static constexpr int OFF_DO = OFF_Q + QST * TILE_BYTES;
+  static constexpr int OFF_DSH = OFF_DO + DOST * TILE_BYTES;  // [2][128 keys][64 q] bf16
+  static constexpr int OFF_DSL = OFF_DSH + 32768;
+  static constexpr int OFF_LSE = OFF_DSL + 32768;             // [QST][128] fp32
+  static constexpr int OFF_DELTA = OFF_LSE + QST * 512;       // [QST][128] fp32
+  static constexpr int OFF_BAR = OFF_DELTA + QST * 512;
   static constexpr int NUM_BARS = 24;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
+  static constexpr int SMEM_USED = OFF_MISC + 64;
+  static constexpr int SMEM_BYTES =
+      SMEM_USED + 1024 <= kMaxDynSmem ? SMEM_USED + 1024 : SMEM_USED;
+  static_assert(SMEM_USED <= kMaxDynSmem, "shared memory layout too large");
+  static_assert(128 * D * 4 <= 65536, "dQ staging must fit the dS buffers");
   // TMEM columns
   static constexpr bool ALIAS_DQ = 256 + 3 * D > 512;
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
@@ -165,9 +203,9 @@ struct BwdCfg {
 };
 
 enum : int {
-  BB_KV = 0, BB_QFULL = 1, BB_DOFULL = 3, BB_QDOEMPTY = 5, BB_SFULL = 7, BB_STFREE = 8,
-  BB_DPFULL = 9, BB_DPTFREE = 10, BB_PTFULL = 11, BB_PTFREE = 12, BB_DSFULL = 13,
-  BB_DSFREE = 14, BB_DQFULL = 15, BB_DQEMPTY = 16, BB_DRAIN = 17
+  BB_KV = 0, BB_QFULL = 1, BB_QEMPTY = 3, BB_DOFULL = 5, BB_DOEMPTY = 7, BB_SFULL = 9,
+  BB_DPFULL = 10, BB_PFULL = 11, BB_PTDONE = 12, BB_DSFULL = 13, BB_DSDONE = 14,
+  BB_DQFULL = 15, BB_DQEMPTY = 16, BB_DKDONE = 17, BB_DRAIN = 18
 };
 
 template <int D>
@@ -178,11 +216,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
            const __grid_constant__ CUtensorMap tmDQacc, const BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = aligned_smem(smem_raw, C::SMEM_USED);
+  if (smem == nullptr) return;  // uniform over the CTA: nothing touched yet
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sK = sbase + C::OFF_K, sV = sbase + C::OFF_V;
-  const uint32_t sPt = sbase + C::OFF_PT, sdSt = sbase + C::OFF_DST, sDQ = sbase + C::OFF_DQ;
+  const uint32_t sDSH = sbase + C::OFF_DSH, sDSL = sbase + C::OFF_DSL;
   auto bar = [&](int i) { return sbase + C::OFF_BAR + 8u * i; };
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
@@ -198,21 +236,23 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(bar(BB_KV), 1);
-    for (int s = 0; s < C::ST; ++s) {
+    for (int s = 0; s < C::QST; ++s) {
       mbar_init(bar(BB_QFULL + s), 1);
+      mbar_init(bar(BB_QEMPTY + s), 1);
+    }
+    for (int s = 0; s < C::DOST; ++s) {
       mbar_init(bar(BB_DOFULL + s), 1);
-      mbar_init(bar(BB_QDOEMPTY + s), 1);
+      mbar_init(bar(BB_DOEMPTY + s), 1);
     }
     mbar_init(bar(BB_SFULL), 1);
-    mbar_init(bar(BB_STFREE), 128);
     mbar_init(bar(BB_DPFULL), 1);
-    mbar_init(bar(BB_DPTFREE), 128);
-    mbar_init(bar(BB_PTFULL), 128);
-    mbar_init(bar(BB_PTFREE), 1);
-    mbar_init(bar(BB_DSFULL), 128);
-    mbar_init(bar(BB_DSFREE), 1);
+    mbar_init(bar(BB_PFULL), 256);
+    mbar_init(bar(BB_PTDONE), 1);
+    mbar_init(bar(BB_DSFULL), 256);
+    mbar_init(bar(BB_DSDONE), 1);
     mbar_init(bar(BB_DQFULL), 1);
-    mbar_init(bar(BB_DQEMPTY), 128);
+    mbar_init(bar(BB_DQEMPTY), 256);
+    mbar_init(bar(BB_DKDONE), 1);
     mbar_init(bar(BB_DRAIN), 1);
     fence_mbar_init();
   }
@@ -237,52 +277,52 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         tma_load_3d(sK + b * C::BLOCK_BYTES, &tmK, bar(BB_KV), b * C::CB, kt * 128, bh);
         tma_load_3d(sV + b * C::BLOCK_BYTES, &tmV, bar(BB_KV), b * C::CB, kt * 128, bh);
       }
-      int n_issued = 0;
+      int nq = 0, ndo = 0;  // loads issued
       for (int i = 0; i < n_iter; ++i) {
-        const int st = i % C::ST;
         const int qi = kt + i;
-        if (i >= C::ST) wait1(w, bar(BB_QDOEMPTY + st), ((i / C::ST) - 1) & 1, 1);
-        if (*abort_flag) break;
-        n_issued = i + 1;
-        const uint32_t sQ = sbase + C::OFF_Q + st * C::TILE_BYTES;
-        const uint32_t sDO = sbase + C::OFF_DO + st * C::TILE_BYTES;
         const size_t vec = static_cast<size_t>(bh) * p.T_pad + static_cast<size_t>(qi) * 128;
-        mbar_arrive_expect_tx(bar(BB_QFULL + st), C::TILE_BYTES + 512);
+        const int qs = i % C::QST;
+        if (i >= C::QST) wait1(w, bar(BB_QEMPTY + qs), ((i / C::QST) - 1) & 1, 1);
+        if (*abort_flag) break;
+        const uint32_t sQ = sbase + C::OFF_Q + qs * C::TILE_BYTES;
+        mbar_arrive_expect_tx(bar(BB_QFULL + qs), C::TILE_BYTES + 1024);
         for (int b = 0; b < C::NCB; ++b)
-          tma_load_3d(sQ + b * C::BLOCK_BYTES, &tmQ, bar(BB_QFULL + st), b * C::CB, qi * 128, bh);
-        bulk_load(sbase + C::OFF_LSE + st * 512, p.lse2 + vec, 512, bar(BB_QFULL + st));
-        mbar_arrive_expect_tx(bar(BB_DOFULL + st), C::TILE_BYTES + 512);
+          tma_load_3d(sQ + b * C::BLOCK_BYTES, &tmQ, bar(BB_QFULL + qs), b * C::CB, qi * 128, bh);
+        bulk_load(sbase + C::OFF_LSE + qs * 512, p.lse2 + vec, 512, bar(BB_QFULL + qs));
+        bulk_load(sbase + C::OFF_DELTA + qs * 512, p.delta + vec, 512, bar(BB_QFULL + qs));
+        nq = i + 1;
+        const int ds = i % C::DOST;
+        if (i >= C::DOST) wait1(w, bar(BB_DOEMPTY + ds), ((i / C::DOST) - 1) & 1, 2);
+        if (*abort_flag) break;
+        const uint32_t sDO = sbase + C::OFF_DO + ds * C::TILE_BYTES;
+        mbar_arrive_expect_tx(bar(BB_DOFULL + ds), C::TILE_BYTES);
         for (int b = 0; b < C::NCB; ++b)
-          tma_load_3d(sDO + b * C::BLOCK_BYTES, &tmDO, bar(BB_DOFULL + st), b * C::CB, qi * 128, bh);
-        bulk_load(sbase + C::OFF_DELTA + st * 512, p.delta + vec, 512, bar(BB_DOFULL + st));
+          tma_load_3d(sDO + b * C::BLOCK_BYTES, &tmDO, bar(BB_DOFULL + ds), b * C::CB, qi * 128,
+                      bh);
+        ndo = i + 1;
       }
       if (*abort_flag) {
+        // wait (bounded, ignoring the abort flag) for loads nobody consumed
         int zero = 0;
         WaitCtx wd{p.timeout_ns, &zero, 2u};
         wait1(wd, bar(BB_KV), 0, 20);
-        for (int i = (n_issued > C::ST ? n_issued - C::ST : 0); i < n_issued; ++i) {
-          const int st = i % C::ST;
-          wait1(wd, bar(BB_QFULL + st), (i / C::ST) & 1, 21);
-          wait1(wd, bar(BB_DOFULL + st), (i / C::ST) & 1, 22);
-        }
+        for (int i = (nq > C::QST ? nq - C::QST : 0); i < nq; ++i)
+          wait1(wd, bar(BB_QFULL + i % C::QST), (i / C::QST) & 1, 21);
+        for (int i = (ndo > C::DOST ? ndo - C::DOST : 0); i < ndo; ++i)
+          wait1(wd, bar(BB_DOFULL + i % C::DOST), (i / C::DOST) & 1, 22);
       }
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idSS = idesc_bf16(128, 128, 0, 0);  // S^T, dP^T
-      constexpr uint32_t idKD = idesc_bf16(128, D, 0, 1);    // dV, dK: A K-major, B MN-major
+      constexpr uint32_t idKD = idesc_bf16(128, D, 0, 1);    // dV, dK: B MN-major
       constexpr uint32_t idQ = idesc_bf16(128, D, 1, 1);     // dQ: A (dS) MN-major
-      wait1(w, bar(BB_KV), 0, 2);
-      for (int i = 0; i < n_iter; ++i) {
-        const int st = i % C::ST;
-        const uint32_t ph = (i / C::ST) & 1;
-        const uint32_t sQ = sbase + C::OFF_Q + st * C::TILE_BYTES;
-        const uint32_t sDO = sbase + C::OFF_DO + st * C::TILE_BYTES;
-        // S^T = K Q^T  (M = keys, N = queries, K = D)
-        wait1(w, bar(BB_QFULL + st), ph, 3);
-        if (i >= 1) wait1(w, bar(BB_STFREE), (i - 1) & 1, 4);
+      auto issue_s = [&](int i) {  // S^T = K Q_i^T
+        const int qs = i % C::QST;
+        wait1(w, bar(BB_QFULL + qs), (i / C::QST) & 1, 3);
         tc_fence_after();
+        const uint32_t sQ = sbase + C::OFF_Q + qs * C::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int blk = (kk * 16) / C::CB;
@@ -293,11 +333,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                  kk > 0 ? 1u : 0u);
         }
         mma_commit(bar(BB_SFULL));
-        // dP^T = V dO^T
-        wait1(w, bar(BB_DOFULL + st), ph, 5);
-        if (i >= 1) wait1(w, bar(BB_DPTFREE), (i - 1) & 1, 6);
-        if (C::ALIAS_DQ && i >= 1) wait1(w, bar(BB_DQEMPTY), (i - 1) & 1, 7);
+      };
+      auto issue_dp = [&](int i) {  // dP^T = V dO_i^T
+        const int ds = i % C::DOST;
+        wait1(w, bar(BB_DOFULL + ds), (i / C::DOST) & 1, 4);
         tc_fence_after();
+        const uint32_t sDO = sbase + C::OFF_DO + ds * C::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int blk = (kk * 16) / C::CB;
@@ -308,216 +349,262 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                  kk > 0 ? 1u : 0u);
         }
         mma_commit(bar(BB_DPFULL));
-        // dV += P^T dO  (M = keys, K = queries, N = D)
-        wait1(w, bar(BB_PTFULL), i & 1, 8);
+      };
+      wait1(w, bar(BB_KV), 0, 5);
+      issue_s(0);
+      issue_dp(0);
+      for (int i = 0; i < n_iter; ++i) {
+        const int qs = i % C::QST;
+        const int ds = i % C::DOST;
+        const uint32_t sQ = sbase + C::OFF_Q + qs * C::TILE_BYTES;
+        const uint32_t sDO = sbase + C::OFF_DO + ds * C::TILE_BYTES;
+        // dV += P^T dO_i  (A = P^T hi/lo in TMEM over S^T; K = 128 queries)
+        wait1(w, bar(BB_PFULL), i & 1, 6);
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          mma_ss(tbase + C::COL_DV, smem_desc(sPt + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, 2),
-                 smem_desc(sDO + kk * 16 * C::RB, C::BLOCK_BYTES, 8 * C::RB, C::SW), idKD,
-                 (i > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t acol = C::COL_S + (kk >> 2) * 64 + (kk & 3) * 8;
+          const uint64_t b = smem_desc(sDO + kk * 16 * C::RB, C::BLOCK_BYTES, 8 * C::RB, C::SW);
+          mma_ts(tbase + C::COL_DV, tbase + acol, b, idKD, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tbase + C::COL_DV, tbase + acol + 32, b, idKD, 1u);
         }
-        mma_commit(bar(BB_PTFREE));
-        // dK += dS^T Q ; dQ = dS K
-        wait1(w, bar(BB_DSFULL), i & 1, 9);
-        if (!C::ALIAS_DQ && i >= 1) wait1(w, bar(BB_DQEMPTY), (i - 1) & 1, 10);
+        mma_commit(bar(BB_PTDONE));
+        mma_commit(bar(BB_DOEMPTY + ds));
+        // S(i+1) overwrites P^T(i): only after dV(i) has read it
+        if (i + 1 < n_iter) {
+          wait1(w, bar(BB_PTDONE), i & 1, 7);
+          issue_s(i + 1);
+        }
+        // dK += dS^T Q_i (A = dS^T hi/lo in TMEM over dP^T)
+        wait1(w, bar(BB_DSFULL), i & 1, 8);
+        if (!C::ALIAS_DQ && i >= 1) wait1(w, bar(BB_DQEMPTY), (i - 1) & 1, 9);
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          mma_ss(tbase + C::COL_DK,
-                 smem_desc(sdSt + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, 2),
-                 smem_desc(sQ + kk * 16 * C::RB, C::BLOCK_BYTES, 8 * C::RB, C::SW), idKD,
-                 (i > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t acol = C::COL_DP + (kk >> 2) * 64 + (kk & 3) * 8;
+          const uint64_t b = smem_desc(sQ + kk * 16 * C::RB, C::BLOCK_BYTES, 8 * C::RB, C::SW);
+          mma_ts(tbase + C::COL_DK, tbase + acol, b, idKD, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tbase + C::COL_DK, tbase + acol + 32, b, idKD, 1u);
         }
+        mma_commit(bar(BB_QEMPTY + qs));
+        if (C::ALIAS_DQ) {  // dQ below overwrites the dS^T that dK just read
+          mma_commit(bar(BB_DKDONE));
+          wait1(w, bar(BB_DKDONE), i & 1, 10);
+          tc_fence_after();
+        }
+        // dQ_i = dS K  (A = dS hi/lo in shared, MN-major; K = 128 keys)
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // K = 128 keys, 16 per MMA
-          mma_ss(tbase + C::COL_DQ, smem_desc(sdSt + kk * 2048, 16384, 1024, 2),
-                 smem_desc(sK + kk * 16 * C::RB, C::BLOCK_BYTES, 8 * C::RB, C::SW), idQ,
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t b = smem_desc(sK + kk * 16 * C::RB, C::BLOCK_BYTES, 8 * C::RB, C::SW);
+          mma_ss(tbase + C::COL_DQ, smem_desc(sDSH + kk * 2048, 16384, 1024, 2), b, idQ,
                  kk > 0 ? 1u : 0u);
+          mma_ss(tbase + C::COL_DQ, smem_desc(sDSL + kk * 2048, 16384, 1024, 2), b, idQ, 1u);
         }
+        mma_commit(bar(BB_DSDONE));
         mma_commit(bar(BB_DQFULL));
-        mma_commit(bar(BB_DSFREE));
-        mma_commit(bar(BB_QDOEMPTY + st));
+        // dP(i+1) overwrites dS^T(i) (and, aliased, dQ(i))
+        if (i + 1 < n_iter) {
+          wait1(w, bar(BB_DSDONE), i & 1, 11);
+          if (C::ALIAS_DQ) wait1(w, bar(BB_DQEMPTY), i & 1, 12);
+          issue_dp(i + 1);
+        }
       }
       mma_commit(bar(BB_DRAIN));
       int zero = 0;
       WaitCtx wd{p.timeout_ns, &zero, 2u};
-      wait1(wd, bar(BB_DRAIN), 0, 11);
-    }
-  } else if (warp < 4) {
-    // ------------------------------------------------- P and dS (row = key)
-    const int r = threadIdx.x;                   // key row in tile == TMEM lane
-    const uint32_t lane_base = (warp * 32) << 16;
-    const float sl2 = p.scale_log2;
-    float pr[128];
-    for (int i = 0; i < n_iter; ++i) {
-      const int st = i % C::ST;
-      const uint32_t ph = (i / C::ST) & 1;
-      wait_warp(w, bar(BB_SFULL), i & 1, 12);
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tbase + lane_base + C::COL_S + c * 32, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) pr[c * 32 + e] = __uint_as_float(v[e]);
-      }
-      tc_fence_before();
-      mbar_arrive(bar(BB_STFREE));
-      wait_warp(w, bar(BB_QFULL + st), ph, 13);  // makes the LSE vector visible
-      const uint32_t sL = sbase + C::OFF_LSE + st * 512;
-#pragma unroll
-      for (int c = 0; c < 128; c += 4) {
-        float l0, l1, l2, l3;
-        ld_shared_v4f(sL + c * 4, l0, l1, l2, l3);
-        pr[c] = ex2(fmaf(pr[c], sl2, -l0));
-        pr[c + 1] = ex2(fmaf(pr[c + 1], sl2, -l1));
-        pr[c + 2] = ex2(fmaf(pr[c + 2], sl2, -l2));
-        pr[c + 3] = ex2(fmaf(pr[c + 3], sl2, -l3));
-      }
-      if (i == 0) {  // diagonal tile: query c sees key r only if r <= c
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c < r) pr[c] = 0.f;
-      }
-      if (i >= 1) wait_warp(w, bar(BB_PTFREE), (i - 1) & 1, 14);
-#pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        const int c0 = ch * 8;
-        st_shared_v4(sPt + (c0 >> 6) * 16384 + swz<128>(r * 128 + ((c0 & 63) >> 3) * 16),
-                     pack_bf16(pr[c0], pr[c0 + 1]), pack_bf16(pr[c0 + 2], pr[c0 + 3]),
-                     pack_bf16(pr[c0 + 4], pr[c0 + 5]), pack_bf16(pr[c0 + 6], pr[c0 + 7]));
-      }
-      fence_async_smem();
-      mbar_arrive(bar(BB_PTFULL));
-
-      wait_warp(w, bar(BB_DPFULL), i & 1, 15);
-      tc_fence_after();
-      wait_warp(w, bar(BB_DOFULL + st), ph, 16);  // makes the Delta vector visible
-      if (i >= 1) wait_warp(w, bar(BB_DSFREE), (i - 1) & 1, 17);
-      const uint32_t sD = sbase + C::OFF_DELTA + st * 512;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tbase + lane_base + C::COL_DP + c * 32, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const int c0 = c * 32 + ch * 8;
-          float d[8];
-          ld_shared_v4f(sD + c0 * 4, d[0], d[1], d[2], d[3]);
-          ld_shared_v4f(sD + c0 * 4 + 16, d[4], d[5], d[6], d[7]);
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float a0 = pr[c0 + 2 * e] * (__uint_as_float(v[ch * 8 + 2 * e]) - d[2 * e]);
-            const float a1 =
-                pr[c0 + 2 * e + 1] * (__uint_as_float(v[ch * 8 + 2 * e + 1]) - d[2 * e + 1]);
-            pk[e] = pack_bf16(a0, a1);
-          }
-          st_shared_v4(sdSt + (c0 >> 6) * 16384 + swz<128>(r * 128 + ((c0 & 63) >> 3) * 16),
-                       pk[0], pk[1], pk[2], pk[3]);
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(bar(BB_DPTFREE));
-      fence_async_smem();
-      mbar_arrive(bar(BB_DSFULL));
-    }
-
-    // ------------------------------------------------ dK, dV epilogue
-    wait_warp(w, bar(BB_DQFULL), (n_iter - 1) & 1, 18);  // every MMA has completed
-    tc_fence_after();
-#pragma unroll
-    for (int which = 0; which < 2; ++which) {  // 0: dV -> sPt, 1: dK -> sdSt
-      const uint32_t col = tbase + lane_base + (which ? C::COL_DK : C::COL_DV);
-      const uint32_t dst = which ? sdSt : sPt;
-      const float mul = which ? p.scale : 1.f;
-#pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
-        uint32_t v[16];
-        tmem_ld16(col + c * 16, v);
-        tmem_wait_ld();
-        uint32_t pk[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          pk[e] = pack_bf16(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
-        const int d0 = c * 16;
-        const int blk = d0 / C::CB;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int dd = (d0 % C::CB) + h * 8;
-          st_shared_v4(dst + blk * C::BLOCK_BYTES + swz<C::RB>(r * C::RB + dd * 2), pk[4 * h],
-                       pk[4 * h + 1], pk[4 * h + 2], pk[4 * h + 3]);
-        }
-      }
-    }
-    tc_fence_before();
-    fence_async_smem();
-    named_bar_sync(1, 128);
-    if (threadIdx.x == 0 && !*abort_flag) {
-      for (int b = 0; b < C::NCB; ++b) {
-        tma_store_3d(&tmDV, sPt + b * C::BLOCK_BYTES, b * C::CB, kt * 128, bh);
-        tma_store_3d(&tmDK, sdSt + b * C::BLOCK_BYTES, b * C::CB, kt * 128, bh);
-      }
-      bulk_commit();
-      bulk_wait0();
+      wait1(wd, bar(BB_DRAIN), 0, 13);
     }
   } else {
-    // ------------------------------------------------ dQ drain (row = query)
-    const int r = threadIdx.x - 128;
-    const uint32_t lane_base = ((warp - 4) * 32) << 16;
-    const bool leader = (r == 0);
-    for (int i = 0; i < n_iter; ++i) {
-      const int qi = kt + i;
-      wait_warp(w, bar(BB_DQFULL), i & 1, 19);
+    // ------------------------------------------- compute warps (row = key)
+    const int quarter = warp & 3;
+    const int h = warp >> 2;                     // query half of the tile
+    const int r = quarter * 32 + lane;           // key row == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const float sl2 = p.scale_log2;
+    const bool leader = threadIdx.x == 0;
+
+    // dQ(t) drain: TMEM (lane = query row) -> fp32 staging in the dS
+    // buffers -> TMA reduce-add into the accumulator.
+    auto drain_dq = [&](int t) {
+      wait_warp(w, bar(BB_DQFULL), t & 1, 14);
       tc_fence_after();
-      float acc[D];
-      if constexpr (D >= 32) {
+      constexpr int NC = D / 2;                  // columns per thread
+      float acc[NC];
+      const uint32_t src = tbase + lane_base + C::COL_DQ + h * NC;
+      if constexpr (NC >= 32) {
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < NC / 32; ++c) {
           uint32_t v[32];
-          tmem_ld32(tbase + lane_base + C::COL_DQ + c * 32, v);
+          tmem_ld32(src + c * 32, v);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) acc[c * 32 + e] = __uint_as_float(v[e]);
         }
-      } else {
+      } else if constexpr (NC == 16) {
         uint32_t v[16];
-        tmem_ld16(tbase + lane_base + C::COL_DQ, v);
+        tmem_ld16(src, v);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(v[e]);
+      } else {
+        uint32_t v[8];
+        tmem_ld8(src, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = __uint_as_float(v[e]);
       }
       tc_fence_before();
       mbar_arrive(bar(BB_DQEMPTY));
+      // staging: blocks of [128 rows][CBQ floats], swizzled
 #pragma unroll
-      for (int ch = 0; ch < D / C::QCHUNK; ++ch) {
-        // stage [128][QCHUNK] fp32 as QCHUNK/CBQ swizzled blocks
+      for (int e = 0; e < NC; e += 4) {
+        const int f = h * NC + e;
+        const int blk = f / C::CBQ;
+        const int within = (f % C::CBQ) * 4;
+        st_shared_v4(sDSH + blk * 128 * C::RBQ + swz<C::RBQ>(r * C::RBQ + within),
+                     __float_as_uint(acc[e]), __float_as_uint(acc[e + 1]),
+                     __float_as_uint(acc[e + 2]), __float_as_uint(acc[e + 3]));
+      }
+      fence_async_smem();
+      named_bar_sync(1, 256);
+      if (leader && !*abort_flag) {
 #pragma unroll
-        for (int e = 0; e < C::QCHUNK; e += 4) {
-          const int blk = e / C::CBQ;
-          const int within = (e % C::CBQ) * 4;
-          const float* a = &acc[ch * C::QCHUNK + e];
-          st_shared_v4(sDQ + blk * 128 * C::RBQ + swz<C::RBQ>(r * C::RBQ + within),
-                       __float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]),
-                       __float_as_uint(a[3]));
+        for (int blk = 0; blk < D / C::CBQ; ++blk)
+          tma_reduce_add_3d(&tmDQacc, sDSH + blk * 128 * C::RBQ, blk * C::CBQ, (kt + t) * 128,
+                            bh);
+        bulk_commit();
+      }
+    };
+    // the dS buffers may be rewritten once the reduce has read them
+    auto staging_free = [&]() {
+      if (leader) bulk_wait_read0();
+      named_bar_sync(1, 256);
+    };
+
+    float pv[64];
+    for (int i = 0; i < n_iter; ++i) {
+      const int qs = i % C::QST;
+      // ---- P phase
+      wait_warp(w, bar(BB_SFULL), i & 1, 15);
+      tc_fence_after();
+      {
+        uint32_t v[32];
+        tmem_ld32(tbase + lane_base + C::COL_S + h * 64, v);
+        uint32_t u[32];
+        tmem_ld32(tbase + lane_base + C::COL_S + h * 64 + 32, u);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          pv[e] = __uint_as_float(v[e]);
+          pv[32 + e] = __uint_as_float(u[e]);
         }
-        fence_async_smem();
-        named_bar_sync(2, 128);
-        if (leader && !*abort_flag) {
+      }
+      wait_warp(w, bar(BB_QFULL + qs), (i / C::QST) & 1, 16);  // LSE2 visibility
+      const uint32_t sL = sbase + C::OFF_LSE + qs * 512 + h * 256;
 #pragma unroll
-          for (int blk = 0; blk < C::QCHUNK / C::CBQ; ++blk)
-            tma_reduce_add_3d(&tmDQacc, sDQ + blk * 128 * C::RBQ,
-                              ch * C::QCHUNK + blk * C::CBQ, qi * 128, bh);
-          bulk_commit();
-          bulk_wait_read0();
+      for (int c = 0; c < 64; c += 4) {
+        float l0, l1, l2, l3;
+        ld_shared_v4f(sL + c * 4, l0, l1, l2, l3);
+        pv[c] = ex2(fmaf(pv[c], sl2, -l0));
+        pv[c + 1] = ex2(fmaf(pv[c + 1], sl2, -l1));
+        pv[c + 2] = ex2(fmaf(pv[c + 2], sl2, -l2));
+        pv[c + 3] = ex2(fmaf(pv[c + 3], sl2, -l3));
+      }
+      if (i == 0) {  // diagonal tile: query (64h + c) sees key r only if r <= query
+        const int lim = r - h * 64;
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (c < lim) pv[c] = 0.f;
+      }
+      {
+        uint32_t hi[32], lo[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) split_bf16x2(pv[2 * e], pv[2 * e + 1], hi[e], lo[e]);
+        tmem_st32(tbase + lane_base + C::COL_S + h * 64, hi);
+        tmem_st32(tbase + lane_base + C::COL_S + h * 64 + 32, lo);
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      mbar_arrive(bar(BB_PFULL));
+
+      // ---- dQ of the previous query tile (its MMA ran during this P phase)
+      if (i >= 1) drain_dq(i - 1);
+
+      // ---- dS phase
+      wait_warp(w, bar(BB_DPFULL), i & 1, 17);
+      tc_fence_after();
+      // (the Delta vector arrived with Q_i, whose barrier was waited above)
+      const uint32_t sD = sbase + C::OFF_DELTA + qs * 512 + h * 256;
+      uint32_t hi[32], lo[32];
+#pragma unroll
+      for (int c2 = 0; c2 < 2; ++c2) {
+        uint32_t v[32];
+        tmem_ld32(tbase + lane_base + C::COL_DP + h * 64 + c2 * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          float d0, d1, d2, d3;
+          ld_shared_v4f(sD + (c2 * 32 + e) * 4, d0, d1, d2, d3);
+          const float s0 = pv[c2 * 32 + e] * (__uint_as_float(v[e]) - d0);
+          const float s1 = pv[c2 * 32 + e + 1] * (__uint_as_float(v[e + 1]) - d1);
+          const float s2 = pv[c2 * 32 + e + 2] * (__uint_as_float(v[e + 2]) - d2);
+          const float s3 = pv[c2 * 32 + e + 3] * (__uint_as_float(v[e + 3]) - d3);
+          split_bf16x2(s0, s1, hi[c2 * 16 + e / 2], lo[c2 * 16 + e / 2]);
+          split_bf16x2(s2, s3, hi[c2 * 16 + e / 2 + 1], lo[c2 * 16 + e / 2 + 1]);
         }
-        named_bar_sync(2, 128);
+      }
+      tmem_st32(tbase + lane_base + C::COL_DP + h * 64, hi);
+      tmem_st32(tbase + lane_base + C::COL_DP + h * 64 + 32, lo);
+      // dS (hi, lo) -> shared for the dQ MMA: [2][128 keys][64 queries]
+      if (i >= 1) staging_free();
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        const uint32_t off = h * 16384 + swz<128>(r * 128 + ch * 16);
+        st_shared_v4(sDSH + off, hi[4 * ch], hi[4 * ch + 1], hi[4 * ch + 2], hi[4 * ch + 3]);
+        st_shared_v4(sDSL + off, lo[4 * ch], lo[4 * ch + 1], lo[4 * ch + 2], lo[4 * ch + 3]);
+      }
+      fence_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(BB_DSFULL));
+    }
+    drain_dq(n_iter - 1);  // waits for the last MMAs: everything is complete
+    staging_free();
+
+    // ---- dK, dV epilogue: TMEM -> bf16 -> shared (dS buffers) -> TMA store
+    constexpr int NC = D / 2;
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {  // 0: dV -> sDSH, 1: dK -> sDSL
+      const uint32_t col = tbase + lane_base + (which ? C::COL_DK : C::COL_DV) + h * NC;
+      const uint32_t dst = which ? sDSL : sDSH;
+      const float mul = which ? p.scale : 1.f;
+#pragma unroll
+      for (int c = 0; c < NC; c += 8) {
+        uint32_t v[8];
+        tmem_ld8(col + c, v);
+        tmem_wait_ld();
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          pk[e] = pack_bf16(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+        const int d0 = h * NC + c;
+        const int blk = d0 / C::CB;
+        const int dd = d0 % C::CB;
+        st_shared_v4(dst + blk * C::BLOCK_BYTES + swz<C::RB>(r * C::RB + dd * 2), pk[0], pk[1],
+                     pk[2], pk[3]);
       }
     }
-    if (leader) bulk_wait0();
+    tc_fence_before();
+    fence_async_smem();
+    named_bar_sync(1, 256);
+    if (leader && !*abort_flag) {
+      for (int b = 0; b < C::NCB; ++b) {
+        tma_store_3d(&tmDV, sDSH + b * C::BLOCK_BYTES, b * C::CB, kt * 128, bh);
+        tma_store_3d(&tmDK, sDSL + b * C::BLOCK_BYTES, b * C::CB, kt * 128, bh);
+      }
+      bulk_commit();
+    }
+    if (leader) bulk_wait0();  // the dQ reduces and the stores have completed
   }
 
   tc_fence_before();

@@ -33,6 +33,7 @@ namespace cattn {
 
 struct FwdParams {
   float* lse;          // (BH, T) fp32 out
+  int write_o_lo;      // also write O_lo = bf16(O - bf16(O)) through tmOlo
   int T;
   int n_qtiles;
   float scale_log2;    // scale * log2(e)
@@ -60,6 +61,7 @@ struct FwdCfg {
   static constexpr int SMEM_USED = OFF_MISC + 64;
   // keep one CTA per SM: the TMEM allocation below takes all 512 columns
   static constexpr int SMEM_BYTES = (SMEM_USED < 120 * 1024 ? 120 * 1024 : SMEM_USED) + 1024;
+  static_assert(SMEM_BYTES <= kMaxDynSmem, "shared memory layout too large");
   // TMEM columns
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O = 256;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -76,12 +78,12 @@ template <int D>
 __global__ void __launch_bounds__(192, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-           const FwdParams p) {
+           const __grid_constant__ CUtensorMap tmOlo, const FwdParams p) {
   using C = FwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte align the working area (swizzle atoms)
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = aligned_smem(smem_raw, C::SMEM_USED);
+  if (smem == nullptr) return;  // uniform over the CTA: nothing touched yet
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase + C::OFF_Q;
   const uint32_t sP = sbase + C::OFF_P;
@@ -293,31 +295,39 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     tc_fence_after();
     const float inv_l = 1.f / l;
     const uint32_t ocol = tbase + lane_base + C::COL_O;
-    // O staging reuses the Q tile (every MMA that read Q has completed)
+    // O staging reuses the Q tile and O_lo staging the first K stage: every
+    // MMA that read them has completed and no load is in flight.
+    const uint32_t sOlo = sbase + C::OFF_K;
 #pragma unroll
     for (int c = 0; c < D / 16; ++c) {
       uint32_t r[16];
       tmem_ld16(ocol + c * 16, r);
       tmem_wait_ld();
-      uint32_t pk[8];
+      uint32_t pk[8], lo[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e)
-        pk[e] = pack_bf16(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
+        split_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l,
+                     pk[e], lo[e]);
       const int d0 = c * 16;
       const int blk = d0 / C::CB;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int dd = (d0 % C::CB) + h * 8;
-        const uint32_t addr = sQ + blk * C::BLOCK_BYTES + swz<C::RB>(row * C::RB + dd * 2);
-        st_shared_v4(addr, pk[4 * h], pk[4 * h + 1], pk[4 * h + 2], pk[4 * h + 3]);
+        const uint32_t off = blk * C::BLOCK_BYTES + swz<C::RB>(row * C::RB + dd * 2);
+        st_shared_v4(sQ + off, pk[4 * h], pk[4 * h + 1], pk[4 * h + 2], pk[4 * h + 3]);
+        if (p.write_o_lo)
+          st_shared_v4(sOlo + off, lo[4 * h], lo[4 * h + 1], lo[4 * h + 2], lo[4 * h + 3]);
       }
     }
     tc_fence_before();
     fence_async_smem();
     named_bar_sync(1, 128);
     if (threadIdx.x == 0 && !*abort_flag) {
-      for (int b = 0; b < C::NCB; ++b)
+      for (int b = 0; b < C::NCB; ++b) {
         tma_store_3d(&tmO, sQ + b * C::BLOCK_BYTES, b * C::CB, qt * C::BM, bh);
+        if (p.write_o_lo)
+          tma_store_3d(&tmOlo, sOlo + b * C::BLOCK_BYTES, b * C::CB, qt * C::BM, bh);
+      }
       bulk_commit();
       bulk_wait_read0();
     }

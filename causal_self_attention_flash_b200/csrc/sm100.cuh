@@ -34,6 +34,27 @@ __device__ __forceinline__ void record_timeout(unsigned int where) {
   if (atomicCAS(&g_status, 0u, kStatusTimeout) == 0u) g_status_where = where;
 }
 
+constexpr unsigned int kStatusUnsupported = 2;  // == CATTN_ERR_UNSUPPORTED
+constexpr int kMaxDynSmem = 232448;              // 227 KB opt-in limit per CTA
+
+// Shared-memory layouts assume 1024-byte aligned tiles.  The host asks for
+// `used + 1024` bytes when that fits, else exactly `used`; here the kernel
+// finds the aligned start and checks it fits what it was given.  Returns
+// nullptr (after recording CATTN_ERR_UNSUPPORTED) if not: the caller must
+// then return before touching any barrier, copy or tensor memory.
+__device__ __forceinline__ uint8_t* aligned_smem(uint8_t* raw, uint32_t used) {
+  uint32_t dyn;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
+  const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(raw));
+  const uint32_t pad = (1024u - (base & 1023u)) & 1023u;
+  if (pad + used > dyn) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0)
+      atomicCAS(&g_status, 0u, kStatusUnsupported);
+    return nullptr;
+  }
+  return raw + pad;
+}
+
 // ---------------------------------------------------------------------------
 // Shared-memory addresses
 // ---------------------------------------------------------------------------
@@ -280,6 +301,27 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32"
+      " [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16,"
+      " %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32"
@@ -364,6 +406,16 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// bf16 hi/lo split of two floats: hi = bf16(x) (round to nearest even) and
+// lo = bf16(x - hi), packed as bf16x2 (first element in the low half).
+// hi + lo carries x to about 16 significant bits.
+__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16(x0, x1);
+  const float h0 = __uint_as_float(hi << 16);
+  const float h1 = __uint_as_float(hi & 0xffff0000u);
+  lo = pack_bf16(x0 - h0, x1 - h1);
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,

@@ -77,6 +77,19 @@ CATTN_API cattn_status attn_fwd(const void* q, const void* k, const void* v, flo
                       int B, int H, int T, int D,
                       void* o, float* lse, void* stream);
 
+/* attn_fwd that can also write the rounding residual of its output:
+ *   o_lo : out, bf16 (B,H,T,D) or NULL; o_lo = bf16(O - o) where O is the
+ *          fp32 result before rounding and o = bf16(O) is the output above.
+ * o + o_lo carries O to about 16 significant bits.  Handing o_lo to
+ * attn_bwd_ex makes the backward's row term Delta = rowsum(dO * O) exact to
+ * fp32 rounding instead of inheriting o's bf16 rounding (which, on long
+ * sequences with peaked softmax, is the largest error in dQ and dK).
+ * With o_lo == NULL this is exactly attn_fwd.  Errors as attn_fwd; o_lo
+ * must be 16-byte aligned. */
+CATTN_API cattn_status attn_fwd_ex(const void* q, const void* k, const void* v, float scale,
+                                   int B, int H, int T, int D, void* o, float* lse, void* o_lo,
+                                   void* stream);
+
 /* Bytes of device workspace attn_bwd needs for this shape (0 on bad
  * arguments).  The layout is internal: an fp32 dQ accumulator of
  * B*H*T*D floats, fp32 Delta and scaled-LSE vectors of B*H*roundup(T,128)
@@ -99,7 +112,10 @@ CATTN_API cattn_status attn_bwd_preprocess(const void* o, const void* dout,
 /* Backward pass of a scalar loss L with dL/dO = dout:
  *   dV = P^T dO;  dP = dO V^T;  Delta = rowsum(dO * O);
  *   dS = P * (dP - Delta);  dQ = scale dS K;  dK = scale dS^T Q
- * P is recomputed from q, k and lse per key tile (never stored).
+ * P is recomputed from q, k and lse per key tile (never stored).  P and
+ * dS enter the tensor-core products as bf16 hi/lo pairs (about 16
+ * significant bits); Delta is computed from the bf16 o given here (use
+ * attn_bwd_ex with the forward's o_lo for an exact Delta).
  *   q, k, v, o, dout : in, bf16 (B,H,T,D); o and lse as produced by attn_fwd
  *   lse              : in, fp32 (B,H,T)
  *   dq, dk, dv       : out, bf16 (B,H,T,D)
@@ -114,6 +130,14 @@ CATTN_API cattn_status attn_bwd(const void* q, const void* k, const void* v,
                       float scale, int B, int H, int T, int D,
                       void* dq, void* dk, void* dv,
                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* attn_bwd with the forward's residual o_lo (see attn_fwd_ex): Delta is
+ * computed from o + o_lo.  o_lo may be NULL, which is exactly attn_bwd. */
+CATTN_API cattn_status attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
+                                   const void* o_lo, const float* lse, const void* dout,
+                                   float scale, int B, int H, int T, int D, void* dq, void* dk,
+                                   void* dv, void* workspace, size_t workspace_bytes,
+                                   void* stream);
 
 /* Library-global device status word: CATTN_OK, or the first
  * CATTN_ERR_TIMEOUT recorded by a kernel since the last clear.  Reads it

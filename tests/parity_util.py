@@ -33,6 +33,21 @@ def check_bf16(name, gpu, ref, max_abs=MAX_ABS, rel_l2=REL_L2):
     return ma, rl
 
 
+def check_bf16_beyond_rounding(name, gpu, ref, max_abs=MAX_ABS, rel_l2=REL_L2):
+    """For cases outside the five workloads whose values are so large that
+    bf16's own rounding (half an ulp, up to 2^-8 |x|) exceeds max_abs: the
+    error beyond that rounding must stay within max_abs, and rel-L2 within
+    rel_l2."""
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    excess = float((np.abs(gpu - ref) - 2.0 ** -8 * np.abs(ref)).max())
+    _, rl = errors(gpu, ref)
+    assert excess <= max_abs and rl <= rel_l2, (
+        f"{name}: error beyond bf16 rounding {excess:.3e} (tol {max_abs}), "
+        f"rel-L2 {rl:.3e} (tol {rel_l2})")
+    return excess, rl
+
+
 def check_lse(gpu, ref, tol=LSE_ABS):
     ma, _ = errors(gpu, ref)
     assert ma <= tol, f"lse: max-abs {ma:.3e} (tol {tol})"

@@ -107,6 +107,17 @@ def test_misaligned_fwd(which):
     assert fwd(lse=ALIGNED + 2) == cattn.ERR_INVALID_ARG
 
 
+def test_residual_entry_points_check_alignment():
+    args = (ALIGNED, ALIGNED, ALIGNED, 0.125, 1, 1, 8, 64, ALIGNED, ALIGNED)
+    assert cattn.LIB.attn_fwd_ex(*args, ALIGNED + 8, None) == cattn.ERR_INVALID_ARG
+    assert cattn.LIB.attn_fwd_ex(ALIGNED, ALIGNED, ALIGNED, 0.125, 1, 1, 8, 48, ALIGNED,
+                                 ALIGNED, None, None) == cattn.ERR_UNSUPPORTED
+    p = [ALIGNED] * 4
+    assert cattn.LIB.attn_bwd_ex(*p, ALIGNED + 8, ALIGNED, ALIGNED, 0.125, 1, 1, 8, 64,
+                                 ALIGNED, ALIGNED, ALIGNED, ALIGNED, 1 << 30,
+                                 None) == cattn.ERR_INVALID_ARG
+
+
 def test_misaligned_or_small_workspace():
     assert bwd(ws=ALIGNED + 128) == cattn.ERR_INVALID_ARG
     need = cattn.attn_bwd_workspace_bytes(1, 1, 8, 64)
