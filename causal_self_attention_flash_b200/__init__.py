@@ -111,33 +111,39 @@ def attn_bwd_preprocess(o, do, delta=None, stream=None):
 
 
 def attn_bwd(q, k, v, o, lse, do, scale=None, dq=None, dk=None, dv=None,
-             workspace=None, stream=None, o_lo=None):
+             workspace=None, stream=None, o_lo=None, grad_dtype=torch.bfloat16):
     """(dq, dk, dv) of causal attention; workspace allocated with torch if
     not given (a uint8 CUDA tensor of attn_bwd_workspace_bytes bytes).
-    With the forward's o_lo (attn_fwd_ex) this calls attn_bwd_ex."""
+    With the forward's o_lo or grad_dtype=torch.float32 this calls
+    attn_bwd_ex."""
     _inputs(q, k, v, o, do)
     B, H, T, D = _shape(q)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if lse.dtype != torch.float32 or not lse.is_contiguous():
         raise ValueError("lse must be contiguous fp32 (B, H, T)")
-    dq = _want(dq, q, torch.bfloat16, (B, H, T, D))
-    dk = _want(dk, q, torch.bfloat16, (B, H, T, D))
-    dv = _want(dv, q, torch.bfloat16, (B, H, T, D))
+    if grad_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("grad_dtype must be torch.bfloat16 or torch.float32")
+    dq = _want(dq, q, grad_dtype, (B, H, T, D))
+    dk = _want(dk, q, grad_dtype, (B, H, T, D))
+    dv = _want(dv, q, grad_dtype, (B, H, T, D))
     need = attn_bwd_workspace_bytes(B, H, T, D)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    if o_lo is None:
+    if o_lo is None and grad_dtype == torch.bfloat16:
         st = LIB.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                           lse.data_ptr(), do.data_ptr(), float(scale), B, H, T, D,
                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
                           workspace.numel(), _stream(stream))
         _check("attn_bwd", st)
     else:
-        _inputs(o_lo)
+        if o_lo is not None:
+            _inputs(o_lo)
         st = LIB.attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                             o_lo.data_ptr(), lse.data_ptr(), do.data_ptr(), float(scale),
-                             B, H, T, D, dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                             o_lo.data_ptr() if o_lo is not None else None, lse.data_ptr(),
+                             do.data_ptr(), float(scale), B, H, T, D, dq.data_ptr(),
+                             dk.data_ptr(), dv.data_ptr(),
+                             1 if grad_dtype == torch.float32 else 0,
                              workspace.data_ptr(), workspace.numel(), _stream(stream))
         _check("attn_bwd_ex", st)
     return dq, dk, dv

@@ -34,7 +34,7 @@ SIGNATURES = {
     "attn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _f, _i, _i, _i, _i,
                       _vp, _vp, _vp, _vp, _sz, _vp]),
     "attn_bwd_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _f, _i, _i, _i, _i,
-                         _vp, _vp, _vp, _vp, _sz, _vp]),
+                         _vp, _vp, _vp, _i, _vp, _sz, _vp]),
     "cattn_get_device_status": (_i, [_i, _vp]),
     "cattn_set_wait_timeout_us": (None, [_u32]),
     "cattn_selftest_wait_timeout": (_i, [_u32, _vp]),

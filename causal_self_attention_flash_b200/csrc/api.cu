@@ -219,7 +219,7 @@ cattn_status fwd_impl(int dev, const void* q, const void* k, const void* v, floa
   p.n_qtiles = (T + 127) / 128;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_timeout_ns;
-  dim3 grid(BH, p.n_qtiles);
+  dim3 grid(BH, (p.n_qtiles + 1) / 2);  // two query tiles per CTA
   {
     LaunchTimer t(K_FWD, s);
     fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, molo, p);
@@ -276,7 +276,8 @@ cattn_status pre_impl(const void* o, const void* o_lo, const void* dout, const f
 template <int D>
 cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, const void* o,
                       const void* o_lo, const float* lse, const void* dout, float scale, int BH,
-                      int T, void* dq, void* dk, void* dv, void* ws, cudaStream_t s) {
+                      int T, void* dq, void* dk, void* dv, bool grad_f32, void* ws,
+                      cudaStream_t s) {
   using C = BwdCfg<D>;
   clear_stale_error();
   cattn_status st = ensure_smem(dev, 4 + (D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3),
@@ -294,8 +295,10 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   if ((st = make_bf16_map(&mk, k, D, T, BH)) != CATTN_OK) return st;
   if ((st = make_bf16_map(&mv, v, D, T, BH)) != CATTN_OK) return st;
   if ((st = make_bf16_map(&mdo, dout, D, T, BH)) != CATTN_OK) return st;
-  if ((st = make_bf16_map(&mdk, dk, D, T, BH)) != CATTN_OK) return st;
-  if ((st = make_bf16_map(&mdv, dv, D, T, BH)) != CATTN_OK) return st;
+  // with fp32 gradients the kernel stores dK, dV directly and never uses
+  // these two maps; they then describe q instead
+  if ((st = make_bf16_map(&mdk, grad_f32 ? q : dk, D, T, BH)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mdv, grad_f32 ? q : dv, D, T, BH)) != CATTN_OK) return st;
   if ((st = make_tmap(&mdq, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, T, BH, C::CBQ, 128)) !=
       CATTN_OK)
     return st;
@@ -307,6 +310,8 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   BwdParams p;
   p.lse2 = lse2;
   p.delta = delta;
+  p.dk_f32 = grad_f32 ? static_cast<float*>(dk) : nullptr;
+  p.dv_f32 = grad_f32 ? static_cast<float*>(dv) : nullptr;
   p.T = T;
   p.T_pad = L.T_pad;
   p.n_tiles = L.T_pad / 128;
@@ -321,8 +326,12 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   if ((st = launch_status()) != CATTN_OK) return st;
   {
     LaunchTimer t(K_DQ_CONVERT, s);
-    dq_convert_kernel<<<grid_for(n_dq / 8, 256), 256, 0, s>>>(
-        reinterpret_cast<const float4*>(dq_acc), static_cast<uint4*>(dq), n_dq / 8, scale);
+    if (grad_f32)
+      dq_convert_f32_kernel<<<grid_for(n_dq / 4, 256), 256, 0, s>>>(
+          reinterpret_cast<const float4*>(dq_acc), static_cast<float4*>(dq), n_dq / 4, scale);
+    else
+      dq_convert_kernel<<<grid_for(n_dq / 8, 256), 256, 0, s>>>(
+          reinterpret_cast<const float4*>(dq_acc), static_cast<uint4*>(dq), n_dq / 8, scale);
   }
   return launch_status();
 }
@@ -408,8 +417,8 @@ cattn_status attn_bwd_preprocess(const void* o, const void* dout, int B, int H, 
 
 cattn_status attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
                          const void* o_lo, const float* lse, const void* dout, float scale, int B,
-                         int H, int T, int D, void* dq, void* dk, void* dv, void* workspace,
-                         size_t workspace_bytes, void* stream) {
+                         int H, int T, int D, void* dq, void* dk, void* dv, int grad_dtype,
+                         void* workspace, size_t workspace_bytes, void* stream) {
   cattn_status st = check_shape(B, H, T, D);
   if (st != CATTN_OK) return st;
   if (!(scale > 0.f) || !isfinite(scale)) return CATTN_ERR_INVALID_ARG;
@@ -422,19 +431,22 @@ cattn_status attn_bwd_ex(const void* q, const void* k, const void* v, const void
     return CATTN_ERR_INVALID_ARG;
   const int BH = B * H;
   if (workspace_bytes < ws_layout(BH, T, D).total) return CATTN_ERR_INVALID_ARG;
+  if (grad_dtype != CATTN_DTYPE_BF16 && grad_dtype != CATTN_DTYPE_F32)
+    return CATTN_ERR_INVALID_ARG;
+  const bool f32 = grad_dtype == CATTN_DTYPE_F32;
   int dev;
   if ((st = check_device(&dev)) != CATTN_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (D) {
     case 16:
-      return bwd_impl<16>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, workspace, s);
+      return bwd_impl<16>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, f32, workspace, s);
     case 32:
-      return bwd_impl<32>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, workspace, s);
+      return bwd_impl<32>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, f32, workspace, s);
     case 64:
-      return bwd_impl<64>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, workspace, s);
+      return bwd_impl<64>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, f32, workspace, s);
     case 128:
-      return bwd_impl<128>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, workspace,
-                           s);
+      return bwd_impl<128>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, f32,
+                           workspace, s);
   }
   return CATTN_ERR_UNSUPPORTED;
 }
@@ -443,8 +455,8 @@ cattn_status attn_bwd(const void* q, const void* k, const void* v, const void* o
                       const float* lse, const void* dout, float scale, int B, int H, int T, int D,
                       void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
                       void* stream) {
-  return attn_bwd_ex(q, k, v, o, nullptr, lse, dout, scale, B, H, T, D, dq, dk, dv, workspace,
-                     workspace_bytes, stream);
+  return attn_bwd_ex(q, k, v, o, nullptr, lse, dout, scale, B, H, T, D, dq, dk, dv,
+                     CATTN_DTYPE_BF16, workspace, workspace_bytes, stream);
 }
 
 cattn_status cattn_get_device_status(int clear, void* stream) {

@@ -19,7 +19,8 @@
 //                    tiles at or after it (causal), accumulating dK and dV in
 //                    TMEM and adding each dQ tile into the fp32 accumulator
 //                    with a TMA reduce-add.
-//   dq_convert_kernel dQ = bf16(scale * accumulator).
+//   dq_convert_kernel dQ = bf16(scale * accumulator), or fp32 when the caller
+//                    asks for fp32 gradients.
 //
 // Precision: P and dS enter the gradient MMAs as a bf16 hi/lo pair
 // (x = hi + lo to ~16 bits), so dV, dK and dQ carry fp32-level error instead
@@ -107,6 +108,17 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
 // dQ convert
 // ---------------------------------------------------------------------------
 
+__global__ void __launch_bounds__(256) dq_convert_f32_kernel(const float4* __restrict__ acc,
+                                                             float4* __restrict__ dq, size_t n4,
+                                                             float scale) {
+  const size_t tid = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const size_t nth = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t i = tid; i < n4; i += nth) {
+    const float4 a = acc[i];
+    dq[i] = make_float4(a.x * scale, a.y * scale, a.z * scale, a.w * scale);
+  }
+}
+
 __global__ void __launch_bounds__(256) dq_convert_kernel(const float4* __restrict__ acc,
                                                          uint4* __restrict__ dq, size_t n8,
                                                          float scale) {
@@ -156,6 +168,8 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float4* __restric
 struct BwdParams {
   const float* lse2;   // (BH, T_pad) LSE * log2(e); +inf on padding rows
   const float* delta;  // (BH, T_pad); 0 on padding rows
+  float* dk_f32;       // fp32 gradient outputs (BH, T, D), or null for bf16
+  float* dv_f32;       //   through the tensor maps
   int T;
   int T_pad;
   int n_tiles;
@@ -571,8 +585,35 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     drain_dq(n_iter - 1);  // waits for the last MMAs: everything is complete
     staging_free();
 
-    // ---- dK, dV epilogue: TMEM -> bf16 -> shared (dS buffers) -> TMA store
+    // ---- dK, dV epilogue
     constexpr int NC = D / 2;
+    if (p.dk_f32 != nullptr) {
+      // fp32 outputs: straight from TMEM to global, this thread's row half
+      const int key = kt * 128 + r;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = tbase + lane_base + (which ? C::COL_DK : C::COL_DV) + h * NC;
+        float* out = (which ? p.dk_f32 : p.dv_f32) +
+                     (static_cast<size_t>(bh) * p.T + key) * D + h * NC;
+        const float mul = which ? p.scale : 1.f;
+#pragma unroll
+        for (int c = 0; c < NC; c += 8) {
+          uint32_t v[8];
+          tmem_ld8(col + c, v);
+          tmem_wait_ld();
+          if (key < p.T) {
+            reinterpret_cast<float4*>(out + c)[0] =
+                make_float4(__uint_as_float(v[0]) * mul, __uint_as_float(v[1]) * mul,
+                            __uint_as_float(v[2]) * mul, __uint_as_float(v[3]) * mul);
+            reinterpret_cast<float4*>(out + c)[1] =
+                make_float4(__uint_as_float(v[4]) * mul, __uint_as_float(v[5]) * mul,
+                            __uint_as_float(v[6]) * mul, __uint_as_float(v[7]) * mul);
+          }
+        }
+      }
+      if (leader) bulk_wait0();  // the dQ reduces have completed
+    } else {
+    // bf16 outputs: TMEM -> bf16 -> shared (dS buffers) -> TMA store
 #pragma unroll
     for (int which = 0; which < 2; ++which) {  // 0: dV -> sDSH, 1: dK -> sDSL
       const uint32_t col = tbase + lane_base + (which ? C::COL_DK : C::COL_DV) + h * NC;
@@ -605,6 +646,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       bulk_commit();
     }
     if (leader) bulk_wait0();  // the dQ reduces and the stores have completed
+    }
   }
 
   tc_fence_before();

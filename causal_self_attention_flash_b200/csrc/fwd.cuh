@@ -1,5 +1,5 @@
-// Forward kernel: O = softmax(scale * Q K^T + causal mask) V and LSE, one
-// CTA per (head, 128-row query tile), never materialising the T x T matrix.
+// Forward kernel: O = softmax(scale * Q K^T + causal mask) V and LSE,
+// never materialising the T x T matrix.
 //
 // Definition ("nanoGPT: a real GPT in two 300-line files", section 2 "How
 // the code works", CausalSelfAttention, the written-out attention): scores
@@ -8,18 +8,24 @@
 // that softmax: a running maximum m and running sum l per row, with the
 // partial output rescaled whenever m moves.
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax: thread t owns query row t of the tile, which is TMEM
-//              lane t.  Reads S from TMEM, masks the diagonal tile, updates
-//              m and l, writes P (bf16) to shared memory, rescales O in
-//              TMEM when needed; at the end normalises O and writes O, LSE.
-//   warp 4     TMA producer: Q once, then K_j, V_j through a 2-stage ring.
-//   warp 5     MMA issuer (one thread) and TMEM owner:
-//              S_j = Q K_j^T into one of two TMEM buffers, then
-//              O += P_{j-1} V_{j-1}, so S_j overlaps the softmax of j-1.
+// One CTA serves two 128-row query tiles (2c, 2c+1) of one head, so the
+// tensor core alternates between them: while one softmax warpgroup works
+// on its scores, the MMAs of the other run.
 //
-// Causal tile skipping: tile i only visits key tiles 0..i (BM = BN = 128);
-// only the last (diagonal) one is masked.
+// Warp roles (320 threads):
+//   warps 0-3, 4-7  softmax warpgroups g = 0, 1 for query tiles 2c+g;
+//              thread t of a group owns query row t, which is TMEM lane t.
+//              It reads S_g from TMEM, masks the diagonal tile, updates m
+//              and l, and writes P back over S_g as bf16 hi/lo pairs
+//              (P = hi + lo to ~16 bits); at the end it normalises O_g and
+//              writes O (bf16), optionally O_lo = bf16(O - bf16(O)), and LSE.
+//   warp 8     TMA producer: both Q tiles once, then K_j, V_j through a ring.
+//   warp 9     MMA issuer and TMEM owner.  Per key tile j and group g:
+//              O_g += P_hi V_j + P_lo V_j (A from TMEM), then
+//              S_g(j+1) = Q_g K_{j+1}^T into the same columns.
+//
+// Causal tile skipping: query tile t visits key tiles 0..t only
+// (BM = BN = 128); only the last (diagonal) one is masked.
 //
 // Lazy rescaling: m is only moved when the new tile maximum exceeds it by
 // more than 8 (log2 units).  The exponentials then stay below 2^8, and
@@ -48,45 +54,44 @@ struct FwdCfg {
   static constexpr int NCB = D / CB;              // column blocks
   static constexpr int BLOCK_BYTES = 128 * RB;    // one [128][CB] block
   static constexpr int TILE_BYTES = 128 * D * 2;  // [128][D] bf16
-  static constexpr int STAGES = 2;
+  static constexpr int STAGES = D <= 64 ? 3 : 2;  // K/V ring depth
   static constexpr uint32_t SW = swizzle_code(RB);
   // shared memory map (all tiles 1024-aligned)
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + TILE_BYTES;
+  static constexpr int OFF_Q = 0;                              // [2] query tiles
+  static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
-  static constexpr int OFF_P = OFF_V + STAGES * TILE_BYTES;   // [2][128][64] bf16
-  static constexpr int OFF_BAR = OFF_P + 128 * 128 * 2;
-  static constexpr int NUM_BARS = 16;
+  static constexpr int OFF_BAR = OFF_V + STAGES * TILE_BYTES;
+  static constexpr int NUM_BARS = 20;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_USED = OFF_MISC + 64;
-  // keep one CTA per SM: the TMEM allocation below takes all 512 columns
-  static constexpr int SMEM_BYTES = (SMEM_USED < 120 * 1024 ? 120 * 1024 : SMEM_USED) + 1024;
-  static_assert(SMEM_BYTES <= kMaxDynSmem, "shared memory layout too large");
-  // TMEM columns
-  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O = 256;
+  // at least 116 KB so that one CTA holds an SM (it takes all 512 TMEM columns)
+  static constexpr int SMEM_WANT = SMEM_USED + 1024 < 116 * 1024 ? 116 * 1024 : SMEM_USED + 1024;
+  static constexpr int SMEM_BYTES = SMEM_WANT <= kMaxDynSmem ? SMEM_WANT : SMEM_USED;
+  static_assert(SMEM_USED <= kMaxDynSmem, "shared memory layout too large");
+  // TMEM columns: S_0, S_1 (P hi/lo written over them), O_0, O_1
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 320;
 };
 
 // barrier indices
 enum : int {
-  FB_Q = 0, FB_KFULL = 1, FB_VFULL = 3, FB_KVEMPTY = 5, FB_SFULL = 7, FB_SEMPTY = 9,
-  FB_PFULL = 11, FB_OFULL = 12, FB_DRAIN = 13
+  FB_Q = 0, FB_KFULL = 1, FB_VFULL = 4, FB_KVEMPTY = 7, FB_SFULL = 10, FB_PFULL = 12,
+  FB_ODONE = 14, FB_DRAIN = 16
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
            const __grid_constant__ CUtensorMap tmOlo, const FwdParams p) {
   using C = FwdCfg<D>;
+  static_assert(FB_DRAIN < C::NUM_BARS, "barrier count");
+  static_assert(FB_KVEMPTY + C::STAGES <= FB_SFULL, "barrier map");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  // 1024-byte align the working area (swizzle atoms)
   uint8_t* smem = aligned_smem(smem_raw, C::SMEM_USED);
   if (smem == nullptr) return;  // uniform over the CTA: nothing touched yet
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t sQ = sbase + C::OFF_Q;
-  const uint32_t sP = sbase + C::OFF_P;
   auto bar = [&](int i) { return sbase + C::OFF_BAR + 8u * i; };
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
@@ -94,8 +99,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int bh = blockIdx.x;
-  const int qt = p.n_qtiles - 1 - blockIdx.y;  // longest (most key tiles) first
-  const int n_kv = qt + 1;
+  const int n_pairs = (p.n_qtiles + 1) >> 1;
+  const int c = n_pairs - 1 - blockIdx.y;  // longest (most key tiles) first
+  const int t0 = 2 * c;                    // query tiles t0, t0 + 1
+  const bool has1 = t0 + 1 < p.n_qtiles;
+  const int n0 = t0 + 1;                   // key tiles seen by query tile t0
+  const int n1 = has1 ? t0 + 2 : 0;
+  const int n_kv = has1 ? n1 : n0;
 
   WaitCtx w{p.timeout_ns, abort_flag, 1u};
 
@@ -107,16 +117,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       mbar_init(bar(FB_VFULL + s), 1);
       mbar_init(bar(FB_KVEMPTY + s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(FB_SFULL + b), 1);
-      mbar_init(bar(FB_SEMPTY + b), 128);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(bar(FB_SFULL + g), 1);
+      mbar_init(bar(FB_PFULL + g), 128);
+      mbar_init(bar(FB_ODONE + g), 1);
     }
-    mbar_init(bar(FB_PFULL), 128);
-    mbar_init(bar(FB_OFULL), 1);
     mbar_init(bar(FB_DRAIN), 1);
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(sbase + C::OFF_MISC, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -125,16 +134,17 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   tc_fence_after();
   const uint32_t tbase = misc[0];
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      const int q0 = qt * C::BM;
-      mbar_arrive_expect_tx(bar(FB_Q), C::TILE_BYTES);
-      for (int b = 0; b < C::NCB; ++b)
-        tma_load_3d(sQ + b * C::BLOCK_BYTES, &tmQ, bar(FB_Q), b * C::CB, q0, bh);
+      mbar_arrive_expect_tx(bar(FB_Q), (has1 ? 2 : 1) * C::TILE_BYTES);
+      for (int g = 0; g < (has1 ? 2 : 1); ++g)
+        for (int b = 0; b < C::NCB; ++b)
+          tma_load_3d(sbase + C::OFF_Q + g * C::TILE_BYTES + b * C::BLOCK_BYTES, &tmQ,
+                      bar(FB_Q), b * C::CB, (t0 + g) * C::BM, bh);
       int n_issued = 0;
       for (int j = 0; j < n_kv; ++j) {
         const int st = j % C::STAGES;
@@ -163,46 +173,62 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         wait1(wd, bar(FB_Q), 0, 13);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);  // Q K-major, K K-major
-      constexpr uint32_t idO = idesc_bf16(128, D, 0, 1);    // P K-major, V MN-major
-      auto issue_pv = [&](int jj) {
-        const int st = jj % C::STAGES;
-        wait1(w, bar(FB_PFULL), jj & 1, 2);
-        wait1(w, bar(FB_VFULL + st), (jj / C::STAGES) & 1, 3);
-        tc_fence_after();
-        const uint32_t sV = sbase + C::OFF_V + st * C::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // 128 keys, 16 per MMA
-          const uint64_t a = smem_desc(sP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, 2);
-          const uint64_t b = smem_desc(sV + kk * 16 * C::RB, C::BLOCK_BYTES, 8 * C::RB, C::SW);
-          mma_ss(tbase + C::COL_O, a, b, idO, (jj > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(bar(FB_OFULL));
-        mma_commit(bar(FB_KVEMPTY + st));
-      };
-      wait1(w, bar(FB_Q), 0, 4);
-      for (int j = 0; j < n_kv; ++j) {
+      constexpr uint32_t idO = idesc_bf16(128, D, 0, 1);    // P (TMEM), V MN-major
+      auto issue_s = [&](int g, int j) {  // S_g = Q_g K_j^T
         const int st = j % C::STAGES;
-        const int sb = j & 1;
-        wait1(w, bar(FB_KFULL + st), (j / C::STAGES) & 1, 5);
-        if (j >= 2) wait1(w, bar(FB_SEMPTY + sb), ((j >> 1) - 1) & 1, 6);
+        wait1(w, bar(FB_KFULL + st), (j / C::STAGES) & 1, 2);
         tc_fence_after();
+        const uint32_t sQ = sbase + C::OFF_Q + g * C::TILE_BYTES;
         const uint32_t sK = sbase + C::OFF_K + st * C::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int blk = (kk * 16) / C::CB;
           const int off = ((kk * 16) % C::CB) * 2;
-          const uint64_t a = smem_desc(sQ + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW);
-          const uint64_t b = smem_desc(sK + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW);
-          mma_ss(tbase + (sb ? C::COL_S1 : C::COL_S0), a, b, idS, kk > 0 ? 1u : 0u);
+          mma_ss(tbase + (g ? C::COL_S1 : C::COL_S0),
+                 smem_desc(sQ + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW),
+                 smem_desc(sK + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW), idS,
+                 kk > 0 ? 1u : 0u);
         }
-        mma_commit(bar(FB_SFULL + sb));
-        if (j >= 1) issue_pv(j - 1);
+        mma_commit(bar(FB_SFULL + g));
+      };
+      auto issue_pv = [&](int g, int j) {  // O_g += (P_hi + P_lo) V_j
+        const int st = j % C::STAGES;
+        wait1(w, bar(FB_PFULL + g), j & 1, 3);
+        wait1(w, bar(FB_VFULL + st), (j / C::STAGES) & 1, 4);
+        tc_fence_after();
+        const uint32_t sV = sbase + C::OFF_V + st * C::TILE_BYTES;
+        const uint32_t pcol = tbase + (g ? C::COL_S1 : C::COL_S0);
+        const uint32_t ocol = tbase + (g ? C::COL_O1 : C::COL_O0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // 128 keys, 16 per MMA
+          const uint64_t b = smem_desc(sV + kk * 16 * C::RB, C::BLOCK_BYTES, 8 * C::RB, C::SW);
+          mma_ts(ocol, pcol + kk * 8, b, idO, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(ocol, pcol + 64 + kk * 8, b, idO, 1u);
+        }
+        mma_commit(bar(FB_ODONE + g));
+      };
+      wait1(w, bar(FB_Q), 0, 5);
+      issue_s(0, 0);
+      if (has1) issue_s(1, 0);
+      for (int j = 0; j < n_kv; ++j) {
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          const int ng = g ? n1 : n0;
+          if (j < ng) {
+            issue_pv(g, j);
+            if (j + 1 < ng) {
+              // S_g(j+1) overwrites P_g(j): only after PV_g(j) has read it
+              wait1(w, bar(FB_ODONE + g), j & 1, 6);
+              issue_s(g, j + 1);
+            }
+          }
+        }
+        mma_commit(bar(FB_KVEMPTY + j % C::STAGES));
       }
-      issue_pv(n_kv - 1);
       // drain: everything issued above has completed before TMEM is freed
       mma_commit(bar(FB_DRAIN));
       int zero = 0;
@@ -211,39 +237,53 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int row = threadIdx.x;            // 0..127 == TMEM lane
-    const uint32_t lane_base = (warp * 32) << 16;
-    const int q_row = qt * C::BM + row;
+    const int g = warp >> 2;                 // warpgroup = query tile t0 + g
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;     // query row in tile == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const int ng = g ? n1 : n0;
+    const int tile = t0 + g;
+    const int q_row = tile * C::BM + row;
+    const uint32_t scol = tbase + lane_base + (g ? C::COL_S1 : C::COL_S0);
+    const uint32_t ocol = tbase + lane_base + (g ? C::COL_O1 : C::COL_O0);
     const float sl2 = p.scale_log2;
     float m_used = -INFINITY;  // running max, scaled log2 units
     float l = 0.f;
     float s[128];
-    for (int j = 0; j < n_kv; ++j) {
-      const int sb = j & 1;
-      wait_warp(w, bar(FB_SFULL + sb), (j >> 1) & 1, 8);
+    for (int j = 0; j < ng; ++j) {
+      wait_warp(w, bar(FB_SFULL + g), j & 1, 8);
       tc_fence_after();
-      const uint32_t scol = tbase + lane_base + (sb ? C::COL_S1 : C::COL_S0);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(scol + c * 32, r);
+      {
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        tmem_ld32(scol, r0);
+        tmem_ld32(scol + 32, r1);
+        tmem_ld32(scol + 64, r2);
+        tmem_ld32(scol + 96, r3);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]);
+        for (int e = 0; e < 32; ++e) {
+          s[e] = __uint_as_float(r0[e]);
+          s[32 + e] = __uint_as_float(r1[e]);
+          s[64 + e] = __uint_as_float(r2[e]);
+          s[96 + e] = __uint_as_float(r3[e]);
+        }
       }
-      tc_fence_before();
-      mbar_arrive(bar(FB_SEMPTY + sb));
-
-      if (j == n_kv - 1) {  // diagonal tile: key index > query index is future
-        const int lim = q_row - j * C::BN;  // keys c <= lim are visible
+      if (j == ng - 1) {  // diagonal tile: key column > query row is future
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c > lim) s[c] = -INFINITY;
+        for (int cc = 0; cc < 128; ++cc)
+          if (cc > row) s[cc] = -INFINITY;
       }
-      float mx = s[0];
+      float mx[4];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
-      const float m_tile = mx * sl2;
+      for (int i = 0; i < 4; ++i) mx[i] = fmax3(s[i], s[4 + i], s[8 + i]);
+#pragma unroll
+      for (int cc = 12; cc < 124; cc += 8)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mx[i] = fmax3(mx[i], s[cc + i], s[cc + 4 + i]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) mx[i] = fmaxf(mx[i], s[124 + i]);
+      const float mxa = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
+      const float m_tile = mxa * sl2;
       float alpha = 1.f;
       const bool move = (j == 0) || (m_tile > m_used + 8.f);
       if (move) {
@@ -251,95 +291,114 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         alpha = ex2(m_used - m_new);  // 0 on the first tile (m_used = -inf)
         m_used = m_new;
       }
-      float sum = 0.f;
+      // O_g is stable here: S_g(j) was issued after PV_g(j-1) completed
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        s[c] = ex2(fmaf(s[c], sl2, -m_used));
-        sum += s[c];
-      }
-      l = l * alpha + sum;
-
-      if (j > 0) {
-        // P buffer and O accumulator are free once PV_{j-1} has completed
-        wait_warp(w, bar(FB_OFULL), (j - 1) & 1, 9);
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-          const uint32_t ocol = tbase + lane_base + C::COL_O;
+        for (int cc = 0; cc < D / 16; ++cc) {
+          uint32_t r[16];
+          tmem_ld16(ocol + cc * 16, r);
+          tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < D / 16; ++c) {
-            uint32_t r[16];
-            tmem_ld16(ocol + c * 16, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st16(ocol + c * 16, r);
-          }
-          tmem_wait_st();
+          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st16(ocol + cc * 16, r);
         }
       }
-      // P (bf16) -> shared, K-major 128B-swizzled [2][128 rows][64 keys]
+      const float neg_m = -m_used;
+      float sum[4];
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        const int c0 = ch * 8;
-        const uint32_t addr = sP + (c0 >> 6) * 16384 + swz<128>(row * 128 + ((c0 & 63) >> 3) * 16);
-        st_shared_v4(addr, pack_bf16(s[c0], s[c0 + 1]), pack_bf16(s[c0 + 2], s[c0 + 3]),
-                     pack_bf16(s[c0 + 4], s[c0 + 5]), pack_bf16(s[c0 + 6], s[c0 + 7]));
+      for (int i = 0; i < 4; ++i) sum[i] = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {  // 16 columns per chunk
+        uint32_t hi[8], lo[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float x0 = ex2(fmaf(s[ch * 16 + 2 * e], sl2, neg_m));
+          const float x1 = ex2(fmaf(s[ch * 16 + 2 * e + 1], sl2, neg_m));
+          sum[(2 * e) & 3] += x0;
+          sum[(2 * e + 1) & 3] += x1;
+          split_bf16x2(x0, x1, hi[e], lo[e]);
+        }
+        tmem_st8(scol + ch * 8, hi);
+        tmem_st8(scol + 64 + ch * 8, lo);
       }
-      fence_async_smem();
+      l = l * alpha + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(FB_PFULL));
+      mbar_arrive(bar(FB_PFULL + g));
     }
 
     // ---------------------------------------------------------- epilogue
-    wait_warp(w, bar(FB_OFULL), (n_kv - 1) & 1, 10);
-    tc_fence_after();
-    const float inv_l = 1.f / l;
-    const uint32_t ocol = tbase + lane_base + C::COL_O;
-    // O staging reuses the Q tile and O_lo staging the first K stage: every
-    // MMA that read them has completed and no load is in flight.
-    const uint32_t sOlo = sbase + C::OFF_K;
+    if (ng > 0) {
+      wait_warp(w, bar(FB_ODONE + g), (ng - 1) & 1, 10);
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      // staging: this group's Q tile (every MMA that read it has completed);
+      // O first, then O_lo through the same buffer
+      const uint32_t sQg = sbase + C::OFF_Q + g * C::TILE_BYTES;
+      const uint32_t nbar = 1 + g;
+      uint32_t lo_all[D / 2];
 #pragma unroll
-    for (int c = 0; c < D / 16; ++c) {
-      uint32_t r[16];
-      tmem_ld16(ocol + c * 16, r);
-      tmem_wait_ld();
-      uint32_t pk[8], lo[8];
+      for (int cc = 0; cc < D / 16; ++cc) {
+        uint32_t r[16];
+        tmem_ld16(ocol + cc * 16, r);
+        tmem_wait_ld();
+        uint32_t pk[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
-        split_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l,
-                     pk[e], lo[e]);
-      const int d0 = c * 16;
-      const int blk = d0 / C::CB;
+        for (int e = 0; e < 8; ++e)
+          split_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l,
+                       pk[e], lo_all[cc * 8 + e]);
+        const int d0 = cc * 16;
+        const int blk = d0 / C::CB;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int dd = (d0 % C::CB) + h * 8;
-        const uint32_t off = blk * C::BLOCK_BYTES + swz<C::RB>(row * C::RB + dd * 2);
-        st_shared_v4(sQ + off, pk[4 * h], pk[4 * h + 1], pk[4 * h + 2], pk[4 * h + 3]);
-        if (p.write_o_lo)
-          st_shared_v4(sOlo + off, lo[4 * h], lo[4 * h + 1], lo[4 * h + 2], lo[4 * h + 3]);
+        for (int hh = 0; hh < 2; ++hh) {
+          const int dd = (d0 % C::CB) + hh * 8;
+          st_shared_v4(sQg + blk * C::BLOCK_BYTES + swz<C::RB>(row * C::RB + dd * 2), pk[4 * hh],
+                       pk[4 * hh + 1], pk[4 * hh + 2], pk[4 * hh + 3]);
+        }
       }
-    }
-    tc_fence_before();
-    fence_async_smem();
-    named_bar_sync(1, 128);
-    if (threadIdx.x == 0 && !*abort_flag) {
-      for (int b = 0; b < C::NCB; ++b) {
-        tma_store_3d(&tmO, sQ + b * C::BLOCK_BYTES, b * C::CB, qt * C::BM, bh);
-        if (p.write_o_lo)
-          tma_store_3d(&tmOlo, sOlo + b * C::BLOCK_BYTES, b * C::CB, qt * C::BM, bh);
+      tc_fence_before();
+      fence_async_smem();
+      named_bar_sync(nbar, 128);
+      const bool leader = (threadIdx.x & 127) == 0;
+      if (leader && !*abort_flag) {
+        for (int b = 0; b < C::NCB; ++b)
+          tma_store_3d(&tmO, sQg + b * C::BLOCK_BYTES, b * C::CB, tile * C::BM, bh);
+        bulk_commit();
       }
-      bulk_commit();
-      bulk_wait_read0();
-    }
-    if (q_row < p.T) {
-      // natural-log LSE: m_used is in log2 units of the scaled score
-      p.lse[static_cast<size_t>(bh) * p.T + q_row] = m_used * 0.69314718055994531f + logf(l);
+      if (p.write_o_lo) {
+        if (leader) bulk_wait_read0();
+        named_bar_sync(nbar, 128);
+#pragma unroll
+        for (int cc = 0; cc < D / 16; ++cc) {
+          const int d0 = cc * 16;
+          const int blk = d0 / C::CB;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int dd = (d0 % C::CB) + hh * 8;
+            st_shared_v4(sQg + blk * C::BLOCK_BYTES + swz<C::RB>(row * C::RB + dd * 2),
+                         lo_all[cc * 8 + 4 * hh], lo_all[cc * 8 + 4 * hh + 1],
+                         lo_all[cc * 8 + 4 * hh + 2], lo_all[cc * 8 + 4 * hh + 3]);
+          }
+        }
+        fence_async_smem();
+        named_bar_sync(nbar, 128);
+        if (leader && !*abort_flag) {
+          for (int b = 0; b < C::NCB; ++b)
+            tma_store_3d(&tmOlo, sQg + b * C::BLOCK_BYTES, b * C::CB, tile * C::BM, bh);
+          bulk_commit();
+        }
+      }
+      if (leader) bulk_wait_read0();
+      if (q_row < p.T) {
+        // natural-log LSE: m_used is in log2 units of the scaled score
+        p.lse[static_cast<size_t>(bh) * p.T + q_row] = m_used * 0.69314718055994531f + logf(l);
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tbase, C::TMEM_COLS);
   }

@@ -24,11 +24,6 @@ __device__ unsigned int g_status_where = 0;
 
 constexpr unsigned int kStatusTimeout = 4;  // == CATTN_ERR_TIMEOUT
 
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
 
 __device__ __forceinline__ void record_timeout(unsigned int where) {
   if (atomicCAS(&g_status, 0u, kStatusTimeout) == 0u) g_status_where = where;
@@ -98,28 +93,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Per-CTA wait context: a deadline in ns and a shared abort flag.  Once any
+// Per-CTA wait context: a time limit and a shared abort flag.  Once any
 // thread of the CTA gives up, every later wait returns at once, so all
 // warps run to the end of the kernel (where TMEM is freed and copies in
 // flight are drained) instead of hanging.
+//
+// The limit is counted in SM clock cycles (clock64, cheap to read) at 2.1
+// cycles per ns: at or below the 1965 MHz maximum SM clock the real limit
+// is at least the requested time.
 struct WaitCtx {
   uint64_t timeout_ns;
   volatile int* abort;  // in shared memory
   unsigned int kernel_id;
 };
 
+__device__ __forceinline__ uint64_t cycles_now() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
+  return t;
+}
+
 // Single-thread bounded wait.  Returns false on timeout/abort.
 __device__ __forceinline__ bool wait1(const WaitCtx& w, uint32_t bar, uint32_t parity,
                                       unsigned int bar_id) {
   if (mbar_try_wait(bar, parity)) return true;
-  if (*w.abort) return false;
-  const uint64_t t0 = globaltimer_ns();
+  const uint64_t t0 = cycles_now();
+  const uint64_t limit = w.timeout_ns * 21 / 10;
   while (true) {
 #pragma unroll 1
-    for (int i = 0; i < 32; ++i)
+    for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (*w.abort) return false;
-    if (globaltimer_ns() - t0 > w.timeout_ns) {
+    if (cycles_now() - t0 > limit) {
       *w.abort = 1;
       record_timeout((w.kernel_id << 8) | bar_id);
       return false;
@@ -230,6 +235,18 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
                : "memory");
 }
 
+// Per-warpgroup register re-balancing (all four warps of a warpgroup run
+// the same one).  The totals must stay within what the block was launched
+// with: threads x registers per thread at launch.
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -322,6 +339,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::
+                   "r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+               "r"(r[7])
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32"
@@ -400,6 +425,13 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// max of three (sm_100 three-input form)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {

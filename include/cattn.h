@@ -131,13 +131,23 @@ CATTN_API cattn_status attn_bwd(const void* q, const void* k, const void* v,
                       void* dq, void* dk, void* dv,
                       void* workspace, size_t workspace_bytes, void* stream);
 
-/* attn_bwd with the forward's residual o_lo (see attn_fwd_ex): Delta is
- * computed from o + o_lo.  o_lo may be NULL, which is exactly attn_bwd. */
+/* Element types of gradient outputs (attn_bwd_ex). */
+enum { CATTN_DTYPE_BF16 = 0, CATTN_DTYPE_F32 = 1 };
+
+/* attn_bwd with two options:
+ *   o_lo       : the forward's residual (see attn_fwd_ex) or NULL; with it
+ *                Delta is computed from o + o_lo.
+ *   grad_dtype : CATTN_DTYPE_BF16 (dq, dk, dv as in attn_bwd) or
+ *                CATTN_DTYPE_F32: dq, dk, dv are fp32 (B,H,T,D), written
+ *                without the final bf16 rounding (whose half-ulp alone is
+ *                2^-8 |x|, 0.03 for gradients of magnitude 8..16).
+ * o_lo == NULL with CATTN_DTYPE_BF16 is exactly attn_bwd.  Errors as
+ * attn_bwd, plus CATTN_ERR_INVALID_ARG for an unknown grad_dtype. */
 CATTN_API cattn_status attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
                                    const void* o_lo, const float* lse, const void* dout,
                                    float scale, int B, int H, int T, int D, void* dq, void* dk,
-                                   void* dv, void* workspace, size_t workspace_bytes,
-                                   void* stream);
+                                   void* dv, int grad_dtype, void* workspace,
+                                   size_t workspace_bytes, void* stream);
 
 /* Library-global device status word: CATTN_OK, or the first
  * CATTN_ERR_TIMEOUT recorded by a kernel since the last clear.  Reads it

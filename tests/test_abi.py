@@ -114,8 +114,12 @@ def test_residual_entry_points_check_alignment():
                                  ALIGNED, None, None) == cattn.ERR_UNSUPPORTED
     p = [ALIGNED] * 4
     assert cattn.LIB.attn_bwd_ex(*p, ALIGNED + 8, ALIGNED, ALIGNED, 0.125, 1, 1, 8, 64,
-                                 ALIGNED, ALIGNED, ALIGNED, ALIGNED, 1 << 30,
+                                 ALIGNED, ALIGNED, ALIGNED, 0, ALIGNED, 1 << 30,
                                  None) == cattn.ERR_INVALID_ARG
+    for bad_dtype in (-1, 2, 7):
+        assert cattn.LIB.attn_bwd_ex(*p, None, ALIGNED, ALIGNED, 0.125, 1, 1, 8, 64,
+                                     ALIGNED, ALIGNED, ALIGNED, bad_dtype, ALIGNED, 1 << 30,
+                                     None) == cattn.ERR_INVALID_ARG
 
 
 def test_misaligned_or_small_workspace():

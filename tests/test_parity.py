@@ -77,35 +77,79 @@ def test_workload_plain_entry_points(lib, index):
     print(w.name, "plain", rep)
 
 
+def bf16_floor(ref):
+    """max |bf16(ref) - ref|: the error of a perfect kernel with bf16 output."""
+    return float(np.abs(as_f64(torch.tensor(ref).to(torch.bfloat16)) - ref).max())
+
+
 def test_long_context_sampled_heads(lib):
     """T = 8192, D = 128, logit std 4: two whole heads through the full
-    oracle (fwd + bwd), plus single rows of O/LSE on eight more heads."""
+    oracle (fwd + bwd), plus single rows of O/LSE on eight more heads.
+
+    On these heads |dQ| and |dK| exceed 8, where bf16's own rounding (half
+    an ulp, up to 0.031) is above the 2e-2 max-abs bar.  So: the bf16
+    gradients are held to 2e-2 beyond their own rounding (the stated
+    figures are printed as they are), and the same call with fp32 gradient
+    outputs is held to the stated 2e-2 / 1e-2 exactly."""
     index = 4
     w = WORKLOADS[index]
     q, k, v, do = workload_inputs(index)
-    got = run_gpu(lib, q, k, v, do, w.scale)
     heads = sample_heads(w.BH, 2, seed=seed_for(index))
     qn, kn, vn, don = (as_f64(t) for t in (q, k, v, do))
     ro, rl = oracle.attention_forward_heads(qn, kn, vn, w.scale, heads)
     rq, rk, rv = oracle.attention_backward_heads(qn, kn, vn, don, w.scale, heads)
-    flat = {n: got[n].reshape(w.BH, w.T, -1) for n in ("o", "dq", "dk", "dv")}
-    flat["lse"] = got["lse"].reshape(w.BH, w.T)
-    rep = {}
-    for n, ref in (("o", ro), ("dq", rq), ("dk", rk), ("dv", rv)):
-        rep[n] = check_bf16(n, flat[n][heads], ref)
-    rep["lse"] = check_lse(flat["lse"][heads], rl)
-    print(w.name, heads, rep)
+    refs = (("o", ro), ("dq", rq), ("dk", rk), ("dv", rv))
+
+    dev = torch.device("cuda:0")
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o, lse, o_lo = lib.attn_fwd_ex(qd, kd, vd, w.scale)
+    bf = lib.attn_bwd(qd, kd, vd, o, lse, dod, w.scale, o_lo=o_lo)
+    f32 = lib.attn_bwd(qd, kd, vd, o, lse, dod, w.scale, o_lo=o_lo, grad_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert lib.cattn_get_device_status() == lib.OK
+    got_bf = dict(o=as_f64(o), dq=as_f64(bf[0]), dk=as_f64(bf[1]), dv=as_f64(bf[2]))
+    got_32 = dict(dq=as_f64(f32[0]), dk=as_f64(f32[1]), dv=as_f64(f32[2]))
+
+    def head_view(x):
+        return x.reshape(w.BH, w.T, -1)[heads]
+
+    check_bf16("o", head_view(got_bf["o"]), ro)
+    check_lse(as_f64(lse).reshape(w.BH, w.T)[heads], rl)
+    for n, ref in refs[1:]:
+        stated = errors(head_view(got_bf[n]), ref)
+        print(f"{w.name} {n} bf16: max-abs {stated[0]:.4f} rel-L2 {stated[1]:.2e} "
+              f"(bf16 floor {bf16_floor(ref):.4f})")
+        check_bf16_beyond_rounding(n, head_view(got_bf[n]), ref)
+        ma, rl2 = check_bf16(n + " fp32", head_view(got_32[n]), ref)
+        print(f"{w.name} {n} fp32: max-abs {ma:.2e} rel-L2 {rl2:.2e}")
     # the plain entry points on the same heads: Delta from the bf16 O
     plain = run_gpu(lib, q, k, v, do, w.scale, residual=False)
-    prep = {n: errors(plain[n].reshape(w.BH, w.T, -1)[heads], ref)
-            for n, ref in (("o", ro), ("dq", rq), ("dk", rk), ("dv", rv))}
+    prep = {n: errors(plain[n].reshape(w.BH, w.T, -1)[heads], ref) for n, ref in refs}
     print(w.name, "plain entry points", prep)
     rows = [0, 1, 127, 128, 4095, 8191]
     for f in sample_heads(w.BH, 8, seed=seed_for(index) + 1):
         b, h = divmod(f, w.H)
         o_rows, lse_rows = oracle.attention_rows(qn, kn, vn, w.scale, b, h, rows)
-        check_bf16("o rows", got["o"][b, h, rows], o_rows)
-        check_lse(got["lse"][b, h, rows], lse_rows)
+        check_bf16("o rows", got_bf["o"][b, h, rows], o_rows)
+        check_lse(as_f64(lse)[b, h, rows], lse_rows)
+
+
+@pytest.mark.parametrize("index", [1, 2, 3])
+def test_workload_fp32_gradients(lib, index):
+    """The fp32-gradient option on the GPT-shaped workloads: stated
+    tolerance with no output rounding."""
+    w = WORKLOADS[index]
+    q, k, v, do = workload_inputs(index)
+    dev = torch.device("cuda:0")
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o, lse, o_lo = lib.attn_fwd_ex(qd, kd, vd, w.scale)
+    dq, dk, dv = lib.attn_bwd(qd, kd, vd, o, lse, dod, w.scale, o_lo=o_lo,
+                              grad_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ref = full_oracle(q, k, v, do, w.scale)
+    for n, g in (("dq", dq), ("dk", dk), ("dv", dv)):
+        ma, rl = check_bf16(n + " fp32", as_f64(g), ref[n])
+        print(w.name, n, "fp32", ma, rl)
 
 
 RAGGED_T = [1, 17, 63, 64, 65, 127, 128, 129, 255, 1000]
