@@ -16,8 +16,9 @@ import math
 
 import torch
 
-from ._binding import (ERR_CUDA, ERR_INVALID_ARG, ERR_TIMEOUT,
-                       ERR_UNSUPPORTED, LIB, LIB_PATH, OK, CattnError)
+from ._binding import (ERR_CUDA, ERR_INVALID_ARG, ERR_TIMEOUT, ERR_TOO_LARGE,
+                       ERR_UNSUPPORTED, LIB, LIB_PATH, NOALLOC_SCRATCH_BYTES, OK,
+                       CattnError)
 
 __all__ = [
     "attn_fwd", "attn_bwd", "attn_fwd_ex", "attn_bwd_ex", "attn_bwd_preprocess",
@@ -26,7 +27,8 @@ __all__ = [
     "cattn_selftest_wait_timeout", "cattn_status_string", "cattn_version",
     "cattn_timing_enable", "cattn_timing_read", "KERNEL_NAMES",
     "CausalAttention", "CattnError", "LIB", "LIB_PATH",
-    "OK", "ERR_INVALID_ARG", "ERR_UNSUPPORTED", "ERR_CUDA", "ERR_TIMEOUT",
+    "OK", "ERR_INVALID_ARG", "ERR_UNSUPPORTED", "ERR_CUDA", "ERR_TIMEOUT", "ERR_TOO_LARGE",
+    "attn_bwd_noalloc", "NOALLOC_SCRATCH_BYTES",
 ]
 
 
@@ -150,6 +152,26 @@ def attn_bwd(q, k, v, o, lse, do, scale=None, dq=None, dk=None, dv=None,
 
 
 attn_bwd_ex = attn_bwd
+
+
+def attn_bwd_noalloc(q, k, v, o, lse, do, scale=None, dq=None, dk=None, dv=None,
+                     stream=None):
+    """attn_bwd without a workspace: the library's fixed scratch of
+    NOALLOC_SCRATCH_BYTES is used instead (see include/cattn.h; calls that
+    overlap on the GPU race).  Only the outputs, if not given, are
+    allocated here, by torch; the C call itself allocates nothing."""
+    _inputs(q, k, v, o, do)
+    B, H, T, D = _shape(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = _want(dq, q, torch.bfloat16, (B, H, T, D))
+    dk = _want(dk, q, torch.bfloat16, (B, H, T, D))
+    dv = _want(dv, q, torch.bfloat16, (B, H, T, D))
+    st = LIB.attn_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              lse.data_ptr(), do.data_ptr(), float(scale), B, H, T, D,
+                              dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), _stream(stream))
+    _check("attn_bwd_noalloc", st)
+    return dq, dk, dv
 
 
 def cattn_get_device_status(clear=False, stream=None):

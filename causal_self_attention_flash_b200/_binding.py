@@ -18,10 +18,11 @@ ERR_INVALID_ARG = 1
 ERR_UNSUPPORTED = 2
 ERR_CUDA = 3
 ERR_TIMEOUT = 4
+ERR_TOO_LARGE = 5
 
 STATUS_NAMES = {OK: "CATTN_OK", ERR_INVALID_ARG: "CATTN_ERR_INVALID_ARG",
                 ERR_UNSUPPORTED: "CATTN_ERR_UNSUPPORTED", ERR_CUDA: "CATTN_ERR_CUDA",
-                ERR_TIMEOUT: "CATTN_ERR_TIMEOUT"}
+                ERR_TIMEOUT: "CATTN_ERR_TIMEOUT", ERR_TOO_LARGE: "CATTN_ERR_TOO_LARGE"}
 
 # name -> (restype, argtypes), mirroring include/cattn.h
 _vp, _i, _f, _sz, _u32 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_float,
@@ -35,6 +36,8 @@ SIGNATURES = {
                       _vp, _vp, _vp, _vp, _sz, _vp]),
     "attn_bwd_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _f, _i, _i, _i, _i,
                          _vp, _vp, _vp, _i, _vp, _sz, _vp]),
+    "attn_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _f, _i, _i, _i, _i,
+                              _vp, _vp, _vp, _vp]),
     "cattn_get_device_status": (_i, [_i, _vp]),
     "cattn_set_wait_timeout_us": (None, [_u32]),
     "cattn_selftest_wait_timeout": (_i, [_u32, _vp]),
@@ -66,5 +69,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         fn.argtypes = args
     return lib
 
+
+# CATTN_NOALLOC_SCRATCH_BYTES of include/cattn.h
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 LIB = load()

@@ -14,6 +14,12 @@
 #include "bwd.cuh"
 #include "fwd.cuh"
 
+// Scratch of attn_bwd_noalloc: one fixed array per device, owned by the
+// library for the process's lifetime.  Host code must not use this name as
+// a device address (on the host it is only a stand-in for the symbol); the
+// address is looked up with cudaGetSymbolAddress per device.
+static __device__ __align__(256) unsigned char cattn_noalloc_scratch[CATTN_NOALLOC_SCRATCH_BYTES];
+
 namespace cattn {
 namespace {
 
@@ -459,6 +465,58 @@ cattn_status attn_bwd(const void* q, const void* k, const void* v, const void* o
                      CATTN_DTYPE_BF16, workspace, workspace_bytes, stream);
 }
 
+// Device addresses of cattn_noalloc_scratch, looked up once per device.
+static void* g_noalloc_scratch_ptr[kMaxDevices];
+
+cattn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                              const float* lse, const void* dout, float scale, int B, int H,
+                              int T, int D, void* dq, void* dk, void* dv, void* stream) {
+  cattn_status st = check_shape(B, H, T, D);
+  if (st != CATTN_OK) return st;
+  if (!(scale > 0.f) || !isfinite(scale)) return CATTN_ERR_INVALID_ARG;
+  if (empty_shape(B, H, T)) return CATTN_OK;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return CATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      !aligned(lse, 4))
+    return CATTN_ERR_INVALID_ARG;
+  const int BH = B * H;
+  if (ws_layout(BH, T, D).total > CATTN_NOALLOC_SCRATCH_BYTES) return CATTN_ERR_TOO_LARGE;
+  int dev;
+  if ((st = check_device(&dev)) != CATTN_OK) return st;
+  void* scratch = nullptr;
+  {
+    // set-up, once per device, with that device current (check_device
+    // bound it to this thread): the array's device address
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_noalloc_scratch_ptr[dev] == nullptr) {
+      void* ptr = nullptr;
+      const cudaError_t e = cudaGetSymbolAddress(&ptr, cattn_noalloc_scratch);
+      if (e != cudaSuccess || ptr == nullptr) return cuda_fail(e != cudaSuccess ? e : cudaErrorUnknown);
+      g_noalloc_scratch_ptr[dev] = ptr;
+    }
+    scratch = g_noalloc_scratch_ptr[dev];
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the backward clears what must start at zero (the dQ accumulator) and
+  // overwrites the rest on every call
+  switch (D) {
+    case 16:
+      return bwd_impl<16>(dev, q, k, v, o, nullptr, lse, dout, scale, BH, T, dq, dk, dv, false,
+                          scratch, s);
+    case 32:
+      return bwd_impl<32>(dev, q, k, v, o, nullptr, lse, dout, scale, BH, T, dq, dk, dv, false,
+                          scratch, s);
+    case 64:
+      return bwd_impl<64>(dev, q, k, v, o, nullptr, lse, dout, scale, BH, T, dq, dk, dv, false,
+                          scratch, s);
+    case 128:
+      return bwd_impl<128>(dev, q, k, v, o, nullptr, lse, dout, scale, BH, T, dq, dk, dv, false,
+                           scratch, s);
+  }
+  return CATTN_ERR_UNSUPPORTED;
+}
+
 cattn_status cattn_get_device_status(int clear, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return cuda_fail(cudaGetLastError());
@@ -522,6 +580,7 @@ const char* cattn_status_string(cattn_status s) {
     case CATTN_ERR_UNSUPPORTED: return "unsupported (head size or device)";
     case CATTN_ERR_CUDA: return "CUDA error";
     case CATTN_ERR_TIMEOUT: return "kernel wait timed out";
+    case CATTN_ERR_TOO_LARGE: return "shape exceeds the fixed scratch of attn_bwd_noalloc";
   }
   return "unknown status";
 }

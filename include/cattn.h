@@ -60,7 +60,8 @@ typedef enum {
   CATTN_ERR_INVALID_ARG = 1, /* null pointer, bad size, misalignment, small workspace */
   CATTN_ERR_UNSUPPORTED = 2, /* head size D not instantiated; device not sm_100 */
   CATTN_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
-  CATTN_ERR_TIMEOUT = 4      /* a kernel's bounded wait ran out (device status) */
+  CATTN_ERR_TIMEOUT = 4,     /* a kernel's bounded wait ran out (device status) */
+  CATTN_ERR_TOO_LARGE = 5    /* shape needs more than attn_bwd_noalloc's scratch */
 } cattn_status;
 
 /* Forward pass: o = softmax(scale*q k^T + causal mask) v and its
@@ -148,6 +149,40 @@ CATTN_API cattn_status attn_bwd_ex(const void* q, const void* k, const void* v, 
                                    float scale, int B, int H, int T, int D, void* dq, void* dk,
                                    void* dv, int grad_dtype, void* workspace,
                                    size_t workspace_bytes, void* stream);
+
+/* Backward pass for callers that cannot allocate device memory.
+ *
+ * Same computation, arguments and results as attn_bwd, minus the workspace:
+ * its scratch (the fp32 dQ accumulator and the per-row LSE and Delta
+ * vectors) lives in one fixed array of CATTN_NOALLOC_SCRATCH_BYTES inside
+ * the library, which every GPU that loads the library holds until the
+ * process exits.  Some callers have no way to allocate: code hosted by a
+ * runtime that owns all device memory and hands a plugin only its input
+ * and output buffers, or latency-critical code that must not call
+ * cudaMalloc / cudaFree in steady state because those calls can
+ * synchronize the device.  This call allocates nothing and calls no
+ * allocating routine.
+ *
+ * Limits and sharing:
+ *  - shapes whose attn_bwd_workspace_bytes(B,H,T,D) exceeds
+ *    CATTN_NOALLOC_SCRATCH_BYTES are refused with CATTN_ERR_TOO_LARGE
+ *    before anything launches (the GPT-2 124M and 1558M layers fit; the
+ *    T = 8192, D = 128 case does not);
+ *  - every call on a device uses the same array: calls that may overlap on
+ *    the GPU (different streams, or other threads) race and give wrong
+ *    results; serialise them.  Each call clears and rewrites what it needs,
+ *    so contents left by an earlier call do not matter;
+ *  - the first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and caches it; make
+ *    that first call before any stream capture.
+ * The pages have no counterpart of this call: it exists for callers of
+ * this library that cannot allocate.
+ * Errors as attn_bwd, plus CATTN_ERR_TOO_LARGE. */
+#define CATTN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+CATTN_API cattn_status attn_bwd_noalloc(const void* q, const void* k, const void* v,
+                                        const void* o, const float* lse, const void* dout,
+                                        float scale, int B, int H, int T, int D, void* dq,
+                                        void* dk, void* dv, void* stream);
 
 /* Library-global device status word: CATTN_OK, or the first
  * CATTN_ERR_TIMEOUT recorded by a kernel since the last clear.  Reads it

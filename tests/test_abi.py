@@ -122,6 +122,22 @@ def test_residual_entry_points_check_alignment():
                                      None) == cattn.ERR_INVALID_ARG
 
 
+def test_static_scratch_backward_refuses_oversized_shapes():
+    """attn_bwd_noalloc: shapes beyond its fixed scratch are refused before
+    any device call (here, on a host without a GPU)."""
+    p = [ALIGNED] * 6
+    out = [ALIGNED] * 3
+    B, H, T, D = 2, 16, 8192, 128          # needs ~135 MB of scratch
+    assert cattn.attn_bwd_workspace_bytes(B, H, T, D) > cattn.NOALLOC_SCRATCH_BYTES
+    assert cattn.LIB.attn_bwd_noalloc(*p, 0.125, B, H, T, D, *out, None) == cattn.ERR_TOO_LARGE
+    assert cattn.attn_bwd_workspace_bytes(8, 25, 1024, 64) <= cattn.NOALLOC_SCRATCH_BYTES
+    assert cattn.LIB.attn_bwd_noalloc(*p, 0.125, 1, 1, 8, 48, *out, None) == \
+        cattn.ERR_UNSUPPORTED
+    assert cattn.LIB.attn_bwd_noalloc(*p[:5], None, 0.125, 1, 1, 8, 64, *out, None) == \
+        cattn.ERR_INVALID_ARG
+    assert "scratch" in cattn.cattn_status_string(cattn.ERR_TOO_LARGE)
+
+
 def test_misaligned_or_small_workspace():
     assert bwd(ws=ALIGNED + 128) == cattn.ERR_INVALID_ARG
     need = cattn.attn_bwd_workspace_bytes(1, 1, 8, 64)
