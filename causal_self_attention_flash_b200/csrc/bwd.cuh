@@ -384,11 +384,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         }
         mma_commit(bar(BB_PTDONE));
         mma_commit(bar(BB_DOEMPTY + ds));
-        // S(i+1) overwrites P^T(i): only after dV(i) has read it
-        if (i + 1 < n_iter) {
-          wait1(w, bar(BB_PTDONE), i & 1, 7);
-          issue_s(i + 1);
-        }
+        // S(i+1) overwrites P^T(i); the MMAs execute in issue order, so it
+        // cannot before dV(i) has read it
+        if (i + 1 < n_iter) issue_s(i + 1);
         // dK += dS^T Q_i (A = dS^T hi/lo in TMEM over dP^T)
         wait1(w, bar(BB_DSFULL), i & 1, 8);
         if (!C::ALIAS_DQ && i >= 1) wait1(w, bar(BB_DQEMPTY), (i - 1) & 1, 9);
@@ -401,11 +399,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           mma_ts(tbase + C::COL_DK, tbase + acol + 32, b, idKD, 1u);
         }
         mma_commit(bar(BB_QEMPTY + qs));
-        if (C::ALIAS_DQ) {  // dQ below overwrites the dS^T that dK just read
-          mma_commit(bar(BB_DKDONE));
-          wait1(w, bar(BB_DKDONE), i & 1, 10);
-          tc_fence_after();
-        }
+        // (aliased, dQ below overwrites the dS^T that dK just read: in order)
         // dQ_i = dS K  (A = dS hi/lo in shared, MN-major; K = 128 keys)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -416,9 +410,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         }
         mma_commit(bar(BB_DSDONE));
         mma_commit(bar(BB_DQFULL));
-        // dP(i+1) overwrites dS^T(i) (and, aliased, dQ(i))
+        // dP(i+1) overwrites dS^T(i) (in order behind dK(i)) and, aliased,
+        // dQ(i), which the compute warps must have drained first
         if (i + 1 < n_iter) {
-          wait1(w, bar(BB_DSDONE), i & 1, 11);
           if (C::ALIAS_DQ) wait1(w, bar(BB_DQEMPTY), i & 1, 12);
           issue_dp(i + 1);
         }

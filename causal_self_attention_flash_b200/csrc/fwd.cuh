@@ -22,7 +22,10 @@
 //   warp 8     TMA producer: both Q tiles once, then K_j, V_j through a ring.
 //   warp 9     MMA issuer and TMEM owner.  Per key tile j and group g:
 //              O_g += P_hi V_j + P_lo V_j (A from TMEM), then
-//              S_g(j+1) = Q_g K_{j+1}^T into the same columns.
+//              S_g(j+1) = Q_g K_{j+1}^T into the same columns.  The MMAs one
+//              thread issues execute in issue order, so S_g(j+1) is issued
+//              right behind PV_g(j) and cannot overwrite P_g(j) before PV_g(j)
+//              has read it.
 //
 // Causal tile skipping: query tile t visits key tiles 0..t only
 // (BM = BN = 128); only the last (diagonal) one is masked.
@@ -182,16 +185,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const int st = j % C::STAGES;
         wait1(w, bar(FB_KFULL + st), (j / C::STAGES) & 1, 2);
         tc_fence_after();
-        const uint32_t sQ = sbase + C::OFF_Q + g * C::TILE_BYTES;
-        const uint32_t sK = sbase + C::OFF_K + st * C::TILE_BYTES;
+        const uint64_t dq = smem_desc(sbase + C::OFF_Q + g * C::TILE_BYTES, 16, 8 * C::RB, C::SW);
+        const uint64_t dk = smem_desc(sbase + C::OFF_K + st * C::TILE_BYTES, 16, 8 * C::RB, C::SW);
+        const uint32_t dcol = tbase + (g ? C::COL_S1 : C::COL_S0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int blk = (kk * 16) / C::CB;
-          const int off = ((kk * 16) % C::CB) * 2;
-          mma_ss(tbase + (g ? C::COL_S1 : C::COL_S0),
-                 smem_desc(sQ + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW),
-                 smem_desc(sK + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW), idS,
-                 kk > 0 ? 1u : 0u);
+          const uint32_t off = (blk * C::BLOCK_BYTES + ((kk * 16) % C::CB) * 2) >> 4;
+          mma_ss(dcol, dq + off, dk + off, idS, kk > 0 ? 1u : 0u);
         }
         mma_commit(bar(FB_SFULL + g));
       };
@@ -200,12 +201,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         wait1(w, bar(FB_PFULL + g), j & 1, 3);
         wait1(w, bar(FB_VFULL + st), (j / C::STAGES) & 1, 4);
         tc_fence_after();
-        const uint32_t sV = sbase + C::OFF_V + st * C::TILE_BYTES;
+        const uint64_t dv = smem_desc(sbase + C::OFF_V + st * C::TILE_BYTES, C::BLOCK_BYTES,
+                                      8 * C::RB, C::SW);
         const uint32_t pcol = tbase + (g ? C::COL_S1 : C::COL_S0);
         const uint32_t ocol = tbase + (g ? C::COL_O1 : C::COL_O0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // 128 keys, 16 per MMA
-          const uint64_t b = smem_desc(sV + kk * 16 * C::RB, C::BLOCK_BYTES, 8 * C::RB, C::SW);
+          const uint64_t b = dv + ((kk * 16 * C::RB) >> 4);
           mma_ts(ocol, pcol + kk * 8, b, idO, (j > 0 || kk > 0) ? 1u : 0u);
           mma_ts(ocol, pcol + 64 + kk * 8, b, idO, 1u);
         }
@@ -220,11 +222,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           const int ng = g ? n1 : n0;
           if (j < ng) {
             issue_pv(g, j);
-            if (j + 1 < ng) {
-              // S_g(j+1) overwrites P_g(j): only after PV_g(j) has read it
-              wait1(w, bar(FB_ODONE + g), j & 1, 6);
-              issue_s(g, j + 1);
-            }
+            if (j + 1 < ng) issue_s(g, j + 1);  // in order behind PV_g(j)
           }
         }
         mma_commit(bar(FB_KVEMPTY + j % C::STAGES));
@@ -291,7 +289,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         alpha = ex2(m_used - m_new);  // 0 on the first tile (m_used = -inf)
         m_used = m_new;
       }
-      // O_g is stable here: S_g(j) was issued after PV_g(j-1) completed
+      // O_g is stable here: S_g(j), whose completion was just observed, was
+      // issued after PV_g(j-1), and the MMAs complete in issue order
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
         for (int cc = 0; cc < D / 16; ++cc) {
@@ -303,25 +302,27 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           tmem_st16(ocol + cc * 16, r);
         }
       }
-      const float neg_m = -m_used;
-      float sum[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) sum[i] = 0.f;
+      const uint64_t sl2x2 = f2(sl2, sl2);
+      const uint64_t negm2 = f2(-m_used, -m_used);
+      uint64_t sum2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {  // 16 columns per chunk
         uint32_t hi[8], lo[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float x0 = ex2(fmaf(s[ch * 16 + 2 * e], sl2, neg_m));
-          const float x1 = ex2(fmaf(s[ch * 16 + 2 * e + 1], sl2, neg_m));
-          sum[(2 * e) & 3] += x0;
-          sum[(2 * e + 1) & 3] += x1;
-          split_bf16x2(x0, x1, hi[e], lo[e]);
+          float x0, x1;
+          f2_split(fma2(f2(s[ch * 16 + 2 * e], s[ch * 16 + 2 * e + 1]), sl2x2, negm2), x0, x1);
+          const uint64_t p2 = f2(ex2(x0), ex2(x1));
+          sum2[e & 1] = add2(sum2[e & 1], p2);
+          split_bf16x2_p(p2, hi[e], lo[e]);
         }
         tmem_st8(scol + ch * 8, hi);
         tmem_st8(scol + 64 + ch * 8, lo);
       }
-      l = l * alpha + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
+      float sa, sb, sc2, sd;
+      f2_split(sum2[0], sa, sb);
+      f2_split(sum2[1], sc2, sd);
+      l = l * alpha + ((sa + sb) + (sc2 + sd));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(FB_PFULL + g));

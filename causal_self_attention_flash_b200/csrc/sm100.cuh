@@ -440,6 +440,48 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return r;
 }
 
+// Packed pairs of fp32 in one 64-bit register: sm_100 executes add, mul
+// and fma on both halves with one instruction.
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// hi/lo split of a packed pair: hi = bf16x2(x), lo = bf16x2(x - hi).
+__device__ __forceinline__ void split_bf16x2_p(uint64_t x, uint32_t& hi, uint32_t& lo) {
+  float x0, x1;
+  f2_split(x, x0, x1);
+  hi = pack_bf16(x0, x1);
+  const uint64_t h = f2(__uint_as_float(hi << 16), __uint_as_float(hi & 0xffff0000u));
+  float r0, r1;
+  f2_split(sub2(x, h), r0, r1);
+  lo = pack_bf16(r0, r1);
+}
+
 // bf16 hi/lo split of two floats: hi = bf16(x) (round to nearest even) and
 // lo = bf16(x - hi), packed as bf16x2 (first element in the low half).
 // hi + lo carries x to about 16 significant bits.
