@@ -203,13 +203,14 @@ struct LaunchTimer {
 
 // ------------------------------------------------------------------ forward
 
-template <int D>
+unsigned d_index(int D) { return D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3; }
+
+template <int D, bool PLO>
 cattn_status fwd_impl(int dev, const void* q, const void* k, const void* v, float scale, int BH,
                       int T, void* o, float* lse, void* o_lo, cudaStream_t s) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, PLO>;
   clear_stale_error();
-  cattn_status st = ensure_smem(dev, 0 + (D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3),
-                                fwd_kernel<D>, C::SMEM_BYTES);
+  cattn_status st = ensure_smem(dev, 0 + 2 * d_index(D) + PLO, fwd_kernel<D, PLO>, C::SMEM_BYTES);
   if (st != CATTN_OK) return st;
   CUtensorMap mq, mk, mv, mo, molo;
   if ((st = make_bf16_map(&mq, q, D, T, BH)) != CATTN_OK) return st;
@@ -228,7 +229,7 @@ cattn_status fwd_impl(int dev, const void* q, const void* k, const void* v, floa
   dim3 grid(BH, (p.n_qtiles + 1) / 2);  // two query tiles per CTA
   {
     LaunchTimer t(K_FWD, s);
-    fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, molo, p);
+    fwd_kernel<D, PLO><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, molo, p);
   }
   return launch_status();
 }
@@ -279,15 +280,14 @@ cattn_status pre_impl(const void* o, const void* o_lo, const void* dout, const f
   return launch_status();
 }
 
-template <int D>
+template <int D, bool SLO>
 cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, const void* o,
                       const void* o_lo, const float* lse, const void* dout, float scale, int BH,
                       int T, void* dq, void* dk, void* dv, bool grad_f32, void* ws,
                       cudaStream_t s) {
-  using C = BwdCfg<D>;
+  using C = BwdCfg<D, SLO>;
   clear_stale_error();
-  cattn_status st = ensure_smem(dev, 4 + (D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3),
-                                bwd_kernel<D>, C::SMEM_BYTES);
+  cattn_status st = ensure_smem(dev, 8 + 2 * d_index(D) + SLO, bwd_kernel<D, SLO>, C::SMEM_BYTES);
   if (st != CATTN_OK) return st;
   const WsLayout L = ws_layout(BH, T, D);
   uint8_t* wb = static_cast<uint8_t*>(ws);
@@ -327,7 +327,8 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   dim3 grid(BH, p.n_tiles);
   {
     LaunchTimer t(K_BWD_MAIN, s);
-    bwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mdo, mdk, mdv, mdq, p);
+    bwd_kernel<D, SLO><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mdo, mdk, mdv, mdq,
+                                                               p);
   }
   if ((st = launch_status()) != CATTN_OK) return st;
   {
@@ -340,6 +341,17 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
           reinterpret_cast<const float4*>(dq_acc), static_cast<uint4*>(dq), n_dq / 8, scale);
   }
   return launch_status();
+}
+
+template <int D>
+cattn_status bwd_dispatch(bool slo, int dev, const void* q, const void* k, const void* v,
+                          const void* o, const void* o_lo, const float* lse, const void* dout,
+                          float scale, int BH, int T, void* dq, void* dk, void* dv, bool f32,
+                          void* ws, cudaStream_t s) {
+  return slo ? bwd_impl<D, true>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, f32,
+                                 ws, s)
+             : bwd_impl<D, false>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv,
+                                  f32, ws, s);
 }
 
 // ---------------------------------------------------------- hang-guard test
@@ -382,10 +394,18 @@ cattn_status attn_fwd_ex(const void* q, const void* k, const void* v, float scal
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int BH = B * H;
   switch (D) {
-    case 16: return fwd_impl<16>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s);
-    case 32: return fwd_impl<32>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s);
-    case 64: return fwd_impl<64>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s);
-    case 128: return fwd_impl<128>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s);
+    case 16:
+      return o_lo ? fwd_impl<16, true>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s)
+                  : fwd_impl<16, false>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s);
+    case 32:
+      return o_lo ? fwd_impl<32, true>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s)
+                  : fwd_impl<32, false>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s);
+    case 64:
+      return o_lo ? fwd_impl<64, true>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s)
+                  : fwd_impl<64, false>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s);
+    case 128:
+      return o_lo ? fwd_impl<128, true>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s)
+                  : fwd_impl<128, false>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s);
   }
   return CATTN_ERR_UNSUPPORTED;
 }
@@ -443,16 +463,13 @@ cattn_status attn_bwd_ex(const void* q, const void* k, const void* v, const void
   int dev;
   if ((st = check_device(&dev)) != CATTN_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // dS as a hi/lo pair when the caller asks for gradients accurate to ~fp32
+  const bool slo = o_lo != nullptr || f32;
   switch (D) {
-    case 16:
-      return bwd_impl<16>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, f32, workspace, s);
-    case 32:
-      return bwd_impl<32>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, f32, workspace, s);
-    case 64:
-      return bwd_impl<64>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, f32, workspace, s);
-    case 128:
-      return bwd_impl<128>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, f32,
-                           workspace, s);
+    case 16: return bwd_dispatch<16>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, f32, workspace, s);
+    case 32: return bwd_dispatch<32>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, f32, workspace, s);
+    case 64: return bwd_dispatch<64>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, f32, workspace, s);
+    case 128: return bwd_dispatch<128>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, f32, workspace, s);
   }
   return CATTN_ERR_UNSUPPORTED;
 }
@@ -502,16 +519,16 @@ cattn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const
   // overwrites the rest on every call
   switch (D) {
     case 16:
-      return bwd_impl<16>(dev, q, k, v, o, nullptr, lse, dout, scale, BH, T, dq, dk, dv, false,
+      return bwd_impl<16, false>(dev, q, k, v, o, nullptr, lse, dout, scale, BH, T, dq, dk, dv, false,
                           scratch, s);
     case 32:
-      return bwd_impl<32>(dev, q, k, v, o, nullptr, lse, dout, scale, BH, T, dq, dk, dv, false,
+      return bwd_impl<32, false>(dev, q, k, v, o, nullptr, lse, dout, scale, BH, T, dq, dk, dv, false,
                           scratch, s);
     case 64:
-      return bwd_impl<64>(dev, q, k, v, o, nullptr, lse, dout, scale, BH, T, dq, dk, dv, false,
+      return bwd_impl<64, false>(dev, q, k, v, o, nullptr, lse, dout, scale, BH, T, dq, dk, dv, false,
                           scratch, s);
     case 128:
-      return bwd_impl<128>(dev, q, k, v, o, nullptr, lse, dout, scale, BH, T, dq, dk, dv, false,
+      return bwd_impl<128, false>(dev, q, k, v, o, nullptr, lse, dout, scale, BH, T, dq, dk, dv, false,
                            scratch, s);
   }
   return CATTN_ERR_UNSUPPORTED;

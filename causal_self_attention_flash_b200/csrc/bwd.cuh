@@ -22,9 +22,11 @@
 //   dq_convert_kernel dQ = bf16(scale * accumulator), or fp32 when the caller
 //                    asks for fp32 gradients.
 //
-// Precision: P and dS enter the gradient MMAs as a bf16 hi/lo pair
-// (x = hi + lo to ~16 bits), so dV, dK and dQ carry fp32-level error instead
-// of bf16's 2^-9; the only bf16 rounding left is that of the outputs.
+// Precision: P enters the dV MMA as a bf16 hi/lo pair (x = hi + lo to ~14
+// bits).  dS enters the dK and dQ MMAs as bf16 (SLO = false, the usual mixed
+// precision) or also as a hi/lo pair (SLO = true, used with the forward's
+// O_lo residual or with fp32 gradient outputs, where the aim is gradients
+// accurate to ~fp32).
 #pragma once
 
 #include "sm100.cuh"
@@ -153,15 +155,16 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float4* __restric
 //          drained to shared memory and added into the fp32 accumulator
 //          with a TMA reduce-add.
 //
-// Warp roles (320 threads):
-//   warps 0-7  compute: warp w serves TMEM lanes 32*(w%4).. (key rows) and
-//              query columns 64*(w/4) .. +64 of the tile; they also drain
-//              dQ and write dK, dV at the end.
-//   warp 8     TMA producer: K_j, V_j once; Q_i with the LSE2 and Delta
+// Warp roles (576 threads):
+//   warps 0-15 compute: warp w serves TMEM lanes 32*(w%4).. (key rows) and
+//              query columns 32*(w/4) .. +32 of the tile (four warps per SM
+//              sub-partition, to hide the latency of the exponentials and
+//              tensor-memory loads); they also drain dQ and write dK, dV.
+//   warp 16    TMA producer: K_j, V_j once; Q_i with the LSE2 and Delta
 //              vectors through a 2-stage ring (freed after dK(i), which
 //              follows every read of them), dO_i through a 2-stage
 //              (D <= 64) or 1-stage ring (freed after dV(i)).
-//   warp 9     MMA issuer and TMEM owner.  Order per iteration:
+//   warp 17    MMA issuer and TMEM owner.  Order per iteration:
 //              dV(i), S(i+1), dK(i), dQ(i), dP(i+1) -- so S(i+1) runs while
 //              dS(i) is computed and dK/dQ(i), dP(i+1) while P(i+1) is.
 
@@ -178,7 +181,7 @@ struct BwdParams {
   uint64_t timeout_ns;
 };
 
-template <int D>
+template <int D, bool SLO>
 struct BwdCfg {
   static constexpr int CB = D < 64 ? D : 64;       // bf16 columns per swizzle block
   static constexpr int RB = CB * 2;
@@ -208,12 +211,18 @@ struct BwdCfg {
       SMEM_USED + 1024 <= kMaxDynSmem ? SMEM_USED + 1024 : SMEM_USED;
   static_assert(SMEM_USED <= kMaxDynSmem, "shared memory layout too large");
   static_assert(128 * D * 4 <= 65536, "dQ staging must fit the dS buffers");
-  // TMEM columns
+  // TMEM columns.  MMAs that accumulate into one TMEM tile run back to back
+  // at about half the rate of independent ones, so where columns allow, the
+  // P_lo products of dV get their own accumulator dV' (summed at the end)
+  // and dK, dQ are issued interleaved.
   static constexpr bool ALIAS_DQ = 256 + 3 * D > 512;
+  static constexpr bool SPLIT_DV = 256 + 4 * D <= 512;
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
   static constexpr uint32_t COL_DQ = ALIAS_DQ ? COL_DP : 256 + 2 * D;
+  static constexpr uint32_t COL_DVL = SPLIT_DV ? 256 + 3 * D : COL_DV;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 576;
+  static constexpr int NCOMP = 512;   // compute threads
 };
 
 enum : int {
@@ -222,13 +231,13 @@ enum : int {
   BB_DQFULL = 15, BB_DQEMPTY = 16, BB_DKDONE = 17, BB_DRAIN = 18
 };
 
-template <int D>
-__global__ void __launch_bounds__(320, 1)
+template <int D, bool SLO>
+__global__ void __launch_bounds__(576, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
            const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
            const __grid_constant__ CUtensorMap tmDQacc, const BwdParams p) {
-  using C = BwdCfg<D>;
+  using C = BwdCfg<D, SLO>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = aligned_smem(smem_raw, C::SMEM_USED);
   if (smem == nullptr) return;  // uniform over the CTA: nothing touched yet
@@ -260,17 +269,17 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     }
     mbar_init(bar(BB_SFULL), 1);
     mbar_init(bar(BB_DPFULL), 1);
-    mbar_init(bar(BB_PFULL), 256);
+    mbar_init(bar(BB_PFULL), C::NCOMP);
     mbar_init(bar(BB_PTDONE), 1);
-    mbar_init(bar(BB_DSFULL), 256);
+    mbar_init(bar(BB_DSFULL), C::NCOMP);
     mbar_init(bar(BB_DSDONE), 1);
     mbar_init(bar(BB_DQFULL), 1);
-    mbar_init(bar(BB_DQEMPTY), 256);
+    mbar_init(bar(BB_DQEMPTY), C::NCOMP);
     mbar_init(bar(BB_DKDONE), 1);
     mbar_init(bar(BB_DRAIN), 1);
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == 17) {
     tmem_alloc(sbase + C::OFF_MISC, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -279,7 +288,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   tc_fence_after();
   const uint32_t tbase = misc[0];
 
-  if (warp == 8) {
+  if (warp == 16) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
@@ -326,7 +335,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           wait1(wd, bar(BB_DOFULL + i % C::DOST), (i / C::DOST) & 1, 22);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 17) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idSS = idesc_bf16(128, 128, 0, 0);  // S^T, dP^T
@@ -375,12 +384,14 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // dV += P^T dO_i  (A = P^T hi/lo in TMEM over S^T; K = 128 queries)
         wait1(w, bar(BB_PFULL), i & 1, 6);
         tc_fence_after();
+        const uint64_t ddo = smem_desc(sDO, C::BLOCK_BYTES, 8 * C::RB, C::SW);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t acol = C::COL_S + (kk >> 2) * 64 + (kk & 3) * 8;
-          const uint64_t b = smem_desc(sDO + kk * 16 * C::RB, C::BLOCK_BYTES, 8 * C::RB, C::SW);
-          mma_ts(tbase + C::COL_DV, tbase + acol, b, idKD, (i > 0 || kk > 0) ? 1u : 0u);
-          mma_ts(tbase + C::COL_DV, tbase + acol + 32, b, idKD, 1u);
+          const uint32_t acol = C::COL_S + (kk >> 1) * 32 + (kk & 1) * 8;
+          const uint64_t b = ddo + ((kk * 16 * C::RB) >> 4);
+          const uint32_t first = (i > 0 || kk > 0) ? 1u : 0u;
+          mma_ts(tbase + C::COL_DV, tbase + acol, b, idKD, first);
+          mma_ts(tbase + C::COL_DVL, tbase + acol + 16, b, idKD, C::SPLIT_DV ? first : 1u);
         }
         mma_commit(bar(BB_PTDONE));
         mma_commit(bar(BB_DOEMPTY + ds));
@@ -391,22 +402,45 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         wait1(w, bar(BB_DSFULL), i & 1, 8);
         if (!C::ALIAS_DQ && i >= 1) wait1(w, bar(BB_DQEMPTY), (i - 1) & 1, 9);
         tc_fence_after();
+        const uint64_t dqq = smem_desc(sQ, C::BLOCK_BYTES, 8 * C::RB, C::SW);
+        const uint64_t dkk = smem_desc(sK, C::BLOCK_BYTES, 8 * C::RB, C::SW);
+        const uint64_t dsh = smem_desc(sDSH, 16384, 1024, 2);
+        const uint64_t dsl = smem_desc(sDSL, 16384, 1024, 2);
+        // dK += dS^T Q_i (A = dS^T hi/lo in TMEM over dP^T) and
+        // dQ_i = dS K (A = dS hi/lo in shared, MN-major; K = 128 keys)
+        auto dk_step = [&](int kk, int lo) {
+          if (!SLO && lo) return;
+          const uint32_t acol = C::COL_DP + (kk >> 1) * 32 + (kk & 1) * 8 + (lo ? 16 : 0);
+          mma_ts(tbase + C::COL_DK, tbase + acol, dqq + ((kk * 16 * C::RB) >> 4), idKD,
+                 (i > 0 || kk > 0 || lo) ? 1u : 0u);
+        };
+        auto dq_step = [&](int kk, int lo) {
+          if (!SLO && lo) return;
+          mma_ss(tbase + C::COL_DQ, (lo ? dsl : dsh) + ((kk * 2048) >> 4),
+                 dkk + ((kk * 16 * C::RB) >> 4), idQ, (kk > 0 || lo) ? 1u : 0u);
+        };
+        if constexpr (C::ALIAS_DQ) {
+          // dQ overwrites the dS^T that dK reads: all of dK first (in order)
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t acol = C::COL_DP + (kk >> 2) * 64 + (kk & 3) * 8;
-          const uint64_t b = smem_desc(sQ + kk * 16 * C::RB, C::BLOCK_BYTES, 8 * C::RB, C::SW);
-          mma_ts(tbase + C::COL_DK, tbase + acol, b, idKD, (i > 0 || kk > 0) ? 1u : 0u);
-          mma_ts(tbase + C::COL_DK, tbase + acol + 32, b, idKD, 1u);
-        }
-        mma_commit(bar(BB_QEMPTY + qs));
-        // (aliased, dQ below overwrites the dS^T that dK just read: in order)
-        // dQ_i = dS K  (A = dS hi/lo in shared, MN-major; K = 128 keys)
+          for (int kk = 0; kk < 8; ++kk) {
+            dk_step(kk, 0);
+            dk_step(kk, 1);
+          }
+          mma_commit(bar(BB_QEMPTY + qs));
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t b = smem_desc(sK + kk * 16 * C::RB, C::BLOCK_BYTES, 8 * C::RB, C::SW);
-          mma_ss(tbase + C::COL_DQ, smem_desc(sDSH + kk * 2048, 16384, 1024, 2), b, idQ,
-                 kk > 0 ? 1u : 0u);
-          mma_ss(tbase + C::COL_DQ, smem_desc(sDSL + kk * 2048, 16384, 1024, 2), b, idQ, 1u);
+          for (int kk = 0; kk < 8; ++kk) {
+            dq_step(kk, 0);
+            dq_step(kk, 1);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            dk_step(kk, 0);
+            dq_step(kk, 0);
+            dk_step(kk, 1);
+            dq_step(kk, 1);
+          }
+          mma_commit(bar(BB_QEMPTY + qs));
         }
         mma_commit(bar(BB_DSDONE));
         mma_commit(bar(BB_DQFULL));
@@ -424,49 +458,56 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     }
   } else {
     // ------------------------------------------- compute warps (row = key)
+    // Thread (warp w, lane l): key row r = 32*(w%4) + l, query columns
+    // [32g, 32g+32) of each tile with g = w/4.  In tensor memory, P^T and
+    // dS^T of query block g sit in columns 32g .. 32g+31 of their regions:
+    // 16 columns of bf16 pairs (hi), then 16 (lo).
     const int quarter = warp & 3;
-    const int h = warp >> 2;                     // query half of the tile
+    const int grp = warp >> 2;                   // query column group 0..3
     const int r = quarter * 32 + lane;           // key row == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const float sl2 = p.scale_log2;
     const bool leader = threadIdx.x == 0;
+    constexpr int NQ = D / 4;                    // dQ / dK / dV columns per thread
 
     // dQ(t) drain: TMEM (lane = query row) -> fp32 staging in the dS
     // buffers -> TMA reduce-add into the accumulator.
     auto drain_dq = [&](int t) {
       wait_warp(w, bar(BB_DQFULL), t & 1, 14);
       tc_fence_after();
-      constexpr int NC = D / 2;                  // columns per thread
-      float acc[NC];
-      const uint32_t src = tbase + lane_base + C::COL_DQ + h * NC;
-      if constexpr (NC >= 32) {
+      float acc[NQ];
+      const uint32_t src = tbase + lane_base + C::COL_DQ + grp * NQ;
+      if constexpr (NQ == 32) {
+        uint32_t v[32];
+        tmem_ld32(src, v);
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < NC / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(src + c * 32, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) acc[c * 32 + e] = __uint_as_float(v[e]);
-        }
-      } else if constexpr (NC == 16) {
+        for (int e = 0; e < 32; ++e) acc[e] = __uint_as_float(v[e]);
+      } else if constexpr (NQ == 16) {
         uint32_t v[16];
         tmem_ld16(src, v);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(v[e]);
-      } else {
+      } else if constexpr (NQ == 8) {
         uint32_t v[8];
         tmem_ld8(src, v);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = __uint_as_float(v[e]);
+      } else {
+        uint32_t v[4];
+        tmem_ld4(src, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[e] = __uint_as_float(v[e]);
       }
       tc_fence_before();
       mbar_arrive(bar(BB_DQEMPTY));
       // staging: blocks of [128 rows][CBQ floats], swizzled
 #pragma unroll
-      for (int e = 0; e < NC; e += 4) {
-        const int f = h * NC + e;
+      for (int e = 0; e < NQ; e += 4) {
+        const int f = grp * NQ + e;
         const int blk = f / C::CBQ;
         const int within = (f % C::CBQ) * 4;
         st_shared_v4(sDSH + blk * 128 * C::RBQ + swz<C::RBQ>(r * C::RBQ + within),
@@ -474,7 +515,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                      __float_as_uint(acc[e + 2]), __float_as_uint(acc[e + 3]));
       }
       fence_async_smem();
-      named_bar_sync(1, 256);
+      named_bar_sync(1, C::NCOMP);
       if (leader && !*abort_flag) {
 #pragma unroll
         for (int blk = 0; blk < D / C::CBQ; ++blk)
@@ -486,10 +527,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     // the dS buffers may be rewritten once the reduce has read them
     auto staging_free = [&]() {
       if (leader) bulk_wait_read0();
-      named_bar_sync(1, 256);
+      named_bar_sync(1, C::NCOMP);
     };
 
-    float pv[64];
+    float pv[32];
     for (int i = 0; i < n_iter; ++i) {
       const int qs = i % C::QST;
       // ---- P phase
@@ -497,20 +538,15 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       tc_fence_after();
       {
         uint32_t v[32];
-        tmem_ld32(tbase + lane_base + C::COL_S + h * 64, v);
-        uint32_t u[32];
-        tmem_ld32(tbase + lane_base + C::COL_S + h * 64 + 32, u);
+        tmem_ld32(tbase + lane_base + C::COL_S + grp * 32, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          pv[e] = __uint_as_float(v[e]);
-          pv[32 + e] = __uint_as_float(u[e]);
-        }
+        for (int e = 0; e < 32; ++e) pv[e] = __uint_as_float(v[e]);
       }
       wait_warp(w, bar(BB_QFULL + qs), (i / C::QST) & 1, 16);  // LSE2 visibility
-      const uint32_t sL = sbase + C::OFF_LSE + qs * 512 + h * 256;
+      const uint32_t sL = sbase + C::OFF_LSE + qs * 512 + grp * 128;
 #pragma unroll
-      for (int c = 0; c < 64; c += 4) {
+      for (int c = 0; c < 32; c += 4) {
         float l0, l1, l2, l3;
         ld_shared_v4f(sL + c * 4, l0, l1, l2, l3);
         pv[c] = ex2(fmaf(pv[c], sl2, -l0));
@@ -518,18 +554,18 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         pv[c + 2] = ex2(fmaf(pv[c + 2], sl2, -l2));
         pv[c + 3] = ex2(fmaf(pv[c + 3], sl2, -l3));
       }
-      if (i == 0) {  // diagonal tile: query (64h + c) sees key r only if r <= query
-        const int lim = r - h * 64;
+      if (i == 0) {  // diagonal tile: query (32g + c) sees key r only if r <= query
+        const int lim = r - grp * 32;
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
+        for (int c = 0; c < 32; ++c)
           if (c < lim) pv[c] = 0.f;
       }
       {
-        uint32_t hi[32], lo[32];
+        uint32_t hi[16], lo[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) split_bf16x2(pv[2 * e], pv[2 * e + 1], hi[e], lo[e]);
-        tmem_st32(tbase + lane_base + C::COL_S + h * 64, hi);
-        tmem_st32(tbase + lane_base + C::COL_S + h * 64 + 32, lo);
+        for (int e = 0; e < 16; ++e) split_bf16x2_p(f2(pv[2 * e], pv[2 * e + 1]), hi[e], lo[e]);
+        tmem_st16(tbase + lane_base + C::COL_S + grp * 32, hi);
+        tmem_st16(tbase + lane_base + C::COL_S + grp * 32 + 16, lo);
         tmem_wait_st();
       }
       tc_fence_before();
@@ -542,34 +578,40 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       wait_warp(w, bar(BB_DPFULL), i & 1, 17);
       tc_fence_after();
       // (the Delta vector arrived with Q_i, whose barrier was waited above)
-      const uint32_t sD = sbase + C::OFF_DELTA + qs * 512 + h * 256;
-      uint32_t hi[32], lo[32];
-#pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
+      const uint32_t sD = sbase + C::OFF_DELTA + qs * 512 + grp * 128;
+      uint32_t hi[16], lo[16];
+      {
         uint32_t v[32];
-        tmem_ld32(tbase + lane_base + C::COL_DP + h * 64 + c2 * 32, v);
+        tmem_ld32(tbase + lane_base + C::COL_DP + grp * 32, v);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           float d0, d1, d2, d3;
-          ld_shared_v4f(sD + (c2 * 32 + e) * 4, d0, d1, d2, d3);
-          const float s0 = pv[c2 * 32 + e] * (__uint_as_float(v[e]) - d0);
-          const float s1 = pv[c2 * 32 + e + 1] * (__uint_as_float(v[e + 1]) - d1);
-          const float s2 = pv[c2 * 32 + e + 2] * (__uint_as_float(v[e + 2]) - d2);
-          const float s3 = pv[c2 * 32 + e + 3] * (__uint_as_float(v[e + 3]) - d3);
-          split_bf16x2(s0, s1, hi[c2 * 16 + e / 2], lo[c2 * 16 + e / 2]);
-          split_bf16x2(s2, s3, hi[c2 * 16 + e / 2 + 1], lo[c2 * 16 + e / 2 + 1]);
+          ld_shared_v4f(sD + e * 4, d0, d1, d2, d3);
+          const float s0 = pv[e] * (__uint_as_float(v[e]) - d0);
+          const float s1 = pv[e + 1] * (__uint_as_float(v[e + 1]) - d1);
+          const float s2 = pv[e + 2] * (__uint_as_float(v[e + 2]) - d2);
+          const float s3 = pv[e + 3] * (__uint_as_float(v[e + 3]) - d3);
+          if (SLO) {
+            split_bf16x2_p(f2(s0, s1), hi[e / 2], lo[e / 2]);
+            split_bf16x2_p(f2(s2, s3), hi[e / 2 + 1], lo[e / 2 + 1]);
+          } else {
+            hi[e / 2] = pack_bf16(s0, s1);
+            hi[e / 2 + 1] = pack_bf16(s2, s3);
+          }
         }
       }
-      tmem_st32(tbase + lane_base + C::COL_DP + h * 64, hi);
-      tmem_st32(tbase + lane_base + C::COL_DP + h * 64 + 32, lo);
-      // dS (hi, lo) -> shared for the dQ MMA: [2][128 keys][64 queries]
+      tmem_st16(tbase + lane_base + C::COL_DP + grp * 32, hi);
+      if (SLO) tmem_st16(tbase + lane_base + C::COL_DP + grp * 32 + 16, lo);
+      // dS (hi, lo) -> shared for the dQ MMA: [2][128 keys][64 queries];
+      // query block g is half g/2, chunks 4*(g%2) .. +3 of the row
       if (i >= 1) staging_free();
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const uint32_t off = h * 16384 + swz<128>(r * 128 + ch * 16);
+      for (int ch = 0; ch < 4; ++ch) {
+        const uint32_t off = (grp >> 1) * 16384 + swz<128>(r * 128 + ((grp & 1) * 4 + ch) * 16);
         st_shared_v4(sDSH + off, hi[4 * ch], hi[4 * ch + 1], hi[4 * ch + 2], hi[4 * ch + 3]);
-        st_shared_v4(sDSL + off, lo[4 * ch], lo[4 * ch + 1], lo[4 * ch + 2], lo[4 * ch + 3]);
+        if (SLO)
+          st_shared_v4(sDSL + off, lo[4 * ch], lo[4 * ch + 1], lo[4 * ch + 2], lo[4 * ch + 3]);
       }
       fence_async_smem();
       tmem_wait_st();
@@ -579,73 +621,99 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     drain_dq(n_iter - 1);  // waits for the last MMAs: everything is complete
     staging_free();
 
-    // ---- dK, dV epilogue
-    constexpr int NC = D / 2;
-    if (p.dk_f32 != nullptr) {
-      // fp32 outputs: straight from TMEM to global, this thread's row half
-      const int key = kt * 128 + r;
+    // ---- dK, dV epilogue: this thread's NQ columns of its key row
+    auto load_cols = [&](uint32_t col, float (&x)[NQ]) {
+      if constexpr (NQ == 32) {
+        uint32_t v[32];
+        tmem_ld32(col, v);
+        tmem_wait_ld();
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t col = tbase + lane_base + (which ? C::COL_DK : C::COL_DV) + h * NC;
-        float* out = (which ? p.dk_f32 : p.dv_f32) +
-                     (static_cast<size_t>(bh) * p.T + key) * D + h * NC;
-        const float mul = which ? p.scale : 1.f;
+        for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(v[e]);
+      } else if constexpr (NQ == 16) {
+        uint32_t v[16];
+        tmem_ld16(col, v);
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < NC; c += 8) {
-          uint32_t v[8];
-          tmem_ld8(col + c, v);
-          tmem_wait_ld();
-          if (key < p.T) {
-            reinterpret_cast<float4*>(out + c)[0] =
-                make_float4(__uint_as_float(v[0]) * mul, __uint_as_float(v[1]) * mul,
-                            __uint_as_float(v[2]) * mul, __uint_as_float(v[3]) * mul);
-            reinterpret_cast<float4*>(out + c)[1] =
-                make_float4(__uint_as_float(v[4]) * mul, __uint_as_float(v[5]) * mul,
-                            __uint_as_float(v[6]) * mul, __uint_as_float(v[7]) * mul);
-          }
-        }
+        for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(v[e]);
+      } else if constexpr (NQ == 8) {
+        uint32_t v[8];
+        tmem_ld8(col, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(v[e]);
+      } else {
+        uint32_t v[4];
+        tmem_ld4(col, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = __uint_as_float(v[e]);
       }
-      if (leader) bulk_wait0();  // the dQ reduces have completed
-    } else {
-    // bf16 outputs: TMEM -> bf16 -> shared (dS buffers) -> TMA store
+    };
+    const bool f32out = p.dk_f32 != nullptr;
 #pragma unroll
-    for (int which = 0; which < 2; ++which) {  // 0: dV -> sDSH, 1: dK -> sDSL
-      const uint32_t col = tbase + lane_base + (which ? C::COL_DK : C::COL_DV) + h * NC;
-      const uint32_t dst = which ? sDSL : sDSH;
+    for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
+      float x[NQ];
+      load_cols(tbase + lane_base + (which ? C::COL_DK : C::COL_DV) + grp * NQ, x);
+      if (C::SPLIT_DV && which == 0) {  // dV = dV + dV'
+        float x2[NQ];
+        load_cols(tbase + lane_base + C::COL_DVL + grp * NQ, x2);
+#pragma unroll
+        for (int e = 0; e < NQ; ++e) x[e] += x2[e];
+      }
       const float mul = which ? p.scale : 1.f;
 #pragma unroll
-      for (int c = 0; c < NC; c += 8) {
-        uint32_t v[8];
-        tmem_ld8(col + c, v);
-        tmem_wait_ld();
-        uint32_t pk[4];
+      for (int e = 0; e < NQ; ++e) x[e] *= mul;
+      if (f32out) {
+        // fp32 outputs: straight to global
+        const int key = kt * 128 + r;
+        if (key < p.T) {
+          float* out = (which ? p.dk_f32 : p.dv_f32) +
+                       (static_cast<size_t>(bh) * p.T + key) * D + grp * NQ;
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          pk[e] = pack_bf16(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
-        const int d0 = h * NC + c;
-        const int blk = d0 / C::CB;
-        const int dd = d0 % C::CB;
-        st_shared_v4(dst + blk * C::BLOCK_BYTES + swz<C::RB>(r * C::RB + dd * 2), pk[0], pk[1],
-                     pk[2], pk[3]);
+          for (int e = 0; e < NQ; e += 4)
+            reinterpret_cast<float4*>(out + e)[0] = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+        }
+      } else {
+        // bf16 outputs: staged in the dS buffers (dV in sDSH, dK in sDSL)
+        // as the TMA store layout [NCB][128][CB], then stored by TMA
+        const uint32_t dst = which ? sDSL : sDSH;
+        if constexpr (NQ >= 8) {
+#pragma unroll
+          for (int e = 0; e < NQ; e += 8) {
+            const int d0 = grp * NQ + e;  // a multiple of 8: one 16-byte chunk
+            st_shared_v4(dst + (d0 / C::CB) * C::BLOCK_BYTES +
+                             swz<C::RB>(r * C::RB + (d0 % C::CB) * 2),
+                         pack_bf16(x[e], x[e + 1]), pack_bf16(x[e + 2], x[e + 3]),
+                         pack_bf16(x[e + 4], x[e + 5]), pack_bf16(x[e + 6], x[e + 7]));
+          }
+        } else {
+          const int d0 = grp * NQ;      // 4 columns: half of a 16-byte chunk
+          st_shared_v2(dst + (d0 / C::CB) * C::BLOCK_BYTES +
+                           swz<C::RB>(r * C::RB + ((d0 % C::CB) & ~7) * 2) + (d0 & 7) * 2,
+                       pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]));
+        }
       }
     }
-    tc_fence_before();
-    fence_async_smem();
-    named_bar_sync(1, 256);
-    if (leader && !*abort_flag) {
-      for (int b = 0; b < C::NCB; ++b) {
-        tma_store_3d(&tmDV, sDSH + b * C::BLOCK_BYTES, b * C::CB, kt * 128, bh);
-        tma_store_3d(&tmDK, sDSL + b * C::BLOCK_BYTES, b * C::CB, kt * 128, bh);
+    if (f32out) {
+      if (leader) bulk_wait0();  // the dQ reduces have completed
+    } else {
+      tc_fence_before();
+      fence_async_smem();
+      named_bar_sync(1, C::NCOMP);
+      if (leader && !*abort_flag) {
+        for (int b = 0; b < C::NCB; ++b) {
+          tma_store_3d(&tmDV, sDSH + b * C::BLOCK_BYTES, b * C::CB, kt * 128, bh);
+          tma_store_3d(&tmDK, sDSL + b * C::BLOCK_BYTES, b * C::CB, kt * 128, bh);
+        }
+        bulk_commit();
       }
-      bulk_commit();
-    }
-    if (leader) bulk_wait0();  // the dQ reduces and the stores have completed
+      if (leader) bulk_wait0();  // the dQ reduces and the stores have completed
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 17) {
     tc_fence_after();
     tmem_dealloc(tbase, C::TMEM_COLS);
   }

@@ -16,12 +16,18 @@
 //   warps 0-3, 4-7  softmax warpgroups g = 0, 1 for query tiles 2c+g;
 //              thread t of a group owns query row t, which is TMEM lane t.
 //              It reads S_g from TMEM, masks the diagonal tile, updates m
-//              and l, and writes P back over S_g as bf16 hi/lo pairs
-//              (P = hi + lo to ~16 bits); at the end it normalises O_g and
-//              writes O (bf16), optionally O_lo = bf16(O - bf16(O)), and LSE.
+//              and l, and writes P back over S_g: as bf16 (PLO = false, the
+//              usual mixed precision), or as bf16 hi/lo pairs (PLO = true,
+//              P = hi + lo to ~14 bits, used when the caller wants the O_lo
+//              residual, whose purpose is an O accurate to ~fp32); at the end
+//              it normalises O_g and writes O (bf16), with PLO also
+//              O_lo = bf16(O - bf16(O)), and LSE.
 //   warp 8     TMA producer: both Q tiles once, then K_j, V_j through a ring.
 //   warp 9     MMA issuer and TMEM owner.  Per key tile j and group g:
-//              O_g += P_hi V_j + P_lo V_j (A from TMEM), then
+//              O_g += P_hi V_j and O'_g += P_lo V_j (A from TMEM; for D <= 64
+//              into two accumulators, summed at the end, because MMAs that
+//              accumulate into one TMEM tile run back to back at about half
+//              the rate of independent ones), then
 //              S_g(j+1) = Q_g K_{j+1}^T into the same columns.  The MMAs one
 //              thread issues execute in issue order, so S_g(j+1) is issued
 //              right behind PV_g(j) and cannot overwrite P_g(j) before PV_g(j)
@@ -49,7 +55,7 @@ struct FwdParams {
   uint64_t timeout_ns;
 };
 
-template <int D>
+template <int D, bool PLO>
 struct FwdCfg {
   static constexpr int BM = 128, BN = 128;
   static constexpr int CB = D < 64 ? D : 64;      // columns per swizzle block
@@ -71,8 +77,12 @@ struct FwdCfg {
   static constexpr int SMEM_WANT = SMEM_USED + 1024 < 116 * 1024 ? 116 * 1024 : SMEM_USED + 1024;
   static constexpr int SMEM_BYTES = SMEM_WANT <= kMaxDynSmem ? SMEM_WANT : SMEM_USED;
   static_assert(SMEM_USED <= kMaxDynSmem, "shared memory layout too large");
-  // TMEM columns: S_0, S_1 (P hi/lo written over them), O_0, O_1
+  // TMEM columns: S_0, S_1 (P hi/lo written over them), O_0, O_1, and for
+  // D <= 64 the second accumulators O'_0, O'_1 of the P_lo products
+  static constexpr bool SPLIT = PLO && 256 + 4 * D <= 512;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
+  static constexpr uint32_t COL_OL0 = SPLIT ? 256 + 2 * D : COL_O0;
+  static constexpr uint32_t COL_OL1 = SPLIT ? 256 + 3 * D : COL_O1;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int THREADS = 320;
 };
@@ -83,12 +93,12 @@ enum : int {
   FB_ODONE = 14, FB_DRAIN = 16
 };
 
-template <int D>
+template <int D, bool PLO>
 __global__ void __launch_bounds__(320, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
            const __grid_constant__ CUtensorMap tmOlo, const FwdParams p) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, PLO>;
   static_assert(FB_DRAIN < C::NUM_BARS, "barrier count");
   static_assert(FB_KVEMPTY + C::STAGES <= FB_SFULL, "barrier map");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -205,11 +215,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                                       8 * C::RB, C::SW);
         const uint32_t pcol = tbase + (g ? C::COL_S1 : C::COL_S0);
         const uint32_t ocol = tbase + (g ? C::COL_O1 : C::COL_O0);
+        const uint32_t olcol = tbase + (g ? C::COL_OL1 : C::COL_OL0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // 128 keys, 16 per MMA
           const uint64_t b = dv + ((kk * 16 * C::RB) >> 4);
-          mma_ts(ocol, pcol + kk * 8, b, idO, (j > 0 || kk > 0) ? 1u : 0u);
-          mma_ts(ocol, pcol + 64 + kk * 8, b, idO, 1u);
+          const uint32_t first = (j > 0 || kk > 0) ? 1u : 0u;
+          mma_ts(ocol, pcol + kk * 8, b, idO, first);
+          if (PLO) mma_ts(olcol, pcol + 64 + kk * 8, b, idO, C::SPLIT ? first : 1u);
         }
         mma_commit(bar(FB_ODONE + g));
       };
@@ -244,6 +256,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const int q_row = tile * C::BM + row;
     const uint32_t scol = tbase + lane_base + (g ? C::COL_S1 : C::COL_S0);
     const uint32_t ocol = tbase + lane_base + (g ? C::COL_O1 : C::COL_O0);
+    const uint32_t olcol = tbase + lane_base + (g ? C::COL_OL1 : C::COL_OL0);
     const float sl2 = p.scale_log2;
     float m_used = -INFINITY;  // running max, scaled log2 units
     float l = 0.f;
@@ -293,13 +306,17 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       // issued after PV_g(j-1), and the MMAs complete in issue order
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-        for (int cc = 0; cc < D / 16; ++cc) {
-          uint32_t r[16];
-          tmem_ld16(ocol + cc * 16, r);
-          tmem_wait_ld();
+        for (int acc = 0; acc < (C::SPLIT ? 2 : 1); ++acc) {
+          const uint32_t col = acc ? olcol : ocol;
 #pragma unroll
-          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st16(ocol + cc * 16, r);
+          for (int cc = 0; cc < D / 16; ++cc) {
+            uint32_t r[16];
+            tmem_ld16(col + cc * 16, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            tmem_st16(col + cc * 16, r);
+          }
         }
       }
       const uint64_t sl2x2 = f2(sl2, sl2);
@@ -312,12 +329,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         for (int e = 0; e < 8; ++e) {
           float x0, x1;
           f2_split(fma2(f2(s[ch * 16 + 2 * e], s[ch * 16 + 2 * e + 1]), sl2x2, negm2), x0, x1);
-          const uint64_t p2 = f2(ex2(x0), ex2(x1));
+          const float p0 = ex2(x0), p1 = ex2(x1);
+          const uint64_t p2 = f2(p0, p1);
           sum2[e & 1] = add2(sum2[e & 1], p2);
-          split_bf16x2_p(p2, hi[e], lo[e]);
+          if (PLO) split_bf16x2_p(p2, hi[e], lo[e]);
+          else hi[e] = pack_bf16(p0, p1);
         }
         tmem_st8(scol + ch * 8, hi);
-        tmem_st8(scol + 64 + ch * 8, lo);
+        if (PLO) tmem_st8(scol + 64 + ch * 8, lo);
       }
       float sa, sb, sc2, sd;
       f2_split(sum2[0], sa, sb);
@@ -342,7 +361,16 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       for (int cc = 0; cc < D / 16; ++cc) {
         uint32_t r[16];
         tmem_ld16(ocol + cc * 16, r);
-        tmem_wait_ld();
+        if (C::SPLIT) {
+          uint32_t r2[16];
+          tmem_ld16(olcol + cc * 16, r2);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            r[e] = __float_as_uint(__uint_as_float(r[e]) + __uint_as_float(r2[e]));
+        } else {
+          tmem_wait_ld();
+        }
         uint32_t pk[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e)

@@ -318,6 +318,12 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
@@ -471,15 +477,57 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// hi/lo split of a packed pair: hi = bf16x2(x), lo = bf16x2(x - hi).
+// 2^x for a packed pair on the FMA pipes (no ex2 unit): 2^x = 2^j * p(f)
+// with j = round(x) and f = x - j in [-1/2, 1/2]; p is the degree-4 minimax
+// fit of 2^f for relative error (Remez exchange; gen_exp2_poly.py prints
+// these coefficients), max relative error 2.7e-6.  j is formed by adding
+// 1.5 * 2^23, which leaves round(x) in the low mantissa bits; those bits
+// shifted into the exponent field scale p by 2^j.  Inputs are clamped to
+// x >= -126 (results below 2^-126 come out as 2^-126 instead of 0: callers
+// that need exact zeros, e.g. masked scores, must not use this).
+constexpr float kExp2C0 = 0.9999992847442627f;
+constexpr float kExp2C1 = 0.6931217908859253f;
+constexpr float kExp2C2 = 0.240247443318367f;
+constexpr float kExp2C3 = 0.05591785907745361f;
+constexpr float kExp2C4 = 0.009570102207362652f;
+
+__device__ __forceinline__ uint64_t exp2_poly2(float x0, float x1) {
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  const uint64_t magic = f2(12582912.f, 12582912.f);
+  const uint64_t x = f2(x0, x1);
+  const uint64_t t = add2(x, magic);
+  const uint64_t f = sub2(x, sub2(t, magic));
+  uint64_t p = fma2(f2(kExp2C4, kExp2C4), f, f2(kExp2C3, kExp2C3));
+  p = fma2(p, f, f2(kExp2C2, kExp2C2));
+  p = fma2(p, f, f2(kExp2C1, kExp2C1));
+  p = fma2(p, f, f2(kExp2C0, kExp2C0));
+  float t0, t1, p0, p1;
+  f2_split(t, t0, t1);
+  f2_split(p, p0, p1);
+  return f2(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
+            __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
+}
+
+// hi/lo split of a packed pair without conversion instructions: hi is the
+// top half of each fp32 word (bf16 rounded toward zero), lo = x - hi, which
+// is exact in fp32, likewise truncated to bf16.  |x - hi - lo| < 2^-7 |lo|
+// < 2^-14 |x|.  Each bf16x2 word is assembled with one byte permute.
+__device__ __forceinline__ uint32_t top_halves(uint32_t a, uint32_t b) {
+  uint32_t d;  // low half = a's top 16 bits, high half = b's top 16 bits
+  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 __device__ __forceinline__ void split_bf16x2_p(uint64_t x, uint32_t& hi, uint32_t& lo) {
   float x0, x1;
   f2_split(x, x0, x1);
-  hi = pack_bf16(x0, x1);
-  const uint64_t h = f2(__uint_as_float(hi << 16), __uint_as_float(hi & 0xffff0000u));
+  const uint32_t b0 = __float_as_uint(x0), b1 = __float_as_uint(x1);
+  hi = top_halves(b0, b1);
+  const uint64_t h = f2(__uint_as_float(b0 & 0xffff0000u), __uint_as_float(b1 & 0xffff0000u));
   float r0, r1;
   f2_split(sub2(x, h), r0, r1);
-  lo = pack_bf16(r0, r1);
+  lo = top_halves(__float_as_uint(r0), __float_as_uint(r1));
 }
 
 // bf16 hi/lo split of two floats: hi = bf16(x) (round to nearest even) and
@@ -497,6 +545,10 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
                "r"(d)
                : "memory");
+}
+
+__device__ __forceinline__ void st_shared_v2(uint32_t addr, uint32_t a, uint32_t b) {
+  asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
 }
 
 __device__ __forceinline__ void ld_shared_v4f(uint32_t addr, float& a, float& b, float& c,
