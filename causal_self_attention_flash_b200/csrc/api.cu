@@ -305,7 +305,8 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   // these two maps; they then describe q instead
   if ((st = make_bf16_map(&mdk, grad_f32 ? q : dk, D, T, BH)) != CATTN_OK) return st;
   if ((st = make_bf16_map(&mdv, grad_f32 ? q : dv, D, T, BH)) != CATTN_OK) return st;
-  if ((st = make_tmap(&mdq, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, T, BH, C::CBQ, 128)) !=
+  if ((st = make_tmap(&mdq, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, T, BH,
+                      C::WARP_DQ ? D / 4 : C::CBQ, C::WARP_DQ ? 32 : 128)) !=
       CATTN_OK)
     return st;
 

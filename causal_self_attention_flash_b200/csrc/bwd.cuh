@@ -203,7 +203,15 @@ struct BwdCfg {
   static constexpr int OFF_DSL = OFF_DSH + 32768;
   static constexpr int OFF_LSE = OFF_DSL + 32768;             // [QST][128] fp32
   static constexpr int OFF_DELTA = OFF_LSE + QST * 512;       // [QST][128] fp32
-  static constexpr int OFF_BAR = OFF_DELTA + QST * 512;
+  // WARP_DQ (D <= 64): every compute warp drains its own [32 rows][D/4]
+  // slice of dQ through its own fp32 staging tile and TMA reduce, so no
+  // CTA-wide barrier is needed; otherwise the CTA stages all of dQ in the dS
+  // buffers and one thread issues the reduce.
+  static constexpr bool WARP_DQ = D <= 64;
+  static constexpr int RBW = D;                                // (D/4) floats per row
+  static constexpr int WARP_STAGE = (32 * RBW + 1023) / 1024 * 1024;
+  static constexpr int OFF_DQW = (OFF_DELTA + QST * 512 + 1023) / 1024 * 1024;
+  static constexpr int OFF_BAR = WARP_DQ ? OFF_DQW + 16 * WARP_STAGE : OFF_DELTA + QST * 512;
   static constexpr int NUM_BARS = 24;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_USED = OFF_MISC + 64;
@@ -504,6 +512,25 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       }
       tc_fence_before();
       mbar_arrive(bar(BB_DQEMPTY));
+      if constexpr (C::WARP_DQ) {
+        // this warp's tile [32 rows][NQ floats]; its previous reduce must
+        // have finished reading it
+        const uint32_t sW = sbase + C::OFF_DQW + warp * C::WARP_STAGE;
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+#pragma unroll
+        for (int e = 0; e < NQ; e += 4)
+          st_shared_v4(sW + swz<C::RBW>(lane * C::RBW + e * 4), __float_as_uint(acc[e]),
+                       __float_as_uint(acc[e + 1]), __float_as_uint(acc[e + 2]),
+                       __float_as_uint(acc[e + 3]));
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0 && !*abort_flag) {
+          tma_reduce_add_3d(&tmDQacc, sW, grp * NQ, (kt + t) * 128 + quarter * 32, bh);
+          bulk_commit();
+        }
+        return;
+      }
       // staging: blocks of [128 rows][CBQ floats], swizzled
 #pragma unroll
       for (int e = 0; e < NQ; e += 4) {
@@ -526,6 +553,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     };
     // the dS buffers may be rewritten once the reduce has read them
     auto staging_free = [&]() {
+      if constexpr (C::WARP_DQ) return;
       if (leader) bulk_wait_read0();
       named_bar_sync(1, C::NCOMP);
     };
@@ -694,6 +722,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         }
       }
     }
+    if (C::WARP_DQ && lane == 0) bulk_wait0();  // this warp's dQ reduces have completed
     if (f32out) {
       if (leader) bulk_wait0();  // the dQ reduces have completed
     } else {

@@ -12,26 +12,34 @@
 // tensor core alternates between them: while one softmax warpgroup works
 // on its scores, the MMAs of the other run.
 //
-// Warp roles (320 threads):
+// Warp roles (352 threads):
 //   warps 0-3, 4-7  softmax warpgroups g = 0, 1 for query tiles 2c+g;
 //              thread t of a group owns query row t, which is TMEM lane t.
 //              It reads S_g from TMEM, masks the diagonal tile, updates m
-//              and l, and writes P back over S_g: as bf16 (PLO = false, the
-//              usual mixed precision), or as bf16 hi/lo pairs (PLO = true,
-//              P = hi + lo to ~14 bits, used when the caller wants the O_lo
-//              residual, whose purpose is an O accurate to ~fp32); at the end
-//              it normalises O_g and writes O (bf16), with PLO also
+//              and l, and writes P to TMEM: as bf16 (PLO = false, the usual
+//              mixed precision), or as bf16 hi/lo pairs (PLO = true, P = hi +
+//              lo to ~14 bits, used when the caller wants the O_lo residual,
+//              whose purpose is an O accurate to ~fp32); at the end it
+//              normalises O_g and writes O (bf16), with PLO also
 //              O_lo = bf16(O - bf16(O)), and LSE.
 //   warp 8     TMA producer: both Q tiles once, then K_j, V_j through a ring.
-//   warp 9     MMA issuer and TMEM owner.  Per key tile j and group g:
-//              O_g += P_hi V_j and O'_g += P_lo V_j (A from TMEM; for D <= 64
-//              into two accumulators, summed at the end, because MMAs that
-//              accumulate into one TMEM tile run back to back at about half
-//              the rate of independent ones), then
-//              S_g(j+1) = Q_g K_{j+1}^T into the same columns.  The MMAs one
-//              thread issues execute in issue order, so S_g(j+1) is issued
-//              right behind PV_g(j) and cannot overwrite P_g(j) before PV_g(j)
-//              has read it.
+//   warps 9, 10  MMA issuers for groups 0, 1 (warp 9 also owns TMEM).  Two
+//              issuing threads keep the tensor core fed where one thread's
+//              issue rate would not (N = D <= 64 MMAs).  Per key tile j:
+//              O_g += P_hi V_j (A from TMEM), with PLO also O'_g += P_lo V_j
+//              (for D <= 64 into a second accumulator, summed at the end,
+//              because MMAs that accumulate into one TMEM tile run back to
+//              back at about half the rate of independent ones), and
+//              S_g(j+1) = Q_g K_{j+1}^T.
+//
+// Where P lives decides when S_g(j+1) can start (the MMAs one thread issues
+// execute in issue order):
+//   EARLY (bf16 P, D <= 64): P_g has its own TMEM columns.  S_g(j+1) is
+//              issued as soon as the softmax has loaded S_g(j) into registers,
+//              so it runs during the softmax of tile j; the softmax waits for
+//              PV_g(j-1) before it rescales O_g or overwrites P_g.
+//   otherwise  P_g is written over S_g (TMEM holds no room for separate P
+//              columns), and S_g(j+1) is issued right behind PV_g(j).
 //
 // Causal tile skipping: query tile t visits key tiles 0..t only
 // (BM = BN = 128); only the last (diagonal) one is masked.
@@ -70,37 +78,103 @@ struct FwdCfg {
   static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_V + STAGES * TILE_BYTES;
-  static constexpr int NUM_BARS = 20;
+  static constexpr int NUM_BARS = 32;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_USED = OFF_MISC + 64;
   // at least 116 KB so that one CTA holds an SM (it takes all 512 TMEM columns)
   static constexpr int SMEM_WANT = SMEM_USED + 1024 < 116 * 1024 ? 116 * 1024 : SMEM_USED + 1024;
   static constexpr int SMEM_BYTES = SMEM_WANT <= kMaxDynSmem ? SMEM_WANT : SMEM_USED;
   static_assert(SMEM_USED <= kMaxDynSmem, "shared memory layout too large");
-  // TMEM columns: S_0, S_1 (P hi/lo written over them), O_0, O_1, and for
-  // D <= 64 the second accumulators O'_0, O'_1 of the P_lo products
+  // EARLY (bf16 P, D <= 64): P_g has its own 64 TMEM columns, so S_g(j+1)
+  // can be computed while the softmax still works on tile j.  Otherwise P
+  // (bf16, or hi/lo pairs) is written over S_g.
+  static constexpr bool EARLY = !PLO && D <= 64;
+  // TMEM columns: S_0, S_1, [P_0, P_1 if EARLY], O_0, O_1, and with P hi/lo
+  // for D <= 64 the second accumulators O'_0, O'_1 of the P_lo products
   static constexpr bool SPLIT = PLO && 256 + 4 * D <= 512;
-  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128;
+  static constexpr uint32_t COL_P0 = EARLY ? 256 : COL_S0, COL_P1 = EARLY ? 320 : COL_S1;
+  static constexpr uint32_t COL_O0 = EARLY ? 384 : 256, COL_O1 = COL_O0 + D;
   static constexpr uint32_t COL_OL0 = SPLIT ? 256 + 2 * D : COL_O0;
   static constexpr uint32_t COL_OL1 = SPLIT ? 256 + 3 * D : COL_O1;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 352;
 };
+
+// named (hardware) barriers: 1 + g for a group's epilogue, and the turn
+// taking of the two groups' exponential phases
+constexpr uint32_t kBarTurn0 = 3, kBarTurn1 = 4;
 
 // barrier indices
+// (KVEMPTY: one per group and stage, index FB_KVEMPTY + 3 * g + stage; the
+// other per-group barriers at base + g)
 enum : int {
-  FB_Q = 0, FB_KFULL = 1, FB_VFULL = 4, FB_KVEMPTY = 7, FB_SFULL = 10, FB_PFULL = 12,
-  FB_ODONE = 14, FB_DRAIN = 16
+  FB_Q = 0, FB_KFULL = 1, FB_VFULL = 4, FB_KVEMPTY = 7, FB_SFULL = 13, FB_ODONE = 15,
+  FB_SFREE = 17, FB_DRAIN = 19, FB_PFULL = 21  // FB_PFULL + 4 * g + part
 };
 
+// Pairs of score columns whose exponential is taken by exp2_poly2 on the FMA
+// pipes instead of the ex2 unit, as a bit mask over the pair index within a
+// 16-column chunk (3 of 8 pairs): the ex2 unit does 16 per clock per SM, so
+// moving part of the work keeps both pipes busy.  Only used on tiles without
+// masked entries (exp2_poly2 has no exact zero).
+constexpr uint32_t kFwdPolyPairs = 0x00u;
+
+// P_g(j) is handed to the MMA warp in kPvParts parts (of 128 / kPvParts
+// keys each), so PV_g(j) starts while the later exponentials are computed.
+constexpr int kPvParts = 2;
+
+// Turn taking of the two groups' exponential phases (see the softmax loop).
+constexpr bool kFwdTurns = false;
+
+// P = 2^(s * scale_log2 - m) for one row of a 128-column tile: written to
+// TMEM as bf16 (or bf16 hi/lo), the row sum accumulated in sum2.
+template <bool POLY, bool PLO>
+__device__ __forceinline__ void fwd_exp_row(const float (&s)[128], uint64_t sl2x2, uint64_t negm2,
+                                            uint32_t scol, uint64_t (&sum2)[2], uint32_t pfull0) {
+#pragma unroll
+  for (int ch = 0; ch < 8; ++ch) {  // 16 columns per chunk
+    uint32_t hi[8], lo[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const uint64_t x2 = fma2(f2(s[ch * 16 + 2 * e], s[ch * 16 + 2 * e + 1]), sl2x2, negm2);
+      uint64_t p2;
+      if (POLY && ((kFwdPolyPairs >> e) & 1u)) {
+        float x0, x1;
+        f2_split(x2, x0, x1);
+        p2 = exp2_poly2(x0, x1);
+      } else {
+        float x0, x1;
+        f2_split(x2, x0, x1);
+        p2 = f2(ex2(x0), ex2(x1));
+      }
+      sum2[e & 1] = add2(sum2[e & 1], p2);
+      if (PLO) {
+        split_bf16x2_p(p2, hi[e], lo[e]);
+      } else {
+        float p0, p1;
+        f2_split(p2, p0, p1);
+        hi[e] = pack_bf16(p0, p1);
+      }
+    }
+    tmem_st8(scol + ch * 8, hi);
+    if (PLO) tmem_st8(scol + 64 + ch * 8, lo);
+    if ((ch + 1) % (8 / kPvParts) == 0) {  // a part of P is complete: the MMA may read it
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(pfull0 + 8u * ((ch + 1) / (8 / kPvParts) - 1));
+    }
+  }
+}
+
 template <int D, bool PLO>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
            const __grid_constant__ CUtensorMap tmOlo, const FwdParams p) {
   using C = FwdCfg<D, PLO>;
-  static_assert(FB_DRAIN < C::NUM_BARS, "barrier count");
-  static_assert(FB_KVEMPTY + C::STAGES <= FB_SFULL, "barrier map");
+  static_assert(FB_PFULL + 8 <= C::NUM_BARS, "barrier count");
+  static_assert(C::STAGES <= 3, "barrier map");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = aligned_smem(smem_raw, C::SMEM_USED);
   if (smem == nullptr) return;  // uniform over the CTA: nothing touched yet
@@ -129,13 +203,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       mbar_init(bar(FB_KFULL + s), 1);
       mbar_init(bar(FB_VFULL + s), 1);
       mbar_init(bar(FB_KVEMPTY + s), 1);
+      mbar_init(bar(FB_KVEMPTY + 3 + s), 1);
     }
     for (int g = 0; g < 2; ++g) {
       mbar_init(bar(FB_SFULL + g), 1);
-      mbar_init(bar(FB_PFULL + g), 128);
+      for (int h = 0; h < kPvParts; ++h) mbar_init(bar(FB_PFULL + 4 * g + h), 128);
       mbar_init(bar(FB_ODONE + g), 1);
+      mbar_init(bar(FB_SFREE + g), 128);
+      mbar_init(bar(FB_DRAIN + g), 1);
     }
-    mbar_init(bar(FB_DRAIN), 1);
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -161,7 +237,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       int n_issued = 0;
       for (int j = 0; j < n_kv; ++j) {
         const int st = j % C::STAGES;
-        if (j >= C::STAGES) wait1(w, bar(FB_KVEMPTY + st), ((j / C::STAGES) - 1) & 1, 1);
+        if (j >= C::STAGES) {  // the tile this stage held must be released by its users
+          const int jj = j - C::STAGES;
+          const uint32_t ph = (jj / C::STAGES) & 1;
+          if (jj < n0) wait1(w, bar(FB_KVEMPTY + st), ph, 1);
+          if (jj < n1) wait1(w, bar(FB_KVEMPTY + 3 + st), ph, 1);
+        }
         if (*abort_flag) break;
         n_issued = j + 1;
         const uint32_t sK = sbase + C::OFF_K + st * C::TILE_BYTES;
@@ -186,64 +267,67 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         wait1(wd, bar(FB_Q), 0, 13);
       }
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+  } else if (warp >= 9) {
+    // ------------------------------------------------- MMA issuers (one per group)
+    const int g = warp - 9;
+    const int ng = g ? n1 : n0;
+    if (lane == 0 && ng > 0) {
       constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);  // Q K-major, K K-major
       constexpr uint32_t idO = idesc_bf16(128, D, 0, 1);    // P (TMEM), V MN-major
-      auto issue_s = [&](int g, int j) {  // S_g = Q_g K_j^T
+      const uint64_t dq = smem_desc(sbase + C::OFF_Q + g * C::TILE_BYTES, 16, 8 * C::RB, C::SW);
+      const uint32_t scol_t = tbase + (g ? C::COL_S1 : C::COL_S0);
+      const uint32_t pcol_t = tbase + (g ? C::COL_P1 : C::COL_P0);
+      const uint32_t ocol_t = tbase + (g ? C::COL_O1 : C::COL_O0);
+      const uint32_t olcol_t = tbase + (g ? C::COL_OL1 : C::COL_OL0);
+      auto issue_s = [&](int j) {  // S_g = Q_g K_j^T
         const int st = j % C::STAGES;
         wait1(w, bar(FB_KFULL + st), (j / C::STAGES) & 1, 2);
         tc_fence_after();
-        const uint64_t dq = smem_desc(sbase + C::OFF_Q + g * C::TILE_BYTES, 16, 8 * C::RB, C::SW);
         const uint64_t dk = smem_desc(sbase + C::OFF_K + st * C::TILE_BYTES, 16, 8 * C::RB, C::SW);
-        const uint32_t dcol = tbase + (g ? C::COL_S1 : C::COL_S0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int blk = (kk * 16) / C::CB;
           const uint32_t off = (blk * C::BLOCK_BYTES + ((kk * 16) % C::CB) * 2) >> 4;
-          mma_ss(dcol, dq + off, dk + off, idS, kk > 0 ? 1u : 0u);
+          mma_ss(scol_t, dq + off, dk + off, idS, kk > 0 ? 1u : 0u);
         }
         mma_commit(bar(FB_SFULL + g));
       };
-      auto issue_pv = [&](int g, int j) {  // O_g += (P_hi + P_lo) V_j
+      auto issue_pv = [&](int j) {  // O_g += (P_hi + P_lo) V_j
         const int st = j % C::STAGES;
-        wait1(w, bar(FB_PFULL + g), j & 1, 3);
         wait1(w, bar(FB_VFULL + st), (j / C::STAGES) & 1, 4);
-        tc_fence_after();
         const uint64_t dv = smem_desc(sbase + C::OFF_V + st * C::TILE_BYTES, C::BLOCK_BYTES,
                                       8 * C::RB, C::SW);
-        const uint32_t pcol = tbase + (g ? C::COL_S1 : C::COL_S0);
-        const uint32_t ocol = tbase + (g ? C::COL_O1 : C::COL_O0);
-        const uint32_t olcol = tbase + (g ? C::COL_OL1 : C::COL_OL0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // 128 keys, 16 per MMA
+          if (kk % (8 / kPvParts) == 0) {  // the next part of P_g(j) is in TMEM
+            wait1(w, bar(FB_PFULL + 4 * g + kk / (8 / kPvParts)), j & 1, 3);
+            tc_fence_after();
+          }
           const uint64_t b = dv + ((kk * 16 * C::RB) >> 4);
           const uint32_t first = (j > 0 || kk > 0) ? 1u : 0u;
-          mma_ts(ocol, pcol + kk * 8, b, idO, first);
-          if (PLO) mma_ts(olcol, pcol + 64 + kk * 8, b, idO, C::SPLIT ? first : 1u);
+          mma_ts(ocol_t, pcol_t + kk * 8, b, idO, first);
+          if (PLO) mma_ts(olcol_t, pcol_t + 64 + kk * 8, b, idO, C::SPLIT ? first : 1u);
         }
         mma_commit(bar(FB_ODONE + g));
       };
       wait1(w, bar(FB_Q), 0, 5);
-      issue_s(0, 0);
-      if (has1) issue_s(1, 0);
-      for (int j = 0; j < n_kv; ++j) {
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          const int ng = g ? n1 : n0;
-          if (j < ng) {
-            issue_pv(g, j);
-            if (j + 1 < ng) issue_s(g, j + 1);  // in order behind PV_g(j)
-          }
+      issue_s(0);
+      for (int j = 0; j < ng; ++j) {
+        if (C::EARLY && j + 1 < ng) {
+          // S_g(j+1) as soon as the softmax has S_g(j) in registers
+          wait1(w, bar(FB_SFREE + g), j & 1, 6);
+          issue_s(j + 1);
         }
-        mma_commit(bar(FB_KVEMPTY + j % C::STAGES));
+        issue_pv(j);
+        // P over S: S_g(j+1) goes in order behind PV_g(j), which reads P_g(j)
+        if (!C::EARLY && j + 1 < ng) issue_s(j + 1);
+        mma_commit(bar(FB_KVEMPTY + 3 * g + j % C::STAGES));
       }
       // drain: everything issued above has completed before TMEM is freed
-      mma_commit(bar(FB_DRAIN));
+      mma_commit(bar(FB_DRAIN + g));
       int zero = 0;
       WaitCtx wd{p.timeout_ns, &zero, 1u};  // the drain wait ignores the abort flag
-      wait1(wd, bar(FB_DRAIN), 0, 7);
+      wait1(wd, bar(FB_DRAIN + g), 0, 7);
     }
   } else {
     // ------------------------------------------------------------ softmax
@@ -255,6 +339,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const int tile = t0 + g;
     const int q_row = tile * C::BM + row;
     const uint32_t scol = tbase + lane_base + (g ? C::COL_S1 : C::COL_S0);
+    const uint32_t pcol = tbase + lane_base + (g ? C::COL_P1 : C::COL_P0);
     const uint32_t ocol = tbase + lane_base + (g ? C::COL_O1 : C::COL_O0);
     const uint32_t olcol = tbase + lane_base + (g ? C::COL_OL1 : C::COL_OL0);
     const float sl2 = p.scale_log2;
@@ -279,6 +364,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           s[96 + e] = __uint_as_float(r3[e]);
         }
       }
+      if (C::EARLY) {  // S_g may now be overwritten by S_g(j+1)
+        tc_fence_before();
+        mbar_arrive(bar(FB_SFREE + g));
+      }
       if (j == ng - 1) {  // diagonal tile: key column > query row is future
 #pragma unroll
         for (int cc = 0; cc < 128; ++cc)
@@ -302,8 +391,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         alpha = ex2(m_used - m_new);  // 0 on the first tile (m_used = -inf)
         m_used = m_new;
       }
-      // O_g is stable here: S_g(j), whose completion was just observed, was
-      // issued after PV_g(j-1), and the MMAs complete in issue order
+      // O_g must be stable before it is rescaled, and P_g(j-1) read before
+      // P_g(j) is written.  Over S (not EARLY): S_g(j), whose completion was
+      // just observed, was issued after PV_g(j-1), and MMAs complete in issue
+      // order.  EARLY: wait for PV_g(j-1) itself.
+      if (C::EARLY && j > 0) {
+        wait_warp(w, bar(FB_ODONE + g), (j - 1) & 1, 9);
+        tc_fence_after();
+      }
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
         for (int acc = 0; acc < (C::SPLIT ? 2 : 1); ++acc) {
@@ -322,29 +417,27 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       const uint64_t sl2x2 = f2(sl2, sl2);
       const uint64_t negm2 = f2(-m_used, -m_used);
       uint64_t sum2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {  // 16 columns per chunk
-        uint32_t hi[8], lo[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float x0, x1;
-          f2_split(fma2(f2(s[ch * 16 + 2 * e], s[ch * 16 + 2 * e + 1]), sl2x2, negm2), x0, x1);
-          const float p0 = ex2(x0), p1 = ex2(x1);
-          const uint64_t p2 = f2(p0, p1);
-          sum2[e & 1] = add2(sum2[e & 1], p2);
-          if (PLO) split_bf16x2_p(p2, hi[e], lo[e]);
-          else hi[e] = pack_bf16(p0, p1);
+      // The two groups take turns at the exponentials (g0 tile j, g1 tile j,
+      // g0 tile j+1, ...): the ex2 unit is the scarcest resource of the
+      // softmax, and while one group uses it the other does its loads, row
+      // maxima and rescaling.  Group 1 has one tile more than group 0.
+      if (kFwdTurns && has1) {
+        if (g == 0) {
+          if (j > 0) named_bar_sync(kBarTurn1, 256);    // g1 finished tile j-1
+        } else if (j < n0) {
+          named_bar_sync(kBarTurn0, 256);               // g0 finished tile j
         }
-        tmem_st8(scol + ch * 8, hi);
-        if (PLO) tmem_st8(scol + 64 + ch * 8, lo);
+      }
+      if (j == ng - 1) fwd_exp_row<false, PLO>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g));
+      else fwd_exp_row<true, PLO>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g));
+      if (kFwdTurns && has1) {
+        if (g == 0) named_bar_arrive(kBarTurn0, 256);
+        else if (j + 1 < n0) named_bar_arrive(kBarTurn1, 256);
       }
       float sa, sb, sc2, sd;
       f2_split(sum2[0], sa, sb);
       f2_split(sum2[1], sc2, sd);
       l = l * alpha + ((sa + sb) + (sc2 + sd));
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(FB_PFULL + g));
     }
 
     // ---------------------------------------------------------- epilogue
