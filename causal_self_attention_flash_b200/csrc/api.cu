@@ -42,6 +42,7 @@ cattn_status cuda_fail(int code) {
 }
 int g_dev_ok[kMaxDevices];           // 0 unknown, 1 sm_100, -1 other
 unsigned g_attr_done[kMaxDevices];   // bit per kernel instance
+int g_sm_count[kMaxDevices];         // multiprocessors (persistent grids)
 
 cattn_status init_encode() {
   std::lock_guard<std::mutex> lk(g_mu);
@@ -76,6 +77,10 @@ cattn_status check_device(int* dev_out) {
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
       return cuda_fail(cudaGetLastError());
     }
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return cuda_fail(cudaGetLastError());
+    g_sm_count[dev] = sms > 0 ? sms : 1;
     g_dev_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
   }
   if (g_dev_ok[dev] != 1) return CATTN_ERR_UNSUPPORTED;
@@ -223,10 +228,15 @@ cattn_status fwd_impl(int dev, const void* q, const void* k, const void* v, floa
   p.lse = lse;
   p.write_o_lo = o_lo != nullptr;
   p.T = T;
+  p.BH = BH;
   p.n_qtiles = (T + 127) / 128;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_timeout_ns;
-  dim3 grid(BH, (p.n_qtiles + 1) / 2);  // two query tiles per CTA
+  // persistent: one CTA per SM (it holds all of an SM's TMEM), each looping
+  // over work items of two query tiles
+  const long long n_items = static_cast<long long>(BH) * ((p.n_qtiles + 1) / 2);
+  if (n_items > 0x7fffffffLL) return CATTN_ERR_INVALID_ARG;
+  dim3 grid(static_cast<unsigned>(n_items < g_sm_count[dev] ? n_items : g_sm_count[dev]));
   {
     LaunchTimer t(K_FWD, s);
     fwd_kernel<D, PLO><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, molo, p);

@@ -529,33 +529,35 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           tma_reduce_add_3d(&tmDQacc, sW, grp * NQ, (kt + t) * 128 + quarter * 32, bh);
           bulk_commit();
         }
-        return;
-      }
-      // staging: blocks of [128 rows][CBQ floats], swizzled
+      } else {
+        // staging: blocks of [128 rows][CBQ floats], swizzled
 #pragma unroll
-      for (int e = 0; e < NQ; e += 4) {
-        const int f = grp * NQ + e;
-        const int blk = f / C::CBQ;
-        const int within = (f % C::CBQ) * 4;
-        st_shared_v4(sDSH + blk * 128 * C::RBQ + swz<C::RBQ>(r * C::RBQ + within),
-                     __float_as_uint(acc[e]), __float_as_uint(acc[e + 1]),
-                     __float_as_uint(acc[e + 2]), __float_as_uint(acc[e + 3]));
-      }
-      fence_async_smem();
-      named_bar_sync(1, C::NCOMP);
-      if (leader && !*abort_flag) {
+        for (int e = 0; e < NQ; e += 4) {
+          const int f = grp * NQ + e;
+          const int blk = f / C::CBQ;
+          const int within = (f % C::CBQ) * 4;
+          st_shared_v4(sDSH + blk * 128 * C::RBQ + swz<C::RBQ>(r * C::RBQ + within),
+                       __float_as_uint(acc[e]), __float_as_uint(acc[e + 1]),
+                       __float_as_uint(acc[e + 2]), __float_as_uint(acc[e + 3]));
+        }
+        fence_async_smem();
+        named_bar_sync(1, C::NCOMP);
+        if (leader && !*abort_flag) {
 #pragma unroll
-        for (int blk = 0; blk < D / C::CBQ; ++blk)
-          tma_reduce_add_3d(&tmDQacc, sDSH + blk * 128 * C::RBQ, blk * C::CBQ, (kt + t) * 128,
-                            bh);
-        bulk_commit();
+          for (int blk = 0; blk < D / C::CBQ; ++blk)
+            tma_reduce_add_3d(&tmDQacc, sDSH + blk * 128 * C::RBQ, blk * C::CBQ,
+                              (kt + t) * 128, bh);
+          bulk_commit();
+        }
       }
     };
-    // the dS buffers may be rewritten once the reduce has read them
+    // the dS buffers may be rewritten once the reduce has read them (CTA
+    // staging only)
     auto staging_free = [&]() {
-      if constexpr (C::WARP_DQ) return;
-      if (leader) bulk_wait_read0();
-      named_bar_sync(1, C::NCOMP);
+      if constexpr (!C::WARP_DQ) {
+        if (leader) bulk_wait_read0();
+        named_bar_sync(1, C::NCOMP);
+      }
     };
 
     float pv[32];
@@ -722,9 +724,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         }
       }
     }
-    if (C::WARP_DQ && lane == 0) bulk_wait0();  // this warp's dQ reduces have completed
+    // before the CTA exits, its bulk copies must have read their shared
+    // memory sources (their global writes complete on their own; the next
+    // kernel on the stream sees them)
+    if (C::WARP_DQ && lane == 0) bulk_wait_read0();
     if (f32out) {
-      if (leader) bulk_wait0();  // the dQ reduces have completed
+      if (leader) bulk_wait_read0();
     } else {
       tc_fence_before();
       fence_async_smem();
@@ -736,7 +741,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         }
         bulk_commit();
       }
-      if (leader) bulk_wait0();  // the dQ reduces and the stores have completed
+      if (leader) bulk_wait_read0();
     }
   }
 

@@ -58,6 +58,7 @@ struct FwdParams {
   float* lse;          // (BH, T) fp32 out
   int write_o_lo;      // also write O_lo = bf16(O - bf16(O)) through tmOlo
   int T;
+  int BH;
   int n_qtiles;
   float scale_log2;    // scale * log2(e)
   uint64_t timeout_ns;
@@ -77,8 +78,12 @@ struct FwdCfg {
   static constexpr int OFF_Q = 0;                              // [2] query tiles
   static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_V + STAGES * TILE_BYTES;
-  static constexpr int NUM_BARS = 32;
+  // SEP_O: the O epilogue has its own staging tiles (where they fit), so the
+  // next item's Q can be loaded while this item's O is stored
+  static constexpr int OFF_OST = OFF_V + STAGES * TILE_BYTES;
+  static constexpr bool SEP_O = OFF_OST + 2 * TILE_BYTES + 1024 <= kMaxDynSmem;
+  static constexpr int OFF_BAR = OFF_OST + (SEP_O ? 2 * TILE_BYTES : 0);
+  static constexpr int NUM_BARS = 34;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_USED = OFF_MISC + 64;
   // at least 116 KB so that one CTA holds an SM (it takes all 512 TMEM columns)
@@ -101,16 +106,14 @@ struct FwdCfg {
   static constexpr int THREADS = 352;
 };
 
-// named (hardware) barriers: 1 + g for a group's epilogue, and the turn
-// taking of the two groups' exponential phases
-constexpr uint32_t kBarTurn0 = 3, kBarTurn1 = 4;
-
+// named (hardware) barriers: 1 + g for a group's epilogue
 // barrier indices
 // (KVEMPTY: one per group and stage, index FB_KVEMPTY + 3 * g + stage; the
 // other per-group barriers at base + g)
 enum : int {
-  FB_Q = 0, FB_KFULL = 1, FB_VFULL = 4, FB_KVEMPTY = 7, FB_SFULL = 13, FB_ODONE = 15,
-  FB_SFREE = 17, FB_DRAIN = 19, FB_PFULL = 21  // FB_PFULL + 4 * g + part
+  FB_KFULL = 0, FB_VFULL = 3, FB_KVEMPTY = 6, FB_QFULL = 12, FB_QFREE = 14, FB_SFULL = 16,
+  FB_ODONE = 18, FB_OFREE = 20, FB_SFREE = 22, FB_DRAIN = 24,
+  FB_PFULL = 26  // FB_PFULL + 4 * g + part
 };
 
 // Pairs of score columns whose exponential is taken by exp2_poly2 on the FMA
@@ -123,9 +126,6 @@ constexpr uint32_t kFwdPolyPairs = 0x00u;
 // P_g(j) is handed to the MMA warp in kPvParts parts (of 128 / kPvParts
 // keys each), so PV_g(j) starts while the later exponentials are computed.
 constexpr int kPvParts = 2;
-
-// Turn taking of the two groups' exponential phases (see the softmax loop).
-constexpr bool kFwdTurns = false;
 
 // P = 2^(s * scale_log2 - m) for one row of a 128-column tile: written to
 // TMEM as bf16 (or bf16 hi/lo), the row sum accumulated in sum2.
@@ -167,6 +167,32 @@ __device__ __forceinline__ void fwd_exp_row(const float (&s)[128], uint64_t sl2x
   }
 }
 
+// Work items: pairs (c, bh) of query tiles 2c, 2c+1 of head bh, numbered
+// longest first (u = 0 .. BH*n_pairs-1: c = n_pairs-1 - u / BH, bh = u % BH).
+// The grid is persistent (at most one CTA per SM); CTA b takes items in
+// passes over the grid, alternating direction, so that every CTA gets a
+// similar mix of long and short items: pass k takes item k*G + b (k even)
+// or k*G + G-1-b (k odd).  Returns -1 past the last item.
+__device__ __forceinline__ int fwd_item(int k, int b, int G, int n_items) {
+  const int u = k * G + ((k & 1) ? G - 1 - b : b);
+  return u < n_items ? u : -1;
+}
+
+struct FwdItem {
+  int bh, t0, n0, n1, n_kv;  // query tiles t0 (n0 key tiles), t0+1 (n1, 0 if absent)
+};
+
+__device__ __forceinline__ FwdItem fwd_item_info(int u, int BH, int n_pairs, int n_qtiles) {
+  FwdItem it;
+  const int c = n_pairs - 1 - u / BH;
+  it.bh = u % BH;
+  it.t0 = 2 * c;
+  it.n0 = it.t0 + 1;
+  it.n1 = it.t0 + 1 < n_qtiles ? it.t0 + 2 : 0;
+  it.n_kv = it.n1 ? it.n1 : it.n0;
+  return it;
+}
+
 template <int D, bool PLO>
 __global__ void __launch_bounds__(352, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -185,20 +211,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
   const int n_pairs = (p.n_qtiles + 1) >> 1;
-  const int c = n_pairs - 1 - blockIdx.y;  // longest (most key tiles) first
-  const int t0 = 2 * c;                    // query tiles t0, t0 + 1
-  const bool has1 = t0 + 1 < p.n_qtiles;
-  const int n0 = t0 + 1;                   // key tiles seen by query tile t0
-  const int n1 = has1 ? t0 + 2 : 0;
-  const int n_kv = has1 ? n1 : n0;
+  const int n_items = p.BH * n_pairs;
+  const int G = gridDim.x, b = blockIdx.x;
 
   WaitCtx w{p.timeout_ns, abort_flag, 1u};
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    mbar_init(bar(FB_Q), 1);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(bar(FB_KFULL + s), 1);
       mbar_init(bar(FB_VFULL + s), 1);
@@ -206,9 +226,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       mbar_init(bar(FB_KVEMPTY + 3 + s), 1);
     }
     for (int g = 0; g < 2; ++g) {
+      mbar_init(bar(FB_QFULL + g), 1);
+      mbar_init(bar(FB_QFREE + g), C::SEP_O ? 1 : 2);
       mbar_init(bar(FB_SFULL + g), 1);
       for (int h = 0; h < kPvParts; ++h) mbar_init(bar(FB_PFULL + 4 * g + h), 128);
       mbar_init(bar(FB_ODONE + g), 1);
+      mbar_init(bar(FB_OFREE + g), 128);
       mbar_init(bar(FB_SFREE + g), 128);
       mbar_init(bar(FB_DRAIN + g), 1);
     }
@@ -225,53 +248,69 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
+    // Per item: Q_g once the previous item no longer needs the Q_g buffer,
+    // then K_j, V_j through a ring that runs on across items (tk counts the
+    // CTA's K/V tiles).
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(bar(FB_Q), (has1 ? 2 : 1) * C::TILE_BYTES);
-      for (int g = 0; g < (has1 ? 2 : 1); ++g)
-        for (int b = 0; b < C::NCB; ++b)
-          tma_load_3d(sbase + C::OFF_Q + g * C::TILE_BYTES + b * C::BLOCK_BYTES, &tmQ,
-                      bar(FB_Q), b * C::CB, (t0 + g) * C::BM, bh);
-      int n_issued = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        const int st = j % C::STAGES;
-        if (j >= C::STAGES) {  // the tile this stage held must be released by its users
-          const int jj = j - C::STAGES;
-          const uint32_t ph = (jj / C::STAGES) & 1;
-          if (jj < n0) wait1(w, bar(FB_KVEMPTY + st), ph, 1);
-          if (jj < n1) wait1(w, bar(FB_KVEMPTY + 3 + st), ph, 1);
+      int tk = 0, aq[2] = {0, 0};
+      for (int k = 0;; ++k) {
+        const int u = fwd_item(k, b, G, n_items);
+        if (u < 0 || *abort_flag) break;
+        const FwdItem it = fwd_item_info(u, p.BH, n_pairs, p.n_qtiles);
+        for (int g = 0; g < 2; ++g) {
+          if ((g ? it.n1 : it.n0) == 0) continue;
+          if (aq[g] > 0) wait1(w, bar(FB_QFREE + g), (aq[g] - 1) & 1, 1);
+          mbar_arrive_expect_tx(bar(FB_QFULL + g), C::TILE_BYTES);
+          for (int bb = 0; bb < C::NCB; ++bb)
+            tma_load_3d(sbase + C::OFF_Q + g * C::TILE_BYTES + bb * C::BLOCK_BYTES, &tmQ,
+                        bar(FB_QFULL + g), bb * C::CB, (it.t0 + g) * C::BM, it.bh);
+          ++aq[g];
         }
-        if (*abort_flag) break;
-        n_issued = j + 1;
-        const uint32_t sK = sbase + C::OFF_K + st * C::TILE_BYTES;
-        const uint32_t sV = sbase + C::OFF_V + st * C::TILE_BYTES;
-        mbar_arrive_expect_tx(bar(FB_KFULL + st), C::TILE_BYTES);
-        for (int b = 0; b < C::NCB; ++b)
-          tma_load_3d(sK + b * C::BLOCK_BYTES, &tmK, bar(FB_KFULL + st), b * C::CB, j * C::BN, bh);
-        mbar_arrive_expect_tx(bar(FB_VFULL + st), C::TILE_BYTES);
-        for (int b = 0; b < C::NCB; ++b)
-          tma_load_3d(sV + b * C::BLOCK_BYTES, &tmV, bar(FB_VFULL + st), b * C::CB, j * C::BN, bh);
+        for (int j = 0; j < it.n_kv; ++j, ++tk) {
+          const int st = tk % C::STAGES;
+          if (tk >= C::STAGES) {  // both groups have released the tile this stage held
+            const uint32_t ph = ((tk / C::STAGES) - 1) & 1;
+            wait1(w, bar(FB_KVEMPTY + st), ph, 1);
+            wait1(w, bar(FB_KVEMPTY + 3 + st), ph, 1);
+          }
+          if (*abort_flag) break;
+          const uint32_t sK = sbase + C::OFF_K + st * C::TILE_BYTES;
+          const uint32_t sV = sbase + C::OFF_V + st * C::TILE_BYTES;
+          mbar_arrive_expect_tx(bar(FB_KFULL + st), C::TILE_BYTES);
+          for (int bb = 0; bb < C::NCB; ++bb)
+            tma_load_3d(sK + bb * C::BLOCK_BYTES, &tmK, bar(FB_KFULL + st), bb * C::CB,
+                        j * C::BN, it.bh);
+          mbar_arrive_expect_tx(bar(FB_VFULL + st), C::TILE_BYTES);
+          for (int bb = 0; bb < C::NCB; ++bb)
+            tma_load_3d(sV + bb * C::BLOCK_BYTES, &tmV, bar(FB_VFULL + st), bb * C::CB,
+                        j * C::BN, it.bh);
+        }
       }
       if (*abort_flag) {
-        // abort path: wait (bounded, ignoring the abort flag) for the loads
-        // this thread issued that nobody consumed, before the CTA exits
+        // abort path: wait (bounded, ignoring the abort flag) for the last
+        // loads this thread issued, which may not have been consumed, before
+        // the CTA exits
         int zero = 0;
         WaitCtx wd{p.timeout_ns, &zero, 1u};
-        for (int j = (n_issued > C::STAGES ? n_issued - C::STAGES : 0); j < n_issued; ++j) {
-          const int st = j % C::STAGES;
-          wait1(wd, bar(FB_KFULL + st), (j / C::STAGES) & 1, 11);
-          wait1(wd, bar(FB_VFULL + st), (j / C::STAGES) & 1, 12);
+        for (int t = (tk > C::STAGES ? tk - C::STAGES : 0); t < tk; ++t) {
+          const int st = t % C::STAGES;
+          wait1(wd, bar(FB_KFULL + st), (t / C::STAGES) & 1, 11);
+          wait1(wd, bar(FB_VFULL + st), (t / C::STAGES) & 1, 12);
         }
-        wait1(wd, bar(FB_Q), 0, 13);
+        for (int g = 0; g < 2; ++g)
+          if (aq[g] > 0) wait1(wd, bar(FB_QFULL + g), (aq[g] - 1) & 1, 13);
       }
     }
   } else if (warp >= 9) {
     // ------------------------------------------------- MMA issuers (one per group)
+    // Running counters across items: tg = tiles of this group so far (the
+    // phase of its S/P/O barriers), aq = items of this group so far (Q and
+    // O hand-over), tk = K/V ring position.
     const int g = warp - 9;
-    const int ng = g ? n1 : n0;
-    if (lane == 0 && ng > 0) {
+    if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);  // Q K-major, K K-major
       constexpr uint32_t idO = idesc_bf16(128, D, 0, 1);    // P (TMEM), V MN-major
       const uint64_t dq = smem_desc(sbase + C::OFF_Q + g * C::TILE_BYTES, 16, 8 * C::RB, C::SW);
@@ -279,9 +318,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       const uint32_t pcol_t = tbase + (g ? C::COL_P1 : C::COL_P0);
       const uint32_t ocol_t = tbase + (g ? C::COL_O1 : C::COL_O0);
       const uint32_t olcol_t = tbase + (g ? C::COL_OL1 : C::COL_OL0);
-      auto issue_s = [&](int j) {  // S_g = Q_g K_j^T
-        const int st = j % C::STAGES;
-        wait1(w, bar(FB_KFULL + st), (j / C::STAGES) & 1, 2);
+      int tg = 0, aq = 0, tk = 0;
+      auto issue_s = [&](int j, int tkj) {  // S_g = Q_g K_j^T
+        const int st = tkj % C::STAGES;
+        wait1(w, bar(FB_KFULL + st), (tkj / C::STAGES) & 1, 2);
         tc_fence_after();
         const uint64_t dk = smem_desc(sbase + C::OFF_K + st * C::TILE_BYTES, 16, 8 * C::RB, C::SW);
 #pragma unroll
@@ -292,36 +332,66 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         }
         mma_commit(bar(FB_SFULL + g));
       };
-      auto issue_pv = [&](int j) {  // O_g += (P_hi + P_lo) V_j
-        const int st = j % C::STAGES;
-        wait1(w, bar(FB_VFULL + st), (j / C::STAGES) & 1, 4);
+      auto issue_pv = [&](int j, int tkj, int tgj) {  // O_g += (P_hi + P_lo) V_j
+        const int st = tkj % C::STAGES;
+        wait1(w, bar(FB_VFULL + st), (tkj / C::STAGES) & 1, 4);
         const uint64_t dv = smem_desc(sbase + C::OFF_V + st * C::TILE_BYTES, C::BLOCK_BYTES,
                                       8 * C::RB, C::SW);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // 128 keys, 16 per MMA
           if (kk % (8 / kPvParts) == 0) {  // the next part of P_g(j) is in TMEM
-            wait1(w, bar(FB_PFULL + 4 * g + kk / (8 / kPvParts)), j & 1, 3);
+            wait1(w, bar(FB_PFULL + 4 * g + kk / (8 / kPvParts)), tgj & 1, 3);
             tc_fence_after();
           }
-          const uint64_t b = dv + ((kk * 16 * C::RB) >> 4);
+          const uint64_t bdesc = dv + ((kk * 16 * C::RB) >> 4);
           const uint32_t first = (j > 0 || kk > 0) ? 1u : 0u;
-          mma_ts(ocol_t, pcol_t + kk * 8, b, idO, first);
-          if (PLO) mma_ts(olcol_t, pcol_t + 64 + kk * 8, b, idO, C::SPLIT ? first : 1u);
+          mma_ts(ocol_t, pcol_t + kk * 8, bdesc, idO, first);
+          if (PLO) mma_ts(olcol_t, pcol_t + 64 + kk * 8, bdesc, idO, C::SPLIT ? first : 1u);
         }
         mma_commit(bar(FB_ODONE + g));
       };
-      wait1(w, bar(FB_Q), 0, 5);
-      issue_s(0);
-      for (int j = 0; j < ng; ++j) {
-        if (C::EARLY && j + 1 < ng) {
-          // S_g(j+1) as soon as the softmax has S_g(j) in registers
-          wait1(w, bar(FB_SFREE + g), j & 1, 6);
-          issue_s(j + 1);
+      for (int k = 0;; ++k) {
+        const int u = fwd_item(k, b, G, n_items);
+        if (u < 0) break;
+        const FwdItem it = fwd_item_info(u, p.BH, n_pairs, p.n_qtiles);
+        const int ng = g ? it.n1 : it.n0;
+        if (ng > 0) {
+          wait1(w, bar(FB_QFULL + g), aq & 1, 5);
+          // EARLY: S_g is read by the softmax before S_g(0) may overwrite it
+          if (C::EARLY && tg > 0) wait1(w, bar(FB_SFREE + g), (tg - 1) & 1, 6);
+          issue_s(0, tk);
+          if (ng == 1) mma_commit(bar(FB_QFREE + g));  // last read of Q_g issued
+          for (int j = 0; j < ng; ++j) {
+            if (C::EARLY && j + 1 < ng) {
+              // S_g(j+1) as soon as the softmax has S_g(j) in registers
+              wait1(w, bar(FB_SFREE + g), (tg + j) & 1, 6);
+              issue_s(j + 1, tk + j + 1);
+              if (j + 2 == ng) mma_commit(bar(FB_QFREE + g));
+            }
+            // O_g is overwritten by PV_g(0): the epilogue of the previous
+            // item must have read it
+            if (j == 0 && aq > 0) wait1(w, bar(FB_OFREE + g), (aq - 1) & 1, 8);
+            issue_pv(j, tk + j, tg + j);
+            // P over S: S_g(j+1) goes in order behind PV_g(j), which reads P_g(j)
+            if (!C::EARLY && j + 1 < ng) {
+              issue_s(j + 1, tk + j + 1);
+              if (j + 2 == ng) mma_commit(bar(FB_QFREE + g));
+            }
+            mma_commit(bar(FB_KVEMPTY + 3 * g + (tk + j) % C::STAGES));
+          }
+          tg += ng;
+          ++aq;
         }
-        issue_pv(j);
-        // P over S: S_g(j+1) goes in order behind PV_g(j), which reads P_g(j)
-        if (!C::EARLY && j + 1 < ng) issue_s(j + 1);
-        mma_commit(bar(FB_KVEMPTY + 3 * g + j % C::STAGES));
+        // K/V tiles of this item that this group does not use: released once
+        // loaded (never earlier: a release of a tile not yet loaded would
+        // complete two phases of the stage's barrier before the producer
+        // waits, and its parity wait would then not see them)
+        for (int j = ng; j < it.n_kv; ++j) {
+          const int t = tk + j;
+          wait1(w, bar(FB_KFULL + t % C::STAGES), (t / C::STAGES) & 1, 2);
+          mma_commit(bar(FB_KVEMPTY + 3 * g + t % C::STAGES));
+        }
+        tk += it.n_kv;
       }
       // drain: everything issued above has completed before TMEM is freed
       mma_commit(bar(FB_DRAIN + g));
@@ -335,121 +405,114 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;     // query row in tile == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const int ng = g ? n1 : n0;
-    const int tile = t0 + g;
-    const int q_row = tile * C::BM + row;
     const uint32_t scol = tbase + lane_base + (g ? C::COL_S1 : C::COL_S0);
     const uint32_t pcol = tbase + lane_base + (g ? C::COL_P1 : C::COL_P0);
     const uint32_t ocol = tbase + lane_base + (g ? C::COL_O1 : C::COL_O0);
     const uint32_t olcol = tbase + lane_base + (g ? C::COL_OL1 : C::COL_OL0);
+    const uint32_t sQg = sbase + C::OFF_Q + g * C::TILE_BYTES;
+    const uint32_t sOg = C::SEP_O ? sbase + C::OFF_OST + g * C::TILE_BYTES : sQg;
+    const uint32_t nbar = 1 + g;
+    const bool leader = (threadIdx.x & 127) == 0;
     const float sl2 = p.scale_log2;
-    float m_used = -INFINITY;  // running max, scaled log2 units
-    float l = 0.f;
+    int tg = 0;
     float s[128];
-    for (int j = 0; j < ng; ++j) {
-      wait_warp(w, bar(FB_SFULL + g), j & 1, 8);
-      tc_fence_after();
-      {
-        uint32_t r0[32], r1[32], r2[32], r3[32];
-        tmem_ld32(scol, r0);
-        tmem_ld32(scol + 32, r1);
-        tmem_ld32(scol + 64, r2);
-        tmem_ld32(scol + 96, r3);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          s[e] = __uint_as_float(r0[e]);
-          s[32 + e] = __uint_as_float(r1[e]);
-          s[64 + e] = __uint_as_float(r2[e]);
-          s[96 + e] = __uint_as_float(r3[e]);
-        }
-      }
-      if (C::EARLY) {  // S_g may now be overwritten by S_g(j+1)
-        tc_fence_before();
-        mbar_arrive(bar(FB_SFREE + g));
-      }
-      if (j == ng - 1) {  // diagonal tile: key column > query row is future
-#pragma unroll
-        for (int cc = 0; cc < 128; ++cc)
-          if (cc > row) s[cc] = -INFINITY;
-      }
-      float mx[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) mx[i] = fmax3(s[i], s[4 + i], s[8 + i]);
-#pragma unroll
-      for (int cc = 12; cc < 124; cc += 8)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) mx[i] = fmax3(mx[i], s[cc + i], s[cc + 4 + i]);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) mx[i] = fmaxf(mx[i], s[124 + i]);
-      const float mxa = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
-      const float m_tile = mxa * sl2;
-      float alpha = 1.f;
-      const bool move = (j == 0) || (m_tile > m_used + 8.f);
-      if (move) {
-        const float m_new = fmaxf(m_used, m_tile);
-        alpha = ex2(m_used - m_new);  // 0 on the first tile (m_used = -inf)
-        m_used = m_new;
-      }
-      // O_g must be stable before it is rescaled, and P_g(j-1) read before
-      // P_g(j) is written.  Over S (not EARLY): S_g(j), whose completion was
-      // just observed, was issued after PV_g(j-1), and MMAs complete in issue
-      // order.  EARLY: wait for PV_g(j-1) itself.
-      if (C::EARLY && j > 0) {
-        wait_warp(w, bar(FB_ODONE + g), (j - 1) & 1, 9);
+    for (int k = 0;; ++k) {
+      const int u = fwd_item(k, b, G, n_items);
+      if (u < 0) break;
+      const FwdItem it = fwd_item_info(u, p.BH, n_pairs, p.n_qtiles);
+      const int ng = g ? it.n1 : it.n0;
+      if (ng == 0) continue;
+      float m_used = -INFINITY;  // running max, scaled log2 units
+      float l = 0.f;
+      for (int j = 0; j < ng; ++j) {
+        const int tgj = tg + j;
+        wait_warp(w, bar(FB_SFULL + g), tgj & 1, 8);
         tc_fence_after();
-      }
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        {
+          uint32_t r0[32], r1[32], r2[32], r3[32];
+          tmem_ld32(scol, r0);
+          tmem_ld32(scol + 32, r1);
+          tmem_ld32(scol + 64, r2);
+          tmem_ld32(scol + 96, r3);
+          tmem_wait_ld();
 #pragma unroll
-        for (int acc = 0; acc < (C::SPLIT ? 2 : 1); ++acc) {
-          const uint32_t col = acc ? olcol : ocol;
-#pragma unroll
-          for (int cc = 0; cc < D / 16; ++cc) {
-            uint32_t r[16];
-            tmem_ld16(col + cc * 16, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st16(col + cc * 16, r);
+          for (int e = 0; e < 32; ++e) {
+            s[e] = __uint_as_float(r0[e]);
+            s[32 + e] = __uint_as_float(r1[e]);
+            s[64 + e] = __uint_as_float(r2[e]);
+            s[96 + e] = __uint_as_float(r3[e]);
           }
         }
-      }
-      const uint64_t sl2x2 = f2(sl2, sl2);
-      const uint64_t negm2 = f2(-m_used, -m_used);
-      uint64_t sum2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
-      // The two groups take turns at the exponentials (g0 tile j, g1 tile j,
-      // g0 tile j+1, ...): the ex2 unit is the scarcest resource of the
-      // softmax, and while one group uses it the other does its loads, row
-      // maxima and rescaling.  Group 1 has one tile more than group 0.
-      if (kFwdTurns && has1) {
-        if (g == 0) {
-          if (j > 0) named_bar_sync(kBarTurn1, 256);    // g1 finished tile j-1
-        } else if (j < n0) {
-          named_bar_sync(kBarTurn0, 256);               // g0 finished tile j
+        if (C::EARLY) {  // S_g may now be overwritten by the next score tile
+          tc_fence_before();
+          mbar_arrive(bar(FB_SFREE + g));
         }
+        if (j == ng - 1) {  // diagonal tile: key column > query row is future
+#pragma unroll
+          for (int cc = 0; cc < 128; ++cc)
+            if (cc > row) s[cc] = -INFINITY;
+        }
+        float mx[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mx[i] = fmax3(s[i], s[4 + i], s[8 + i]);
+#pragma unroll
+        for (int cc = 12; cc < 124; cc += 8)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) mx[i] = fmax3(mx[i], s[cc + i], s[cc + 4 + i]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mx[i] = fmaxf(mx[i], s[124 + i]);
+        const float mxa = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
+        const float m_tile = mxa * sl2;
+        float alpha = 1.f;
+        const bool move = (j == 0) || (m_tile > m_used + 8.f);
+        if (move) {
+          const float m_new = fmaxf(m_used, m_tile);
+          alpha = ex2(m_used - m_new);  // 0 on the first tile (m_used = -inf)
+          m_used = m_new;
+        }
+        // O_g must be stable before it is rescaled, and P_g(j-1) read before
+        // P_g(j) is written.  Over S (not EARLY): S_g(j), whose completion
+        // was just observed, was issued after PV_g(j-1), and MMAs complete
+        // in issue order.  EARLY: wait for PV_g(j-1) itself.  (For j = 0,
+        // the previous item's epilogue waited for its last PV.)
+        if (C::EARLY && j > 0) {
+          wait_warp(w, bar(FB_ODONE + g), (tgj - 1) & 1, 9);
+          tc_fence_after();
+        }
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int acc = 0; acc < (C::SPLIT ? 2 : 1); ++acc) {
+            const uint32_t col = acc ? olcol : ocol;
+#pragma unroll
+            for (int cc = 0; cc < D / 16; ++cc) {
+              uint32_t r[16];
+              tmem_ld16(col + cc * 16, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+              tmem_st16(col + cc * 16, r);
+            }
+          }
+        }
+        const uint64_t sl2x2 = f2(sl2, sl2);
+        const uint64_t negm2 = f2(-m_used, -m_used);
+        uint64_t sum2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
+        if (j == ng - 1)
+          fwd_exp_row<false, PLO>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g));
+        else
+          fwd_exp_row<true, PLO>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g));
+        float sa, sb, sc2, sd;
+        f2_split(sum2[0], sa, sb);
+        f2_split(sum2[1], sc2, sd);
+        l = l * alpha + ((sa + sb) + (sc2 + sd));
       }
-      if (j == ng - 1) fwd_exp_row<false, PLO>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g));
-      else fwd_exp_row<true, PLO>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g));
-      if (kFwdTurns && has1) {
-        if (g == 0) named_bar_arrive(kBarTurn0, 256);
-        else if (j + 1 < n0) named_bar_arrive(kBarTurn1, 256);
-      }
-      float sa, sb, sc2, sd;
-      f2_split(sum2[0], sa, sb);
-      f2_split(sum2[1], sc2, sd);
-      l = l * alpha + ((sa + sb) + (sc2 + sd));
-    }
 
-    // ---------------------------------------------------------- epilogue
-    if (ng > 0) {
-      wait_warp(w, bar(FB_ODONE + g), (ng - 1) & 1, 10);
+      // -------------------------------------------------------- epilogue
+      wait_warp(w, bar(FB_ODONE + g), (tg + ng - 1) & 1, 10);
       tc_fence_after();
       const float inv_l = 1.f / l;
-      // staging: this group's Q tile (every MMA that read it has completed);
-      // O first, then O_lo through the same buffer
-      const uint32_t sQg = sbase + C::OFF_Q + g * C::TILE_BYTES;
-      const uint32_t nbar = 1 + g;
-      uint32_t lo_all[D / 2];
+      // O (and O') into registers; then TMEM is free for the next item
+      uint32_t o_all[D / 2], lo_all[D / 2];
 #pragma unroll
       for (int cc = 0; cc < D / 16; ++cc) {
         uint32_t r[16];
@@ -464,32 +527,17 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         } else {
           tmem_wait_ld();
         }
-        uint32_t pk[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e)
           split_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l,
-                       pk[e], lo_all[cc * 8 + e]);
-        const int d0 = cc * 16;
-        const int blk = d0 / C::CB;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int dd = (d0 % C::CB) + hh * 8;
-          st_shared_v4(sQg + blk * C::BLOCK_BYTES + swz<C::RB>(row * C::RB + dd * 2), pk[4 * hh],
-                       pk[4 * hh + 1], pk[4 * hh + 2], pk[4 * hh + 3]);
-        }
+                       o_all[cc * 8 + e], lo_all[cc * 8 + e]);
       }
       tc_fence_before();
-      fence_async_smem();
-      named_bar_sync(nbar, 128);
-      const bool leader = (threadIdx.x & 127) == 0;
-      if (leader && !*abort_flag) {
-        for (int b = 0; b < C::NCB; ++b)
-          tma_store_3d(&tmO, sQg + b * C::BLOCK_BYTES, b * C::CB, tile * C::BM, bh);
-        bulk_commit();
-      }
-      if (p.write_o_lo) {
-        if (leader) bulk_wait_read0();
-        named_bar_sync(nbar, 128);
+      mbar_arrive(bar(FB_OFREE + g));
+      // staging (the separate O tile, or this group's Q tile, which every
+      // MMA that read it has finished with): O, then O_lo through the same
+      // buffer
+      auto stage = [&](const uint32_t (&x)[D / 2]) {
 #pragma unroll
         for (int cc = 0; cc < D / 16; ++cc) {
           const int d0 = cc * 16;
@@ -497,24 +545,45 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             const int dd = (d0 % C::CB) + hh * 8;
-            st_shared_v4(sQg + blk * C::BLOCK_BYTES + swz<C::RB>(row * C::RB + dd * 2),
-                         lo_all[cc * 8 + 4 * hh], lo_all[cc * 8 + 4 * hh + 1],
-                         lo_all[cc * 8 + 4 * hh + 2], lo_all[cc * 8 + 4 * hh + 3]);
+            st_shared_v4(sOg + blk * C::BLOCK_BYTES + swz<C::RB>(row * C::RB + dd * 2),
+                         x[cc * 8 + 4 * hh], x[cc * 8 + 4 * hh + 1], x[cc * 8 + 4 * hh + 2],
+                         x[cc * 8 + 4 * hh + 3]);
           }
         }
+      };
+      const int tile = it.t0 + g;
+      stage(o_all);
+      fence_async_smem();
+      named_bar_sync(nbar, 128);
+      if (leader && !*abort_flag) {
+        for (int bb = 0; bb < C::NCB; ++bb)
+          tma_store_3d(&tmO, sOg + bb * C::BLOCK_BYTES, bb * C::CB, tile * C::BM, it.bh);
+        bulk_commit();
+      }
+      if (p.write_o_lo) {
+        if (leader) bulk_wait_read0();
+        named_bar_sync(nbar, 128);
+        stage(lo_all);
         fence_async_smem();
         named_bar_sync(nbar, 128);
         if (leader && !*abort_flag) {
-          for (int b = 0; b < C::NCB; ++b)
-            tma_store_3d(&tmOlo, sQg + b * C::BLOCK_BYTES, b * C::CB, tile * C::BM, bh);
+          for (int bb = 0; bb < C::NCB; ++bb)
+            tma_store_3d(&tmOlo, sOg + bb * C::BLOCK_BYTES, bb * C::CB, tile * C::BM, it.bh);
           bulk_commit();
         }
       }
-      if (leader) bulk_wait_read0();
+      // the staging tile is rewritten by the next item (separate O tile) or
+      // by the next Q load (the producer waits for this arrival)
+      if (leader) {
+        bulk_wait_read0();
+        if (!C::SEP_O) mbar_arrive(bar(FB_QFREE + g));
+      }
+      const int q_row = tile * C::BM + row;
       if (q_row < p.T) {
         // natural-log LSE: m_used is in log2 units of the scaled score
-        p.lse[static_cast<size_t>(bh) * p.T + q_row] = m_used * 0.69314718055994531f + logf(l);
+        p.lse[static_cast<size_t>(it.bh) * p.T + q_row] = m_used * 0.69314718055994531f + logf(l);
       }
+      tg += ng;
     }
   }
 
