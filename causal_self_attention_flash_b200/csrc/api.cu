@@ -306,15 +306,11 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   float* delta = reinterpret_cast<float*>(wb + L.delta_off);
   const size_t n_dq = static_cast<size_t>(BH) * T * D;
 
-  CUtensorMap mq, mk, mv, mdo, mdk, mdv, mdq;
+  CUtensorMap mq, mk, mv, mdo, mdq;
   if ((st = make_bf16_map(&mq, q, D, T, BH)) != CATTN_OK) return st;
   if ((st = make_bf16_map(&mk, k, D, T, BH)) != CATTN_OK) return st;
   if ((st = make_bf16_map(&mv, v, D, T, BH)) != CATTN_OK) return st;
   if ((st = make_bf16_map(&mdo, dout, D, T, BH)) != CATTN_OK) return st;
-  // with fp32 gradients the kernel stores dK, dV directly and never uses
-  // these two maps; they then describe q instead
-  if ((st = make_bf16_map(&mdk, grad_f32 ? q : dk, D, T, BH)) != CATTN_OK) return st;
-  if ((st = make_bf16_map(&mdv, grad_f32 ? q : dv, D, T, BH)) != CATTN_OK) return st;
   if ((st = make_tmap(&mdq, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, T, BH,
                       C::WARP_DQ ? D / 4 : C::CBQ, C::WARP_DQ ? 32 : 128)) !=
       CATTN_OK)
@@ -329,17 +325,22 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   p.delta = delta;
   p.dk_f32 = grad_f32 ? static_cast<float*>(dk) : nullptr;
   p.dv_f32 = grad_f32 ? static_cast<float*>(dv) : nullptr;
+  p.dk_bf16 = grad_f32 ? nullptr : static_cast<__nv_bfloat16*>(dk);
+  p.dv_bf16 = grad_f32 ? nullptr : static_cast<__nv_bfloat16*>(dv);
+  p.BH = BH;
   p.T = T;
   p.T_pad = L.T_pad;
   p.n_tiles = L.T_pad / 128;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_timeout_ns;
-  dim3 grid(BH, p.n_tiles);
+  // persistent: one CTA per SM, each looping over key tiles
+  const long long n_items = static_cast<long long>(BH) * p.n_tiles;
+  if (n_items > 0x7fffffffLL) return CATTN_ERR_INVALID_ARG;
+  dim3 grid(static_cast<unsigned>(n_items < g_sm_count[dev] ? n_items : g_sm_count[dev]));
   {
     LaunchTimer t(K_BWD_MAIN, s);
-    bwd_kernel<D, SLO><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mdo, mdk, mdv, mdq,
-                                                               p);
+    bwd_kernel<D, SLO><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mdo, mdq, p);
   }
   if ((st = launch_status()) != CATTN_OK) return st;
   {

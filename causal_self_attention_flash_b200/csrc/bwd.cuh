@@ -171,11 +171,14 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float4* __restric
 struct BwdParams {
   const float* lse2;   // (BH, T_pad) LSE * log2(e); +inf on padding rows
   const float* delta;  // (BH, T_pad); 0 on padding rows
-  float* dk_f32;       // fp32 gradient outputs (BH, T, D), or null for bf16
-  float* dv_f32;       //   through the tensor maps
+  float* dk_f32;       // fp32 gradient outputs (BH, T, D), or null
+  float* dv_f32;
+  __nv_bfloat16* dk_bf16;  // bf16 gradient outputs, used when dk_f32 is null
+  __nv_bfloat16* dv_bf16;
   int T;
   int T_pad;
   int n_tiles;
+  int BH;
   float scale;
   float scale_log2;
   uint64_t timeout_ns;
@@ -191,18 +194,10 @@ struct BwdCfg {
   static constexpr int QST = 2;                     // Q ring depth
   static constexpr int DOST = D <= 64 ? 2 : 1;      // dO ring depth
   static constexpr uint32_t SW = swizzle_code(RB);
-  // fp32 dQ staging (in the dS buffers): blocks of [128 rows][CBQ floats]
+  // fp32 dQ staging in the dS buffers (CTA-wide drain): blocks of
+  // [128 rows][CBQ floats]
   static constexpr int CBQ = D < 32 ? D : 32;
   static constexpr int RBQ = CBQ * 4;
-  // shared memory map
-  static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = OFF_K + TILE_BYTES;
-  static constexpr int OFF_Q = OFF_V + TILE_BYTES;
-  static constexpr int OFF_DO = OFF_Q + QST * TILE_BYTES;
-  static constexpr int OFF_DSH = OFF_DO + DOST * TILE_BYTES;  // [2][128 keys][64 q] bf16
-  static constexpr int OFF_DSL = OFF_DSH + 32768;
-  static constexpr int OFF_LSE = OFF_DSL + 32768;             // [QST][128] fp32
-  static constexpr int OFF_DELTA = OFF_LSE + QST * 512;       // [QST][128] fp32
   // WARP_DQ (D <= 64): every compute warp drains its own [32 rows][D/4]
   // slice of dQ through its own fp32 staging tile and TMA reduce, so no
   // CTA-wide barrier is needed; otherwise the CTA stages all of dQ in the dS
@@ -210,6 +205,23 @@ struct BwdCfg {
   static constexpr bool WARP_DQ = D <= 64;
   static constexpr int RBW = D;                                // (D/4) floats per row
   static constexpr int WARP_STAGE = (32 * RBW + 1023) / 1024 * 1024;
+  // dS lo buffer: with SLO, and as the second half of the CTA dQ staging
+  static constexpr int DSL_BYTES = (SLO || !WARP_DQ) ? 32768 : 0;
+  // shared memory map; KVB = 2 K/V buffers (the next work item's K, V load
+  // while the current one finishes) where they fit
+  static constexpr int layout_end(int kvb) {
+    return ((kvb * 2 * TILE_BYTES + (QST + DOST) * TILE_BYTES + 32768 + DSL_BYTES +
+             QST * 1024 + 1023) / 1024 * 1024) +
+           (WARP_DQ ? 16 * WARP_STAGE : 0) + 24 * 8 + 64;
+  }
+  static constexpr int KVB = layout_end(2) + 1024 <= kMaxDynSmem ? 2 : 1;
+  static constexpr int OFF_KV = 0;                             // [KVB][K, V]
+  static constexpr int OFF_Q = OFF_KV + KVB * 2 * TILE_BYTES;
+  static constexpr int OFF_DO = OFF_Q + QST * TILE_BYTES;
+  static constexpr int OFF_DSH = OFF_DO + DOST * TILE_BYTES;  // [2][128 keys][64 q] bf16
+  static constexpr int OFF_DSL = OFF_DSH + 32768;
+  static constexpr int OFF_LSE = OFF_DSL + DSL_BYTES;         // [QST][128] fp32
+  static constexpr int OFF_DELTA = OFF_LSE + QST * 512;       // [QST][128] fp32
   static constexpr int OFF_DQW = (OFF_DELTA + QST * 512 + 1023) / 1024 * 1024;
   static constexpr int OFF_BAR = WARP_DQ ? OFF_DQW + 16 * WARP_STAGE : OFF_DELTA + QST * 512;
   static constexpr int NUM_BARS = 24;
@@ -218,7 +230,7 @@ struct BwdCfg {
   static constexpr int SMEM_BYTES =
       SMEM_USED + 1024 <= kMaxDynSmem ? SMEM_USED + 1024 : SMEM_USED;
   static_assert(SMEM_USED <= kMaxDynSmem, "shared memory layout too large");
-  static_assert(128 * D * 4 <= 65536, "dQ staging must fit the dS buffers");
+  static_assert(WARP_DQ || 128 * D * 4 <= 32768 + DSL_BYTES, "dQ staging must fit the dS buffers");
   // TMEM columns.  MMAs that accumulate into one TMEM tile run back to back
   // at about half the rate of independent ones, so where columns allow, the
   // P_lo products of dV get their own accumulator dV' (summed at the end)
@@ -233,40 +245,55 @@ struct BwdCfg {
   static constexpr int NCOMP = 512;   // compute threads
 };
 
+// barrier indices (two of each K/V buffer barrier, QST of the Q ring's,
+// DOST (<= 2) of the dO ring's)
 enum : int {
-  BB_KV = 0, BB_QFULL = 1, BB_QEMPTY = 3, BB_DOFULL = 5, BB_DOEMPTY = 7, BB_SFULL = 9,
-  BB_DPFULL = 10, BB_PFULL = 11, BB_PTDONE = 12, BB_DSFULL = 13, BB_DSDONE = 14,
-  BB_DQFULL = 15, BB_DQEMPTY = 16, BB_DKDONE = 17, BB_DRAIN = 18
+  BB_KVFULL = 0, BB_KVFREE = 2, BB_QFULL = 4, BB_QEMPTY = 6, BB_DOFULL = 8, BB_DOEMPTY = 10,
+  BB_SFULL = 12, BB_DPFULL = 13, BB_PFULL = 14, BB_DSFULL = 15, BB_DQFULL = 16,
+  BB_DQEMPTY = 17, BB_ACCFREE = 18, BB_DRAIN = 19
 };
+
+// Work items: key tiles (kt, bh), numbered longest first (u = 0 ..
+// BH*n_tiles-1: kt = u / BH, bh = u % BH; key tile kt meets n_tiles - kt
+// query tiles).  The grid is persistent (at most one CTA per SM); CTA b
+// takes items in passes over the grid, alternating direction: pass k takes
+// item k*G + b (k even) or k*G + G-1-b (k odd).  Returns -1 past the end.
+__device__ __forceinline__ int bwd_item(int k, int b, int G, int n_items) {
+  const int u = k * G + ((k & 1) ? G - 1 - b : b);
+  return u < n_items ? u : -1;
+}
 
 template <int D, bool SLO>
 __global__ void __launch_bounds__(576, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-           const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
            const __grid_constant__ CUtensorMap tmDQacc, const BwdParams p) {
   using C = BwdCfg<D, SLO>;
+  static_assert(BB_DRAIN < C::NUM_BARS, "barrier count");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = aligned_smem(smem_raw, C::SMEM_USED);
   if (smem == nullptr) return;  // uniform over the CTA: nothing touched yet
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t sK = sbase + C::OFF_K, sV = sbase + C::OFF_V;
   const uint32_t sDSH = sbase + C::OFF_DSH, sDSL = sbase + C::OFF_DSL;
   auto bar = [&](int i) { return sbase + C::OFF_BAR + 8u * i; };
+  auto sK = [&](int kvb) { return sbase + C::OFF_KV + kvb * 2 * C::TILE_BYTES; };
+  auto sV = [&](int kvb) { return sbase + C::OFF_KV + kvb * 2 * C::TILE_BYTES + C::TILE_BYTES; };
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
-  const int kt = blockIdx.y;            // key tile; tile 0 has the most work
-  const int n_iter = p.n_tiles - kt;    // query tiles kt .. n_tiles-1
+  const int n_items = p.BH * p.n_tiles;
+  const int G = gridDim.x, b = blockIdx.x;
 
   WaitCtx w{p.timeout_ns, abort_flag, 2u};
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    mbar_init(bar(BB_KV), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(BB_KVFULL + s), 1);
+      mbar_init(bar(BB_KVFREE + s), 1);
+    }
     for (int s = 0; s < C::QST; ++s) {
       mbar_init(bar(BB_QFULL + s), 1);
       mbar_init(bar(BB_QEMPTY + s), 1);
@@ -278,12 +305,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     mbar_init(bar(BB_SFULL), 1);
     mbar_init(bar(BB_DPFULL), 1);
     mbar_init(bar(BB_PFULL), C::NCOMP);
-    mbar_init(bar(BB_PTDONE), 1);
     mbar_init(bar(BB_DSFULL), C::NCOMP);
-    mbar_init(bar(BB_DSDONE), 1);
     mbar_init(bar(BB_DQFULL), 1);
     mbar_init(bar(BB_DQEMPTY), C::NCOMP);
-    mbar_init(bar(BB_DKDONE), 1);
+    mbar_init(bar(BB_ACCFREE), C::NCOMP);
     mbar_init(bar(BB_DRAIN), 1);
     fence_mbar_init();
   }
@@ -296,6 +321,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   tc_fence_after();
   const uint32_t tbase = misc[0];
 
+  // Running counters across the CTA's items: t = query tiles processed so
+  // far (one per iteration: the phase of the per-iteration barriers and the
+  // position in the Q and dO rings), n = items so far (K/V buffer n % KVB).
   if (warp == 16) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -303,44 +331,66 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmDO);
-      mbar_arrive_expect_tx(bar(BB_KV), 2 * C::TILE_BYTES);
-      for (int b = 0; b < C::NCB; ++b) {
-        tma_load_3d(sK + b * C::BLOCK_BYTES, &tmK, bar(BB_KV), b * C::CB, kt * 128, bh);
-        tma_load_3d(sV + b * C::BLOCK_BYTES, &tmV, bar(BB_KV), b * C::CB, kt * 128, bh);
-      }
-      int nq = 0, ndo = 0;  // loads issued
-      for (int i = 0; i < n_iter; ++i) {
-        const int qi = kt + i;
+      int tq = 0, tdo = 0, n = 0;  // loads issued
+      auto load_q = [&](int qi, int bh) {
+        const int qs = tq % C::QST;
+        if (tq >= C::QST) wait1(w, bar(BB_QEMPTY + qs), ((tq / C::QST) - 1) & 1, 1);
+        if (*abort_flag) return;
         const size_t vec = static_cast<size_t>(bh) * p.T_pad + static_cast<size_t>(qi) * 128;
-        const int qs = i % C::QST;
-        if (i >= C::QST) wait1(w, bar(BB_QEMPTY + qs), ((i / C::QST) - 1) & 1, 1);
-        if (*abort_flag) break;
         const uint32_t sQ = sbase + C::OFF_Q + qs * C::TILE_BYTES;
         mbar_arrive_expect_tx(bar(BB_QFULL + qs), C::TILE_BYTES + 1024);
-        for (int b = 0; b < C::NCB; ++b)
-          tma_load_3d(sQ + b * C::BLOCK_BYTES, &tmQ, bar(BB_QFULL + qs), b * C::CB, qi * 128, bh);
+        for (int bb = 0; bb < C::NCB; ++bb)
+          tma_load_3d(sQ + bb * C::BLOCK_BYTES, &tmQ, bar(BB_QFULL + qs), bb * C::CB, qi * 128, bh);
         bulk_load(sbase + C::OFF_LSE + qs * 512, p.lse2 + vec, 512, bar(BB_QFULL + qs));
         bulk_load(sbase + C::OFF_DELTA + qs * 512, p.delta + vec, 512, bar(BB_QFULL + qs));
-        nq = i + 1;
-        const int ds = i % C::DOST;
-        if (i >= C::DOST) wait1(w, bar(BB_DOEMPTY + ds), ((i / C::DOST) - 1) & 1, 2);
-        if (*abort_flag) break;
+        ++tq;
+      };
+      auto load_do = [&](int qi, int bh) {
+        const int ds = tdo % C::DOST;
+        if (tdo >= C::DOST) wait1(w, bar(BB_DOEMPTY + ds), ((tdo / C::DOST) - 1) & 1, 2);
+        if (*abort_flag) return;
         const uint32_t sDO = sbase + C::OFF_DO + ds * C::TILE_BYTES;
         mbar_arrive_expect_tx(bar(BB_DOFULL + ds), C::TILE_BYTES);
-        for (int b = 0; b < C::NCB; ++b)
-          tma_load_3d(sDO + b * C::BLOCK_BYTES, &tmDO, bar(BB_DOFULL + ds), b * C::CB, qi * 128,
+        for (int bb = 0; bb < C::NCB; ++bb)
+          tma_load_3d(sDO + bb * C::BLOCK_BYTES, &tmDO, bar(BB_DOFULL + ds), bb * C::CB, qi * 128,
                       bh);
-        ndo = i + 1;
+        ++tdo;
+      };
+      for (int k = 0;; ++k) {
+        const int u = bwd_item(k, b, G, n_items);
+        if (u < 0 || *abort_flag) break;
+        const int kt = u / p.BH, bh = u % p.BH;
+        const int n_iter = p.n_tiles - kt;
+        // in the order the MMAs consume them: Q_0 (S), K and V, dO_0 (dP)
+        load_q(kt, bh);
+        const int kvb = n % C::KVB;
+        if (n >= C::KVB) wait1(w, bar(BB_KVFREE + kvb), ((n / C::KVB) - 1) & 1, 3);
+        if (*abort_flag) break;
+        mbar_arrive_expect_tx(bar(BB_KVFULL + kvb), 2 * C::TILE_BYTES);
+        for (int bb = 0; bb < C::NCB; ++bb) {
+          tma_load_3d(sK(kvb) + bb * C::BLOCK_BYTES, &tmK, bar(BB_KVFULL + kvb), bb * C::CB,
+                      kt * 128, bh);
+          tma_load_3d(sV(kvb) + bb * C::BLOCK_BYTES, &tmV, bar(BB_KVFULL + kvb), bb * C::CB,
+                      kt * 128, bh);
+        }
+        ++n;
+        load_do(kt, bh);
+        for (int i = 1; i < n_iter && !*abort_flag; ++i) {
+          load_q(kt + i, bh);
+          load_do(kt + i, bh);
+        }
       }
       if (*abort_flag) {
-        // wait (bounded, ignoring the abort flag) for loads nobody consumed
+        // wait (bounded, ignoring the abort flag) for the last loads issued,
+        // which nobody may consume, before the CTA exits
         int zero = 0;
         WaitCtx wd{p.timeout_ns, &zero, 2u};
-        wait1(wd, bar(BB_KV), 0, 20);
-        for (int i = (nq > C::QST ? nq - C::QST : 0); i < nq; ++i)
-          wait1(wd, bar(BB_QFULL + i % C::QST), (i / C::QST) & 1, 21);
-        for (int i = (ndo > C::DOST ? ndo - C::DOST : 0); i < ndo; ++i)
-          wait1(wd, bar(BB_DOFULL + i % C::DOST), (i / C::DOST) & 1, 22);
+        for (int j = (n > C::KVB ? n - C::KVB : 0); j < n; ++j)
+          wait1(wd, bar(BB_KVFULL + j % C::KVB), (j / C::KVB) & 1, 20);
+        for (int j = (tq > C::QST ? tq - C::QST : 0); j < tq; ++j)
+          wait1(wd, bar(BB_QFULL + j % C::QST), (j / C::QST) & 1, 21);
+        for (int j = (tdo > C::DOST ? tdo - C::DOST : 0); j < tdo; ++j)
+          wait1(wd, bar(BB_DOFULL + j % C::DOST), (j / C::DOST) & 1, 22);
       }
     }
   } else if (warp == 17) {
@@ -349,9 +399,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       constexpr uint32_t idSS = idesc_bf16(128, 128, 0, 0);  // S^T, dP^T
       constexpr uint32_t idKD = idesc_bf16(128, D, 0, 1);    // dV, dK: B MN-major
       constexpr uint32_t idQ = idesc_bf16(128, D, 1, 1);     // dQ: A (dS) MN-major
-      auto issue_s = [&](int i) {  // S^T = K Q_i^T
-        const int qs = i % C::QST;
-        wait1(w, bar(BB_QFULL + qs), (i / C::QST) & 1, 3);
+      auto issue_s = [&](int t, uint32_t k_s) {  // S^T = K Q_t^T
+        const int qs = t % C::QST;
+        wait1(w, bar(BB_QFULL + qs), (t / C::QST) & 1, 4);
         tc_fence_after();
         const uint32_t sQ = sbase + C::OFF_Q + qs * C::TILE_BYTES;
 #pragma unroll
@@ -359,15 +409,18 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           const int blk = (kk * 16) / C::CB;
           const int off = ((kk * 16) % C::CB) * 2;
           mma_ss(tbase + C::COL_S,
-                 smem_desc(sK + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW),
+                 smem_desc(k_s + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW),
                  smem_desc(sQ + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW), idSS,
                  kk > 0 ? 1u : 0u);
         }
         mma_commit(bar(BB_SFULL));
       };
-      auto issue_dp = [&](int i) {  // dP^T = V dO_i^T
-        const int ds = i % C::DOST;
-        wait1(w, bar(BB_DOFULL + ds), (i / C::DOST) & 1, 4);
+      auto issue_dp = [&](int t, uint32_t v_s) {  // dP^T = V dO_t^T
+        const int ds = t % C::DOST;
+        wait1(w, bar(BB_DOFULL + ds), (t / C::DOST) & 1, 5);
+        // dP overwrites dS^T(t-1), which dK(t-1) read in order before it,
+        // and, aliased, dQ(t-1), which the compute warps must have drained
+        if (C::ALIAS_DQ && t >= 1) wait1(w, bar(BB_DQEMPTY), (t - 1) & 1, 12);
         tc_fence_after();
         const uint32_t sDO = sbase + C::OFF_DO + ds * C::TILE_BYTES;
 #pragma unroll
@@ -375,89 +428,97 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           const int blk = (kk * 16) / C::CB;
           const int off = ((kk * 16) % C::CB) * 2;
           mma_ss(tbase + C::COL_DP,
-                 smem_desc(sV + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW),
+                 smem_desc(v_s + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW),
                  smem_desc(sDO + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW), idSS,
                  kk > 0 ? 1u : 0u);
         }
         mma_commit(bar(BB_DPFULL));
       };
-      wait1(w, bar(BB_KV), 0, 5);
-      issue_s(0);
-      issue_dp(0);
-      for (int i = 0; i < n_iter; ++i) {
-        const int qs = i % C::QST;
-        const int ds = i % C::DOST;
-        const uint32_t sQ = sbase + C::OFF_Q + qs * C::TILE_BYTES;
-        const uint32_t sDO = sbase + C::OFF_DO + ds * C::TILE_BYTES;
-        // dV += P^T dO_i  (A = P^T hi/lo in TMEM over S^T; K = 128 queries)
-        wait1(w, bar(BB_PFULL), i & 1, 6);
-        tc_fence_after();
-        const uint64_t ddo = smem_desc(sDO, C::BLOCK_BYTES, 8 * C::RB, C::SW);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t acol = C::COL_S + (kk >> 1) * 32 + (kk & 1) * 8;
-          const uint64_t b = ddo + ((kk * 16 * C::RB) >> 4);
-          const uint32_t first = (i > 0 || kk > 0) ? 1u : 0u;
-          mma_ts(tbase + C::COL_DV, tbase + acol, b, idKD, first);
-          mma_ts(tbase + C::COL_DVL, tbase + acol + 16, b, idKD, C::SPLIT_DV ? first : 1u);
-        }
-        mma_commit(bar(BB_PTDONE));
-        mma_commit(bar(BB_DOEMPTY + ds));
-        // S(i+1) overwrites P^T(i); the MMAs execute in issue order, so it
-        // cannot before dV(i) has read it
-        if (i + 1 < n_iter) issue_s(i + 1);
-        // dK += dS^T Q_i (A = dS^T hi/lo in TMEM over dP^T)
-        wait1(w, bar(BB_DSFULL), i & 1, 8);
-        if (!C::ALIAS_DQ && i >= 1) wait1(w, bar(BB_DQEMPTY), (i - 1) & 1, 9);
-        tc_fence_after();
-        const uint64_t dqq = smem_desc(sQ, C::BLOCK_BYTES, 8 * C::RB, C::SW);
-        const uint64_t dkk = smem_desc(sK, C::BLOCK_BYTES, 8 * C::RB, C::SW);
-        const uint64_t dsh = smem_desc(sDSH, 16384, 1024, 2);
-        const uint64_t dsl = smem_desc(sDSL, 16384, 1024, 2);
-        // dK += dS^T Q_i (A = dS^T hi/lo in TMEM over dP^T) and
-        // dQ_i = dS K (A = dS hi/lo in shared, MN-major; K = 128 keys)
-        auto dk_step = [&](int kk, int lo) {
-          if (!SLO && lo) return;
-          const uint32_t acol = C::COL_DP + (kk >> 1) * 32 + (kk & 1) * 8 + (lo ? 16 : 0);
-          mma_ts(tbase + C::COL_DK, tbase + acol, dqq + ((kk * 16 * C::RB) >> 4), idKD,
-                 (i > 0 || kk > 0 || lo) ? 1u : 0u);
-        };
-        auto dq_step = [&](int kk, int lo) {
-          if (!SLO && lo) return;
-          mma_ss(tbase + C::COL_DQ, (lo ? dsl : dsh) + ((kk * 2048) >> 4),
-                 dkk + ((kk * 16 * C::RB) >> 4), idQ, (kk > 0 || lo) ? 1u : 0u);
-        };
-        if constexpr (C::ALIAS_DQ) {
-          // dQ overwrites the dS^T that dK reads: all of dK first (in order)
+      int t = 0, n = 0;
+      for (int k = 0;; ++k) {
+        const int u = bwd_item(k, b, G, n_items);
+        if (u < 0) break;
+        const int kt = u / p.BH;
+        const int n_iter = p.n_tiles - kt;
+        const int kvb = n % C::KVB;
+        const uint32_t k_s = sK(kvb), v_s = sV(kvb);
+        wait1(w, bar(BB_KVFULL + kvb), (n / C::KVB) & 1, 6);
+        // S(t) overwrites P^T(t-1), read by dV(t-1) before it in order
+        issue_s(t, k_s);
+        issue_dp(t, v_s);
+        for (int i = 0; i < n_iter; ++i, ++t) {
+          const int qs = t % C::QST;
+          const int ds = t % C::DOST;
+          const uint32_t sQ = sbase + C::OFF_Q + qs * C::TILE_BYTES;
+          const uint32_t sDO = sbase + C::OFF_DO + ds * C::TILE_BYTES;
+          // dV += P^T dO_t  (A = P^T hi/lo in TMEM over S^T; K = 128 queries)
+          wait1(w, bar(BB_PFULL), t & 1, 7);
+          // the first dV, dK of an item overwrite the accumulators: the
+          // previous item's epilogue must have read them
+          if (i == 0 && n > 0) wait1(w, bar(BB_ACCFREE), (n - 1) & 1, 8);
+          tc_fence_after();
+          const uint64_t ddo = smem_desc(sDO, C::BLOCK_BYTES, 8 * C::RB, C::SW);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            dk_step(kk, 0);
-            dk_step(kk, 1);
+            const uint32_t acol = C::COL_S + (kk >> 1) * 32 + (kk & 1) * 8;
+            const uint64_t bd = ddo + ((kk * 16 * C::RB) >> 4);
+            const uint32_t first = (i > 0 || kk > 0) ? 1u : 0u;
+            mma_ts(tbase + C::COL_DV, tbase + acol, bd, idKD, first);
+            mma_ts(tbase + C::COL_DVL, tbase + acol + 16, bd, idKD, C::SPLIT_DV ? first : 1u);
           }
-          mma_commit(bar(BB_QEMPTY + qs));
+          mma_commit(bar(BB_DOEMPTY + ds));
+          // S(t+1) overwrites P^T(t); the MMAs execute in issue order, so it
+          // cannot before dV(t) has read it
+          if (i + 1 < n_iter) issue_s(t + 1, k_s);
+          // dK += dS^T Q_t (A = dS^T hi/lo in TMEM over dP^T) and
+          // dQ_t = dS K (A = dS hi/lo in shared, MN-major; K = 128 keys)
+          wait1(w, bar(BB_DSFULL), t & 1, 9);
+          if (!C::ALIAS_DQ && t >= 1) wait1(w, bar(BB_DQEMPTY), (t - 1) & 1, 10);
+          tc_fence_after();
+          const uint64_t dqq = smem_desc(sQ, C::BLOCK_BYTES, 8 * C::RB, C::SW);
+          const uint64_t dkk = smem_desc(k_s, C::BLOCK_BYTES, 8 * C::RB, C::SW);
+          const uint64_t dsh = smem_desc(sDSH, 16384, 1024, 2);
+          const uint64_t dsl = smem_desc(sDSL, 16384, 1024, 2);
+          auto dk_step = [&](int kk, int lo) {
+            if (!SLO && lo) return;
+            const uint32_t acol = C::COL_DP + (kk >> 1) * 32 + (kk & 1) * 8 + (lo ? 16 : 0);
+            mma_ts(tbase + C::COL_DK, tbase + acol, dqq + ((kk * 16 * C::RB) >> 4), idKD,
+                   (i > 0 || kk > 0 || lo) ? 1u : 0u);
+          };
+          auto dq_step = [&](int kk, int lo) {
+            if (!SLO && lo) return;
+            mma_ss(tbase + C::COL_DQ, (lo ? dsl : dsh) + ((kk * 2048) >> 4),
+                   dkk + ((kk * 16 * C::RB) >> 4), idQ, (kk > 0 || lo) ? 1u : 0u);
+          };
+          if constexpr (C::ALIAS_DQ) {
+            // dQ overwrites the dS^T that dK reads: all of dK first (in order)
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            dq_step(kk, 0);
-            dq_step(kk, 1);
-          }
-        } else {
+            for (int kk = 0; kk < 8; ++kk) {
+              dk_step(kk, 0);
+              dk_step(kk, 1);
+            }
+            mma_commit(bar(BB_QEMPTY + qs));
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            dk_step(kk, 0);
-            dq_step(kk, 0);
-            dk_step(kk, 1);
-            dq_step(kk, 1);
+            for (int kk = 0; kk < 8; ++kk) {
+              dq_step(kk, 0);
+              dq_step(kk, 1);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              dk_step(kk, 0);
+              dq_step(kk, 0);
+              dk_step(kk, 1);
+              dq_step(kk, 1);
+            }
+            mma_commit(bar(BB_QEMPTY + qs));
           }
-          mma_commit(bar(BB_QEMPTY + qs));
+          mma_commit(bar(BB_DQFULL));
+          if (i + 1 < n_iter) issue_dp(t + 1, v_s);
         }
-        mma_commit(bar(BB_DSDONE));
-        mma_commit(bar(BB_DQFULL));
-        // dP(i+1) overwrites dS^T(i) (in order behind dK(i)) and, aliased,
-        // dQ(i), which the compute warps must have drained first
-        if (i + 1 < n_iter) {
-          if (C::ALIAS_DQ) wait1(w, bar(BB_DQEMPTY), i & 1, 12);
-          issue_dp(i + 1);
-        }
+        // every MMA that reads this item's K, V has been issued
+        mma_commit(bar(BB_KVFREE + kvb));
+        ++n;
       }
       mma_commit(bar(BB_DRAIN));
       int zero = 0;
@@ -478,180 +539,6 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const bool leader = threadIdx.x == 0;
     constexpr int NQ = D / 4;                    // dQ / dK / dV columns per thread
 
-    // dQ(t) drain: TMEM (lane = query row) -> fp32 staging in the dS
-    // buffers -> TMA reduce-add into the accumulator.
-    auto drain_dq = [&](int t) {
-      wait_warp(w, bar(BB_DQFULL), t & 1, 14);
-      tc_fence_after();
-      float acc[NQ];
-      const uint32_t src = tbase + lane_base + C::COL_DQ + grp * NQ;
-      if constexpr (NQ == 32) {
-        uint32_t v[32];
-        tmem_ld32(src, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) acc[e] = __uint_as_float(v[e]);
-      } else if constexpr (NQ == 16) {
-        uint32_t v[16];
-        tmem_ld16(src, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(v[e]);
-      } else if constexpr (NQ == 8) {
-        uint32_t v[8];
-        tmem_ld8(src, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = __uint_as_float(v[e]);
-      } else {
-        uint32_t v[4];
-        tmem_ld4(src, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[e] = __uint_as_float(v[e]);
-      }
-      tc_fence_before();
-      mbar_arrive(bar(BB_DQEMPTY));
-      if constexpr (C::WARP_DQ) {
-        // this warp's tile [32 rows][NQ floats]; its previous reduce must
-        // have finished reading it
-        const uint32_t sW = sbase + C::OFF_DQW + warp * C::WARP_STAGE;
-        if (lane == 0) bulk_wait_read0();
-        __syncwarp();
-#pragma unroll
-        for (int e = 0; e < NQ; e += 4)
-          st_shared_v4(sW + swz<C::RBW>(lane * C::RBW + e * 4), __float_as_uint(acc[e]),
-                       __float_as_uint(acc[e + 1]), __float_as_uint(acc[e + 2]),
-                       __float_as_uint(acc[e + 3]));
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0 && !*abort_flag) {
-          tma_reduce_add_3d(&tmDQacc, sW, grp * NQ, (kt + t) * 128 + quarter * 32, bh);
-          bulk_commit();
-        }
-      } else {
-        // staging: blocks of [128 rows][CBQ floats], swizzled
-#pragma unroll
-        for (int e = 0; e < NQ; e += 4) {
-          const int f = grp * NQ + e;
-          const int blk = f / C::CBQ;
-          const int within = (f % C::CBQ) * 4;
-          st_shared_v4(sDSH + blk * 128 * C::RBQ + swz<C::RBQ>(r * C::RBQ + within),
-                       __float_as_uint(acc[e]), __float_as_uint(acc[e + 1]),
-                       __float_as_uint(acc[e + 2]), __float_as_uint(acc[e + 3]));
-        }
-        fence_async_smem();
-        named_bar_sync(1, C::NCOMP);
-        if (leader && !*abort_flag) {
-#pragma unroll
-          for (int blk = 0; blk < D / C::CBQ; ++blk)
-            tma_reduce_add_3d(&tmDQacc, sDSH + blk * 128 * C::RBQ, blk * C::CBQ,
-                              (kt + t) * 128, bh);
-          bulk_commit();
-        }
-      }
-    };
-    // the dS buffers may be rewritten once the reduce has read them (CTA
-    // staging only)
-    auto staging_free = [&]() {
-      if constexpr (!C::WARP_DQ) {
-        if (leader) bulk_wait_read0();
-        named_bar_sync(1, C::NCOMP);
-      }
-    };
-
-    float pv[32];
-    for (int i = 0; i < n_iter; ++i) {
-      const int qs = i % C::QST;
-      // ---- P phase
-      wait_warp(w, bar(BB_SFULL), i & 1, 15);
-      tc_fence_after();
-      {
-        uint32_t v[32];
-        tmem_ld32(tbase + lane_base + C::COL_S + grp * 32, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) pv[e] = __uint_as_float(v[e]);
-      }
-      wait_warp(w, bar(BB_QFULL + qs), (i / C::QST) & 1, 16);  // LSE2 visibility
-      const uint32_t sL = sbase + C::OFF_LSE + qs * 512 + grp * 128;
-#pragma unroll
-      for (int c = 0; c < 32; c += 4) {
-        float l0, l1, l2, l3;
-        ld_shared_v4f(sL + c * 4, l0, l1, l2, l3);
-        pv[c] = ex2(fmaf(pv[c], sl2, -l0));
-        pv[c + 1] = ex2(fmaf(pv[c + 1], sl2, -l1));
-        pv[c + 2] = ex2(fmaf(pv[c + 2], sl2, -l2));
-        pv[c + 3] = ex2(fmaf(pv[c + 3], sl2, -l3));
-      }
-      if (i == 0) {  // diagonal tile: query (32g + c) sees key r only if r <= query
-        const int lim = r - grp * 32;
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (c < lim) pv[c] = 0.f;
-      }
-      {
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) split_bf16x2_p(f2(pv[2 * e], pv[2 * e + 1]), hi[e], lo[e]);
-        tmem_st16(tbase + lane_base + C::COL_S + grp * 32, hi);
-        tmem_st16(tbase + lane_base + C::COL_S + grp * 32 + 16, lo);
-        tmem_wait_st();
-      }
-      tc_fence_before();
-      mbar_arrive(bar(BB_PFULL));
-
-      // ---- dQ of the previous query tile (its MMA ran during this P phase)
-      if (i >= 1) drain_dq(i - 1);
-
-      // ---- dS phase
-      wait_warp(w, bar(BB_DPFULL), i & 1, 17);
-      tc_fence_after();
-      // (the Delta vector arrived with Q_i, whose barrier was waited above)
-      const uint32_t sD = sbase + C::OFF_DELTA + qs * 512 + grp * 128;
-      uint32_t hi[16], lo[16];
-      {
-        uint32_t v[32];
-        tmem_ld32(tbase + lane_base + C::COL_DP + grp * 32, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          float d0, d1, d2, d3;
-          ld_shared_v4f(sD + e * 4, d0, d1, d2, d3);
-          const float s0 = pv[e] * (__uint_as_float(v[e]) - d0);
-          const float s1 = pv[e + 1] * (__uint_as_float(v[e + 1]) - d1);
-          const float s2 = pv[e + 2] * (__uint_as_float(v[e + 2]) - d2);
-          const float s3 = pv[e + 3] * (__uint_as_float(v[e + 3]) - d3);
-          if (SLO) {
-            split_bf16x2_p(f2(s0, s1), hi[e / 2], lo[e / 2]);
-            split_bf16x2_p(f2(s2, s3), hi[e / 2 + 1], lo[e / 2 + 1]);
-          } else {
-            hi[e / 2] = pack_bf16(s0, s1);
-            hi[e / 2 + 1] = pack_bf16(s2, s3);
-          }
-        }
-      }
-      tmem_st16(tbase + lane_base + C::COL_DP + grp * 32, hi);
-      if (SLO) tmem_st16(tbase + lane_base + C::COL_DP + grp * 32 + 16, lo);
-      // dS (hi, lo) -> shared for the dQ MMA: [2][128 keys][64 queries];
-      // query block g is half g/2, chunks 4*(g%2) .. +3 of the row
-      if (i >= 1) staging_free();
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        const uint32_t off = (grp >> 1) * 16384 + swz<128>(r * 128 + ((grp & 1) * 4 + ch) * 16);
-        st_shared_v4(sDSH + off, hi[4 * ch], hi[4 * ch + 1], hi[4 * ch + 2], hi[4 * ch + 3]);
-        if (SLO)
-          st_shared_v4(sDSL + off, lo[4 * ch], lo[4 * ch + 1], lo[4 * ch + 2], lo[4 * ch + 3]);
-      }
-      fence_async_smem();
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(BB_DSFULL));
-    }
-    drain_dq(n_iter - 1);  // waits for the last MMAs: everything is complete
-    staging_free();
-
-    // ---- dK, dV epilogue: this thread's NQ columns of its key row
     auto load_cols = [&](uint32_t col, float (&x)[NQ]) {
       if constexpr (NQ == 32) {
         uint32_t v[32];
@@ -679,69 +566,225 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         for (int e = 0; e < 4; ++e) x[e] = __uint_as_float(v[e]);
       }
     };
-    const bool f32out = p.dk_f32 != nullptr;
+
+    // dQ(t) drain: TMEM (lane = query row) -> fp32 staging -> TMA
+    // reduce-add into the accumulator, rows q0 .. q0+127 of head bh
+    auto drain_dq = [&](int t, int q0, int bh) {
+      wait_warp(w, bar(BB_DQFULL), t & 1, 14);
+      tc_fence_after();
+      float acc[NQ];
+      load_cols(tbase + lane_base + C::COL_DQ + grp * NQ, acc);
+      tc_fence_before();
+      mbar_arrive(bar(BB_DQEMPTY));
+      if constexpr (C::WARP_DQ) {
+        // this warp's tile [32 rows][NQ floats]; its previous reduce must
+        // have finished reading it
+        const uint32_t sW = sbase + C::OFF_DQW + warp * C::WARP_STAGE;
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
 #pragma unroll
-    for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
-      float x[NQ];
-      load_cols(tbase + lane_base + (which ? C::COL_DK : C::COL_DV) + grp * NQ, x);
-      if (C::SPLIT_DV && which == 0) {  // dV = dV + dV'
-        float x2[NQ];
-        load_cols(tbase + lane_base + C::COL_DVL + grp * NQ, x2);
+        for (int e = 0; e < NQ; e += 4)
+          st_shared_v4(sW + swz<C::RBW>(lane * C::RBW + e * 4), __float_as_uint(acc[e]),
+                       __float_as_uint(acc[e + 1]), __float_as_uint(acc[e + 2]),
+                       __float_as_uint(acc[e + 3]));
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0 && !*abort_flag) {
+          tma_reduce_add_3d(&tmDQacc, sW, grp * NQ, q0 + quarter * 32, bh);
+          bulk_commit();
+        }
+      } else {
+        // staging: blocks of [128 rows][CBQ floats], swizzled
 #pragma unroll
-        for (int e = 0; e < NQ; ++e) x[e] += x2[e];
+        for (int e = 0; e < NQ; e += 4) {
+          const int f = grp * NQ + e;
+          const int blk = f / C::CBQ;
+          const int within = (f % C::CBQ) * 4;
+          st_shared_v4(sDSH + blk * 128 * C::RBQ + swz<C::RBQ>(r * C::RBQ + within),
+                       __float_as_uint(acc[e]), __float_as_uint(acc[e + 1]),
+                       __float_as_uint(acc[e + 2]), __float_as_uint(acc[e + 3]));
+        }
+        fence_async_smem();
+        named_bar_sync(1, C::NCOMP);
+        if (leader && !*abort_flag) {
+#pragma unroll
+          for (int blk = 0; blk < D / C::CBQ; ++blk)
+            tma_reduce_add_3d(&tmDQacc, sDSH + blk * 128 * C::RBQ, blk * C::CBQ, q0, bh);
+          bulk_commit();
+        }
       }
-      const float mul = which ? p.scale : 1.f;
+    };
+    // the dS buffers may be rewritten once the reduce has read them (CTA
+    // staging only)
+    auto staging_free = [&]() {
+      if constexpr (!C::WARP_DQ) {
+        if (leader) bulk_wait_read0();
+        named_bar_sync(1, C::NCOMP);
+      }
+    };
+
+    // dK, dV epilogue of key tile kt of head bh: this thread's NQ columns of
+    // its key row, straight from TMEM to global memory.  (The accumulators
+    // are complete: the dQ drain of the item's last iteration waited for
+    // the MMAs that finished them.)
+    auto epilogue = [&](int kt, int bh) {
+      const int key = kt * 128 + r;
+      const size_t off = (static_cast<size_t>(bh) * p.T + (key < p.T ? key : 0)) * D + grp * NQ;
+      // which = 0: dV (+ dV'), 1: dK * scale; the accumulators are released
+      // after the last TMEM load
 #pragma unroll
-      for (int e = 0; e < NQ; ++e) x[e] *= mul;
-      if (f32out) {
-        // fp32 outputs: straight to global
-        const int key = kt * 128 + r;
-        if (key < p.T) {
-          float* out = (which ? p.dk_f32 : p.dv_f32) +
-                       (static_cast<size_t>(bh) * p.T + key) * D + grp * NQ;
+      for (int which = 0; which < 2; ++which) {
+        float x[NQ];
+        load_cols(tbase + lane_base + (which ? C::COL_DK : C::COL_DV) + grp * NQ, x);
+        if (C::SPLIT_DV && which == 0) {
+          float x2[NQ];
+          load_cols(tbase + lane_base + C::COL_DVL + grp * NQ, x2);
+#pragma unroll
+          for (int e = 0; e < NQ; ++e) x[e] += x2[e];
+        }
+        if (which == 1) {
+          tc_fence_before();
+          mbar_arrive(bar(BB_ACCFREE));
+        }
+        const float mul = which ? p.scale : 1.f;
+#pragma unroll
+        for (int e = 0; e < NQ; ++e) x[e] *= mul;
+        if (key >= p.T) continue;
+        if (p.dk_f32 != nullptr) {
+          float* out = (which ? p.dk_f32 : p.dv_f32) + off;
 #pragma unroll
           for (int e = 0; e < NQ; e += 4)
             reinterpret_cast<float4*>(out + e)[0] = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
-        }
-      } else {
-        // bf16 outputs: staged in the dS buffers (dV in sDSH, dK in sDSL)
-        // as the TMA store layout [NCB][128][CB], then stored by TMA
-        const uint32_t dst = which ? sDSL : sDSH;
-        if constexpr (NQ >= 8) {
+        } else if constexpr (NQ >= 8) {
+          __nv_bfloat16* out = (which ? p.dk_bf16 : p.dv_bf16) + off;
 #pragma unroll
-          for (int e = 0; e < NQ; e += 8) {
-            const int d0 = grp * NQ + e;  // a multiple of 8: one 16-byte chunk
-            st_shared_v4(dst + (d0 / C::CB) * C::BLOCK_BYTES +
-                             swz<C::RB>(r * C::RB + (d0 % C::CB) * 2),
-                         pack_bf16(x[e], x[e + 1]), pack_bf16(x[e + 2], x[e + 3]),
-                         pack_bf16(x[e + 4], x[e + 5]), pack_bf16(x[e + 6], x[e + 7]));
-          }
+          for (int e = 0; e < NQ; e += 8)
+            reinterpret_cast<uint4*>(out + e)[0] =
+                make_uint4(pack_bf16(x[e], x[e + 1]), pack_bf16(x[e + 2], x[e + 3]),
+                           pack_bf16(x[e + 4], x[e + 5]), pack_bf16(x[e + 6], x[e + 7]));
         } else {
-          const int d0 = grp * NQ;      // 4 columns: half of a 16-byte chunk
-          st_shared_v2(dst + (d0 / C::CB) * C::BLOCK_BYTES +
-                           swz<C::RB>(r * C::RB + ((d0 % C::CB) & ~7) * 2) + (d0 & 7) * 2,
-                       pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]));
+          __nv_bfloat16* out = (which ? p.dk_bf16 : p.dv_bf16) + off;
+          reinterpret_cast<uint2*>(out)[0] =
+              make_uint2(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]));
         }
       }
+    };
+
+    float pv[32];
+    int t = 0;
+    // the previous query tile (its dQ is drained in the next iteration) and
+    // the previous item (its epilogue follows the first P phase of the next)
+    int prev_q0 = 0, prev_bh = 0, prev_kt = -1;
+    for (int k = 0;; ++k) {
+      const int u = bwd_item(k, b, G, n_items);
+      if (u < 0) break;
+      const int kt = u / p.BH, bh = u % p.BH;
+      const int n_iter = p.n_tiles - kt;
+      for (int i = 0; i < n_iter; ++i, ++t) {
+        const int qs = t % C::QST;
+        // ---- P phase
+        wait_warp(w, bar(BB_SFULL), t & 1, 15);
+        tc_fence_after();
+        {
+          uint32_t v[32];
+          tmem_ld32(tbase + lane_base + C::COL_S + grp * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) pv[e] = __uint_as_float(v[e]);
+        }
+        wait_warp(w, bar(BB_QFULL + qs), (t / C::QST) & 1, 16);  // LSE2 visibility
+        const uint32_t sL = sbase + C::OFF_LSE + qs * 512 + grp * 128;
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          float l0, l1, l2, l3;
+          ld_shared_v4f(sL + c * 4, l0, l1, l2, l3);
+          pv[c] = ex2(fmaf(pv[c], sl2, -l0));
+          pv[c + 1] = ex2(fmaf(pv[c + 1], sl2, -l1));
+          pv[c + 2] = ex2(fmaf(pv[c + 2], sl2, -l2));
+          pv[c + 3] = ex2(fmaf(pv[c + 3], sl2, -l3));
+        }
+        if (i == 0) {  // diagonal tile: query (32g + c) sees key r only if r <= query
+          const int lim = r - grp * 32;
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (c < lim) pv[c] = 0.f;
+        }
+        {
+          uint32_t hi[16], lo[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) split_bf16x2_p(f2(pv[2 * e], pv[2 * e + 1]), hi[e], lo[e]);
+          tmem_st16(tbase + lane_base + C::COL_S + grp * 32, hi);
+          tmem_st16(tbase + lane_base + C::COL_S + grp * 32 + 16, lo);
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        mbar_arrive(bar(BB_PFULL));
+
+        // ---- dQ of the previous query tile (its MMA ran during this P phase)
+        if (t >= 1) drain_dq(t - 1, prev_q0, prev_bh);
+        // ---- the previous item's dK, dV (complete since that drain)
+        if (i == 0 && prev_kt >= 0) epilogue(prev_kt, prev_bh);
+
+        // ---- dS phase
+        wait_warp(w, bar(BB_DPFULL), t & 1, 17);
+        tc_fence_after();
+        // (the Delta vector arrived with Q_t, whose barrier was waited above)
+        const uint32_t sD = sbase + C::OFF_DELTA + qs * 512 + grp * 128;
+        uint32_t hi[16], lo[16];
+        {
+          uint32_t v[32];
+          tmem_ld32(tbase + lane_base + C::COL_DP + grp * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            float d0, d1, d2, d3;
+            ld_shared_v4f(sD + e * 4, d0, d1, d2, d3);
+            const float s0 = pv[e] * (__uint_as_float(v[e]) - d0);
+            const float s1 = pv[e + 1] * (__uint_as_float(v[e + 1]) - d1);
+            const float s2 = pv[e + 2] * (__uint_as_float(v[e + 2]) - d2);
+            const float s3 = pv[e + 3] * (__uint_as_float(v[e + 3]) - d3);
+            if (SLO) {
+              split_bf16x2_p(f2(s0, s1), hi[e / 2], lo[e / 2]);
+              split_bf16x2_p(f2(s2, s3), hi[e / 2 + 1], lo[e / 2 + 1]);
+            } else {
+              hi[e / 2] = pack_bf16(s0, s1);
+              hi[e / 2 + 1] = pack_bf16(s2, s3);
+            }
+          }
+        }
+        tmem_st16(tbase + lane_base + C::COL_DP + grp * 32, hi);
+        if (SLO) tmem_st16(tbase + lane_base + C::COL_DP + grp * 32 + 16, lo);
+        // dS (hi, lo) -> shared for the dQ MMA: [2][128 keys][64 queries];
+        // query block g is half g/2, chunks 4*(g%2) .. +3 of the row.  (dQ(t-1),
+        // which read the previous dS, is complete: drained above.)
+        if (t >= 1) staging_free();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const uint32_t off = (grp >> 1) * 16384 + swz<128>(r * 128 + ((grp & 1) * 4 + ch) * 16);
+          st_shared_v4(sDSH + off, hi[4 * ch], hi[4 * ch + 1], hi[4 * ch + 2], hi[4 * ch + 3]);
+          if (SLO)
+            st_shared_v4(sDSL + off, lo[4 * ch], lo[4 * ch + 1], lo[4 * ch + 2], lo[4 * ch + 3]);
+        }
+        fence_async_smem();
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(BB_DSFULL));
+        prev_q0 = (kt + i) * 128;
+        prev_bh = bh;
+      }
+      prev_kt = kt;
+    }
+    if (t >= 1) {
+      drain_dq(t - 1, prev_q0, prev_bh);  // waits for the last MMAs: everything is complete
+      epilogue(prev_kt, prev_bh);
     }
     // before the CTA exits, its bulk copies must have read their shared
     // memory sources (their global writes complete on their own; the next
     // kernel on the stream sees them)
-    if (C::WARP_DQ && lane == 0) bulk_wait_read0();
-    if (f32out) {
-      if (leader) bulk_wait_read0();
-    } else {
-      tc_fence_before();
-      fence_async_smem();
-      named_bar_sync(1, C::NCOMP);
-      if (leader && !*abort_flag) {
-        for (int b = 0; b < C::NCB; ++b) {
-          tma_store_3d(&tmDV, sDSH + b * C::BLOCK_BYTES, b * C::CB, kt * 128, bh);
-          tma_store_3d(&tmDK, sDSL + b * C::BLOCK_BYTES, b * C::CB, kt * 128, bh);
-        }
-        bulk_commit();
-      }
-      if (leader) bulk_wait_read0();
+    if (C::WARP_DQ) {
+      if (lane == 0) bulk_wait_read0();
+    } else if (leader) {
+      bulk_wait_read0();
     }
   }
 
