@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float4* __restric
 // Main backward kernel
 // ---------------------------------------------------------------------------
 //
-// One CTA per (head, 128-key tile j).  For each query tile i >= j:
+// Work item: (head, 128-key tile j).  For each query tile i >= j:
 //   S^T  = K_j Q_i^T               (TMEM, fp32; lane = key)
 //   P^T  = exp2(S^T*scale*log2e - LSE2_i); masked on the diagonal tile;
 //          written back over S^T as bf16 hi/lo pairs
@@ -155,18 +155,19 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float4* __restric
 //          drained to shared memory and added into the fp32 accumulator
 //          with a TMA reduce-add.
 //
-// Warp roles (576 threads):
+// Warp roles (608 threads):
 //   warps 0-15 compute: warp w serves TMEM lanes 32*(w%4).. (key rows) and
 //              query columns 32*(w/4) .. +32 of the tile (four warps per SM
 //              sub-partition, to hide the latency of the exponentials and
 //              tensor-memory loads); they also drain dQ and write dK, dV.
-//   warp 16    TMA producer: K_j, V_j once; Q_i with the LSE2 and Delta
-//              vectors through a 2-stage ring (freed after dK(i), which
-//              follows every read of them), dO_i through a 2-stage
-//              (D <= 64) or 1-stage ring (freed after dV(i)).
-//   warp 17    MMA issuer and TMEM owner.  Order per iteration:
-//              dV(i), S(i+1), dK(i), dQ(i), dP(i+1) -- so S(i+1) runs while
-//              dS(i) is computed and dK/dQ(i), dP(i+1) while P(i+1) is.
+//   warp 16    TMA producer: per work item K, V (double-buffered where
+//              shared memory allows); Q_t with the LSE2 and Delta vectors
+//              through a 2-stage ring, dO_t through a 2-stage (D <= 64) or
+//              1-stage ring, both running on across items.
+//   warp 17    MMA issuer A and TMEM owner: S(t+1) as soon as dV(t) has read
+//              P^T(t), dQ(t), dP(t+1) once dK(t) has read dS^T(t).
+//   warp 18    MMA issuer B: dV(t), dK(t).
+// The kernel is persistent: CTA b loops over work items (key tiles).
 
 struct BwdParams {
   const float* lse2;   // (BH, T_pad) LSE * log2(e); +inf on padding rows
@@ -241,7 +242,7 @@ struct BwdCfg {
   static constexpr uint32_t COL_DQ = ALIAS_DQ ? COL_DP : 256 + 2 * D;
   static constexpr uint32_t COL_DVL = SPLIT_DV ? 256 + 3 * D : COL_DV;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int THREADS = 576;
+  static constexpr int THREADS = 608;
   static constexpr int NCOMP = 512;   // compute threads
 };
 
@@ -250,7 +251,7 @@ struct BwdCfg {
 enum : int {
   BB_KVFULL = 0, BB_KVFREE = 2, BB_QFULL = 4, BB_QEMPTY = 6, BB_DOFULL = 8, BB_DOEMPTY = 10,
   BB_SFULL = 12, BB_DPFULL = 13, BB_PFULL = 14, BB_DSFULL = 15, BB_DQFULL = 16,
-  BB_DQEMPTY = 17, BB_ACCFREE = 18, BB_DRAIN = 19
+  BB_DQEMPTY = 17, BB_ACCFREE = 18, BB_PTDONE = 19, BB_DKDONE = 20, BB_DRAIN = 21  // + 0, 1
 };
 
 // Work items: key tiles (kt, bh), numbered longest first (u = 0 ..
@@ -264,12 +265,12 @@ __device__ __forceinline__ int bwd_item(int k, int b, int G, int n_items) {
 }
 
 template <int D, bool SLO>
-__global__ void __launch_bounds__(576, 1)
+__global__ void __launch_bounds__(608, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
            const __grid_constant__ CUtensorMap tmDQacc, const BwdParams p) {
   using C = BwdCfg<D, SLO>;
-  static_assert(BB_DRAIN < C::NUM_BARS, "barrier count");
+  static_assert(BB_DRAIN + 2 <= C::NUM_BARS, "barrier count");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = aligned_smem(smem_raw, C::SMEM_USED);
   if (smem == nullptr) return;  // uniform over the CTA: nothing touched yet
@@ -300,7 +301,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     }
     for (int s = 0; s < C::DOST; ++s) {
       mbar_init(bar(BB_DOFULL + s), 1);
-      mbar_init(bar(BB_DOEMPTY + s), 1);
+      mbar_init(bar(BB_DOEMPTY + s), 2);  // released by dP (warp 17) and dV (warp 18)
     }
     mbar_init(bar(BB_SFULL), 1);
     mbar_init(bar(BB_DPFULL), 1);
@@ -309,7 +310,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     mbar_init(bar(BB_DQFULL), 1);
     mbar_init(bar(BB_DQEMPTY), C::NCOMP);
     mbar_init(bar(BB_ACCFREE), C::NCOMP);
+    mbar_init(bar(BB_PTDONE), 1);
+    mbar_init(bar(BB_DKDONE), 1);
     mbar_init(bar(BB_DRAIN), 1);
+    mbar_init(bar(BB_DRAIN + 1), 1);
     fence_mbar_init();
   }
   if (warp == 17) {
@@ -393,137 +397,174 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           wait1(wd, bar(BB_DOFULL + j % C::DOST), (j / C::DOST) & 1, 22);
       }
     }
-  } else if (warp == 17) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 17 || warp == 18) {
+    // -------------------------------------------------- MMA issuers
+    // warp 17 (A): S, dP, dQ -- the products that read K and V;
+    // warp 18 (B): dV, dK -- the accumulations.  One thread issues an
+    // N = 64 MMA only every ~50 cycles, so two issuers keep the tensor core
+    // busier.  What one issuer's in-order execution guaranteed is now
+    // explicit: S(t+1) waits for dV(t) (PTDONE), dP(t+1) for dK(t) (DKDONE).
     if (lane == 0) {
       constexpr uint32_t idSS = idesc_bf16(128, 128, 0, 0);  // S^T, dP^T
       constexpr uint32_t idKD = idesc_bf16(128, D, 0, 1);    // dV, dK: B MN-major
       constexpr uint32_t idQ = idesc_bf16(128, D, 1, 1);     // dQ: A (dS) MN-major
-      auto issue_s = [&](int t, uint32_t k_s) {  // S^T = K Q_t^T
-        const int qs = t % C::QST;
-        wait1(w, bar(BB_QFULL + qs), (t / C::QST) & 1, 4);
-        tc_fence_after();
-        const uint32_t sQ = sbase + C::OFF_Q + qs * C::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int blk = (kk * 16) / C::CB;
-          const int off = ((kk * 16) % C::CB) * 2;
-          mma_ss(tbase + C::COL_S,
-                 smem_desc(k_s + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW),
-                 smem_desc(sQ + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW), idSS,
-                 kk > 0 ? 1u : 0u);
-        }
-        mma_commit(bar(BB_SFULL));
-      };
-      auto issue_dp = [&](int t, uint32_t v_s) {  // dP^T = V dO_t^T
-        const int ds = t % C::DOST;
-        wait1(w, bar(BB_DOFULL + ds), (t / C::DOST) & 1, 5);
-        // dP overwrites dS^T(t-1), which dK(t-1) read in order before it,
-        // and, aliased, dQ(t-1), which the compute warps must have drained
-        if (C::ALIAS_DQ && t >= 1) wait1(w, bar(BB_DQEMPTY), (t - 1) & 1, 12);
-        tc_fence_after();
-        const uint32_t sDO = sbase + C::OFF_DO + ds * C::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int blk = (kk * 16) / C::CB;
-          const int off = ((kk * 16) % C::CB) * 2;
-          mma_ss(tbase + C::COL_DP,
-                 smem_desc(v_s + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW),
-                 smem_desc(sDO + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW), idSS,
-                 kk > 0 ? 1u : 0u);
-        }
-        mma_commit(bar(BB_DPFULL));
-      };
-      int t = 0, n = 0;
-      for (int k = 0;; ++k) {
-        const int u = bwd_item(k, b, G, n_items);
-        if (u < 0) break;
-        const int kt = u / p.BH;
-        const int n_iter = p.n_tiles - kt;
-        const int kvb = n % C::KVB;
-        const uint32_t k_s = sK(kvb), v_s = sV(kvb);
-        wait1(w, bar(BB_KVFULL + kvb), (n / C::KVB) & 1, 6);
-        // S(t) overwrites P^T(t-1), read by dV(t-1) before it in order
-        issue_s(t, k_s);
-        issue_dp(t, v_s);
-        for (int i = 0; i < n_iter; ++i, ++t) {
+      if (warp == 17) {
+        auto issue_s = [&](int t, uint32_t k_s) {  // S^T = K Q_t^T
           const int qs = t % C::QST;
-          const int ds = t % C::DOST;
+          wait1(w, bar(BB_QFULL + qs), (t / C::QST) & 1, 4);
+          // S overwrites P^T(t-1), which dV(t-1) reads
+          if (t >= 1) wait1(w, bar(BB_PTDONE), (t - 1) & 1, 24);
+          tc_fence_after();
           const uint32_t sQ = sbase + C::OFF_Q + qs * C::TILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int blk = (kk * 16) / C::CB;
+            const int off = ((kk * 16) % C::CB) * 2;
+            mma_ss(tbase + C::COL_S,
+                   smem_desc(k_s + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW),
+                   smem_desc(sQ + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW), idSS,
+                   kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(BB_SFULL));
+        };
+        auto issue_dp = [&](int t, uint32_t v_s) {  // dP^T = V dO_t^T
+          const int ds = t % C::DOST;
+          wait1(w, bar(BB_DOFULL + ds), (t / C::DOST) & 1, 5);
+          // dP overwrites dS^T(t-1), which dK(t-1) reads, and, aliased,
+          // dQ(t-1), which the compute warps must have drained
+          if (t >= 1) wait1(w, bar(BB_DKDONE), (t - 1) & 1, 25);
+          if (C::ALIAS_DQ && t >= 1) wait1(w, bar(BB_DQEMPTY), (t - 1) & 1, 12);
+          tc_fence_after();
           const uint32_t sDO = sbase + C::OFF_DO + ds * C::TILE_BYTES;
-          // dV += P^T dO_t  (A = P^T hi/lo in TMEM over S^T; K = 128 queries)
-          wait1(w, bar(BB_PFULL), t & 1, 7);
-          // the first dV, dK of an item overwrite the accumulators: the
-          // previous item's epilogue must have read them
-          if (i == 0 && n > 0) wait1(w, bar(BB_ACCFREE), (n - 1) & 1, 8);
-          tc_fence_after();
-          const uint64_t ddo = smem_desc(sDO, C::BLOCK_BYTES, 8 * C::RB, C::SW);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t acol = C::COL_S + (kk >> 1) * 32 + (kk & 1) * 8;
-            const uint64_t bd = ddo + ((kk * 16 * C::RB) >> 4);
-            const uint32_t first = (i > 0 || kk > 0) ? 1u : 0u;
-            mma_ts(tbase + C::COL_DV, tbase + acol, bd, idKD, first);
-            mma_ts(tbase + C::COL_DVL, tbase + acol + 16, bd, idKD, C::SPLIT_DV ? first : 1u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int blk = (kk * 16) / C::CB;
+            const int off = ((kk * 16) % C::CB) * 2;
+            mma_ss(tbase + C::COL_DP,
+                   smem_desc(v_s + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW),
+                   smem_desc(sDO + blk * C::BLOCK_BYTES + off, 16, 8 * C::RB, C::SW), idSS,
+                   kk > 0 ? 1u : 0u);
           }
-          mma_commit(bar(BB_DOEMPTY + ds));
-          // S(t+1) overwrites P^T(t); the MMAs execute in issue order, so it
-          // cannot before dV(t) has read it
-          if (i + 1 < n_iter) issue_s(t + 1, k_s);
-          // dK += dS^T Q_t (A = dS^T hi/lo in TMEM over dP^T) and
-          // dQ_t = dS K (A = dS hi/lo in shared, MN-major; K = 128 keys)
-          wait1(w, bar(BB_DSFULL), t & 1, 9);
-          if (!C::ALIAS_DQ && t >= 1) wait1(w, bar(BB_DQEMPTY), (t - 1) & 1, 10);
-          tc_fence_after();
-          const uint64_t dqq = smem_desc(sQ, C::BLOCK_BYTES, 8 * C::RB, C::SW);
-          const uint64_t dkk = smem_desc(k_s, C::BLOCK_BYTES, 8 * C::RB, C::SW);
-          const uint64_t dsh = smem_desc(sDSH, 16384, 1024, 2);
-          const uint64_t dsl = smem_desc(sDSL, 16384, 1024, 2);
-          auto dk_step = [&](int kk, int lo) {
-            if (!SLO && lo) return;
-            const uint32_t acol = C::COL_DP + (kk >> 1) * 32 + (kk & 1) * 8 + (lo ? 16 : 0);
-            mma_ts(tbase + C::COL_DK, tbase + acol, dqq + ((kk * 16 * C::RB) >> 4), idKD,
-                   (i > 0 || kk > 0 || lo) ? 1u : 0u);
-          };
-          auto dq_step = [&](int kk, int lo) {
-            if (!SLO && lo) return;
-            mma_ss(tbase + C::COL_DQ, (lo ? dsl : dsh) + ((kk * 2048) >> 4),
-                   dkk + ((kk * 16 * C::RB) >> 4), idQ, (kk > 0 || lo) ? 1u : 0u);
-          };
-          if constexpr (C::ALIAS_DQ) {
-            // dQ overwrites the dS^T that dK reads: all of dK first (in order)
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              dk_step(kk, 0);
-              dk_step(kk, 1);
+          mma_commit(bar(BB_DPFULL));
+          mma_commit(bar(BB_DOEMPTY + ds));  // one of the slot's two releases
+        };
+        // a flat walk over the CTA's (item, query tile) pairs, one ahead:
+        // S and dP of the next pair are issued as early as their operands
+        // and buffers allow, across item boundaries when the next item's
+        // K, V have their own buffer
+        int k = 0, u = bwd_item(0, b, G, n_items);
+        if (u >= 0) {
+          int kt = u / p.BH, n_iter = p.n_tiles - kt, i = 0, n = 0, t = 0;
+          wait1(w, bar(BB_KVFULL + 0), 0, 6);
+          issue_s(0, sK(0));
+          issue_dp(0, sV(0));
+          while (true) {
+            // the pair after (n, i)
+            int u2 = u, i2 = i + 1, n2 = n;
+            if (i2 == n_iter) {
+              u2 = bwd_item(k + 1, b, G, n_items);
+              i2 = 0;
+              n2 = n + 1;
             }
-            mma_commit(bar(BB_QEMPTY + qs));
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              dq_step(kk, 0);
-              dq_step(kk, 1);
+            const bool has_next = u2 >= 0;
+            const bool new_item = has_next && n2 != n;
+            const int kvb2 = n2 % C::KVB;
+            const bool early = has_next && (!new_item || C::KVB == 2);
+            if (early) {
+              if (new_item) wait1(w, bar(BB_KVFULL + kvb2), (n2 / C::KVB) & 1, 6);
+              issue_s(t + 1, sK(kvb2));
             }
-          } else {
+            // dQ_t = dS K (A = dS hi/lo in shared, MN-major; K = 128 keys)
+            wait1(w, bar(BB_DSFULL), t & 1, 9);
+            if (!C::ALIAS_DQ && t >= 1) wait1(w, bar(BB_DQEMPTY), (t - 1) & 1, 10);
+            if (C::ALIAS_DQ) wait1(w, bar(BB_DKDONE), t & 1, 26);  // dQ overwrites dS^T
+            tc_fence_after();
+            {
+              const uint64_t dkk = smem_desc(sK(n % C::KVB), C::BLOCK_BYTES, 8 * C::RB, C::SW);
+              const uint64_t dsh = smem_desc(sDSH, 16384, 1024, 2);
+              const uint64_t dsl = smem_desc(sDSL, 16384, 1024, 2);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              dk_step(kk, 0);
-              dq_step(kk, 0);
-              dk_step(kk, 1);
-              dq_step(kk, 1);
+              for (int kk = 0; kk < 8; ++kk) {
+                mma_ss(tbase + C::COL_DQ, dsh + ((kk * 2048) >> 4), dkk + ((kk * 16 * C::RB) >> 4),
+                       idQ, kk > 0 ? 1u : 0u);
+                if (SLO)
+                  mma_ss(tbase + C::COL_DQ, dsl + ((kk * 2048) >> 4),
+                         dkk + ((kk * 16 * C::RB) >> 4), idQ, 1u);
+              }
             }
-            mma_commit(bar(BB_QEMPTY + qs));
+            mma_commit(bar(BB_DQFULL));
+            // every MMA that reads this item's K, V has been issued
+            if (!has_next || new_item) mma_commit(bar(BB_KVFREE + n % C::KVB));
+            if (!has_next) break;
+            if (!early) {
+              wait1(w, bar(BB_KVFULL + kvb2), (n2 / C::KVB) & 1, 6);
+              issue_s(t + 1, sK(kvb2));
+            }
+            issue_dp(t + 1, sV(kvb2));
+            if (new_item) {
+              k = k + 1;
+              u = u2;
+              kt = u / p.BH;
+              n_iter = p.n_tiles - kt;
+            }
+            i = i2;
+            n = n2;
+            ++t;
           }
-          mma_commit(bar(BB_DQFULL));
-          if (i + 1 < n_iter) issue_dp(t + 1, v_s);
         }
-        // every MMA that reads this item's K, V has been issued
-        mma_commit(bar(BB_KVFREE + kvb));
-        ++n;
+      } else {
+        int t = 0, n = 0;
+        for (int k = 0;; ++k) {
+          const int u = bwd_item(k, b, G, n_items);
+          if (u < 0) break;
+          const int n_iter = p.n_tiles - u / p.BH;
+          for (int i = 0; i < n_iter; ++i, ++t) {
+            const int qs = t % C::QST;
+            const int ds = t % C::DOST;
+            const uint32_t sQ = sbase + C::OFF_Q + qs * C::TILE_BYTES;
+            const uint32_t sDO = sbase + C::OFF_DO + ds * C::TILE_BYTES;
+            // dV += P^T dO_t  (A = P^T hi/lo in TMEM over S^T; K = 128 queries)
+            wait1(w, bar(BB_PFULL), t & 1, 7);
+            // the first dV, dK of an item overwrite the accumulators: the
+            // previous item's epilogue must have read them
+            if (i == 0 && n > 0) wait1(w, bar(BB_ACCFREE), (n - 1) & 1, 8);
+            wait1(w, bar(BB_DOFULL + ds), (t / C::DOST) & 1, 27);  // (visibility)
+            tc_fence_after();
+            const uint64_t ddo = smem_desc(sDO, C::BLOCK_BYTES, 8 * C::RB, C::SW);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t acol = C::COL_S + (kk >> 1) * 32 + (kk & 1) * 8;
+              const uint64_t bd = ddo + ((kk * 16 * C::RB) >> 4);
+              const uint32_t first = (i > 0 || kk > 0) ? 1u : 0u;
+              mma_ts(tbase + C::COL_DV, tbase + acol, bd, idKD, first);
+              mma_ts(tbase + C::COL_DVL, tbase + acol + 16, bd, idKD, C::SPLIT_DV ? first : 1u);
+            }
+            mma_commit(bar(BB_PTDONE));
+            mma_commit(bar(BB_DOEMPTY + ds));  // the slot's other release
+            // dK += dS^T Q_t (A = dS^T hi/lo in TMEM over dP^T)
+            wait1(w, bar(BB_DSFULL), t & 1, 9);
+            wait1(w, bar(BB_QFULL + qs), (t / C::QST) & 1, 28);  // (visibility)
+            tc_fence_after();
+            const uint64_t dqq = smem_desc(sQ, C::BLOCK_BYTES, 8 * C::RB, C::SW);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t acol = C::COL_DP + (kk >> 1) * 32 + (kk & 1) * 8;
+              mma_ts(tbase + C::COL_DK, tbase + acol, dqq + ((kk * 16 * C::RB) >> 4), idKD,
+                     (i > 0 || kk > 0) ? 1u : 0u);
+              if (SLO)
+                mma_ts(tbase + C::COL_DK, tbase + acol + 16, dqq + ((kk * 16 * C::RB) >> 4), idKD,
+                       1u);
+            }
+            mma_commit(bar(BB_DKDONE));
+            mma_commit(bar(BB_QEMPTY + qs));  // S(t), which also read Q_t, completed long ago
+          }
+          ++n;
+        }
       }
-      mma_commit(bar(BB_DRAIN));
+      mma_commit(bar(BB_DRAIN + (warp - 17)));
       int zero = 0;
       WaitCtx wd{p.timeout_ns, &zero, 2u};
-      wait1(wd, bar(BB_DRAIN), 0, 13);
+      wait1(wd, bar(BB_DRAIN + (warp - 17)), 0, 13);
     }
   } else {
     // ------------------------------------------- compute warps (row = key)
@@ -623,11 +664,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       }
     };
 
-    // dK, dV epilogue of key tile kt of head bh: this thread's NQ columns of
-    // its key row, straight from TMEM to global memory.  (The accumulators
-    // are complete: the dQ drain of the item's last iteration waited for
-    // the MMAs that finished them.)
-    auto epilogue = [&](int kt, int bh) {
+    // dK, dV epilogue of key tile kt of head bh, whose last query tile was
+    // t_last: this thread's NQ columns of its key row, straight from TMEM
+    // to global memory, once dK(t_last) (and so every dV, dK) is complete
+    auto epilogue = [&](int kt, int bh, int t_last) {
+      wait_warp(w, bar(BB_DKDONE), t_last & 1, 29);
+      tc_fence_after();
       const int key = kt * 128 + r;
       const size_t off = (static_cast<size_t>(bh) * p.T + (key < p.T ? key : 0)) * D + grp * NQ;
       // which = 0: dV (+ dV'), 1: dK * scale; the accumulators are released
@@ -723,7 +765,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // ---- dQ of the previous query tile (its MMA ran during this P phase)
         if (t >= 1) drain_dq(t - 1, prev_q0, prev_bh);
         // ---- the previous item's dK, dV (complete since that drain)
-        if (i == 0 && prev_kt >= 0) epilogue(prev_kt, prev_bh);
+        if (i == 0 && prev_kt >= 0) epilogue(prev_kt, prev_bh, t - 1);
 
         // ---- dS phase
         wait_warp(w, bar(BB_DPFULL), t & 1, 17);
@@ -776,7 +818,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     }
     if (t >= 1) {
       drain_dq(t - 1, prev_q0, prev_bh);  // waits for the last MMAs: everything is complete
-      epilogue(prev_kt, prev_bh);
+      epilogue(prev_kt, prev_bh, t - 1);
     }
     // before the CTA exits, its bulk copies must have read their shared
     // memory sources (their global writes complete on their own; the next
