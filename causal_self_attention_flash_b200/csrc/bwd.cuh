@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float4* __restric
 //          drained to shared memory and added into the fp32 accumulator
 //          with a TMA reduce-add.
 //
-// Warp roles (608 threads):
+// Warp roles (640 threads):
 //   warps 0-15 compute: warp w serves TMEM lanes 32*(w%4).. (key rows) and
 //              query columns 32*(w/4) .. +32 of the tile (four warps per SM
 //              sub-partition, to hide the latency of the exponentials and
@@ -166,7 +166,9 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float4* __restric
 //              1-stage ring, both running on across items.
 //   warp 17    MMA issuer A and TMEM owner: S(t+1) as soon as dV(t) has read
 //              P^T(t), dQ(t), dP(t+1) once dK(t) has read dS^T(t).
-//   warp 18    MMA issuer B: dV(t), dK(t).
+//   warp 18    MMA issuer B: dV(t) (P^T_hi part), dK(t).
+//   warp 19    MMA issuer C: the P^T_lo part of dV(t), into dV' (where TMEM
+//              holds a separate dV' accumulator; otherwise warp 18 does it).
 // The kernel is persistent: CTA b loops over work items (key tiles).
 
 struct BwdParams {
@@ -225,7 +227,7 @@ struct BwdCfg {
   static constexpr int OFF_DELTA = OFF_LSE + QST * 512;       // [QST][128] fp32
   static constexpr int OFF_DQW = (OFF_DELTA + QST * 512 + 1023) / 1024 * 1024;
   static constexpr int OFF_BAR = WARP_DQ ? OFF_DQW + 16 * WARP_STAGE : OFF_DELTA + QST * 512;
-  static constexpr int NUM_BARS = 24;
+  static constexpr int NUM_BARS = 26;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_USED = OFF_MISC + 64;
   static constexpr int SMEM_BYTES =
@@ -242,7 +244,7 @@ struct BwdCfg {
   static constexpr uint32_t COL_DQ = ALIAS_DQ ? COL_DP : 256 + 2 * D;
   static constexpr uint32_t COL_DVL = SPLIT_DV ? 256 + 3 * D : COL_DV;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int THREADS = 608;
+  static constexpr int THREADS = 640;
   static constexpr int NCOMP = 512;   // compute threads
 };
 
@@ -251,7 +253,9 @@ struct BwdCfg {
 enum : int {
   BB_KVFULL = 0, BB_KVFREE = 2, BB_QFULL = 4, BB_QEMPTY = 6, BB_DOFULL = 8, BB_DOEMPTY = 10,
   BB_SFULL = 12, BB_DPFULL = 13, BB_PFULL = 14, BB_DSFULL = 15, BB_DQFULL = 16,
-  BB_DQEMPTY = 17, BB_ACCFREE = 18, BB_PTDONE = 19, BB_DKDONE = 20, BB_DRAIN = 21  // + 0, 1
+  BB_DQEMPTY = 17, BB_ACCFREE = 18, BB_PTDONE = 19, BB_DKDONE = 20,
+  BB_DRAIN = 21,  // + issuer 0, 1, 2
+  BB_PFULL2 = 24  // second half of P^T (BB_PFULL is the first)
 };
 
 // Work items: key tiles (kt, bh), numbered longest first (u = 0 ..
@@ -265,12 +269,12 @@ __device__ __forceinline__ int bwd_item(int k, int b, int G, int n_items) {
 }
 
 template <int D, bool SLO>
-__global__ void __launch_bounds__(608, 1)
+__global__ void __launch_bounds__(640, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
            const __grid_constant__ CUtensorMap tmDQacc, const BwdParams p) {
   using C = BwdCfg<D, SLO>;
-  static_assert(BB_DRAIN + 2 <= C::NUM_BARS, "barrier count");
+  static_assert(BB_PFULL2 + 1 <= C::NUM_BARS, "barrier count");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = aligned_smem(smem_raw, C::SMEM_USED);
   if (smem == nullptr) return;  // uniform over the CTA: nothing touched yet
@@ -301,19 +305,22 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     }
     for (int s = 0; s < C::DOST; ++s) {
       mbar_init(bar(BB_DOFULL + s), 1);
-      mbar_init(bar(BB_DOEMPTY + s), 2);  // released by dP (warp 17) and dV (warp 18)
+      // released by dP (warp 17) and dV (warp 18, and 19 with a dV' accumulator)
+      mbar_init(bar(BB_DOEMPTY + s), C::SPLIT_DV ? 3 : 2);
     }
     mbar_init(bar(BB_SFULL), 1);
     mbar_init(bar(BB_DPFULL), 1);
     mbar_init(bar(BB_PFULL), C::NCOMP);
+    mbar_init(bar(BB_PFULL2), C::NCOMP);
     mbar_init(bar(BB_DSFULL), C::NCOMP);
     mbar_init(bar(BB_DQFULL), 1);
     mbar_init(bar(BB_DQEMPTY), C::NCOMP);
     mbar_init(bar(BB_ACCFREE), C::NCOMP);
-    mbar_init(bar(BB_PTDONE), 1);
+    mbar_init(bar(BB_PTDONE), C::SPLIT_DV ? 2 : 1);  // dV by warps 18 (and 19)
     mbar_init(bar(BB_DKDONE), 1);
     mbar_init(bar(BB_DRAIN), 1);
     mbar_init(bar(BB_DRAIN + 1), 1);
+    mbar_init(bar(BB_DRAIN + 2), 1);
     fence_mbar_init();
   }
   if (warp == 17) {
@@ -397,14 +404,14 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           wait1(wd, bar(BB_DOFULL + j % C::DOST), (j / C::DOST) & 1, 22);
       }
     }
-  } else if (warp == 17 || warp == 18) {
+  } else if (warp >= 17) {
     // -------------------------------------------------- MMA issuers
     // warp 17 (A): S, dP, dQ -- the products that read K and V;
-    // warp 18 (B): dV, dK -- the accumulations.  One thread issues an
-    // N = 64 MMA only every ~50 cycles, so two issuers keep the tensor core
-    // busier.  What one issuer's in-order execution guaranteed is now
+    // warps 18, 19 (B, C): dV, dK -- the accumulations.  One thread issues
+    // an N = 64 MMA only every ~50 cycles, so several issuers keep the
+    // tensor core busier.  What one issuer's in-order execution guaranteed is now
     // explicit: S(t+1) waits for dV(t) (PTDONE), dP(t+1) for dK(t) (DKDONE).
-    if (lane == 0) {
+    if (lane == 0 && (warp != 19 || C::SPLIT_DV)) {
       constexpr uint32_t idSS = idesc_bf16(128, 128, 0, 0);  // S^T, dP^T
       constexpr uint32_t idKD = idesc_bf16(128, D, 0, 1);    // dV, dK: B MN-major
       constexpr uint32_t idQ = idesc_bf16(128, D, 1, 1);     // dQ: A (dS) MN-major
@@ -523,24 +530,35 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             const int ds = t % C::DOST;
             const uint32_t sQ = sbase + C::OFF_Q + qs * C::TILE_BYTES;
             const uint32_t sDO = sbase + C::OFF_DO + ds * C::TILE_BYTES;
-            // dV += P^T dO_t  (A = P^T hi/lo in TMEM over S^T; K = 128 queries)
-            wait1(w, bar(BB_PFULL), t & 1, 7);
+            // dV += P^T dO_t  (A = P^T hi/lo in TMEM over S^T; K = 128 queries),
+            // in two halves as the compute warps hand P^T over: MMA kk
+            // reads queries 16kk.., i.e. half kk % 2 of query block kk / 2.
+            // Warp 18 adds P^T_hi (and, without a dV' accumulator, P^T_lo),
+            // warp 19 adds P^T_lo into dV'.
+            const bool lo_role = warp == 19;
             // the first dV, dK of an item overwrite the accumulators: the
             // previous item's epilogue must have read them
             if (i == 0 && n > 0) wait1(w, bar(BB_ACCFREE), (n - 1) & 1, 8);
             wait1(w, bar(BB_DOFULL + ds), (t / C::DOST) & 1, 27);  // (visibility)
-            tc_fence_after();
             const uint64_t ddo = smem_desc(sDO, C::BLOCK_BYTES, 8 * C::RB, C::SW);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t acol = C::COL_S + (kk >> 1) * 32 + (kk & 1) * 8;
-              const uint64_t bd = ddo + ((kk * 16 * C::RB) >> 4);
-              const uint32_t first = (i > 0 || kk > 0) ? 1u : 0u;
-              mma_ts(tbase + C::COL_DV, tbase + acol, bd, idKD, first);
-              mma_ts(tbase + C::COL_DVL, tbase + acol + 16, bd, idKD, C::SPLIT_DV ? first : 1u);
+            for (int h = 0; h < 2; ++h) {
+              wait1(w, bar(h ? BB_PFULL2 : BB_PFULL), t & 1, 7);
+              tc_fence_after();
+#pragma unroll
+              for (int g4 = 0; g4 < 4; ++g4) {
+                const int kk = 2 * g4 + h;
+                const uint32_t acol = C::COL_S + g4 * 32 + h * 8;
+                const uint64_t bd = ddo + ((kk * 16 * C::RB) >> 4);
+                const uint32_t first = (i > 0 || kk > 0) ? 1u : 0u;
+                if (!lo_role) mma_ts(tbase + C::COL_DV, tbase + acol, bd, idKD, first);
+                if (lo_role || !C::SPLIT_DV)
+                  mma_ts(tbase + C::COL_DVL, tbase + acol + 16, bd, idKD, C::SPLIT_DV ? first : 1u);
+              }
             }
             mma_commit(bar(BB_PTDONE));
-            mma_commit(bar(BB_DOEMPTY + ds));  // the slot's other release
+            mma_commit(bar(BB_DOEMPTY + ds));  // one of the slot's releases
+            if (lo_role) continue;
             // dK += dS^T Q_t (A = dS^T hi/lo in TMEM over dP^T)
             wait1(w, bar(BB_DSFULL), t & 1, 9);
             wait1(w, bar(BB_QFULL + qs), (t / C::QST) & 1, 28);  // (visibility)
@@ -669,6 +687,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     // to global memory, once dK(t_last) (and so every dV, dK) is complete
     auto epilogue = [&](int kt, int bh, int t_last) {
       wait_warp(w, bar(BB_DKDONE), t_last & 1, 29);
+      wait_warp(w, bar(BB_PTDONE), t_last & 1, 30);  // dV' (warp 19) complete too
       tc_fence_after();
       const int key = kt * 128 + r;
       const size_t off = (static_cast<size_t>(bh) * p.T + (key < p.T ? key : 0)) * D + grp * NQ;
@@ -736,31 +755,35 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         }
         wait_warp(w, bar(BB_QFULL + qs), (t / C::QST) & 1, 16);  // LSE2 visibility
         const uint32_t sL = sbase + C::OFF_LSE + qs * 512 + grp * 128;
+        // in two halves of 16 queries, each handed to the dV MMAs as soon
+        // as it is in TMEM (hi at columns 32g + 8h, lo at 32g + 16 + 8h)
 #pragma unroll
-        for (int c = 0; c < 32; c += 4) {
-          float l0, l1, l2, l3;
-          ld_shared_v4f(sL + c * 4, l0, l1, l2, l3);
-          pv[c] = ex2(fmaf(pv[c], sl2, -l0));
-          pv[c + 1] = ex2(fmaf(pv[c + 1], sl2, -l1));
-          pv[c + 2] = ex2(fmaf(pv[c + 2], sl2, -l2));
-          pv[c + 3] = ex2(fmaf(pv[c + 3], sl2, -l3));
-        }
-        if (i == 0) {  // diagonal tile: query (32g + c) sees key r only if r <= query
-          const int lim = r - grp * 32;
+        for (int h = 0; h < 2; ++h) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (c < lim) pv[c] = 0.f;
-        }
-        {
-          uint32_t hi[16], lo[16];
+          for (int c = 16 * h; c < 16 * h + 16; c += 4) {
+            float l0, l1, l2, l3;
+            ld_shared_v4f(sL + c * 4, l0, l1, l2, l3);
+            pv[c] = ex2(fmaf(pv[c], sl2, -l0));
+            pv[c + 1] = ex2(fmaf(pv[c + 1], sl2, -l1));
+            pv[c + 2] = ex2(fmaf(pv[c + 2], sl2, -l2));
+            pv[c + 3] = ex2(fmaf(pv[c + 3], sl2, -l3));
+          }
+          if (i == 0) {  // diagonal tile: query (32g + c) sees key r only if r <= query
+            const int lim = r - grp * 32;
 #pragma unroll
-          for (int e = 0; e < 16; ++e) split_bf16x2_p(f2(pv[2 * e], pv[2 * e + 1]), hi[e], lo[e]);
-          tmem_st16(tbase + lane_base + C::COL_S + grp * 32, hi);
-          tmem_st16(tbase + lane_base + C::COL_S + grp * 32 + 16, lo);
+            for (int c = 16 * h; c < 16 * h + 16; ++c)
+              if (c < lim) pv[c] = 0.f;
+          }
+          uint32_t hi[8], lo[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            split_bf16x2_p(f2(pv[16 * h + 2 * e], pv[16 * h + 2 * e + 1]), hi[e], lo[e]);
+          tmem_st8(tbase + lane_base + C::COL_S + grp * 32 + 8 * h, hi);
+          tmem_st8(tbase + lane_base + C::COL_S + grp * 32 + 16 + 8 * h, lo);
           tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(h ? BB_PFULL2 : BB_PFULL));
         }
-        tc_fence_before();
-        mbar_arrive(bar(BB_PFULL));
 
         // ---- dQ of the previous query tile (its MMA ran during this P phase)
         if (t >= 1) drain_dq(t - 1, prev_q0, prev_bh);
