@@ -422,7 +422,7 @@ def run_cattn(args, w, index, world, rank, local):
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": sum(c for _, c in ktimes.values()),
             "clocks": clocks,
             "device_status": status,
         }
