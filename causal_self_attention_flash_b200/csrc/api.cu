@@ -217,16 +217,14 @@ cattn_status fwd_impl(int dev, const void* q, const void* k, const void* v, floa
   clear_stale_error();
   cattn_status st = ensure_smem(dev, 0 + 2 * d_index(D) + PLO, fwd_kernel<D, PLO>, C::SMEM_BYTES);
   if (st != CATTN_OK) return st;
-  CUtensorMap mq, mk, mv, mo, molo;
+  CUtensorMap mq, mk, mv;
   if ((st = make_bf16_map(&mq, q, D, T, BH)) != CATTN_OK) return st;
   if ((st = make_bf16_map(&mk, k, D, T, BH)) != CATTN_OK) return st;
   if ((st = make_bf16_map(&mv, v, D, T, BH)) != CATTN_OK) return st;
-  if ((st = make_bf16_map(&mo, o, D, T, BH)) != CATTN_OK) return st;
-  // without O_lo the kernel never touches this map; it reuses O's
-  if ((st = make_bf16_map(&molo, o_lo ? o_lo : o, D, T, BH)) != CATTN_OK) return st;
   FwdParams p;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_lo = static_cast<__nv_bfloat16*>(o_lo);
   p.lse = lse;
-  p.write_o_lo = o_lo != nullptr;
   p.T = T;
   p.BH = BH;
   p.n_qtiles = (T + 127) / 128;
@@ -239,7 +237,7 @@ cattn_status fwd_impl(int dev, const void* q, const void* k, const void* v, floa
   dim3 grid(static_cast<unsigned>(n_items < g_sm_count[dev] ? n_items : g_sm_count[dev]));
   {
     LaunchTimer t(K_FWD, s);
-    fwd_kernel<D, PLO><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, molo, p);
+    fwd_kernel<D, PLO><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, p);
   }
   return launch_status();
 }

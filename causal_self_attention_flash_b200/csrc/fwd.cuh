@@ -55,8 +55,9 @@
 namespace cattn {
 
 struct FwdParams {
+  __nv_bfloat16* o;     // (BH, T, D) bf16 out
+  __nv_bfloat16* o_lo;  // O_lo = bf16(O - bf16(O)) out, or null
   float* lse;          // (BH, T) fp32 out
-  int write_o_lo;      // also write O_lo = bf16(O - bf16(O)) through tmOlo
   int T;
   int BH;
   int n_qtiles;
@@ -78,11 +79,7 @@ struct FwdCfg {
   static constexpr int OFF_Q = 0;                              // [2] query tiles
   static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
-  // SEP_O: the O epilogue has its own staging tiles (where they fit), so the
-  // next item's Q can be loaded while this item's O is stored
-  static constexpr int OFF_OST = OFF_V + STAGES * TILE_BYTES;
-  static constexpr bool SEP_O = OFF_OST + 2 * TILE_BYTES + 1024 <= kMaxDynSmem;
-  static constexpr int OFF_BAR = OFF_OST + (SEP_O ? 2 * TILE_BYTES : 0);
+  static constexpr int OFF_BAR = OFF_V + STAGES * TILE_BYTES;
   static constexpr int NUM_BARS = 34;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_USED = OFF_MISC + 64;
@@ -196,8 +193,7 @@ __device__ __forceinline__ FwdItem fwd_item_info(int u, int BH, int n_pairs, int
 template <int D, bool PLO>
 __global__ void __launch_bounds__(352, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-           const __grid_constant__ CUtensorMap tmOlo, const FwdParams p) {
+           const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = FwdCfg<D, PLO>;
   static_assert(FB_PFULL + 8 <= C::NUM_BARS, "barrier count");
   static_assert(C::STAGES <= 3, "barrier map");
@@ -227,7 +223,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     }
     for (int g = 0; g < 2; ++g) {
       mbar_init(bar(FB_QFULL + g), 1);
-      mbar_init(bar(FB_QFREE + g), C::SEP_O ? 1 : 2);
+      mbar_init(bar(FB_QFREE + g), 1);
       mbar_init(bar(FB_SFULL + g), 1);
       for (int h = 0; h < kPvParts; ++h) mbar_init(bar(FB_PFULL + 4 * g + h), 128);
       mbar_init(bar(FB_ODONE + g), 1);
@@ -409,10 +405,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const uint32_t pcol = tbase + lane_base + (g ? C::COL_P1 : C::COL_P0);
     const uint32_t ocol = tbase + lane_base + (g ? C::COL_O1 : C::COL_O0);
     const uint32_t olcol = tbase + lane_base + (g ? C::COL_OL1 : C::COL_OL0);
-    const uint32_t sQg = sbase + C::OFF_Q + g * C::TILE_BYTES;
-    const uint32_t sOg = C::SEP_O ? sbase + C::OFF_OST + g * C::TILE_BYTES : sQg;
-    const uint32_t nbar = 1 + g;
-    const bool leader = (threadIdx.x & 127) == 0;
     const float sl2 = p.scale_log2;
     int tg = 0;
     float s[128];
@@ -512,7 +504,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       tc_fence_after();
       const float inv_l = 1.f / l;
       // O (and O') into registers; then TMEM is free for the next item
-      uint32_t o_all[D / 2], lo_all[D / 2];
+      uint32_t o_all[D / 2], lo_all[PLO ? D / 2 : 1];
 #pragma unroll
       for (int cc = 0; cc < D / 16; ++cc) {
         uint32_t r[16];
@@ -528,58 +520,32 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           tmem_wait_ld();
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          split_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l,
-                       o_all[cc * 8 + e], lo_all[cc * 8 + e]);
+        for (int e = 0; e < 8; ++e) {
+          const float x0 = __uint_as_float(r[2 * e]) * inv_l;
+          const float x1 = __uint_as_float(r[2 * e + 1]) * inv_l;
+          if constexpr (PLO) split_bf16x2(x0, x1, o_all[cc * 8 + e], lo_all[cc * 8 + e]);
+          else o_all[cc * 8 + e] = pack_bf16(x0, x1);
+        }
       }
       tc_fence_before();
       mbar_arrive(bar(FB_OFREE + g));
-      // staging (the separate O tile, or this group's Q tile, which every
-      // MMA that read it has finished with): O, then O_lo through the same
-      // buffer
-      auto stage = [&](const uint32_t (&x)[D / 2]) {
-#pragma unroll
-        for (int cc = 0; cc < D / 16; ++cc) {
-          const int d0 = cc * 16;
-          const int blk = d0 / C::CB;
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int dd = (d0 % C::CB) + hh * 8;
-            st_shared_v4(sOg + blk * C::BLOCK_BYTES + swz<C::RB>(row * C::RB + dd * 2),
-                         x[cc * 8 + 4 * hh], x[cc * 8 + 4 * hh + 1], x[cc * 8 + 4 * hh + 2],
-                         x[cc * 8 + 4 * hh + 3]);
-          }
-        }
-      };
+      // each thread writes its own row (D contiguous bf16) straight to
+      // global memory: no staging, no barrier, no wait
       const int tile = it.t0 + g;
-      stage(o_all);
-      fence_async_smem();
-      named_bar_sync(nbar, 128);
-      if (leader && !*abort_flag) {
-        for (int bb = 0; bb < C::NCB; ++bb)
-          tma_store_3d(&tmO, sOg + bb * C::BLOCK_BYTES, bb * C::CB, tile * C::BM, it.bh);
-        bulk_commit();
-      }
-      if (p.write_o_lo) {
-        if (leader) bulk_wait_read0();
-        named_bar_sync(nbar, 128);
-        stage(lo_all);
-        fence_async_smem();
-        named_bar_sync(nbar, 128);
-        if (leader && !*abort_flag) {
-          for (int bb = 0; bb < C::NCB; ++bb)
-            tma_store_3d(&tmOlo, sOg + bb * C::BLOCK_BYTES, bb * C::CB, tile * C::BM, it.bh);
-          bulk_commit();
-        }
-      }
-      // the staging tile is rewritten by the next item (separate O tile) or
-      // by the next Q load (the producer waits for this arrival)
-      if (leader) {
-        bulk_wait_read0();
-        if (!C::SEP_O) mbar_arrive(bar(FB_QFREE + g));
-      }
       const int q_row = tile * C::BM + row;
       if (q_row < p.T) {
+        const size_t off = (static_cast<size_t>(it.bh) * p.T + q_row) * D;
+        uint4* orow = reinterpret_cast<uint4*>(p.o + off);
+#pragma unroll
+        for (int e = 0; e < D / 8; ++e)
+          orow[e] = make_uint4(o_all[4 * e], o_all[4 * e + 1], o_all[4 * e + 2], o_all[4 * e + 3]);
+        if (PLO && p.o_lo != nullptr) {
+          uint4* lrow = reinterpret_cast<uint4*>(p.o_lo + off);
+#pragma unroll
+          for (int e = 0; e < D / 8; ++e)
+            lrow[e] = make_uint4(lo_all[4 * e], lo_all[4 * e + 1], lo_all[4 * e + 2],
+                                 lo_all[4 * e + 3]);
+        }
         // natural-log LSE: m_used is in log2 units of the scaled score
         p.lse[static_cast<size_t>(it.bh) * p.T + q_row] = m_used * 0.69314718055994531f + logf(l);
       }
