@@ -62,26 +62,45 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
   const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
   constexpr float kLog2e = 1.4426950408889634f;
 
-  for (long long base = warp_global * RPW; base < p.n_rows; base += n_warps * RPW) {
-    const long long pr = base + lane / TPR;
-    const bool in_range = pr < p.n_rows;
-    long long bh = 0;
-    int t = 0;
-    if (in_range) {
-      bh = pr / p.row_stride;
-      t = static_cast<int>(pr - bh * p.row_stride);
+  // two row groups per step, their loads issued before either is reduced
+  constexpr int U = 2;
+  const bool small = p.n_rows <= 0x7fffffffLL;  // 32-bit index arithmetic
+  for (long long base = warp_global * (RPW * U); base < p.n_rows; base += n_warps * (RPW * U)) {
+    long long pr[U];
+    long long bh[U];
+    int t[U];
+    bool valid[U];
+    uint4 a[U], bb[U], c[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      pr[u] = base + u * RPW + lane / TPR;
+      bh[u] = 0;
+      t[u] = 0;
+      if (pr[u] < p.n_rows) {
+        if (small) {
+          const unsigned q = static_cast<unsigned>(pr[u]) / static_cast<unsigned>(p.row_stride);
+          bh[u] = q;
+          t[u] = static_cast<int>(static_cast<unsigned>(pr[u]) - q * static_cast<unsigned>(p.row_stride));
+        } else {
+          bh[u] = pr[u] / p.row_stride;
+          t[u] = static_cast<int>(pr[u] - bh[u] * p.row_stride);
+        }
+      }
+      valid[u] = pr[u] < p.n_rows && t[u] < p.T;
+      a[u] = bb[u] = c[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (valid[u]) {
+        const size_t off = (static_cast<size_t>(bh[u]) * p.T + t[u]) * D + sub * 8;
+        a[u] = *reinterpret_cast<const uint4*>(p.o + off);
+        bb[u] = *reinterpret_cast<const uint4*>(p.dout + off);
+        if (p.o_lo != nullptr) c[u] = *reinterpret_cast<const uint4*>(p.o_lo + off);
+      }
     }
-    const bool valid = in_range && t < p.T;
-    float acc = 0.f;
-    if (valid) {
-      const size_t off = (static_cast<size_t>(bh) * p.T + t) * D + sub * 8;
-      const uint4 a = *reinterpret_cast<const uint4*>(p.o + off);
-      const uint4 b = *reinterpret_cast<const uint4*>(p.dout + off);
-      uint4 c = make_uint4(0u, 0u, 0u, 0u);
-      if (p.o_lo != nullptr) c = *reinterpret_cast<const uint4*>(p.o_lo + off);
-      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
-      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
-      const __nv_bfloat162* c2 = reinterpret_cast<const __nv_bfloat162*>(&c);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float acc = 0.f;
+      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a[u]);
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&bb[u]);
+      const __nv_bfloat162* c2 = reinterpret_cast<const __nv_bfloat162*>(&c[u]);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 fa = __bfloat1622float2(a2[e]);
@@ -90,13 +109,14 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
         acc = fmaf(fa.x + fc.x, fb.x, acc);
         acc = fmaf(fa.y + fc.y, fb.y, acc);
       }
-    }
 #pragma unroll
-    for (int o = TPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (in_range && sub == 0) {
-      p.delta[pr] = acc;  // 0 on padding rows
-      if (p.lse2 != nullptr)
-        p.lse2[pr] = valid ? p.lse[static_cast<size_t>(bh) * p.T + t] * kLog2e : INFINITY;
+      for (int o = TPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (pr[u] < p.n_rows && sub == 0) {
+        p.delta[pr[u]] = acc;  // 0 on padding rows
+        if (p.lse2 != nullptr)
+          p.lse2[pr[u]] =
+              valid[u] ? p.lse[static_cast<size_t>(bh[u]) * p.T + t[u]] * kLog2e : INFINITY;
+      }
     }
   }
   if (p.zero != nullptr) {

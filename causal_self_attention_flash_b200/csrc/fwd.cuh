@@ -13,7 +13,7 @@
 // on its scores, the MMAs of the other run.
 //
 // Warp roles (352 threads):
-//   warps 0-3, 4-7  softmax warpgroups g = 0, 1 for query tiles 2c+g;
+//   warps 0-3, 4-7  softmax warpgroups g = 0, 1, one query tile each per item;
 //              thread t of a group owns query row t, which is TMEM lane t.
 //              It reads S_g from TMEM, masks the diagonal tile, updates m
 //              and l, and writes P to TMEM: as bf16 (PLO = false, the usual
@@ -175,18 +175,30 @@ __device__ __forceinline__ int fwd_item(int k, int b, int G, int n_items) {
   return u < n_items ? u : -1;
 }
 
+// An item's two query tiles go to the two softmax groups, the longer one
+// (one key tile more) to group 1 on even passes k and to group 0 on odd
+// ones, so that over its items a CTA's groups carry about equal work.
 struct FwdItem {
-  int bh, t0, n0, n1, n_kv;  // query tiles t0 (n0 key tiles), t0+1 (n1, 0 if absent)
+  int bh;
+  int tile[2];  // query tile of group g
+  int n[2];     // key tiles group g visits (0: no tile)
+  int n_kv;     // key tiles loaded for the item
 };
 
-__device__ __forceinline__ FwdItem fwd_item_info(int u, int BH, int n_pairs, int n_qtiles) {
+__device__ __forceinline__ FwdItem fwd_item_info(int u, int k, int BH, int n_pairs,
+                                                  int n_qtiles) {
   FwdItem it;
   const int c = n_pairs - 1 - u / BH;
   it.bh = u % BH;
-  it.t0 = 2 * c;
-  it.n0 = it.t0 + 1;
-  it.n1 = it.t0 + 1 < n_qtiles ? it.t0 + 2 : 0;
-  it.n_kv = it.n1 ? it.n1 : it.n0;
+  const int t0 = 2 * c;
+  const int nlo = t0 + 1;                           // tile t0
+  const int nhi = t0 + 1 < n_qtiles ? t0 + 2 : 0;   // tile t0 + 1, if any
+  const int s = k & 1;
+  it.tile[s] = t0 + 1;
+  it.n[s] = nhi;
+  it.tile[s ^ 1] = t0;
+  it.n[s ^ 1] = nlo;
+  it.n_kv = nhi ? nhi : nlo;
   return it;
 }
 
@@ -255,14 +267,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       for (int k = 0;; ++k) {
         const int u = fwd_item(k, b, G, n_items);
         if (u < 0 || *abort_flag) break;
-        const FwdItem it = fwd_item_info(u, p.BH, n_pairs, p.n_qtiles);
+        const FwdItem it = fwd_item_info(u, k, p.BH, n_pairs, p.n_qtiles);
         for (int g = 0; g < 2; ++g) {
-          if ((g ? it.n1 : it.n0) == 0) continue;
+          if (it.n[g] == 0) continue;
           if (aq[g] > 0) wait1(w, bar(FB_QFREE + g), (aq[g] - 1) & 1, 1);
           mbar_arrive_expect_tx(bar(FB_QFULL + g), C::TILE_BYTES);
           for (int bb = 0; bb < C::NCB; ++bb)
             tma_load_3d(sbase + C::OFF_Q + g * C::TILE_BYTES + bb * C::BLOCK_BYTES, &tmQ,
-                        bar(FB_QFULL + g), bb * C::CB, (it.t0 + g) * C::BM, it.bh);
+                        bar(FB_QFULL + g), bb * C::CB, it.tile[g] * C::BM, it.bh);
           ++aq[g];
         }
         for (int j = 0; j < it.n_kv; ++j, ++tk) {
@@ -349,8 +361,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       for (int k = 0;; ++k) {
         const int u = fwd_item(k, b, G, n_items);
         if (u < 0) break;
-        const FwdItem it = fwd_item_info(u, p.BH, n_pairs, p.n_qtiles);
-        const int ng = g ? it.n1 : it.n0;
+        const FwdItem it = fwd_item_info(u, k, p.BH, n_pairs, p.n_qtiles);
+        const int ng = it.n[g];
         if (ng > 0) {
           wait1(w, bar(FB_QFULL + g), aq & 1, 5);
           // EARLY: S_g is read by the softmax before S_g(0) may overwrite it
@@ -397,7 +409,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int g = warp >> 2;                 // warpgroup = query tile t0 + g
+    const int g = warp >> 2;                 // warpgroup: one query tile per item
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;     // query row in tile == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
@@ -411,8 +423,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     for (int k = 0;; ++k) {
       const int u = fwd_item(k, b, G, n_items);
       if (u < 0) break;
-      const FwdItem it = fwd_item_info(u, p.BH, n_pairs, p.n_qtiles);
-      const int ng = g ? it.n1 : it.n0;
+      const FwdItem it = fwd_item_info(u, k, p.BH, n_pairs, p.n_qtiles);
+      const int ng = it.n[g];
       if (ng == 0) continue;
       float m_used = -INFINITY;  // running max, scaled log2 units
       float l = 0.f;
@@ -531,7 +543,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       mbar_arrive(bar(FB_OFREE + g));
       // each thread writes its own row (D contiguous bf16) straight to
       // global memory: no staging, no barrier, no wait
-      const int tile = it.t0 + g;
+      const int tile = it.tile[g];
       const int q_row = tile * C::BM + row;
       if (q_row < p.T) {
         const size_t off = (static_cast<size_t>(it.bh) * p.T + q_row) * D;
