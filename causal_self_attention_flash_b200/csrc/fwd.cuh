@@ -8,9 +8,11 @@
 // that softmax: a running maximum m and running sum l per row, with the
 // partial output rescaled whenever m moves.
 //
-// One CTA serves two 128-row query tiles (2c, 2c+1) of one head, so the
-// tensor core alternates between them: while one softmax warpgroup works
-// on its scores, the MMAs of the other run.
+// The kernel is persistent: one CTA per SM loops over work items, each a
+// pair of 128-row query tiles (2c, 2c+1) of one head.  The two tiles go to
+// two softmax warpgroups, so the tensor core alternates between them: while
+// one warpgroup works on its scores, the MMAs of the other run.  The next
+// item's Q and K/V are loaded while the current item finishes.
 //
 // Warp roles (352 threads):
 //   warps 0-3, 4-7  softmax warpgroups g = 0, 1, one query tile each per item;
@@ -21,8 +23,11 @@
 //              lo to ~14 bits, used when the caller wants the O_lo residual,
 //              whose purpose is an O accurate to ~fp32); at the end it
 //              normalises O_g and writes O (bf16), with PLO also
-//              O_lo = bf16(O - bf16(O)), and LSE.
-//   warp 8     TMA producer: both Q tiles once, then K_j, V_j through a ring.
+//              O_lo = bf16(O - bf16(O)), and LSE, each thread its own row
+//              straight from registers.
+//   warp 8     TMA producer: per item each group's Q tile (once the previous
+//              item's S MMAs are done with the buffer), then K_j, V_j through
+//              a ring that runs on across items.
 //   warps 9, 10  MMA issuers for groups 0, 1 (warp 9 also owns TMEM).  Two
 //              issuing threads keep the tensor core fed where one thread's
 //              issue rate would not (N = D <= 64 MMAs).  Per key tile j:
