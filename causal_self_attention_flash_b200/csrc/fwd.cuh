@@ -108,7 +108,8 @@ struct FwdCfg {
   static constexpr int THREADS = 352;
 };
 
-// named (hardware) barriers: 1 + g for a group's epilogue
+// named (hardware) barrier for the one-time offset of the two groups
+constexpr uint32_t kBarOffset = 3;
 // barrier indices
 // (KVEMPTY: one per group and stage, index FB_KVEMPTY + 3 * g + stage; the
 // other per-group barriers at base + g)
@@ -506,10 +507,18 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const uint64_t sl2x2 = f2(sl2, sl2);
         const uint64_t negm2 = f2(-m_used, -m_used);
         uint64_t sum2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
+        // Once per CTA, group 1's first exponential phase waits for group
+        // 0's: the two groups then stay out of step, so their exponential
+        // phases overlap less on the ex2 unit.  (Exactly one arrive and one
+        // wait per CTA on this named barrier, both taken only when both
+        // groups have a tile in the first item.)
+        const bool offset = k == 0 && j == 0 && it.n[0] > 0 && it.n[1] > 0;
+        if (offset && g == 1) named_bar_sync(kBarOffset, 256);
         if (j == ng - 1)
           fwd_exp_row<false, PLO>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g));
         else
           fwd_exp_row<true, PLO>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g));
+        if (offset && g == 0) named_bar_arrive(kBarOffset, 256);
         float sa, sb, sc2, sd;
         f2_split(sum2[0], sa, sb);
         f2_split(sum2[1], sc2, sd);
