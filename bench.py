@@ -274,6 +274,88 @@ def run_reference(args, w, index, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def compulsory_bytes(w):
+    """HBM bytes a fwd+bwd step must move: the forward reads Q, K, V and
+    writes O, LSE; the preprocess reads O, dO and writes Delta; the backward
+    reads Q, K, V, dO, LSE, Delta and writes dQ, dK, dV (no L2-served
+    re-reads, no fp32 dQ accumulator traffic)."""
+    t = w.B * w.H * w.T * w.D * 2
+    v = w.B * w.H * w.T * 4
+    return (4 * t + v) + (2 * t + v) + (7 * t + 2 * v)
+
+
+def measure_detail(args, w, sets, olos, step, stream, cattn):
+    n = max(args.steps, 20)
+
+    def timed(fn, count):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(count + 1)]
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for i in range(count):
+            fn(i)
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        return [ev[i].elapsed_time(ev[i + 1]) for i in range(count)]
+
+    def pct(xs, q):
+        ys = sorted(xs)
+        return ys[min(len(ys) - 1, int(q * (len(ys) - 1) + 0.5))]
+
+    per_step = timed(step, n)
+    tf = lambda flops, ms: flops / (ms / 1e3) / 1e12  # noqa: E731
+
+    def fwd_only(i):
+        qd, kd, vd, dod, o, lse, dq, dk, dv, ws = sets[i % N_SETS]
+        if olos[i % N_SETS] is not None:
+            cattn.attn_fwd_ex(qd, kd, vd, w.scale, o=o, lse=lse, o_lo=olos[i % N_SETS],
+                              stream=stream)
+        else:
+            cattn.attn_fwd(qd, kd, vd, w.scale, o=o, lse=lse, stream=stream)
+
+    def bwd_only(i):
+        qd, kd, vd, dod, o, lse, dq, dk, dv, ws = sets[i % N_SETS]
+        cattn.attn_bwd(qd, kd, vd, o, lse, dod, w.scale, dq=dq, dk=dk, dv=dv, workspace=ws,
+                       stream=stream, o_lo=olos[i % N_SETS])
+
+    for i in range(N_SETS):
+        fwd_only(i)
+    fwd_ms = timed(fwd_only, n)
+    bwd_ms = timed(bwd_only, n)
+    one_set = timed(lambda i: step(0), n)
+    med = pct(per_step, 0.5)
+    detail = {
+        "step_ms": {"median": med, "p10": pct(per_step, 0.1), "p90": pct(per_step, 0.9),
+                    "samples": n},
+        "fwd_alone": {"tflops": tf(fwd_flops(w), pct(fwd_ms, 0.5)), "ms_median": pct(fwd_ms, 0.5)},
+        "bwd_alone": {"tflops": tf(2.5 * fwd_flops(w), pct(bwd_ms, 0.5)),
+                      "ms_median": pct(bwd_ms, 0.5),
+                      "includes": "preprocess + main + dQ convert"},
+        "single_input_set": {"tflops": tf(step_flops(w), pct(one_set, 0.5)),
+                             "note": "no rotation: whatever of the step fits stays in L2"},
+        "hbm_compulsory": {"bytes_per_step": compulsory_bytes(w),
+                           "gbs_at_median_step": compulsory_bytes(w) / (med / 1e3) / 1e9},
+    }
+    # context: torch.nn.functional.scaled_dot_product_attention (a library
+    # kernel; run and timed only) on the same inputs and shapes
+    try:
+        qd, kd, vd, dod = (t.detach() for t in sets[0][:4])
+        q_, k_, v_ = (t.clone().requires_grad_(True) for t in (qd, kd, vd))
+
+        def sdpa(i):
+            out = torch.nn.functional.scaled_dot_product_attention(q_, k_, v_, is_causal=True,
+                                                                   scale=w.scale)
+            out.backward(dod)
+
+        for i in range(3):
+            sdpa(i)
+        sd = timed(sdpa, n)
+        detail["context_torch_sdpa"] = {"tflops_fwd_bwd": tf(step_flops(w), pct(sd, 0.5)),
+                                        "ms_median": pct(sd, 0.5)}
+    except Exception as e:  # noqa: BLE001  (context only)
+        detail["context_torch_sdpa"] = {"unavailable": str(e)[:120]}
+    return detail
+
+
 def run_cattn(args, w, index, world, rank, local):
     import causal_self_attention_flash_b200 as cattn
     dev = torch.device("cuda", local)
@@ -359,6 +441,13 @@ def run_cattn(args, w, index, world, rank, local):
     except (OSError, ValueError):
         pass
 
+    # ---- detail (rank 0): step-time spread, forward and backward alone, a
+    # single (unrotated) input set, HBM rate on the compulsory bytes, and
+    # torch's own fused attention on the same inputs as a context row
+    detail = None
+    if rank == 0:
+        detail = measure_detail(args, w, sets, olos, step, stream, cattn)
+
     # ---- end to end: pinned host buffers -> device -> fwd+bwd -> host
     host_in = [t.pin_memory() for t in (q0, k0, v0, do0)]
     host_out = [torch.empty(w.B, w.H, w.T, w.D, dtype=torch.bfloat16).pin_memory()
@@ -425,6 +514,7 @@ def run_cattn(args, w, index, world, rank, local):
             "gpu_launches": sum(c for _, c in ktimes.values()),
             "clocks": clocks,
             "device_status": status,
+            "detail": detail,
         }
         print(json.dumps(line), flush=True)
 
