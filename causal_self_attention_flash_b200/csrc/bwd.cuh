@@ -755,6 +755,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       }
     };
 
+    // kLateDrain (own dQ staging, dQ not aliased): drain dQ(t-1) after the
+    // dS phase of tile t rather than after its P phase, so that dS(t) (and
+    // dK(t), dQ(t) after it) come earlier and the drain fills the wait for
+    // S(t+1).
+    constexpr bool kLateDrain = C::WARP_DQ && !C::ALIAS_DQ;
     float pv[32];
     int t = 0;
     // the previous query tile (its dQ is drained in the next iteration) and
@@ -810,8 +815,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         }
 
         // ---- dQ of the previous query tile (its MMA ran during this P phase)
-        if (t >= 1) drain_dq(t - 1, prev_q0, prev_bh);
-        // ---- the previous item's dK, dV (complete since that drain)
+        // (kLateDrain: after the dS phase instead, see there)
+        if (!kLateDrain && t >= 1) drain_dq(t - 1, prev_q0, prev_bh);
+        // ---- the previous item's dK, dV
         if (i == 0 && prev_kt >= 0) epilogue(prev_kt, prev_bh, t - 1);
 
         // ---- dS phase
@@ -846,6 +852,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // dS (hi, lo) -> shared for the dQ MMA: [2][128 keys][64 queries];
         // query block g is half g/2, chunks 4*(g%2) .. +3 of the row.  (dQ(t-1),
         // which read the previous dS, is complete: drained above.)
+        // the previous dQ MMA, which read the previous dS, must be complete
+        if (kLateDrain && t >= 1) {
+          wait_warp(w, bar(BB_DQFULL), (t - 1) & 1, 31);
+          tc_fence_after();
+        }
         if (t >= 1) staging_free();
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
@@ -858,6 +869,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(BB_DSFULL));
+        // ---- kLateDrain: the previous query tile's dQ, while the next S is
+        // computed (the compute warps would otherwise wait for it)
+        if (kLateDrain && t >= 1) drain_dq(t - 1, prev_q0, prev_bh);
         prev_q0 = (kt + i) * 128;
         prev_bh = bh;
       }
