@@ -237,7 +237,7 @@ struct BwdCfg {
   static constexpr int layout_end(int kvb) {
     return ((kvb * 2 * TILE_BYTES + (QST + DOST) * TILE_BYTES + 32768 + DSL_BYTES +
              QST * 1024 + 1023) / 1024 * 1024) +
-           (WARP_DQ ? 16 * WARP_STAGE : 0) + 32 * 8 + 64;
+           (WARP_DQ ? 16 * WARP_STAGE : 0) + 40 * 8 + 64;
   }
   static constexpr int KVB = layout_end(2) + 1024 <= kMaxDynSmem ? 2 : 1;
   static constexpr int OFF_KV = 0;                             // [KVB][K, V]
@@ -249,7 +249,7 @@ struct BwdCfg {
   static constexpr int OFF_DELTA = OFF_LSE + QST * 512;       // [QST][128] fp32
   static constexpr int OFF_DQW = (OFF_DELTA + QST * 512 + 1023) / 1024 * 1024;
   static constexpr int OFF_BAR = WARP_DQ ? OFF_DQW + 16 * WARP_STAGE : OFF_DELTA + QST * 512;
-  static constexpr int NUM_BARS = 29;
+  static constexpr int NUM_BARS = 33;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_USED = OFF_MISC + 64;
   static constexpr int SMEM_BYTES =
@@ -272,13 +272,13 @@ struct BwdCfg {
 
 // barrier indices (two of each K/V buffer barrier, QST of the Q ring's,
 // DOST (<= 2) of the dO ring's)
-// (room for up to 4 Q stages and 2 dO stages)
+// (room for up to 4 Q stages and 4 dO stages)
 enum : int {
-  BB_KVFULL = 0, BB_KVFREE = 2, BB_QFULL = 4, BB_QEMPTY = 8, BB_DOFULL = 12, BB_DOEMPTY = 14,
-  BB_SFULL = 16, BB_DPFULL = 17, BB_PFULL = 18, BB_DSFULL = 19, BB_DQFULL = 20,
-  BB_DQEMPTY = 21, BB_ACCFREE = 22, BB_PTDONE = 23, BB_DKDONE = 24,
-  BB_DRAIN = 25,  // + issuer 0, 1, 2
-  BB_PFULL2 = 28  // second half of P^T (BB_PFULL is the first)
+  BB_KVFULL = 0, BB_KVFREE = 2, BB_QFULL = 4, BB_QEMPTY = 8, BB_DOFULL = 12, BB_DOEMPTY = 16,
+  BB_SFULL = 20, BB_DPFULL = 21, BB_PFULL = 22, BB_DSFULL = 23, BB_DQFULL = 24,
+  BB_DQEMPTY = 25, BB_ACCFREE = 26, BB_PTDONE = 27, BB_DKDONE = 28,
+  BB_DRAIN = 29,  // + issuer 0, 1, 2
+  BB_PFULL2 = 32  // second half of P^T (BB_PFULL is the first)
 };
 
 // Work items: key tiles (kt, bh), numbered longest first (u = 0 ..
@@ -298,7 +298,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
            const __grid_constant__ CUtensorMap tmDQacc, const BwdParams p) {
   using C = BwdCfg<D, SLO>;
   static_assert(BB_PFULL2 + 1 <= C::NUM_BARS, "barrier count");
-  static_assert(C::QST <= 4 && C::DOST <= 2, "barrier map");
+  static_assert(C::QST <= 4 && C::DOST <= 4, "barrier map");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = aligned_smem(smem_raw, C::SMEM_USED);
   if (smem == nullptr) return;  // uniform over the CTA: nothing touched yet
