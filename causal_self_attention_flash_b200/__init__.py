@@ -7,7 +7,10 @@ and raise CattnError on a non-zero status.  Nothing here computes: torch
 only provides device memory and streams.
 
 Layout: q, k, v, o, do, dq, dk, dv are bf16 (B, H, T, D) contiguous; lse
-and delta are fp32 (B, H, T).
+and delta are fp32 (B, H, T).  The _strided calls take (B, H, T, D) views
+with any strides whose last one is 1 (e.g. the parts of a fused (B, T, 3C)
+projection, see split_qkv), and CausalAttentionQKV goes from that fused
+projection straight to a (B, T, C) output with no transposes.
 """
 
 from __future__ import annotations
@@ -18,7 +21,7 @@ import torch
 
 from ._binding import (ERR_CUDA, ERR_INVALID_ARG, ERR_TIMEOUT, ERR_TOO_LARGE,
                        ERR_UNSUPPORTED, LIB, LIB_PATH, NOALLOC_SCRATCH_BYTES, OK,
-                       CattnError)
+                       CattnError, Layout)
 
 __all__ = [
     "attn_fwd", "attn_bwd", "attn_fwd_ex", "attn_bwd_ex", "attn_bwd_preprocess",
@@ -29,6 +32,7 @@ __all__ = [
     "CausalAttention", "CattnError", "LIB", "LIB_PATH",
     "OK", "ERR_INVALID_ARG", "ERR_UNSUPPORTED", "ERR_CUDA", "ERR_TIMEOUT", "ERR_TOO_LARGE",
     "attn_bwd_noalloc", "NOALLOC_SCRATCH_BYTES",
+    "attn_fwd_strided", "attn_bwd_strided", "split_qkv", "CausalAttentionQKV", "Layout",
 ]
 
 
@@ -209,6 +213,123 @@ def cattn_status_string(st: int) -> str:
 
 def cattn_version() -> int:
     return int(LIB.cattn_version())
+
+
+def _layout(t, dtype, what):
+    """cattn_layout of a (B, H, T, D) view whose last stride is 1."""
+    if t.dim() != 4 or t.stride(3) != 1:
+        raise ValueError(f"{what}: expected a (B, H, T, D) view with unit last stride")
+    if t.dtype != dtype or not t.is_cuda:
+        raise ValueError(f"{what}: expected a {dtype} CUDA tensor")
+    return Layout(t.stride(0), t.stride(1), t.stride(2))
+
+
+def split_qkv(qkv, n_head):
+    """(q, k, v) as (B, H, T, D) views into a fused (B, T, 3C) projection,
+    as the pages' c_attn produces it.  View arithmetic only: no copies."""
+    B, T, C3 = qkv.shape
+    C = C3 // 3
+    D = C // n_head
+    parts = qkv.split(C, dim=2)
+    return tuple(x.view(B, T, n_head, D).transpose(1, 2) for x in parts)
+
+
+def attn_fwd_strided(q, k, v, scale=None, o=None, lse=None, o_lo=None, stream=None):
+    """attn_fwd_ex on strided (B, H, T, D) views.  o (and o_lo) may be views
+    too, e.g. of a (B, T, C) buffer (o_lo must share o's strides); if not
+    given they are allocated contiguous.  Returns (o, lse, o_lo)."""
+    B, H, T, D = _shape(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    lq, lk, lv = (_layout(t, torch.bfloat16, n) for t, n in ((q, "q"), (k, "k"), (v, "v")))
+    if o is None:
+        o = torch.empty((B, H, T, D), dtype=torch.bfloat16, device=q.device)
+    lo = _layout(o, torch.bfloat16, "o")
+    if o_lo is not None and (o_lo.stride() != o.stride() or o_lo.dtype != torch.bfloat16):
+        raise ValueError("o_lo must be a bf16 view with o's strides")
+    lse = _want(lse, q, torch.float32, (B, H, T))
+    st = LIB.attn_fwd_strided(q.data_ptr(), lq, k.data_ptr(), lk, v.data_ptr(), lv, float(scale),
+                              B, H, T, D, o.data_ptr(), lo, lse.data_ptr(),
+                              o_lo.data_ptr() if o_lo is not None else None, _stream(stream))
+    _check("attn_fwd_strided", st)
+    return o, lse, o_lo
+
+
+def attn_bwd_strided(q, k, v, o, lse, do, scale=None, dq=None, dk=None, dv=None,
+                     workspace=None, stream=None, o_lo=None, grad_dtype=torch.bfloat16):
+    """attn_bwd_ex on strided (B, H, T, D) views of q, k, v, o (o_lo with o's
+    strides), do and the outputs dq, dk, dv (allocated contiguous if not
+    given; e.g. the three parts of one (B, T, 3C) gradient buffer)."""
+    B, H, T, D = _shape(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous fp32 (B, H, T)")
+    if grad_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("grad_dtype must be torch.bfloat16 or torch.float32")
+    ins = [_layout(t, torch.bfloat16, n)
+           for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do"))]
+    if o_lo is not None and (o_lo.stride() != o.stride() or o_lo.dtype != torch.bfloat16):
+        raise ValueError("o_lo must be a bf16 view with o's strides")
+    outs = []
+    for t in (dq, dk, dv):
+        outs.append(t if t is not None else
+                    torch.empty((B, H, T, D), dtype=grad_dtype, device=q.device))
+    dq, dk, dv = outs
+    louts = [_layout(t, grad_dtype, n) for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv"))]
+    need = attn_bwd_workspace_bytes(B, H, T, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = LIB.attn_bwd_strided(q.data_ptr(), ins[0], k.data_ptr(), ins[1], v.data_ptr(), ins[2],
+                              o.data_ptr(), ins[3],
+                              o_lo.data_ptr() if o_lo is not None else None, lse.data_ptr(),
+                              do.data_ptr(), ins[4], float(scale), B, H, T, D,
+                              dq.data_ptr(), louts[0], dk.data_ptr(), louts[1],
+                              dv.data_ptr(), louts[2],
+                              1 if grad_dtype == torch.float32 else 0,
+                              workspace.data_ptr(), workspace.numel(), _stream(stream))
+    _check("attn_bwd_strided", st)
+    return dq, dk, dv
+
+
+class CausalAttentionQKV(torch.autograd.Function):
+    """autograd wrapper from the fused projection to the merged output:
+    qkv (B, T, 3C) bf16 -> y (B, T, C) bf16 = the heads of causal attention
+    side by side, as the pages' CausalSelfAttention glues them together
+    before c_proj.  Forward and backward read and write those layouts in
+    place (attn_fwd_strided / attn_bwd_strided); dqkv comes back as one
+    (B, T, 3C) tensor."""
+
+    @staticmethod
+    def forward(ctx, qkv, n_head, scale=None):
+        B, T, C3 = qkv.shape
+        C = C3 // 3
+        D = C // n_head
+        q, k, v = split_qkv(qkv, n_head)
+        y = torch.empty((B, T, C), dtype=torch.bfloat16, device=qkv.device)
+        y_lo = torch.empty_like(y)
+        o = y.view(B, T, n_head, D).transpose(1, 2)
+        o_lo = y_lo.view(B, T, n_head, D).transpose(1, 2)
+        _, lse, _ = attn_fwd_strided(q, k, v, scale, o=o, o_lo=o_lo)
+        ctx.save_for_backward(qkv, y, y_lo, lse)
+        ctx.n_head, ctx.scale = n_head, scale
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        qkv, y, y_lo, lse = ctx.saved_tensors
+        n_head = ctx.n_head
+        B, T, C = y.shape
+        D = C // n_head
+        q, k, v = split_qkv(qkv, n_head)
+        o = y.view(B, T, n_head, D).transpose(1, 2)
+        o_lo = y_lo.view(B, T, n_head, D).transpose(1, 2)
+        dy = dy.contiguous()
+        do = dy.view(B, T, n_head, D).transpose(1, 2)
+        dqkv = torch.empty_like(qkv)
+        dq, dk, dv = split_qkv(dqkv, n_head)
+        attn_bwd_strided(q, k, v, o, lse, do, ctx.scale, dq=dq, dk=dk, dv=dv, o_lo=o_lo)
+        return dqkv, None, None
 
 
 class CausalAttention(torch.autograd.Function):

@@ -24,9 +24,17 @@ STATUS_NAMES = {OK: "CATTN_OK", ERR_INVALID_ARG: "CATTN_ERR_INVALID_ARG",
                 ERR_UNSUPPORTED: "CATTN_ERR_UNSUPPORTED", ERR_CUDA: "CATTN_ERR_CUDA",
                 ERR_TIMEOUT: "CATTN_ERR_TIMEOUT", ERR_TOO_LARGE: "CATTN_ERR_TOO_LARGE"}
 
+
+
+class Layout(ctypes.Structure):
+    """cattn_layout: element strides (b, h, t) of a (B, H, T, D) tensor."""
+    _fields_ = [("b", ctypes.c_longlong), ("h", ctypes.c_longlong), ("t", ctypes.c_longlong)]
+
+
 # name -> (restype, argtypes), mirroring include/cattn.h
 _vp, _i, _f, _sz, _u32 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_float,
                           ctypes.c_size_t, ctypes.c_uint32)
+_L = Layout
 SIGNATURES = {
     "attn_fwd": (_i, [_vp, _vp, _vp, _f, _i, _i, _i, _i, _vp, _vp, _vp]),
     "attn_fwd_ex": (_i, [_vp, _vp, _vp, _f, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
@@ -38,6 +46,10 @@ SIGNATURES = {
                          _vp, _vp, _vp, _i, _vp, _sz, _vp]),
     "attn_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _f, _i, _i, _i, _i,
                               _vp, _vp, _vp, _vp]),
+    "attn_fwd_strided": (_i, [_vp, _L, _vp, _L, _vp, _L, _f, _i, _i, _i, _i, _vp, _L, _vp, _vp,
+                              _vp]),
+    "attn_bwd_strided": (_i, [_vp, _L, _vp, _L, _vp, _L, _vp, _L, _vp, _vp, _vp, _L, _f,
+                              _i, _i, _i, _i, _vp, _L, _vp, _L, _vp, _L, _i, _vp, _sz, _vp]),
     "cattn_get_device_status": (_i, [_i, _vp]),
     "cattn_set_wait_timeout_us": (None, [_u32]),
     "cattn_selftest_wait_timeout": (_i, [_u32, _vp]),

@@ -136,9 +136,50 @@ cattn_status make_tmap(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, 
   return r == CUDA_SUCCESS ? CATTN_OK : cuda_fail(10000 + static_cast<int>(r));
 }
 
-cattn_status make_bf16_map(CUtensorMap* m, const void* ptr, int D, int T, long long BH) {
+cattn_layout contiguous_layout(int H, int T, int D) {
+  cattn_layout l;
+  l.b = static_cast<long long>(H) * T * D;
+  l.h = static_cast<long long>(T) * D;
+  l.t = D;
+  return l;
+}
+
+bool is_contiguous(cattn_layout l, int H, int T, int D) {
+  const cattn_layout c = contiguous_layout(H, T, D);
+  return l.b == c.b && l.h == c.h && l.t == c.t;
+}
+
+// Element strides the kernels accept: positive multiples of 8 (rows start
+// on 16-byte boundaries, as the TMA and the 16-byte stores need), each below
+// 2^38 so that byte offsets stay far inside the TMA's 2^40 stride limit.
+bool layout_ok(cattn_layout l) {
+  const long long lim = 1LL << 38;
+  return l.b > 0 && l.h > 0 && l.t > 0 && l.b % 8 == 0 && l.h % 8 == 0 && l.t % 8 == 0 &&
+         l.b < lim && l.h < lim && l.t < lim;
+}
+
+// 4-D tensor map {x = d, y = t, z = h, w = b} over a bf16 (B, H, T, D)
+// tensor with element strides lay (the d stride is 1); boxes of
+// [128 rows][min(D, 64) columns], swizzled by the box's row bytes.
+cattn_status make_bf16_map(CUtensorMap* m, const void* ptr, int D, int T, int H, int B,
+                           cattn_layout lay) {
   const int cb = D < 64 ? D : 64;
-  return make_tmap(m, ptr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, T, BH, cb, 128);
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(T),
+                              static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(lay.t) * 2,
+                                 static_cast<cuuint64_t>(lay.h) * 2,
+                                 static_cast<cuuint64_t>(lay.b) * 2};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(cb), 128, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const int row_bytes = cb * 2;
+  CUtensorMapSwizzle sw = row_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                          : row_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                            : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CATTN_OK : cuda_fail(10000 + static_cast<int>(r));
 }
 
 cattn_status launch_status() {
@@ -211,20 +252,26 @@ struct LaunchTimer {
 unsigned d_index(int D) { return D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3; }
 
 template <int D, bool PLO>
-cattn_status fwd_impl(int dev, const void* q, const void* k, const void* v, float scale, int BH,
-                      int T, void* o, float* lse, void* o_lo, cudaStream_t s) {
+cattn_status fwd_impl(int dev, const void* q, cattn_layout lq, const void* k, cattn_layout lk,
+                      const void* v, cattn_layout lv, float scale, int B, int H, int T, void* o,
+                      cattn_layout lo, float* lse, void* o_lo, cudaStream_t s) {
+  const int BH = B * H;
   using C = FwdCfg<D, PLO>;
   clear_stale_error();
   cattn_status st = ensure_smem(dev, 0 + 2 * d_index(D) + PLO, fwd_kernel<D, PLO>, C::SMEM_BYTES);
   if (st != CATTN_OK) return st;
   CUtensorMap mq, mk, mv;
-  if ((st = make_bf16_map(&mq, q, D, T, BH)) != CATTN_OK) return st;
-  if ((st = make_bf16_map(&mk, k, D, T, BH)) != CATTN_OK) return st;
-  if ((st = make_bf16_map(&mv, v, D, T, BH)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mq, q, D, T, H, B, lq)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mk, k, D, T, H, B, lk)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mv, v, D, T, H, B, lv)) != CATTN_OK) return st;
   FwdParams p;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.o_lo = static_cast<__nv_bfloat16*>(o_lo);
+  p.o_sb = lo.b;
+  p.o_sh = lo.h;
+  p.o_st = lo.t;
   p.lse = lse;
+  p.H = H;
   p.T = T;
   p.BH = BH;
   p.n_qtiles = (T + 127) / 128;
@@ -262,14 +309,22 @@ WsLayout ws_layout(long long BH, int T, int D) {
 }
 
 template <int D>
-cattn_status pre_impl(const void* o, const void* o_lo, const void* dout, const float* lse,
-                      float* delta, float* lse2, float4* zero, size_t zero_n4, long long BH,
-                      int T, int row_stride, cudaStream_t s) {
+cattn_status pre_impl(const void* o, cattn_layout lo, const void* o_lo, const void* dout,
+                      cattn_layout ldo, const float* lse, float* delta, float* lse2, float4* zero,
+                      size_t zero_n4, int B, int H, int T, int row_stride, cudaStream_t s) {
   clear_stale_error();
+  const long long BH = static_cast<long long>(B) * H;
   PreParams p;
   p.o = static_cast<const __nv_bfloat16*>(o);
   p.o_lo = static_cast<const __nv_bfloat16*>(o_lo);
   p.dout = static_cast<const __nv_bfloat16*>(dout);
+  p.o_sb = lo.b;
+  p.o_sh = lo.h;
+  p.o_st = lo.t;
+  p.do_sb = ldo.b;
+  p.do_sh = ldo.h;
+  p.do_st = ldo.t;
+  p.H = H;
   p.lse = lse;
   p.delta = delta;
   p.lse2 = lse2;
@@ -288,12 +343,23 @@ cattn_status pre_impl(const void* o, const void* o_lo, const void* dout, const f
   return launch_status();
 }
 
+// The strides of one backward call (element strides of each tensor).
+struct BwdLayouts {
+  cattn_layout q, k, v, o, dout, dq, dk, dv;
+};
+
+BwdLayouts contiguous_bwd_layouts(int H, int T, int D) {
+  const cattn_layout c = contiguous_layout(H, T, D);
+  return BwdLayouts{c, c, c, c, c, c, c, c};
+}
+
 template <int D, bool SLO>
 cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, const void* o,
-                      const void* o_lo, const float* lse, const void* dout, float scale, int BH,
-                      int T, void* dq, void* dk, void* dv, bool grad_f32, void* ws,
-                      cudaStream_t s) {
+                      const void* o_lo, const float* lse, const void* dout, float scale, int B,
+                      int H, int T, void* dq, void* dk, void* dv, const BwdLayouts& ly,
+                      bool grad_f32, void* ws, cudaStream_t s) {
   using C = BwdCfg<D, SLO>;
+  const int BH = B * H;
   clear_stale_error();
   cattn_status st = ensure_smem(dev, 8 + 2 * d_index(D) + SLO, bwd_kernel<D, SLO>, C::SMEM_BYTES);
   if (st != CATTN_OK) return st;
@@ -305,17 +371,17 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   const size_t n_dq = static_cast<size_t>(BH) * T * D;
 
   CUtensorMap mq, mk, mv, mdo, mdq;
-  if ((st = make_bf16_map(&mq, q, D, T, BH)) != CATTN_OK) return st;
-  if ((st = make_bf16_map(&mk, k, D, T, BH)) != CATTN_OK) return st;
-  if ((st = make_bf16_map(&mv, v, D, T, BH)) != CATTN_OK) return st;
-  if ((st = make_bf16_map(&mdo, dout, D, T, BH)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mq, q, D, T, H, B, ly.q)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mk, k, D, T, H, B, ly.k)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mv, v, D, T, H, B, ly.v)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mdo, dout, D, T, H, B, ly.dout)) != CATTN_OK) return st;
   if ((st = make_tmap(&mdq, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, T, BH,
                       C::WARP_DQ ? D / 4 : C::CBQ, C::WARP_DQ ? 32 : 128)) !=
       CATTN_OK)
     return st;
 
-  st = pre_impl<D>(o, o_lo, dout, lse, delta, lse2, reinterpret_cast<float4*>(dq_acc), n_dq / 4, BH, T,
-                   L.T_pad, s);
+  st = pre_impl<D>(o, ly.o, o_lo, dout, ly.dout, lse, delta, lse2,
+                   reinterpret_cast<float4*>(dq_acc), n_dq / 4, B, H, T, L.T_pad, s);
   if (st != CATTN_OK) return st;
 
   BwdParams p;
@@ -325,6 +391,13 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   p.dv_f32 = grad_f32 ? static_cast<float*>(dv) : nullptr;
   p.dk_bf16 = grad_f32 ? nullptr : static_cast<__nv_bfloat16*>(dk);
   p.dv_bf16 = grad_f32 ? nullptr : static_cast<__nv_bfloat16*>(dv);
+  p.dk_sb = ly.dk.b;
+  p.dk_sh = ly.dk.h;
+  p.dk_st = ly.dk.t;
+  p.dv_sb = ly.dv.b;
+  p.dv_sh = ly.dv.h;
+  p.dv_st = ly.dv.t;
+  p.H = H;
   p.BH = BH;
   p.T = T;
   p.T_pad = L.T_pad;
@@ -343,7 +416,18 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   if ((st = launch_status()) != CATTN_OK) return st;
   {
     LaunchTimer t(K_DQ_CONVERT, s);
-    if (grad_f32)
+    if (!is_contiguous(ly.dq, H, T, D)) {
+      const long long n8 = static_cast<long long>(n_dq / 8);
+      const int g = grid_for(static_cast<size_t>(n8), 256);
+      if (grad_f32)
+        dq_convert_strided_kernel<D, true><<<g, 256, 0, s>>>(
+            reinterpret_cast<const float4*>(dq_acc), dq, H, T, n8, ly.dq.b, ly.dq.h, ly.dq.t,
+            scale);
+      else
+        dq_convert_strided_kernel<D, false><<<g, 256, 0, s>>>(
+            reinterpret_cast<const float4*>(dq_acc), dq, H, T, n8, ly.dq.b, ly.dq.h, ly.dq.t,
+            scale);
+    } else if (grad_f32)
       dq_convert_f32_kernel<<<grid_for(n_dq / 4, 256), 256, 0, s>>>(
           reinterpret_cast<const float4*>(dq_acc), static_cast<float4*>(dq), n_dq / 4, scale);
     else
@@ -356,12 +440,12 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
 template <int D>
 cattn_status bwd_dispatch(bool slo, int dev, const void* q, const void* k, const void* v,
                           const void* o, const void* o_lo, const float* lse, const void* dout,
-                          float scale, int BH, int T, void* dq, void* dk, void* dv, bool f32,
-                          void* ws, cudaStream_t s) {
-  return slo ? bwd_impl<D, true>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, f32,
-                                 ws, s)
-             : bwd_impl<D, false>(dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv,
-                                  f32, ws, s);
+                          float scale, int B, int H, int T, void* dq, void* dk, void* dv,
+                          const BwdLayouts& ly, bool f32, void* ws, cudaStream_t s) {
+  return slo ? bwd_impl<D, true>(dev, q, k, v, o, o_lo, lse, dout, scale, B, H, T, dq, dk, dv, ly,
+                                 f32, ws, s)
+             : bwd_impl<D, false>(dev, q, k, v, o, o_lo, lse, dout, scale, B, H, T, dq, dk, dv,
+                                  ly, f32, ws, s);
 }
 
 // ---------------------------------------------------------- hang-guard test
@@ -389,8 +473,10 @@ using namespace cattn;
 
 extern "C" {
 
-cattn_status attn_fwd_ex(const void* q, const void* k, const void* v, float scale, int B, int H,
-                         int T, int D, void* o, float* lse, void* o_lo, void* stream) {
+cattn_status attn_fwd_strided(const void* q, cattn_layout lq, const void* k, cattn_layout lk,
+                              const void* v, cattn_layout lv, float scale, int B, int H, int T,
+                              int D, void* o, cattn_layout lo, float* lse, void* o_lo,
+                              void* stream) {
   cattn_status st = check_shape(B, H, T, D);
   if (st != CATTN_OK) return st;
   if (!(scale > 0.f) || !isfinite(scale)) return CATTN_ERR_INVALID_ARG;
@@ -399,25 +485,28 @@ cattn_status attn_fwd_ex(const void* q, const void* k, const void* v, float scal
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
       !aligned(lse, 4) || !aligned(o_lo, 16))
     return CATTN_ERR_INVALID_ARG;
+  if (!layout_ok(lq) || !layout_ok(lk) || !layout_ok(lv) || !layout_ok(lo))
+    return CATTN_ERR_INVALID_ARG;
   int dev;
   if ((st = check_device(&dev)) != CATTN_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int BH = B * H;
+#define CATTN_FWD(DD)                                                                         \
+  return o_lo ? fwd_impl<DD, true>(dev, q, lq, k, lk, v, lv, scale, B, H, T, o, lo, lse, o_lo, s) \
+              : fwd_impl<DD, false>(dev, q, lq, k, lk, v, lv, scale, B, H, T, o, lo, lse, o_lo, s)
   switch (D) {
-    case 16:
-      return o_lo ? fwd_impl<16, true>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s)
-                  : fwd_impl<16, false>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s);
-    case 32:
-      return o_lo ? fwd_impl<32, true>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s)
-                  : fwd_impl<32, false>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s);
-    case 64:
-      return o_lo ? fwd_impl<64, true>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s)
-                  : fwd_impl<64, false>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s);
-    case 128:
-      return o_lo ? fwd_impl<128, true>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s)
-                  : fwd_impl<128, false>(dev, q, k, v, scale, BH, T, o, lse, o_lo, s);
+    case 16: CATTN_FWD(16);
+    case 32: CATTN_FWD(32);
+    case 64: CATTN_FWD(64);
+    case 128: CATTN_FWD(128);
   }
+#undef CATTN_FWD
   return CATTN_ERR_UNSUPPORTED;
+}
+
+cattn_status attn_fwd_ex(const void* q, const void* k, const void* v, float scale, int B, int H,
+                         int T, int D, void* o, float* lse, void* o_lo, void* stream) {
+  const cattn_layout c = contiguous_layout(H, T, D);
+  return attn_fwd_strided(q, c, k, c, v, c, scale, B, H, T, D, o, c, lse, o_lo, stream);
 }
 
 cattn_status attn_fwd(const void* q, const void* k, const void* v, float scale, int B, int H,
@@ -441,20 +530,23 @@ cattn_status attn_bwd_preprocess(const void* o, const void* dout, int B, int H, 
   int dev;
   if ((st = check_device(&dev)) != CATTN_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const long long BH = static_cast<long long>(B) * H;
+  const cattn_layout c = contiguous_layout(H, T, D);
   switch (D) {
-    case 16: return pre_impl<16>(o, nullptr, dout, nullptr, delta, nullptr, nullptr, 0, BH, T, T, s);
-    case 32: return pre_impl<32>(o, nullptr, dout, nullptr, delta, nullptr, nullptr, 0, BH, T, T, s);
-    case 64: return pre_impl<64>(o, nullptr, dout, nullptr, delta, nullptr, nullptr, 0, BH, T, T, s);
-    case 128: return pre_impl<128>(o, nullptr, dout, nullptr, delta, nullptr, nullptr, 0, BH, T, T, s);
+    case 16: return pre_impl<16>(o, c, nullptr, dout, c, nullptr, delta, nullptr, nullptr, 0, B, H, T, T, s);
+    case 32: return pre_impl<32>(o, c, nullptr, dout, c, nullptr, delta, nullptr, nullptr, 0, B, H, T, T, s);
+    case 64: return pre_impl<64>(o, c, nullptr, dout, c, nullptr, delta, nullptr, nullptr, 0, B, H, T, T, s);
+    case 128: return pre_impl<128>(o, c, nullptr, dout, c, nullptr, delta, nullptr, nullptr, 0, B, H, T, T, s);
   }
   return CATTN_ERR_UNSUPPORTED;
 }
 
-cattn_status attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
-                         const void* o_lo, const float* lse, const void* dout, float scale, int B,
-                         int H, int T, int D, void* dq, void* dk, void* dv, int grad_dtype,
-                         void* workspace, size_t workspace_bytes, void* stream) {
+cattn_status attn_bwd_strided(const void* q, cattn_layout lq, const void* k, cattn_layout lk,
+                              const void* v, cattn_layout lv, const void* o, cattn_layout lo,
+                              const void* o_lo, const float* lse, const void* dout,
+                              cattn_layout ldo, float scale, int B, int H, int T, int D, void* dq,
+                              cattn_layout ldq, void* dk, cattn_layout ldk, void* dv,
+                              cattn_layout ldv, int grad_dtype, void* workspace,
+                              size_t workspace_bytes, void* stream) {
   cattn_status st = check_shape(B, H, T, D);
   if (st != CATTN_OK) return st;
   if (!(scale > 0.f) || !isfinite(scale)) return CATTN_ERR_INVALID_ARG;
@@ -465,6 +557,9 @@ cattn_status attn_bwd_ex(const void* q, const void* k, const void* v, const void
       !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
       !aligned(lse, 4) || !aligned(workspace, 256) || !aligned(o_lo, 16))
     return CATTN_ERR_INVALID_ARG;
+  if (!layout_ok(lq) || !layout_ok(lk) || !layout_ok(lv) || !layout_ok(lo) || !layout_ok(ldo) ||
+      !layout_ok(ldq) || !layout_ok(ldk) || !layout_ok(ldv))
+    return CATTN_ERR_INVALID_ARG;
   const int BH = B * H;
   if (workspace_bytes < ws_layout(BH, T, D).total) return CATTN_ERR_INVALID_ARG;
   if (grad_dtype != CATTN_DTYPE_BF16 && grad_dtype != CATTN_DTYPE_F32)
@@ -473,15 +568,25 @@ cattn_status attn_bwd_ex(const void* q, const void* k, const void* v, const void
   int dev;
   if ((st = check_device(&dev)) != CATTN_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const BwdLayouts ly{lq, lk, lv, lo, ldo, ldq, ldk, ldv};
   // dS as a hi/lo pair when the caller asks for gradients accurate to ~fp32
   const bool slo = o_lo != nullptr || f32;
   switch (D) {
-    case 16: return bwd_dispatch<16>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, f32, workspace, s);
-    case 32: return bwd_dispatch<32>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, f32, workspace, s);
-    case 64: return bwd_dispatch<64>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, f32, workspace, s);
-    case 128: return bwd_dispatch<128>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, BH, T, dq, dk, dv, f32, workspace, s);
+    case 16: return bwd_dispatch<16>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, B, H, T, dq, dk, dv, ly, f32, workspace, s);
+    case 32: return bwd_dispatch<32>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, B, H, T, dq, dk, dv, ly, f32, workspace, s);
+    case 64: return bwd_dispatch<64>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, B, H, T, dq, dk, dv, ly, f32, workspace, s);
+    case 128: return bwd_dispatch<128>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, B, H, T, dq, dk, dv, ly, f32, workspace, s);
   }
   return CATTN_ERR_UNSUPPORTED;
+}
+
+cattn_status attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
+                         const void* o_lo, const float* lse, const void* dout, float scale, int B,
+                         int H, int T, int D, void* dq, void* dk, void* dv, int grad_dtype,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  const cattn_layout c = contiguous_layout(H, T, D);
+  return attn_bwd_strided(q, c, k, c, v, c, o, c, o_lo, lse, dout, c, scale, B, H, T, D, dq, c,
+                          dk, c, dv, c, grad_dtype, workspace, workspace_bytes, stream);
 }
 
 cattn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
@@ -527,19 +632,20 @@ cattn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the backward clears what must start at zero (the dQ accumulator) and
   // overwrites the rest on every call
+  const BwdLayouts ly = contiguous_bwd_layouts(H, T, D);
   switch (D) {
     case 16:
-      return bwd_impl<16, false>(dev, q, k, v, o, nullptr, lse, dout, scale, BH, T, dq, dk, dv, false,
-                          scratch, s);
+      return bwd_impl<16, false>(dev, q, k, v, o, nullptr, lse, dout, scale, B, H, T, dq, dk, dv, ly,
+                                 false, scratch, s);
     case 32:
-      return bwd_impl<32, false>(dev, q, k, v, o, nullptr, lse, dout, scale, BH, T, dq, dk, dv, false,
-                          scratch, s);
+      return bwd_impl<32, false>(dev, q, k, v, o, nullptr, lse, dout, scale, B, H, T, dq, dk, dv, ly,
+                                 false, scratch, s);
     case 64:
-      return bwd_impl<64, false>(dev, q, k, v, o, nullptr, lse, dout, scale, BH, T, dq, dk, dv, false,
-                          scratch, s);
+      return bwd_impl<64, false>(dev, q, k, v, o, nullptr, lse, dout, scale, B, H, T, dq, dk, dv, ly,
+                                 false, scratch, s);
     case 128:
-      return bwd_impl<128, false>(dev, q, k, v, o, nullptr, lse, dout, scale, BH, T, dq, dk, dv, false,
-                           scratch, s);
+      return bwd_impl<128, false>(dev, q, k, v, o, nullptr, lse, dout, scale, B, H, T, dq, dk, dv, ly,
+                                 false, scratch, s);
   }
   return CATTN_ERR_UNSUPPORTED;
 }

@@ -38,9 +38,11 @@ namespace cattn {
 // ---------------------------------------------------------------------------
 
 struct PreParams {
-  const __nv_bfloat16* o;
-  const __nv_bfloat16* o_lo;  // may be null
-  const __nv_bfloat16* dout;
+  const __nv_bfloat16* o;     // (B, H, T, D), element strides o_sb, o_sh, o_st
+  const __nv_bfloat16* o_lo;  // may be null; the strides of o
+  const __nv_bfloat16* dout;  // element strides do_sb, do_sh, do_st
+  long long o_sb, o_sh, o_st, do_sb, do_sh, do_st;
+  int H;
   const float* lse;      // may be null (no lse2 output)
   float* delta;          // (BH, row_stride)
   float* lse2;           // (BH, row_stride) or null
@@ -89,9 +91,11 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
       valid[u] = pr[u] < p.n_rows && t[u] < p.T;
       a[u] = bb[u] = c[u] = make_uint4(0u, 0u, 0u, 0u);
       if (valid[u]) {
-        const size_t off = (static_cast<size_t>(bh[u]) * p.T + t[u]) * D + sub * 8;
+        const long long b_ = bh[u] / p.H, h_ = bh[u] - b_ * p.H;
+        const long long off = b_ * p.o_sb + h_ * p.o_sh + t[u] * p.o_st + sub * 8;
+        const long long doff = b_ * p.do_sb + h_ * p.do_sh + t[u] * p.do_st + sub * 8;
         a[u] = *reinterpret_cast<const uint4*>(p.o + off);
-        bb[u] = *reinterpret_cast<const uint4*>(p.dout + off);
+        bb[u] = *reinterpret_cast<const uint4*>(p.dout + doff);
         if (p.o_lo != nullptr) c[u] = *reinterpret_cast<const uint4*>(p.o_lo + off);
       }
     }
@@ -158,6 +162,41 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float4* __restric
   }
 }
 
+// dQ into an output with any (b, h, t) element strides: one thread per 8
+// elements, the accumulator (B*H, T, D) read contiguously.
+template <int D, bool F32>
+__global__ void __launch_bounds__(256) dq_convert_strided_kernel(const float4* __restrict__ acc,
+                                                                 void* __restrict__ dq, int H,
+                                                                 int T, long long n8,
+                                                                 long long sb, long long sh,
+                                                                 long long st, float scale) {
+  constexpr int C8 = D / 8;  // 8-element chunks per row
+  const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long nth = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = tid; i < n8; i += nth) {
+    const long long row = i / C8;
+    const int c8 = static_cast<int>(i - row * C8);
+    const long long bh = row / T;
+    const long long t = row - bh * T;
+    const long long b = bh / H, h = bh - b * H;
+    const long long off = b * sb + h * sh + t * st + c8 * 8;
+    const float4 a = acc[2 * i];
+    const float4 c = acc[2 * i + 1];
+    if constexpr (F32) {
+      float4* out = reinterpret_cast<float4*>(static_cast<float*>(dq) + off);
+      out[0] = make_float4(a.x * scale, a.y * scale, a.z * scale, a.w * scale);
+      out[1] = make_float4(c.x * scale, c.y * scale, c.z * scale, c.w * scale);
+    } else {
+      uint4 r;
+      r.x = pack_bf16(a.x * scale, a.y * scale);
+      r.y = pack_bf16(a.z * scale, a.w * scale);
+      r.z = pack_bf16(c.x * scale, c.y * scale);
+      r.w = pack_bf16(c.z * scale, c.w * scale);
+      reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dq) + off)[0] = r;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Main backward kernel
 // ---------------------------------------------------------------------------
@@ -198,6 +237,9 @@ struct BwdParams {
   float* dv_f32;
   __nv_bfloat16* dk_bf16;  // bf16 gradient outputs, used when dk_f32 is null
   __nv_bfloat16* dv_bf16;
+  // element strides (b, h, t) of the dK and dV outputs (either type)
+  long long dk_sb, dk_sh, dk_st, dv_sb, dv_sh, dv_st;
+  int H;
   int T;
   int T_pad;
   int n_tiles;
@@ -375,7 +417,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const uint32_t sQ = sbase + C::OFF_Q + qs * C::TILE_BYTES;
         mbar_arrive_expect_tx(bar(BB_QFULL + qs), C::TILE_BYTES + 1024);
         for (int bb = 0; bb < C::NCB; ++bb)
-          tma_load_3d(sQ + bb * C::BLOCK_BYTES, &tmQ, bar(BB_QFULL + qs), bb * C::CB, qi * 128, bh);
+          tma_load_4d(sQ + bb * C::BLOCK_BYTES, &tmQ, bar(BB_QFULL + qs), bb * C::CB, qi * 128,
+                      bh % p.H, bh / p.H);
         bulk_load(sbase + C::OFF_LSE + qs * 512, p.lse2 + vec, 512, bar(BB_QFULL + qs));
         bulk_load(sbase + C::OFF_DELTA + qs * 512, p.delta + vec, 512, bar(BB_QFULL + qs));
         ++tq;
@@ -387,8 +430,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const uint32_t sDO = sbase + C::OFF_DO + ds * C::TILE_BYTES;
         mbar_arrive_expect_tx(bar(BB_DOFULL + ds), C::TILE_BYTES);
         for (int bb = 0; bb < C::NCB; ++bb)
-          tma_load_3d(sDO + bb * C::BLOCK_BYTES, &tmDO, bar(BB_DOFULL + ds), bb * C::CB, qi * 128,
-                      bh);
+          tma_load_4d(sDO + bb * C::BLOCK_BYTES, &tmDO, bar(BB_DOFULL + ds), bb * C::CB, qi * 128,
+                      bh % p.H, bh / p.H);
         ++tdo;
       };
       for (int k = 0;; ++k) {
@@ -403,10 +446,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         if (*abort_flag) break;
         mbar_arrive_expect_tx(bar(BB_KVFULL + kvb), 2 * C::TILE_BYTES);
         for (int bb = 0; bb < C::NCB; ++bb) {
-          tma_load_3d(sK(kvb) + bb * C::BLOCK_BYTES, &tmK, bar(BB_KVFULL + kvb), bb * C::CB,
-                      kt * 128, bh);
-          tma_load_3d(sV(kvb) + bb * C::BLOCK_BYTES, &tmV, bar(BB_KVFULL + kvb), bb * C::CB,
-                      kt * 128, bh);
+          tma_load_4d(sK(kvb) + bb * C::BLOCK_BYTES, &tmK, bar(BB_KVFULL + kvb), bb * C::CB,
+                      kt * 128, bh % p.H, bh / p.H);
+          tma_load_4d(sV(kvb) + bb * C::BLOCK_BYTES, &tmV, bar(BB_KVFULL + kvb), bb * C::CB,
+                      kt * 128, bh % p.H, bh / p.H);
         }
         ++n;
         load_do(kt, bh);
@@ -714,7 +757,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       wait_warp(w, bar(BB_PTDONE), t_last & 1, 30);  // dV' (warp 19) complete too
       tc_fence_after();
       const int key = kt * 128 + r;
-      const size_t off = (static_cast<size_t>(bh) * p.T + (key < p.T ? key : 0)) * D + grp * NQ;
+      const long long kb = bh / p.H, kh = bh % p.H, kr = key < p.T ? key : 0;
       // which = 0: dV (+ dV'), 1: dK * scale; the accumulators are released
       // after the last TMEM load
 #pragma unroll
@@ -735,6 +778,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 #pragma unroll
         for (int e = 0; e < NQ; ++e) x[e] *= mul;
         if (key >= p.T) continue;
+        const long long off = which ? kb * p.dk_sb + kh * p.dk_sh + kr * p.dk_st + grp * NQ
+                                    : kb * p.dv_sb + kh * p.dv_sh + kr * p.dv_st + grp * NQ;
         if (p.dk_f32 != nullptr) {
           float* out = (which ? p.dk_f32 : p.dv_f32) + off;
 #pragma unroll

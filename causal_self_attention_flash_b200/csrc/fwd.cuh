@@ -60,9 +60,11 @@
 namespace cattn {
 
 struct FwdParams {
-  __nv_bfloat16* o;     // (BH, T, D) bf16 out
-  __nv_bfloat16* o_lo;  // O_lo = bf16(O - bf16(O)) out, or null
-  float* lse;          // (BH, T) fp32 out
+  __nv_bfloat16* o;     // (B, H, T, D) bf16 out, element strides o_sb, o_sh, o_st
+  __nv_bfloat16* o_lo;  // O_lo = bf16(O - bf16(O)) out (same strides), or null
+  long long o_sb, o_sh, o_st;
+  float* lse;          // (B, H, T) fp32 out, contiguous
+  int H;
   int T;
   int BH;
   int n_qtiles;
@@ -283,8 +285,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           if (aq[g] > 0) wait1(w, bar(FB_QFREE + g), (aq[g] - 1) & 1, 1);
           mbar_arrive_expect_tx(bar(FB_QFULL + g), C::TILE_BYTES);
           for (int bb = 0; bb < C::NCB; ++bb)
-            tma_load_3d(sbase + C::OFF_Q + g * C::TILE_BYTES + bb * C::BLOCK_BYTES, &tmQ,
-                        bar(FB_QFULL + g), bb * C::CB, it.tile[g] * C::BM, it.bh);
+            tma_load_4d(sbase + C::OFF_Q + g * C::TILE_BYTES + bb * C::BLOCK_BYTES, &tmQ,
+                        bar(FB_QFULL + g), bb * C::CB, it.tile[g] * C::BM, it.bh % p.H,
+                        it.bh / p.H);
           ++aq[g];
         }
         for (int j = 0; j < it.n_kv; ++j, ++tk) {
@@ -299,12 +302,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           const uint32_t sV = sbase + C::OFF_V + st * C::TILE_BYTES;
           mbar_arrive_expect_tx(bar(FB_KFULL + st), C::TILE_BYTES);
           for (int bb = 0; bb < C::NCB; ++bb)
-            tma_load_3d(sK + bb * C::BLOCK_BYTES, &tmK, bar(FB_KFULL + st), bb * C::CB,
-                        j * C::BN, it.bh);
+            tma_load_4d(sK + bb * C::BLOCK_BYTES, &tmK, bar(FB_KFULL + st), bb * C::CB,
+                        j * C::BN, it.bh % p.H, it.bh / p.H);
           mbar_arrive_expect_tx(bar(FB_VFULL + st), C::TILE_BYTES);
           for (int bb = 0; bb < C::NCB; ++bb)
-            tma_load_3d(sV + bb * C::BLOCK_BYTES, &tmV, bar(FB_VFULL + st), bb * C::CB,
-                        j * C::BN, it.bh);
+            tma_load_4d(sV + bb * C::BLOCK_BYTES, &tmV, bar(FB_VFULL + st), bb * C::CB,
+                        j * C::BN, it.bh % p.H, it.bh / p.H);
         }
       }
       if (*abort_flag) {
@@ -564,7 +567,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       const int tile = it.tile[g];
       const int q_row = tile * C::BM + row;
       if (q_row < p.T) {
-        const size_t off = (static_cast<size_t>(it.bh) * p.T + q_row) * D;
+        const long long off = static_cast<long long>(it.bh / p.H) * p.o_sb +
+                              static_cast<long long>(it.bh % p.H) * p.o_sh +
+                              static_cast<long long>(q_row) * p.o_st;
         uint4* orow = reinterpret_cast<uint4*>(p.o + off);
 #pragma unroll
         for (int e = 0; e < D / 8; ++e)

@@ -150,6 +150,50 @@ CATTN_API cattn_status attn_bwd_ex(const void* q, const void* k, const void* v, 
                                    void* dv, int grad_dtype, void* workspace,
                                    size_t workspace_bytes, void* stream);
 
+/* Strided tensors.
+ *
+ * The pages build q, k and v by splitting one projection of shape
+ * (B, T, 3C) and reshaping each part to (B, T, H, D) before moving the head
+ * axis forward ("nanoGPT: a real GPT in two 300-line files", section 2,
+ * CausalSelfAttention: c_attn, then the heads are glued back together into
+ * (B, T, C) after attention).  The _strided calls read and write such
+ * views in place, with no transposes: each (B, H, T, D) operand is given by
+ * its base pointer and its element strides.
+ *
+ *   cattn_layout { b, h, t }: element strides of the batch, head and
+ *   position axes.  The d axis has stride 1.  Each stride must be a
+ *   positive multiple of 8 elements (16 bytes for bf16; rows then start on
+ *   16-byte boundaries) and below 2^38.  The contiguous (B, H, T, D)
+ *   layout is { H*T*D, T*D, D }.  For the c_attn split, q = base,
+ *   k = base + C, v = base + 2C, each with { T*3C, D, 3C }.
+ *   Output (B, T, H*D) is { T*C, D, C }.
+ *
+ * LSE stays a contiguous (B, H, T) fp32 vector; o_lo (if given) shares o's
+ * layout.  Inputs may overlap one another (q, k, v in one buffer).  Outputs
+ * must not overlap each other or any input: they would race.
+ * Errors: as the contiguous calls, plus CATTN_ERR_INVALID_ARG for a stride
+ * outside these limits. */
+typedef struct { long long b, h, t; } cattn_layout;
+
+/* attn_fwd_ex with strided q, k, v and o (o_lo uses o's layout). */
+CATTN_API cattn_status attn_fwd_strided(const void* q, cattn_layout lq, const void* k,
+                                        cattn_layout lk, const void* v, cattn_layout lv,
+                                        float scale, int B, int H, int T, int D, void* o,
+                                        cattn_layout lo, float* lse, void* o_lo, void* stream);
+
+/* attn_bwd_ex with strided q, k, v, o (and o_lo), dout, dq, dk, dv.  dq,
+ * dk and dv may be the three parts of one (B, T, 3C) gradient buffer, the
+ * layout the c_attn backward wants.  With CATTN_DTYPE_F32 the strides count
+ * fp32 elements of dq, dk, dv. */
+CATTN_API cattn_status attn_bwd_strided(const void* q, cattn_layout lq, const void* k,
+                                        cattn_layout lk, const void* v, cattn_layout lv,
+                                        const void* o, cattn_layout lo, const void* o_lo,
+                                        const float* lse, const void* dout, cattn_layout ldo,
+                                        float scale, int B, int H, int T, int D, void* dq,
+                                        cattn_layout ldq, void* dk, cattn_layout ldk, void* dv,
+                                        cattn_layout ldv, int grad_dtype, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
 /* Backward pass for callers that cannot allocate device memory.
  *
  * Same computation, arguments and results as attn_bwd, minus the workspace:

@@ -180,3 +180,59 @@ def test_product_has_no_oracle_dependency():
                     src = fh.read()
                 assert "oracle" not in src, f
                 assert "workloads" not in src, f
+
+
+# ------------------------------------------------------------ strided calls
+
+def contiguous(H, T, D):
+    return _binding.Layout(H * T * D, T * D, D)
+
+
+def fwd_strided(lay=None, lo=None, B=1, H=2, T=8, D=64):
+    c = contiguous(H, T, D)
+    lq = lay or c
+    return cattn.LIB.attn_fwd_strided(ALIGNED, lq, ALIGNED, c, ALIGNED, c, 0.125, B, H, T, D,
+                                      ALIGNED, lo or c, ALIGNED, None, None)
+
+
+def bwd_strided(bad_index=None, bad=None, B=1, H=2, T=8, D=64):
+    c = contiguous(H, T, D)
+    lays = [c] * 8   # q, k, v, o, dout, dq, dk, dv
+    if bad_index is not None:
+        lays[bad_index] = bad
+    return cattn.LIB.attn_bwd_strided(ALIGNED, lays[0], ALIGNED, lays[1], ALIGNED, lays[2],
+                                      ALIGNED, lays[3], None, ALIGNED, ALIGNED, lays[4], 0.125,
+                                      B, H, T, D, ALIGNED, lays[5], ALIGNED, lays[6],
+                                      ALIGNED, lays[7], 0, ALIGNED, 1 << 30, None)
+
+
+@pytest.mark.parametrize("bad", [(0, 64, 8), (512, 64, 0), (512, -64, 8), (512, 64, 12),
+                                 (516, 64, 64), (1 << 38, 64, 64), (512, 3, 64)])
+def test_strided_calls_reject_bad_strides(bad):
+    lay = _binding.Layout(*bad)
+    assert fwd_strided(lay=lay) == cattn.ERR_INVALID_ARG
+    assert fwd_strided(lo=lay) == cattn.ERR_INVALID_ARG
+    for i in range(8):
+        assert bwd_strided(i, lay) == cattn.ERR_INVALID_ARG
+
+
+def test_strided_calls_check_shapes_and_empty():
+    assert fwd_strided(D=48) == cattn.ERR_UNSUPPORTED
+    assert bwd_strided(D=48) == cattn.ERR_UNSUPPORTED
+    assert fwd_strided(T=0) == cattn.OK
+    assert bwd_strided(B=0) == cattn.OK
+
+
+def test_split_qkv_views_share_the_fused_buffer():
+    import torch as t
+    B, T, H, D = 2, 16, 4, 32
+    qkv = t.arange(B * T * 3 * H * D, dtype=t.float32).view(B, T, 3 * H * D)
+    q, k, v = cattn.split_qkv(qkv, H)
+    C = H * D
+    assert q.shape == (B, H, T, D)
+    assert q.stride() == (T * 3 * C, D, 3 * C, 1) == k.stride() == v.stride()
+    assert k.data_ptr() - q.data_ptr() == C * qkv.element_size()
+    assert v.data_ptr() - q.data_ptr() == 2 * C * qkv.element_size()
+    # element (b, h, t, d) of q is qkv[b, t, h*D + d]
+    assert float(q[1, 2, 3, 4]) == float(qkv[1, 3, 2 * D + 4])
+    assert float(v[0, 3, 5, 1]) == float(qkv[0, 5, 2 * C + 3 * D + 1])
