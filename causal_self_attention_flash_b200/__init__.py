@@ -15,13 +15,14 @@ projection straight to a (B, T, C) output with no transposes.
 
 from __future__ import annotations
 
+import ctypes
 import math
 
 import torch
 
 from ._binding import (ERR_CUDA, ERR_INVALID_ARG, ERR_TIMEOUT, ERR_TOO_LARGE,
                        ERR_UNSUPPORTED, LIB, LIB_PATH, NOALLOC_SCRATCH_BYTES, OK,
-                       CattnError, Layout)
+                       CattnError, Dropout, Layout)
 
 __all__ = [
     "attn_fwd", "attn_bwd", "attn_fwd_ex", "attn_bwd_ex", "attn_bwd_preprocess",
@@ -33,6 +34,7 @@ __all__ = [
     "OK", "ERR_INVALID_ARG", "ERR_UNSUPPORTED", "ERR_CUDA", "ERR_TIMEOUT", "ERR_TOO_LARGE",
     "attn_bwd_noalloc", "NOALLOC_SCRATCH_BYTES",
     "attn_fwd_strided", "attn_bwd_strided", "split_qkv", "CausalAttentionQKV", "Layout",
+    "Dropout", "dropout_params",
 ]
 
 
@@ -234,10 +236,20 @@ def split_qkv(qkv, n_head):
     return tuple(x.view(B, T, n_head, D).transpose(1, 2) for x in parts)
 
 
-def attn_fwd_strided(q, k, v, scale=None, o=None, lse=None, o_lo=None, stream=None):
+def dropout_params(p, seed=0, offset=0):
+    """cattn_dropout for drop probability p (0 <= p < 1), a 64-bit seed and
+    a 32-bit counter offset; None for p == 0 (or None)."""
+    if p is None or p == 0:
+        return None
+    return Dropout(float(p), int(seed) & 0xFFFFFFFFFFFFFFFF, int(offset) & 0xFFFFFFFF)
+
+
+def attn_fwd_strided(q, k, v, scale=None, o=None, lse=None, o_lo=None, stream=None,
+                     dropout=None):
     """attn_fwd_ex on strided (B, H, T, D) views.  o (and o_lo) may be views
     too, e.g. of a (B, T, C) buffer (o_lo must share o's strides); if not
-    given they are allocated contiguous.  Returns (o, lse, o_lo)."""
+    given they are allocated contiguous.  dropout: a Dropout (see
+    dropout_params) for attention dropout.  Returns (o, lse, o_lo)."""
     B, H, T, D = _shape(q)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
@@ -248,18 +260,27 @@ def attn_fwd_strided(q, k, v, scale=None, o=None, lse=None, o_lo=None, stream=No
     if o_lo is not None and (o_lo.stride() != o.stride() or o_lo.dtype != torch.bfloat16):
         raise ValueError("o_lo must be a bf16 view with o's strides")
     lse = _want(lse, q, torch.float32, (B, H, T))
-    st = LIB.attn_fwd_strided(q.data_ptr(), lq, k.data_ptr(), lk, v.data_ptr(), lv, float(scale),
-                              B, H, T, D, o.data_ptr(), lo, lse.data_ptr(),
-                              o_lo.data_ptr() if o_lo is not None else None, _stream(stream))
-    _check("attn_fwd_strided", st)
+    olo_ptr = o_lo.data_ptr() if o_lo is not None else None
+    if dropout is None:
+        st = LIB.attn_fwd_strided(q.data_ptr(), lq, k.data_ptr(), lk, v.data_ptr(), lv,
+                                  float(scale), B, H, T, D, o.data_ptr(), lo, lse.data_ptr(),
+                                  olo_ptr, _stream(stream))
+        _check("attn_fwd_strided", st)
+    else:
+        st = LIB.attn_fwd_dropout(q.data_ptr(), lq, k.data_ptr(), lk, v.data_ptr(), lv,
+                                  float(scale), B, H, T, D, ctypes.byref(dropout), o.data_ptr(),
+                                  lo, lse.data_ptr(), olo_ptr, _stream(stream))
+        _check("attn_fwd_dropout", st)
     return o, lse, o_lo
 
 
 def attn_bwd_strided(q, k, v, o, lse, do, scale=None, dq=None, dk=None, dv=None,
-                     workspace=None, stream=None, o_lo=None, grad_dtype=torch.bfloat16):
+                     workspace=None, stream=None, o_lo=None, grad_dtype=torch.bfloat16,
+                     dropout=None):
     """attn_bwd_ex on strided (B, H, T, D) views of q, k, v, o (o_lo with o's
     strides), do and the outputs dq, dk, dv (allocated contiguous if not
-    given; e.g. the three parts of one (B, T, 3C) gradient buffer)."""
+    given; e.g. the three parts of one (B, T, 3C) gradient buffer).  dropout:
+    the forward's Dropout, for attention dropout."""
     B, H, T, D = _shape(q)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
@@ -280,15 +301,24 @@ def attn_bwd_strided(q, k, v, o, lse, do, scale=None, dq=None, dk=None, dv=None,
     need = attn_bwd_workspace_bytes(B, H, T, D)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    st = LIB.attn_bwd_strided(q.data_ptr(), ins[0], k.data_ptr(), ins[1], v.data_ptr(), ins[2],
-                              o.data_ptr(), ins[3],
-                              o_lo.data_ptr() if o_lo is not None else None, lse.data_ptr(),
-                              do.data_ptr(), ins[4], float(scale), B, H, T, D,
-                              dq.data_ptr(), louts[0], dk.data_ptr(), louts[1],
-                              dv.data_ptr(), louts[2],
-                              1 if grad_dtype == torch.float32 else 0,
-                              workspace.data_ptr(), workspace.numel(), _stream(stream))
-    _check("attn_bwd_strided", st)
+    olo_ptr = o_lo.data_ptr() if o_lo is not None else None
+    f32 = 1 if grad_dtype == torch.float32 else 0
+    if dropout is None:
+        st = LIB.attn_bwd_strided(q.data_ptr(), ins[0], k.data_ptr(), ins[1], v.data_ptr(),
+                                  ins[2], o.data_ptr(), ins[3], olo_ptr, lse.data_ptr(),
+                                  do.data_ptr(), ins[4], float(scale), B, H, T, D,
+                                  dq.data_ptr(), louts[0], dk.data_ptr(), louts[1],
+                                  dv.data_ptr(), louts[2], f32,
+                                  workspace.data_ptr(), workspace.numel(), _stream(stream))
+        _check("attn_bwd_strided", st)
+    else:
+        st = LIB.attn_bwd_dropout(q.data_ptr(), ins[0], k.data_ptr(), ins[1], v.data_ptr(),
+                                  ins[2], o.data_ptr(), ins[3], olo_ptr, lse.data_ptr(),
+                                  do.data_ptr(), ins[4], float(scale), B, H, T, D,
+                                  ctypes.byref(dropout), dq.data_ptr(), louts[0],
+                                  dk.data_ptr(), louts[1], dv.data_ptr(), louts[2], f32,
+                                  workspace.data_ptr(), workspace.numel(), _stream(stream))
+        _check("attn_bwd_dropout", st)
     return dq, dk, dv
 
 
@@ -298,10 +328,12 @@ class CausalAttentionQKV(torch.autograd.Function):
     side by side, as the pages' CausalSelfAttention glues them together
     before c_proj.  Forward and backward read and write those layouts in
     place (attn_fwd_strided / attn_bwd_strided); dqkv comes back as one
-    (B, T, 3C) tensor."""
+    (B, T, 3C) tensor.  apply(qkv, n_head, scale=None, dropout_p=0.0,
+    seed=0, offset=0): with dropout_p > 0, attention dropout with the mask
+    of (seed, offset), the same in the backward."""
 
     @staticmethod
-    def forward(ctx, qkv, n_head, scale=None):
+    def forward(ctx, qkv, n_head, scale=None, dropout_p=0.0, seed=0, offset=0):
         B, T, C3 = qkv.shape
         C = C3 // 3
         D = C // n_head
@@ -310,9 +342,10 @@ class CausalAttentionQKV(torch.autograd.Function):
         y_lo = torch.empty_like(y)
         o = y.view(B, T, n_head, D).transpose(1, 2)
         o_lo = y_lo.view(B, T, n_head, D).transpose(1, 2)
-        _, lse, _ = attn_fwd_strided(q, k, v, scale, o=o, o_lo=o_lo)
+        drop = dropout_params(dropout_p, seed, offset)
+        _, lse, _ = attn_fwd_strided(q, k, v, scale, o=o, o_lo=o_lo, dropout=drop)
         ctx.save_for_backward(qkv, y, y_lo, lse)
-        ctx.n_head, ctx.scale = n_head, scale
+        ctx.n_head, ctx.scale, ctx.drop = n_head, scale, drop
         return y
 
     @staticmethod
@@ -328,8 +361,9 @@ class CausalAttentionQKV(torch.autograd.Function):
         do = dy.view(B, T, n_head, D).transpose(1, 2)
         dqkv = torch.empty_like(qkv)
         dq, dk, dv = split_qkv(dqkv, n_head)
-        attn_bwd_strided(q, k, v, o, lse, do, ctx.scale, dq=dq, dk=dk, dv=dv, o_lo=o_lo)
-        return dqkv, None, None
+        attn_bwd_strided(q, k, v, o, lse, do, ctx.scale, dq=dq, dk=dk, dv=dv, o_lo=o_lo,
+                         dropout=ctx.drop)
+        return dqkv, None, None, None, None, None
 
 
 class CausalAttention(torch.autograd.Function):

@@ -31,10 +31,16 @@ class Layout(ctypes.Structure):
     _fields_ = [("b", ctypes.c_longlong), ("h", ctypes.c_longlong), ("t", ctypes.c_longlong)]
 
 
+class Dropout(ctypes.Structure):
+    """cattn_dropout: drop probability p, generator seed and counter offset."""
+    _fields_ = [("p", ctypes.c_float), ("seed", ctypes.c_ulonglong), ("offset", ctypes.c_uint)]
+
+
 # name -> (restype, argtypes), mirroring include/cattn.h
 _vp, _i, _f, _sz, _u32 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_float,
                           ctypes.c_size_t, ctypes.c_uint32)
 _L = Layout
+_DP = ctypes.POINTER(Dropout)
 SIGNATURES = {
     "attn_fwd": (_i, [_vp, _vp, _vp, _f, _i, _i, _i, _i, _vp, _vp, _vp]),
     "attn_fwd_ex": (_i, [_vp, _vp, _vp, _f, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
@@ -50,6 +56,10 @@ SIGNATURES = {
                               _vp]),
     "attn_bwd_strided": (_i, [_vp, _L, _vp, _L, _vp, _L, _vp, _L, _vp, _vp, _vp, _L, _f,
                               _i, _i, _i, _i, _vp, _L, _vp, _L, _vp, _L, _i, _vp, _sz, _vp]),
+    "attn_fwd_dropout": (_i, [_vp, _L, _vp, _L, _vp, _L, _f, _i, _i, _i, _i, _DP, _vp, _L, _vp,
+                              _vp, _vp]),
+    "attn_bwd_dropout": (_i, [_vp, _L, _vp, _L, _vp, _L, _vp, _L, _vp, _vp, _vp, _L, _f,
+                              _i, _i, _i, _i, _DP, _vp, _L, _vp, _L, _vp, _L, _i, _vp, _sz, _vp]),
     "cattn_get_device_status": (_i, [_i, _vp]),
     "cattn_set_wait_timeout_us": (None, [_u32]),
     "cattn_selftest_wait_timeout": (_i, [_u32, _vp]),

@@ -41,7 +41,7 @@ cattn_status cuda_fail(int code) {
   return CATTN_ERR_CUDA;
 }
 int g_dev_ok[kMaxDevices];           // 0 unknown, 1 sm_100, -1 other
-unsigned g_attr_done[kMaxDevices];   // bit per kernel instance
+uint64_t g_attr_done[kMaxDevices];   // bit per kernel instance
 int g_sm_count[kMaxDevices];         // multiprocessors (persistent grids)
 
 cattn_status init_encode() {
@@ -91,13 +91,13 @@ cattn_status check_device(int* dev_out) {
 // Set the dynamic shared-memory limit of a kernel once per device.
 template <typename K>
 cattn_status ensure_smem(int dev, unsigned bit, K kernel, int bytes) {
-  if (g_attr_done[dev] & (1u << bit)) return CATTN_OK;
+  if (g_attr_done[dev] & (1ull << bit)) return CATTN_OK;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
       cudaSuccess) {
     return cuda_fail(cudaGetLastError());
   }
   std::lock_guard<std::mutex> lk(g_mu);
-  g_attr_done[dev] |= 1u << bit;
+  g_attr_done[dev] |= 1ull << bit;
   return CATTN_OK;
 }
 
@@ -117,12 +117,17 @@ cattn_status check_shape(int B, int H, int T, int D) {
 bool empty_shape(int B, int H, int T) { return B == 0 || H == 0 || T == 0; }
 
 // 3-D tensor map over a contiguous (BH, T, D) tensor: x = d, y = t, z = head.
+// 3-D tensor map {x = d, y = t, z = b*H + h} with element strides t_stride
+// and bh_stride (0: the contiguous D and T*D).
 cattn_status make_tmap(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int elem_bytes,
-                       int D, int T, long long BH, int box_x, int box_y) {
+                       int D, int T, long long BH, int box_x, int box_y, long long t_stride = 0,
+                       long long bh_stride = 0) {
+  if (t_stride == 0) t_stride = D;
+  if (bh_stride == 0) bh_stride = static_cast<long long>(T) * D;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(T),
                               static_cast<cuuint64_t>(BH)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * elem_bytes,
-                                 static_cast<cuuint64_t>(D) * T * elem_bytes};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(t_stride) * elem_bytes,
+                                 static_cast<cuuint64_t>(bh_stride) * elem_bytes};
   const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_x), static_cast<cuuint32_t>(box_y), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const int row_bytes = box_x * elem_bytes;
@@ -161,9 +166,16 @@ bool layout_ok(cattn_layout l) {
 // 4-D tensor map {x = d, y = t, z = h, w = b} over a bf16 (B, H, T, D)
 // tensor with element strides lay (the d stride is 1); boxes of
 // [128 rows][min(D, 64) columns], swizzled by the box's row bytes.
+// A (B, H, T, D) layout whose batch stride is H head strides: (b, h) then
+// address like the single index b*H + h.
+bool collapses(cattn_layout l, int H) { return l.b == static_cast<long long>(H) * l.h; }
+
 cattn_status make_bf16_map(CUtensorMap* m, const void* ptr, int D, int T, int H, int B,
-                           cattn_layout lay) {
+                           cattn_layout lay, bool flat) {
   const int cb = D < 64 ? D : 64;
+  if (flat)  // a layout that collapses: 3-D over the b*H + h axis
+    return make_tmap(m, ptr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, T,
+                     static_cast<long long>(B) * H, cb, 128, lay.t, lay.h);
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(T),
                               static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(lay.t) * 2,
@@ -251,19 +263,21 @@ struct LaunchTimer {
 
 unsigned d_index(int D) { return D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3; }
 
-template <int D, bool PLO>
+template <int D, bool PLO, bool DROP, bool FLAT>
 cattn_status fwd_impl(int dev, const void* q, cattn_layout lq, const void* k, cattn_layout lk,
                       const void* v, cattn_layout lv, float scale, int B, int H, int T, void* o,
-                      cattn_layout lo, float* lse, void* o_lo, cudaStream_t s) {
+                      cattn_layout lo, float* lse, void* o_lo, const DropParams& dp,
+                      cudaStream_t s) {
   const int BH = B * H;
   using C = FwdCfg<D, PLO>;
   clear_stale_error();
-  cattn_status st = ensure_smem(dev, 0 + 2 * d_index(D) + PLO, fwd_kernel<D, PLO>, C::SMEM_BYTES);
+  cattn_status st = ensure_smem(dev, (FLAT ? 32 : 0) + (DROP ? 16 : 0) + 2 * d_index(D) + PLO,
+                                fwd_kernel<D, PLO, DROP, FLAT>, C::SMEM_BYTES);
   if (st != CATTN_OK) return st;
   CUtensorMap mq, mk, mv;
-  if ((st = make_bf16_map(&mq, q, D, T, H, B, lq)) != CATTN_OK) return st;
-  if ((st = make_bf16_map(&mk, k, D, T, H, B, lk)) != CATTN_OK) return st;
-  if ((st = make_bf16_map(&mv, v, D, T, H, B, lv)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mq, q, D, T, H, B, lq, FLAT)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mk, k, D, T, H, B, lk, FLAT)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mv, v, D, T, H, B, lv, FLAT)) != CATTN_OK) return st;
   FwdParams p;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.o_lo = static_cast<__nv_bfloat16*>(o_lo);
@@ -277,6 +291,7 @@ cattn_status fwd_impl(int dev, const void* q, cattn_layout lq, const void* k, ca
   p.n_qtiles = (T + 127) / 128;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_timeout_ns;
+  p.drop = dp;
   // persistent: one CTA per SM (it holds all of an SM's TMEM), each looping
   // over work items of two query tiles
   const long long n_items = static_cast<long long>(BH) * ((p.n_qtiles + 1) / 2);
@@ -284,9 +299,24 @@ cattn_status fwd_impl(int dev, const void* q, cattn_layout lq, const void* k, ca
   dim3 grid(static_cast<unsigned>(n_items < g_sm_count[dev] ? n_items : g_sm_count[dev]));
   {
     LaunchTimer t(K_FWD, s);
-    fwd_kernel<D, PLO><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, p);
+    fwd_kernel<D, PLO, DROP, FLAT><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, p);
   }
   return launch_status();
+}
+
+// One forward instance per (PLO, DROP, FLAT); each line picks exactly one.
+template <int D>
+cattn_status fwd_dispatch(bool plo, bool drop, bool flat, int dev, const void* q, cattn_layout lq,
+                          const void* k, cattn_layout lk, const void* v, cattn_layout lv,
+                          float scale, int B, int H, int T, void* o, cattn_layout lo, float* lse,
+                          void* o_lo, const DropParams& dp, cudaStream_t s) {
+#define CATTN_FWD(PL, DR, FL) \
+  fwd_impl<D, PL, DR, FL>(dev, q, lq, k, lk, v, lv, scale, B, H, T, o, lo, lse, o_lo, dp, s)
+  if (plo && drop) return flat ? CATTN_FWD(true, true, true) : CATTN_FWD(true, true, false);
+  if (plo) return flat ? CATTN_FWD(true, false, true) : CATTN_FWD(true, false, false);
+  if (drop) return flat ? CATTN_FWD(false, true, true) : CATTN_FWD(false, true, false);
+  return flat ? CATTN_FWD(false, false, true) : CATTN_FWD(false, false, false);
+#undef CATTN_FWD
 }
 
 // ----------------------------------------------------------------- backward
@@ -337,8 +367,11 @@ cattn_status pre_impl(const void* o, cattn_layout lo, const void* o_lo, const vo
   const size_t work = static_cast<size_t>(p.n_rows);
   {
     LaunchTimer t(K_BWD_PRE, s);
-    bwd_pre_kernel<D><<<grid_for(work > zero_n4 / 64 ? work : zero_n4 / 64, rows_per_block), 256,
-                        0, s>>>(p);
+    const unsigned g = grid_for(work > zero_n4 / 64 ? work : zero_n4 / 64, rows_per_block);
+    if (is_contiguous(lo, H, T, D) && is_contiguous(ldo, H, T, D))
+      bwd_pre_kernel<D, true><<<g, 256, 0, s>>>(p);
+    else
+      bwd_pre_kernel<D, false><<<g, 256, 0, s>>>(p);
   }
   return launch_status();
 }
@@ -353,15 +386,16 @@ BwdLayouts contiguous_bwd_layouts(int H, int T, int D) {
   return BwdLayouts{c, c, c, c, c, c, c, c};
 }
 
-template <int D, bool SLO>
+template <int D, bool SLO, bool DROP, bool FLAT>
 cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, const void* o,
                       const void* o_lo, const float* lse, const void* dout, float scale, int B,
                       int H, int T, void* dq, void* dk, void* dv, const BwdLayouts& ly,
-                      bool grad_f32, void* ws, cudaStream_t s) {
+                      bool grad_f32, void* ws, const DropParams& dp, cudaStream_t s) {
   using C = BwdCfg<D, SLO>;
   const int BH = B * H;
   clear_stale_error();
-  cattn_status st = ensure_smem(dev, 8 + 2 * d_index(D) + SLO, bwd_kernel<D, SLO>, C::SMEM_BYTES);
+  cattn_status st = ensure_smem(dev, (FLAT ? 32 : 0) + (DROP ? 24 : 8) + 2 * d_index(D) + SLO,
+                                bwd_kernel<D, SLO, DROP, FLAT>, C::SMEM_BYTES);
   if (st != CATTN_OK) return st;
   const WsLayout L = ws_layout(BH, T, D);
   uint8_t* wb = static_cast<uint8_t*>(ws);
@@ -371,10 +405,10 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   const size_t n_dq = static_cast<size_t>(BH) * T * D;
 
   CUtensorMap mq, mk, mv, mdo, mdq;
-  if ((st = make_bf16_map(&mq, q, D, T, H, B, ly.q)) != CATTN_OK) return st;
-  if ((st = make_bf16_map(&mk, k, D, T, H, B, ly.k)) != CATTN_OK) return st;
-  if ((st = make_bf16_map(&mv, v, D, T, H, B, ly.v)) != CATTN_OK) return st;
-  if ((st = make_bf16_map(&mdo, dout, D, T, H, B, ly.dout)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mq, q, D, T, H, B, ly.q, FLAT)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mk, k, D, T, H, B, ly.k, FLAT)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mv, v, D, T, H, B, ly.v, FLAT)) != CATTN_OK) return st;
+  if ((st = make_bf16_map(&mdo, dout, D, T, H, B, ly.dout, FLAT)) != CATTN_OK) return st;
   if ((st = make_tmap(&mdq, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, T, BH,
                       C::WARP_DQ ? D / 4 : C::CBQ, C::WARP_DQ ? 32 : 128)) !=
       CATTN_OK)
@@ -405,13 +439,14 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_timeout_ns;
+  p.drop = dp;
   // persistent: one CTA per SM, each looping over key tiles
   const long long n_items = static_cast<long long>(BH) * p.n_tiles;
   if (n_items > 0x7fffffffLL) return CATTN_ERR_INVALID_ARG;
   dim3 grid(static_cast<unsigned>(n_items < g_sm_count[dev] ? n_items : g_sm_count[dev]));
   {
     LaunchTimer t(K_BWD_MAIN, s);
-    bwd_kernel<D, SLO><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mdo, mdq, p);
+    bwd_kernel<D, SLO, DROP, FLAT><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mdo, mdq, p);
   }
   if ((st = launch_status()) != CATTN_OK) return st;
   {
@@ -441,11 +476,40 @@ template <int D>
 cattn_status bwd_dispatch(bool slo, int dev, const void* q, const void* k, const void* v,
                           const void* o, const void* o_lo, const float* lse, const void* dout,
                           float scale, int B, int H, int T, void* dq, void* dk, void* dv,
-                          const BwdLayouts& ly, bool f32, void* ws, cudaStream_t s) {
-  return slo ? bwd_impl<D, true>(dev, q, k, v, o, o_lo, lse, dout, scale, B, H, T, dq, dk, dv, ly,
-                                 f32, ws, s)
-             : bwd_impl<D, false>(dev, q, k, v, o, o_lo, lse, dout, scale, B, H, T, dq, dk, dv,
-                                  ly, f32, ws, s);
+                          const BwdLayouts& ly, bool f32, void* ws, const DropParams& dp,
+                          cudaStream_t s) {
+  // FLAT: every tensor the main kernel addresses by (b, h) collapses to one
+  // b*H + h axis (the contiguous layout among others): 3-D tensor maps and
+  // no division by H in the kernel
+  const bool flat = collapses(ly.q, H) && collapses(ly.k, H) && collapses(ly.v, H) &&
+                    collapses(ly.dout, H) && collapses(ly.dk, H) && collapses(ly.dv, H);
+  // one instance per (SLO, DROP, FLAT); each line picks exactly one
+  const bool drop = dp.t16x != 0;
+#define CATTN_BWD(SS, DR, FL) \
+  bwd_impl<D, SS, DR, FL>(dev, q, k, v, o, o_lo, lse, dout, scale, B, H, T, dq, dk, dv, ly, f32, ws, dp, s)
+  if (slo && drop) return flat ? CATTN_BWD(true, true, true) : CATTN_BWD(true, true, false);
+  if (slo) return flat ? CATTN_BWD(true, false, true) : CATTN_BWD(true, false, false);
+  if (drop) return flat ? CATTN_BWD(false, true, true) : CATTN_BWD(false, true, false);
+  return flat ? CATTN_BWD(false, false, true) : CATTN_BWD(false, false, false);
+#undef CATTN_BWD
+}
+
+// Dropout parameters of a call: t = round(p * 65536) (the drop threshold on
+// 16 random bits), 1 / (1 - t / 65536) as the keep scale; false for a
+// probability outside [0, 1).  t = 0 (no dropout, p < 2^-17) selects the
+// kernels without the mask, whose result is then the same.
+bool drop_params(const cattn_dropout* d, DropParams* out) {
+  *out = DropParams{0u, 0u, 0u, 0u, 1.f};
+  if (d == nullptr) return true;
+  if (!(d->p >= 0.f) || !(d->p < 1.f)) return false;
+  long t = lrint(static_cast<double>(d->p) * 65536.0);
+  if (t > 65535) t = 65535;
+  out->t16x = static_cast<uint32_t>(t) << 16;
+  out->k0 = static_cast<uint32_t>(d->seed & 0xffffffffull);
+  out->k1 = static_cast<uint32_t>(d->seed >> 32);
+  out->offset = d->offset;
+  out->inv_keep = static_cast<float>(65536.0 / (65536.0 - static_cast<double>(t)));
+  return true;
 }
 
 // ---------------------------------------------------------- hang-guard test
@@ -473,13 +537,15 @@ using namespace cattn;
 
 extern "C" {
 
-cattn_status attn_fwd_strided(const void* q, cattn_layout lq, const void* k, cattn_layout lk,
+cattn_status attn_fwd_dropout(const void* q, cattn_layout lq, const void* k, cattn_layout lk,
                               const void* v, cattn_layout lv, float scale, int B, int H, int T,
-                              int D, void* o, cattn_layout lo, float* lse, void* o_lo,
-                              void* stream) {
+                              int D, const cattn_dropout* dropout, void* o, cattn_layout lo,
+                              float* lse, void* o_lo, void* stream) {
   cattn_status st = check_shape(B, H, T, D);
   if (st != CATTN_OK) return st;
   if (!(scale > 0.f) || !isfinite(scale)) return CATTN_ERR_INVALID_ARG;
+  DropParams dp;
+  if (!drop_params(dropout, &dp)) return CATTN_ERR_INVALID_ARG;
   if (empty_shape(B, H, T)) return CATTN_OK;
   if (!q || !k || !v || !o || !lse) return CATTN_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
@@ -490,17 +556,24 @@ cattn_status attn_fwd_strided(const void* q, cattn_layout lq, const void* k, cat
   int dev;
   if ((st = check_device(&dev)) != CATTN_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-#define CATTN_FWD(DD)                                                                         \
-  return o_lo ? fwd_impl<DD, true>(dev, q, lq, k, lk, v, lv, scale, B, H, T, o, lo, lse, o_lo, s) \
-              : fwd_impl<DD, false>(dev, q, lq, k, lk, v, lv, scale, B, H, T, o, lo, lse, o_lo, s)
+  // FLAT: q, k, v and o all collapse to one b*H + h axis (see bwd_dispatch)
+  const bool flat = collapses(lq, H) && collapses(lk, H) && collapses(lv, H) && collapses(lo, H);
+  const bool plo = o_lo != nullptr, drop = dp.t16x != 0;
   switch (D) {
-    case 16: CATTN_FWD(16);
-    case 32: CATTN_FWD(32);
-    case 64: CATTN_FWD(64);
-    case 128: CATTN_FWD(128);
+    case 16: return fwd_dispatch<16>(plo, drop, flat, dev, q, lq, k, lk, v, lv, scale, B, H, T, o, lo, lse, o_lo, dp, s);
+    case 32: return fwd_dispatch<32>(plo, drop, flat, dev, q, lq, k, lk, v, lv, scale, B, H, T, o, lo, lse, o_lo, dp, s);
+    case 64: return fwd_dispatch<64>(plo, drop, flat, dev, q, lq, k, lk, v, lv, scale, B, H, T, o, lo, lse, o_lo, dp, s);
+    case 128: return fwd_dispatch<128>(plo, drop, flat, dev, q, lq, k, lk, v, lv, scale, B, H, T, o, lo, lse, o_lo, dp, s);
   }
-#undef CATTN_FWD
   return CATTN_ERR_UNSUPPORTED;
+}
+
+cattn_status attn_fwd_strided(const void* q, cattn_layout lq, const void* k, cattn_layout lk,
+                              const void* v, cattn_layout lv, float scale, int B, int H, int T,
+                              int D, void* o, cattn_layout lo, float* lse, void* o_lo,
+                              void* stream) {
+  return attn_fwd_dropout(q, lq, k, lk, v, lv, scale, B, H, T, D, nullptr, o, lo, lse, o_lo,
+                          stream);
 }
 
 cattn_status attn_fwd_ex(const void* q, const void* k, const void* v, float scale, int B, int H,
@@ -540,16 +613,18 @@ cattn_status attn_bwd_preprocess(const void* o, const void* dout, int B, int H, 
   return CATTN_ERR_UNSUPPORTED;
 }
 
-cattn_status attn_bwd_strided(const void* q, cattn_layout lq, const void* k, cattn_layout lk,
+cattn_status attn_bwd_dropout(const void* q, cattn_layout lq, const void* k, cattn_layout lk,
                               const void* v, cattn_layout lv, const void* o, cattn_layout lo,
                               const void* o_lo, const float* lse, const void* dout,
-                              cattn_layout ldo, float scale, int B, int H, int T, int D, void* dq,
-                              cattn_layout ldq, void* dk, cattn_layout ldk, void* dv,
-                              cattn_layout ldv, int grad_dtype, void* workspace,
-                              size_t workspace_bytes, void* stream) {
+                              cattn_layout ldo, float scale, int B, int H, int T, int D,
+                              const cattn_dropout* dropout, void* dq, cattn_layout ldq, void* dk,
+                              cattn_layout ldk, void* dv, cattn_layout ldv, int grad_dtype,
+                              void* workspace, size_t workspace_bytes, void* stream) {
   cattn_status st = check_shape(B, H, T, D);
   if (st != CATTN_OK) return st;
   if (!(scale > 0.f) || !isfinite(scale)) return CATTN_ERR_INVALID_ARG;
+  DropParams dp;
+  if (!drop_params(dropout, &dp)) return CATTN_ERR_INVALID_ARG;
   if (empty_shape(B, H, T)) return CATTN_OK;
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
     return CATTN_ERR_INVALID_ARG;
@@ -572,12 +647,24 @@ cattn_status attn_bwd_strided(const void* q, cattn_layout lq, const void* k, cat
   // dS as a hi/lo pair when the caller asks for gradients accurate to ~fp32
   const bool slo = o_lo != nullptr || f32;
   switch (D) {
-    case 16: return bwd_dispatch<16>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, B, H, T, dq, dk, dv, ly, f32, workspace, s);
-    case 32: return bwd_dispatch<32>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, B, H, T, dq, dk, dv, ly, f32, workspace, s);
-    case 64: return bwd_dispatch<64>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, B, H, T, dq, dk, dv, ly, f32, workspace, s);
-    case 128: return bwd_dispatch<128>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, B, H, T, dq, dk, dv, ly, f32, workspace, s);
+    case 16: return bwd_dispatch<16>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, B, H, T, dq, dk, dv, ly, f32, workspace, dp, s);
+    case 32: return bwd_dispatch<32>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, B, H, T, dq, dk, dv, ly, f32, workspace, dp, s);
+    case 64: return bwd_dispatch<64>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, B, H, T, dq, dk, dv, ly, f32, workspace, dp, s);
+    case 128: return bwd_dispatch<128>(slo, dev, q, k, v, o, o_lo, lse, dout, scale, B, H, T, dq, dk, dv, ly, f32, workspace, dp, s);
   }
   return CATTN_ERR_UNSUPPORTED;
+}
+
+cattn_status attn_bwd_strided(const void* q, cattn_layout lq, const void* k, cattn_layout lk,
+                              const void* v, cattn_layout lv, const void* o, cattn_layout lo,
+                              const void* o_lo, const float* lse, const void* dout,
+                              cattn_layout ldo, float scale, int B, int H, int T, int D, void* dq,
+                              cattn_layout ldq, void* dk, cattn_layout ldk, void* dv,
+                              cattn_layout ldv, int grad_dtype, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  return attn_bwd_dropout(q, lq, k, lk, v, lv, o, lo, o_lo, lse, dout, ldo, scale, B, H, T, D,
+                          nullptr, dq, ldq, dk, ldk, dv, ldv, grad_dtype, workspace,
+                          workspace_bytes, stream);
 }
 
 cattn_status attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
@@ -633,19 +720,20 @@ cattn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const
   // the backward clears what must start at zero (the dQ accumulator) and
   // overwrites the rest on every call
   const BwdLayouts ly = contiguous_bwd_layouts(H, T, D);
+  const DropParams no_drop{0u, 0u, 0u, 0u, 1.f};
   switch (D) {
     case 16:
-      return bwd_impl<16, false>(dev, q, k, v, o, nullptr, lse, dout, scale, B, H, T, dq, dk, dv, ly,
-                                 false, scratch, s);
+      return bwd_impl<16, false, false, true>(dev, q, k, v, o, nullptr, lse, dout, scale, B, H, T, dq, dk,
+                                        dv, ly, false, scratch, no_drop, s);
     case 32:
-      return bwd_impl<32, false>(dev, q, k, v, o, nullptr, lse, dout, scale, B, H, T, dq, dk, dv, ly,
-                                 false, scratch, s);
+      return bwd_impl<32, false, false, true>(dev, q, k, v, o, nullptr, lse, dout, scale, B, H, T, dq, dk,
+                                        dv, ly, false, scratch, no_drop, s);
     case 64:
-      return bwd_impl<64, false>(dev, q, k, v, o, nullptr, lse, dout, scale, B, H, T, dq, dk, dv, ly,
-                                 false, scratch, s);
+      return bwd_impl<64, false, false, true>(dev, q, k, v, o, nullptr, lse, dout, scale, B, H, T, dq, dk,
+                                        dv, ly, false, scratch, no_drop, s);
     case 128:
-      return bwd_impl<128, false>(dev, q, k, v, o, nullptr, lse, dout, scale, B, H, T, dq, dk, dv, ly,
-                                 false, scratch, s);
+      return bwd_impl<128, false, false, true>(dev, q, k, v, o, nullptr, lse, dout, scale, B, H, T, dq, dk,
+                                        dv, ly, false, scratch, no_drop, s);
   }
   return CATTN_ERR_UNSUPPORTED;
 }

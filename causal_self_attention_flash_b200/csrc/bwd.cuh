@@ -29,6 +29,7 @@
 // accurate to ~fp32).
 #pragma once
 
+#include "philox.cuh"
 #include "sm100.cuh"
 
 namespace cattn {
@@ -54,7 +55,8 @@ struct PreParams {
 };
 
 // Threads per row: each handles 8 bf16 (16 bytes) of O and of dO.
-template <int D>
+// CONTIG: O and dO are contiguous (B, H, T, D), addressed as rows of D.
+template <int D, bool CONTIG>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
   constexpr int TPR = D / 8;
   constexpr int RPW = 32 / TPR;  // rows per warp per step
@@ -91,9 +93,16 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
       valid[u] = pr[u] < p.n_rows && t[u] < p.T;
       a[u] = bb[u] = c[u] = make_uint4(0u, 0u, 0u, 0u);
       if (valid[u]) {
-        const long long b_ = bh[u] / p.H, h_ = bh[u] - b_ * p.H;
-        const long long off = b_ * p.o_sb + h_ * p.o_sh + t[u] * p.o_st + sub * 8;
-        const long long doff = b_ * p.do_sb + h_ * p.do_sh + t[u] * p.do_st + sub * 8;
+        long long off, doff;
+        if constexpr (CONTIG) {
+          off = doff = (static_cast<long long>(bh[u]) * p.T + t[u]) * D + sub * 8;
+        } else {
+          // (B*H < 2^31: a 32-bit division)
+          const unsigned hb = static_cast<unsigned>(bh[u]) / static_cast<unsigned>(p.H);
+          const long long b_ = hb, h_ = static_cast<long long>(bh[u]) - b_ * p.H;
+          off = b_ * p.o_sb + h_ * p.o_sh + t[u] * p.o_st + sub * 8;
+          doff = b_ * p.do_sb + h_ * p.do_sh + t[u] * p.do_st + sub * 8;
+        }
         a[u] = *reinterpret_cast<const uint4*>(p.o + off);
         bb[u] = *reinterpret_cast<const uint4*>(p.dout + doff);
         if (p.o_lo != nullptr) c[u] = *reinterpret_cast<const uint4*>(p.o_lo + off);
@@ -174,11 +183,13 @@ __global__ void __launch_bounds__(256) dq_convert_strided_kernel(const float4* _
   const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long nth = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long i = tid; i < n8; i += nth) {
-    const long long row = i / C8;
+    const long long row = i / C8;  // C8 is a power of two: a shift
     const int c8 = static_cast<int>(i - row * C8);
-    const long long bh = row / T;
+    const long long bh = row <= 0xffffffffLL
+                             ? static_cast<long long>(static_cast<unsigned>(row) / static_cast<unsigned>(T))
+                             : row / T;
     const long long t = row - bh * T;
-    const long long b = bh / H, h = bh - b * H;
+    const long long b = static_cast<unsigned>(bh) / static_cast<unsigned>(H), h = bh - b * H;
     const long long off = b * sb + h * sh + t * st + c8 * 8;
     const float4 a = acc[2 * i];
     const float4 c = acc[2 * i + 1];
@@ -247,6 +258,7 @@ struct BwdParams {
   float scale;
   float scale_log2;
   uint64_t timeout_ns;
+  DropParams drop;  // attention dropout (kernels instantiated with DROP only)
 };
 
 template <int D, bool SLO>
@@ -333,7 +345,10 @@ __device__ __forceinline__ int bwd_item(int k, int b, int G, int n_items) {
   return u < n_items ? u : -1;
 }
 
-template <int D, bool SLO>
+// FLAT: Q, K, V, dO, dK and dV address (b, h) as one b*H + h axis (3-D
+// tensor maps, dK/dV offsets bh * d?_sh); otherwise 4-D maps with (h, b)
+// coordinates.
+template <int D, bool SLO, bool DROP, bool FLAT>
 __global__ void __launch_bounds__(640, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -409,6 +424,16 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmDO);
       int tq = 0, tdo = 0, n = 0;  // loads issued
+      // one [128][CB] box at column x, row y of head bh: a 4-D map takes
+      // (h, b) coordinates, a 3-D map (the (B*H, T, D) layout) takes bh
+      auto load_tile = [&](uint32_t dst, const CUtensorMap* m, int bit, uint32_t mbar, int x,
+                           int y, int bh) {
+        (void)bit;
+        if constexpr (FLAT)
+          tma_load_3d(dst, m, mbar, x, y, bh);
+        else
+          tma_load_4d(dst, m, mbar, x, y, bh % p.H, bh / p.H);
+      };
       auto load_q = [&](int qi, int bh) {
         const int qs = tq % C::QST;
         if (tq >= C::QST) wait1(w, bar(BB_QEMPTY + qs), ((tq / C::QST) - 1) & 1, 1);
@@ -417,8 +442,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const uint32_t sQ = sbase + C::OFF_Q + qs * C::TILE_BYTES;
         mbar_arrive_expect_tx(bar(BB_QFULL + qs), C::TILE_BYTES + 1024);
         for (int bb = 0; bb < C::NCB; ++bb)
-          tma_load_4d(sQ + bb * C::BLOCK_BYTES, &tmQ, bar(BB_QFULL + qs), bb * C::CB, qi * 128,
-                      bh % p.H, bh / p.H);
+          load_tile(sQ + bb * C::BLOCK_BYTES, &tmQ, 1, bar(BB_QFULL + qs), bb * C::CB, qi * 128,
+                    bh);
         bulk_load(sbase + C::OFF_LSE + qs * 512, p.lse2 + vec, 512, bar(BB_QFULL + qs));
         bulk_load(sbase + C::OFF_DELTA + qs * 512, p.delta + vec, 512, bar(BB_QFULL + qs));
         ++tq;
@@ -430,8 +455,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const uint32_t sDO = sbase + C::OFF_DO + ds * C::TILE_BYTES;
         mbar_arrive_expect_tx(bar(BB_DOFULL + ds), C::TILE_BYTES);
         for (int bb = 0; bb < C::NCB; ++bb)
-          tma_load_4d(sDO + bb * C::BLOCK_BYTES, &tmDO, bar(BB_DOFULL + ds), bb * C::CB, qi * 128,
-                      bh % p.H, bh / p.H);
+          load_tile(sDO + bb * C::BLOCK_BYTES, &tmDO, 8, bar(BB_DOFULL + ds), bb * C::CB,
+                    qi * 128, bh);
         ++tdo;
       };
       for (int k = 0;; ++k) {
@@ -446,10 +471,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         if (*abort_flag) break;
         mbar_arrive_expect_tx(bar(BB_KVFULL + kvb), 2 * C::TILE_BYTES);
         for (int bb = 0; bb < C::NCB; ++bb) {
-          tma_load_4d(sK(kvb) + bb * C::BLOCK_BYTES, &tmK, bar(BB_KVFULL + kvb), bb * C::CB,
-                      kt * 128, bh % p.H, bh / p.H);
-          tma_load_4d(sV(kvb) + bb * C::BLOCK_BYTES, &tmV, bar(BB_KVFULL + kvb), bb * C::CB,
-                      kt * 128, bh % p.H, bh / p.H);
+          load_tile(sK(kvb) + bb * C::BLOCK_BYTES, &tmK, 2, bar(BB_KVFULL + kvb), bb * C::CB,
+                    kt * 128, bh);
+          load_tile(sV(kvb) + bb * C::BLOCK_BYTES, &tmV, 4, bar(BB_KVFULL + kvb), bb * C::CB,
+                    kt * 128, bh);
         }
         ++n;
         load_do(kt, bh);
@@ -757,7 +782,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       wait_warp(w, bar(BB_PTDONE), t_last & 1, 30);  // dV' (warp 19) complete too
       tc_fence_after();
       const int key = kt * 128 + r;
-      const long long kb = bh / p.H, kh = bh % p.H, kr = key < p.T ? key : 0;
+      const long long kb = FLAT ? 0 : bh / p.H, kh = FLAT ? 0 : bh % p.H;
+      const long long kr = key < p.T ? key : 0;
       // which = 0: dV (+ dV'), 1: dK * scale; the accumulators are released
       // after the last TMEM load
 #pragma unroll
@@ -774,12 +800,14 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           tc_fence_before();
           mbar_arrive(bar(BB_ACCFREE));
         }
-        const float mul = which ? p.scale : 1.f;
+        const float mul = which ? p.scale : (DROP ? p.drop.inv_keep : 1.f);
 #pragma unroll
         for (int e = 0; e < NQ; ++e) x[e] *= mul;
         if (key >= p.T) continue;
-        const long long off = which ? kb * p.dk_sb + kh * p.dk_sh + kr * p.dk_st + grp * NQ
-                                    : kb * p.dv_sb + kh * p.dv_sh + kr * p.dv_st + grp * NQ;
+        const long long off =
+            FLAT ? (which ? bh * p.dk_sh + kr * p.dk_st : bh * p.dv_sh + kr * p.dv_st) + grp * NQ
+                 : (which ? kb * p.dk_sb + kh * p.dk_sh + kr * p.dk_st
+                          : kb * p.dv_sb + kh * p.dv_sh + kr * p.dv_st) + grp * NQ;
         if (p.dk_f32 != nullptr) {
           float* out = (which ? p.dk_f32 : p.dv_f32) + off;
 #pragma unroll
@@ -817,6 +845,25 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       const int n_iter = p.n_tiles - kt;
       for (int i = 0; i < n_iter; ++i, ++t) {
         const int qs = t % C::QST;
+        // ---- dropout keep bits (DROP), while S is on its way: bit c of
+        // keepm is this key row's bit for query column 32g + c.  Lane l
+        // draws the bits of keys 8*(l/8) .. +7 of its warp for query
+        // 8s + l%8 (one generator block each); a shuffle per query hands
+        // every lane the bit of its own key.
+        [[maybe_unused]] uint32_t keepm = 0u;
+        if constexpr (DROP) {
+          const uint32_t jg = static_cast<uint32_t>((kt * 128 + quarter * 32) / 8 + (lane >> 3));
+          const uint32_t qb = static_cast<uint32_t>((kt + i) * 128 + grp * 32 + (lane & 7));
+#pragma unroll
+          for (int s8 = 0; s8 < 4; ++s8) {
+            const uint32_t byte = keep_byte(jg, qb + 8 * s8, static_cast<uint32_t>(bh), p.drop);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const uint32_t v8 = __shfl_sync(0xffffffffu, byte, (lane & ~7) | q);
+              keepm |= ((v8 >> (lane & 7)) & 1u) << (8 * s8 + q);
+            }
+          }
+        }
         // ---- P phase
         wait_warp(w, bar(BB_SFULL), t & 1, 15);
         tc_fence_after();
@@ -849,9 +896,18 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
               if (c < lim) pv[c] = 0.f;
           }
           uint32_t hi[8], lo[8];
+          if constexpr (DROP) {  // dV takes the dropped P (scaled in the epilogue)
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            split_bf16x2_p(f2(pv[16 * h + 2 * e], pv[16 * h + 2 * e + 1]), hi[e], lo[e]);
+            for (int e = 0; e < 8; ++e) {
+              const float a0 = ((keepm >> (16 * h + 2 * e)) & 1u) ? pv[16 * h + 2 * e] : 0.f;
+              const float a1 = ((keepm >> (16 * h + 2 * e + 1)) & 1u) ? pv[16 * h + 2 * e + 1] : 0.f;
+              split_bf16x2_p(f2(a0, a1), hi[e], lo[e]);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              split_bf16x2_p(f2(pv[16 * h + 2 * e], pv[16 * h + 2 * e + 1]), hi[e], lo[e]);
+          }
           tmem_st8(tbase + lane_base + C::COL_S + grp * 32 + 8 * h, hi);
           tmem_st8(tbase + lane_base + C::COL_S + grp * 32 + 16 + 8 * h, lo);
           tmem_wait_st();
@@ -879,10 +935,23 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           for (int e = 0; e < 32; e += 4) {
             float d0, d1, d2, d3;
             ld_shared_v4f(sD + e * 4, d0, d1, d2, d3);
-            const float s0 = pv[e] * (__uint_as_float(v[e]) - d0);
-            const float s1 = pv[e + 1] * (__uint_as_float(v[e + 1]) - d1);
-            const float s2 = pv[e + 2] * (__uint_as_float(v[e + 2]) - d2);
-            const float s3 = pv[e + 3] * (__uint_as_float(v[e + 3]) - d3);
+            float s0, s1, s2, s3;
+            if constexpr (DROP) {  // dP = dP~ * mask / (1 - p)
+              const float kp = p.drop.inv_keep;
+              const float g0 = ((keepm >> e) & 1u) ? __uint_as_float(v[e]) * kp : 0.f;
+              const float g1 = ((keepm >> (e + 1)) & 1u) ? __uint_as_float(v[e + 1]) * kp : 0.f;
+              const float g2 = ((keepm >> (e + 2)) & 1u) ? __uint_as_float(v[e + 2]) * kp : 0.f;
+              const float g3 = ((keepm >> (e + 3)) & 1u) ? __uint_as_float(v[e + 3]) * kp : 0.f;
+              s0 = pv[e] * (g0 - d0);
+              s1 = pv[e + 1] * (g1 - d1);
+              s2 = pv[e + 2] * (g2 - d2);
+              s3 = pv[e + 3] * (g3 - d3);
+            } else {
+              s0 = pv[e] * (__uint_as_float(v[e]) - d0);
+              s1 = pv[e + 1] * (__uint_as_float(v[e + 1]) - d1);
+              s2 = pv[e + 2] * (__uint_as_float(v[e + 2]) - d2);
+              s3 = pv[e + 3] * (__uint_as_float(v[e + 3]) - d3);
+            }
             if (SLO) {
               split_bf16x2_p(f2(s0, s1), hi[e / 2], lo[e / 2]);
               split_bf16x2_p(f2(s2, s3), hi[e / 2 + 1], lo[e / 2 + 1]);

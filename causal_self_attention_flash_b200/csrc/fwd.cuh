@@ -55,6 +55,7 @@
 // unchanged: it is still exactly the softmax, as the online rewrite is.
 #pragma once
 
+#include "philox.cuh"
 #include "sm100.cuh"
 
 namespace cattn {
@@ -70,6 +71,7 @@ struct FwdParams {
   int n_qtiles;
   float scale_log2;    // scale * log2(e)
   uint64_t timeout_ns;
+  DropParams drop;     // attention dropout (kernels instantiated with DROP only)
 };
 
 template <int D, bool PLO>
@@ -138,9 +140,12 @@ constexpr int kPvParts = 2;
 
 // P = 2^(s * scale_log2 - m) for one row of a 128-column tile: written to
 // TMEM as bf16 (or bf16 hi/lo), the row sum accumulated in sum2.
-template <bool POLY, bool PLO>
+// DROP: P entries whose bit in keep (bit c of keep[c / 32] for column c) is
+// clear are written as 0; the row sum still takes every entry.
+template <bool POLY, bool PLO, bool DROP>
 __device__ __forceinline__ void fwd_exp_row(const float (&s)[128], uint64_t sl2x2, uint64_t negm2,
-                                            uint32_t scol, uint64_t (&sum2)[2], uint32_t pfull0) {
+                                            uint32_t scol, uint64_t (&sum2)[2], uint32_t pfull0,
+                                            const uint32_t* keep) {
 #pragma unroll
   for (int ch = 0; ch < 8; ++ch) {  // 16 columns per chunk
     uint32_t hi[8], lo[8];
@@ -158,6 +163,14 @@ __device__ __forceinline__ void fwd_exp_row(const float (&s)[128], uint64_t sl2x
         p2 = f2(ex2(x0), ex2(x1));
       }
       sum2[e & 1] = add2(sum2[e & 1], p2);
+      if constexpr (DROP) {
+        const int c = ch * 16 + 2 * e;
+        float p0, p1;
+        f2_split(p2, p0, p1);
+        p0 = ((keep[c >> 5] >> (c & 31)) & 1u) ? p0 : 0.f;
+        p1 = ((keep[c >> 5] >> ((c + 1) & 31)) & 1u) ? p1 : 0.f;
+        p2 = f2(p0, p1);
+      }
       if (PLO) {
         split_bf16x2_p(p2, hi[e], lo[e]);
       } else {
@@ -214,7 +227,9 @@ __device__ __forceinline__ FwdItem fwd_item_info(int u, int k, int BH, int n_pai
   return it;
 }
 
-template <int D, bool PLO>
+// FLAT: Q, K, V and O address (b, h) as one b*H + h axis (3-D tensor
+// maps, O offsets bh * o_sh); otherwise 4-D maps with (h, b) coordinates.
+template <int D, bool PLO, bool DROP, bool FLAT>
 __global__ void __launch_bounds__(352, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -276,6 +291,16 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       int tk = 0, aq[2] = {0, 0};
+      // one [128][CB] box at column x, row y of head bh: a 4-D map takes
+      // (h, b) coordinates, a 3-D map (the (B*H, T, D) layout) takes bh
+      auto load_tile = [&](uint32_t dst, const CUtensorMap* m, int bit, uint32_t mbar, int x,
+                           int y, int bh) {
+        (void)bit;
+        if constexpr (FLAT)
+          tma_load_3d(dst, m, mbar, x, y, bh);
+        else
+          tma_load_4d(dst, m, mbar, x, y, bh % p.H, bh / p.H);
+      };
       for (int k = 0;; ++k) {
         const int u = fwd_item(k, b, G, n_items);
         if (u < 0 || *abort_flag) break;
@@ -285,9 +310,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           if (aq[g] > 0) wait1(w, bar(FB_QFREE + g), (aq[g] - 1) & 1, 1);
           mbar_arrive_expect_tx(bar(FB_QFULL + g), C::TILE_BYTES);
           for (int bb = 0; bb < C::NCB; ++bb)
-            tma_load_4d(sbase + C::OFF_Q + g * C::TILE_BYTES + bb * C::BLOCK_BYTES, &tmQ,
-                        bar(FB_QFULL + g), bb * C::CB, it.tile[g] * C::BM, it.bh % p.H,
-                        it.bh / p.H);
+            load_tile(sbase + C::OFF_Q + g * C::TILE_BYTES + bb * C::BLOCK_BYTES, &tmQ, 1,
+                      bar(FB_QFULL + g), bb * C::CB, it.tile[g] * C::BM, it.bh);
           ++aq[g];
         }
         for (int j = 0; j < it.n_kv; ++j, ++tk) {
@@ -302,12 +326,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           const uint32_t sV = sbase + C::OFF_V + st * C::TILE_BYTES;
           mbar_arrive_expect_tx(bar(FB_KFULL + st), C::TILE_BYTES);
           for (int bb = 0; bb < C::NCB; ++bb)
-            tma_load_4d(sK + bb * C::BLOCK_BYTES, &tmK, bar(FB_KFULL + st), bb * C::CB,
-                        j * C::BN, it.bh % p.H, it.bh / p.H);
+            load_tile(sK + bb * C::BLOCK_BYTES, &tmK, 2, bar(FB_KFULL + st), bb * C::CB,
+                      j * C::BN, it.bh);
           mbar_arrive_expect_tx(bar(FB_VFULL + st), C::TILE_BYTES);
           for (int bb = 0; bb < C::NCB; ++bb)
-            tma_load_4d(sV + bb * C::BLOCK_BYTES, &tmV, bar(FB_VFULL + st), bb * C::CB,
-                        j * C::BN, it.bh % p.H, it.bh / p.H);
+            load_tile(sV + bb * C::BLOCK_BYTES, &tmV, 4, bar(FB_VFULL + st), bb * C::CB,
+                      j * C::BN, it.bh);
         }
       }
       if (*abort_flag) {
@@ -443,6 +467,18 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       float l = 0.f;
       for (int j = 0; j < ng; ++j) {
         const int tgj = tg + j;
+        // dropout keep bits of this row's 128 keys of tile j, computed while
+        // the scores are still on their way
+        [[maybe_unused]] uint32_t keep[4] = {0u, 0u, 0u, 0u};
+        if constexpr (DROP) {
+          const uint32_t qi = static_cast<uint32_t>(it.tile[g] * C::BM + row);
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4)
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+              keep[c4] |= keep_byte(static_cast<uint32_t>(j * 16 + c4 * 4 + x), qi,
+                                    static_cast<uint32_t>(it.bh), p.drop) << (8 * x);
+        }
         wait_warp(w, bar(FB_SFULL + g), tgj & 1, 8);
         tc_fence_after();
         {
@@ -522,9 +558,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const bool offset = k == 0 && j == 0 && it.n[0] > 0 && it.n[1] > 0;
         if (offset && g == 1) named_bar_sync(kBarOffset, 256);
         if (j == ng - 1)
-          fwd_exp_row<false, PLO>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g));
+          fwd_exp_row<false, PLO, DROP>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g),
+                                        DROP ? keep : nullptr);
         else
-          fwd_exp_row<true, PLO>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g));
+          fwd_exp_row<true, PLO, DROP>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g),
+                                       DROP ? keep : nullptr);
         if (offset && g == 0) named_bar_arrive(kBarOffset, 256);
         float sa, sb, sc2, sd;
         f2_split(sum2[0], sa, sb);
@@ -535,7 +573,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       // -------------------------------------------------------- epilogue
       wait_warp(w, bar(FB_ODONE + g), (tg + ng - 1) & 1, 10);
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      // (DROP: O = P~ V with P~ = P * mask / (1 - p): the keep scale is
+      // applied here, once per row)
+      const float inv_l = DROP ? p.drop.inv_keep / l : 1.f / l;
       // O (and O') into registers; then TMEM is free for the next item
       uint32_t o_all[D / 2], lo_all[PLO ? D / 2 : 1];
 #pragma unroll
@@ -567,9 +607,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       const int tile = it.tile[g];
       const int q_row = tile * C::BM + row;
       if (q_row < p.T) {
-        const long long off = static_cast<long long>(it.bh / p.H) * p.o_sb +
-                              static_cast<long long>(it.bh % p.H) * p.o_sh +
-                              static_cast<long long>(q_row) * p.o_st;
+        const long long off =
+            FLAT ? static_cast<long long>(it.bh) * p.o_sh + static_cast<long long>(q_row) * p.o_st
+                 : static_cast<long long>(it.bh / p.H) * p.o_sb +
+                       static_cast<long long>(it.bh % p.H) * p.o_sh +
+                       static_cast<long long>(q_row) * p.o_st;
         uint4* orow = reinterpret_cast<uint4*>(p.o + off);
 #pragma unroll
         for (int e = 0; e < D / 8; ++e)

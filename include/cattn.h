@@ -194,6 +194,58 @@ CATTN_API cattn_status attn_bwd_strided(const void* q, cattn_layout lq, const vo
                                         cattn_layout ldv, int grad_dtype, void* workspace,
                                         size_t workspace_bytes, void* stream);
 
+/* Attention dropout.
+ *
+ * While training, the pages' CausalSelfAttention passes its dropout rate to
+ * the fused attention ("nanoGPT: a real GPT in two 300-line files",
+ * section 2, model.py; 0.2 for the Shakespeare model in section 3).  It is
+ * inverted dropout on the attention probabilities after the softmax:
+ *
+ *   P~ = P * M / (1 - p),  O = P~ V,  M_ij kept with probability 1 - p,
+ *
+ * LSE is that of the undropped scores, and the backward holds M fixed:
+ * dV = P~^T dO, dP = (dO V^T) * M / (1 - p), dS = P * (dP - Delta).
+ *
+ * M comes from Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random
+ * numbers: as easy as 1, 2, 3", SC 2011), key = (seed low 32 bits, seed
+ * high 32 bits).  Element (b, h, i, j) (query i, key j) uses the block with
+ * counter (j >> 3, i, b*H + h, offset), word (j & 7) >> 1, low 16 bits for
+ * even j and high 16 bits for odd j; it is dropped iff those 16 bits are
+ * below t = round(p * 65536) (t at most 65535), and kept entries are scaled
+ * by 65536 / (65536 - t).  So the drop probability is t / 65536 (p to within
+ * 2^-17) and E[P~] = P exactly.  The mask depends only on (seed, offset,
+ * b*H + h, i, j): the forward and backward of one step must get the same
+ * seed and offset; use another offset (or seed) for every call that wants a
+ * fresh mask (each layer, each step).
+ *
+ * dropout = NULL or p with t = 0 runs the calls without dropout (same
+ * results as the _strided calls).  Errors: CATTN_ERR_INVALID_ARG for p
+ * outside [0, 1) (NaN included), otherwise as the _strided calls.  The
+ * Delta = rowsum(dO * O) of the backward holds with dropout too. */
+typedef struct {
+  float p;                 /* drop probability, 0 <= p < 1 */
+  unsigned long long seed; /* generator key */
+  unsigned int offset;     /* counter word 3 */
+} cattn_dropout;
+
+/* attn_fwd_strided with attention dropout. */
+CATTN_API cattn_status attn_fwd_dropout(const void* q, cattn_layout lq, const void* k,
+                                        cattn_layout lk, const void* v, cattn_layout lv,
+                                        float scale, int B, int H, int T, int D,
+                                        const cattn_dropout* dropout, void* o, cattn_layout lo,
+                                        float* lse, void* o_lo, void* stream);
+
+/* attn_bwd_strided with attention dropout (the forward's dropout argument). */
+CATTN_API cattn_status attn_bwd_dropout(const void* q, cattn_layout lq, const void* k,
+                                        cattn_layout lk, const void* v, cattn_layout lv,
+                                        const void* o, cattn_layout lo, const void* o_lo,
+                                        const float* lse, const void* dout, cattn_layout ldo,
+                                        float scale, int B, int H, int T, int D,
+                                        const cattn_dropout* dropout, void* dq, cattn_layout ldq,
+                                        void* dk, cattn_layout ldk, void* dv, cattn_layout ldv,
+                                        int grad_dtype, void* workspace, size_t workspace_bytes,
+                                        void* stream);
+
 /* Backward pass for callers that cannot allocate device memory.
  *
  * Same computation, arguments and results as attn_bwd, minus the workspace:

@@ -236,3 +236,42 @@ def test_split_qkv_views_share_the_fused_buffer():
     # element (b, h, t, d) of q is qkv[b, t, h*D + d]
     assert float(q[1, 2, 3, 4]) == float(qkv[1, 3, 2 * D + 4])
     assert float(v[0, 3, 5, 1]) == float(qkv[0, 5, 2 * C + 3 * D + 1])
+
+
+# ------------------------------------------------------------ dropout calls
+
+def fwd_dropout(drop, B=1, H=2, T=8, D=64):
+    c = contiguous(H, T, D)
+    return cattn.LIB.attn_fwd_dropout(ALIGNED, c, ALIGNED, c, ALIGNED, c, 0.125, B, H, T, D,
+                                      drop, ALIGNED, c, ALIGNED, None, None)
+
+
+def bwd_dropout(drop, B=1, H=2, T=8, D=64):
+    c = contiguous(H, T, D)
+    return cattn.LIB.attn_bwd_dropout(ALIGNED, c, ALIGNED, c, ALIGNED, c, ALIGNED, c, None,
+                                      ALIGNED, ALIGNED, c, 0.125, B, H, T, D, drop,
+                                      ALIGNED, c, ALIGNED, c, ALIGNED, c, 0, ALIGNED, 1 << 30,
+                                      None)
+
+
+@pytest.mark.parametrize("p", [1.0, -0.01, float("nan"), float("inf"), 7.0])
+def test_dropout_calls_reject_bad_probability(p):
+    import ctypes
+    d = ctypes.byref(_binding.Dropout(p, 1, 2))
+    assert fwd_dropout(d) == cattn.ERR_INVALID_ARG
+    assert bwd_dropout(d) == cattn.ERR_INVALID_ARG
+
+
+def test_dropout_calls_accept_empty_and_null():
+    import ctypes
+    d = ctypes.byref(_binding.Dropout(0.2, 1, 2))
+    assert fwd_dropout(d, T=0) == cattn.OK
+    assert bwd_dropout(d, B=0) == cattn.OK
+    assert fwd_dropout(d, D=48) == cattn.ERR_UNSUPPORTED
+    assert fwd_dropout(None, T=0) == cattn.OK
+
+
+def test_dropout_params_helper():
+    assert cattn.dropout_params(0.0) is None and cattn.dropout_params(None) is None
+    d = cattn.dropout_params(0.2, seed=-1, offset=1 << 33)
+    assert d.seed == (1 << 64) - 1 and d.offset == 0 and abs(d.p - 0.2) < 1e-7

@@ -124,3 +124,30 @@ def test_fp32_gradients_strided(lib):
     assert torch.equal(dks, ref[1]) and torch.equal(dvs, ref[2])
     assert torch.allclose(dqs, ref[0], rtol=1e-5, atol=1e-5 * ref[0].abs().max().item())
     assert not torch.isnan(g).any()
+
+
+def test_plain_and_residual_calls_run_different_kernels(lib):
+    """The plain calls (bf16 P, bf16 dS) and the residual calls (hi/lo P
+    and dS) are different kernels: their outputs differ in low bits.  Guards
+    the dispatch: a plain call that ran the residual kernel would still
+    pass every tolerance test."""
+    B, H, T, D = 1, 4, 384, 64
+    dev = torch.device("cuda:0")
+    q, k, v, do = (t.to(dev) for t in bf16_inputs(B, H, T, D, seed=1001, qk_std=1.0))
+    scale = D ** -0.5
+    for strided in (False, True):
+        if strided:
+            qkv = fused(q, k, v)
+            qs, ks, vs = lib.split_qkv(qkv, H)
+            o1, l1, _ = lib.attn_fwd_strided(qs, ks, vs, scale)
+            o2, l2, olo = lib.attn_fwd_strided(qs, ks, vs, scale, o_lo=torch.empty_like(q))
+            g1 = lib.attn_bwd_strided(qs, ks, vs, o1, l1, do, scale)
+            g2 = lib.attn_bwd_strided(qs, ks, vs, o2, l2, do, scale, o_lo=olo)
+        else:
+            o1, l1 = lib.attn_fwd(q, k, v, scale)
+            o2, l2, olo = lib.attn_fwd_ex(q, k, v, scale)
+            g1 = lib.attn_bwd(q, k, v, o1, l1, do, scale)
+            g2 = lib.attn_bwd(q, k, v, o2, l2, do, scale, o_lo=olo)
+        torch.cuda.synchronize()
+        assert not torch.equal(o1, o2), strided
+        assert not torch.equal(g1[1], g2[1]), strided
