@@ -29,7 +29,7 @@ def header_functions():
     return re.findall(r"^CATTN_API\s+[\w\s\*]+?\b(\w+)\s*\(", src, flags=re.M)
 
 
-def test_header_declares_the_north_star_calls():
+def test_header_declares_the_forward_and_backward_calls():
     names = header_functions()
     for n in ("attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "attn_bwd_preprocess"):
         assert n in names
