@@ -34,7 +34,7 @@ __all__ = [
     "OK", "ERR_INVALID_ARG", "ERR_UNSUPPORTED", "ERR_CUDA", "ERR_TIMEOUT", "ERR_TOO_LARGE",
     "attn_bwd_noalloc", "NOALLOC_SCRATCH_BYTES",
     "attn_fwd_strided", "attn_bwd_strided", "split_qkv", "CausalAttentionQKV", "Layout",
-    "Dropout", "dropout_params",
+    "Dropout", "dropout_params", "attn_decode", "attn_decode_workspace_bytes",
 ]
 
 
@@ -320,6 +320,38 @@ def attn_bwd_strided(q, k, v, o, lse, do, scale=None, dq=None, dk=None, dv=None,
                                   workspace.data_ptr(), workspace.numel(), _stream(stream))
         _check("attn_bwd_dropout", st)
     return dq, dk, dv
+
+
+def attn_decode_workspace_bytes(B, H, Tq, L, D):
+    return int(LIB.attn_decode_workspace_bytes(B, H, Tq, L, D))
+
+
+def attn_decode(q, k, v, L, scale=None, o=None, lse=None, workspace=None, stream=None):
+    """Causal attention of the Tq newest positions against a key/value
+    cache: q (B, H, Tq, D) holds the query rows at positions L-Tq .. L-1,
+    k and v (B, H, >= L, D) views of the cache whose first L rows are the
+    sequence so far (any strides with unit last stride).  Returns (o, lse),
+    o (B, H, Tq, D) bf16 and lse (B, H, Tq) fp32."""
+    B, H, Tq, D = _shape(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    lq, lk, lv = (_layout(t, torch.bfloat16, n) for t, n in ((q, "q"), (k, "k"), (v, "v")))
+    if k.shape[:2] != (B, H) or v.shape[:2] != (B, H) or k.shape[3] != D or v.shape[3] != D:
+        raise ValueError("k, v must be (B, H, >= L, D) views matching q")
+    if k.shape[2] < L or v.shape[2] < L:
+        raise ValueError("the cache holds fewer than L positions")
+    if o is None:
+        o = torch.empty((B, H, Tq, D), dtype=torch.bfloat16, device=q.device)
+    lo = _layout(o, torch.bfloat16, "o")
+    lse = _want(lse, q, torch.float32, (B, H, Tq))
+    need = attn_decode_workspace_bytes(B, H, Tq, L, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = LIB.attn_decode(q.data_ptr(), lq, k.data_ptr(), lk, v.data_ptr(), lv, float(scale),
+                         B, H, Tq, int(L), D, o.data_ptr(), lo, lse.data_ptr(),
+                         workspace.data_ptr(), workspace.numel(), _stream(stream))
+    _check("attn_decode", st)
+    return o, lse
 
 
 class CausalAttentionQKV(torch.autograd.Function):

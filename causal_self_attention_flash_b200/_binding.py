@@ -60,6 +60,9 @@ SIGNATURES = {
                               _vp, _vp]),
     "attn_bwd_dropout": (_i, [_vp, _L, _vp, _L, _vp, _L, _vp, _L, _vp, _vp, _vp, _L, _f,
                               _i, _i, _i, _i, _DP, _vp, _L, _vp, _L, _vp, _L, _i, _vp, _sz, _vp]),
+    "attn_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
+    "attn_decode": (_i, [_vp, _L, _vp, _L, _vp, _L, _f, _i, _i, _i, _i, _i, _vp, _L, _vp, _vp,
+                         _sz, _vp]),
     "cattn_get_device_status": (_i, [_i, _vp]),
     "cattn_set_wait_timeout_us": (None, [_u32]),
     "cattn_selftest_wait_timeout": (_i, [_u32, _vp]),

@@ -12,6 +12,7 @@
 
 #include "cattn.h"
 #include "bwd.cuh"
+#include "decode.cuh"
 #include "fwd.cuh"
 
 // Scratch of attn_bwd_noalloc: one fixed array per device, owned by the
@@ -116,7 +117,6 @@ cattn_status check_shape(int B, int H, int T, int D) {
 
 bool empty_shape(int B, int H, int T) { return B == 0 || H == 0 || T == 0; }
 
-// 3-D tensor map over a contiguous (BH, T, D) tensor: x = d, y = t, z = head.
 // 3-D tensor map {x = d, y = t, z = b*H + h} with element strides t_stride
 // and bh_stride (0: the contiguous D and T*D).
 cattn_status make_tmap(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int elem_bytes,
@@ -530,6 +530,27 @@ __global__ void selftest_wait_kernel(uint64_t timeout_ns) {
   __syncthreads();
 }
 
+// ------------------------------------------------------------------ decode
+
+// Key chunks per head, and the workspace of their partial results.
+int decode_splits(int L) { return (L + kDecodeChunk - 1) / kDecodeChunk; }
+
+size_t decode_ws_bytes(long long BH, int Tq, int L, int D) {
+  const size_t rows = static_cast<size_t>(BH) * decode_splits(L) * Tq;
+  return round256(rows * 2 * sizeof(float)) + round256(rows * D * sizeof(float));
+}
+
+template <int D>
+cattn_status decode_impl(const DecodeParams& p, long long BH, cudaStream_t s) {
+  clear_stale_error();
+  dim3 grid(static_cast<unsigned>(BH), static_cast<unsigned>(p.n_split));
+  decode_partial_kernel<D><<<grid, kDecodeWarps * 32, 0, s>>>(p);
+  cattn_status st = launch_status();
+  if (st != CATTN_OK) return st;
+  decode_combine_kernel<D><<<static_cast<unsigned>(BH * p.Tq), D, 0, s>>>(p);
+  return launch_status();
+}
+
 }  // namespace
 }  // namespace cattn
 
@@ -585,6 +606,62 @@ cattn_status attn_fwd_ex(const void* q, const void* k, const void* v, float scal
 cattn_status attn_fwd(const void* q, const void* k, const void* v, float scale, int B, int H,
                       int T, int D, void* o, float* lse, void* stream) {
   return attn_fwd_ex(q, k, v, scale, B, H, T, D, o, lse, nullptr, stream);
+}
+
+size_t attn_decode_workspace_bytes(int B, int H, int Tq, int L, int D) {
+  if (check_shape(B, H, L, D) != CATTN_OK || Tq < 1 || Tq > kDecodeMaxTq || L < Tq) return 0;
+  if (empty_shape(B, H, L)) return 0;
+  return decode_ws_bytes(static_cast<long long>(B) * H, Tq, L, D);
+}
+
+cattn_status attn_decode(const void* q, cattn_layout lq, const void* k, cattn_layout lk,
+                         const void* v, cattn_layout lv, float scale, int B, int H, int Tq, int L,
+                         int D, void* o, cattn_layout lo, float* lse, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  cattn_status st = check_shape(B, H, L, D);
+  if (st != CATTN_OK) return st;
+  if (!(scale > 0.f) || !isfinite(scale)) return CATTN_ERR_INVALID_ARG;
+  if (Tq > kDecodeMaxTq) return CATTN_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0) return CATTN_OK;
+  if (Tq < 1 || L < Tq) return CATTN_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !lse || !workspace) return CATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4) || !aligned(workspace, 256))
+    return CATTN_ERR_INVALID_ARG;
+  if (!layout_ok(lq) || !layout_ok(lk) || !layout_ok(lv) || !layout_ok(lo))
+    return CATTN_ERR_INVALID_ARG;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH * Tq > 0x7fffffffLL) return CATTN_ERR_INVALID_ARG;
+  if (workspace_bytes < decode_ws_bytes(BH, Tq, L, D)) return CATTN_ERR_INVALID_ARG;
+  int dev;
+  if ((st = check_device(&dev)) != CATTN_OK) return st;
+  DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.q_sb = lq.b; p.q_sh = lq.h; p.q_st = lq.t;
+  p.k_sb = lk.b; p.k_sh = lk.h; p.k_st = lk.t;
+  p.v_sb = lv.b; p.v_sh = lv.h; p.v_st = lv.t;
+  const size_t rows = static_cast<size_t>(BH) * decode_splits(L) * Tq;
+  uint8_t* wb = static_cast<uint8_t*>(workspace);
+  p.part_ml = reinterpret_cast<float*>(wb);
+  p.part_o = reinterpret_cast<float*>(wb + round256(rows * 2 * sizeof(float)));
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_sb = lo.b; p.o_sh = lo.h; p.o_st = lo.t;
+  p.lse = lse;
+  p.H = H;
+  p.Tq = Tq;
+  p.L = L;
+  p.n_split = decode_splits(L);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (D) {
+    case 16: return decode_impl<16>(p, BH, s);
+    case 32: return decode_impl<32>(p, BH, s);
+    case 64: return decode_impl<64>(p, BH, s);
+    case 128: return decode_impl<128>(p, BH, s);
+  }
+  return CATTN_ERR_UNSUPPORTED;
 }
 
 size_t attn_bwd_workspace_bytes(int B, int H, int T, int D) {

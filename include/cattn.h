@@ -246,6 +246,37 @@ CATTN_API cattn_status attn_bwd_dropout(const void* q, cattn_layout lq, const vo
                                         int grad_dtype, void* workspace, size_t workspace_bytes,
                                         void* stream);
 
+/* Decode attention over a key/value cache.
+ *
+ * generate() in "nanoGPT: a real GPT in two 300-line files" (section 2,
+ * "How the code works") runs the model once per new token; with a
+ * key/value cache (as nanochat's inference does, "Karpathy's nano lineage:
+ * nanoGPT, llm.c, and nanochat") a step needs causal attention only for the
+ * Tq newest positions.  attn_decode computes it for query rows at positions
+ * L - Tq .. L - 1 of a sequence whose first L keys and values are in k and
+ * v: row r sees keys 0 .. L - Tq + r.  The result is exactly the last Tq
+ * rows of attn_fwd over the whole sequence (up to rounding).
+ *
+ *   q      bf16 (B, H, Tq, D), layout lq
+ *   k, v   bf16 (B, H, >= L, D), layouts lk, lv (rows beyond L are not
+ *          read; a (B, Tmax, H, D) cache is { Tmax*H*D, D, H*D })
+ *   o      bf16 (B, H, Tq, D) out, layout lo;  lse fp32 (B, H, Tq) out,
+ *          contiguous, natural log
+ *   workspace  attn_decode_workspace_bytes(B, H, Tq, L, D) bytes of device
+ *          memory, 256-byte aligned (the per-chunk partial results)
+ *
+ * The keys of each head are processed in chunks of 256 by separate CTAs and
+ * merged by a second kernel; both run on `stream`.  1 <= Tq <= L; Tq above
+ * 8 returns CATTN_ERR_UNSUPPORTED (use attn_fwd for a prefill).  Layout
+ * rules as for the _strided calls; B = 0 or H = 0 is a no-op. */
+CATTN_API size_t attn_decode_workspace_bytes(int B, int H, int Tq, int L, int D);
+
+CATTN_API cattn_status attn_decode(const void* q, cattn_layout lq, const void* k,
+                                   cattn_layout lk, const void* v, cattn_layout lv, float scale,
+                                   int B, int H, int Tq, int L, int D, void* o, cattn_layout lo,
+                                   float* lse, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
 /* Backward pass for callers that cannot allocate device memory.
  *
  * Same computation, arguments and results as attn_bwd, minus the workspace:

@@ -275,3 +275,33 @@ def test_dropout_params_helper():
     assert cattn.dropout_params(0.0) is None and cattn.dropout_params(None) is None
     d = cattn.dropout_params(0.2, seed=-1, offset=1 << 33)
     assert d.seed == (1 << 64) - 1 and d.offset == 0 and abs(d.p - 0.2) < 1e-7
+
+
+# ------------------------------------------------------------ decode call
+
+def decode(Tq=1, L=8, B=1, H=2, D=64, lay=None, ws_bytes=1 << 20):
+    c = _binding.Layout(H * L * D, L * D, D)
+    return cattn.LIB.attn_decode(ALIGNED, lay or c, ALIGNED, c, ALIGNED, c, 0.125, B, H, Tq, L,
+                                 D, ALIGNED, c, ALIGNED, ALIGNED, ws_bytes, None)
+
+
+def test_decode_checks_arguments_before_the_device():
+    assert decode(Tq=9) == cattn.ERR_UNSUPPORTED
+    assert decode(Tq=0) == cattn.ERR_INVALID_ARG
+    assert decode(Tq=4, L=3) == cattn.ERR_INVALID_ARG
+    assert decode(D=48) == cattn.ERR_UNSUPPORTED
+    assert decode(B=0) == cattn.OK
+    assert decode(lay=_binding.Layout(512, 64, 12)) == cattn.ERR_INVALID_ARG
+    assert decode(ws_bytes=16) == cattn.ERR_INVALID_ARG
+
+
+def test_decode_workspace_formula():
+    # per (head, chunk of 256 keys, query row): (m, l) and D partial outputs
+    def r256(x):
+        return (x + 255) // 256 * 256
+    for B, H, Tq, L, D in [(1, 1, 1, 1, 16), (2, 3, 4, 257, 64), (16, 12, 1, 1024, 64),
+                           (1, 2, 8, 4096, 128)]:
+        rows = B * H * ((L + 255) // 256) * Tq
+        assert cattn.attn_decode_workspace_bytes(B, H, Tq, L, D) == r256(rows * 8) + r256(rows * D * 4)
+    assert cattn.attn_decode_workspace_bytes(1, 1, 9, 16, 64) == 0
+    assert cattn.attn_decode_workspace_bytes(1, 1, 2, 1, 64) == 0

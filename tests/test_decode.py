@@ -1,0 +1,73 @@
+"""GPU parity of decode attention (attn_decode) against the fp64 decode
+oracle: the Tq newest query rows of a sequence against its first L cached
+keys and values, with contiguous and (B, Tmax, H, D) cache layouts."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.decode as odec
+from parity_util import check_bf16, check_lse
+from workloads import as_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def draw(seed, *shape):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn(*shape, generator=g).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("B,H,L,Tq,D", [(1, 2, 1, 1, 16), (2, 3, 300, 1, 64), (2, 2, 257, 8, 128),
+                                         (1, 4, 513, 2, 32), (2, 2, 64, 8, 16), (3, 2, 1000, 4, 64),
+                                         (1, 2, 4096, 1, 128), (16, 12, 1024, 1, 64)])
+@pytest.mark.parametrize("cache_layout", ["bhtd", "bthd"])
+def test_decode_against_oracle(lib, B, H, L, Tq, D, cache_layout):
+    dev = torch.device("cuda:0")
+    Tmax = L + 37                       # cache capacity beyond the live length
+    q = draw(11 + L, B, H, Tq, D)
+    if cache_layout == "bhtd":
+        k = draw(12 + L, B, H, Tmax, D)
+        v = draw(13 + L, B, H, Tmax, D)
+        kd, vd = k.to(dev), v.to(dev)
+    else:                               # (B, Tmax, H, D) storage, (B, H, Tmax, D) views
+        k = draw(12 + L, B, Tmax, H, D).transpose(1, 2)
+        v = draw(13 + L, B, Tmax, H, D).transpose(1, 2)
+        kd = k.transpose(1, 2).contiguous().to(dev).transpose(1, 2)
+        vd = v.transpose(1, 2).contiguous().to(dev).transpose(1, 2)
+        assert kd.stride(2) == H * D
+    # poison the rows past L: they must not be read into the result
+    kd[:, :, L:] = float("nan")
+    vd[:, :, L:] = float("nan")
+    scale = D ** -0.5
+    o, lse = lib.attn_decode(q.to(dev), kd, vd, L, scale)
+    torch.cuda.synchronize()
+    ro, rl = odec.decode_attention(as_f64(q), as_f64(k), as_f64(v), scale, L)
+    check_bf16("o", as_f64(o), ro)
+    check_lse(as_f64(lse), rl)
+
+
+def test_decode_matches_forward_rows(lib):
+    """the decode of the last rows agrees with the full forward's last rows"""
+    B, H, T, D, Tq = 2, 3, 700, 64, 5
+    dev = torch.device("cuda:0")
+    q, k, v = (draw(s, B, H, T, D).to(dev) for s in (21, 22, 23))
+    o_full, lse_full = lib.attn_fwd(q, k, v)
+    o, lse = lib.attn_decode(q[:, :, T - Tq:].contiguous(), k, v, T)
+    torch.cuda.synchronize()
+    assert torch.allclose(lse, lse_full[:, :, T - Tq:], atol=1e-4, rtol=0)
+    diff = (o.float() - o_full[:, :, T - Tq:].float()).abs().max().item()
+    assert diff < 2e-2, diff
+
+
+def test_decode_argument_errors(lib):
+    dev = torch.device("cuda:0")
+    q = torch.zeros(1, 1, 9, 64, dtype=torch.bfloat16, device=dev)
+    k = torch.zeros(1, 1, 16, 64, dtype=torch.bfloat16, device=dev)
+    with pytest.raises(lib.CattnError):        # Tq above 8
+        lib.attn_decode(q, k, k, 16)
+    with pytest.raises(lib.CattnError):        # L < Tq
+        lib.attn_decode(q[:, :, :4], k, k, 3)
+    ws = torch.empty(16, dtype=torch.uint8, device=dev)
+    with pytest.raises(lib.CattnError):        # workspace too small
+        lib.attn_decode(q[:, :, :1], k, k, 16, workspace=ws)
