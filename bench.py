@@ -353,7 +353,59 @@ def measure_detail(args, w, sets, olos, step, stream, cattn):
                                         "ms_median": pct(sd, 0.5)}
     except Exception as e:  # noqa: BLE001  (context only)
         detail["context_torch_sdpa"] = {"unavailable": str(e)[:120]}
+    try:
+        detail["decode"] = measure_decode(w, sets, stream, cattn, n)
+    except Exception as e:  # noqa: BLE001  (a side measurement; the step stands)
+        detail["decode"] = {"unavailable": str(e)[:120]}
     return detail
+
+
+def decode_bytes(B, H, L, D, Tq=1) -> int:
+    """Compulsory HBM bytes of one decode call: the L cached K and V rows of
+    every head (bf16), the Tq query rows and outputs (bf16), LSE (fp32)."""
+    return 2 * B * H * L * D * 2 + 2 * B * H * Tq * D * 2 + B * H * Tq * 4
+
+
+def measure_decode(w, sets, stream, cattn, n):
+    """attn_decode of the newest position (Tq = 1) against the whole
+    sequence's K and V as the cache, rotating over the input sets (their
+    K, V together exceed L2); device time from the library's own timer."""
+    import ctypes
+    B, H, T, D = w.B, w.H, w.T, w.D
+    ws = torch.empty(max(cattn.attn_decode_workspace_bytes(B, H, 1, T, D), 1),
+                     dtype=torch.uint8, device=sets[0][0].device)
+    outs = [(torch.empty((B, H, 1, D), dtype=torch.bfloat16, device=ws.device),
+             torch.empty((B, H, 1), dtype=torch.float32, device=ws.device))
+            for _ in range(N_SETS)]
+
+    def call(i):
+        qd, kd, vd = sets[i % N_SETS][:3]
+        o, lse = outs[i % N_SETS]
+        cattn.attn_decode(qd[:, :, T - 1:], kd, vd, T, w.scale, o=o, lse=lse, workspace=ws,
+                          stream=stream)
+
+    for i in range(N_SETS):
+        call(i)
+    torch.cuda.synchronize()
+    ms = (ctypes.c_float * 5)()
+    cnt = (ctypes.c_int * 5)()
+    cattn.LIB.cattn_timing_enable(1)
+    cattn.LIB.cattn_timing_read(ms, cnt, 5)
+    for i in range(n):
+        call(i)
+    torch.cuda.synchronize()
+    st = cattn.LIB.cattn_timing_read(ms, cnt, 5)
+    cattn.LIB.cattn_timing_enable(0)
+    if st != 0 or cnt[4] == 0:
+        return {"unavailable": f"timer status {st}, {cnt[4]} launches"}
+    per_ms = ms[4] / cnt[4]
+    byts = decode_bytes(B, H, T, D)
+    peaks, src = load_peaks()
+    gbs = byts / (per_ms / 1e3) / 1e9
+    return {"shape": f"B={B} H={H} L={T} D={D} Tq=1", "us_per_call": per_ms * 1e3,
+            "calls": cnt[4], "bytes_per_call": byts, "gbs": gbs,
+            "frac_of_hbm": gbs / peaks["hbm_gbs"], "peak_source": src,
+            "kernels": "decode_partial_kernel + decode_combine_kernel"}
 
 
 def run_cattn(args, w, index, world, rank, local):

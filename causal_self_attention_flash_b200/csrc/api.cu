@@ -216,7 +216,9 @@ int grid_for(size_t work_items, int per_block) {
 // Optional CUDA-event timing of each launch, on the launching stream (a
 // benchmarking aid; off by default, and then it costs nothing).
 
-enum KernelId { K_FWD = 0, K_BWD_PRE = 1, K_BWD_MAIN = 2, K_DQ_CONVERT = 3, K_COUNT = 4 };
+enum KernelId {
+  K_FWD = 0, K_BWD_PRE = 1, K_BWD_MAIN = 2, K_DQ_CONVERT = 3, K_DECODE = 4, K_COUNT = 5
+};
 
 bool g_timing = false;
 struct TimingRec {
@@ -544,6 +546,7 @@ template <int D>
 cattn_status decode_impl(const DecodeParams& p, long long BH, cudaStream_t s) {
   clear_stale_error();
   dim3 grid(static_cast<unsigned>(BH), static_cast<unsigned>(p.n_split));
+  LaunchTimer t(K_DECODE, s);  // both kernels, as one entry
   decode_partial_kernel<D><<<grid, kDecodeWarps * 32, 0, s>>>(p);
   cattn_status st = launch_status();
   if (st != CATTN_OK) return st;

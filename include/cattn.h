@@ -337,7 +337,8 @@ CATTN_API cattn_status cattn_selftest_wait_timeout(uint32_t timeout_us, void* st
  * launching stream.  cattn_timing_read() waits for the recorded events and
  * returns, per kernel, the summed device time in ms and the launch count,
  * then forgets them.  Kernel index: 0 forward, 1 backward preprocess,
- * 2 backward main, 3 dQ convert.  n = length of both output arrays.  Not
+ * 2 backward main, 3 dQ convert, 4 decode (its two kernels together).
+ * n = length of both output arrays (indices >= n are dropped).  Not
  * for use while a stream is being captured into a CUDA graph. */
 CATTN_API void cattn_timing_enable(int enable);
 CATTN_API cattn_status cattn_timing_read(float* total_ms, int* launches, int n);

@@ -47,3 +47,12 @@ def test_kernel_algorithmic_units(bench):
     amount, unit, bound = bench.kernel_algorithmic(w, "dq_convert_kernel")
     assert (unit, bound) == ("byte", "hbm")
     assert amount == w.B * w.H * w.T * w.D * 6   # fp32 read + bf16 write
+
+
+def test_decode_bytes(bench):
+    # GPT-2 layer as a cache: K and V of 16 x 12 heads x 1024 positions x 64
+    # (bf16), plus one query row, one output row and one LSE per head
+    kv = 2 * 16 * 12 * 1024 * 64 * 2
+    assert bench.decode_bytes(16, 12, 1024, 64) == kv + 2 * 16 * 12 * 64 * 2 + 16 * 12 * 4
+    assert bench.decode_bytes(16, 12, 1024, 64) == pytest.approx(50.4e6, rel=1e-3)
+    assert bench.decode_bytes(1, 1, 1, 16, 1) == 2 * 16 * 2 + 2 * 16 * 2 + 4
