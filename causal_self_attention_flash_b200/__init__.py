@@ -56,17 +56,60 @@ def _shape(q):
 
 
 def _want(t, like, dtype, shape):
+    """An output buffer: allocated like `like` if None, else checked (the
+    library writes through its pointer, so it must be device memory of the
+    right size on like's device)."""
     if t is None:
         return torch.empty(shape, dtype=dtype, device=like.device)
     if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
-        raise ValueError(f"output must be contiguous {dtype} of shape {shape}")
+        raise ValueError(f"output must be contiguous {dtype} of shape {tuple(shape)}")
+    if not t.is_cuda or t.device != like.device:
+        raise ValueError(f"output must be on {like.device}")
     return t
 
 
+def _same_device(ref):
+    if ref.device.index != torch.cuda.current_device():
+        raise ValueError(f"tensors are on {ref.device}, the current device is "
+                         f"cuda:{torch.cuda.current_device()}: call under torch.cuda.device")
+
+
 def _inputs(*ts):
+    """Inputs: one (B, H, T, D) shape (the first tensor's), then contiguous
+    bf16 tensors on the current CUDA device."""
+    ref = ts[0]
+    for t in ts:
+        if t.dim() != 4 or tuple(t.shape) != tuple(ref.shape):
+            raise ValueError(f"inputs must share the (B, H, T, D) shape {tuple(ref.shape)}, "
+                             f"got {tuple(t.shape)}")
     for t in ts:
         if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
             raise ValueError("inputs must be contiguous bf16 CUDA tensors")
+        if t.device != ref.device:
+            raise ValueError("inputs must be on one device")
+    _same_device(ref)
+
+
+def _vector(x, like, shape, what):
+    """A contiguous fp32 (B, H, T) input such as LSE, on like's device."""
+    if tuple(x.shape) != tuple(shape):
+        raise ValueError(f"{what} must have shape {tuple(shape)}, got {tuple(x.shape)}")
+    if x.dtype != torch.float32 or not x.is_contiguous() or not x.is_cuda or x.device != like.device:
+        raise ValueError(f"{what} must be contiguous fp32 on {like.device}")
+
+
+def _workspace(ws, like, need):
+    """A caller-given workspace: device memory on like's device; returns its
+    size in bytes (the library checks it against `need`)."""
+    if ws is None:
+        return torch.empty(max(need, 1), dtype=torch.uint8, device=like.device)
+    if not ws.is_cuda or ws.device != like.device or not ws.is_contiguous():
+        raise ValueError(f"workspace must be contiguous device memory on {like.device}")
+    return ws
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
 
 
 def attn_fwd_ex(q, k, v, scale=None, o=None, lse=None, o_lo=None, want_o_lo=True,
@@ -128,31 +171,28 @@ def attn_bwd(q, k, v, o, lse, do, scale=None, dq=None, dk=None, dv=None,
     B, H, T, D = _shape(q)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    if lse.dtype != torch.float32 or not lse.is_contiguous():
-        raise ValueError("lse must be contiguous fp32 (B, H, T)")
+    _vector(lse, q, (B, H, T), "lse")
     if grad_dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("grad_dtype must be torch.bfloat16 or torch.float32")
     dq = _want(dq, q, grad_dtype, (B, H, T, D))
     dk = _want(dk, q, grad_dtype, (B, H, T, D))
     dv = _want(dv, q, grad_dtype, (B, H, T, D))
-    need = attn_bwd_workspace_bytes(B, H, T, D)
-    if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    workspace = _workspace(workspace, q, attn_bwd_workspace_bytes(B, H, T, D))
     if o_lo is None and grad_dtype == torch.bfloat16:
         st = LIB.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                           lse.data_ptr(), do.data_ptr(), float(scale), B, H, T, D,
                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
-                          workspace.numel(), _stream(stream))
+                          _nbytes(workspace), _stream(stream))
         _check("attn_bwd", st)
     else:
         if o_lo is not None:
-            _inputs(o_lo)
+            _inputs(q, o_lo)
         st = LIB.attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                              o_lo.data_ptr() if o_lo is not None else None, lse.data_ptr(),
                              do.data_ptr(), float(scale), B, H, T, D, dq.data_ptr(),
                              dk.data_ptr(), dv.data_ptr(),
                              1 if grad_dtype == torch.float32 else 0,
-                             workspace.data_ptr(), workspace.numel(), _stream(stream))
+                             workspace.data_ptr(), _nbytes(workspace), _stream(stream))
         _check("attn_bwd_ex", st)
     return dq, dk, dv
 
@@ -170,6 +210,7 @@ def attn_bwd_noalloc(q, k, v, o, lse, do, scale=None, dq=None, dk=None, dv=None,
     B, H, T, D = _shape(q)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
+    _vector(lse, q, (B, H, T), "lse")
     dq = _want(dq, q, torch.bfloat16, (B, H, T, D))
     dk = _want(dk, q, torch.bfloat16, (B, H, T, D))
     dv = _want(dv, q, torch.bfloat16, (B, H, T, D))
@@ -217,12 +258,17 @@ def cattn_version() -> int:
     return int(LIB.cattn_version())
 
 
-def _layout(t, dtype, what):
-    """cattn_layout of a (B, H, T, D) view whose last stride is 1."""
+def _layout(t, dtype, what, shape=None, device=None):
+    """cattn_layout of a (B, H, T, D) view whose last stride is 1 (checked
+    against the expected shape and device when given)."""
     if t.dim() != 4 or t.stride(3) != 1:
         raise ValueError(f"{what}: expected a (B, H, T, D) view with unit last stride")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{what}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
     if t.dtype != dtype or not t.is_cuda:
         raise ValueError(f"{what}: expected a {dtype} CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{what}: expected a tensor on {device}")
     return Layout(t.stride(0), t.stride(1), t.stride(2))
 
 
@@ -253,12 +299,17 @@ def attn_fwd_strided(q, k, v, scale=None, o=None, lse=None, o_lo=None, stream=No
     B, H, T, D = _shape(q)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    lq, lk, lv = (_layout(t, torch.bfloat16, n) for t, n in ((q, "q"), (k, "k"), (v, "v")))
+    shp = (B, H, T, D)
+    lq, lk, lv = (_layout(t, torch.bfloat16, n, shp, q.device)
+                  for t, n in ((q, "q"), (k, "k"), (v, "v")))
+    _same_device(q)
     if o is None:
-        o = torch.empty((B, H, T, D), dtype=torch.bfloat16, device=q.device)
-    lo = _layout(o, torch.bfloat16, "o")
-    if o_lo is not None and (o_lo.stride() != o.stride() or o_lo.dtype != torch.bfloat16):
-        raise ValueError("o_lo must be a bf16 view with o's strides")
+        o = torch.empty(shp, dtype=torch.bfloat16, device=q.device)
+    lo = _layout(o, torch.bfloat16, "o", shp, q.device)
+    if o_lo is not None:
+        _layout(o_lo, torch.bfloat16, "o_lo", shp, q.device)
+        if o_lo.stride() != o.stride():
+            raise ValueError("o_lo must be a bf16 view with o's strides")
     lse = _want(lse, q, torch.float32, (B, H, T))
     olo_ptr = o_lo.data_ptr() if o_lo is not None else None
     if dropout is None:
@@ -284,23 +335,24 @@ def attn_bwd_strided(q, k, v, o, lse, do, scale=None, dq=None, dk=None, dv=None,
     B, H, T, D = _shape(q)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    if lse.dtype != torch.float32 or not lse.is_contiguous():
-        raise ValueError("lse must be contiguous fp32 (B, H, T)")
+    shp = (B, H, T, D)
     if grad_dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("grad_dtype must be torch.bfloat16 or torch.float32")
-    ins = [_layout(t, torch.bfloat16, n)
+    ins = [_layout(t, torch.bfloat16, n, shp, q.device)
            for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do"))]
-    if o_lo is not None and (o_lo.stride() != o.stride() or o_lo.dtype != torch.bfloat16):
-        raise ValueError("o_lo must be a bf16 view with o's strides")
+    _same_device(q)
+    _vector(lse, q, (B, H, T), "lse")
+    if o_lo is not None:
+        _layout(o_lo, torch.bfloat16, "o_lo", shp, q.device)
+        if o_lo.stride() != o.stride():
+            raise ValueError("o_lo must be a bf16 view with o's strides")
     outs = []
     for t in (dq, dk, dv):
-        outs.append(t if t is not None else
-                    torch.empty((B, H, T, D), dtype=grad_dtype, device=q.device))
+        outs.append(t if t is not None else torch.empty(shp, dtype=grad_dtype, device=q.device))
     dq, dk, dv = outs
-    louts = [_layout(t, grad_dtype, n) for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv"))]
-    need = attn_bwd_workspace_bytes(B, H, T, D)
-    if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    louts = [_layout(t, grad_dtype, n, shp, q.device)
+             for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv"))]
+    workspace = _workspace(workspace, q, attn_bwd_workspace_bytes(B, H, T, D))
     olo_ptr = o_lo.data_ptr() if o_lo is not None else None
     f32 = 1 if grad_dtype == torch.float32 else 0
     if dropout is None:
@@ -309,7 +361,7 @@ def attn_bwd_strided(q, k, v, o, lse, do, scale=None, dq=None, dk=None, dv=None,
                                   do.data_ptr(), ins[4], float(scale), B, H, T, D,
                                   dq.data_ptr(), louts[0], dk.data_ptr(), louts[1],
                                   dv.data_ptr(), louts[2], f32,
-                                  workspace.data_ptr(), workspace.numel(), _stream(stream))
+                                  workspace.data_ptr(), _nbytes(workspace), _stream(stream))
         _check("attn_bwd_strided", st)
     else:
         st = LIB.attn_bwd_dropout(q.data_ptr(), ins[0], k.data_ptr(), ins[1], v.data_ptr(),
@@ -317,7 +369,7 @@ def attn_bwd_strided(q, k, v, o, lse, do, scale=None, dq=None, dk=None, dv=None,
                                   do.data_ptr(), ins[4], float(scale), B, H, T, D,
                                   ctypes.byref(dropout), dq.data_ptr(), louts[0],
                                   dk.data_ptr(), louts[1], dv.data_ptr(), louts[2], f32,
-                                  workspace.data_ptr(), workspace.numel(), _stream(stream))
+                                  workspace.data_ptr(), _nbytes(workspace), _stream(stream))
         _check("attn_bwd_dropout", st)
     return dq, dk, dv
 
@@ -335,21 +387,23 @@ def attn_decode(q, k, v, L, scale=None, o=None, lse=None, workspace=None, stream
     B, H, Tq, D = _shape(q)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    lq, lk, lv = (_layout(t, torch.bfloat16, n) for t, n in ((q, "q"), (k, "k"), (v, "v")))
-    if k.shape[:2] != (B, H) or v.shape[:2] != (B, H) or k.shape[3] != D or v.shape[3] != D:
-        raise ValueError("k, v must be (B, H, >= L, D) views matching q")
-    if k.shape[2] < L or v.shape[2] < L:
-        raise ValueError("the cache holds fewer than L positions")
+    for t, n in ((k, "k"), (v, "v")):
+        if t.dim() != 4 or tuple(t.shape[:2]) != (B, H) or t.shape[3] != D:
+            raise ValueError(f"{n} must be a (B, H, >= L, D) view matching q")
+        if t.shape[2] < L:
+            raise ValueError(f"{n}: the cache holds fewer than L positions")
+    lq = _layout(q, torch.bfloat16, "q", None, q.device)
+    lk = _layout(k, torch.bfloat16, "k", None, q.device)
+    lv = _layout(v, torch.bfloat16, "v", None, q.device)
+    _same_device(q)
     if o is None:
         o = torch.empty((B, H, Tq, D), dtype=torch.bfloat16, device=q.device)
-    lo = _layout(o, torch.bfloat16, "o")
+    lo = _layout(o, torch.bfloat16, "o", (B, H, Tq, D), q.device)
     lse = _want(lse, q, torch.float32, (B, H, Tq))
-    need = attn_decode_workspace_bytes(B, H, Tq, L, D)
-    if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    workspace = _workspace(workspace, q, attn_decode_workspace_bytes(B, H, Tq, L, D))
     st = LIB.attn_decode(q.data_ptr(), lq, k.data_ptr(), lk, v.data_ptr(), lv, float(scale),
                          B, H, Tq, int(L), D, o.data_ptr(), lo, lse.data_ptr(),
-                         workspace.data_ptr(), workspace.numel(), _stream(stream))
+                         workspace.data_ptr(), _nbytes(workspace), _stream(stream))
     _check("attn_decode", st)
     return o, lse
 

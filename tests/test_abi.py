@@ -305,3 +305,38 @@ def test_decode_workspace_formula():
         assert cattn.attn_decode_workspace_bytes(B, H, Tq, L, D) == r256(rows * 8) + r256(rows * D * 4)
     assert cattn.attn_decode_workspace_bytes(1, 1, 9, 16, 64) == 0
     assert cattn.attn_decode_workspace_bytes(1, 1, 2, 1, 64) == 0
+
+
+# ------------------------------------------------------------ Python checks
+
+def test_python_calls_reject_mismatched_shapes_before_any_launch():
+    import torch as t
+    q = t.zeros(1, 2, 16, 64, dtype=t.bfloat16)
+    short = t.zeros(1, 2, 8, 64, dtype=t.bfloat16)
+    with pytest.raises(ValueError, match="share the"):
+        cattn.attn_fwd(q, short, q)
+    with pytest.raises(ValueError, match="share the"):
+        cattn.attn_fwd_ex(q, q, short)
+    lse = t.zeros(1, 2, 16)
+    with pytest.raises(ValueError, match="share the"):
+        cattn.attn_bwd(q, q, q, q, lse, short)
+    with pytest.raises(ValueError, match="share the"):
+        cattn.attn_bwd_noalloc(q, q, short, q, lse, q)
+    with pytest.raises(ValueError, match="share the"):
+        cattn.attn_bwd_preprocess(q, short)
+
+
+def test_python_buffers_must_be_device_memory_of_the_right_shape():
+    import torch as t
+    like = t.zeros(1, 2, 16, 64, dtype=t.bfloat16)
+    with pytest.raises(ValueError, match="output must be on"):
+        cattn._want(t.zeros(1, 2, 16, 64, dtype=t.bfloat16), like, t.bfloat16, (1, 2, 16, 64))
+    with pytest.raises(ValueError, match="shape"):
+        cattn._want(t.zeros(1, 2, 8, 64, dtype=t.bfloat16), like, t.bfloat16, (1, 2, 16, 64))
+    with pytest.raises(ValueError, match="workspace"):
+        cattn._workspace(t.zeros(1024, dtype=t.uint8), like, 512)
+    with pytest.raises(ValueError, match="lse must have shape"):
+        cattn._vector(t.zeros(1, 2, 8), like, (1, 2, 16), "lse")
+    with pytest.raises(ValueError, match="fp32"):
+        cattn._vector(t.zeros(1, 2, 16), like, (1, 2, 16), "lse")   # a CPU tensor
+    assert cattn._nbytes(t.zeros(10, dtype=t.float32)) == 40
