@@ -191,11 +191,13 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(world, x: float) -> float:
+def max_over_ranks(world, x: float, device: str = "cuda") -> float:
+    """The maximum of x over all ranks (every rank gets it); device is where
+    the reduction tensor lives ("cuda" for NCCL, "cpu" for gloo)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
