@@ -35,6 +35,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import sys
 import threading
@@ -80,14 +81,29 @@ KERNEL_SOURCES = {
 }
 
 
+def code_only(src: str) -> str:
+    """C++ source without its comments and blank lines (so that a comment
+    edit does not count as a change of the kernel)."""
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    lines = []
+    for line in src.splitlines():
+        cut = line.find("//")
+        if cut >= 0 and line.count('"', 0, cut) % 2 == 0:
+            line = line[:cut]
+        if line.strip():
+            lines.append(line.rstrip())
+    return "\n".join(lines)
+
+
 def source_hash(kernel: str) -> str:
-    """Hash of the device sources a kernel is compiled from (its ncu traffic
-    figure is reported only while this matches the one stored with it)."""
+    """Hash of the device code a kernel is compiled from, comments aside
+    (its ncu traffic figure is reported only while this matches the one
+    stored with it)."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(CSRC, f), "rb") as fh:
+        with open(os.path.join(CSRC, f), encoding="utf-8") as fh:
             h.update(f.encode())
-            h.update(fh.read())
+            h.update(code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -27,6 +27,18 @@
 // precision) or also as a hi/lo pair (SLO = true, used with the forward's
 // O_lo residual or with fp32 gradient outputs, where the aim is gradients
 // accurate to ~fp32).
+//
+// Instances bwd_kernel<D, SLO, DROP, FLAT>:
+//   DROP   attention dropout with the forward's mask (philox.cuh): a compute
+//          thread owns one key and 32 queries, so each lane draws the bits
+//          of 8 keys for one query and a warp shuffle per query hands every
+//          lane its own bit; dV takes the dropped P^T (the keep scale is
+//          applied in the epilogue) and dS = P * (dP~ * mask / (1 - p) -
+//          Delta).
+//   FLAT   Q, K, V, dO, dK and dV address (b, h) as one b*H + h index (3-D
+//          tensor maps); otherwise 4-D maps take any element strides.
+// bwd_pre_kernel<D, CONTIG> and the dQ convert have contiguous and strided
+// forms too.
 #pragma once
 
 #include "philox.cuh"

@@ -53,6 +53,15 @@
 // more than 8 (log2 units).  The exponentials then stay below 2^8, and
 // because O and l are accumulated against the same m the final O / l is
 // unchanged: it is still exactly the softmax, as the online rewrite is.
+//
+// Instances fwd_kernel<D, PLO, DROP, FLAT>:
+//   DROP   attention dropout (philox.cuh): each softmax thread draws its
+//          row's keep bits for a key tile before that tile's scores arrive,
+//          writes the dropped P entries as 0 (the row sum l still takes
+//          every entry) and folds the keep scale 1 / (1 - p) into 1 / l.
+//   FLAT   Q, K, V and O address (b, h) as one b*H + h index (3-D tensor
+//          maps); otherwise 4-D maps {d, t, h, b} take any element strides,
+//          e.g. q, k, v as views into one fused (B, T, 3C) projection.
 #pragma once
 
 #include "philox.cuh"

@@ -56,3 +56,21 @@ def test_decode_bytes(bench):
     assert bench.decode_bytes(16, 12, 1024, 64) == kv + 2 * 16 * 12 * 64 * 2 + 16 * 12 * 4
     assert bench.decode_bytes(16, 12, 1024, 64) == pytest.approx(50.4e6, rel=1e-3)
     assert bench.decode_bytes(1, 1, 1, 16, 1) == 2 * 16 * 2 + 2 * 16 * 2 + 4
+
+
+def test_source_hash_ignores_comments_only(bench):
+    a = "int f(int x) {  // doubles\n  return 2 * x;  /* twice */\n}\n"
+    b = "// header\nint f(int x) {\n\n  return 2 * x;\n}\n"
+    c = "int f(int x) {\n  return 3 * x;\n}\n"
+    assert bench.code_only(a) == bench.code_only(b)
+    assert bench.code_only(a) != bench.code_only(c)
+
+
+def test_traffic_entries_match_the_current_kernels(bench):
+    """profiles/traffic.json was captured from the kernels as they are"""
+    import json
+    with open(bench.TRAFFIC_FILE) as f:
+        tr = json.load(f)
+    for name, ent in tr.items():
+        assert ent["source_hash"] == bench.source_hash(name), name
+        assert ent["bytes_per_launch"] == ent["dram_read_bytes"] + ent["dram_write_bytes"]
