@@ -151,3 +151,34 @@ def test_plain_and_residual_calls_run_different_kernels(lib):
         torch.cuda.synchronize()
         assert not torch.equal(o1, o2), strided
         assert not torch.equal(g1[1], g2[1]), strided
+
+
+@pytest.mark.parametrize("D", [32, 64, 128])
+def test_padded_rows_collapse_to_the_flat_kernels(lib, D):
+    """(B, H, T, D) views of buffers whose rows are padded to D + 16: the
+    batch stride is still H head strides, so the FLAT instances run (3-D
+    tensor maps with a row stride other than D, the strided preprocess)."""
+    B, H, T = 2, 3, 200
+    dev = torch.device("cuda:0")
+    q, k, v, do = (t.to(dev) for t in bf16_inputs(B, H, T, D, seed=606 + D, qk_std=1.0))
+    scale = D ** -0.5
+
+    def padded(x):
+        buf = torch.full((B, H, T, D + 16), float("nan"), dtype=x.dtype, device=dev)
+        buf[..., :D] = x
+        return buf[..., :D]
+
+    o_c, lse_c, olo_c = lib.attn_fwd_ex(q, k, v, scale)
+    g_c = lib.attn_bwd(q, k, v, o_c, lse_c, do, scale, o_lo=olo_c)
+    qp, kp, vp, dop = (padded(t) for t in (q, k, v, do))
+    o_p = padded(torch.zeros_like(q))
+    olo_p = padded(torch.zeros_like(q))
+    _, lse_p, _ = lib.attn_fwd_strided(qp, kp, vp, scale, o=o_p, o_lo=olo_p)
+    gp = [padded(torch.zeros_like(q)) for _ in range(3)]
+    lib.attn_bwd_strided(qp, kp, vp, o_p, lse_p, dop, scale, dq=gp[0], dk=gp[1], dv=gp[2],
+                         o_lo=olo_p)
+    torch.cuda.synchronize()
+    assert lib.cattn_get_device_status() == lib.OK
+    assert torch.equal(o_p, o_c) and torch.equal(lse_p, lse_c) and torch.equal(olo_p, olo_c)
+    assert torch.equal(gp[1], g_c[1]) and torch.equal(gp[2], g_c[2])
+    close_bf16_steps(gp[0], g_c[0], "dq")
