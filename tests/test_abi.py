@@ -340,3 +340,29 @@ def test_python_buffers_must_be_device_memory_of_the_right_shape():
     with pytest.raises(ValueError, match="fp32"):
         cattn._vector(t.zeros(1, 2, 16), like, (1, 2, 16), "lse")   # a CPU tensor
     assert cattn._nbytes(t.zeros(10, dtype=t.float32)) == 40
+
+
+# ------------------------------------------------------------ the header as C
+
+@pytest.mark.parametrize("lang,std", [("c", "c99"), ("c", "c11"), ("c++", "c++17")])
+def test_header_is_plain_c_and_cpp(lang, std, tmp_path):
+    """include/cattn.h compiles on its own, warning-free, as C and as C++,
+    and a C program can take the address of every entry point (the ABI has
+    no C++ types in it)."""
+    import re
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc" if lang == "c" else "g++")
+    if cc is None:
+        pytest.skip("no host compiler")
+    inc = os.path.join(ROOT, "include")
+    names = re.findall(r"CATTN_API\s+[\w\s\*]+?\b(\w+)\s*\(",
+                       open(os.path.join(inc, "cattn.h")).read())
+    assert "attn_fwd" in names and "attn_decode" in names and "attn_bwd_dropout" in names
+    src = tmp_path / ("t.c" if lang == "c" else "t.cpp")
+    body = "\n".join(f"  p = (fn)&{n}; (void)p;" for n in names)
+    src.write_text(f'#include "cattn.h"\ntypedef void (*fn)(void);\nint main(void) {{\n'
+                   f'  fn p;\n{body}\n  return 0;\n}}\n')
+    r = subprocess.run([cc, f"-std={std}", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                        "-fsyntax-only", "-I", inc, str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
