@@ -35,6 +35,7 @@ __all__ = [
     "attn_bwd_noalloc", "NOALLOC_SCRATCH_BYTES",
     "attn_fwd_strided", "attn_bwd_strided", "split_qkv", "CausalAttentionQKV", "Layout",
     "Dropout", "dropout_params", "attn_decode", "attn_decode_workspace_bytes",
+    "SUPPORTED_HEAD_SIZES", "padded_head_size", "pad_qkv_projection", "pad_out_projection",
 ]
 
 
@@ -406,6 +407,50 @@ def attn_decode(q, k, v, L, scale=None, o=None, lse=None, workspace=None, stream
                          workspace.data_ptr(), _nbytes(workspace), _stream(stream))
     _check("attn_decode", st)
     return o, lse
+
+
+SUPPORTED_HEAD_SIZES = (16, 32, 64, 128)
+
+
+def padded_head_size(d: int) -> int:
+    """The smallest head size the kernels take that holds d (e.g. 12 -> 16)."""
+    for s in SUPPORTED_HEAD_SIZES:
+        if d <= s:
+            return s
+    raise ValueError(f"head size {d} above {SUPPORTED_HEAD_SIZES[-1]}")
+
+
+def pad_qkv_projection(weight, bias, n_head, d, d_pad=None):
+    """One-time set-up for head sizes the kernels do not take (12, say):
+    the c_attn projection (weight (3C, C_in), bias (3C,) or None, rows
+    [q heads | k heads | v heads], d rows per head) re-laid so that each
+    head gets d_pad rows, the extra ones zero.  Its output is then a
+    (B, T, 3 * n_head * d_pad) buffer whose zero-padded heads the d_pad
+    kernels process exactly (padded q and k add nothing to the scores;
+    padded v columns give zero output columns); pass scale = 1/sqrt(d).
+    Not on the per-step path: a model does this once to its weights."""
+    d_pad = d_pad or padded_head_size(d)
+    w = weight.reshape(3, n_head, d, -1)
+    wp = weight.new_zeros(3, n_head, d_pad, w.shape[-1])
+    wp[:, :, :d] = w
+    bp = None
+    if bias is not None:
+        bp = bias.new_zeros(3, n_head, d_pad)
+        bp[:, :, :d] = bias.reshape(3, n_head, d)
+        bp = bp.reshape(-1)
+    return wp.reshape(3 * n_head * d_pad, -1), bp
+
+
+def pad_out_projection(weight, n_head, d, d_pad=None):
+    """The matching c_proj weight (C_out, n_head * d) with zero columns for
+    the padded head columns, so that y (B, T, n_head * d_pad) from the
+    kernels feeds it unchanged (the padded columns of y are zero, and the
+    zero columns keep their gradient zero)."""
+    d_pad = d_pad or padded_head_size(d)
+    w = weight.reshape(weight.shape[0], n_head, d)
+    wp = weight.new_zeros(weight.shape[0], n_head, d_pad)
+    wp[:, :, :d] = w
+    return wp.reshape(weight.shape[0], n_head * d_pad)
 
 
 class CausalAttentionQKV(torch.autograd.Function):
