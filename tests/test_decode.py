@@ -20,7 +20,8 @@ def draw(seed, *shape):
 
 @pytest.mark.parametrize("B,H,L,Tq,D", [(1, 2, 1, 1, 16), (2, 3, 300, 1, 64), (2, 2, 257, 8, 128),
                                          (1, 4, 513, 2, 32), (2, 2, 64, 8, 16), (3, 2, 1000, 4, 64),
-                                         (1, 2, 4096, 1, 128), (16, 12, 1024, 1, 64)])
+                                         (1, 2, 4096, 1, 128), (16, 12, 1024, 1, 64),
+                                         (2, 2, 8, 8, 64), (1, 1, 257, 8, 32)])
 @pytest.mark.parametrize("cache_layout", ["bhtd", "bthd"])
 def test_decode_against_oracle(lib, B, H, L, Tq, D, cache_layout):
     dev = torch.device("cuda:0")
