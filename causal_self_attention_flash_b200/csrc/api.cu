@@ -547,7 +547,15 @@ cattn_status decode_impl(const DecodeParams& p, long long BH, cudaStream_t s) {
   clear_stale_error();
   dim3 grid(static_cast<unsigned>(BH), static_cast<unsigned>(p.n_split));
   LaunchTimer t(K_DECODE, s);  // both kernels, as one entry
-  decode_partial_kernel<D><<<grid, kDecodeWarps * 32, 0, s>>>(p);
+  // query rows per thread: Tq rounded up to 1, 2, 4 or 8
+  if (p.Tq <= 1)
+    decode_partial_kernel<D, 1><<<grid, kDecodeWarps * 32, 0, s>>>(p);
+  else if (p.Tq <= 2)
+    decode_partial_kernel<D, 2><<<grid, kDecodeWarps * 32, 0, s>>>(p);
+  else if (p.Tq <= 4)
+    decode_partial_kernel<D, 4><<<grid, kDecodeWarps * 32, 0, s>>>(p);
+  else
+    decode_partial_kernel<D, 8><<<grid, kDecodeWarps * 32, 0, s>>>(p);
   cattn_status st = launch_status();
   if (st != CATTN_OK) return st;
   decode_combine_kernel<D><<<static_cast<unsigned>(BH * p.Tq), D, 0, s>>>(p);

@@ -12,14 +12,17 @@
 //
 // There is almost no arithmetic per byte (2 * Tq flops per key element), so
 // the work is bound by reading K and V once from HBM.  The keys of each head
-// are split into chunks of kDecodeChunk, one CTA per (chunk, head), so even a
+// are split into chunks of kDecodeChunk, one CTA per (head, chunk), so even a
 // batch of one sequence spreads over the SMs ("split-K"):
-//   decode_partial_kernel  per CTA: 4 warps stream the chunk's K and V rows
-//                          with coalesced 4- or 8-byte lane loads, several
-//                          keys in flight per warp; each lane group keeps an
-//                          online softmax (running max m, sum l, output o)
-//                          per query; the groups are merged in shared memory
-//                          and the CTA writes its (m, l, o) to the workspace.
+//   decode_partial_kernel<D, TQ>  per CTA: 4 warps stream the chunk's K and
+//                          V rows, 16 bytes per lane and several keys per
+//                          warp load, kDecodeUnroll loads per lane in flight
+//                          (enough bytes in flight per SM to cover the DRAM
+//                          latency); each lane group keeps an online softmax
+//                          (running max m, sum l, output o) per query row,
+//                          updated once per batch of keys; the groups are
+//                          merged in shared memory and the CTA writes its
+//                          (m, l, o) to the workspace.
 //   decode_combine_kernel  per (head, query): merges the chunks' (m, l, o)
 //                          (o = sum 2^(m_c - M) o_c / sum 2^(m_c - M) l_c)
 //                          and writes O (bf16) and LSE (natural log).
@@ -36,7 +39,7 @@ namespace cattn {
 constexpr int kDecodeMaxTq = 8;     // query rows per call
 constexpr int kDecodeChunk = 256;   // keys per CTA
 constexpr int kDecodeWarps = 4;
-constexpr int kDecodeUnroll = 4;    // keys in flight per lane group
+constexpr int kDecodeUnroll = 4;    // key rows in flight per lane group
 
 struct DecodeParams {
   const __nv_bfloat16* q;  // (B, H, Tq, D), element strides q_sb, q_sh, q_st
@@ -52,43 +55,42 @@ struct DecodeParams {
   float scale_log2;        // scale * log2(e)
 };
 
-// Lane layout: EPL consecutive elements per lane, LPK lanes per key row,
-// KPW keys side by side in a warp.
+// Lane layout: 8 consecutive elements (one 16-byte load) per lane, LPK
+// lanes per key row, KPW keys side by side in a warp.
 template <int D>
 struct DecodeCfg {
-  static constexpr int EPL = D >= 128 ? 4 : 2;
-  static constexpr int LPK = D / EPL;
-  static constexpr int KPW = 32 / LPK;
-  static constexpr int SLOTS = kDecodeWarps * KPW;   // lane groups per CTA
+  static constexpr int EPL = 8;
+  static constexpr int LPK = D / EPL;                 // 2, 4, 8, 16 lanes per row
+  static constexpr int KPW = 32 / LPK;                // 16, 8, 4, 2 keys per warp load
+  static constexpr int SLOTS = kDecodeWarps * KPW;    // lane groups per CTA
   static constexpr int STEP = SLOTS * kDecodeUnroll;  // keys per CTA iteration
   static_assert(LPK * EPL == D && KPW * LPK == 32, "lane layout");
   static_assert(kDecodeChunk % STEP == 0, "chunk");
 };
 
-template <int EPL>
-__device__ __forceinline__ void load_row(const __nv_bfloat16* src, float (&x)[EPL]) {
-  if constexpr (EPL == 2) {
-    const __nv_bfloat162 t = *reinterpret_cast<const __nv_bfloat162*>(src);
-    const float2 f = __bfloat1622float2(t);
-    x[0] = f.x;
-    x[1] = f.y;
-  } else {
-    const uint2 t = *reinterpret_cast<const uint2*>(src);
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&t.x));
-    const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&t.y));
-    x[0] = a.x;
-    x[1] = a.y;
-    x[2] = c.x;
-    x[3] = c.y;
+// 8 bf16 (one 16-byte load) -> 8 floats
+__device__ __forceinline__ void unpack8(const uint4& t, float (&x)[8]) {
+  const unsigned w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
   }
 }
 
-template <int D>
+// TQ: query rows held per thread (Tq rounded up to 1, 2, 4 or 8; rows at or
+// past Tq are idle).  Per iteration every lane group loads kDecodeUnroll
+// keys' K and V rows at once (4 x 2 x 16 bytes per lane in flight), forms
+// their scores, and then updates its online softmax once for the batch:
+// m' = max(m, s_1..s_U), l' = l 2^(m - m') + sum 2^(s_u - m'),
+// o' = o 2^(m - m') + sum 2^(s_u - m') v_u.
+template <int D, int TQ>
 __global__ void __launch_bounds__(kDecodeWarps * 32) decode_partial_kernel(const DecodeParams p) {
   using C = DecodeCfg<D>;
-  constexpr int EPL = C::EPL, LPK = C::LPK, KPW = C::KPW;
-  __shared__ float s_ml[C::SLOTS][kDecodeMaxTq][2];
-  __shared__ float s_o[C::SLOTS][kDecodeMaxTq][D];
+  constexpr int EPL = C::EPL, LPK = C::LPK, KPW = C::KPW, U = kDecodeUnroll;
+  __shared__ float s_ml[C::SLOTS][TQ][2];
+  __shared__ float s_o[C::SLOTS][TQ][D];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kslot = lane / LPK, sub = lane % LPK;   // key slot in the warp, lane in the row
@@ -99,10 +101,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_partial_kernel(const
   const int k0 = split * kDecodeChunk;
   const int k1 = min(p.L, k0 + kDecodeChunk);
 
-  float qr[kDecodeMaxTq][EPL];
-  float m[kDecodeMaxTq], l[kDecodeMaxTq], o[kDecodeMaxTq][EPL];
+  float qr[TQ][EPL];
+  float m[TQ], l[TQ], o[TQ][EPL];
 #pragma unroll
-  for (int r = 0; r < kDecodeMaxTq; ++r) {
+  for (int r = 0; r < TQ; ++r) {
     m[r] = -INFINITY;
     l[r] = 0.f;
 #pragma unroll
@@ -111,7 +113,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_partial_kernel(const
       qr[r][e] = 0.f;
     }
     if (r < Tq) {
-      load_row<EPL>(p.q + b * p.q_sb + h * p.q_sh + r * p.q_st + sub * EPL, qr[r]);
+      const uint4 t = *reinterpret_cast<const uint4*>(p.q + b * p.q_sb + h * p.q_sh +
+                                                      r * p.q_st + sub * EPL);
+      unpack8(t, qr[r]);
 #pragma unroll
       for (int e = 0; e < EPL; ++e) qr[r][e] *= p.scale_log2;
     }
@@ -123,50 +127,69 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_partial_kernel(const
   // warp-uniform trip count: every lane runs every iteration (the shuffles
   // below take the full warp); keys past the chunk are masked, not skipped
   for (int base = k0; base < k1; base += C::STEP) {
-    float kx[kDecodeUnroll][EPL], vx[kDecodeUnroll][EPL];
-    int key[kDecodeUnroll];
+    uint4 kraw[U], vraw[U];
+    int key[U];
 #pragma unroll
-    for (int u = 0; u < kDecodeUnroll; ++u) {
+    for (int u = 0; u < U; ++u) {
       key[u] = base + (u * kDecodeWarps + warp) * KPW + kslot;
       if (key[u] < k1) {
-        load_row<EPL>(kbase + static_cast<long long>(key[u]) * p.k_st, kx[u]);
-        load_row<EPL>(vbase + static_cast<long long>(key[u]) * p.v_st, vx[u]);
+        kraw[u] = *reinterpret_cast<const uint4*>(kbase + static_cast<long long>(key[u]) * p.k_st);
+        vraw[u] = *reinterpret_cast<const uint4*>(vbase + static_cast<long long>(key[u]) * p.v_st);
       } else {
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) kx[u][e] = vx[u][e] = 0.f;
+        kraw[u] = vraw[u] = uint4{0u, 0u, 0u, 0u};
       }
     }
+    // scores of the batch: s[r][u], -inf where not visible
+    float s[TQ][U];
 #pragma unroll
-    for (int u = 0; u < kDecodeUnroll; ++u) {
+    for (int u = 0; u < U; ++u) {
+      float kx[EPL];
+      unpack8(kraw[u], kx);
 #pragma unroll
-      for (int r = 0; r < kDecodeMaxTq; ++r) {
-        if (r >= Tq) break;  // uniform over the CTA
+      for (int r = 0; r < TQ; ++r) {
         float d = 0.f;
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) d = fmaf(qr[r][e], kx[u][e], d);
+        for (int e = 0; e < EPL; ++e) d = fmaf(qr[r][e], kx[e], d);
 #pragma unroll
         for (int off = LPK / 2; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-        // visible: inside the chunk and not after the query's position
-        if (key[u] < k1 && key[u] <= pos0 + r) {
-          if (d > m[r]) {
-            const float alpha = exp2f(m[r] - d);  // 0 while m is -inf
-            l[r] *= alpha;
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) o[r][e] *= alpha;
-            m[r] = d;
-          }
-          const float pe = exp2f(d - m[r]);
-          l[r] += pe;
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) o[r][e] = fmaf(pe, vx[u][e], o[r][e]);
-        }
+        s[r][u] = (key[u] < k1 && key[u] <= pos0 + r) ? d : -INFINITY;
       }
+    }
+    // one online-softmax update per row for the whole batch; the scores
+    // become the batch's weights 2^(s - m') in place
+#pragma unroll
+    for (int r = 0; r < TQ; ++r) {
+      float mn = m[r];
+#pragma unroll
+      for (int u = 0; u < U; ++u) mn = fmaxf(mn, s[r][u]);
+      // nothing visible yet: keep everything at zero (and avoid -inf - -inf)
+      const float mu = mn == -INFINITY ? 0.f : mn;
+      const float alpha = exp2f(m[r] - mu);  // 0 while m is -inf
+      float lsum = 0.f;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        s[r][u] = exp2f(s[r][u] - mu);         // 0 for a masked key
+        lsum += s[r][u];
+      }
+      l[r] = fmaf(l[r], alpha, lsum);
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) o[r][e] *= alpha;
+      m[r] = mn;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float vx[EPL];
+      unpack8(vraw[u], vx);
+#pragma unroll
+      for (int r = 0; r < TQ; ++r)
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) o[r][e] = fmaf(s[r][u], vx[e], o[r][e]);
     }
   }
 
   // lane groups -> shared memory -> one (m, l, o) per query for the CTA
 #pragma unroll
-  for (int r = 0; r < kDecodeMaxTq; ++r) {
+  for (int r = 0; r < TQ; ++r) {
     if (r >= Tq) break;
 #pragma unroll
     for (int e = 0; e < EPL; ++e) s_o[slot][r][sub * EPL + e] = o[r][e];
@@ -179,13 +202,13 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_partial_kernel(const
   for (int t = threadIdx.x; t < Tq * D; t += blockDim.x) {
     const int r = t / D, d = t - (t / D) * D;
     float M = -INFINITY;
-    for (int s = 0; s < C::SLOTS; ++s) M = fmaxf(M, s_ml[s][r][0]);
+    for (int sl = 0; sl < C::SLOTS; ++sl) M = fmaxf(M, s_ml[sl][r][0]);
     float lsum = 0.f, osum = 0.f;
     if (M > -INFINITY) {  // otherwise no key of this chunk is visible to the row
-      for (int s = 0; s < C::SLOTS; ++s) {
-        const float w = exp2f(s_ml[s][r][0] - M);  // 0 for a slot that saw nothing
-        lsum = fmaf(s_ml[s][r][1], w, lsum);
-        osum = fmaf(s_o[s][r][d], w, osum);
+      for (int sl = 0; sl < C::SLOTS; ++sl) {
+        const float w = exp2f(s_ml[sl][r][0] - M);  // 0 for a slot that saw nothing
+        lsum = fmaf(s_ml[sl][r][1], w, lsum);
+        osum = fmaf(s_o[sl][r][d], w, osum);
       }
     }
     const size_t row = (static_cast<size_t>(bh) * p.n_split + split) * Tq + r;

@@ -25,7 +25,15 @@ static T* exact(size_t n) {
 
 template <int D>
 static void run(DecodeParams p, int BH) {
-  emu::launch(dim3(BH, p.n_split), kDecodeWarps * 32, decode_partial_kernel<D>, p);
+  const dim3 grid(BH, p.n_split);
+  if (p.Tq <= 1)
+    emu::launch(grid, kDecodeWarps * 32, decode_partial_kernel<D, 1>, p);
+  else if (p.Tq <= 2)
+    emu::launch(grid, kDecodeWarps * 32, decode_partial_kernel<D, 2>, p);
+  else if (p.Tq <= 4)
+    emu::launch(grid, kDecodeWarps * 32, decode_partial_kernel<D, 4>, p);
+  else
+    emu::launch(grid, kDecodeWarps * 32, decode_partial_kernel<D, 8>, p);
   emu::launch(dim3(BH * p.Tq), D, decode_combine_kernel<D>, p);
 }
 

@@ -50,7 +50,9 @@ def from_bits(b: np.ndarray) -> np.ndarray:
 
 @pytest.mark.parametrize("B,H,Tq,L,D,layout", [
     (1, 1, 1, 1, 16, 0), (2, 2, 1, 300, 64, 0), (1, 2, 3, 257, 128, 1), (1, 1, 8, 8, 32, 0),
-    (2, 1, 8, 513, 16, 1), (1, 3, 2, 256, 64, 1), (1, 1, 5, 1000, 128, 0)])
+    (2, 1, 8, 513, 16, 1), (1, 3, 2, 256, 64, 1), (1, 1, 5, 1000, 128, 0),
+    (1, 2, 4, 37, 64, 0), (2, 1, 2, 70, 32, 1), (1, 1, 7, 520, 64, 1), (1, 1, 1, 255, 128, 1),
+    (3, 1, 6, 129, 16, 0)])
 def test_decode_kernels_on_the_host(emu_exe, tmp_path, B, H, Tq, L, D, layout):
     g = torch.Generator().manual_seed(1000 * L + D + Tq)
     Tmax = L       # a tight cache: a read past row L - 1 leaves the buffer
