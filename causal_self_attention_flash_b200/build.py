@@ -19,7 +19,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libcattn.so")
 
 SOURCES = ["api.cu"]
-DEPS = ["api.cu", "fwd.cuh", "bwd.cuh", "sm100.cuh"]
+# every device source and header: a change to any of them rebuilds
+DEPS = sorted(f for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh")))
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
