@@ -366,3 +366,37 @@ def test_header_is_plain_c_and_cpp(lang, std, tmp_path):
     r = subprocess.run([cc, f"-std={std}", "-Wall", "-Wextra", "-Werror", "-pedantic",
                         "-fsyntax-only", "-I", inc, str(src)], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_strided_dropout_and_decode_calls_check_alignment_and_nulls():
+    """Every pointer of the newer entry points is checked before anything
+    runs: bf16 tensors 16-byte aligned, LSE 4, workspace 256; nulls
+    refused."""
+    import ctypes
+    c = contiguous(2, 8, 64)
+    d = ctypes.byref(_binding.Dropout(0.1, 1, 2))
+    fwd_args = lambda q=ALIGNED, k=ALIGNED, v=ALIGNED, o=ALIGNED, lse=ALIGNED, olo=None: (  # noqa: E731
+        q, c, k, c, v, c, 0.125, 1, 2, 8, 64, d, o, c, lse, olo, None)
+    for bad in (dict(q=ALIGNED + 8), dict(k=ALIGNED + 2), dict(v=ALIGNED + 8), dict(o=ALIGNED + 8),
+                dict(lse=ALIGNED + 2), dict(olo=ALIGNED + 8), dict(q=None), dict(lse=None)):
+        assert cattn.LIB.attn_fwd_dropout(*fwd_args(**bad)) == cattn.ERR_INVALID_ARG, bad
+    ptrs = [ALIGNED] * 10   # q k v o o_lo lse do dq dk dv
+    for i, bad in ((0, ALIGNED + 8), (3, ALIGNED + 8), (4, ALIGNED + 8), (5, ALIGNED + 2),
+                   (6, ALIGNED + 8), (7, ALIGNED + 8), (8, None), (9, ALIGNED + 8)):
+        p = list(ptrs)
+        p[i] = bad
+        r = cattn.LIB.attn_bwd_dropout(p[0], c, p[1], c, p[2], c, p[3], c, p[4], p[5], p[6], c,
+                                       0.125, 1, 2, 8, 64, d, p[7], c, p[8], c, p[9], c, 0,
+                                       ALIGNED, 1 << 30, None)
+        assert r == cattn.ERR_INVALID_ARG, (i, bad)
+    r = cattn.LIB.attn_bwd_dropout(*[x for t in zip(ptrs[:4], [c] * 4) for x in t], ALIGNED,
+                                   ALIGNED, ALIGNED, c, 0.125, 1, 2, 8, 64, d, ALIGNED, c,
+                                   ALIGNED, c, ALIGNED, c, 0, ALIGNED + 128, 1 << 30, None)
+    assert r == cattn.ERR_INVALID_ARG    # workspace not 256-byte aligned
+    for kw in (dict(q=ALIGNED + 8), dict(k=ALIGNED + 8), dict(o=ALIGNED + 8),
+               dict(lse=ALIGNED + 2), dict(ws=ALIGNED + 16), dict(v=None)):
+        a = dict(q=ALIGNED, k=ALIGNED, v=ALIGNED, o=ALIGNED, lse=ALIGNED, ws=ALIGNED)
+        a.update(kw)
+        r = cattn.LIB.attn_decode(a["q"], c, a["k"], c, a["v"], c, 0.125, 1, 2, 1, 8, 64,
+                                  a["o"], c, a["lse"], a["ws"], 1 << 20, None)
+        assert r == cattn.ERR_INVALID_ARG, kw
