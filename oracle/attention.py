@@ -143,6 +143,38 @@ def attention_backward_heads(q, k, v, do, scale, heads):
     return tuple(out)
 
 
+def attention_backward_given_o(q, k, v, do, o_heads, scale, heads):
+    """Backward pass with the row term taken from a GIVEN output instead of
+    the exact one, for a subset of flat head indices (b*H + h).
+
+    The chain rule above writes Delta either as sum_j P_ij dP_ij or as
+    sum_d dO_id O_id; a backward that receives O from the caller (the pages'
+    interface passes it in bf16) can only use the second form with the O
+    it was given.  Here Delta_i = sum_d dO_id o_id with o from ``o_heads``
+    ((n, T, D), one row block per listed head), and then, as in
+    attention_backward, dS = P * (dP - Delta), dQ = scale dS K,
+    dK = scale dS^T Q, dV = P^T dO.  With o equal to the exact output this
+    is attention_backward; with o = bf16(exact output) it is the exact
+    gradient reachable through that interface.  Returns (dq, dk, dv), each
+    (n, T, D).
+    """
+    q, k, v = _check(q, k, v)
+    do = np.asarray(do, dtype=np.float64)
+    o_heads = np.asarray(o_heads, dtype=np.float64)
+    B, H, T, D = q.shape
+    out = [np.empty((len(heads), T, D)) for _ in range(3)]
+    for n, f in enumerate(heads):
+        b, h = divmod(f, H)
+        p, _ = head_probs(q[b, h], k[b, h], scale)
+        dp_n = do[b, h] @ v[b, h].T
+        dlt_o = (o_heads[n] * do[b, h]).sum(axis=1)    # Delta from the given O
+        ds_n = p * (dp_n - dlt_o[:, None])
+        out[0][n] = scale * (ds_n @ k[b, h])
+        out[1][n] = scale * (ds_n.T @ q[b, h])
+        out[2][n] = p.T @ do[b, h]
+    return tuple(out)
+
+
 def attention_rows(q, k, v, scale, b, h, rows):
     """O and LSE of chosen query rows of one head, one row at a time.
 

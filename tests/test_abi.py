@@ -158,8 +158,23 @@ def test_workspace_formula(B, H, T, D):
     def r256(x):
         return (x + 255) // 256 * 256
     tpad = (T + 127) // 128 * 128
-    want = r256(B * H * T * D * 4) + 2 * r256(B * H * tpad * 4)
+    # the call's status words (256 bytes), the dQ accumulator, the arrival
+    # counters (one word per head, 128-row query tile and 32-row quarter),
+    # LSE2, Delta
+    want = (256 + r256(B * H * T * D * 4) + r256(B * H * (tpad // 128) * 4 * 4)
+            + 2 * r256(B * H * tpad * 4))
     assert cattn.attn_bwd_workspace_bytes(B, H, T, D) == want
+
+
+def test_last_device_status_checks_its_workspace_pointer():
+    """cattn_last_device_status reads the status words at the start of a
+    backward workspace; a null or misaligned workspace is refused before
+    any device call."""
+    assert cattn.LIB.cattn_last_device_status(None, None) == cattn.ERR_INVALID_ARG
+    assert cattn.LIB.cattn_last_device_status(ALIGNED + 16, None) == cattn.ERR_INVALID_ARG
+    assert cattn.LIB.cattn_selftest_wait_timeout_ws(1000, None, None) == cattn.ERR_INVALID_ARG
+    assert cattn.LIB.cattn_selftest_wait_timeout_ws(1000, ALIGNED + 128, None) == \
+        cattn.ERR_INVALID_ARG
 
 
 def test_binding_refuses_cpu_tensors():
@@ -214,6 +229,34 @@ def test_strided_calls_reject_bad_strides(bad):
     assert fwd_strided(lo=lay) == cattn.ERR_INVALID_ARG
     for i in range(8):
         assert bwd_strided(i, lay) == cattn.ERR_INVALID_ARG
+
+
+def test_self_overlapping_output_layouts_are_refused():
+    """An output whose own elements would share addresses (rows closer than
+    D, heads closer than a head's span, ...) is refused before anything
+    runs; the same strides on an input only read, and pass the check."""
+    B, H, T, D = 1, 2, 8, 64
+    overlapping = [_binding.Layout(H * T * D, T * D, 8),      # rows overlap
+                   _binding.Layout(H * T * D, 64, D),         # heads overlap rows
+                   _binding.Layout(T * D, T * D, D),          # batches overlap heads
+                   _binding.Layout(H * T * D, 8, 128)]        # heads 8 apart, D = 64 wide
+    for lay in overlapping:
+        assert fwd_strided(lo=lay, B=2) == cattn.ERR_INVALID_ARG, (lay.b, lay.h, lay.t)
+        for i in (5, 6, 7):      # dq, dk, dv
+            assert bwd_strided(i, lay, B=2) == cattn.ERR_INVALID_ARG, (i, lay.b, lay.h, lay.t)
+        # as an input the layout only reads: the argument check lets it through
+        # (what follows is the device check, which fails on a host without a GPU)
+        assert fwd_strided(lay=lay, B=2) != cattn.ERR_INVALID_ARG
+    C = H * D   # (B, T, C) output: heads interleaved within each row, no overlap
+    btc = _binding.Layout(T * C, D, C)
+    assert fwd_strided(lo=btc, B=2) != cattn.ERR_INVALID_ARG
+    padded = _binding.Layout(H * T * (D + 16), T * (D + 16), D + 16)
+    assert fwd_strided(lo=padded, B=2) != cattn.ERR_INVALID_ARG
+    # decode: its (B, H, Tq, D) output is checked the same way
+    c = _binding.Layout(H * 8 * D, 8 * D, D)
+    assert cattn.LIB.attn_decode(ALIGNED, c, ALIGNED, c, ALIGNED, c, 0.125, 1, H, 2, 8, D,
+                                 ALIGNED, _binding.Layout(H * 2 * D, 2 * D, 16), ALIGNED,
+                                 ALIGNED, 1 << 20, None) == cattn.ERR_INVALID_ARG
 
 
 def test_strided_calls_check_shapes_and_empty():

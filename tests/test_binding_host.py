@@ -166,3 +166,14 @@ def test_decode_call(fake):
         cattn.attn_decode(q, k, k, Tmax + 1, o=o, lse=lse, workspace=ws)
     with pytest.raises(ValueError, match="matching q"):
         cattn.attn_decode(q, FakeDev((B, H + 1, Tmax, D)), k, L, o=o, lse=lse, workspace=ws)
+
+
+def test_status_word_readers_take_device_workspaces_only():
+    """cattn_last_device_status and the workspace self-test read a backward
+    workspace's status words: a host tensor is refused in Python, before
+    any C call."""
+    host_ws = torch.zeros(4096, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="device memory"):
+        cattn.cattn_last_device_status(host_ws)
+    with pytest.raises(ValueError, match="device memory"):
+        cattn.cattn_selftest_wait_timeout(1000, workspace=host_ws)

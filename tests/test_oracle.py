@@ -92,6 +92,64 @@ def test_row_and_head_helpers_match_full():
     np.testing.assert_allclose(oracle.delta_from_o(o, do), delta, rtol=0, atol=1e-12)
 
 
+def _given_o_pins(given_o):
+    """Facts outside attention_backward_given_o that pin it:
+    (1) given the exact output it is the ordinary backward (the two forms of
+    Delta agree, sum_j P_ij dP_ij = sum_d dO_id O_id);
+    (2) its change under a perturbation e of the given output is the closed
+    form of the chain rule: Delta moves by delta_i = sum_d dO_id e_id, so dS
+    moves by -P_ij delta_i, dQ_i by -scale delta_i (P K)_i, dK_j by
+    -scale sum_i P_ij delta_i Q_i, and dV not at all;
+    (3) it is linear in the output (the perturbation doubled doubles the
+    change)."""
+    q, k, v, do = (as_f64(t) for t in bf16_inputs(1, 3, 37, 8, seed=21))
+    scale = 0.41
+    heads = [0, 2]
+    o, _ = oracle.attention_forward_heads(q, k, v, scale, heads)
+    exact = oracle.attention_backward_heads(q, k, v, do, scale, heads)
+    given = given_o(q, k, v, do, o, scale, heads)
+    for a, b_ in zip(given, exact):
+        np.testing.assert_allclose(a, b_, rtol=0, atol=1e-13)
+    rng = np.random.default_rng(5)
+    e = rng.standard_normal(o.shape) * 1e-3
+    moved = given_o(q, k, v, do, o + e, scale, heads)
+    moved2 = given_o(q, k, v, do, o + 2 * e, scale, heads)
+    for n, f in enumerate(heads):
+        b, h = divmod(f, 3)
+        p, _ = oracle.head_probs(q[b, h], k[b, h], scale)
+        dlt = (do[b, h] * e[n]).sum(axis=1)
+        want_dq = -scale * dlt[:, None] * (p @ k[b, h])
+        want_dk = -scale * (p * dlt[:, None]).T @ q[b, h]
+        np.testing.assert_allclose(moved[0][n] - exact[0][n], want_dq, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(moved[1][n] - exact[1][n], want_dk, rtol=0, atol=1e-12)
+        np.testing.assert_array_equal(moved[2][n], exact[2][n])
+        np.testing.assert_allclose(moved2[0][n] - exact[0][n], 2 * want_dq, rtol=0, atol=1e-12)
+
+
+def test_backward_given_o_is_pinned():
+    _given_o_pins(oracle.attention_backward_given_o)
+
+
+GIVEN_O_MUTANTS = [
+    ("exact Delta instead of the given output's",
+     "dlt_o = (o_heads[n] * do[b, h]).sum(axis=1)", "dlt_o = (p * dp_n).sum(axis=1)"),
+    ("given output of the wrong head", "(o_heads[n] * do[b, h])", "(o_heads[-1] * do[b, h])"),
+    ("Delta subtracted column-wise", "ds_n = p * (dp_n - dlt_o[:, None])",
+     "ds_n = p * (dp_n - dlt_o[None, :])"),
+]
+
+
+@pytest.mark.parametrize("desc,old,new", GIVEN_O_MUTANTS, ids=[m[0] for m in GIVEN_O_MUTANTS])
+def test_given_o_planted_mistake_is_caught(desc, old, new):
+    with open(oracle_mod.__file__) as f:
+        src = f.read()
+    assert src.count(old) == 1, old
+    mod = types.ModuleType("oracle_given_o_mutant")
+    exec(compile(src.replace(old, new), "oracle_given_o_mutant", "exec"), mod.__dict__)
+    with pytest.raises(AssertionError):
+        _given_o_pins(mod.attention_backward_given_o)
+
+
 def test_tiny_workload_fp32_and_bf16_inputs():
     """The tiny check runs on its raw fp32 draws as well as on the bf16
     rounding the GPU sees; the two results differ only by input rounding."""

@@ -46,3 +46,28 @@ def test_static_scratch_backward_matches_workspace_backward(lib):
         assert lib.cattn_get_device_status() == lib.OK
         for name, g, w in zip(("dq", "dk", "dv"), got, want):
             check_bf16(f"{name} B{B} H{H} T{T} D{D}", as_f64(g), as_f64(w))
+
+
+def test_second_call_allocates_no_device_memory(lib):
+    """The call's promise: after the first call on a device (which looks up
+    the array's address), a call leaves the device's free memory unchanged.
+    The outputs are allocated before the measurement and passed in; this
+    goes through the Python wrapper, whose only work is marshalling."""
+    B, H, T, D = 2, 3, 300, 64
+    scale = 1.0 / math.sqrt(D)
+    q, k, v, do = (t.cuda() for t in bf16_inputs(B, H, T, D, seed=4104))
+    o, lse = lib.attn_fwd(q, k, v, scale)
+    outs = [torch.empty_like(q) for _ in range(3)]
+    lib.attn_bwd_noalloc(q, k, v, o, lse, do, scale, dq=outs[0], dk=outs[1], dv=outs[2])
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    got = lib.attn_bwd_noalloc(q, k, v, o, lse, do, scale, dq=outs[0], dk=outs[1], dv=outs[2])
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, (free0, free1)
+    assert all(g is w for g, w in zip(got, outs))
+    want = lib.attn_bwd(q, k, v, o, lse, do, scale)
+    torch.cuda.synchronize()
+    assert lib.cattn_get_device_status() == lib.OK
+    for name, g, w in zip(("dq", "dk", "dv"), got, want):
+        check_bf16(f"{name} (Python wrapper)", as_f64(g), as_f64(w))
