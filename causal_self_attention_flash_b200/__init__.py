@@ -29,6 +29,7 @@ __all__ = [
     "attn_bwd_workspace_bytes",
     "cattn_get_device_status", "cattn_set_wait_timeout_us",
     "cattn_selftest_wait_timeout", "cattn_status_string", "cattn_version",
+    "cattn_last_device_status",
     "cattn_timing_enable", "cattn_timing_read", "KERNEL_NAMES",
     "CausalAttention", "CattnError", "LIB", "LIB_PATH",
     "OK", "ERR_INVALID_ARG", "ERR_UNSUPPORTED", "ERR_CUDA", "ERR_TIMEOUT", "ERR_TOO_LARGE",
@@ -230,8 +231,23 @@ def cattn_set_wait_timeout_us(us: int):
     LIB.cattn_set_wait_timeout_us(int(us))
 
 
-def cattn_selftest_wait_timeout(timeout_us: int, stream=None):
-    return int(LIB.cattn_selftest_wait_timeout(int(timeout_us), _stream(stream)))
+def cattn_selftest_wait_timeout(timeout_us: int, stream=None, workspace=None):
+    """The hang guard's self-test; with a workspace (a uint8 CUDA tensor of
+    a backward's workspace) it records into that workspace's status words."""
+    if workspace is None:
+        return int(LIB.cattn_selftest_wait_timeout(int(timeout_us), _stream(stream)))
+    if not workspace.is_cuda:
+        raise ValueError("workspace must be device memory")
+    return int(LIB.cattn_selftest_wait_timeout_ws(int(timeout_us), workspace.data_ptr(),
+                                                  _stream(stream)))
+
+
+def cattn_last_device_status(workspace, stream=None):
+    """Status recorded by the last backward call that used this workspace
+    (waits for `stream`)."""
+    if not workspace.is_cuda:
+        raise ValueError("workspace must be device memory")
+    return int(LIB.cattn_last_device_status(workspace.data_ptr(), _stream(stream)))
 
 
 KERNEL_NAMES = ("fwd_kernel", "bwd_pre_kernel", "bwd_kernel", "dq_convert_kernel")

@@ -66,6 +66,8 @@ SIGNATURES = {
     "cattn_get_device_status": (_i, [_i, _vp]),
     "cattn_set_wait_timeout_us": (None, [_u32]),
     "cattn_selftest_wait_timeout": (_i, [_u32, _vp]),
+    "cattn_last_device_status": (_i, [_vp, _vp]),
+    "cattn_selftest_wait_timeout_ws": (_i, [_u32, _vp, _vp]),
     "cattn_timing_enable": (None, [_i]),
     "cattn_timing_read": (_i, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int), _i]),
     "cattn_status_string": (ctypes.c_char_p, [_i]),

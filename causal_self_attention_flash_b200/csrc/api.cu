@@ -89,10 +89,19 @@ cattn_status check_device(int* dev_out) {
   return init_encode();
 }
 
-// Set the dynamic shared-memory limit of a kernel once per device.
+// Set the dynamic shared-memory limit of a kernel once per device.  A
+// kernel that re-balances registers between its warpgroups (setmaxnreg)
+// assumes it is launched with `launch_regs` registers per thread: with
+// fewer, its increase would wait forever, so a build where the compiler
+// chose another count is refused (CATTN_ERR_UNSUPPORTED) instead of run.
 template <typename K>
-cattn_status ensure_smem(int dev, unsigned bit, K kernel, int bytes) {
+cattn_status ensure_smem(int dev, unsigned bit, K kernel, int bytes, int launch_regs = 0) {
   if (g_attr_done[dev] & (1ull << bit)) return CATTN_OK;
+  if (launch_regs > 0) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return cuda_fail(cudaGetLastError());
+    if (fa.numRegs != launch_regs) return CATTN_ERR_UNSUPPORTED;
+  }
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
       cudaSuccess) {
     return cuda_fail(cudaGetLastError());
@@ -161,6 +170,26 @@ bool layout_ok(cattn_layout l) {
   const long long lim = 1LL << 38;
   return l.b > 0 && l.h > 0 && l.t > 0 && l.b % 8 == 0 && l.h % 8 == 0 && l.t % 8 == 0 &&
          l.b < lim && l.h < lim && l.t < lim;
+}
+
+// An output layout must not make two of its own elements share an address
+// (16-byte stores from different threads would race).  Sufficient test:
+// with the axes of extent > 1 taken in increasing stride order (d first,
+// stride 1), every stride must exceed the span the smaller ones cover.
+// This admits the contiguous layout, padded rows and head-interleaved
+// (B, T, C) outputs alike.
+bool output_layout_ok(cattn_layout l, int B, int H, int T, int D) {
+  struct Ax { long long stride, extent; } ax[3] = {{l.t, T}, {l.h, H}, {l.b, B}};
+  for (int i = 0; i < 3; ++i)      // sort by stride (three elements)
+    for (int j = i + 1; j < 3; ++j)
+      if (ax[j].stride < ax[i].stride) { Ax x = ax[i]; ax[i] = ax[j]; ax[j] = x; }
+  long long span = D;  // the d axis: elements 0 .. D-1
+  for (int i = 0; i < 3; ++i) {
+    if (ax[i].extent <= 1) continue;
+    if (ax[i].stride < span) return false;
+    span += ax[i].stride * (ax[i].extent - 1);
+  }
+  return true;
 }
 
 // 4-D tensor map {x = d, y = t, z = h, w = b} over a bf16 (B, H, T, D)
@@ -274,7 +303,7 @@ cattn_status fwd_impl(int dev, const void* q, cattn_layout lq, const void* k, ca
   using C = FwdCfg<D, PLO>;
   clear_stale_error();
   cattn_status st = ensure_smem(dev, (FLAT ? 32 : 0) + (DROP ? 16 : 0) + 2 * d_index(D) + PLO,
-                                fwd_kernel<D, PLO, DROP, FLAT>, C::SMEM_BYTES);
+                                fwd_kernel<D, PLO, DROP, FLAT>, C::SMEM_BYTES, C::LAUNCH_REGS);
   if (st != CATTN_OK) return st;
   CUtensorMap mq, mk, mv;
   if ((st = make_bf16_map(&mq, q, D, T, H, B, lq, FLAT)) != CATTN_OK) return st;
@@ -323,8 +352,16 @@ cattn_status fwd_dispatch(bool plo, bool drop, bool flat, int dev, const void* q
 
 // ----------------------------------------------------------------- backward
 
+// Workspace of a backward call: the call's status words {code, where}
+// (CATTN_OK = 0, else the first error a kernel recorded; read back by
+// cattn_last_device_status), the fp32 dQ accumulator, the arrival counters
+// of its query-tile quarters (one 32-bit word per (head, 128-row tile,
+// 32-row quarter)), then the LSE * log2(e) and Delta vectors; every part
+// 256-byte aligned.  The accumulator and the counters are one contiguous
+// range that the preprocess kernel zeroes.
 struct WsLayout {
-  size_t dq_off, lse2_off, delta_off, total;
+  size_t status_off, dq_off, cnt_off, lse2_off, delta_off, total;
+  size_t zero_bytes;  // accumulator + counters
   int T_pad;
 };
 
@@ -333,8 +370,11 @@ size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 WsLayout ws_layout(long long BH, int T, int D) {
   WsLayout L;
   L.T_pad = (T + 127) / 128 * 128;
-  L.dq_off = 0;
-  L.lse2_off = round256(static_cast<size_t>(BH) * T * D * 4);
+  L.status_off = 0;
+  L.dq_off = 256;
+  L.cnt_off = L.dq_off + round256(static_cast<size_t>(BH) * T * D * 4);
+  L.lse2_off = L.cnt_off + round256(static_cast<size_t>(BH) * (L.T_pad / 128) * 4 * 4);
+  L.zero_bytes = L.lse2_off - L.dq_off;
   L.delta_off = L.lse2_off + round256(static_cast<size_t>(BH) * L.T_pad * 4);
   L.total = L.delta_off + round256(static_cast<size_t>(BH) * L.T_pad * 4);
   return L;
@@ -343,7 +383,8 @@ WsLayout ws_layout(long long BH, int T, int D) {
 template <int D>
 cattn_status pre_impl(const void* o, cattn_layout lo, const void* o_lo, const void* dout,
                       cattn_layout ldo, const float* lse, float* delta, float* lse2, float4* zero,
-                      size_t zero_n4, int B, int H, int T, int row_stride, cudaStream_t s) {
+                      size_t zero_n4, int B, int H, int T, int row_stride,
+                      unsigned int* status, cudaStream_t s) {
   clear_stale_error();
   const long long BH = static_cast<long long>(B) * H;
   PreParams p;
@@ -362,6 +403,7 @@ cattn_status pre_impl(const void* o, cattn_layout lo, const void* o_lo, const vo
   p.lse2 = lse2;
   p.zero = zero;
   p.zero_n4 = zero_n4;
+  p.status = status;
   p.T = T;
   p.row_stride = row_stride;
   p.n_rows = BH * row_stride;
@@ -404,6 +446,8 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   float* dq_acc = reinterpret_cast<float*>(wb + L.dq_off);
   float* lse2 = reinterpret_cast<float*>(wb + L.lse2_off);
   float* delta = reinterpret_cast<float*>(wb + L.delta_off);
+  unsigned int* status = reinterpret_cast<unsigned int*>(wb + L.status_off);
+  unsigned int* cnt = reinterpret_cast<unsigned int*>(wb + L.cnt_off);
   const size_t n_dq = static_cast<size_t>(BH) * T * D;
 
   CUtensorMap mq, mk, mv, mdo, mdq;
@@ -412,12 +456,13 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   if ((st = make_bf16_map(&mv, v, D, T, H, B, ly.v, FLAT)) != CATTN_OK) return st;
   if ((st = make_bf16_map(&mdo, dout, D, T, H, B, ly.dout, FLAT)) != CATTN_OK) return st;
   if ((st = make_tmap(&mdq, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, T, BH,
-                      C::WARP_DQ ? D / 4 : C::CBQ, C::WARP_DQ ? 32 : 128)) !=
+                      C::WARP_DQ ? C::DCB : C::CBQ, C::WARP_DQ ? 32 : 128)) !=
       CATTN_OK)
     return st;
 
   st = pre_impl<D>(o, ly.o, o_lo, dout, ly.dout, lse, delta, lse2,
-                   reinterpret_cast<float4*>(dq_acc), n_dq / 4, B, H, T, L.T_pad, s);
+                   reinterpret_cast<float4*>(dq_acc), L.zero_bytes / 16, B, H, T, L.T_pad,
+                   status, s);
   if (st != CATTN_OK) return st;
 
   BwdParams p;
@@ -442,6 +487,16 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_timeout_ns;
   p.drop = dp;
+  p.status = status;
+  // dQ output: with WARP_DQ the kernel's drain warps convert each query
+  // tile's rows once their last contribution has been added
+  p.dq_cnt = cnt;
+  p.dq_acc = dq_acc;
+  p.dq_out = dq;
+  p.dq_f32 = grad_f32 ? 1 : 0;
+  p.dq_sb = ly.dq.b;
+  p.dq_sh = ly.dq.h;
+  p.dq_st = ly.dq.t;
   // persistent: one CTA per SM, each looping over key tiles
   const long long n_items = static_cast<long long>(BH) * p.n_tiles;
   if (n_items > 0x7fffffffLL) return CATTN_ERR_INVALID_ARG;
@@ -451,6 +506,7 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
     bwd_kernel<D, SLO, DROP, FLAT><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mdo, mdq, p);
   }
   if ((st = launch_status()) != CATTN_OK) return st;
+  if (C::WARP_DQ) return CATTN_OK;  // dQ written by the main kernel
   {
     LaunchTimer t(K_DQ_CONVERT, s);
     if (!is_contiguous(ly.dq, H, T, D)) {
@@ -516,7 +572,7 @@ bool drop_params(const cattn_dropout* d, DropParams* out) {
 
 // ---------------------------------------------------------- hang-guard test
 
-__global__ void selftest_wait_kernel(uint64_t timeout_ns) {
+__global__ void selftest_wait_kernel(uint64_t timeout_ns, unsigned int* call_status) {
   __shared__ __align__(8) uint64_t mbar;
   __shared__ int abort_flag;
   if (threadIdx.x == 0) {
@@ -526,7 +582,7 @@ __global__ void selftest_wait_kernel(uint64_t timeout_ns) {
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    WaitCtx w{timeout_ns, &abort_flag, 15u};
+    WaitCtx w{timeout_ns, &abort_flag, 15u, call_status};
     wait1(w, smem_u32(&mbar), 0, 1);  // nothing ever arrives
   }
   __syncthreads();
@@ -585,6 +641,7 @@ cattn_status attn_fwd_dropout(const void* q, cattn_layout lq, const void* k, cat
     return CATTN_ERR_INVALID_ARG;
   if (!layout_ok(lq) || !layout_ok(lk) || !layout_ok(lv) || !layout_ok(lo))
     return CATTN_ERR_INVALID_ARG;
+  if (!output_layout_ok(lo, B, H, T, D)) return CATTN_ERR_INVALID_ARG;
   int dev;
   if ((st = check_device(&dev)) != CATTN_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -641,6 +698,7 @@ cattn_status attn_decode(const void* q, cattn_layout lq, const void* k, cattn_la
     return CATTN_ERR_INVALID_ARG;
   if (!layout_ok(lq) || !layout_ok(lk) || !layout_ok(lv) || !layout_ok(lo))
     return CATTN_ERR_INVALID_ARG;
+  if (!output_layout_ok(lo, B, H, Tq, D)) return CATTN_ERR_INVALID_ARG;
   const long long BH = static_cast<long long>(B) * H;
   if (BH * Tq > 0x7fffffffLL) return CATTN_ERR_INVALID_ARG;
   if (workspace_bytes < decode_ws_bytes(BH, Tq, L, D)) return CATTN_ERR_INVALID_ARG;
@@ -693,10 +751,10 @@ cattn_status attn_bwd_preprocess(const void* o, const void* dout, int B, int H, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const cattn_layout c = contiguous_layout(H, T, D);
   switch (D) {
-    case 16: return pre_impl<16>(o, c, nullptr, dout, c, nullptr, delta, nullptr, nullptr, 0, B, H, T, T, s);
-    case 32: return pre_impl<32>(o, c, nullptr, dout, c, nullptr, delta, nullptr, nullptr, 0, B, H, T, T, s);
-    case 64: return pre_impl<64>(o, c, nullptr, dout, c, nullptr, delta, nullptr, nullptr, 0, B, H, T, T, s);
-    case 128: return pre_impl<128>(o, c, nullptr, dout, c, nullptr, delta, nullptr, nullptr, 0, B, H, T, T, s);
+    case 16: return pre_impl<16>(o, c, nullptr, dout, c, nullptr, delta, nullptr, nullptr, 0, B, H, T, T, nullptr, s);
+    case 32: return pre_impl<32>(o, c, nullptr, dout, c, nullptr, delta, nullptr, nullptr, 0, B, H, T, T, nullptr, s);
+    case 64: return pre_impl<64>(o, c, nullptr, dout, c, nullptr, delta, nullptr, nullptr, 0, B, H, T, T, nullptr, s);
+    case 128: return pre_impl<128>(o, c, nullptr, dout, c, nullptr, delta, nullptr, nullptr, 0, B, H, T, T, nullptr, s);
   }
   return CATTN_ERR_UNSUPPORTED;
 }
@@ -722,6 +780,9 @@ cattn_status attn_bwd_dropout(const void* q, cattn_layout lq, const void* k, cat
     return CATTN_ERR_INVALID_ARG;
   if (!layout_ok(lq) || !layout_ok(lk) || !layout_ok(lv) || !layout_ok(lo) || !layout_ok(ldo) ||
       !layout_ok(ldq) || !layout_ok(ldk) || !layout_ok(ldv))
+    return CATTN_ERR_INVALID_ARG;
+  if (!output_layout_ok(ldq, B, H, T, D) || !output_layout_ok(ldk, B, H, T, D) ||
+      !output_layout_ok(ldv, B, H, T, D))
     return CATTN_ERR_INVALID_ARG;
   const int BH = B * H;
   if (workspace_bytes < ws_layout(BH, T, D).total) return CATTN_ERR_INVALID_ARG;
@@ -842,6 +903,44 @@ cattn_status cattn_get_device_status(int clear, void* stream) {
   return v == 0 ? CATTN_OK : static_cast<cattn_status>(v);
 }
 
+cattn_status cattn_last_device_status(void* workspace, void* stream) {
+  if (workspace == nullptr || !aligned(workspace, 256)) return CATTN_ERR_INVALID_ARG;
+  int dev;
+  cattn_status st = check_device(&dev);
+  if (st != CATTN_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return cuda_fail(cudaGetLastError());
+  unsigned int v = 0;
+  if (cudaMemcpy(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return cuda_fail(cudaGetLastError());
+  return v == 0 ? CATTN_OK : static_cast<cattn_status>(v);
+}
+
+cattn_status cattn_selftest_wait_timeout_ws(uint32_t timeout_us, void* workspace, void* stream) {
+  if (workspace == nullptr || !aligned(workspace, 256)) return CATTN_ERR_INVALID_ARG;
+  int dev;
+  cattn_status st = check_device(&dev);
+  if (st != CATTN_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned int before = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess ||
+      cudaMemcpyFromSymbol(&before, g_status, sizeof(before)) != cudaSuccess ||
+      cudaMemsetAsync(workspace, 0, 8, s) != cudaSuccess)
+    return cuda_fail(cudaGetLastError());
+  clear_stale_error();
+  selftest_wait_kernel<<<1, 32, 0, s>>>(static_cast<uint64_t>(timeout_us) * 1000ull,
+                                        static_cast<unsigned int*>(workspace));
+  if (launch_status() != CATTN_OK) return CATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return cuda_fail(cudaGetLastError());
+  if (before == 0) {  // leave the global word as it was found
+    const unsigned int z = 0;
+    if (cudaMemcpyToSymbol(g_status, &z, sizeof(z)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_status_where, &z, sizeof(z)) != cudaSuccess)
+      return cuda_fail(cudaGetLastError());
+  }
+  return cattn_last_device_status(workspace, stream);
+}
+
 void cattn_set_wait_timeout_us(uint32_t us) {
   g_timeout_ns = us == 0 ? kDefaultTimeoutNs : static_cast<uint64_t>(us) * 1000ull;
 }
@@ -850,7 +949,7 @@ cattn_status cattn_selftest_wait_timeout(uint32_t timeout_us, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cattn_status st = cattn_get_device_status(1, stream);  // start from a clear word
   if (st != CATTN_OK && st != CATTN_ERR_TIMEOUT) return st;
-  selftest_wait_kernel<<<1, 32, 0, s>>>(static_cast<uint64_t>(timeout_us) * 1000ull);
+  selftest_wait_kernel<<<1, 32, 0, s>>>(static_cast<uint64_t>(timeout_us) * 1000ull, nullptr);
   if (launch_status() != CATTN_OK) return CATTN_ERR_CUDA;
   st = cattn_get_device_status(1, stream);
   return st;

@@ -14,7 +14,7 @@
 // one warpgroup works on its scores, the MMAs of the other run.  The next
 // item's Q and K/V are loaded while the current item finishes.
 //
-// Warp roles (352 threads):
+// Warp roles (384 threads):
 //   warps 0-3, 4-7  softmax warpgroups g = 0, 1, one query tile each per item;
 //              thread t of a group owns query row t, which is TMEM lane t.
 //              It reads S_g from TMEM, masks the diagonal tile, updates m
@@ -28,6 +28,8 @@
 //   warp 8     TMA producer: per item each group's Q tile (once the previous
 //              item's S MMAs are done with the buffer), then K_j, V_j through
 //              a ring that runs on across items.
+//   warp 11    idle; it completes the third warpgroup (warps 8-11), whose
+//              registers go to the softmax warpgroups.
 //   warps 9, 10  MMA issuers for groups 0, 1 (warp 9 also owns TMEM).  Two
 //              issuing threads keep the tensor core fed where one thread's
 //              issue rate would not (N = D <= 64 MMAs).  Per key tile j:
@@ -100,7 +102,7 @@ struct FwdCfg {
   static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_V + STAGES * TILE_BYTES;
-  static constexpr int NUM_BARS = 46;
+  static constexpr int NUM_BARS = 47;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_USED = OFF_MISC + 64;
   // at least 116 KB so that one CTA holds an SM (it takes all 512 TMEM columns)
@@ -120,11 +122,19 @@ struct FwdCfg {
   static constexpr uint32_t COL_OL0 = SPLIT ? 256 + 2 * D : COL_O0;
   static constexpr uint32_t COL_OL1 = SPLIT ? 256 + 3 * D : COL_O1;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int THREADS = 352;
+  // 12 warps: two softmax warpgroups, then the producer, two MMA issuers
+  // and one idle warp, which complete the third warpgroup so that its
+  // registers can be handed to the softmax warps (setmaxnreg acts on whole
+  // warpgroups).  At launch every thread holds LAUNCH_REGS (65536 / 384,
+  // rounded down to 8); the third warpgroup then drops to REGS_OTHER and
+  // the softmax warpgroups rise to REGS_SOFTMAX, within the launch total.
+  static constexpr int THREADS = 384;
+  static constexpr int LAUNCH_REGS = 168;
+  static constexpr int REGS_SOFTMAX = 216, REGS_OTHER = 64;
+  static_assert(256 * REGS_SOFTMAX + 128 * REGS_OTHER <= THREADS * LAUNCH_REGS,
+                "register split exceeds the launch allocation");
 };
 
-// named (hardware) barrier for the one-time offset of the two groups
-constexpr uint32_t kBarOffset = 3;
 // barrier indices
 // (KVEMPTY: one per group and stage, index FB_KVEMPTY + kMaxStages * g + stage; the
 // other per-group barriers at base + g)
@@ -133,7 +143,8 @@ enum : int {
   FB_KFULL = 0, FB_VFULL = kMaxStages, FB_KVEMPTY = 2 * kMaxStages, FB_QFULL = 4 * kMaxStages,
   FB_QFREE = FB_QFULL + 2, FB_SFULL = FB_QFULL + 4, FB_ODONE = FB_QFULL + 6,
   FB_OFREE = FB_QFULL + 8, FB_SFREE = FB_QFULL + 10, FB_DRAIN = FB_QFULL + 12,
-  FB_PFULL = FB_QFULL + 14  // FB_PFULL + 4 * g + part
+  FB_PFULL = FB_QFULL + 14,  // FB_PFULL + 4 * g + part
+  FB_OFFSET = FB_PFULL + 8   // the one-time start offset of the two groups
 };
 
 // Pairs of score columns whose exponential is taken by exp2_poly2 on the FMA
@@ -151,12 +162,13 @@ constexpr int kPvParts = 2;
 // TMEM as bf16 (or bf16 hi/lo), the row sum accumulated in sum2.
 // DROP: P entries whose bit in keep (bit c of keep[c / 32] for column c) is
 // clear are written as 0; the row sum still takes every entry.
-template <bool POLY, bool PLO, bool DROP>
+// Chunks [CH0, CH1) of 16 columns each (the whole row is chunks 0 .. 7).
+template <bool POLY, bool PLO, bool DROP, int CH0 = 0, int CH1 = 8>
 __device__ __forceinline__ void fwd_exp_row(const float (&s)[128], uint64_t sl2x2, uint64_t negm2,
                                             uint32_t scol, uint64_t (&sum2)[2], uint32_t pfull0,
                                             const uint32_t* keep) {
 #pragma unroll
-  for (int ch = 0; ch < 8; ++ch) {  // 16 columns per chunk
+  for (int ch = CH0; ch < CH1; ++ch) {  // 16 columns per chunk
     uint32_t hi[8], lo[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -239,14 +251,14 @@ __device__ __forceinline__ FwdItem fwd_item_info(int u, int k, int BH, int n_pai
 // FLAT: Q, K, V and O address (b, h) as one b*H + h axis (3-D tensor
 // maps, O offsets bh * o_sh); otherwise 4-D maps with (h, b) coordinates.
 template <int D, bool PLO, bool DROP, bool FLAT>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(384, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = FwdCfg<D, PLO>;
-  static_assert(FB_PFULL + 8 <= C::NUM_BARS, "barrier count");
+  static_assert(FB_OFFSET + 1 <= C::NUM_BARS, "barrier count");
   static_assert(C::STAGES <= kMaxStages, "barrier map");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = aligned_smem(smem_raw, C::SMEM_USED);
+  uint8_t* smem = aligned_smem(smem_raw, C::SMEM_USED, nullptr);
   if (smem == nullptr) return;  // uniform over the CTA: nothing touched yet
   const uint32_t sbase = smem_u32(smem);
   auto bar = [&](int i) { return sbase + C::OFF_BAR + 8u * i; };
@@ -259,7 +271,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   const int n_items = p.BH * n_pairs;
   const int G = gridDim.x, b = blockIdx.x;
 
-  WaitCtx w{p.timeout_ns, abort_flag, 1u};
+  WaitCtx w{p.timeout_ns, abort_flag, 1u, nullptr};
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -279,6 +291,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       mbar_init(bar(FB_SFREE + g), 128);
       mbar_init(bar(FB_DRAIN + g), 1);
     }
+    mbar_init(bar(FB_OFFSET), 128);
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -290,6 +303,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   tc_fence_after();
   const uint32_t tbase = misc[0];
 
+  if (warp >= 8) {
+  // third warpgroup: producer, MMA issuers, one idle warp
+  regs_dec<C::REGS_OTHER>();
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     // Per item: Q_g once the previous item no longer needs the Q_g buffer,
@@ -348,7 +364,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // loads this thread issued, which may not have been consumed, before
         // the CTA exits
         int zero = 0;
-        WaitCtx wd{p.timeout_ns, &zero, 1u};
+        WaitCtx wd{p.timeout_ns, &zero, 1u, nullptr};
         for (int t = (tk > C::STAGES ? tk - C::STAGES : 0); t < tk; ++t) {
           const int st = t % C::STAGES;
           wait1(wd, bar(FB_KFULL + st), (t / C::STAGES) & 1, 11);
@@ -358,7 +374,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           if (aq[g] > 0) wait1(wd, bar(FB_QFULL + g), (aq[g] - 1) & 1, 13);
       }
     }
-  } else if (warp >= 9) {
+  } else if (warp <= 10) {
     // ------------------------------------------------- MMA issuers (one per group)
     // Running counters across items: tg = tiles of this group so far (the
     // phase of its S/P/O barriers), aq = items of this group so far (Q and
@@ -450,10 +466,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       // drain: everything issued above has completed before TMEM is freed
       mma_commit(bar(FB_DRAIN + g));
       int zero = 0;
-      WaitCtx wd{p.timeout_ns, &zero, 1u};  // the drain wait ignores the abort flag
+      WaitCtx wd{p.timeout_ns, &zero, 1u, nullptr};  // the drain wait ignores the abort flag
       wait1(wd, bar(FB_DRAIN + g), 0, 7);
     }
+  }
   } else {
+    regs_inc<C::REGS_SOFTMAX>();
     // ------------------------------------------------------------ softmax
     const int g = warp >> 2;                 // warpgroup: one query tile per item
     const int quarter = warp & 3;
@@ -474,6 +492,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       if (ng == 0) continue;
       float m_used = -INFINITY;  // running max, scaled log2 units
       float l = 0.f;
+      // EARLY: S_g(j+1) is computed while tile j's exponentials run, so its
+      // first 64 columns are loaded during the second half of them (`pre`:
+      // s[0..63] already hold them when tile j+1 starts)
+      bool pre = false;
       for (int j = 0; j < ng; ++j) {
         const int tgj = tg + j;
         // dropout keep bits of this row's 128 keys of tile j, computed while
@@ -488,9 +510,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
               keep[c4] |= keep_byte(static_cast<uint32_t>(j * 16 + c4 * 4 + x), qi,
                                     static_cast<uint32_t>(it.bh), p.drop) << (8 * x);
         }
-        wait_warp(w, bar(FB_SFULL + g), tgj & 1, 8);
-        tc_fence_after();
-        {
+        if (!pre) {
+          wait_warp(w, bar(FB_SFULL + g), tgj & 1, 8);
+          tc_fence_after();
           uint32_t r0[32], r1[32], r2[32], r3[32];
           tmem_ld32(scol, r0);
           tmem_ld32(scol + 32, r1);
@@ -501,6 +523,16 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           for (int e = 0; e < 32; ++e) {
             s[e] = __uint_as_float(r0[e]);
             s[32 + e] = __uint_as_float(r1[e]);
+            s[64 + e] = __uint_as_float(r2[e]);
+            s[96 + e] = __uint_as_float(r3[e]);
+          }
+        } else {  // the first half arrived during the previous tile
+          uint32_t r2[32], r3[32];
+          tmem_ld32(scol + 64, r2);
+          tmem_ld32(scol + 96, r3);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
             s[64 + e] = __uint_as_float(r2[e]);
             s[96 + e] = __uint_as_float(r3[e]);
           }
@@ -561,18 +593,43 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         uint64_t sum2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
         // Once per CTA, group 1's first exponential phase waits for group
         // 0's: the two groups then stay out of step, so their exponential
-        // phases overlap less on the ex2 unit.  (Exactly one arrive and one
-        // wait per CTA on this named barrier, both taken only when both
-        // groups have a tile in the first item.)
+        // phases overlap less on the ex2 unit.  Exactly one phase of the
+        // FB_OFFSET barrier per CTA: group 0's 128 threads arrive once,
+        // group 1 waits once (bounded, like every wait), and both take it
+        // only when both groups have a tile in the first item.
         const bool offset = k == 0 && j == 0 && it.n[0] > 0 && it.n[1] > 0;
-        if (offset && g == 1) named_bar_sync(kBarOffset, 256);
-        if (j == ng - 1)
-          fwd_exp_row<false, PLO, DROP>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g),
-                                        DROP ? keep : nullptr);
-        else
-          fwd_exp_row<true, PLO, DROP>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g),
-                                       DROP ? keep : nullptr);
-        if (offset && g == 0) named_bar_arrive(kBarOffset, 256);
+        if (offset && g == 1) wait_warp(w, bar(FB_OFFSET), 0, 11);
+        if (C::EARLY && j + 1 < ng) {
+          // first half of P_g(j); then S_g(j+1), computed meanwhile, starts
+          // loading while the second half of the exponentials runs (the
+          // loaded registers count as written only at the wait)
+          fwd_exp_row<true, PLO, DROP, 0, 4>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g),
+                                             DROP ? keep : nullptr);
+          wait_warp(w, bar(FB_SFULL + g), (tgj + 1) & 1, 8);
+          tc_fence_after();
+          uint32_t r0[32], r1[32];
+          tmem_ld32(scol, r0);
+          tmem_ld32(scol + 32, r1);
+          fwd_exp_row<true, PLO, DROP, 4, 8>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g),
+                                             DROP ? keep : nullptr);
+          tmem_wait_ld_regs(r0);
+          tmem_wait_ld_regs(r1);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            s[e] = __uint_as_float(r0[e]);
+            s[32 + e] = __uint_as_float(r1[e]);
+          }
+          pre = true;
+        } else {
+          if (j == ng - 1)
+            fwd_exp_row<false, PLO, DROP>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g),
+                                          DROP ? keep : nullptr);
+          else
+            fwd_exp_row<true, PLO, DROP>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g),
+                                         DROP ? keep : nullptr);
+          pre = false;
+        }
+        if (offset && g == 0) mbar_arrive(bar(FB_OFFSET));
         float sa, sb, sc2, sd;
         f2_split(sum2[0], sa, sb);
         f2_split(sum2[1], sc2, sd);

@@ -15,18 +15,24 @@ namespace cattn {
 // Status word and hang guard
 // ---------------------------------------------------------------------------
 
-// Library-global device status: 0 = OK, else the first error code recorded.
-// g_status_where holds a code naming the wait that gave up (kernel id << 8 |
-// barrier id) for diagnosis.  The library is one translation unit, which
-// defines them here.
+// Status words.  g_status is the library-global device status: 0 = OK,
+// else the first error code any kernel recorded since it was last cleared;
+// g_status_where names the wait that gave up (kernel id << 8 | barrier id).
+// The library is one translation unit, which defines them here.  A call
+// that has a caller-owned workspace (the backward) also records into the
+// two words {code, where} at the start of that workspace, so that calls on
+// different workspaces (and streams) keep separate records.
 __device__ unsigned int g_status = 0;
 __device__ unsigned int g_status_where = 0;
 
 constexpr unsigned int kStatusTimeout = 4;  // == CATTN_ERR_TIMEOUT
 
-
-__device__ __forceinline__ void record_timeout(unsigned int where) {
-  if (atomicCAS(&g_status, 0u, kStatusTimeout) == 0u) g_status_where = where;
+// Record `code` (first error wins) in the global word and, if given, in a
+// call's own words.
+__device__ __forceinline__ void record_status(unsigned int* call, unsigned int code,
+                                              unsigned int where) {
+  if (atomicCAS(&g_status, 0u, code) == 0u) g_status_where = where;
+  if (call != nullptr && atomicCAS(call, 0u, code) == 0u) call[1] = where;
 }
 
 constexpr unsigned int kStatusUnsupported = 2;  // == CATTN_ERR_UNSUPPORTED
@@ -37,14 +43,15 @@ constexpr int kMaxDynSmem = 232448;              // 227 KB opt-in limit per CTA
 // finds the aligned start and checks it fits what it was given.  Returns
 // nullptr (after recording CATTN_ERR_UNSUPPORTED) if not: the caller must
 // then return before touching any barrier, copy or tensor memory.
-__device__ __forceinline__ uint8_t* aligned_smem(uint8_t* raw, uint32_t used) {
+__device__ __forceinline__ uint8_t* aligned_smem(uint8_t* raw, uint32_t used,
+                                                 unsigned int* call_status) {
   uint32_t dyn;
   asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
   const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(raw));
   const uint32_t pad = (1024u - (base & 1023u)) & 1023u;
   if (pad + used > dyn) {
     if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0)
-      atomicCAS(&g_status, 0u, kStatusUnsupported);
+      record_status(call_status, kStatusUnsupported, 0u);
     return nullptr;
   }
   return raw + pad;
@@ -93,10 +100,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Per-CTA wait context: a time limit and a shared abort flag.  Once any
-// thread of the CTA gives up, every later wait returns at once, so all
-// warps run to the end of the kernel (where TMEM is freed and copies in
-// flight are drained) instead of hanging.
+// Per-CTA wait context: a time limit, a shared abort flag and the call's
+// own status words (null for a call without a workspace).  Once any thread
+// of the CTA gives up, every later wait returns at once, so all warps run
+// to the end of the kernel (where TMEM is freed and copies in flight are
+// drained) instead of hanging.
 //
 // The limit is counted in SM clock cycles (clock64, cheap to read) at 2.1
 // cycles per ns: at or below the 1965 MHz maximum SM clock the real limit
@@ -105,6 +113,7 @@ struct WaitCtx {
   uint64_t timeout_ns;
   volatile int* abort;  // in shared memory
   unsigned int kernel_id;
+  unsigned int* status;  // {code, where} of the call, or null
 };
 
 __device__ __forceinline__ uint64_t cycles_now() {
@@ -126,7 +135,7 @@ __device__ __forceinline__ bool wait1(const WaitCtx& w, uint32_t bar, uint32_t p
     if (*w.abort) return false;
     if (cycles_now() - t0 > limit) {
       *w.abort = 1;
-      record_timeout((w.kernel_id << 8) | bar_id);
+      record_status(w.status, kStatusTimeout, (w.kernel_id << 8) | bar_id);
       return false;
     }
   }
@@ -152,13 +161,6 @@ __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 // ---------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), 3-D tensor maps {x = d, y = t, z = b*H + h}
@@ -228,6 +230,27 @@ __device__ __forceinline__ void bulk_wait_read0() {
 // Wait until the bulk stores have completed (writes performed).
 __device__ __forceinline__ void bulk_wait0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// ... all but the most recent bulk group.
+__device__ __forceinline__ void bulk_wait1() {
+  asm volatile("cp.async.bulk.wait_group 1;" ::: "memory");
+}
+
+// Order this thread's completed async-proxy writes to global memory (bulk
+// reduce-adds) before its later generic-proxy operations.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Atomic add at GPU scope with acquire-release semantics; returns the old
+// value.
+__device__ __forceinline__ unsigned int atom_add_acq_rel_gpu(unsigned int* p, unsigned int v) {
+  unsigned int old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
+               : "=r"(old)
+               : "l"(p), "r"(v)
+               : "memory");
+  return old;
 }
 
 // ---------------------------------------------------------------------------
@@ -301,6 +324,23 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
 
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// tcgen05.wait::ld that also marks 32 registers loaded by an earlier
+// tcgen05.ld as produced here, so that the compiler cannot move any use of
+// them above the wait (the load's own asm statement is where it otherwise
+// believes they are written).
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
+        "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]),
+        "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
+        "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]),
+        "+r"(r[31])
+      :
+      : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");

@@ -36,8 +36,18 @@
  *    been touched.
  *  - The library allocates no device memory for these calls and keeps no
  *    per-call state.  Kernels whose internal waits exceed their poll limit
- *    (a hang guard) record CATTN_ERR_TIMEOUT in a library-global device
- *    status word and exit; read it with cattn_get_device_status().
+ *    (a hang guard) record CATTN_ERR_TIMEOUT and exit.  A backward call
+ *    records it in status words at the start of its own workspace (read
+ *    them with cattn_last_device_status(workspace, stream)), so calls on
+ *    different workspaces keep separate records; every kernel also records
+ *    it in one library-global device word (cattn_get_device_status()),
+ *    which is the only record a forward call has, its signature having no
+ *    workspace.
+ *  - Per-device set-up the library caches (kernel attributes, the address
+ *    of attn_bwd_noalloc's array) belongs to the device's primary CUDA
+ *    context.  After cudaDeviceReset() or any other destruction of that
+ *    context, unload the library (or restart the process) before calling
+ *    it again on that device.
  */
 #ifndef CATTN_H
 #define CATTN_H
@@ -92,10 +102,12 @@ CATTN_API cattn_status attn_fwd_ex(const void* q, const void* k, const void* v, 
                                    void* stream);
 
 /* Bytes of device workspace attn_bwd needs for this shape (0 on bad
- * arguments).  The layout is internal: an fp32 dQ accumulator of
- * B*H*T*D floats, fp32 Delta and scaled-LSE vectors of B*H*roundup(T,128)
- * floats each,
- * each part 256-byte aligned. */
+ * arguments).  Layout: the call's status words (offset 0: CATTN_OK or the
+ * first error a kernel of the call recorded; offset 4: where), then an
+ * fp32 dQ accumulator of B*H*T*D floats and fp32 Delta and scaled-LSE
+ * vectors of B*H*roundup(T,128) floats each; each part 256-byte aligned.
+ * Only the status words are part of the interface (see
+ * cattn_last_device_status). */
 CATTN_API size_t attn_bwd_workspace_bytes(int B, int H, int T, int D);
 
 /* Backward preprocess on its own: delta_i = sum_d dout_id * o_id (fp32),
@@ -170,9 +182,13 @@ CATTN_API cattn_status attn_bwd_ex(const void* q, const void* k, const void* v, 
  *
  * LSE stays a contiguous (B, H, T) fp32 vector; o_lo (if given) shares o's
  * layout.  Inputs may overlap one another (q, k, v in one buffer).  Outputs
- * must not overlap each other or any input: they would race.
+ * must not overlap each other or any input: they would race.  No output
+ * may overlap itself either, and that is checked: taking the axes of
+ * extent > 1 in increasing stride order (d first, stride 1, extent D),
+ * each stride must be at least the span of the axes before it (the
+ * contiguous layout, padded rows and the (B, T, C) output all pass).
  * Errors: as the contiguous calls, plus CATTN_ERR_INVALID_ARG for a stride
- * outside these limits. */
+ * outside these limits or a self-overlapping output layout. */
 typedef struct { long long b, h, t; } cattn_layout;
 
 /* attn_fwd_ex with strided q, k, v and o (o_lo uses o's layout). */
@@ -314,8 +330,25 @@ CATTN_API cattn_status attn_bwd_noalloc(const void* q, const void* k, const void
 /* Library-global device status word: CATTN_OK, or the first
  * CATTN_ERR_TIMEOUT recorded by a kernel since the last clear.  Reads it
  * synchronously (waits for all work on `stream`); clears it when `clear`
- * is non-zero. */
+ * is non-zero.  Every kernel records here, whatever its stream: this is
+ * the process-wide record, and the only one a forward call has. */
 CATTN_API cattn_status cattn_get_device_status(int clear, void* stream);
+
+/* Status of the last backward call that used `workspace` (attn_bwd and
+ * its _ex/_strided/_dropout forms): CATTN_OK, or the first error one of
+ * its kernels recorded (CATTN_ERR_TIMEOUT from the hang guard,
+ * CATTN_ERR_UNSUPPORTED for a launch the kernel could not honour).  The
+ * call's first kernel clears the words, so each call starts clean and the
+ * record is that call's alone; two streams with their own workspaces never
+ * see each other's failures.  Waits for all work on `stream` (the stream
+ * the backward ran on), then reads the word.
+ *   workspace : the call's workspace (device pointer, 256-byte aligned)
+ * Errors: CATTN_ERR_INVALID_ARG for a null or misaligned pointer,
+ * CATTN_ERR_CUDA if the wait or the read fails.  The word lives at offset 0
+ * of the workspace whatever the shape.  ("nanoGPT: a real GPT in two
+ * 300-line files" has no counterpart: PyTorch reports kernel failures
+ * through its own CUDA error state.) */
+CATTN_API cattn_status cattn_last_device_status(void* workspace, void* stream);
 
 /* Time limit of every mbarrier wait inside the kernels (the hang guard), in
  * microseconds.  0 restores the default of 2 s.  Process-global; affects
@@ -331,6 +364,16 @@ CATTN_API void cattn_set_wait_timeout_us(uint32_t us);
  * (CATTN_ERR_TIMEOUT expected), clearing it again.  Faults nothing; the
  * CUDA context stays usable.  Synchronises `stream`. */
 CATTN_API cattn_status cattn_selftest_wait_timeout(uint32_t timeout_us, void* stream);
+
+/* The same self-test recording into a backward workspace's status words:
+ * clears them, runs the waiting kernel on `stream` with `workspace` as its
+ * call's record, and returns cattn_last_device_status(workspace, stream)
+ * (CATTN_ERR_TIMEOUT expected).  The workspace keeps that record until a
+ * backward call reuses it.  The global word is left as it was found if it
+ * was clear before.  Synchronises `stream`.  Errors as
+ * cattn_last_device_status. */
+CATTN_API cattn_status cattn_selftest_wait_timeout_ws(uint32_t timeout_us, void* workspace,
+                                                      void* stream);
 
 /* Kernel timer (benchmarking aid).  While enabled, every kernel this
  * library launches is bracketed by two CUDA events recorded on its own
