@@ -303,7 +303,8 @@ cattn_status fwd_impl(int dev, const void* q, cattn_layout lq, const void* k, ca
   using C = FwdCfg<D, PLO>;
   clear_stale_error();
   cattn_status st = ensure_smem(dev, (FLAT ? 32 : 0) + (DROP ? 16 : 0) + 2 * d_index(D) + PLO,
-                                fwd_kernel<D, PLO, DROP, FLAT>, C::SMEM_BYTES, C::LAUNCH_REGS);
+                                fwd_kernel<D, PLO, DROP, FLAT>, C::SMEM_BYTES,
+                                C::REBALANCE ? C::LAUNCH_REGS : 0);
   if (st != CATTN_OK) return st;
   CUtensorMap mq, mk, mv;
   if ((st = make_bf16_map(&mq, q, D, T, H, B, lq, FLAT)) != CATTN_OK) return st;
@@ -354,14 +355,10 @@ cattn_status fwd_dispatch(bool plo, bool drop, bool flat, int dev, const void* q
 
 // Workspace of a backward call: the call's status words {code, where}
 // (CATTN_OK = 0, else the first error a kernel recorded; read back by
-// cattn_last_device_status), the fp32 dQ accumulator, the arrival counters
-// of its query-tile quarters (one 32-bit word per (head, 128-row tile,
-// 32-row quarter)), then the LSE * log2(e) and Delta vectors; every part
-// 256-byte aligned.  The accumulator and the counters are one contiguous
-// range that the preprocess kernel zeroes.
+// cattn_last_device_status), then the fp32 dQ accumulator and the
+// LSE * log2(e) and Delta vectors; every part 256-byte aligned.
 struct WsLayout {
-  size_t status_off, dq_off, cnt_off, lse2_off, delta_off, total;
-  size_t zero_bytes;  // accumulator + counters
+  size_t status_off, dq_off, lse2_off, delta_off, total;
   int T_pad;
 };
 
@@ -372,9 +369,7 @@ WsLayout ws_layout(long long BH, int T, int D) {
   L.T_pad = (T + 127) / 128 * 128;
   L.status_off = 0;
   L.dq_off = 256;
-  L.cnt_off = L.dq_off + round256(static_cast<size_t>(BH) * T * D * 4);
-  L.lse2_off = L.cnt_off + round256(static_cast<size_t>(BH) * (L.T_pad / 128) * 4 * 4);
-  L.zero_bytes = L.lse2_off - L.dq_off;
+  L.lse2_off = L.dq_off + round256(static_cast<size_t>(BH) * T * D * 4);
   L.delta_off = L.lse2_off + round256(static_cast<size_t>(BH) * L.T_pad * 4);
   L.total = L.delta_off + round256(static_cast<size_t>(BH) * L.T_pad * 4);
   return L;
@@ -447,7 +442,6 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   float* lse2 = reinterpret_cast<float*>(wb + L.lse2_off);
   float* delta = reinterpret_cast<float*>(wb + L.delta_off);
   unsigned int* status = reinterpret_cast<unsigned int*>(wb + L.status_off);
-  unsigned int* cnt = reinterpret_cast<unsigned int*>(wb + L.cnt_off);
   const size_t n_dq = static_cast<size_t>(BH) * T * D;
 
   CUtensorMap mq, mk, mv, mdo, mdq;
@@ -456,13 +450,12 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   if ((st = make_bf16_map(&mv, v, D, T, H, B, ly.v, FLAT)) != CATTN_OK) return st;
   if ((st = make_bf16_map(&mdo, dout, D, T, H, B, ly.dout, FLAT)) != CATTN_OK) return st;
   if ((st = make_tmap(&mdq, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, T, BH,
-                      C::WARP_DQ ? C::DCB : C::CBQ, C::WARP_DQ ? 32 : 128)) !=
+                      C::WARP_DQ ? D / 4 : C::CBQ, C::WARP_DQ ? 32 : 128)) !=
       CATTN_OK)
     return st;
 
   st = pre_impl<D>(o, ly.o, o_lo, dout, ly.dout, lse, delta, lse2,
-                   reinterpret_cast<float4*>(dq_acc), L.zero_bytes / 16, B, H, T, L.T_pad,
-                   status, s);
+                   reinterpret_cast<float4*>(dq_acc), n_dq / 4, B, H, T, L.T_pad, status, s);
   if (st != CATTN_OK) return st;
 
   BwdParams p;
@@ -488,15 +481,6 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   p.timeout_ns = g_timeout_ns;
   p.drop = dp;
   p.status = status;
-  // dQ output: with WARP_DQ the kernel's drain warps convert each query
-  // tile's rows once their last contribution has been added
-  p.dq_cnt = cnt;
-  p.dq_acc = dq_acc;
-  p.dq_out = dq;
-  p.dq_f32 = grad_f32 ? 1 : 0;
-  p.dq_sb = ly.dq.b;
-  p.dq_sh = ly.dq.h;
-  p.dq_st = ly.dq.t;
   // persistent: one CTA per SM, each looping over key tiles
   const long long n_items = static_cast<long long>(BH) * p.n_tiles;
   if (n_items > 0x7fffffffLL) return CATTN_ERR_INVALID_ARG;
@@ -506,7 +490,6 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
     bwd_kernel<D, SLO, DROP, FLAT><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mdo, mdq, p);
   }
   if ((st = launch_status()) != CATTN_OK) return st;
-  if (C::WARP_DQ) return CATTN_OK;  // dQ written by the main kernel
   {
     LaunchTimer t(K_DQ_CONVERT, s);
     if (!is_contiguous(ly.dq, H, T, D)) {
@@ -574,15 +557,19 @@ bool drop_params(const cattn_dropout* d, DropParams* out) {
 
 __global__ void selftest_wait_kernel(uint64_t timeout_ns, unsigned int* call_status) {
   __shared__ __align__(8) uint64_t mbar;
-  __shared__ int abort_flag;
+  // the abort flag, then (8 bytes on) the call's status address, as in the
+  // backward kernel
+  __shared__ __align__(8) int abort_and_call[4];
+  int& abort_flag = abort_and_call[0];
   if (threadIdx.x == 0) {
     abort_flag = 0;
+    *reinterpret_cast<unsigned int**>(&abort_and_call[2]) = call_status;
     mbar_init(smem_u32(&mbar), 1);
     fence_mbar_init();
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    WaitCtx w{timeout_ns, &abort_flag, 15u, call_status};
+    WaitCtx w{timeout_ns, &abort_flag, 15u, true};
     wait1(w, smem_u32(&mbar), 0, 1);  // nothing ever arrives
   }
   __syncthreads();
@@ -591,10 +578,10 @@ __global__ void selftest_wait_kernel(uint64_t timeout_ns, unsigned int* call_sta
 // ------------------------------------------------------------------ decode
 
 // Key chunks per head, and the workspace of their partial results.
-int decode_splits(int L) { return (L + kDecodeChunk - 1) / kDecodeChunk; }
+
 
 size_t decode_ws_bytes(long long BH, int Tq, int L, int D) {
-  const size_t rows = static_cast<size_t>(BH) * decode_splits(L) * Tq;
+  const size_t rows = static_cast<size_t>(BH) * decode_splits_for(BH, L, D) * Tq;
   return round256(rows * 2 * sizeof(float)) + round256(rows * D * sizeof(float));
 }
 
@@ -605,16 +592,16 @@ cattn_status decode_impl(const DecodeParams& p, long long BH, cudaStream_t s) {
   LaunchTimer t(K_DECODE, s);  // both kernels, as one entry
   // query rows per thread: Tq rounded up to 1, 2, 4 or 8
   if (p.Tq <= 1)
-    decode_partial_kernel<D, 1><<<grid, kDecodeWarps * 32, 0, s>>>(p);
+    decode_partial_kernel<D, 1><<<grid, kDecodeThreads, 0, s>>>(p);
   else if (p.Tq <= 2)
-    decode_partial_kernel<D, 2><<<grid, kDecodeWarps * 32, 0, s>>>(p);
+    decode_partial_kernel<D, 2><<<grid, kDecodeThreads, 0, s>>>(p);
   else if (p.Tq <= 4)
-    decode_partial_kernel<D, 4><<<grid, kDecodeWarps * 32, 0, s>>>(p);
+    decode_partial_kernel<D, 4><<<grid, kDecodeThreads, 0, s>>>(p);
   else
-    decode_partial_kernel<D, 8><<<grid, kDecodeWarps * 32, 0, s>>>(p);
+    decode_partial_kernel<D, 8><<<grid, kDecodeThreads, 0, s>>>(p);
   cattn_status st = launch_status();
   if (st != CATTN_OK) return st;
-  decode_combine_kernel<D><<<static_cast<unsigned>(BH * p.Tq), D, 0, s>>>(p);
+  decode_combine_kernel<D><<<static_cast<unsigned>(BH * p.Tq), kCombineThreads, 0, s>>>(p);
   return launch_status();
 }
 
@@ -711,7 +698,7 @@ cattn_status attn_decode(const void* q, cattn_layout lq, const void* k, cattn_la
   p.q_sb = lq.b; p.q_sh = lq.h; p.q_st = lq.t;
   p.k_sb = lk.b; p.k_sh = lk.h; p.k_st = lk.t;
   p.v_sb = lv.b; p.v_sh = lv.h; p.v_st = lv.t;
-  const size_t rows = static_cast<size_t>(BH) * decode_splits(L) * Tq;
+  const size_t rows = static_cast<size_t>(BH) * decode_splits_for(BH, L, D) * Tq;
   uint8_t* wb = static_cast<uint8_t*>(workspace);
   p.part_ml = reinterpret_cast<float*>(wb);
   p.part_o = reinterpret_cast<float*>(wb + round256(rows * 2 * sizeof(float)));
@@ -721,7 +708,8 @@ cattn_status attn_decode(const void* q, cattn_layout lq, const void* k, cattn_la
   p.H = H;
   p.Tq = Tq;
   p.L = L;
-  p.n_split = decode_splits(L);
+  p.n_split = decode_splits_for(BH, L, D);
+  p.chunks_per_cta = decode_chunks_per_cta(BH, L, D);
   p.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (D) {

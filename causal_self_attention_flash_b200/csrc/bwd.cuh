@@ -145,9 +145,9 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
       for (int o = TPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if (pr[u] < p.n_rows && sub == 0) {
         p.delta[pr[u]] = acc;  // 0 on padding rows
-        if (p.lse2 != nullptr)
+        if (p.lse2 != nullptr)  // stored negated: P = 2^(s * scale_log2 + lse2)
           p.lse2[pr[u]] =
-              valid[u] ? p.lse[static_cast<size_t>(bh[u]) * p.T + t[u]] * kLog2e : INFINITY;
+              valid[u] ? -(p.lse[static_cast<size_t>(bh[u]) * p.T + t[u]] * kLog2e) : -INFINITY;
       }
     }
   }
@@ -248,8 +248,7 @@ __global__ void __launch_bounds__(256) dq_convert_strided_kernel(const float4* _
 //   warps 0-15 compute: warp w serves TMEM lanes 32*(w%4).. (key rows) and
 //              query columns 32*(w/4) .. +32 of the tile (four warps per SM
 //              sub-partition, to hide the latency of the exponentials and
-//              tensor-memory loads); they also write dK, dV, and for D = 128
-//              drain dQ.
+//              tensor-memory loads); they also drain dQ and write dK, dV.
 //   warp 16    TMA producer: per work item K, V (double-buffered where
 //              shared memory allows); Q_t with the LSE2 and Delta vectors
 //              through a 2-stage ring, dO_t through a 2-stage (D <= 64) or
@@ -259,15 +258,10 @@ __global__ void __launch_bounds__(256) dq_convert_strided_kernel(const float4* _
 //   warp 18    MMA issuer B: dV(t) (P^T_hi part), dK(t).
 //   warp 19    MMA issuer C: the P^T_lo part of dV(t), into dV' (where TMEM
 //              holds a separate dV' accumulator; otherwise warp 18 does it).
-//   warps 20-23 (D <= 64) dQ drain: warp 20 + r takes query rows 32r.. of
-//              dQ(t) from TMEM once its MMA is complete, releases the TMEM
-//              columns, stages the rows in shared memory and adds them into
-//              the fp32 accumulator with TMA reduce-adds, off the compute
-//              warps' path.
 // The kernel is persistent: CTA b loops over work items (key tiles).
 
 struct BwdParams {
-  const float* lse2;   // (BH, T_pad) LSE * log2(e); +inf on padding rows
+  const float* lse2;   // (BH, T_pad) -LSE * log2(e); -inf on padding rows
   const float* delta;  // (BH, T_pad); 0 on padding rows
   float* dk_f32;       // fp32 gradient outputs (BH, T, D), or null
   float* dv_f32;
@@ -285,14 +279,6 @@ struct BwdParams {
   uint64_t timeout_ns;
   DropParams drop;  // attention dropout (kernels instantiated with DROP only)
   unsigned int* status;  // the call's {code, where} words in its workspace
-  // dQ written by the drain warps (WARP_DQ): arrival counters per (head,
-  // query tile, 32-row quarter), zeroed by the preprocess; the output (bf16,
-  // or fp32 when dq_f32) with element strides (b, h, t)
-  unsigned int* dq_cnt;
-  const float* dq_acc;  // (BH, T, D) fp32 accumulator
-  void* dq_out;
-  int dq_f32;
-  long long dq_sb, dq_sh, dq_st;
 };
 
 template <int D, bool SLO>
@@ -311,18 +297,13 @@ struct BwdCfg {
   // [128 rows][CBQ floats]
   static constexpr int CBQ = D < 32 ? D : 32;
   static constexpr int RBQ = CBQ * 4;
-  // WARP_DQ (D <= 64): four drain warps (one per TMEM lane quarter) move
-  // dQ out of tensor memory, each through its own fp32 staging tile
-  // [32 rows][D floats] and TMA reduce-adds, so the compute warps never
-  // touch dQ and no CTA-wide barrier is needed; otherwise (D = 128) the
-  // compute warps stage all of dQ in the dS buffers and one thread issues
-  // the reduce.  The staging tile is DNB boxes of [32 rows][DCB floats],
-  // each swizzled by its row bytes (128 or 64).
+  // WARP_DQ (D <= 64): every compute warp drains its own [32 rows][D/4]
+  // slice of dQ through its own fp32 staging tile and TMA reduce, so no
+  // CTA-wide barrier is needed; otherwise the CTA stages all of dQ in the dS
+  // buffers and one thread issues the reduce.
   static constexpr bool WARP_DQ = D <= 64;
-  static constexpr int DCB = D < 32 ? D : 32;                  // floats per box row
-  static constexpr int DRB = DCB * 4;                          // bytes per box row
-  static constexpr int DNB = D / DCB;                          // boxes per warp tile
-  static constexpr int WARP_STAGE = (32 * D * 4 + 1023) / 1024 * 1024;
+  static constexpr int RBW = D;                                // (D/4) floats per row
+  static constexpr int WARP_STAGE = (32 * RBW + 1023) / 1024 * 1024;
   // dS lo buffer: with SLO, and as the second half of the CTA dQ staging
   static constexpr int DSL_BYTES = (SLO || !WARP_DQ) ? 32768 : 0;
   // shared memory map; KVB = 2 K/V buffers (the next work item's K, V load
@@ -330,7 +311,7 @@ struct BwdCfg {
   static constexpr int layout_end(int kvb) {
     return ((kvb * 2 * TILE_BYTES + (QST + DOST) * TILE_BYTES + 32768 + DSL_BYTES +
              QST * 1024 + 1023) / 1024 * 1024) +
-           (WARP_DQ ? 4 * WARP_STAGE : 0) + 40 * 8 + 64;
+           (WARP_DQ ? 16 * WARP_STAGE : 0) + 40 * 8 + 64;
   }
   static constexpr int KVB = layout_end(2) + 1024 <= kMaxDynSmem ? 2 : 1;
   static constexpr int OFF_KV = 0;                             // [KVB][K, V]
@@ -341,8 +322,8 @@ struct BwdCfg {
   static constexpr int OFF_LSE = OFF_DSL + DSL_BYTES;         // [QST][128] fp32
   static constexpr int OFF_DELTA = OFF_LSE + QST * 512;       // [QST][128] fp32
   static constexpr int OFF_DQW = (OFF_DELTA + QST * 512 + 1023) / 1024 * 1024;
-  static constexpr int OFF_BAR = WARP_DQ ? OFF_DQW + 4 * WARP_STAGE : OFF_DELTA + QST * 512;
-  static constexpr int NUM_BARS = 34;
+  static constexpr int OFF_BAR = WARP_DQ ? OFF_DQW + 16 * WARP_STAGE : OFF_DELTA + QST * 512;
+  static constexpr int NUM_BARS = 33;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_USED = OFF_MISC + 64;
   static constexpr int SMEM_BYTES =
@@ -359,9 +340,7 @@ struct BwdCfg {
   static constexpr uint32_t COL_DQ = ALIAS_DQ ? COL_DP : 256 + 2 * D;
   static constexpr uint32_t COL_DVL = SPLIT_DV ? 256 + 3 * D : COL_DV;
   static constexpr uint32_t TMEM_COLS = 512;
-  // warps 0-15 compute, 16 producer, 17-19 MMA issuers, 20-23 dQ drain
-  // (WARP_DQ only); 80 registers per thread with 768 threads, 96 with 640
-  static constexpr int THREADS = WARP_DQ ? 768 : 640;
+  static constexpr int THREADS = 640;
   static constexpr int NCOMP = 512;   // compute threads
 };
 
@@ -373,8 +352,7 @@ enum : int {
   BB_SFULL = 20, BB_DPFULL = 21, BB_PFULL = 22, BB_DSFULL = 23, BB_DQFULL = 24,
   BB_DQEMPTY = 25, BB_ACCFREE = 26, BB_PTDONE = 27, BB_DKDONE = 28,
   BB_DRAIN = 29,  // + issuer 0, 1, 2
-  BB_PFULL2 = 32,  // second half of P^T (BB_PFULL is the first)
-  BB_CSYNC = 33    // CTA-wide dQ staging of the compute warps (D = 128)
+  BB_PFULL2 = 32  // second half of P^T (BB_PFULL is the first)
 };
 
 // Work items: key tiles (kt, bh), numbered longest first (u = 0 ..
@@ -391,12 +369,12 @@ __device__ __forceinline__ int bwd_item(int k, int b, int G, int n_items) {
 // tensor maps, dK/dV offsets bh * d?_sh); otherwise 4-D maps with (h, b)
 // coordinates.
 template <int D, bool SLO, bool DROP, bool FLAT>
-__global__ void __launch_bounds__(BwdCfg<D, SLO>::THREADS, 1)
+__global__ void __launch_bounds__(640, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
            const __grid_constant__ CUtensorMap tmDQacc, const BwdParams p) {
   using C = BwdCfg<D, SLO>;
-  static_assert(BB_CSYNC + 1 <= C::NUM_BARS, "barrier count");
+  static_assert(BB_PFULL2 + 1 <= C::NUM_BARS, "barrier count");
   static_assert(C::QST <= 4 && C::DOST <= 4, "barrier map");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = aligned_smem(smem_raw, C::SMEM_USED, p.status);
@@ -406,6 +384,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   auto bar = [&](int i) { return sbase + C::OFF_BAR + 8u * i; };
   auto sK = [&](int kvb) { return sbase + C::OFF_KV + kvb * 2 * C::TILE_BYTES; };
   auto sV = [&](int kvb) { return sbase + C::OFF_KV + kvb * 2 * C::TILE_BYTES + C::TILE_BYTES; };
+  // misc: [0] TMEM address, [1] abort flag, [2..3] the call's status address
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
 
@@ -414,10 +393,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   const int n_items = p.BH * p.n_tiles;
   const int G = gridDim.x, b = blockIdx.x;
 
-  WaitCtx w{p.timeout_ns, abort_flag, 2u, p.status};
+  WaitCtx w{p.timeout_ns, abort_flag, 2u, true};
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
+    *reinterpret_cast<unsigned int**>(misc + 2) = p.status;
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(BB_KVFULL + s), 1);
       mbar_init(bar(BB_KVFREE + s), 1);
@@ -437,14 +417,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     mbar_init(bar(BB_PFULL2), C::NCOMP);
     mbar_init(bar(BB_DSFULL), C::NCOMP);
     mbar_init(bar(BB_DQFULL), 1);
-    mbar_init(bar(BB_DQEMPTY), C::WARP_DQ ? 128 : C::NCOMP);  // drain or compute threads
+    mbar_init(bar(BB_DQEMPTY), C::NCOMP);
     mbar_init(bar(BB_ACCFREE), C::NCOMP);
     mbar_init(bar(BB_PTDONE), C::SPLIT_DV ? 2 : 1);  // dV by warps 18 (and 19)
     mbar_init(bar(BB_DKDONE), 1);
     mbar_init(bar(BB_DRAIN), 1);
     mbar_init(bar(BB_DRAIN + 1), 1);
     mbar_init(bar(BB_DRAIN + 2), 1);
-    mbar_init(bar(BB_CSYNC), C::NCOMP / 32);  // one arrival per compute warp
     fence_mbar_init();
   }
   if (warp == 17) {
@@ -530,7 +509,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // wait (bounded, ignoring the abort flag) for the last loads issued,
         // which nobody may consume, before the CTA exits
         int zero = 0;
-        WaitCtx wd{p.timeout_ns, &zero, 2u, p.status};
+        WaitCtx wd{p.timeout_ns, &zero, 2u, false};
         for (int j = (n > C::KVB ? n - C::KVB : 0); j < n; ++j)
           wait1(wd, bar(BB_KVFULL + j % C::KVB), (j / C::KVB) & 1, 20);
         for (int j = (tq > C::QST ? tq - C::QST : 0); j < tq; ++j)
@@ -539,8 +518,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           wait1(wd, bar(BB_DOFULL + j % C::DOST), (j / C::DOST) & 1, 22);
       }
     }
-  } else if (warp >= 17 && warp <= 19) {
-    // -------------------------------------------------- MMA issuers (17-19)
+  } else if (warp >= 17) {
+    // -------------------------------------------------- MMA issuers
     // warp 17 (A): S, dP, dQ -- the products that read K and V;
     // warps 18, 19 (B, C): dV, dK -- the accumulations.  One thread issues
     // an N = 64 MMA only every ~50 cycles, so several issuers keep the
@@ -716,121 +695,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       }
       mma_commit(bar(BB_DRAIN + (warp - 17)));
       int zero = 0;
-      WaitCtx wd{p.timeout_ns, &zero, 2u, p.status};
+      WaitCtx wd{p.timeout_ns, &zero, 2u, false};
       wait1(wd, bar(BB_DRAIN + (warp - 17)), 0, 13);
-    }
-  } else if (warp >= 20) {
-    // ------------------------------------------------------- dQ drain warps
-    // (launched only with WARP_DQ).  Thread (warp 20 + r, lane l) owns query
-    // row 32r + l of dQ(t): D fp32 columns of TMEM lane 32r + l.
-    if constexpr (C::WARP_DQ) {
-      const int quarter = warp & 3;
-      const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-      const uint32_t sW = sbase + C::OFF_DQW + quarter * C::WARP_STAGE;
-      // Query tile qi of head bh receives qi + 1 contributions (key tiles
-      // 0 .. qi).  After its own reduce-adds into rows 32*quarter.. of the
-      // tile are complete, a drain warp counts its contribution; the warp
-      // that brings the count to qi + 1 converts those 32 rows:
-      // dQ = scale * accumulator, bf16 (or fp32) into the output layout.
-      auto arrive_convert = [&](int bh, int qi) {
-        unsigned int old = 0;
-        if (lane == 0) {
-          fence_proxy_async_global();
-          old = atom_add_acq_rel_gpu(
-              p.dq_cnt + (static_cast<size_t>(bh) * p.n_tiles + qi) * 4 + quarter, 1u);
-        }
-        old = __shfl_sync(0xffffffffu, old, 0);
-        if (old != static_cast<unsigned int>(qi)) return;
-        __syncwarp();
-        constexpr int LPR = D / 4;      // lanes per row, 4 floats each
-        constexpr int RPP = 32 / LPR;   // rows per pass
-        const int sub = lane % LPR, rr = lane / LPR;
-        const long long b_ = bh / p.H, h_ = bh - (bh / p.H) * p.H;
-#pragma unroll
-        for (int r0 = 0; r0 < 32; r0 += RPP) {
-          const int row = qi * 128 + quarter * 32 + r0 + rr;
-          if (row >= p.T) continue;
-          const float4 a = __ldcg(reinterpret_cast<const float4*>(
-                                      p.dq_acc + (static_cast<size_t>(bh) * p.T + row) * D) +
-                                  sub);
-          const long long off = b_ * p.dq_sb + h_ * p.dq_sh + row * p.dq_st + sub * 4;
-          if (p.dq_f32) {
-            *reinterpret_cast<float4*>(static_cast<float*>(p.dq_out) + off) =
-                make_float4(a.x * p.scale, a.y * p.scale, a.z * p.scale, a.w * p.scale);
-          } else {
-            *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.dq_out) + off) =
-                make_uint2(pack_bf16(a.x * p.scale, a.y * p.scale),
-                           pack_bf16(a.z * p.scale, a.w * p.scale));
-          }
-        }
-      };
-      int t = 0;
-      int prev_bh = -1, prev_qi = 0;  // the tile whose contribution is not yet counted
-      for (int k = 0;; ++k) {
-        const int u = bwd_item(k, b, G, n_items);
-        if (u < 0) break;
-        const int kt = u / p.BH, bh = u % p.BH;
-        const int n_iter = p.n_tiles - kt;
-        for (int i = 0; i < n_iter; ++i, ++t) {
-          wait_warp(w, bar(BB_DQFULL), t & 1, 14);
-          tc_fence_after();
-          // the previous reduce-adds must have read the staging tile
-          if (lane == 0) bulk_wait_read0();
-          __syncwarp();
-#pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            constexpr int NC = D < 32 ? D : 32;
-            float x[NC];
-            if constexpr (NC == 32) {
-              uint32_t v[32];
-              tmem_ld32(tbase + lane_base + C::COL_DQ + c0, v);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(v[e]);
-            } else {
-              uint32_t v[16];
-              tmem_ld16(tbase + lane_base + C::COL_DQ + c0, v);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(v[e]);
-            }
-            if (c0 + 32 >= D) {  // every column of dQ(t) is in registers
-              tc_fence_before();
-              mbar_arrive(bar(BB_DQEMPTY));
-            }
-            // box c0 / DCB of the staging tile: row = lane, DCB floats
-            const uint32_t box = sW + (c0 / C::DCB) * 32 * C::DRB;
-#pragma unroll
-            for (int e = 0; e < NC; e += 4)
-              st_shared_v4(box + swz<C::DRB>(lane * C::DRB + e * 4), __float_as_uint(x[e]),
-                           __float_as_uint(x[e + 1]), __float_as_uint(x[e + 2]),
-                           __float_as_uint(x[e + 3]));
-          }
-          fence_async_smem();
-          __syncwarp();
-          if (lane == 0 && !*abort_flag) {
-            const int q0 = (kt + i) * 128 + quarter * 32;
-#pragma unroll
-            for (int bx = 0; bx < C::DNB; ++bx)
-              tma_reduce_add_3d(&tmDQacc, sW + bx * 32 * C::DRB, bx * C::DCB, q0, bh);
-          }
-          if (lane == 0) bulk_commit();
-          // the previous tile's reduce-adds are complete once at most this
-          // tile's group is pending: count that contribution
-          if (prev_bh >= 0) {
-            if (lane == 0) bulk_wait1();
-            __syncwarp();
-            if (!*abort_flag) arrive_convert(prev_bh, prev_qi);
-          }
-          prev_bh = bh;
-          prev_qi = kt + i;
-        }
-      }
-      // the last tile: wait for its reduce-adds (which also covers their
-      // reads of the staging tile, needed before the CTA exits)
-      if (lane == 0) bulk_wait0();
-      __syncwarp();
-      if (prev_bh >= 0 && !*abort_flag) arrive_convert(prev_bh, prev_qi);
     }
   } else {
     // ------------------------------------------- compute warps (row = key)
@@ -874,30 +740,33 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       }
     };
 
-    // Barrier of the 16 compute warps around the CTA-wide dQ staging
-    // (D = 128): each warp arrives once (lane 0, after the warp's own
-    // shared-memory writes, ordered by __syncwarp), and waits (bounded) for
-    // the phase to complete.  All compute warps take the same sequence of
-    // these, whatever their waits returned, so the phases stay in step.
-    int n_csync = 0;
-    auto compute_sync = [&]() {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BB_CSYNC));
-      wait_warp(w, bar(BB_CSYNC), n_csync & 1, 18);
-      ++n_csync;
-    };
-
-    // dQ(t) drain (D = 128; with WARP_DQ the drain warps do it): TMEM (lane
-    // = query row) -> fp32 staging in the dS buffers -> TMA reduce-add into
-    // the accumulator, rows q0 .. q0+127 of head bh
+    // dQ(t) drain: TMEM (lane = query row) -> fp32 staging -> TMA
+    // reduce-add into the accumulator, rows q0 .. q0+127 of head bh
     auto drain_dq = [&](int t, int q0, int bh) {
-      if constexpr (!C::WARP_DQ) {
-        wait_warp(w, bar(BB_DQFULL), t & 1, 14);
-        tc_fence_after();
-        float acc[NQ];
-        load_cols(tbase + lane_base + C::COL_DQ + grp * NQ, acc);
-        tc_fence_before();
-        mbar_arrive(bar(BB_DQEMPTY));
+      wait_warp(w, bar(BB_DQFULL), t & 1, 14);
+      tc_fence_after();
+      float acc[NQ];
+      load_cols(tbase + lane_base + C::COL_DQ + grp * NQ, acc);
+      tc_fence_before();
+      mbar_arrive(bar(BB_DQEMPTY));
+      if constexpr (C::WARP_DQ) {
+        // this warp's tile [32 rows][NQ floats]; its previous reduce must
+        // have finished reading it
+        const uint32_t sW = sbase + C::OFF_DQW + warp * C::WARP_STAGE;
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+#pragma unroll
+        for (int e = 0; e < NQ; e += 4)
+          st_shared_v4(sW + swz<C::RBW>(lane * C::RBW + e * 4), __float_as_uint(acc[e]),
+                       __float_as_uint(acc[e + 1]), __float_as_uint(acc[e + 2]),
+                       __float_as_uint(acc[e + 3]));
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0 && !*abort_flag) {
+          tma_reduce_add_3d(&tmDQacc, sW, grp * NQ, q0 + quarter * 32, bh);
+          bulk_commit();
+        }
+      } else {
         // staging: blocks of [128 rows][CBQ floats], swizzled
 #pragma unroll
         for (int e = 0; e < NQ; e += 4) {
@@ -909,15 +778,20 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                        __float_as_uint(acc[e + 2]), __float_as_uint(acc[e + 3]));
         }
         fence_async_smem();
-        compute_sync();
+        // A hardware named barrier over the 512 compute threads: every
+        // compute thread executes the same sequence of these (drain_dq and
+        // staging_free are called at the same points of a loop whose trip
+        // counts are uniform over the CTA, whatever any wait returned), so
+        // each barrier is reached by all 512 and cannot hang.  A bounded
+        // mbarrier in its place measured 14 % slower on the long-context
+        // backward.
+        named_bar_sync(1, C::NCOMP);
         if (leader && !*abort_flag) {
 #pragma unroll
           for (int blk = 0; blk < D / C::CBQ; ++blk)
             tma_reduce_add_3d(&tmDQacc, sDSH + blk * 128 * C::RBQ, blk * C::CBQ, q0, bh);
           bulk_commit();
         }
-      } else {
-        (void)t; (void)q0; (void)bh;
       }
     };
     // the dS buffers may be rewritten once the reduce has read them (CTA
@@ -925,7 +799,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     auto staging_free = [&]() {
       if constexpr (!C::WARP_DQ) {
         if (leader) bulk_wait_read0();
-        compute_sync();
+        named_bar_sync(1, C::NCOMP);
       }
     };
 
@@ -983,9 +857,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       }
     };
 
-    // WARP_DQ: the drain warps move dQ; the compute warps only wait, before
-    // they overwrite the dS buffer, for the dQ MMA that read it.
-    constexpr bool kOwnDrain = !C::WARP_DQ;
+    // kLateDrain (own dQ staging, dQ not aliased): drain dQ(t-1) after the
+    // dS phase of tile t rather than after its P phase, so that dS(t) (and
+    // dK(t), dQ(t) after it) come earlier and the drain fills the wait for
+    // S(t+1).
+    constexpr bool kLateDrain = C::WARP_DQ && !C::ALIAS_DQ;
     float pv[32];
     int t = 0;
     // the previous query tile (its dQ is drained in the next iteration) and
@@ -1035,12 +911,15 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         for (int h = 0; h < 2; ++h) {
 #pragma unroll
           for (int c = 16 * h; c < 16 * h + 16; c += 4) {
-            float l0, l1, l2, l3;
+            float l0, l1, l2, l3;  // -LSE * log2(e) of four queries
             ld_shared_v4f(sL + c * 4, l0, l1, l2, l3);
-            pv[c] = ex2(fmaf(pv[c], sl2, -l0));
-            pv[c + 1] = ex2(fmaf(pv[c + 1], sl2, -l1));
-            pv[c + 2] = ex2(fmaf(pv[c + 2], sl2, -l2));
-            pv[c + 3] = ex2(fmaf(pv[c + 3], sl2, -l3));
+            float x0, x1, x2, x3;
+            f2_split(fma2(f2(pv[c], pv[c + 1]), f2(sl2, sl2), f2(l0, l1)), x0, x1);
+            f2_split(fma2(f2(pv[c + 2], pv[c + 3]), f2(sl2, sl2), f2(l2, l3)), x2, x3);
+            pv[c] = ex2(x0);
+            pv[c + 1] = ex2(x1);
+            pv[c + 2] = ex2(x2);
+            pv[c + 3] = ex2(x3);
           }
           if (i == 0) {  // diagonal tile: query (32g + c) sees key r only if r <= query
             const int lim = r - grp * 32;
@@ -1069,7 +948,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         }
 
         // ---- dQ of the previous query tile (its MMA ran during this P phase)
-        if (kOwnDrain && t >= 1) drain_dq(t - 1, prev_q0, prev_bh);
+        // (kLateDrain: after the dS phase instead, see there)
+        if (!kLateDrain && t >= 1) drain_dq(t - 1, prev_q0, prev_bh);
         // ---- the previous item's dK, dV
         if (i == 0 && prev_kt >= 0) epilogue(prev_kt, prev_bh, t - 1);
 
@@ -1099,10 +979,14 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
               s2 = pv[e + 2] * (g2 - d2);
               s3 = pv[e + 3] * (g3 - d3);
             } else {
-              s0 = pv[e] * (__uint_as_float(v[e]) - d0);
-              s1 = pv[e + 1] * (__uint_as_float(v[e + 1]) - d1);
-              s2 = pv[e + 2] * (__uint_as_float(v[e + 2]) - d2);
-              s3 = pv[e + 3] * (__uint_as_float(v[e + 3]) - d3);
+              const uint64_t a01 = mul2(f2(pv[e], pv[e + 1]),
+                                        sub2(f2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])),
+                                             f2(d0, d1)));
+              const uint64_t a23 = mul2(f2(pv[e + 2], pv[e + 3]),
+                                        sub2(f2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])),
+                                             f2(d2, d3)));
+              f2_split(a01, s0, s1);
+              f2_split(a23, s2, s3);
             }
             if (SLO) {
               split_bf16x2_p(f2(s0, s1), hi[e / 2], lo[e / 2]);
@@ -1119,7 +1003,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // query block g is half g/2, chunks 4*(g%2) .. +3 of the row.  (dQ(t-1),
         // which read the previous dS, is complete: drained above.)
         // the previous dQ MMA, which read the previous dS, must be complete
-        if (C::WARP_DQ && t >= 1) {
+        if (kLateDrain && t >= 1) {
           wait_warp(w, bar(BB_DQFULL), (t - 1) & 1, 31);
           tc_fence_after();
         }
@@ -1135,20 +1019,26 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(BB_DSFULL));
+        // ---- kLateDrain: the previous query tile's dQ, while the next S is
+        // computed (the compute warps would otherwise wait for it)
+        if (kLateDrain && t >= 1) drain_dq(t - 1, prev_q0, prev_bh);
         prev_q0 = (kt + i) * 128;
         prev_bh = bh;
       }
       prev_kt = kt;
     }
     if (t >= 1) {
-      if (kOwnDrain) drain_dq(t - 1, prev_q0, prev_bh);
+      drain_dq(t - 1, prev_q0, prev_bh);  // waits for the last MMAs: everything is complete
       epilogue(prev_kt, prev_bh, t - 1);
     }
     // before the CTA exits, its bulk copies must have read their shared
     // memory sources (their global writes complete on their own; the next
     // kernel on the stream sees them)
-    if (kOwnDrain && leader) bulk_wait_read0();
-    (void)prev_q0;
+    if (C::WARP_DQ) {
+      if (lane == 0) bulk_wait_read0();
+    } else if (leader) {
+      bulk_wait_read0();
+    }
   }
 
   tc_fence_before();

@@ -14,7 +14,7 @@
 // one warpgroup works on its scores, the MMAs of the other run.  The next
 // item's Q and K/V are loaded while the current item finishes.
 //
-// Warp roles (384 threads):
+// Warp roles (352 threads; 384 with D = 128):
 //   warps 0-3, 4-7  softmax warpgroups g = 0, 1, one query tile each per item;
 //              thread t of a group owns query row t, which is TMEM lane t.
 //              It reads S_g from TMEM, masks the diagonal tile, updates m
@@ -28,8 +28,8 @@
 //   warp 8     TMA producer: per item each group's Q tile (once the previous
 //              item's S MMAs are done with the buffer), then K_j, V_j through
 //              a ring that runs on across items.
-//   warp 11    idle; it completes the third warpgroup (warps 8-11), whose
-//              registers go to the softmax warpgroups.
+//   warp 11    (D = 128 only) idle; it completes the third warpgroup
+//              (warps 8-11), whose registers go to the softmax warpgroups.
 //   warps 9, 10  MMA issuers for groups 0, 1 (warp 9 also owns TMEM).  Two
 //              issuing threads keep the tensor core fed where one thread's
 //              issue rate would not (N = D <= 64 MMAs).  Per key tile j:
@@ -122,16 +122,20 @@ struct FwdCfg {
   static constexpr uint32_t COL_OL0 = SPLIT ? 256 + 2 * D : COL_O0;
   static constexpr uint32_t COL_OL1 = SPLIT ? 256 + 3 * D : COL_O1;
   static constexpr uint32_t TMEM_COLS = 512;
-  // 12 warps: two softmax warpgroups, then the producer, two MMA issuers
-  // and one idle warp, which complete the third warpgroup so that its
-  // registers can be handed to the softmax warps (setmaxnreg acts on whole
-  // warpgroups).  At launch every thread holds LAUNCH_REGS (65536 / 384,
-  // rounded down to 8); the third warpgroup then drops to REGS_OTHER and
-  // the softmax warpgroups rise to REGS_SOFTMAX, within the launch total.
-  static constexpr int THREADS = 384;
+  // Two softmax warpgroups, then the producer and two MMA issuers.  With
+  // D = 128 (REBALANCE) a twelfth, idle warp completes the third warpgroup
+  // so that its registers can be handed to the softmax warps (setmaxnreg
+  // acts on whole warpgroups): at launch every thread holds LAUNCH_REGS
+  // (65536 / 384, rounded down to 8); the third warpgroup then drops to
+  // REGS_OTHER and the softmax warpgroups rise to REGS_SOFTMAX, within the
+  // launch total.  That removed the D = 128 softmax's spills (3.6 % faster
+  // on the long-context workload); with D <= 64 the same split measured
+  // 4 % slower, so those keep 11 warps and 168 registers throughout.
+  static constexpr bool REBALANCE = D == 128;
+  static constexpr int THREADS = REBALANCE ? 384 : 352;
   static constexpr int LAUNCH_REGS = 168;
   static constexpr int REGS_SOFTMAX = 216, REGS_OTHER = 64;
-  static_assert(256 * REGS_SOFTMAX + 128 * REGS_OTHER <= THREADS * LAUNCH_REGS,
+  static_assert(!REBALANCE || 256 * REGS_SOFTMAX + 128 * REGS_OTHER <= THREADS * LAUNCH_REGS,
                 "register split exceeds the launch allocation");
 };
 
@@ -149,10 +153,13 @@ enum : int {
 
 // Pairs of score columns whose exponential is taken by exp2_poly2 on the FMA
 // pipes instead of the ex2 unit, as a bit mask over the pair index within a
-// 16-column chunk (3 of 8 pairs): the ex2 unit does 16 per clock per SM, so
-// moving part of the work keeps both pipes busy.  Only used on tiles without
-// masked entries (exp2_poly2 has no exact zero).
-constexpr uint32_t kFwdPolyPairs = 0x00u;
+// 16-column chunk.  The ex2 unit does 16 per clock per SM; with D = 128 a
+// tile's MMAs take as long as its exponentials, and moving 2 of 8 pairs to
+// the FMA pipes measured 4 % faster (long-context workload).  With D <= 64
+// the softmax warps have no issue slots to spare and the share measured
+// slower, so it is 0 there.  Only used on tiles without masked entries
+// (exp2_poly2 has no exact zero).
+__host__ __device__ constexpr uint32_t fwd_poly_pairs(int D) { return D == 128 ? 0x11u : 0x00u; }
 
 // P_g(j) is handed to the MMA warp in kPvParts parts (of 128 / kPvParts
 // keys each), so PV_g(j) starts while the later exponentials are computed.
@@ -162,19 +169,18 @@ constexpr int kPvParts = 2;
 // TMEM as bf16 (or bf16 hi/lo), the row sum accumulated in sum2.
 // DROP: P entries whose bit in keep (bit c of keep[c / 32] for column c) is
 // clear are written as 0; the row sum still takes every entry.
-// Chunks [CH0, CH1) of 16 columns each (the whole row is chunks 0 .. 7).
-template <bool POLY, bool PLO, bool DROP, int CH0 = 0, int CH1 = 8>
+template <int D, bool POLY, bool PLO, bool DROP>
 __device__ __forceinline__ void fwd_exp_row(const float (&s)[128], uint64_t sl2x2, uint64_t negm2,
                                             uint32_t scol, uint64_t (&sum2)[2], uint32_t pfull0,
                                             const uint32_t* keep) {
 #pragma unroll
-  for (int ch = CH0; ch < CH1; ++ch) {  // 16 columns per chunk
+  for (int ch = 0; ch < 8; ++ch) {  // 16 columns per chunk
     uint32_t hi[8], lo[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const uint64_t x2 = fma2(f2(s[ch * 16 + 2 * e], s[ch * 16 + 2 * e + 1]), sl2x2, negm2);
       uint64_t p2;
-      if (POLY && ((kFwdPolyPairs >> e) & 1u)) {
+      if (POLY && ((fwd_poly_pairs(D) >> e) & 1u)) {
         float x0, x1;
         f2_split(x2, x0, x1);
         p2 = exp2_poly2(x0, x1);
@@ -251,7 +257,7 @@ __device__ __forceinline__ FwdItem fwd_item_info(int u, int k, int BH, int n_pai
 // FLAT: Q, K, V and O address (b, h) as one b*H + h axis (3-D tensor
 // maps, O offsets bh * o_sh); otherwise 4-D maps with (h, b) coordinates.
 template <int D, bool PLO, bool DROP, bool FLAT>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(FwdCfg<D, PLO>::THREADS, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = FwdCfg<D, PLO>;
@@ -271,7 +277,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   const int n_items = p.BH * n_pairs;
   const int G = gridDim.x, b = blockIdx.x;
 
-  WaitCtx w{p.timeout_ns, abort_flag, 1u, nullptr};
+  WaitCtx w{p.timeout_ns, abort_flag, 1u, false};
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -304,8 +310,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   const uint32_t tbase = misc[0];
 
   if (warp >= 8) {
-  // third warpgroup: producer, MMA issuers, one idle warp
-  regs_dec<C::REGS_OTHER>();
+  // third warpgroup: producer, MMA issuers (and with REBALANCE an idle warp)
+  if constexpr (C::REBALANCE) regs_dec<C::REGS_OTHER>();
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     // Per item: Q_g once the previous item no longer needs the Q_g buffer,
@@ -364,7 +370,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // loads this thread issued, which may not have been consumed, before
         // the CTA exits
         int zero = 0;
-        WaitCtx wd{p.timeout_ns, &zero, 1u, nullptr};
+        WaitCtx wd{p.timeout_ns, &zero, 1u, false};
         for (int t = (tk > C::STAGES ? tk - C::STAGES : 0); t < tk; ++t) {
           const int st = t % C::STAGES;
           wait1(wd, bar(FB_KFULL + st), (t / C::STAGES) & 1, 11);
@@ -466,12 +472,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       // drain: everything issued above has completed before TMEM is freed
       mma_commit(bar(FB_DRAIN + g));
       int zero = 0;
-      WaitCtx wd{p.timeout_ns, &zero, 1u, nullptr};  // the drain wait ignores the abort flag
+      WaitCtx wd{p.timeout_ns, &zero, 1u, false};  // the drain wait ignores the abort flag
       wait1(wd, bar(FB_DRAIN + g), 0, 7);
     }
   }
   } else {
-    regs_inc<C::REGS_SOFTMAX>();
+    if constexpr (C::REBALANCE) regs_inc<C::REGS_SOFTMAX>();
     // ------------------------------------------------------------ softmax
     const int g = warp >> 2;                 // warpgroup: one query tile per item
     const int quarter = warp & 3;
@@ -492,10 +498,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       if (ng == 0) continue;
       float m_used = -INFINITY;  // running max, scaled log2 units
       float l = 0.f;
-      // EARLY: S_g(j+1) is computed while tile j's exponentials run, so its
-      // first 64 columns are loaded during the second half of them (`pre`:
-      // s[0..63] already hold them when tile j+1 starts)
-      bool pre = false;
       for (int j = 0; j < ng; ++j) {
         const int tgj = tg + j;
         // dropout keep bits of this row's 128 keys of tile j, computed while
@@ -510,9 +512,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
               keep[c4] |= keep_byte(static_cast<uint32_t>(j * 16 + c4 * 4 + x), qi,
                                     static_cast<uint32_t>(it.bh), p.drop) << (8 * x);
         }
-        if (!pre) {
-          wait_warp(w, bar(FB_SFULL + g), tgj & 1, 8);
-          tc_fence_after();
+        wait_warp(w, bar(FB_SFULL + g), tgj & 1, 8);
+        tc_fence_after();
+        {
           uint32_t r0[32], r1[32], r2[32], r3[32];
           tmem_ld32(scol, r0);
           tmem_ld32(scol + 32, r1);
@@ -523,16 +525,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           for (int e = 0; e < 32; ++e) {
             s[e] = __uint_as_float(r0[e]);
             s[32 + e] = __uint_as_float(r1[e]);
-            s[64 + e] = __uint_as_float(r2[e]);
-            s[96 + e] = __uint_as_float(r3[e]);
-          }
-        } else {  // the first half arrived during the previous tile
-          uint32_t r2[32], r3[32];
-          tmem_ld32(scol + 64, r2);
-          tmem_ld32(scol + 96, r3);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
             s[64 + e] = __uint_as_float(r2[e]);
             s[96 + e] = __uint_as_float(r3[e]);
           }
@@ -599,36 +591,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // only when both groups have a tile in the first item.
         const bool offset = k == 0 && j == 0 && it.n[0] > 0 && it.n[1] > 0;
         if (offset && g == 1) wait_warp(w, bar(FB_OFFSET), 0, 11);
-        if (C::EARLY && j + 1 < ng) {
-          // first half of P_g(j); then S_g(j+1), computed meanwhile, starts
-          // loading while the second half of the exponentials runs (the
-          // loaded registers count as written only at the wait)
-          fwd_exp_row<true, PLO, DROP, 0, 4>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g),
-                                             DROP ? keep : nullptr);
-          wait_warp(w, bar(FB_SFULL + g), (tgj + 1) & 1, 8);
-          tc_fence_after();
-          uint32_t r0[32], r1[32];
-          tmem_ld32(scol, r0);
-          tmem_ld32(scol + 32, r1);
-          fwd_exp_row<true, PLO, DROP, 4, 8>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g),
-                                             DROP ? keep : nullptr);
-          tmem_wait_ld_regs(r0);
-          tmem_wait_ld_regs(r1);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            s[e] = __uint_as_float(r0[e]);
-            s[32 + e] = __uint_as_float(r1[e]);
-          }
-          pre = true;
-        } else {
-          if (j == ng - 1)
-            fwd_exp_row<false, PLO, DROP>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g),
+        if (j == ng - 1)
+          fwd_exp_row<D, false, PLO, DROP>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g),
+                                           DROP ? keep : nullptr);
+        else
+          fwd_exp_row<D, true, PLO, DROP>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g),
                                           DROP ? keep : nullptr);
-          else
-            fwd_exp_row<true, PLO, DROP>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g),
-                                         DROP ? keep : nullptr);
-          pre = false;
-        }
         if (offset && g == 0) mbar_arrive(bar(FB_OFFSET));
         float sa, sb, sc2, sd;
         f2_split(sum2[0], sa, sb);

@@ -100,11 +100,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Per-CTA wait context: a time limit, a shared abort flag and the call's
-// own status words (null for a call without a workspace).  Once any thread
-// of the CTA gives up, every later wait returns at once, so all warps run
-// to the end of the kernel (where TMEM is freed and copies in flight are
-// drained) instead of hanging.
+// Per-CTA wait context: a time limit and a shared abort flag.  Once any
+// thread of the CTA gives up, every later wait returns at once, so all
+// warps run to the end of the kernel (where TMEM is freed and copies in
+// flight are drained) instead of hanging.  With `call_slot`, the 8 bytes
+// after the abort flag (shared memory) hold the address of the call's own
+// status words (or null), read only when a wait gives up: the hot loops
+// carry no extra register for it.
 //
 // The limit is counted in SM clock cycles (clock64, cheap to read) at 2.1
 // cycles per ns: at or below the 1965 MHz maximum SM clock the real limit
@@ -113,13 +115,28 @@ struct WaitCtx {
   uint64_t timeout_ns;
   volatile int* abort;  // in shared memory
   unsigned int kernel_id;
-  unsigned int* status;  // {code, where} of the call, or null
+  bool call_slot;        // the call's status address follows *abort
 };
+
+// The call's status address kept in the 8 bytes after the abort flag.
+__device__ __forceinline__ unsigned int* call_status_of(const WaitCtx& w) {
+  if (!w.call_slot) return nullptr;
+  return *reinterpret_cast<unsigned int* const volatile*>(
+      reinterpret_cast<const volatile char*>(w.abort) + 8);
+}
 
 __device__ __forceinline__ uint64_t cycles_now() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
   return t;
+}
+
+// What a wait that gives up does, out of line: one copy serves every wait
+// site.  Inlined at each of the kernels' ~30 sites, this cold code measured
+// 10 % slower on the backward (instruction-cache pressure in its hot loops).
+__device__ __noinline__ void record_timeout_of(const WaitCtx& w, unsigned int where) {
+  *w.abort = 1;
+  record_status(call_status_of(w), kStatusTimeout, where);
 }
 
 // Single-thread bounded wait.  Returns false on timeout/abort.
@@ -134,8 +151,7 @@ __device__ __forceinline__ bool wait1(const WaitCtx& w, uint32_t bar, uint32_t p
       if (mbar_try_wait(bar, parity)) return true;
     if (*w.abort) return false;
     if (cycles_now() - t0 > limit) {
-      *w.abort = 1;
-      record_status(w.status, kStatusTimeout, (w.kernel_id << 8) | bar_id);
+      record_timeout_of(w, (w.kernel_id << 8) | bar_id);
       return false;
     }
   }
@@ -161,6 +177,12 @@ __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+
+// Hardware named barrier over nthreads threads (a multiple of 32).  Used
+// only where every participating thread provably reaches it.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 
 // ---------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), 3-D tensor maps {x = d, y = t, z = b*H + h}
@@ -231,27 +253,7 @@ __device__ __forceinline__ void bulk_wait_read0() {
 __device__ __forceinline__ void bulk_wait0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
-// ... all but the most recent bulk group.
-__device__ __forceinline__ void bulk_wait1() {
-  asm volatile("cp.async.bulk.wait_group 1;" ::: "memory");
-}
 
-// Order this thread's completed async-proxy writes to global memory (bulk
-// reduce-adds) before its later generic-proxy operations.
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-// Atomic add at GPU scope with acquire-release semantics; returns the old
-// value.
-__device__ __forceinline__ unsigned int atom_add_acq_rel_gpu(unsigned int* p, unsigned int v) {
-  unsigned int old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
-               : "=r"(old)
-               : "l"(p), "r"(v)
-               : "memory");
-  return old;
-}
 
 // ---------------------------------------------------------------------------
 // Tensor memory (TMEM) and tcgen05
@@ -326,22 +328,6 @@ __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// tcgen05.wait::ld that also marks 32 registers loaded by an earlier
-// tcgen05.ld as produced here, so that the compiler cannot move any use of
-// them above the wait (the load's own asm statement is where it otherwise
-// believes they are written).
-__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.wait::ld.sync.aligned;"
-      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
-        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
-        "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]),
-        "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
-        "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]),
-        "+r"(r[31])
-      :
-      : "memory");
-}
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }

@@ -3,10 +3,12 @@
 // AddressSanitizer and UBSan, so any out-of-bounds or misaligned access of
 // the kernels fails the run.
 //
-//   decode_emu B H Tq L D Tmax layout scale in.bin out.bin
+//   decode_emu B H Tq L D Tmax layout scale in.bin out.bin [ctas_per_head]
 //     layout 0: k, v stored (B, H, Tmax, D); 1: stored (B, Tmax, H, D)
 //     in.bin:  q (B, H, Tq, D), k, v (stored layout) as bf16 bit patterns
 //     out.bin: o (B, H, Tq, D) bf16 bit patterns, then lse (B, H, Tq) fp32
+//     ctas_per_head: partial CTAs per head (default: attn_decode's own
+//     choice); fewer CTAs than chunks make each CTA walk several chunks
 // The host set-up (chunk count, workspace split, strides) follows
 // attn_decode in api.cu.
 #include "simt_emu.h"
@@ -27,19 +29,19 @@ template <int D>
 static void run(DecodeParams p, int BH) {
   const dim3 grid(BH, p.n_split);
   if (p.Tq <= 1)
-    emu::launch(grid, kDecodeWarps * 32, decode_partial_kernel<D, 1>, p);
+    emu::launch(grid, kDecodeThreads, decode_partial_kernel<D, 1>, p);
   else if (p.Tq <= 2)
-    emu::launch(grid, kDecodeWarps * 32, decode_partial_kernel<D, 2>, p);
+    emu::launch(grid, kDecodeThreads, decode_partial_kernel<D, 2>, p);
   else if (p.Tq <= 4)
-    emu::launch(grid, kDecodeWarps * 32, decode_partial_kernel<D, 4>, p);
+    emu::launch(grid, kDecodeThreads, decode_partial_kernel<D, 4>, p);
   else
-    emu::launch(grid, kDecodeWarps * 32, decode_partial_kernel<D, 8>, p);
-  emu::launch(dim3(BH * p.Tq), D, decode_combine_kernel<D>, p);
+    emu::launch(grid, kDecodeThreads, decode_partial_kernel<D, 8>, p);
+  emu::launch(dim3(BH * p.Tq), kCombineThreads, decode_combine_kernel<D>, p);
 }
 
 int main(int argc, char** argv) {
-  if (argc != 11) {
-    std::fprintf(stderr, "usage: decode_emu B H Tq L D Tmax layout scale in out\n");
+  if (argc != 11 && argc != 12) {
+    std::fprintf(stderr, "usage: decode_emu B H Tq L D Tmax layout scale in out [ctas_per_head]\n");
     return 2;
   }
   const int B = std::atoi(argv[1]), H = std::atoi(argv[2]), Tq = std::atoi(argv[3]);
@@ -56,7 +58,14 @@ int main(int argc, char** argv) {
     return 3;
   std::fclose(f);
   const int BH = B * H;
-  const int n_split = (L + kDecodeChunk - 1) / kDecodeChunk;
+  const int n_chunks = (L + decode_chunk(D) - 1) / decode_chunk(D);
+  int n_split = decode_splits_for(static_cast<long long>(B) * H, L, D);
+  int cpc = decode_chunks_per_cta(static_cast<long long>(B) * H, L, D);
+  if (argc == 12) {  // a chosen number of CTAs per head
+    const int want = std::atoi(argv[11]);
+    cpc = (n_chunks + want - 1) / want;
+    n_split = (n_chunks + cpc - 1) / cpc;
+  }
   const size_t rows = static_cast<size_t>(BH) * n_split * Tq;
   auto* part_ml = exact<float>(rows * 2);
   auto* part_o = exact<float>(rows * D);
@@ -92,6 +101,7 @@ int main(int argc, char** argv) {
   p.Tq = Tq;
   p.L = L;
   p.n_split = n_split;
+  p.chunks_per_cta = cpc;
   p.scale_log2 = scale * 1.4426950408889634f;
   switch (D) {
     case 16: run<16>(p, BH); break;

@@ -71,6 +71,12 @@ inline thread_local Cta* t_cta = nullptr;
 
 inline void __syncthreads() { emu::t_cta->cta_bar->arrive_and_wait(); }
 
+// warp barrier (full warps only, like the shuffles)
+inline void __syncwarp(unsigned mask = 0xffffffffu) {
+  if (mask != 0xffffffffu) throw std::logic_error("only full-warp __syncwarp is emulated");
+  emu::t_cta->warp_bar[threadIdx.x / 32]->arrive_and_wait();
+}
+
 inline float __shfl_xor_sync(unsigned mask, float v, int lane_mask) {
   if (mask != 0xffffffffu) throw std::logic_error("only full-warp shuffles are emulated");
   emu::Cta* c = emu::t_cta;

@@ -158,11 +158,8 @@ def test_workspace_formula(B, H, T, D):
     def r256(x):
         return (x + 255) // 256 * 256
     tpad = (T + 127) // 128 * 128
-    # the call's status words (256 bytes), the dQ accumulator, the arrival
-    # counters (one word per head, 128-row query tile and 32-row quarter),
-    # LSE2, Delta
-    want = (256 + r256(B * H * T * D * 4) + r256(B * H * (tpad // 128) * 4 * 4)
-            + 2 * r256(B * H * tpad * 4))
+    # the call's status words (256 bytes), the dQ accumulator, LSE2, Delta
+    want = 256 + r256(B * H * T * D * 4) + 2 * r256(B * H * tpad * 4)
     assert cattn.attn_bwd_workspace_bytes(B, H, T, D) == want
 
 
@@ -339,12 +336,22 @@ def test_decode_checks_arguments_before_the_device():
 
 
 def test_decode_workspace_formula():
-    # per (head, chunk of 256 keys, query row): (m, l) and D partial outputs
+    # per (head, partial CTA, query row): (m, l) and D partial outputs.  A
+    # chunk is 16 KB of K (8192 / D keys, at most 256); a head's chunks are
+    # dealt to about 592 / (B*H) CTAs (one wave), each a run of chunks.
     def r256(x):
         return (x + 255) // 256 * 256
+
+    def splits(BH, L, D):
+        chunk = min(8192 // D, 256)
+        n_chunks = (L + chunk - 1) // chunk
+        s = max(1, min(n_chunks, 592 // BH))
+        cpc = (n_chunks + s - 1) // s
+        return (n_chunks + cpc - 1) // cpc
+    assert splits(192, 1024, 64) == 3 and splits(32, 8192, 128) == 16
     for B, H, Tq, L, D in [(1, 1, 1, 1, 16), (2, 3, 4, 257, 64), (16, 12, 1, 1024, 64),
-                           (1, 2, 8, 4096, 128)]:
-        rows = B * H * ((L + 255) // 256) * Tq
+                           (1, 2, 8, 4096, 128), (2, 16, 1, 8192, 128), (64, 12, 2, 300, 32)]:
+        rows = B * H * splits(B * H, L, D) * Tq
         assert cattn.attn_decode_workspace_bytes(B, H, Tq, L, D) == r256(rows * 8) + r256(rows * D * 4)
     assert cattn.attn_decode_workspace_bytes(1, 1, 9, 16, 64) == 0
     assert cattn.attn_decode_workspace_bytes(1, 1, 2, 1, 64) == 0

@@ -48,12 +48,17 @@ def from_bits(b: np.ndarray) -> np.ndarray:
     return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-@pytest.mark.parametrize("B,H,Tq,L,D,layout", [
-    (1, 1, 1, 1, 16, 0), (2, 2, 1, 300, 64, 0), (1, 2, 3, 257, 128, 1), (1, 1, 8, 8, 32, 0),
-    (2, 1, 8, 513, 16, 1), (1, 3, 2, 256, 64, 1), (1, 1, 5, 1000, 128, 0),
-    (1, 2, 4, 37, 64, 0), (2, 1, 2, 70, 32, 1), (1, 1, 7, 520, 64, 1), (1, 1, 1, 255, 128, 1),
-    (3, 1, 6, 129, 16, 0)])
-def test_decode_kernels_on_the_host(emu_exe, tmp_path, B, H, Tq, L, D, layout):
+# (B, H, Tq, L, D, layout, partial CTAs per head or None for attn_decode's
+# own choice); a count below the number of chunks makes each CTA walk
+# several chunks (the cross-chunk merge)
+@pytest.mark.parametrize("B,H,Tq,L,D,layout,ctas", [
+    (1, 1, 1, 1, 16, 0, None), (2, 2, 1, 300, 64, 0, None), (1, 2, 3, 257, 128, 1, None),
+    (1, 1, 8, 8, 32, 0, None), (2, 1, 8, 513, 16, 1, None), (1, 3, 2, 256, 64, 1, None),
+    (1, 1, 5, 1000, 128, 0, None), (1, 2, 4, 37, 64, 0, None), (2, 1, 2, 70, 32, 1, None),
+    (1, 1, 7, 520, 64, 1, None), (1, 1, 1, 255, 128, 1, None), (3, 1, 6, 129, 16, 0, None),
+    (1, 2, 1, 1000, 64, 0, 1), (1, 1, 4, 700, 128, 1, 3), (2, 1, 8, 1100, 32, 0, 2),
+    (1, 1, 3, 600, 16, 1, 1)])
+def test_decode_kernels_on_the_host(emu_exe, tmp_path, B, H, Tq, L, D, layout, ctas):
     g = torch.Generator().manual_seed(1000 * L + D + Tq)
     Tmax = L       # a tight cache: a read past row L - 1 leaves the buffer
     q = torch.randn(B, H, Tq, D, generator=g).to(torch.bfloat16)
@@ -71,8 +76,9 @@ def test_decode_kernels_on_the_host(emu_exe, tmp_path, B, H, Tq, L, D, layout):
         for t in (q, kst, vst):
             f.write(bf16_bits(t).tobytes())
     env = dict(os.environ, ASAN_OPTIONS="detect_leaks=0")
+    extra = [] if ctas is None else [str(ctas)]
     r = subprocess.run([str(emu_exe), str(B), str(H), str(Tq), str(L), str(D), str(Tmax),
-                        str(layout), repr(scale), str(inp), str(out)],
+                        str(layout), repr(scale), str(inp), str(out)] + extra,
                        capture_output=True, text=True, timeout=600, env=env)
     assert r.returncode == 0, r.stderr[-3000:]
     raw = np.fromfile(out, dtype=np.uint8)
