@@ -581,7 +581,7 @@ __global__ void selftest_wait_kernel(uint64_t timeout_ns, unsigned int* call_sta
 
 
 size_t decode_ws_bytes(long long BH, int Tq, int L, int D) {
-  const size_t rows = static_cast<size_t>(BH) * decode_splits_for(BH, L, D) * Tq;
+  const size_t rows = static_cast<size_t>(BH) * decode_splits_for(BH, L, D, Tq) * Tq;
   return round256(rows * 2 * sizeof(float)) + round256(rows * D * sizeof(float));
 }
 
@@ -698,7 +698,7 @@ cattn_status attn_decode(const void* q, cattn_layout lq, const void* k, cattn_la
   p.q_sb = lq.b; p.q_sh = lq.h; p.q_st = lq.t;
   p.k_sb = lk.b; p.k_sh = lk.h; p.k_st = lk.t;
   p.v_sb = lv.b; p.v_sh = lv.h; p.v_st = lv.t;
-  const size_t rows = static_cast<size_t>(BH) * decode_splits_for(BH, L, D) * Tq;
+  const size_t rows = static_cast<size_t>(BH) * decode_splits_for(BH, L, D, Tq) * Tq;
   uint8_t* wb = static_cast<uint8_t*>(workspace);
   p.part_ml = reinterpret_cast<float*>(wb);
   p.part_o = reinterpret_cast<float*>(wb + round256(rows * 2 * sizeof(float)));
@@ -708,8 +708,8 @@ cattn_status attn_decode(const void* q, cattn_layout lq, const void* k, cattn_la
   p.H = H;
   p.Tq = Tq;
   p.L = L;
-  p.n_split = decode_splits_for(BH, L, D);
-  p.chunks_per_cta = decode_chunks_per_cta(BH, L, D);
+  p.n_split = decode_splits_for(BH, L, D, Tq);
+  p.chunks_per_cta = decode_chunks_per_cta(BH, L, D, Tq);
   p.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (D) {

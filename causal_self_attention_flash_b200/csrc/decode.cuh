@@ -48,20 +48,24 @@ constexpr int kDecodeThreads = 256;  // threads per partial CTA
 // Keys per chunk: 16 KB of K (and of V), at most 256 keys.
 __host__ __device__ constexpr int decode_chunk(int D) { return 8192 / D < 256 ? 8192 / D : 256; }
 
-// Partial CTAs per head: about kDecodeCtasTarget CTAs in all (one wave at
-// 4 per SM on a 148-SM B200), at most one per chunk.
-constexpr int kDecodeCtasTarget = 592;
-__host__ __device__ constexpr int decode_splits_for(long long BH, int L, int D) {
+// Resident partial CTAs per SM: 4 for up to 2 query rows (the launch bounds
+// then hold a thread to 64 registers, and the shared memory fits 4), 3 for
+// more rows (left unbounded: their accumulators would spill at 64).
+__host__ __device__ constexpr int decode_ctas_per_sm(int Tq) { return Tq <= 2 ? 4 : 3; }
+
+// Partial CTAs per head: one wave of CTAs on a 148-SM B200, at most one per
+// chunk.
+__host__ __device__ constexpr int decode_splits_for(long long BH, int L, int D, int Tq) {
   const int n_chunks = (L + decode_chunk(D) - 1) / decode_chunk(D);
-  const long long want = BH > 0 ? kDecodeCtasTarget / BH : 1;
+  const long long want = BH > 0 ? 148LL * decode_ctas_per_sm(Tq) / BH : 1;
   const int s = want < 1 ? 1 : (want > n_chunks ? n_chunks : static_cast<int>(want));
   // chunks per CTA, then the CTAs that actually have chunks
   const int cpc = (n_chunks + s - 1) / s;
   return (n_chunks + cpc - 1) / cpc;
 }
-__host__ __device__ constexpr int decode_chunks_per_cta(long long BH, int L, int D) {
+__host__ __device__ constexpr int decode_chunks_per_cta(long long BH, int L, int D, int Tq) {
   const int n_chunks = (L + decode_chunk(D) - 1) / decode_chunk(D);
-  const int s = decode_splits_for(BH, L, D);
+  const int s = decode_splits_for(BH, L, D, Tq);
   return (n_chunks + s - 1) / s;
 }
 
@@ -117,7 +121,8 @@ __device__ __forceinline__ int dec_swz(int row, int c) {
 // loads are already in flight into registers; a running (m, l, o) per row
 // merges the chunks as the online softmax does.
 template <int D, int TQ>
-__global__ void __launch_bounds__(kDecodeThreads) decode_partial_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kDecodeThreads, TQ <= 2 ? 4 : 1)
+    decode_partial_kernel(const DecodeParams p) {
   using C = DecodeCfg<D>;
   constexpr int VPR = C::VPR, CH = C::CHUNK, NT = kDecodeThreads;
   __shared__ uint4 sK[C::PIECES];  // uint4: 16-byte aligned by its type

@@ -490,6 +490,21 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const float sl2 = p.scale_log2;
     int tg = 0;
     float s[128];
+    // Once per CTA, group 1 starts only after group 0's first exponential
+    // phase: the two groups then stay out of step, so their exponential
+    // phases overlap less on the ex2 unit.  Exactly one phase of the
+    // FB_OFFSET barrier per CTA: group 0's 128 threads arrive once (after
+    // the exponentials of the first tile of the first item), group 1 waits
+    // once, here (bounded, like every wait), and both take it only when both
+    // groups have a tile in the first item.  Waiting before the loop keeps
+    // the wait out of the loop body.
+    {
+      const int u0 = fwd_item(0, b, G, n_items);
+      if (u0 >= 0 && g == 1) {
+        const FwdItem it0 = fwd_item_info(u0, 0, p.BH, n_pairs, p.n_qtiles);
+        if (it0.n[0] > 0 && it0.n[1] > 0) wait_warp(w, bar(FB_OFFSET), 0, 11);
+      }
+    }
     for (int k = 0;; ++k) {
       const int u = fwd_item(k, b, G, n_items);
       if (u < 0) break;
@@ -583,14 +598,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const uint64_t sl2x2 = f2(sl2, sl2);
         const uint64_t negm2 = f2(-m_used, -m_used);
         uint64_t sum2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
-        // Once per CTA, group 1's first exponential phase waits for group
-        // 0's: the two groups then stay out of step, so their exponential
-        // phases overlap less on the ex2 unit.  Exactly one phase of the
-        // FB_OFFSET barrier per CTA: group 0's 128 threads arrive once,
-        // group 1 waits once (bounded, like every wait), and both take it
-        // only when both groups have a tile in the first item.
+        // Group 0's side of the one-time offset (see before the item loop).
         const bool offset = k == 0 && j == 0 && it.n[0] > 0 && it.n[1] > 0;
-        if (offset && g == 1) wait_warp(w, bar(FB_OFFSET), 0, 11);
         if (j == ng - 1)
           fwd_exp_row<D, false, PLO, DROP>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g),
                                            DROP ? keep : nullptr);

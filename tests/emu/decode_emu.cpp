@@ -59,8 +59,8 @@ int main(int argc, char** argv) {
   std::fclose(f);
   const int BH = B * H;
   const int n_chunks = (L + decode_chunk(D) - 1) / decode_chunk(D);
-  int n_split = decode_splits_for(static_cast<long long>(B) * H, L, D);
-  int cpc = decode_chunks_per_cta(static_cast<long long>(B) * H, L, D);
+  int n_split = decode_splits_for(static_cast<long long>(B) * H, L, D, Tq);
+  int cpc = decode_chunks_per_cta(static_cast<long long>(B) * H, L, D, Tq);
   if (argc == 12) {  // a chosen number of CTAs per head
     const int want = std::atoi(argv[11]);
     cpc = (n_chunks + want - 1) / want;

@@ -338,20 +338,24 @@ def test_decode_checks_arguments_before_the_device():
 def test_decode_workspace_formula():
     # per (head, partial CTA, query row): (m, l) and D partial outputs.  A
     # chunk is 16 KB of K (8192 / D keys, at most 256); a head's chunks are
-    # dealt to about 592 / (B*H) CTAs (one wave), each a run of chunks.
+    # dealt to about 148 * (4, or 3 above 2 rows) / (B*H) CTAs (one wave),
+    # each a run of chunks.
     def r256(x):
         return (x + 255) // 256 * 256
 
-    def splits(BH, L, D):
+    def splits(BH, L, D, Tq):
         chunk = min(8192 // D, 256)
         n_chunks = (L + chunk - 1) // chunk
-        s = max(1, min(n_chunks, 592 // BH))
+        per_sm = 4 if Tq <= 2 else 3
+        s = max(1, min(n_chunks, 148 * per_sm // BH))
         cpc = (n_chunks + s - 1) // s
         return (n_chunks + cpc - 1) // cpc
-    assert splits(192, 1024, 64) == 3 and splits(32, 8192, 128) == 16
+    assert splits(192, 1024, 64, 1) == 3 and splits(32, 8192, 128, 1) == 16
+    assert splits(192, 1024, 64, 4) == 2
     for B, H, Tq, L, D in [(1, 1, 1, 1, 16), (2, 3, 4, 257, 64), (16, 12, 1, 1024, 64),
-                           (1, 2, 8, 4096, 128), (2, 16, 1, 8192, 128), (64, 12, 2, 300, 32)]:
-        rows = B * H * splits(B * H, L, D) * Tq
+                           (1, 2, 8, 4096, 128), (2, 16, 1, 8192, 128), (64, 12, 2, 300, 32),
+                           (16, 12, 8, 1024, 64)]:
+        rows = B * H * splits(B * H, L, D, Tq) * Tq
         assert cattn.attn_decode_workspace_bytes(B, H, Tq, L, D) == r256(rows * 8) + r256(rows * D * 4)
     assert cattn.attn_decode_workspace_bytes(1, 1, 9, 16, 64) == 0
     assert cattn.attn_decode_workspace_bytes(1, 1, 2, 1, 64) == 0
