@@ -390,11 +390,11 @@ def measure_decode(w, sets, stream, cattn, n):
     """attn_decode of the Tq newest positions (Tq = 1, 4, 8) against the
     whole sequence's K and V as the cache, rotating over the input sets
     (their K, V together exceed L2).  The calls are captured in a CUDA graph
-    and replayed, so the time is the GPU's (two kernels per call, no host
+    and replayed, so the time is the GPU's (one kernel per call, no host
     launch gaps), as a serving loop would run it."""
     B, H, T, D = w.B, w.H, w.T, w.D
     peaks, src = load_peaks()
-    out = {"peak_source": src, "kernels": "decode_partial_kernel + decode_combine_kernel",
+    out = {"peak_source": src, "kernels": "decode_kernel (one launch per call)",
            "timing": "CUDA graph of %d calls, replayed; device time per call" % n}
     for tq in (1, 4, 8):
         if tq > T:

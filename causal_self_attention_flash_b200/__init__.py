@@ -417,10 +417,15 @@ def attn_decode(q, k, v, L, scale=None, o=None, lse=None, workspace=None, stream
         o = torch.empty((B, H, Tq, D), dtype=torch.bfloat16, device=q.device)
     lo = _layout(o, torch.bfloat16, "o", (B, H, Tq, D), q.device)
     lse = _want(lse, q, torch.float32, (B, H, Tq))
-    workspace = _workspace(workspace, q, attn_decode_workspace_bytes(B, H, Tq, L, D))
+    need = attn_decode_workspace_bytes(B, H, Tq, L, D)
+    if workspace is None and need == 0:
+        ws_ptr, ws_n = None, 0
+    else:
+        workspace = _workspace(workspace, q, need)
+        ws_ptr, ws_n = workspace.data_ptr(), _nbytes(workspace)
     st = LIB.attn_decode(q.data_ptr(), lq, k.data_ptr(), lk, v.data_ptr(), lv, float(scale),
                          B, H, Tq, int(L), D, o.data_ptr(), lo, lse.data_ptr(),
-                         workspace.data_ptr(), _nbytes(workspace), _stream(stream))
+                         ws_ptr, ws_n, _stream(stream))
     _check("attn_decode", st)
     return o, lse
 

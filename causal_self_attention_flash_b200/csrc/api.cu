@@ -42,7 +42,7 @@ cattn_status cuda_fail(int code) {
   return CATTN_ERR_CUDA;
 }
 int g_dev_ok[kMaxDevices];           // 0 unknown, 1 sm_100, -1 other
-uint64_t g_attr_done[kMaxDevices];   // bit per kernel instance
+uint64_t g_attr_done[kMaxDevices][2];  // bit per kernel instance (128)
 int g_sm_count[kMaxDevices];         // multiprocessors (persistent grids)
 
 cattn_status init_encode() {
@@ -96,7 +96,7 @@ cattn_status check_device(int* dev_out) {
 // chose another count is refused (CATTN_ERR_UNSUPPORTED) instead of run.
 template <typename K>
 cattn_status ensure_smem(int dev, unsigned bit, K kernel, int bytes, int launch_regs = 0) {
-  if (g_attr_done[dev] & (1ull << bit)) return CATTN_OK;
+  if (g_attr_done[dev][bit >> 6] & (1ull << (bit & 63))) return CATTN_OK;
   if (launch_regs > 0) {
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return cuda_fail(cudaGetLastError());
@@ -107,7 +107,7 @@ cattn_status ensure_smem(int dev, unsigned bit, K kernel, int bytes, int launch_
     return cuda_fail(cudaGetLastError());
   }
   std::lock_guard<std::mutex> lk(g_mu);
-  g_attr_done[dev] |= 1ull << bit;
+  g_attr_done[dev][bit >> 6] |= 1ull << (bit & 63);
   return CATTN_OK;
 }
 
@@ -577,31 +577,29 @@ __global__ void selftest_wait_kernel(uint64_t timeout_ns, unsigned int* call_sta
 
 // ------------------------------------------------------------------ decode
 
-// Key chunks per head, and the workspace of their partial results.
-
-
-size_t decode_ws_bytes(long long BH, int Tq, int L, int D) {
-  const size_t rows = static_cast<size_t>(BH) * decode_splits_for(BH, L, D, Tq) * Tq;
-  return round256(rows * 2 * sizeof(float)) + round256(rows * D * sizeof(float));
-}
+// Resident decode CTAs on the device: its SMs x kDecodeCtasPerSm.
+int decode_slots(int dev) { return g_sm_count[dev] * kDecodeCtasPerSm; }
 
 template <int D>
-cattn_status decode_impl(const DecodeParams& p, long long BH, cudaStream_t s) {
-  clear_stale_error();
-  dim3 grid(static_cast<unsigned>(BH), static_cast<unsigned>(p.n_split));
-  LaunchTimer t(K_DECODE, s);  // both kernels, as one entry
-  // query rows per thread: Tq rounded up to 1, 2, 4 or 8
-  if (p.Tq <= 1)
-    decode_partial_kernel<D, 1><<<grid, kDecodeThreads, 0, s>>>(p);
-  else if (p.Tq <= 2)
-    decode_partial_kernel<D, 2><<<grid, kDecodeThreads, 0, s>>>(p);
-  else if (p.Tq <= 4)
-    decode_partial_kernel<D, 4><<<grid, kDecodeThreads, 0, s>>>(p);
-  else
-    decode_partial_kernel<D, 8><<<grid, kDecodeThreads, 0, s>>>(p);
-  cattn_status st = launch_status();
+cattn_status decode_impl(const DecodeParams& p, long long BH, int dev, cudaStream_t s) {
+  cattn_status st = ensure_smem(dev, 64 + d_index(D), decode_kernel<D>, kDecodeSmemBytes);
   if (st != CATTN_OK) return st;
-  decode_combine_kernel<D><<<static_cast<unsigned>(BH * p.Tq), kCombineThreads, 0, s>>>(p);
+  clear_stale_error();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(BH * p.n_split));
+  cfg.blockDim = dim3(kDecodeThreads);
+  cfg.dynamicSmemBytes = kDecodeSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(p.n_split);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.n_split > 1 ? 1 : 0;
+  LaunchTimer t(K_DECODE, s);
+  if (cudaLaunchKernelEx(&cfg, decode_kernel<D>, p) != cudaSuccess)
+    return cuda_fail(cudaGetLastError());
   return launch_status();
 }
 
@@ -664,9 +662,9 @@ cattn_status attn_fwd(const void* q, const void* k, const void* v, float scale, 
 }
 
 size_t attn_decode_workspace_bytes(int B, int H, int Tq, int L, int D) {
-  if (check_shape(B, H, L, D) != CATTN_OK || Tq < 1 || Tq > kDecodeMaxTq || L < Tq) return 0;
-  if (empty_shape(B, H, L)) return 0;
-  return decode_ws_bytes(static_cast<long long>(B) * H, Tq, L, D);
+  // the CTAs of a head merge their partial results on chip
+  (void)B, (void)H, (void)Tq, (void)L, (void)D;
+  return 0;
 }
 
 cattn_status attn_decode(const void* q, cattn_layout lq, const void* k, cattn_layout lk,
@@ -679,18 +677,19 @@ cattn_status attn_decode(const void* q, cattn_layout lq, const void* k, cattn_la
   if (Tq > kDecodeMaxTq) return CATTN_ERR_UNSUPPORTED;
   if (B == 0 || H == 0) return CATTN_OK;
   if (Tq < 1 || L < Tq) return CATTN_ERR_INVALID_ARG;
-  if (!q || !k || !v || !o || !lse || !workspace) return CATTN_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !lse) return CATTN_ERR_INVALID_ARG;
+  (void)workspace, (void)workspace_bytes;  // none needed
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
-      !aligned(lse, 4) || !aligned(workspace, 256))
+      !aligned(lse, 4))
     return CATTN_ERR_INVALID_ARG;
   if (!layout_ok(lq) || !layout_ok(lk) || !layout_ok(lv) || !layout_ok(lo))
     return CATTN_ERR_INVALID_ARG;
   if (!output_layout_ok(lo, B, H, Tq, D)) return CATTN_ERR_INVALID_ARG;
   const long long BH = static_cast<long long>(B) * H;
-  if (BH * Tq > 0x7fffffffLL) return CATTN_ERR_INVALID_ARG;
-  if (workspace_bytes < decode_ws_bytes(BH, Tq, L, D)) return CATTN_ERR_INVALID_ARG;
   int dev;
   if ((st = check_device(&dev)) != CATTN_OK) return st;
+  const int n_split = decode_splits_for(BH, L, D, decode_slots(dev));
+  if (BH * n_split > 0x7fffffffLL) return CATTN_ERR_INVALID_ARG;
   DecodeParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k = static_cast<const __nv_bfloat16*>(k);
@@ -698,25 +697,21 @@ cattn_status attn_decode(const void* q, cattn_layout lq, const void* k, cattn_la
   p.q_sb = lq.b; p.q_sh = lq.h; p.q_st = lq.t;
   p.k_sb = lk.b; p.k_sh = lk.h; p.k_st = lk.t;
   p.v_sb = lv.b; p.v_sh = lv.h; p.v_st = lv.t;
-  const size_t rows = static_cast<size_t>(BH) * decode_splits_for(BH, L, D, Tq) * Tq;
-  uint8_t* wb = static_cast<uint8_t*>(workspace);
-  p.part_ml = reinterpret_cast<float*>(wb);
-  p.part_o = reinterpret_cast<float*>(wb + round256(rows * 2 * sizeof(float)));
   p.o = static_cast<__nv_bfloat16*>(o);
   p.o_sb = lo.b; p.o_sh = lo.h; p.o_st = lo.t;
   p.lse = lse;
   p.H = H;
   p.Tq = Tq;
   p.L = L;
-  p.n_split = decode_splits_for(BH, L, D, Tq);
-  p.chunks_per_cta = decode_chunks_per_cta(BH, L, D, Tq);
+  p.n_split = n_split;
+  p.chunks_per_cta = decode_chunks_per_cta(BH, L, D, decode_slots(dev));
   p.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (D) {
-    case 16: return decode_impl<16>(p, BH, s);
-    case 32: return decode_impl<32>(p, BH, s);
-    case 64: return decode_impl<64>(p, BH, s);
-    case 128: return decode_impl<128>(p, BH, s);
+    case 16: return decode_impl<16>(p, BH, dev, s);
+    case 32: return decode_impl<32>(p, BH, dev, s);
+    case 64: return decode_impl<64>(p, BH, dev, s);
+    case 128: return decode_impl<128>(p, BH, dev, s);
   }
   return CATTN_ERR_UNSUPPORTED;
 }

@@ -11,61 +11,70 @@
 // forward, for a few rows.
 //
 // There is almost no arithmetic per byte (2 * Tq flops per key element), so
-// the work is bound by reading K and V once from HBM.  The keys of each head
-// are split into chunks of DecodeCfg<D>::CHUNK (16 KB of K and 16 KB of V),
-// one CTA per (head, chunk), so even a batch of one sequence spreads over
-// the SMs ("split-K"):
-//   decode_partial_kernel<D, TQ>  per CTA (256 threads), over a run of
-//   chunks of one head:
-//     1. every thread's 16-byte loads of a chunk's K and V rows go out at
-//        once (the whole chunk in flight, while the previous chunk is
-//        computed), then into shared memory, 16-byte pieces swizzled by row
-//        so that the reads below are free of bank conflicts;
-//     2. scores s[r][key] = q_r . k_key in log2 units (scale * log2(e)
-//        folded into q), one (key, query row) pair per thread, -inf where
-//        the key is not visible to the row or past the cache;
-//     3. one warp per query row: the running maximum m, the weights
-//        2^(s - m) and the running sum l (warp shuffles);
-//     4. o[r][d] = 2^(m_old - m) o[r][d] + sum_key w[r][key] v[key][d],
-//        threads over (part of the keys, r, d);
-//     5. after its last chunk, the CTA's (m, l, o) to the workspace (the
-//        key parts summed through shared memory).
-//   decode_combine_kernel  per (head, query): merges the chunks' (m, l, o)
-//                          (o = sum 2^(m_c - M) o_c / sum 2^(m_c - M) l_c)
-//                          and writes O (bf16) and LSE (natural log).
-// Scores are kept in log2 units, so the exponentials are exp2; exp2f keeps
-// them accurate, as the kernel is not bound by arithmetic.
+// the work is bound by reading K and V once from HBM, and the design is
+// about keeping enough of that read in flight on every SM:
+//   decode_kernel<D>, one launch:
+//     - a head's keys are cut into chunks of decode_chunk(D) keys (4 KB of
+//       K and 4 KB of V) and dealt to a thread-block cluster of n_split CTAs
+//       (a contiguous run of chunks each), so that even a few heads spread
+//       over the SMs ("split-K");
+//     - inside a CTA, chunk j of the run goes to warp j % kDecodeWarps, and
+//       every warp streams its own chunks through a private ring of
+//       kDecodeStages shared-memory slots with cp.async (16-byte pieces,
+//       swizzled by row so that the ldmatrix reads below are free of bank
+//       conflicts): kDecodeStages chunks per warp are always on their way;
+//     - per chunk, the warp computes s = q k^T on the tensor cores
+//       (mma.sync m16n8k16: the query rows, zero-padded to 16, are the A
+//       operand, held in registers for the whole run; K by ldmatrix), the
+//       running maximum m, the weights p = 2^(s scale log2(e) - m) and
+//       running sum l in registers (online softmax), then o += p v (p as
+//       bf16 A fragments straight from the score accumulators, V by
+//       transposed ldmatrix);
+//     - at the end the warps' (m, l, o) are merged through shared memory,
+//       then the cluster's CTAs' through distributed shared memory
+//       (o = sum 2^(m_c - M) o_c / sum 2^(m_c - M) l_c), and O (bf16) and
+//       LSE (natural log) are written.  No workspace and no second kernel.
+// Exponentials are exp2f: the kernel is not bound by arithmetic.
 #pragma once
 
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#ifndef CATTN_HOST_EMULATION
+#include "decode_ptx.cuh"
+#endif
+
 namespace cattn {
 
-constexpr int kDecodeMaxTq = 8;      // query rows per call
-constexpr int kDecodeThreads = 256;  // threads per partial CTA
+constexpr int kDecodeMaxTq = 8;                        // query rows per call
+constexpr int kDecodeWarps = 4;                        // warps per CTA
+constexpr int kDecodeThreads = 32 * kDecodeWarps;
+constexpr int kDecodeStages = 3;                       // chunks in flight per warp
+constexpr int kDecodeChunkBytes = 8192;                // K and V of one chunk
+constexpr int kDecodeSmemBytes = kDecodeWarps * kDecodeStages * kDecodeChunkBytes;
+constexpr int kDecodeCtasPerSm = 2;                    // 2 x 96 KB of shared memory
+constexpr int kDecodeMaxCluster = 8;                   // portable cluster size
 
-// Keys per chunk: 16 KB of K (and of V), at most 256 keys.
-__host__ __device__ constexpr int decode_chunk(int D) { return 8192 / D < 256 ? 8192 / D : 256; }
+// Keys per chunk: 4 KB of K, 4 KB of V (128, 64, 32, 16 keys for D = 16 ..
+// 128).
+__host__ __device__ constexpr int decode_chunk(int D) { return kDecodeChunkBytes / 4 / D; }
 
-// Resident partial CTAs per SM: 4 for up to 2 query rows (the launch bounds
-// then hold a thread to 64 registers, and the shared memory fits 4), 3 for
-// more rows (left unbounded: their accumulators would spill at 64).
-__host__ __device__ constexpr int decode_ctas_per_sm(int Tq) { return Tq <= 2 ? 4 : 3; }
-
-// Partial CTAs per head: one wave of CTAs on a 148-SM B200, at most one per
-// chunk.
-__host__ __device__ constexpr int decode_splits_for(long long BH, int L, int D, int Tq) {
+// CTAs per head (the cluster size): enough to fill `slots` resident CTAs
+// (SMs x kDecodeCtasPerSm), at most kDecodeMaxCluster and at most one per
+// chunk; then the number of CTAs that a run of equal length leaves work
+// for.
+__host__ __device__ constexpr int decode_splits_for(long long BH, int L, int D, int slots) {
   const int n_chunks = (L + decode_chunk(D) - 1) / decode_chunk(D);
-  const long long want = BH > 0 ? 148LL * decode_ctas_per_sm(Tq) / BH : 1;
-  const int s = want < 1 ? 1 : (want > n_chunks ? n_chunks : static_cast<int>(want));
-  // chunks per CTA, then the CTAs that actually have chunks
-  const int cpc = (n_chunks + s - 1) / s;
+  long long want = BH > 0 ? slots / BH : 1;
+  if (want > kDecodeMaxCluster) want = kDecodeMaxCluster;
+  if (want > n_chunks) want = n_chunks;
+  if (want < 1) want = 1;
+  const int cpc = (n_chunks + static_cast<int>(want) - 1) / static_cast<int>(want);
   return (n_chunks + cpc - 1) / cpc;
 }
-__host__ __device__ constexpr int decode_chunks_per_cta(long long BH, int L, int D, int Tq) {
+__host__ __device__ constexpr int decode_chunks_per_cta(long long BH, int L, int D, int slots) {
   const int n_chunks = (L + decode_chunk(D) - 1) / decode_chunk(D);
-  const int s = decode_splits_for(BH, L, D, Tq);
+  const int s = decode_splits_for(BH, L, D, slots);
   return (n_chunks + s - 1) / s;
 }
 
@@ -74,267 +83,251 @@ struct DecodeParams {
   const __nv_bfloat16* k;  // (B, H, >= L, D)
   const __nv_bfloat16* v;
   long long q_sb, q_sh, q_st, k_sb, k_sh, k_st, v_sb, v_sh, v_st;
-  float* part_ml;          // [BH][n_split][Tq][2]: m (log2 units), l
-  float* part_o;           // [BH][n_split][Tq][D]
   __nv_bfloat16* o;        // (B, H, Tq, D), element strides o_sb, o_sh, o_st
   long long o_sb, o_sh, o_st;
   float* lse;              // (B, H, Tq) contiguous, natural log
-  int H, Tq, L, n_split;
-  int chunks_per_cta;      // chunks of CHUNK keys each partial CTA takes
+  int H, Tq, L;
+  int n_split;             // CTAs per head = cluster size
+  int chunks_per_cta;      // chunks of a CTA's run (the last run shorter)
   float scale_log2;        // scale * log2(e)
 };
 
+// Byte offset of 16-byte piece `pc` of row `row` in a chunk tile of D-wide
+// rows.  The 8 rows an ldmatrix reads (consecutive rows, same piece) land
+// in 8 different 16-byte bank groups: the piece index is XORed with the
+// row's position among the rows that share a 128-byte line span.
 template <int D>
-struct DecodeCfg {
-  static constexpr int CHUNK = decode_chunk(D);        // keys per CTA
-  static constexpr int VPR = D / 8;                    // 16-byte pieces per row
-  static constexpr int PIECES = CHUNK * VPR;           // per tensor per chunk
-  static constexpr int LOADS = PIECES / kDecodeThreads;  // per thread per tensor
-  static constexpr int TPK = kDecodeThreads / CHUNK;   // threads per key (scores)
-  static_assert(LOADS * kDecodeThreads == PIECES && TPK * CHUNK == kDecodeThreads, "chunk");
-};
-
-// 8 bf16 (one 16-byte piece) -> 8 floats
-__device__ __forceinline__ void unpack8(const uint4& t, float (&x)[8]) {
-  const unsigned w[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
-    x[2 * i] = f.x;
-    x[2 * i + 1] = f.y;
-  }
+__host__ __device__ constexpr int dec_swz(int row, int pc) {
+  constexpr int P = D / 8;                  // pieces per row
+  constexpr int RPL = P >= 8 ? 1 : 8 / P;   // rows per 128 bytes
+  constexpr int MASK = (P >= 8 ? 8 : P) - 1;
+  return (row * P + (pc ^ ((row / RPL) & MASK))) * 16;
 }
 
-// Shared-memory position of 16-byte piece c of chunk row `row`: pieces are
-// rotated by the row so that consecutive rows' piece c fall in different
-// banks (a thread per row reads its row piece by piece).
-template <int VPR>
-__device__ __forceinline__ int dec_swz(int row, int c) {
-  return row * VPR + (c ^ (row % VPR));
-}
+// Grid: BH * n_split CTAs of kDecodeThreads, clusters of n_split along x
+// (CTA x: head x / n_split, cluster rank x % n_split), kDecodeSmemBytes of
+// dynamic shared memory.
+template <int D>
+__global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
+    decode_kernel(const DecodeParams p) {
+  constexpr int CK = decode_chunk(D);  // keys per chunk
+  constexpr int P = D / 8;             // 16-byte pieces per row
+  constexpr int NS = CK / 8;           // score n-tiles per chunk
+  constexpr int KS = D / 16;           // k-steps of q k^T
+  constexpr int NO = D / 8;            // output n-tiles
+  constexpr int TILE = CK * D * 2;     // bytes of K (of V) per chunk
+  constexpr int NW = kDecodeWarps;
+  static_assert(2 * TILE == kDecodeChunkBytes && TILE / 16 % 32 == 0, "chunk");
+  static_assert(NS % 2 == 0 && D % 16 == 0, "tiles");
 
-// TQ: query rows the CTA is compiled for (Tq rounded up to 1, 2, 4 or 8;
-// rows at or past Tq compute nothing useful and are not written).
-// CTA (bh, split) takes the chunks split*cpc .. split*cpc + cpc - 1 of head
-// bh (cpc = p.chunks_per_cta, the last CTA fewer), so that the grid is one
-// wave.  While it computes a chunk from shared memory, the next chunk's
-// loads are already in flight into registers; a running (m, l, o) per row
-// merges the chunks as the online softmax does.
-template <int D, int TQ>
-__global__ void __launch_bounds__(kDecodeThreads, TQ <= 2 ? 4 : 1)
-    decode_partial_kernel(const DecodeParams p) {
-  using C = DecodeCfg<D>;
-  constexpr int VPR = C::VPR, CH = C::CHUNK, NT = kDecodeThreads;
-  __shared__ uint4 sK[C::PIECES];  // uint4: 16-byte aligned by its type
-  __shared__ uint4 sV[C::PIECES];
-  __shared__ float sQ[TQ][D];         // q rows * scale * log2(e)
-  __shared__ float sW[TQ][CH];        // scores, then weights 2^(s - M)
-  __shared__ float sML[TQ][2];        // running M and l per row
-  __shared__ float sAlpha[TQ];        // this chunk's rescale of the running o
-  constexpr int OUTS = TQ * D;        // outputs per CTA
-  constexpr int PARTS = OUTS >= NT ? 1 : NT / OUTS;  // key parts of the sum
-  constexpr int OPT = OUTS >= NT ? OUTS / NT : 1;    // outputs per thread
-  __shared__ float sO[PARTS][OUTS];
-
+  uint8_t* smem = dec_dynamic_smem();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int bh = blockIdx.x, split = blockIdx.y;
-  const int b = bh / p.H, h = bh - b * p.H;
-  const int Tq = p.Tq;
-  const int pos0 = p.L - Tq;          // position of query row 0
-  const int n_chunks = (p.L + CH - 1) / CH;
+  const int g = lane >> 2, t4 = lane & 3;  // fragment row, column pair
+  const int split = static_cast<int>(blockIdx.x % static_cast<unsigned>(p.n_split));
+  const long long bh = blockIdx.x / static_cast<unsigned>(p.n_split);
+  const long long b = bh / p.H, h = bh - b * p.H;
+  const int Tq = p.Tq, L = p.L, pos0 = L - Tq;  // position of query row 0
+  const int n_chunks = (L + CK - 1) / CK;
   const int c_begin = split * p.chunks_per_cta;
   const int c_end = min(n_chunks, c_begin + p.chunks_per_cta);
   const __nv_bfloat16* kb = p.k + b * p.k_sb + h * p.k_sh;
   const __nv_bfloat16* vb = p.v + b * p.v_sb + h * p.v_sh;
 
-  // loads of chunk c into registers (zero past the cache)
-  uint4 kr[C::LOADS], vr[C::LOADS];
-  auto load_chunk = [&](int c) {
-    const int k0 = c * CH, n = min(CH, p.L - k0);
+  // this warp's chunks: first, first + NW, ... below c_end
+  const int first = c_begin + warp;
+  const int n_my = first < c_end ? (c_end - first + NW - 1) / NW : 0;
+  uint8_t* ring = smem + warp * (kDecodeStages * kDecodeChunkBytes);
+
+  // chunk i of this warp into ring slot i % kDecodeStages; keys past the
+  // cache are zero-filled (and masked below)
+  auto issue = [&](int i) {
+    const int k0 = (first + NW * i) * CK;
+    uint8_t* sk = ring + (i % kDecodeStages) * kDecodeChunkBytes;
+    uint8_t* sv = sk + TILE;
 #pragma unroll
-    for (int u = 0; u < C::LOADS; ++u) {
-      const int i = tid + NT * u, row = i / VPR, pc = i - (i / VPR) * VPR;
-      kr[u] = vr[u] = uint4{0u, 0u, 0u, 0u};
-      if (row < n) {
-        const long long key = k0 + row;
-        kr[u] = *reinterpret_cast<const uint4*>(kb + key * p.k_st + pc * 8);
-        vr[u] = *reinterpret_cast<const uint4*>(vb + key * p.v_st + pc * 8);
-      }
+    for (int u = 0; u < TILE / 16 / 32; ++u) {
+      const int piece = lane + 32 * u, row = piece / P, pc = piece - (piece / P) * P;
+      const int key = k0 + row;
+      const bool ok = key < L;
+      const long long kr = ok ? key : 0;
+      dec_cp_async16(sk + dec_swz<D>(row, pc), kb + kr * p.k_st + pc * 8, ok);
+      dec_cp_async16(sv + dec_swz<D>(row, pc), vb + kr * p.v_st + pc * 8, ok);
     }
   };
-  load_chunk(c_begin);
-  for (int i = tid; i < TQ * D; i += NT) {
-    const int r = i / D, d = i - (i / D) * D;
-    float x = 0.f;
-    if (r < Tq) x = __bfloat162float(p.q[b * p.q_sb + h * p.q_sh + r * p.q_st + d]) * p.scale_log2;
-    sQ[r][d] = x;
-  }
-  if (tid < TQ) {
-    sML[tid][0] = -INFINITY;
-    sML[tid][1] = 0.f;
-  }
-  float o_run[OPT];
+  // one commit group per ring slot, empty when the warp has fewer chunks,
+  // so that "all but the newest kDecodeStages - 1 groups done" is always
+  // "chunk i has landed"
 #pragma unroll
-  for (int j = 0; j < OPT; ++j) o_run[j] = 0.f;
-
-  for (int c = c_begin; c < c_end; ++c) {
-    const int k0 = c * CH, n = min(CH, p.L - k0);
-    // 1. the chunk (loaded into registers) into shared memory; then the
-    //    next chunk's loads go out while this one is computed
-#pragma unroll
-    for (int u = 0; u < C::LOADS; ++u) {
-      const int i = tid + NT * u, row = i / VPR, pc = i - (i / VPR) * VPR;
-      sK[dec_swz<VPR>(row, pc)] = kr[u];
-      sV[dec_swz<VPR>(row, pc)] = vr[u];
-    }
-    __syncthreads();
-    if (c + 1 < c_end) load_chunk(c + 1);
-
-    // 2. scores: thread -> key tid % CH, rows tid / CH, + TPK, ...
-    {
-      const int key = tid % CH;
-      for (int r = tid / CH; r < TQ; r += C::TPK) {
-        float d0 = 0.f, d1 = 0.f;
-#pragma unroll
-        for (int pc = 0; pc < VPR; ++pc) {
-          float x[8];
-          unpack8(sK[dec_swz<VPR>(key, pc)], x);
-#pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-            d0 = fmaf(sQ[r][pc * 8 + e], x[e], d0);
-            d1 = fmaf(sQ[r][pc * 8 + e + 1], x[e + 1], d1);
-          }
-        }
-        const bool visible = key < n && k0 + key <= pos0 + r;
-        sW[r][key] = visible ? d0 + d1 : -INFINITY;
-      }
-    }
-    __syncthreads();
-
-    // 3. one warp per query row: the new running maximum M, the weights
-    //    2^(s - M), the running sum, and alpha = 2^(M_old - M) for o
-    for (int r = warp; r < TQ; r += NT / 32) {
-      float m = -INFINITY;
-      for (int j = lane; j < CH; j += 32) m = fmaxf(m, sW[r][j]);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      const float m_old = sML[r][0];
-      const float M = fmaxf(m_old, m);
-      // no key visible to the row yet: everything stays zero
-      const float mu = M == -INFINITY ? 0.f : M;
-      float l = 0.f;
-      for (int j = lane; j < CH; j += 32) {
-        const float w = exp2f(sW[r][j] - mu);  // 0 for a masked key
-        sW[r][j] = w;
-        l += w;
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-      __syncwarp();
-      if (lane == 0) {
-        const float alpha = exp2f(m_old - mu);  // 0 while m_old is -inf
-        sAlpha[r] = alpha;
-        sML[r][0] = M;
-        sML[r][1] = sML[r][1] * alpha + l;
-      }
-    }
-    __syncthreads();
-
-    // 4. o[r][d] = alpha o[r][d] + sum_key w[r][key] v[key][d]: thread ->
-    //    outputs (tid % OUTS) + NT j over key part tid / OUTS
-    {
-      const __nv_bfloat16* sVh = reinterpret_cast<const __nv_bfloat16*>(sV);
-      const int part = OUTS >= NT ? 0 : tid / OUTS;
-      const int kb0 = part * (CH / PARTS), ke = kb0 + CH / PARTS;
-#pragma unroll
-      for (int j = 0; j < OPT; ++j) {
-        const int out = (OUTS >= NT ? tid + NT * j : tid % OUTS);
-        const int r = out / D, d = out - (out / D) * D;
-        float a0 = 0.f, a1 = 0.f;
-        for (int key = kb0; key < ke; key += 2) {
-          a0 = fmaf(sW[r][key], __bfloat162float(sVh[dec_swz<VPR>(key, d / 8) * 8 + (d & 7)]), a0);
-          a1 = fmaf(sW[r][key + 1],
-                    __bfloat162float(sVh[dec_swz<VPR>(key + 1, d / 8) * 8 + (d & 7)]), a1);
-        }
-        o_run[j] = fmaf(o_run[j], sAlpha[r], a0 + a1);
-      }
-    }
-    __syncthreads();  // shared K, V and W are rewritten by the next chunk
+  for (int i = 0; i < kDecodeStages; ++i) {
+    if (i < n_my) issue(i);
+    dec_cp_async_commit();
   }
 
-  // 5. the CTA's (M, l, o) to the workspace: the key parts summed
+  // the query rows as mma A fragments (rows g >= Tq and 8 .. 15 zero):
+  // qa[kk][0] = q[g][16kk + 2 t4 ..+1], qa[kk][1] = q[g][16kk + 8 + 2 t4 ..+1]
+  uint32_t qa[KS][2];
   {
-    const int part = OUTS >= NT ? 0 : tid / OUTS;
+    const __nv_bfloat16* qr = p.q + b * p.q_sb + h * p.q_sh + static_cast<long long>(g) * p.q_st;
 #pragma unroll
-    for (int j = 0; j < OPT; ++j) sO[part][OUTS >= NT ? tid + NT * j : tid % OUTS] = o_run[j];
-  }
-  __syncthreads();
-  for (int out = tid; out < Tq * D; out += NT) {
-    const int r = out / D, d = out - (out / D) * D;
-    float acc = 0.f;
-#pragma unroll
-    for (int q = 0; q < PARTS; ++q) acc += sO[q][out];
-    const size_t row = (static_cast<size_t>(bh) * p.n_split + split) * Tq + r;
-    p.part_o[row * D + d] = acc;
-    if (d == 0) {
-      p.part_ml[row * 2] = sML[r][0];
-      p.part_ml[row * 2 + 1] = sML[r][1];
+    for (int kk = 0; kk < KS; ++kk) {
+      qa[kk][0] = g < Tq ? *reinterpret_cast<const uint32_t*>(qr + 16 * kk + 2 * t4) : 0u;
+      qa[kk][1] = g < Tq ? *reinterpret_cast<const uint32_t*>(qr + 16 * kk + 8 + 2 * t4) : 0u;
     }
   }
-}
 
-// One CTA of kCombineThreads per (head, query row) merges the chunks:
-// first M = max_c m_c (the threads read the chunks' m in parallel, then a
-// block reduction), then per column d the sums over the chunks of
-// 2^(m_c - M) o_c[d] and 2^(m_c - M) l_c, the chunks dealt to
-// kCombineThreads / D thread groups so that every thread has few,
-// independent loads, then the groups' sums added.  Key 0 is in chunk 0 and
-// visible to every row, so M is finite.
-constexpr int kCombineThreads = 128;
+  // running state of row g (lanes of a quad share it; l is the lane's part)
+  float o[NO][4];
+#pragma unroll
+  for (int j = 0; j < NO; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+  const float sl2 = p.scale_log2;
+  // last key row g sees (padding rows >= Tq: every key of the cache)
+  const int last_visible = min(pos0 + g, L - 1);
 
-template <int D>
-__global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(const DecodeParams p) {
-  constexpr int NT = kCombineThreads;
-  constexpr int PARTS = NT / D;  // thread groups over the chunks (D <= 128)
-  __shared__ float sRed[NT / 32];
-  __shared__ float sO[PARTS][D];
-  __shared__ float sL[PARTS];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int row = blockIdx.x;  // bh * Tq + r
-  const int bh = row / p.Tq, r = row - (row / p.Tq) * p.Tq;
-  const int b = bh / p.H, h = bh - b * p.H;
-  const size_t first = static_cast<size_t>(bh) * p.n_split * p.Tq + r;  // chunk 0's row
-  float m = -INFINITY;
-  for (int c = tid; c < p.n_split; c += NT)
-    m = fmaxf(m, p.part_ml[(first + static_cast<size_t>(c) * p.Tq) * 2]);
+  for (int i = 0; i < n_my; ++i) {
+    dec_cp_async_wait<kDecodeStages - 1>();
+    __syncwarp();  // every lane's pieces of chunk i are in shared memory
+    const uint8_t* sk = ring + (i % kDecodeStages) * kDecodeChunkBytes;
+    const uint8_t* sv = sk + TILE;
+    const int k0 = (first + NW * i) * CK;
+
+    // s = q k^T: n-tile nt holds keys k0 + 8nt .. +7; lane's c0, c1 are
+    // row g, keys 8nt + 2t4, +1
+    float s[NS][4];
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-  if (lane == 0) sRed[warp] = m;
-  __syncthreads();
-  float M = sRed[0];
+    for (int nt = 0; nt < NS; ++nt) {
+      s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+      if constexpr (P >= 4) {
 #pragma unroll
-  for (int i = 1; i < NT / 32; ++i) M = fmaxf(M, sRed[i]);
-  const int d = tid % D, part = tid / D;
-  float o = 0.f, l = 0.f;
-#pragma unroll 4
-  for (int c = part; c < p.n_split; c += PARTS) {
-    const size_t pr = first + static_cast<size_t>(c) * p.Tq;
-    const float w = exp2f(p.part_ml[pr * 2] - M);
-    o = fmaf(w, p.part_o[pr * D + d], o);
-    l = fmaf(p.part_ml[pr * 2 + 1], w, l);
-  }
-  sO[part][d] = o;
-  if (d == 0) sL[part] = l;
-  __syncthreads();
-  if (part == 0) {
-    float os = 0.f, ls = 0.f;
-#pragma unroll
-    for (int q = 0; q < PARTS; ++q) {
-      os += sO[q][d];
-      ls += sL[q];
+        for (int x = 0; x < P / 4; ++x) {
+          uint32_t r[4];
+          dec_ldsm_x4(r, sk + dec_swz<D>(nt * 8 + (lane & 7), 4 * x + (lane >> 3)));
+          dec_mma(s[nt], qa[2 * x][0], 0u, qa[2 * x][1], 0u, r[0], r[1]);
+          dec_mma(s[nt], qa[2 * x + 1][0], 0u, qa[2 * x + 1][1], 0u, r[2], r[3]);
+        }
+      } else {  // D = 16: one k-step, two matrices
+        uint32_t r[2];
+        dec_ldsm_x2(r, sk + dec_swz<D>(nt * 8 + (lane & 7), (lane >> 3) & 1));
+        dec_mma(s[nt], qa[0][0], 0u, qa[0][1], 0u, r[0], r[1]);
+      }
     }
-    p.o[b * p.o_sb + h * p.o_sh + r * p.o_st + d] = __float2bfloat16_rn(os / ls);
-    if (d == 0) p.lse[row] = (M + log2f(ls)) * 0.69314718055994531f;
+    // keys past the cache, and keys after the row's position
+    if (k0 + CK - 1 > pos0) {
+#pragma unroll
+      for (int nt = 0; nt < NS; ++nt)
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+          if (k0 + nt * 8 + 2 * t4 + c > last_visible) s[nt][c] = -INFINITY;
+    }
+
+    // online softmax of row g over this chunk
+    float mx = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < NS; ++nt) mx = fmaxf(mx, fmaxf(s[nt][0], s[nt][1]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m_run, mx * sl2);
+    const float mu = m_new == -INFINITY ? 0.f : m_new;  // no visible key yet
+    const float alpha = exp2f(m_run - mu);               // 0 while m_run is -inf
+    m_run = m_new;
+    uint32_t pk[NS];  // the weights as bf16 pairs (A fragments of p v)
+    float ls = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < NS; ++nt) {
+      const float p0 = exp2f(fmaf(s[nt][0], sl2, -mu));
+      const float p1 = exp2f(fmaf(s[nt][1], sl2, -mu));
+      ls += p0 + p1;
+      pk[nt] = dec_pack_bf16(p0, p1);
+    }
+    l_run = fmaf(l_run, alpha, ls);
+#pragma unroll
+    for (int j = 0; j < NO; ++j) {
+      o[j][0] *= alpha;
+      o[j][1] *= alpha;
+    }
+
+    // o += p v over the chunk's 16-key steps; one transposed x4 covers 16
+    // keys x 16 columns (two output n-tiles)
+#pragma unroll
+    for (int kk = 0; kk < CK / 16; ++kk) {
+#pragma unroll
+      for (int jj = 0; jj < D / 16; ++jj) {
+        const int mi = lane >> 3;
+        uint32_t r[4];
+        dec_ldsm_x4_t(r, sv + dec_swz<D>(kk * 16 + (mi & 1) * 8 + (lane & 7), 2 * jj + (mi >> 1)));
+        dec_mma(o[2 * jj], pk[2 * kk], 0u, pk[2 * kk + 1], 0u, r[0], r[1]);
+        dec_mma(o[2 * jj + 1], pk[2 * kk], 0u, pk[2 * kk + 1], 0u, r[2], r[3]);
+      }
+    }
+    __syncwarp();  // every lane has read the slot: refill it
+    if (i + kDecodeStages < n_my) issue(i + kDecodeStages);
+    dec_cp_async_commit();
+  }
+  dec_cp_async_wait<0>();
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  __syncthreads();  // every warp is done with its ring: reuse it
+
+  // merge area: per warp (m, l, o) of its 8 fragment rows, then the CTA's
+  float* wm = reinterpret_cast<float*>(smem);  // [NW][8]
+  float* wl = wm + NW * 8;                      // [NW][8]
+  float* wo = wl + NW * 8;                      // [NW][8][D]
+  float* cm = wo + NW * 8 * D;                  // [8]
+  float* cl = cm + 8;                           // [8]
+  float* co = cl + 8;                           // [8][D]
+  if (t4 == 0) {
+    wm[warp * 8 + g] = m_run;
+    wl[warp * 8 + g] = l_run;
+  }
+#pragma unroll
+  for (int j = 0; j < NO; ++j)
+    *reinterpret_cast<float2*>(wo + (warp * 8 + g) * D + j * 8 + 2 * t4) = float2{o[j][0], o[j][1]};
+  __syncthreads();
+
+  __nv_bfloat16* ob = p.o + b * p.o_sb + h * p.o_sh;
+  float* lseb = p.lse + bh * Tq;
+  for (int e = tid; e < Tq * D; e += kDecodeThreads) {
+    const int r = e / D, d = e - (e / D) * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, wm[w * 8 + r]);
+    float Ls = 0.f, Os = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float mw = wm[w * 8 + r];
+      const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);  // warp without a visible key
+      Ls = fmaf(f, wl[w * 8 + r], Ls);
+      Os = fmaf(f, wo[(w * 8 + r) * D + d], Os);
+    }
+    if (p.n_split == 1) {  // key 0 is in this CTA: M is finite, Ls > 0
+      ob[r * p.o_st + d] = __float2bfloat16_rn(Os / Ls);
+      if (d == 0) lseb[r] = (M + log2f(Ls)) * 0.69314718055994531f;
+    } else {
+      co[r * D + d] = Os;
+      if (d == 0) {
+        cm[r] = M;
+        cl[r] = Ls;
+      }
+    }
+  }
+  if (p.n_split > 1) {
+    dec_cluster_sync();  // every CTA's partial is in its shared memory
+    const unsigned ns = static_cast<unsigned>(p.n_split);
+    for (int e = split * kDecodeThreads + tid; e < Tq * D; e += p.n_split * kDecodeThreads) {
+      const int r = e / D, d = e - (e / D) * D;
+      float M = -INFINITY;
+      for (unsigned c = 0; c < ns; ++c) M = fmaxf(M, dec_cluster_ld(cm + r, c));
+      float Ls = 0.f, Os = 0.f;  // key 0 is visible to every row: M is finite
+      for (unsigned c = 0; c < ns; ++c) {
+        const float mc = dec_cluster_ld(cm + r, c);
+        const float f = mc == -INFINITY ? 0.f : exp2f(mc - M);
+        Ls = fmaf(f, dec_cluster_ld(cl + r, c), Ls);
+        Os = fmaf(f, dec_cluster_ld(co + r * D + d, c), Os);
+      }
+      ob[r * p.o_st + d] = __float2bfloat16_rn(Os / Ls);
+      if (d == 0) lseb[r] = (M + log2f(Ls)) * 0.69314718055994531f;
+    }
+    dec_cluster_sync();  // no CTA leaves while its shared memory is read
   }
 }
 

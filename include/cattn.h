@@ -278,13 +278,16 @@ CATTN_API cattn_status attn_bwd_dropout(const void* q, cattn_layout lq, const vo
  *          read; a (B, Tmax, H, D) cache is { Tmax*H*D, D, H*D })
  *   o      bf16 (B, H, Tq, D) out, layout lo;  lse fp32 (B, H, Tq) out,
  *          contiguous, natural log
- *   workspace  attn_decode_workspace_bytes(B, H, Tq, L, D) bytes of device
- *          memory, 256-byte aligned (the per-chunk partial results)
+ *   workspace, workspace_bytes  not used (attn_decode_workspace_bytes
+ *          returns 0 for every shape; NULL and 0 are accepted): the CTAs
+ *          that share a head form a thread-block cluster and merge their
+ *          partial results in distributed shared memory
  *
- * The keys of each head are processed in chunks of 256 by separate CTAs and
- * merged by a second kernel; both run on `stream`.  1 <= Tq <= L; Tq above
- * 8 returns CATTN_ERR_UNSUPPORTED (use attn_fwd for a prefill).  Layout
- * rules as for the _strided calls; B = 0 or H = 0 is a no-op. */
+ * One kernel on `stream`: the keys of each head are cut into chunks of 4 KB
+ * of K (2048 / D keys) dealt to a cluster of up to 8 CTAs, four warps per
+ * CTA streaming their chunks.  1 <= Tq <= L; Tq above 8 returns
+ * CATTN_ERR_UNSUPPORTED (use attn_fwd for a prefill).  Layout rules as for
+ * the _strided calls; B = 0 or H = 0 is a no-op. */
 CATTN_API size_t attn_decode_workspace_bytes(int B, int H, int Tq, int L, int D);
 
 CATTN_API cattn_status attn_decode(const void* q, cattn_layout lq, const void* k,

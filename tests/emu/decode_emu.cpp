@@ -1,21 +1,24 @@
-// Runs the decode kernels of decode.cuh (the device source itself) on the
-// host through simt_emu.h, for CPU tests: exactly sized buffers under
-// AddressSanitizer and UBSan, so any out-of-bounds or misaligned access of
-// the kernels fails the run.
+// Runs the decode kernel of decode.cuh (the device source itself) on the
+// host through simt_emu.h and decode_ptx_emu.h, for CPU tests: exactly
+// sized buffers under AddressSanitizer and UBSan, so any out-of-bounds or
+// misaligned access of the kernel fails the run.
 //
 //   decode_emu B H Tq L D Tmax layout scale in.bin out.bin [ctas_per_head]
 //     layout 0: k, v stored (B, H, Tmax, D); 1: stored (B, Tmax, H, D)
 //     in.bin:  q (B, H, Tq, D), k, v (stored layout) as bf16 bit patterns
 //     out.bin: o (B, H, Tq, D) bf16 bit patterns, then lse (B, H, Tq) fp32
-//     ctas_per_head: partial CTAs per head (default: attn_decode's own
-//     choice); fewer CTAs than chunks make each CTA walk several chunks
-// The host set-up (chunk count, workspace split, strides) follows
+//     ctas_per_head: CTAs per head, the cluster size (default: attn_decode's
+//     own choice on a 148-SM B200); fewer CTAs than chunks make each CTA,
+//     and each of its warps, walk several chunks
+// The host set-up (cluster size, chunks per CTA, strides) follows
 // attn_decode in api.cu.
+#define CATTN_HOST_EMULATION 1
 #include "simt_emu.h"
 
 #include <cstdio>
 #include <cstdlib>
 
+#include "decode_ptx_emu.h"
 #include "decode.cuh"
 
 using namespace cattn;
@@ -27,16 +30,8 @@ static T* exact(size_t n) {
 
 template <int D>
 static void run(DecodeParams p, int BH) {
-  const dim3 grid(BH, p.n_split);
-  if (p.Tq <= 1)
-    emu::launch(grid, kDecodeThreads, decode_partial_kernel<D, 1>, p);
-  else if (p.Tq <= 2)
-    emu::launch(grid, kDecodeThreads, decode_partial_kernel<D, 2>, p);
-  else if (p.Tq <= 4)
-    emu::launch(grid, kDecodeThreads, decode_partial_kernel<D, 4>, p);
-  else
-    emu::launch(grid, kDecodeThreads, decode_partial_kernel<D, 8>, p);
-  emu::launch(dim3(BH * p.Tq), kCombineThreads, decode_combine_kernel<D>, p);
+  emu::launch_ex(static_cast<unsigned>(BH * p.n_split), kDecodeThreads, kDecodeSmemBytes,
+                 static_cast<unsigned>(p.n_split), decode_kernel<D>, p);
 }
 
 int main(int argc, char** argv) {
@@ -59,16 +54,14 @@ int main(int argc, char** argv) {
   std::fclose(f);
   const int BH = B * H;
   const int n_chunks = (L + decode_chunk(D) - 1) / decode_chunk(D);
-  int n_split = decode_splits_for(static_cast<long long>(B) * H, L, D, Tq);
-  int cpc = decode_chunks_per_cta(static_cast<long long>(B) * H, L, D, Tq);
+  const int slots = 148 * kDecodeCtasPerSm;
+  int n_split = decode_splits_for(static_cast<long long>(B) * H, L, D, slots);
+  int cpc = decode_chunks_per_cta(static_cast<long long>(B) * H, L, D, slots);
   if (argc == 12) {  // a chosen number of CTAs per head
     const int want = std::atoi(argv[11]);
     cpc = (n_chunks + want - 1) / want;
     n_split = (n_chunks + cpc - 1) / cpc;
   }
-  const size_t rows = static_cast<size_t>(BH) * n_split * Tq;
-  auto* part_ml = exact<float>(rows * 2);
-  auto* part_o = exact<float>(rows * D);
   auto* o = exact<__nv_bfloat16>(nq);
   auto* lse = exact<float>(static_cast<size_t>(BH) * Tq);
   DecodeParams p{};
@@ -90,8 +83,6 @@ int main(int argc, char** argv) {
   p.v_sb = p.k_sb;
   p.v_sh = p.k_sh;
   p.v_st = p.k_st;
-  p.part_ml = part_ml;
-  p.part_o = part_o;
   p.o = o;
   p.o_sb = p.q_sb;
   p.o_sh = p.q_sh;
@@ -118,8 +109,6 @@ int main(int argc, char** argv) {
   std::free(q);
   std::free(k);
   std::free(v);
-  std::free(part_ml);
-  std::free(part_o);
   std::free(o);
   std::free(lse);
   return 0;

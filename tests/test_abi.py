@@ -332,33 +332,15 @@ def test_decode_checks_arguments_before_the_device():
     assert decode(D=48) == cattn.ERR_UNSUPPORTED
     assert decode(B=0) == cattn.OK
     assert decode(lay=_binding.Layout(512, 64, 12)) == cattn.ERR_INVALID_ARG
-    assert decode(ws_bytes=16) == cattn.ERR_INVALID_ARG
 
 
-def test_decode_workspace_formula():
-    # per (head, partial CTA, query row): (m, l) and D partial outputs.  A
-    # chunk is 16 KB of K (8192 / D keys, at most 256); a head's chunks are
-    # dealt to about 148 * (4, or 3 above 2 rows) / (B*H) CTAs (one wave),
-    # each a run of chunks.
-    def r256(x):
-        return (x + 255) // 256 * 256
-
-    def splits(BH, L, D, Tq):
-        chunk = min(8192 // D, 256)
-        n_chunks = (L + chunk - 1) // chunk
-        per_sm = 4 if Tq <= 2 else 3
-        s = max(1, min(n_chunks, 148 * per_sm // BH))
-        cpc = (n_chunks + s - 1) // s
-        return (n_chunks + cpc - 1) // cpc
-    assert splits(192, 1024, 64, 1) == 3 and splits(32, 8192, 128, 1) == 16
-    assert splits(192, 1024, 64, 4) == 2
+def test_decode_needs_no_workspace():
+    # the CTAs of a head (a thread-block cluster) merge their partial
+    # results in distributed shared memory: no workspace for any shape
     for B, H, Tq, L, D in [(1, 1, 1, 1, 16), (2, 3, 4, 257, 64), (16, 12, 1, 1024, 64),
                            (1, 2, 8, 4096, 128), (2, 16, 1, 8192, 128), (64, 12, 2, 300, 32),
-                           (16, 12, 8, 1024, 64)]:
-        rows = B * H * splits(B * H, L, D, Tq) * Tq
-        assert cattn.attn_decode_workspace_bytes(B, H, Tq, L, D) == r256(rows * 8) + r256(rows * D * 4)
-    assert cattn.attn_decode_workspace_bytes(1, 1, 9, 16, 64) == 0
-    assert cattn.attn_decode_workspace_bytes(1, 1, 2, 1, 64) == 0
+                           (16, 12, 8, 1024, 64), (1, 1, 9, 16, 64), (1, 1, 2, 1, 64)]:
+        assert cattn.attn_decode_workspace_bytes(B, H, Tq, L, D) == 0
 
 
 # ------------------------------------------------------------ Python checks
@@ -448,7 +430,7 @@ def test_strided_dropout_and_decode_calls_check_alignment_and_nulls():
                                    ALIGNED, c, ALIGNED, c, 0, ALIGNED + 128, 1 << 30, None)
     assert r == cattn.ERR_INVALID_ARG    # workspace not 256-byte aligned
     for kw in (dict(q=ALIGNED + 8), dict(k=ALIGNED + 8), dict(o=ALIGNED + 8),
-               dict(lse=ALIGNED + 2), dict(ws=ALIGNED + 16), dict(v=None)):
+               dict(lse=ALIGNED + 2), dict(v=None)):
         a = dict(q=ALIGNED, k=ALIGNED, v=ALIGNED, o=ALIGNED, lse=ALIGNED, ws=ALIGNED)
         a.update(kw)
         r = cattn.LIB.attn_decode(a["q"], c, a["k"], c, a["v"], c, 0.125, 1, 2, 1, 8, 64,

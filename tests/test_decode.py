@@ -73,6 +73,7 @@ def test_decode_argument_errors(lib):
         lib.attn_decode(q, k, k, 16)
     with pytest.raises(lib.CattnError):        # L < Tq
         lib.attn_decode(q[:, :, :4], k, k, 3)
-    ws = torch.empty(16, dtype=torch.uint8, device=dev)
-    with pytest.raises(lib.CattnError):        # workspace too small
-        lib.attn_decode(q[:, :, :1], k, k, 16, workspace=ws)
+    # no workspace is needed: an empty one is accepted
+    ws = torch.empty(0, dtype=torch.uint8, device=dev)
+    lib.attn_decode(q[:, :, :1], k, k, 16, workspace=ws)
+    torch.cuda.synchronize()

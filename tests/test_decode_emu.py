@@ -1,8 +1,9 @@
-"""The decode kernels' own source run on the CPU (tests/emu: each CUDA
-thread a host thread, warp shuffles and __syncthreads by barriers), built
-with AddressSanitizer and UBSan over exactly sized buffers.  Any
-out-of-bounds or misaligned access of the kernels' indexing fails the run;
-the outputs are compared with the fp64 decode oracle.  This checks the
+"""The decode kernel's own source run on the CPU (tests/emu: each CUDA
+thread a host thread, warp-level instructions and barriers emulated, the
+CTAs of a cluster together), built with AddressSanitizer and UBSan over
+exactly sized buffers.  Any out-of-bounds or misaligned access of the
+kernel's indexing fails the run; the outputs are compared with the fp64
+decode oracle.  This checks the
 indexing and the split/merge logic on shapes the GPU tests do not reach,
 without a GPU."""
 
@@ -48,16 +49,21 @@ def from_bits(b: np.ndarray) -> np.ndarray:
     return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-# (B, H, Tq, L, D, layout, partial CTAs per head or None for attn_decode's
-# own choice); a count below the number of chunks makes each CTA walk
-# several chunks (the cross-chunk merge)
+# (B, H, Tq, L, D, layout, CTAs per head (the cluster size) or None for
+# attn_decode's own choice); a count below the number of chunks makes each
+# CTA walk several chunks (the cross-chunk merge)
 @pytest.mark.parametrize("B,H,Tq,L,D,layout,ctas", [
     (1, 1, 1, 1, 16, 0, None), (2, 2, 1, 300, 64, 0, None), (1, 2, 3, 257, 128, 1, None),
     (1, 1, 8, 8, 32, 0, None), (2, 1, 8, 513, 16, 1, None), (1, 3, 2, 256, 64, 1, None),
     (1, 1, 5, 1000, 128, 0, None), (1, 2, 4, 37, 64, 0, None), (2, 1, 2, 70, 32, 1, None),
     (1, 1, 7, 520, 64, 1, None), (1, 1, 1, 255, 128, 1, None), (3, 1, 6, 129, 16, 0, None),
     (1, 2, 1, 1000, 64, 0, 1), (1, 1, 4, 700, 128, 1, 3), (2, 1, 8, 1100, 32, 0, 2),
-    (1, 1, 3, 600, 16, 1, 1)])
+    (1, 1, 3, 600, 16, 1, 1),
+    # the last CTA of the cluster holds only key 32, after rows 0-6's
+    # positions: its partial for those rows is empty (m = -inf)
+    (1, 1, 8, 33, 128, 0, None),
+    # Tq = L: row 0 sees key 0 only
+    (1, 2, 8, 8, 64, 1, None)])
 def test_decode_kernels_on_the_host(emu_exe, tmp_path, B, H, Tq, L, D, layout, ctas):
     g = torch.Generator().manual_seed(1000 * L + D + Tq)
     Tmax = L       # a tight cache: a read past row L - 1 leaves the buffer
