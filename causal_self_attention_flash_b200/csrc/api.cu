@@ -577,18 +577,18 @@ __global__ void selftest_wait_kernel(uint64_t timeout_ns, unsigned int* call_sta
 
 // ------------------------------------------------------------------ decode
 
-// Resident decode CTAs on the device: its SMs x kDecodeCtasPerSm.
-int decode_slots(int dev) { return g_sm_count[dev] * kDecodeCtasPerSm; }
+// Resident decode CTAs on the device: its SMs x decode_ctas_per_sm(D).
+int decode_slots(int dev, int D) { return g_sm_count[dev] * decode_ctas_per_sm(D); }
 
 template <int D>
 cattn_status decode_impl(const DecodeParams& p, long long BH, int dev, cudaStream_t s) {
-  cattn_status st = ensure_smem(dev, 64 + d_index(D), decode_kernel<D>, kDecodeSmemBytes);
+  cattn_status st = ensure_smem(dev, 64 + d_index(D), decode_kernel<D>, decode_smem_bytes(D));
   if (st != CATTN_OK) return st;
   clear_stale_error();
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(BH * p.n_split));
   cfg.blockDim = dim3(kDecodeThreads);
-  cfg.dynamicSmemBytes = kDecodeSmemBytes;
+  cfg.dynamicSmemBytes = decode_smem_bytes(D);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -688,7 +688,7 @@ cattn_status attn_decode(const void* q, cattn_layout lq, const void* k, cattn_la
   const long long BH = static_cast<long long>(B) * H;
   int dev;
   if ((st = check_device(&dev)) != CATTN_OK) return st;
-  const int n_split = decode_splits_for(BH, L, D, decode_slots(dev));
+  const int n_split = decode_splits_for(BH, L, D, decode_slots(dev, D));
   if (BH * n_split > 0x7fffffffLL) return CATTN_ERR_INVALID_ARG;
   DecodeParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -704,7 +704,7 @@ cattn_status attn_decode(const void* q, cattn_layout lq, const void* k, cattn_la
   p.Tq = Tq;
   p.L = L;
   p.n_split = n_split;
-  p.chunks_per_cta = decode_chunks_per_cta(BH, L, D, decode_slots(dev));
+  p.chunks_per_cta = decode_chunks_per_cta(BH, L, D, decode_slots(dev, D));
   p.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (D) {

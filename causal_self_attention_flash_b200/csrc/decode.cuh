@@ -50,17 +50,21 @@ constexpr int kDecodeMaxTq = 8;                        // query rows per call
 constexpr int kDecodeWarps = 4;                        // warps per CTA
 constexpr int kDecodeThreads = 32 * kDecodeWarps;
 constexpr int kDecodeStages = 3;                       // chunks in flight per warp
-constexpr int kDecodeChunkBytes = 8192;                // K and V of one chunk
-constexpr int kDecodeSmemBytes = kDecodeWarps * kDecodeStages * kDecodeChunkBytes;
-constexpr int kDecodeCtasPerSm = 2;                    // 2 x 96 KB of shared memory
 constexpr int kDecodeMaxCluster = 8;                   // portable cluster size
 
-// Keys per chunk: 4 KB of K, 4 KB of V (128, 64, 32, 16 keys for D = 16 ..
-// 128).
-__host__ __device__ constexpr int decode_chunk(int D) { return kDecodeChunkBytes / 4 / D; }
+// Bytes of K and V per chunk: 4 KB of K and 4 KB of V.
+__host__ __device__ constexpr int decode_chunk_bytes(int D) { return (void)D, 8192; }
+// Keys per chunk (128, 64, 32, 16 for D = 16 .. 128).
+__host__ __device__ constexpr int decode_chunk(int D) { return decode_chunk_bytes(D) / 4 / D; }
+// Dynamic shared memory per CTA: every warp's ring (96 KB).
+__host__ __device__ constexpr int decode_smem_bytes(int D) {
+  return kDecodeWarps * kDecodeStages * decode_chunk_bytes(D);
+}
+// Resident CTAs per SM (2 x 96 KB of shared memory).
+__host__ __device__ constexpr int decode_ctas_per_sm(int D) { return (void)D, 2; }
 
 // CTAs per head (the cluster size): enough to fill `slots` resident CTAs
-// (SMs x kDecodeCtasPerSm), at most kDecodeMaxCluster and at most one per
+// (SMs x decode_ctas_per_sm(D)), at most kDecodeMaxCluster and at most one per
 // chunk; then the number of CTAs that a run of equal length leaves work
 // for.
 __host__ __device__ constexpr int decode_splits_for(long long BH, int L, int D, int slots) {
@@ -105,10 +109,10 @@ __host__ __device__ constexpr int dec_swz(int row, int pc) {
 }
 
 // Grid: BH * n_split CTAs of kDecodeThreads, clusters of n_split along x
-// (CTA x: head x / n_split, cluster rank x % n_split), kDecodeSmemBytes of
-// dynamic shared memory.
+// (CTA x: head x / n_split, cluster rank x % n_split), decode_smem_bytes(D)
+// of dynamic shared memory.
 template <int D>
-__global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
+__global__ void __launch_bounds__(kDecodeThreads, decode_ctas_per_sm(D))
     decode_kernel(const DecodeParams p) {
   constexpr int CK = decode_chunk(D);  // keys per chunk
   constexpr int P = D / 8;             // 16-byte pieces per row
@@ -117,8 +121,10 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
   constexpr int NO = D / 8;            // output n-tiles
   constexpr int TILE = CK * D * 2;     // bytes of K (of V) per chunk
   constexpr int NW = kDecodeWarps;
-  static_assert(2 * TILE == kDecodeChunkBytes && TILE / 16 % 32 == 0, "chunk");
+  constexpr int CB = decode_chunk_bytes(D);
+  static_assert(2 * TILE == CB && TILE / 16 % 32 == 0, "chunk");
   static_assert(NS % 2 == 0 && D % 16 == 0, "tiles");
+  static_assert((2 * NW * 8 + NW * 8 * D + 16 + 8 * D) * 4 <= decode_smem_bytes(D), "merge area");
 
   uint8_t* smem = dec_dynamic_smem();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -136,13 +142,13 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
   // this warp's chunks: first, first + NW, ... below c_end
   const int first = c_begin + warp;
   const int n_my = first < c_end ? (c_end - first + NW - 1) / NW : 0;
-  uint8_t* ring = smem + warp * (kDecodeStages * kDecodeChunkBytes);
+  uint8_t* ring = smem + warp * (kDecodeStages * CB);
 
   // chunk i of this warp into ring slot i % kDecodeStages; keys past the
   // cache are zero-filled (and masked below)
   auto issue = [&](int i) {
     const int k0 = (first + NW * i) * CK;
-    uint8_t* sk = ring + (i % kDecodeStages) * kDecodeChunkBytes;
+    uint8_t* sk = ring + (i % kDecodeStages) * CB;
     uint8_t* sv = sk + TILE;
 #pragma unroll
     for (int u = 0; u < TILE / 16 / 32; ++u) {
@@ -187,7 +193,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
   for (int i = 0; i < n_my; ++i) {
     dec_cp_async_wait<kDecodeStages - 1>();
     __syncwarp();  // every lane's pieces of chunk i are in shared memory
-    const uint8_t* sk = ring + (i % kDecodeStages) * kDecodeChunkBytes;
+    const uint8_t* sk = ring + (i % kDecodeStages) * CB;
     const uint8_t* sv = sk + TILE;
     const int k0 = (first + NW * i) * CK;
 

@@ -30,7 +30,7 @@ static T* exact(size_t n) {
 
 template <int D>
 static void run(DecodeParams p, int BH) {
-  emu::launch_ex(static_cast<unsigned>(BH * p.n_split), kDecodeThreads, kDecodeSmemBytes,
+  emu::launch_ex(static_cast<unsigned>(BH * p.n_split), kDecodeThreads, decode_smem_bytes(D),
                  static_cast<unsigned>(p.n_split), decode_kernel<D>, p);
 }
 
@@ -54,7 +54,7 @@ int main(int argc, char** argv) {
   std::fclose(f);
   const int BH = B * H;
   const int n_chunks = (L + decode_chunk(D) - 1) / decode_chunk(D);
-  const int slots = 148 * kDecodeCtasPerSm;
+  const int slots = 148 * decode_ctas_per_sm(D);
   int n_split = decode_splits_for(static_cast<long long>(B) * H, L, D, slots);
   int cpc = decode_chunks_per_cta(static_cast<long long>(B) * H, L, D, slots);
   if (argc == 12) {  // a chosen number of CTAs per head
