@@ -300,7 +300,7 @@ cattn_status fwd_impl(int dev, const void* q, cattn_layout lq, const void* k, ca
                       cattn_layout lo, float* lse, void* o_lo, const DropParams& dp,
                       cudaStream_t s) {
   const int BH = B * H;
-  using C = FwdCfg<D, PLO>;
+  using C = FwdCfg<D, PLO, DROP>;
   clear_stale_error();
   cattn_status st = ensure_smem(dev, (FLAT ? 32 : 0) + (DROP ? 16 : 0) + 2 * d_index(D) + PLO,
                                 fwd_kernel<D, PLO, DROP, FLAT>, C::SMEM_BYTES,

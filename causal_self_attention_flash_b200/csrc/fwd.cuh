@@ -57,10 +57,14 @@
 // unchanged: it is still exactly the softmax, as the online rewrite is.
 //
 // Instances fwd_kernel<D, PLO, DROP, FLAT>:
-//   DROP   attention dropout (philox.cuh): each softmax thread draws its
-//          row's keep bits for a key tile before that tile's scores arrive,
-//          writes the dropped P entries as 0 (the row sum l still takes
-//          every entry) and folds the keep scale 1 / (1 - p) into 1 / l.
+//   DROP   attention dropout (philox.cuh): the softmax writes the dropped
+//          P entries as 0 (the row sum l still takes every entry) and folds
+//          the keep scale 1 / (1 - p) into 1 / l.  With D <= 64 a fourth
+//          warpgroup draws the keep bits (one thread per query row, a key
+//          tile ahead of the softmax) into a shared-memory ring, so the
+//          generator's integer work runs beside the softmax instead of in
+//          it; with D = 128 each softmax thread draws its own row's bits
+//          before the tile's scores arrive.
 //   FLAT   Q, K, V and O address (b, h) as one b*H + h index (3-D tensor
 //          maps); otherwise 4-D maps {d, t, h, b} take any element strides,
 //          e.g. q, k, v as views into one fused (B, T, 3C) projection.
@@ -85,7 +89,7 @@ struct FwdParams {
   DropParams drop;     // attention dropout (kernels instantiated with DROP only)
 };
 
-template <int D, bool PLO>
+template <int D, bool PLO, bool DROP = false>
 struct FwdCfg {
   static constexpr int BM = 128, BN = 128;
   static constexpr int CB = D < 64 ? D : 64;      // columns per swizzle block
@@ -101,8 +105,13 @@ struct FwdCfg {
   static constexpr int OFF_Q = 0;                              // [2] query tiles
   static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_V + STAGES * TILE_BYTES;
-  static constexpr int NUM_BARS = 47;
+  // MASKW: dropout keep bits drawn by their own warpgroup into
+  // [2 groups][2 slots][128 rows] x 16 bytes (128 bits per row and key tile)
+  static constexpr bool MASKW = DROP && D <= 64;
+  static constexpr int OFF_MASK = OFF_V + STAGES * TILE_BYTES;
+  static constexpr int MASK_BYTES = MASKW ? 2 * 2 * 128 * 16 : 0;
+  static constexpr int OFF_BAR = OFF_MASK + MASK_BYTES;
+  static constexpr int NUM_BARS = 55;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_USED = OFF_MISC + 64;
   // at least 116 KB so that one CTA holds an SM (it takes all 512 TMEM columns)
@@ -131,11 +140,14 @@ struct FwdCfg {
   // launch total.  That removed the D = 128 softmax's spills (3.6 % faster
   // on the long-context workload); with D <= 64 the same split measured
   // 4 % slower, so those keep 11 warps and 168 registers throughout.
-  static constexpr bool REBALANCE = D == 128;
-  static constexpr int THREADS = REBALANCE ? 384 : 352;
-  static constexpr int LAUNCH_REGS = 168;
-  static constexpr int REGS_SOFTMAX = 216, REGS_OTHER = 64;
-  static_assert(!REBALANCE || 256 * REGS_SOFTMAX + 128 * REGS_OTHER <= THREADS * LAUNCH_REGS,
+  // MASKW adds the keep-bit warpgroup (16 warps): 128 registers at launch,
+  // 184 for the softmax, 72 for the rest.
+  static constexpr bool REBALANCE = D == 128 || MASKW;
+  static constexpr int THREADS = MASKW ? 512 : REBALANCE ? 384 : 352;
+  static constexpr int LAUNCH_REGS = MASKW ? 128 : 168;
+  static constexpr int REGS_SOFTMAX = MASKW ? 184 : 216, REGS_OTHER = MASKW ? 72 : 64;
+  static_assert(!REBALANCE ||
+                    256 * REGS_SOFTMAX + (THREADS - 256) * REGS_OTHER <= THREADS * LAUNCH_REGS,
                 "register split exceeds the launch allocation");
 };
 
@@ -148,7 +160,9 @@ enum : int {
   FB_QFREE = FB_QFULL + 2, FB_SFULL = FB_QFULL + 4, FB_ODONE = FB_QFULL + 6,
   FB_OFREE = FB_QFULL + 8, FB_SFREE = FB_QFULL + 10, FB_DRAIN = FB_QFULL + 12,
   FB_PFULL = FB_QFULL + 14,  // FB_PFULL + 4 * g + part
-  FB_OFFSET = FB_PFULL + 8   // the one-time start offset of the two groups
+  FB_OFFSET = FB_PFULL + 8,  // the one-time start offset of the two groups
+  FB_MFULL = FB_OFFSET + 1,  // keep bits of group g, slot s: FB_MFULL + 2 * g + s
+  FB_MEMPTY = FB_MFULL + 4   // the slot read by all 128 softmax threads
 };
 
 // Pairs of score columns whose exponential is taken by exp2_poly2 on the FMA
@@ -160,6 +174,21 @@ enum : int {
 // slower, so it is 0 there.  Only used on tiles without masked entries
 // (exp2_poly2 has no exact zero).
 __host__ __device__ constexpr uint32_t fwd_poly_pairs(int D) { return D == 128 ? 0x11u : 0x00u; }
+
+// Exponential-phase turns: the two softmax warps of a sub-partition (warp
+// q of group 0 and warp 4 + q of group 1) share its ex2 unit.  When both
+// run their exponential phases at once, each takes twice as long and their
+// other work (score loads, maxima, waits) then overlaps nothing; so a warp
+// about to start its phase first waits, for a bounded number of short
+// sleeps, while its partner's busy flag (shared memory) is set.  Only a
+// scheduling hint: a warp that gives up, or that races its partner past the
+// check, just runs its phase alongside, and no result depends on it.
+// Measured: 4-5 % faster forward with D = 128 (long-context workload, 16
+// polls; 64 and 256 polls gained less), 5 % slower with D = 64, whose
+// phases are short against the waits between them: only D = 128 takes
+// turns.
+__host__ __device__ constexpr bool fwd_exp_turns(int D) { return D == 128; }
+constexpr int kFwdTurnPolls = 16;  // sleeps of ~32 ns before giving up
 
 // P_g(j) is handed to the MMA warp in kPvParts parts (of 128 / kPvParts
 // keys each), so PV_g(j) starts while the later exponentials are computed.
@@ -257,11 +286,11 @@ __device__ __forceinline__ FwdItem fwd_item_info(int u, int k, int BH, int n_pai
 // FLAT: Q, K, V and O address (b, h) as one b*H + h axis (3-D tensor
 // maps, O offsets bh * o_sh); otherwise 4-D maps with (h, b) coordinates.
 template <int D, bool PLO, bool DROP, bool FLAT>
-__global__ void __launch_bounds__(FwdCfg<D, PLO>::THREADS, 1)
+__global__ void __launch_bounds__(FwdCfg<D, PLO, DROP>::THREADS, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using C = FwdCfg<D, PLO>;
-  static_assert(FB_OFFSET + 1 <= C::NUM_BARS, "barrier count");
+  using C = FwdCfg<D, PLO, DROP>;
+  static_assert(FB_MEMPTY + 4 <= C::NUM_BARS, "barrier count");
   static_assert(C::STAGES <= kMaxStages, "barrier map");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = aligned_smem(smem_raw, C::SMEM_USED, nullptr);
@@ -279,8 +308,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 
   WaitCtx w{p.timeout_ns, abort_flag, 1u, false};
 
+  volatile int* exp_busy = reinterpret_cast<volatile int*>(misc + 8);  // [8 softmax warps]
   if (threadIdx.x == 0) {
     *abort_flag = 0;
+    for (int i = 0; i < 8; ++i) exp_busy[i] = 0;
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(bar(FB_KFULL + s), 1);
       mbar_init(bar(FB_VFULL + s), 1);
@@ -298,6 +329,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       mbar_init(bar(FB_DRAIN + g), 1);
     }
     mbar_init(bar(FB_OFFSET), 128);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(bar(FB_MFULL + i), 128);
+      mbar_init(bar(FB_MEMPTY + i), 128);
+    }
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -310,9 +345,53 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   const uint32_t tbase = misc[0];
 
   if (warp >= 8) {
-  // third warpgroup: producer, MMA issuers (and with REBALANCE an idle warp)
+  // third warpgroup: producer, MMA issuers (and with REBALANCE an idle
+  // warp); with MASKW the fourth, keep-bit warpgroup too
   if constexpr (C::REBALANCE) regs_dec<C::REGS_OTHER>();
-  if (warp == 8) {
+  if (warp >= 12) {
+    // ------------------------------------------------ keep bits (MASKW only)
+    // Thread t draws row t's keep bits for every key tile the softmax
+    // groups visit, in their order (tile j of group 0, then of group 1),
+    // into slot (tile count) % 2 of the group's ring, at most two tiles
+    // ahead of the group's softmax.
+    if constexpr (C::MASKW) {
+      const int t = threadIdx.x - 384;  // query row within the tile
+      uint4* mask = reinterpret_cast<uint4*>(smem + C::OFF_MASK);
+      int mg[2] = {0, 0};  // tiles drawn per group
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int u = fwd_item(k, b, G, n_items);
+        if (u < 0) break;
+        const FwdItem it = fwd_item_info(u, k, p.BH, n_pairs, p.n_qtiles);
+        const int jmax = it.n[0] > it.n[1] ? it.n[0] : it.n[1];
+        for (int j = 0; j < jmax && ok; ++j) {
+          for (int g = 0; g < 2; ++g) {
+            if (j >= it.n[g]) continue;
+            const int slot = mg[g] & 1;
+            if (mg[g] >= 2) {
+              const uint32_t ph = ((mg[g] >> 1) - 1) & 1;
+              if (!wait_warp(w, bar(FB_MEMPTY + 2 * g + slot), ph, 15)) {
+                ok = false;
+                break;
+              }
+              (void)mbar_try_wait(bar(FB_MEMPTY + 2 * g + slot), ph);  // acquire, every lane
+            }
+            const uint32_t qi = static_cast<uint32_t>(it.tile[g] * C::BM + t);
+            uint32_t kw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll 2  // fully unrolled, the 16 generator blocks spill at 72 registers
+            for (int c4 = 0; c4 < 4; ++c4)
+#pragma unroll
+              for (int x = 0; x < 4; ++x)
+                kw[c4] |= keep_byte(static_cast<uint32_t>(j * 16 + c4 * 4 + x), qi,
+                                    static_cast<uint32_t>(it.bh), p.drop) << (8 * x);
+            mask[(2 * g + slot) * 128 + t] = make_uint4(kw[0], kw[1], kw[2], kw[3]);
+            mbar_arrive(bar(FB_MFULL + 2 * g + slot));
+            ++mg[g];
+          }
+        }
+      }
+    }
+  } else if (warp == 8) {
     // ------------------------------------------------------------ producer
     // Per item: Q_g once the previous item no longer needs the Q_g buffer,
     // then K_j, V_j through a ring that runs on across items (tk counts the
@@ -518,7 +597,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // dropout keep bits of this row's 128 keys of tile j, computed while
         // the scores are still on their way
         [[maybe_unused]] uint32_t keep[4] = {0u, 0u, 0u, 0u};
-        if constexpr (DROP) {
+        if constexpr (DROP && !C::MASKW) {
           const uint32_t qi = static_cast<uint32_t>(it.tile[g] * C::BM + row);
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4)
@@ -598,14 +677,36 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const uint64_t sl2x2 = f2(sl2, sl2);
         const uint64_t negm2 = f2(-m_used, -m_used);
         uint64_t sum2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
+        if constexpr (C::MASKW) {  // this row's keep bits of tile j, from the ring
+          const int slot = tgj & 1;
+          wait_warp(w, bar(FB_MFULL + 2 * g + slot), (tgj >> 1) & 1, 16);
+          (void)mbar_try_wait(bar(FB_MFULL + 2 * g + slot), (tgj >> 1) & 1);  // acquire, every lane
+          const uint4 kw = reinterpret_cast<const uint4*>(smem + C::OFF_MASK)[(2 * g + slot) * 128 + row];
+          keep[0] = kw.x;
+          keep[1] = kw.y;
+          keep[2] = kw.z;
+          keep[3] = kw.w;
+          mbar_arrive(bar(FB_MEMPTY + 2 * g + slot));
+        }
         // Group 0's side of the one-time offset (see before the item loop).
         const bool offset = k == 0 && j == 0 && it.n[0] > 0 && it.n[1] > 0;
+        if constexpr (fwd_exp_turns(D)) {
+          if (lane == 0) {
+            for (int i = 0; i < kFwdTurnPolls && exp_busy[warp ^ 4]; ++i) __nanosleep(32);
+            exp_busy[warp] = 1;
+          }
+          __syncwarp();
+        }
         if (j == ng - 1)
           fwd_exp_row<D, false, PLO, DROP>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g),
                                            DROP ? keep : nullptr);
         else
           fwd_exp_row<D, true, PLO, DROP>(s, sl2x2, negm2, pcol, sum2, bar(FB_PFULL + 4 * g),
                                           DROP ? keep : nullptr);
+        if constexpr (fwd_exp_turns(D)) {
+          __syncwarp();
+          if (lane == 0) exp_busy[warp] = 0;
+        }
         if (offset && g == 0) mbar_arrive(bar(FB_OFFSET));
         float sa, sb, sc2, sd;
         f2_split(sum2[0], sa, sb);
