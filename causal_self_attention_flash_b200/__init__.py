@@ -35,7 +35,8 @@ __all__ = [
     "OK", "ERR_INVALID_ARG", "ERR_UNSUPPORTED", "ERR_CUDA", "ERR_TIMEOUT", "ERR_TOO_LARGE",
     "attn_bwd_noalloc", "NOALLOC_SCRATCH_BYTES",
     "attn_fwd_strided", "attn_bwd_strided", "split_qkv", "CausalAttentionQKV", "Layout",
-    "Dropout", "dropout_params", "attn_decode", "attn_decode_workspace_bytes",
+    "Dropout", "dropout_params", "attn_dropout_mask_bytes", "attn_dropout_mask",
+    "attn_decode", "attn_decode_workspace_bytes",
     "SUPPORTED_HEAD_SIZES", "padded_head_size", "pad_qkv_projection", "pad_out_projection",
 ]
 
@@ -299,12 +300,33 @@ def split_qkv(qkv, n_head):
     return tuple(x.view(B, T, n_head, D).transpose(1, 2) for x in parts)
 
 
-def dropout_params(p, seed=0, offset=0):
+def dropout_params(p, seed=0, offset=0, mask=None):
     """cattn_dropout for drop probability p (0 <= p < 1), a 64-bit seed and
-    a 32-bit counter offset; None for p == 0 (or None)."""
+    a 32-bit counter offset; None for p == 0 (or None).  mask: an optional
+    uint8 device tensor of attn_dropout_mask_bytes(B, H, T) bytes that the
+    forward fills with its keep bits and the backward then reads (see
+    attn_dropout_mask); the tensor must stay alive until the backward."""
     if p is None or p == 0:
         return None
-    return Dropout(float(p), int(seed) & 0xFFFFFFFFFFFFFFFF, int(offset) & 0xFFFFFFFF)
+    ptr = None
+    if mask is not None:
+        if not mask.is_cuda or not mask.is_contiguous() or mask.dtype != torch.uint8:
+            raise ValueError("mask must be a contiguous uint8 device tensor")
+        ptr = mask.data_ptr()
+    return Dropout(float(p), int(seed) & 0xFFFFFFFFFFFFFFFF, int(offset) & 0xFFFFFFFF, ptr)
+
+
+def attn_dropout_mask_bytes(B, H, T):
+    return int(LIB.attn_dropout_mask_bytes(B, H, T))
+
+
+def attn_dropout_mask(B, H, T, device):
+    """A keep-bit cache buffer (uint8, attn_dropout_mask_bytes(B, H, T)
+    bytes) for dropout_params(..., mask=...)."""
+    n = attn_dropout_mask_bytes(B, H, T)
+    if n == 0:
+        raise ValueError("empty or invalid shape")
+    return torch.empty(n, dtype=torch.uint8, device=device)
 
 
 def attn_fwd_strided(q, k, v, scale=None, o=None, lse=None, o_lo=None, stream=None,
@@ -482,7 +504,9 @@ class CausalAttentionQKV(torch.autograd.Function):
     place (attn_fwd_strided / attn_bwd_strided); dqkv comes back as one
     (B, T, 3C) tensor.  apply(qkv, n_head, scale=None, dropout_p=0.0,
     seed=0, offset=0): with dropout_p > 0, attention dropout with the mask
-    of (seed, offset), the same in the backward."""
+    of (seed, offset), the same in the backward: the forward keeps its keep
+    bits in a cache buffer (attn_dropout_mask, 1 bit per element of the
+    causal tiles) that the backward reads instead of drawing them again."""
 
     @staticmethod
     def forward(ctx, qkv, n_head, scale=None, dropout_p=0.0, seed=0, offset=0):
@@ -494,10 +518,11 @@ class CausalAttentionQKV(torch.autograd.Function):
         y_lo = torch.empty_like(y)
         o = y.view(B, T, n_head, D).transpose(1, 2)
         o_lo = y_lo.view(B, T, n_head, D).transpose(1, 2)
-        drop = dropout_params(dropout_p, seed, offset)
+        mask = attn_dropout_mask(B, n_head, T, qkv.device) if dropout_p else None
+        drop = dropout_params(dropout_p, seed, offset, mask)
         _, lse, _ = attn_fwd_strided(q, k, v, scale, o=o, o_lo=o_lo, dropout=drop)
         ctx.save_for_backward(qkv, y, y_lo, lse)
-        ctx.n_head, ctx.scale, ctx.drop = n_head, scale, drop
+        ctx.n_head, ctx.scale, ctx.drop, ctx.mask = n_head, scale, drop, mask
         return y
 
     @staticmethod

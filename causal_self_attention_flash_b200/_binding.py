@@ -32,8 +32,10 @@ class Layout(ctypes.Structure):
 
 
 class Dropout(ctypes.Structure):
-    """cattn_dropout: drop probability p, generator seed and counter offset."""
-    _fields_ = [("p", ctypes.c_float), ("seed", ctypes.c_ulonglong), ("offset", ctypes.c_uint)]
+    """cattn_dropout: drop probability p, generator seed, counter offset and
+    the optional keep-bit cache (device pointer or None)."""
+    _fields_ = [("p", ctypes.c_float), ("seed", ctypes.c_ulonglong), ("offset", ctypes.c_uint),
+                ("mask", ctypes.c_void_p)]
 
 
 # name -> (restype, argtypes), mirroring include/cattn.h
@@ -61,6 +63,7 @@ SIGNATURES = {
     "attn_bwd_dropout": (_i, [_vp, _L, _vp, _L, _vp, _L, _vp, _L, _vp, _vp, _vp, _L, _f,
                               _i, _i, _i, _i, _DP, _vp, _L, _vp, _L, _vp, _L, _i, _vp, _sz, _vp]),
     "attn_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
+    "attn_dropout_mask_bytes": (_sz, [_i, _i, _i]),
     "attn_decode": (_i, [_vp, _L, _vp, _L, _vp, _L, _f, _i, _i, _i, _i, _i, _vp, _L, _vp, _vp,
                          _sz, _vp]),
     "cattn_get_device_status": (_i, [_i, _vp]),

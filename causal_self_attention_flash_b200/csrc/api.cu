@@ -540,9 +540,11 @@ cattn_status bwd_dispatch(bool slo, int dev, const void* q, const void* k, const
 // probability outside [0, 1).  t = 0 (no dropout, p < 2^-17) selects the
 // kernels without the mask, whose result is then the same.
 bool drop_params(const cattn_dropout* d, DropParams* out) {
-  *out = DropParams{0u, 0u, 0u, 0u, 1.f};
+  *out = DropParams{0u, 0u, 0u, 0u, 1.f, nullptr};
   if (d == nullptr) return true;
   if (!(d->p >= 0.f) || !(d->p < 1.f)) return false;
+  if (!aligned(d->mask, 16)) return false;
+  out->mask = static_cast<uint32_t*>(d->mask);
   long t = lrint(static_cast<double>(d->p) * 65536.0);
   if (t > 65535) t = 65535;
   out->t16x = static_cast<uint32_t>(t) << 16;
@@ -659,6 +661,14 @@ cattn_status attn_fwd_ex(const void* q, const void* k, const void* v, float scal
 cattn_status attn_fwd(const void* q, const void* k, const void* v, float scale, int B, int H,
                       int T, int D, void* o, float* lse, void* stream) {
   return attn_fwd_ex(q, k, v, scale, B, H, T, D, o, lse, nullptr, stream);
+}
+
+size_t attn_dropout_mask_bytes(int B, int H, int T) {
+  if (B <= 0 || H <= 0 || T <= 0 || static_cast<long long>(B) * H > 0x7fffffffLL ||
+      T > (1 << 20))
+    return 0;
+  const int n_tiles = (T + 127) / 128;
+  return keep_cache_block(static_cast<long long>(B) * H, n_tiles, 0, 0) * sizeof(uint32_t);
 }
 
 size_t attn_decode_workspace_bytes(int B, int H, int Tq, int L, int D) {

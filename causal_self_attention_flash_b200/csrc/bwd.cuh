@@ -880,7 +880,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // 8s + l%8 (one generator block each); a shuffle per query hands
         // every lane the bit of its own key.
         [[maybe_unused]] uint32_t keepm = 0u;
-        if constexpr (DROP) {
+        if (DROP && p.drop.mask != nullptr) {  // the forward's copy: one word
+          keepm = p.drop.mask[keep_cache_block(bh, p.n_tiles, kt + i, kt) + r * 4 + grp];
+        } else if constexpr (DROP) {
           const uint32_t jg = static_cast<uint32_t>((kt * 128 + quarter * 32) / 8 + (lane >> 3));
           const uint32_t qb = static_cast<uint32_t>((kt + i) * 128 + grp * 32 + (lane & 7));
 #pragma unroll

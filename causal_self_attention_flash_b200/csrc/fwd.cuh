@@ -386,6 +386,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                                     static_cast<uint32_t>(it.bh), p.drop) << (8 * x);
             mask[(2 * g + slot) * 128 + t] = make_uint4(kw[0], kw[1], kw[2], kw[3]);
             mbar_arrive(bar(FB_MFULL + 2 * g + slot));
+            if (p.drop.mask != nullptr)  // the backward's copy
+              store_keep_block(kw, p.drop.mask + keep_cache_block(it.bh, p.n_qtiles, it.tile[g], j),
+                               t >> 5, lane);
             ++mg[g];
           }
         }
@@ -605,6 +608,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             for (int x = 0; x < 4; ++x)
               keep[c4] |= keep_byte(static_cast<uint32_t>(j * 16 + c4 * 4 + x), qi,
                                     static_cast<uint32_t>(it.bh), p.drop) << (8 * x);
+          if (p.drop.mask != nullptr)  // the backward's copy
+            store_keep_block(keep, p.drop.mask + keep_cache_block(it.bh, p.n_qtiles, it.tile[g], j),
+                             quarter, lane);
         }
         wait_warp(w, bar(FB_SFULL + g), tgj & 1, 8);
         tc_fence_after();

@@ -38,7 +38,42 @@ struct DropParams {
   uint32_t k0, k1;  // seed, low and high word
   uint32_t offset;  // counter word 3
   float inv_keep;   // 65536 / (65536 - t)
+  uint32_t* mask;   // the keep bits kept between forward and backward, or null
 };
+
+// Keep-bit cache: one block of 128 x 4 words per (head bh, query tile qt,
+// key tile kt <= qt) of 128 x 128, at block bh * n_pairs + qt (qt + 1) / 2
+// + kt (n_pairs = n_tiles (n_tiles + 1) / 2); word [kr][w] of a block holds
+// bit c = keep bit of query 128 qt + 32 w + c, key 128 kt + kr.  Keys and
+// queries past T hold generator bits too; nothing reads them.  The forward
+// (thread = query row) writes it, the backward (thread = key row) reads one
+// word per 32 queries.
+__host__ __device__ constexpr size_t keep_cache_block(long long bh, int n_tiles, int qt, int kt) {
+  return (static_cast<size_t>(bh) * (static_cast<size_t>(n_tiles) * (n_tiles + 1) / 2) +
+          static_cast<size_t>(qt) * (qt + 1) / 2 + kt) * 512;
+}
+
+// The calling warp holds 32 consecutive query rows (32 w .. 32 w + 31 of a
+// tile), each lane its row's keep bits for 128 keys (bit c of kw[c / 32]);
+// stores them transposed into cache block `blk`: word [kr][w] gets bit
+// `lane` from lane's key kr.  Each 32 x 32 bit block is transposed across
+// the warp in five exchange rounds: at round j the off-diagonal j x j
+// sub-blocks of every 2j x 2j block swap between lanes l and l ^ j.
+__device__ __forceinline__ void store_keep_block(const uint32_t (&kw)[4], uint32_t* blk, int w,
+                                                 int lane) {
+#pragma unroll
+  for (int kb = 0; kb < 4; ++kb) {
+    uint32_t x = kw[kb];
+#pragma unroll
+    for (int j = 16, i = 0; j > 0; j >>= 1, ++i) {
+      const uint32_t m = i == 0 ? 0x0000FFFFu : i == 1 ? 0x00FF00FFu : i == 2 ? 0x0F0F0F0Fu
+                                                : i == 3 ? 0x33333333u : 0x55555555u;
+      const uint32_t y = __shfl_xor_sync(0xffffffffu, x, j);
+      x = (lane & j) ? ((x & ~m) | ((y >> j) & m)) : ((x & m) | ((y & m) << j));
+    }
+    blk[(32 * kb + lane) * 4 + w] = x;
+  }
+}
 
 __device__ __forceinline__ void philox4x32_10(uint32_t& c0, uint32_t& c1, uint32_t& c2,
                                               uint32_t& c3, uint32_t k0, uint32_t k1) {

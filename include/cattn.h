@@ -236,13 +236,31 @@ CATTN_API cattn_status attn_bwd_strided(const void* q, cattn_layout lq, const vo
  *
  * dropout = NULL or p with t = 0 runs the calls without dropout (same
  * results as the _strided calls).  Errors: CATTN_ERR_INVALID_ARG for p
- * outside [0, 1) (NaN included), otherwise as the _strided calls.  The
- * Delta = rowsum(dO * O) of the backward holds with dropout too. */
+ * outside [0, 1) (NaN included) or a mask not 16-byte aligned, otherwise as
+ * the _strided calls.  The Delta = rowsum(dO * O) of the backward holds
+ * with dropout too.
+ *
+ * mask (optional, NULL to draw the bits in both calls): device memory of
+ * attn_dropout_mask_bytes(B, H, T) bytes, 16-byte aligned.  attn_fwd_dropout
+ * then also stores its keep bits there (1 bit per element of every 128 x 128
+ * tile on or below the diagonal, 2 KB per tile, in the order the backward
+ * reads them), and attn_bwd_dropout given the same mask reads them instead
+ * of running the generator again (the generator is most of the backward's
+ * dropout cost).  The results are bit-identical either way.  The caller
+ * owns the buffer; its contents are valid for the backward of the forward
+ * call that wrote them (same q/k/v shape, p, seed and offset), and nothing
+ * checks that: a mask from another call gives wrong gradients. */
 typedef struct {
   float p;                 /* drop probability, 0 <= p < 1 */
   unsigned long long seed; /* generator key */
   unsigned int offset;     /* counter word 3 */
+  void* mask;              /* keep-bit cache between forward and backward, or NULL */
 } cattn_dropout;
+
+/* Bytes of a dropout keep-bit cache for B x H heads of T positions:
+ * B * H * n (n + 1) / 2 * 2048 with n = ceil(T / 128); 0 for an empty or
+ * invalid shape. */
+CATTN_API size_t attn_dropout_mask_bytes(int B, int H, int T);
 
 /* attn_fwd_strided with attention dropout. */
 CATTN_API cattn_status attn_fwd_dropout(const void* q, cattn_layout lq, const void* k,

@@ -334,6 +334,25 @@ def test_decode_checks_arguments_before_the_device():
     assert decode(lay=_binding.Layout(512, 64, 12)) == cattn.ERR_INVALID_ARG
 
 
+def test_dropout_mask_bytes_formula():
+    # 2 KB (128 x 128 bits) per tile on or below the diagonal, per head
+    for B, H, T in [(1, 1, 1), (2, 3, 128), (2, 3, 129), (16, 12, 1024), (1, 2, 8192)]:
+        n = (T + 127) // 128
+        assert cattn.attn_dropout_mask_bytes(B, H, T) == B * H * n * (n + 1) // 2 * 2048
+    assert cattn.attn_dropout_mask_bytes(0, 1, 64) == 0
+    assert cattn.attn_dropout_mask_bytes(1, 1, 0) == 0
+    assert cattn.attn_dropout_mask_bytes(1, 1, (1 << 20) + 1) == 0
+
+
+def test_dropout_mask_alignment_is_checked_before_the_device():
+    c = _binding.Layout(2 * 8 * 64, 8 * 64, 64)
+    d = _binding.Dropout(0.5, 1, 2, ALIGNED + 8)     # not 16-byte aligned
+    assert cattn.LIB.attn_fwd_dropout(ALIGNED, c, ALIGNED, c, ALIGNED, c, 0.125, 1, 2, 8, 64,
+                                      ctypes.byref(d), ALIGNED, c, ALIGNED, None,
+                                      None) == cattn.ERR_INVALID_ARG
+    assert ctypes.sizeof(_binding.Dropout) == 32
+
+
 def test_decode_needs_no_workspace():
     # the CTAs of a head (a thread-block cluster) merge their partial
     # results in distributed shared memory: no workspace for any shape

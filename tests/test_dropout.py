@@ -166,3 +166,63 @@ def test_autograd_qkv_with_dropout(lib):
     check_bf16("dq", as_f64(view(g[..., :C])), rq)
     check_bf16("dk", as_f64(view(g[..., C:2 * C])), rk)
     check_bf16("dv", as_f64(view(g[..., 2 * C:])), rv)
+
+
+def _unpack_mask(buf, B, H, T):
+    """The keep-bit cache as a (B, H, T, T) bool array [query, key]: block
+    bh * n_pairs + qt (qt + 1) / 2 + kt holds words [kr][w], bit c = query
+    128 qt + 32 w + c, key 128 kt + kr (tiles on or below the diagonal)."""
+    n = (T + 127) // 128
+    n_pairs = n * (n + 1) // 2
+    words = buf.view(torch.int32).cpu().numpy().view(np.uint32).reshape(B * H, n_pairs, 128, 4)
+    bits = (words[..., None] >> np.arange(32, dtype=np.uint32)) & 1  # [bh, blk, kr, w, c]
+    full = np.zeros((B * H, n * 128, n * 128), dtype=bool)
+    for qt in range(n):
+        for kt in range(qt + 1):
+            blk = bits[:, qt * (qt + 1) // 2 + kt].reshape(B * H, 128, 128)  # [kr, 32 w + c]
+            full[:, qt * 128:(qt + 1) * 128, kt * 128:(kt + 1) * 128] = blk.transpose(0, 2, 1)
+    return full[:, :T, :T].reshape(B, H, T, T)
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 300, 64), (2, 1, 260, 128), (1, 1, 129, 16)])
+def test_cached_mask_bits_match_oracle(lib, shape):
+    B, H, T, D = shape
+    p, seed, offset = 0.3, SEED, 99
+    q, k, v, _ = bf16_inputs(B, H, T, D, seed=4242 + T, qk_std=1.0)
+    dev = torch.device("cuda:0")
+    q, k, v = (t.to(dev) for t in (q, k, v))
+    mask = lib.attn_dropout_mask(B, H, T, dev)
+    assert mask.numel() == B * H * ((T + 127) // 128) * ((T + 127) // 128 + 1) // 2 * 2048
+    lib.attn_fwd_strided(q, k, v, D ** -0.5, dropout=lib.dropout_params(p, seed, offset, mask))
+    torch.cuda.synchronize()
+    got = _unpack_mask(mask, B, H, T)
+    causal = np.tril(np.ones((T, T), dtype=bool))
+    for b in range(B):
+        for h in range(H):
+            want = odrop.keep_mask_head(b, h, H, T, p, seed, offset)
+            assert np.array_equal(got[b, h] & causal, want & causal), (b, h)
+
+
+@pytest.mark.parametrize("shape", [(2, 3, 129, 32), (1, 2, 260, 128), (2, 2, 1024, 64)])
+@pytest.mark.parametrize("residual", [False, True])
+def test_backward_with_cached_mask_is_bit_identical(lib, shape, residual):
+    B, H, T, D = shape
+    p, seed, offset = 0.2, SEED, 5
+    q, k, v, do = bf16_inputs(B, H, T, D, seed=777 + T + D, qk_std=1.0)
+    dev = torch.device("cuda:0")
+    q, k, v, do = (t.to(dev) for t in (q, k, v, do))
+    scale = D ** -0.5
+    mask = lib.attn_dropout_mask(B, H, T, dev)
+    drawn = lib.dropout_params(p, seed, offset)
+    cached = lib.dropout_params(p, seed, offset, mask)
+    res = []
+    for drop in (drawn, cached):
+        o = torch.empty_like(q)
+        o_lo = torch.empty_like(q) if residual else None
+        _, lse, _ = lib.attn_fwd_strided(q, k, v, scale, o=o, o_lo=o_lo, dropout=drop)
+        res.append((o, lse) + lib.attn_bwd_strided(q, k, v, o, lse, do, scale, o_lo=o_lo,
+                                                   dropout=drop))
+    torch.cuda.synchronize()
+    assert lib.cattn_get_device_status() == lib.OK
+    for a, b in zip(*res):
+        assert torch.equal(a, b)
