@@ -22,10 +22,13 @@ def draw(seed, *shape):
                                          (1, 4, 513, 2, 32), (2, 2, 64, 8, 16), (3, 2, 1000, 4, 64),
                                          (1, 2, 4096, 1, 128), (16, 12, 1024, 1, 64),
                                          (2, 2, 8, 8, 64), (1, 1, 257, 8, 32),
-                                         # many heads: each partial CTA walks
-                                         # several chunks of its head
+                                         # many heads: each warp walks several
+                                         # chunks of its head
                                          (16, 12, 1024, 4, 64), (8, 25, 1024, 8, 64),
-                                         (2, 16, 8192, 2, 128)])
+                                         (2, 16, 8192, 2, 128),
+                                         # clusters of 8 (one head), 5 and 2 CTAs
+                                         (1, 1, 8192, 8, 128), (1, 50, 1000, 3, 64),
+                                         (1, 99, 300, 1, 32)])
 @pytest.mark.parametrize("cache_layout", ["bhtd", "bthd"])
 def test_decode_against_oracle(lib, B, H, L, Tq, D, cache_layout):
     dev = torch.device("cuda:0")

@@ -63,7 +63,9 @@ def from_bits(b: np.ndarray) -> np.ndarray:
     # positions: its partial for those rows is empty (m = -inf)
     (1, 1, 8, 33, 128, 0, None),
     # Tq = L: row 0 sees key 0 only
-    (1, 2, 8, 8, 64, 1, None)])
+    (1, 2, 8, 8, 64, 1, None),
+    # clusters of 5 and 4 CTAs (7 asked for: 8 chunks give runs of 2)
+    (1, 1, 3, 1000, 64, 0, 5), (1, 1, 8, 900, 16, 1, 7)])
 def test_decode_kernels_on_the_host(emu_exe, tmp_path, B, H, Tq, L, D, layout, ctas):
     g = torch.Generator().manual_seed(1000 * L + D + Tq)
     Tmax = L       # a tight cache: a read past row L - 1 leaves the buffer
