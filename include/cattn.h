@@ -125,9 +125,11 @@ CATTN_API cattn_status attn_bwd_preprocess(const void* o, const void* dout,
 /* Backward pass of a scalar loss L with dL/dO = dout:
  *   dV = P^T dO;  dP = dO V^T;  Delta = rowsum(dO * O);
  *   dS = P * (dP - Delta);  dQ = scale dS K;  dK = scale dS^T Q
- * P is recomputed from q, k and lse per key tile (never stored).  P and
- * dS enter the tensor-core products as bf16 hi/lo pairs (about 16
- * significant bits); Delta is computed from the bf16 o given here (use
+ * P is recomputed from q, k and lse per key tile (never stored).  P
+ * enters the dV product as a bf16 hi/lo pair (about 16 significant bits;
+ * with P alone in bf16, dV missed the 2e-2 tolerance), dS enters the dK and
+ * dQ products in bf16 (attn_bwd_ex with o_lo, or fp32 gradients, give dS a
+ * hi/lo pair too); Delta is computed from the bf16 o given here (use
  * attn_bwd_ex with the forward's o_lo for an exact Delta).
  *   q, k, v, o, dout : in, bf16 (B,H,T,D); o and lse as produced by attn_fwd
  *   lse              : in, fp32 (B,H,T)
