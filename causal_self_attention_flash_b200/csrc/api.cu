@@ -434,7 +434,8 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   const int BH = B * H;
   clear_stale_error();
   cattn_status st = ensure_smem(dev, (FLAT ? 32 : 0) + (DROP ? 24 : 8) + 2 * d_index(D) + SLO,
-                                bwd_kernel<D, SLO, DROP, FLAT>, C::SMEM_BYTES);
+                                bwd_kernel<D, SLO, DROP, FLAT>, C::SMEM_BYTES,
+                                C::REBALANCE ? C::LAUNCH_REGS : 0);
   if (st != CATTN_OK) return st;
   const WsLayout L = ws_layout(BH, T, D);
   uint8_t* wb = static_cast<uint8_t*>(ws);

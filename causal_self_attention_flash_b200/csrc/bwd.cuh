@@ -341,6 +341,13 @@ struct BwdCfg {
   static constexpr uint32_t COL_DVL = SPLIT_DV ? 256 + 3 * D : COL_DV;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int THREADS = 640;
+  // Registers: 96 per thread at launch (65536 / 640, rounded down to 8);
+  // setmaxnreg then gives the compute warpgroups REGS_COMP and the fifth
+  // warpgroup (producer and MMA issuers) REGS_OTHER, within the launch total.
+  static constexpr bool REBALANCE = D <= 64 && !SLO;
+  static constexpr int LAUNCH_REGS = 96, REGS_COMP = 104, REGS_OTHER = 64;
+  static_assert(!REBALANCE || 512 * REGS_COMP + 128 * REGS_OTHER <= THREADS * LAUNCH_REGS,
+                "register split exceeds the launch allocation");
   static constexpr int NCOMP = 512;   // compute threads
 };
 
@@ -438,6 +445,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   // Running counters across the CTA's items: t = query tiles processed so
   // far (one per iteration: the phase of the per-iteration barriers and the
   // position in the Q and dO rings), n = items so far (K/V buffer n % KVB).
+  if (warp >= 16) {
+  // fifth warpgroup: the producer and the MMA issuers
+  if constexpr (C::REBALANCE) regs_dec<C::REGS_OTHER>();
   if (warp == 16) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -518,7 +528,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           wait1(wd, bar(BB_DOFULL + j % C::DOST), (j / C::DOST) & 1, 22);
       }
     }
-  } else if (warp >= 17) {
+  } else {
     // -------------------------------------------------- MMA issuers
     // warp 17 (A): S, dP, dQ -- the products that read K and V;
     // warps 18, 19 (B, C): dV, dK -- the accumulations.  One thread issues
@@ -698,7 +708,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       WaitCtx wd{p.timeout_ns, &zero, 2u, false};
       wait1(wd, bar(BB_DRAIN + (warp - 17)), 0, 13);
     }
+  }
   } else {
+    if constexpr (C::REBALANCE) regs_inc<C::REGS_COMP>();
     // ------------------------------------------- compute warps (row = key)
     // Thread (warp w, lane l): key row r = 32*(w%4) + l, query columns
     // [32g, 32g+32) of each tile with g = w/4.  In tensor memory, P^T and
