@@ -138,15 +138,16 @@ struct FwdCfg {
   // (65536 / 384, rounded down to 8); the third warpgroup then drops to
   // REGS_OTHER and the softmax warpgroups rise to REGS_SOFTMAX, within the
   // launch total.  That removed the D = 128 softmax's spills (3.6 % faster
-  // on the long-context workload).  D = 64 takes 200 and 88 (1 % faster
-  // than 168 throughout; 216 and 64 measured 4 % slower); D <= 32 keeps 11
-  // warps and 168 registers.  MASKW adds the keep-bit warpgroup (16
+  // on the long-context workload, at 216 and 64; 208 and 80 measured 2-4 %
+  // faster still, 224 and 48 between them).  D = 64 takes 200 and 88 (1 %
+  // faster than 168 throughout; 208 and 72 the same; 216 and 64 measured
+  // 4 % slower); D <= 32 keeps 11 warps and 168 registers.  MASKW adds the keep-bit warpgroup (16
   // warps): 128 registers at launch, 184 for the softmax, 72 for the rest.
   static constexpr bool REBALANCE = D >= 64 || MASKW;
   static constexpr int THREADS = MASKW ? 512 : REBALANCE ? 384 : 352;
   static constexpr int LAUNCH_REGS = MASKW ? 128 : 168;
-  static constexpr int REGS_SOFTMAX = MASKW ? 184 : D == 128 ? 216 : 200;
-  static constexpr int REGS_OTHER = MASKW ? 72 : D == 128 ? 64 : 88;
+  static constexpr int REGS_SOFTMAX = MASKW ? 184 : D == 128 ? 208 : 200;
+  static constexpr int REGS_OTHER = MASKW ? 72 : D == 128 ? 80 : 88;
   static_assert(!REBALANCE ||
                     256 * REGS_SOFTMAX + (THREADS - 256) * REGS_OTHER <= THREADS * LAUNCH_REGS,
                 "register split exceeds the launch allocation");
