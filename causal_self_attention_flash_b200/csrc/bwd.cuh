@@ -336,6 +336,11 @@ struct BwdCfg {
   // and dK, dQ are issued interleaved.
   static constexpr bool ALIAS_DQ = 256 + 3 * D > 512;
   static constexpr bool SPLIT_DV = 256 + 4 * D <= 512;
+  // CTA-wide dQ staging (D = 128) over the dS hi buffer (HI_BLOCKS blocks)
+  // and the lo buffer: with bf16 dS the dS phase rewrites the hi buffer
+  // only, so it need not wait for the reduce to read the lo part.
+  static constexpr int HI_BLOCKS = 32768 / (128 * RBQ);
+  static constexpr bool STAGE_SPLIT = !WARP_DQ && !SLO && HI_BLOCKS < D / CBQ;
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
   static constexpr uint32_t COL_DQ = ALIAS_DQ ? COL_DP : 256 + 2 * D;
   static constexpr uint32_t COL_DVL = SPLIT_DV ? 256 + 3 * D : COL_DV;
@@ -779,7 +784,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           bulk_commit();
         }
       } else {
-        // staging: blocks of [128 rows][CBQ floats], swizzled
+        // staging: blocks of [128 rows][CBQ floats], swizzled.  The
+        // previous drain's reduce may still be reading its second group
+        // (the blocks in the dS lo buffer, see staging_free): wait for it.
+        if constexpr (C::STAGE_SPLIT) {
+          if (leader) bulk_wait_read0();
+          named_bar_sync(1, C::NCOMP);
+        }
 #pragma unroll
         for (int e = 0; e < NQ; e += 4) {
           const int f = grp * NQ + e;
@@ -799,18 +810,31 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // backward.
         named_bar_sync(1, C::NCOMP);
         if (leader && !*abort_flag) {
+          // two commit groups: the blocks in the dS hi buffer, then the rest
+          // (STAGE_SPLIT: the next dS phase waits for the first only)
+          constexpr int NB = D / C::CBQ, NH = C::STAGE_SPLIT ? C::HI_BLOCKS : NB;
 #pragma unroll
-          for (int blk = 0; blk < D / C::CBQ; ++blk)
+          for (int blk = 0; blk < NH; ++blk)
             tma_reduce_add_3d(&tmDQacc, sDSH + blk * 128 * C::RBQ, blk * C::CBQ, q0, bh);
           bulk_commit();
+          if constexpr (NH < NB) {
+#pragma unroll
+            for (int blk = NH; blk < NB; ++blk)
+              tma_reduce_add_3d(&tmDQacc, sDSH + blk * 128 * C::RBQ, blk * C::CBQ, q0, bh);
+            bulk_commit();
+          }
         }
       }
     };
     // the dS buffers may be rewritten once the reduce has read them (CTA
-    // staging only)
+    // staging only; STAGE_SPLIT: the dS phase writes the hi buffer only, so
+    // it waits for the first commit group, and the next drain for the rest)
     auto staging_free = [&]() {
       if constexpr (!C::WARP_DQ) {
-        if (leader) bulk_wait_read0();
+        if (leader) {
+          if constexpr (C::STAGE_SPLIT) bulk_wait_read1();
+          else bulk_wait_read0();
+        }
         named_bar_sync(1, C::NCOMP);
       }
     };
