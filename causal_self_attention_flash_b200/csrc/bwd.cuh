@@ -341,6 +341,13 @@ struct BwdCfg {
   // only, so it need not wait for the reduce to read the lo part.
   static constexpr int HI_BLOCKS = 32768 / (128 * RBQ);
   static constexpr bool STAGE_SPLIT = !WARP_DQ && !SLO && HI_BLOCKS < D / CBQ;
+  // DK_SMEM (D = 128, bf16 dS): dK takes dS^T from the shared-memory copy
+  // of dS that the dQ product reads (the [2][128 keys][64 queries] 128-byte
+  // swizzled blocks are dS^T in K-major order), so the compute warps store
+  // dS to shared memory only, and dQ (whose TMEM columns are dP^T's) need
+  // not wait for dK; the CTA-wide staging then waits for dK before it
+  // overwrites the dS blocks.
+  static constexpr bool DK_SMEM = !WARP_DQ && !SLO;
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
   static constexpr uint32_t COL_DQ = ALIAS_DQ ? COL_DP : 256 + 2 * D;
   static constexpr uint32_t COL_DVL = SPLIT_DV ? 256 + 3 * D : COL_DV;
@@ -568,7 +575,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           wait1(w, bar(BB_DOFULL + ds), (t / C::DOST) & 1, 5);
           // dP overwrites dS^T(t-1), which dK(t-1) reads, and, aliased,
           // dQ(t-1), which the compute warps must have drained
-          if (t >= 1) wait1(w, bar(BB_DKDONE), (t - 1) & 1, 25);
+          // (DK_SMEM: dS^T(t-1) is not in TMEM; the compute warps loaded
+          // dP^T(t-1) before draining dQ(t-1), which the wait below covers)
+          if (!C::DK_SMEM && t >= 1) wait1(w, bar(BB_DKDONE), (t - 1) & 1, 25);
           if (C::ALIAS_DQ && t >= 1) wait1(w, bar(BB_DQEMPTY), (t - 1) & 1, 12);
           tc_fence_after();
           const uint32_t sDO = sbase + C::OFF_DO + ds * C::TILE_BYTES;
@@ -613,7 +622,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             // dQ_t = dS K (A = dS hi/lo in shared, MN-major; K = 128 keys)
             wait1(w, bar(BB_DSFULL), t & 1, 9);
             if (!C::ALIAS_DQ && t >= 1) wait1(w, bar(BB_DQEMPTY), (t - 1) & 1, 10);
-            if (C::ALIAS_DQ) wait1(w, bar(BB_DKDONE), t & 1, 26);  // dQ overwrites dS^T
+            if (C::ALIAS_DQ && !C::DK_SMEM)
+              wait1(w, bar(BB_DKDONE), t & 1, 26);  // dQ overwrites dS^T
             tc_fence_after();
             {
               const uint64_t dkk = smem_desc(sK(n % C::KVB), C::BLOCK_BYTES, 8 * C::RB, C::SW);
@@ -688,19 +698,27 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             mma_commit(bar(BB_PTDONE));
             mma_commit(bar(BB_DOEMPTY + ds));  // one of the slot's releases
             if (lo_role) continue;
-            // dK += dS^T Q_t (A = dS^T hi/lo in TMEM over dP^T)
+            // dK += dS^T Q_t (A = dS^T hi/lo in TMEM over dP^T; DK_SMEM: A =
+            // the shared dS hi blocks, K-major, 16 queries = 32 bytes a step)
             wait1(w, bar(BB_DSFULL), t & 1, 9);
             wait1(w, bar(BB_QFULL + qs), (t / C::QST) & 1, 28);  // (visibility)
             tc_fence_after();
             const uint64_t dqq = smem_desc(sQ, C::BLOCK_BYTES, 8 * C::RB, C::SW);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t acol = C::COL_DP + (kk >> 1) * 32 + (kk & 1) * 8;
-              mma_ts(tbase + C::COL_DK, tbase + acol, dqq + ((kk * 16 * C::RB) >> 4), idKD,
-                     (i > 0 || kk > 0) ? 1u : 0u);
-              if (SLO)
-                mma_ts(tbase + C::COL_DK, tbase + acol + 16, dqq + ((kk * 16 * C::RB) >> 4), idKD,
-                       1u);
+              const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+              if constexpr (C::DK_SMEM) {
+                const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
+                mma_ss(tbase + C::COL_DK, smem_desc(sDSH + aoff, 16, 1024, 2),
+                       dqq + ((kk * 16 * C::RB) >> 4), idKD, acc);
+              } else {
+                const uint32_t acol = C::COL_DP + (kk >> 1) * 32 + (kk & 1) * 8;
+                mma_ts(tbase + C::COL_DK, tbase + acol, dqq + ((kk * 16 * C::RB) >> 4), idKD,
+                       acc);
+                if (SLO)
+                  mma_ts(tbase + C::COL_DK, tbase + acol + 16, dqq + ((kk * 16 * C::RB) >> 4),
+                         idKD, 1u);
+              }
             }
             mma_commit(bar(BB_DKDONE));
             mma_commit(bar(BB_QEMPTY + qs));  // S(t), which also read Q_t, completed long ago
@@ -787,6 +805,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // staging: blocks of [128 rows][CBQ floats], swizzled.  The
         // previous drain's reduce may still be reading its second group
         // (the blocks in the dS lo buffer, see staging_free): wait for it.
+        if constexpr (C::DK_SMEM) {  // dK(t) reads the dS blocks the staging overwrites
+          wait_warp(w, bar(BB_DKDONE), t & 1, 34);
+          tc_fence_after();
+        }
         if constexpr (C::STAGE_SPLIT) {
           if (leader) bulk_wait_read0();
           named_bar_sync(1, C::NCOMP);
@@ -1035,8 +1057,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             }
           }
         }
-        tmem_st16(tbase + lane_base + C::COL_DP + grp * 32, hi);
-        if (SLO) tmem_st16(tbase + lane_base + C::COL_DP + grp * 32 + 16, lo);
+        if constexpr (!C::DK_SMEM) {
+          tmem_st16(tbase + lane_base + C::COL_DP + grp * 32, hi);
+          if (SLO) tmem_st16(tbase + lane_base + C::COL_DP + grp * 32 + 16, lo);
+        }
         // dS (hi, lo) -> shared for the dQ MMA: [2][128 keys][64 queries];
         // query block g is half g/2, chunks 4*(g%2) .. +3 of the row.  (dQ(t-1),
         // which read the previous dS, is complete: drained above.)
@@ -1054,7 +1078,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             st_shared_v4(sDSL + off, lo[4 * ch], lo[4 * ch + 1], lo[4 * ch + 2], lo[4 * ch + 3]);
         }
         fence_async_smem();
-        tmem_wait_st();
+        if constexpr (!C::DK_SMEM) tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(BB_DSFULL));
         // ---- kLateDrain: the previous query tile's dQ, while the next S is
