@@ -236,11 +236,12 @@ __global__ void __launch_bounds__(256) dq_convert_strided_kernel(const float4* _
 //   P^T  = exp2(S^T*scale*log2e - LSE2_i); masked on the diagonal tile;
 //          written back over S^T as bf16 hi/lo pairs
 //   dP^T = V_j dO_i^T              (TMEM, fp32)
-//   dS^T = P^T * (dP^T - Delta_i); written back over dP^T as hi/lo pairs,
-//          and (as dS) to shared memory for the dQ MMA
+//   dS^T = P^T * (dP^T - Delta_i); written back over dP^T (bf16, or hi/lo
+//          pairs), and (as dS) to shared memory for the dQ MMA
 //   dV  += P^T_hi dO_i + P^T_lo dO_i        (A from TMEM)
-//   dK  += dS^T_hi Q_i + dS^T_lo Q_i        (A from TMEM)
-//   dQ_i = dS_hi K_j + dS_lo K_j            (A from shared, MN-major),
+//   dK  += dS^T_hi Q_i (+ dS^T_lo Q_i)      (A from TMEM; DK_SMEM: from the
+//                                            shared dS, K-major)
+//   dQ_i = dS_hi K_j (+ dS_lo K_j)          (A from shared, MN-major),
 //          drained to shared memory and added into the fp32 accumulator
 //          with a TMA reduce-add.
 //
@@ -254,7 +255,8 @@ __global__ void __launch_bounds__(256) dq_convert_strided_kernel(const float4* _
 //              through a 2-stage ring, dO_t through a 2-stage (D <= 64) or
 //              1-stage ring, both running on across items.
 //   warp 17    MMA issuer A and TMEM owner: S(t+1) as soon as dV(t) has read
-//              P^T(t), dQ(t), dP(t+1) once dK(t) has read dS^T(t).
+//              P^T(t), dQ(t), dP(t+1) once dK(t) has read dS^T(t) (and, with
+//              dQ in dP^T's columns, once dQ(t) has been drained).
 //   warp 18    MMA issuer B: dV(t) (P^T_hi part), dK(t).
 //   warp 19    MMA issuer C: the P^T_lo part of dV(t), into dV' (where TMEM
 //              holds a separate dV' accumulator; otherwise warp 18 does it).
