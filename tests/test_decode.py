@@ -80,3 +80,28 @@ def test_decode_argument_errors(lib):
     ws = torch.empty(0, dtype=torch.uint8, device=dev)
     lib.attn_decode(q[:, :, :1], k, k, 16, workspace=ws)
     torch.cuda.synchronize()
+
+
+def test_decode_strided_query_and_output(lib):
+    """q and o as (B, Tq, H, D) storage seen as (B, H, Tq, D) views (the
+    layout of a fused projection's rows), the cache (B, Tmax, H, D): every
+    stride of the call differs from the contiguous one."""
+    B, H, Tq, L, D = 3, 5, 6, 700, 64
+    dev = torch.device("cuda:0")
+    Tmax = L + 5
+    qs = draw(31, B, Tq, H, D)
+    ks = draw(32, B, Tmax, H, D)
+    vs = draw(33, B, Tmax, H, D)
+    q = qs.to(dev).transpose(1, 2)
+    k = ks.to(dev).transpose(1, 2)
+    v = vs.to(dev).transpose(1, 2)
+    o_store = torch.full((B, Tq, H, D), float("nan"), dtype=torch.bfloat16, device=dev)
+    o = o_store.transpose(1, 2)
+    scale = D ** -0.5
+    o2, lse = lib.attn_decode(q, k, v, L, scale, o=o)
+    torch.cuda.synchronize()
+    assert o2.data_ptr() == o.data_ptr()
+    ro, rl = odec.decode_attention(as_f64(qs.transpose(1, 2)), as_f64(ks.transpose(1, 2)),
+                                   as_f64(vs.transpose(1, 2)), scale, L)
+    check_bf16("o", as_f64(o), ro)
+    check_lse(as_f64(lse), rl)
