@@ -36,16 +36,19 @@ side implements the same generator on its own; the two agree because both
 follow the definition, which published known-answer vectors pin
 (tests/golden/philox4x32_10_kat.txt).
 
-Element (b, h, i, j) of the mask (query i, key j) takes its 16 bits from
-the Philox block with
+Element (b, h, i, j) of the mask (query i, key j) takes 8 random bits
+from the Philox block with
 
-    counter = (j >> 3, i, b * H + h, offset),   key = (seed low 32, seed high 32)
+    counter = (j >> 4, i, b * H + h, offset),   key = (seed low 32, seed high 32)
 
-word (j & 7) >> 1, half j & 1 (low 16 bits for even j).  The element is
-dropped iff those 16 bits, as an unsigned integer, are below
-t = round(p * 65536); so the drop probability is t / 65536 (p to within
-2^-17) and the kept values are scaled by 65536 / (65536 - t), which makes
-E[P~] = P exactly.
+namely byte j & 3 (bits 8 (j & 3) .. 8 (j & 3) + 7) of output word
+(j & 15) >> 2.  The element is dropped iff that byte, as an unsigned
+integer, is below t = round(p * 256); so the drop probability is t / 256
+(p to within 2^-9) and the kept values are scaled by 256 / (256 - t),
+which makes E[P~] = P exactly.  The pages fix the rate, not how finely it
+is drawn: 8 bits per element is the reading taken here (flash-attention's
+own dropout also draws 8 bits per element), one generator block per 16
+elements.
 """
 
 from __future__ import annotations
@@ -87,37 +90,37 @@ def philox4x32_10(ctr, key):
 
 
 def drop_threshold(p: float) -> int:
-    """t = round(p * 65536) for 0 <= p < 1 (at most 65535)."""
+    """t = round(p * 256) for 0 <= p < 1 (at most 255)."""
     if not 0.0 <= p < 1.0:
         raise ValueError("dropout probability must be in [0, 1)")
-    return min(int(np.rint(p * 65536.0)), 65535)
+    return min(int(np.rint(p * 256.0)), 255)
 
 
 def keep_scale(p: float) -> float:
-    """The factor kept probabilities are multiplied by: 1 / (1 - t/65536)."""
+    """The factor kept probabilities are multiplied by: 1 / (1 - t/256)."""
     t = drop_threshold(p)
-    return 65536.0 / (65536.0 - t)
+    return 256.0 / (256.0 - t)
 
 
-def random16(b, h, H, i, j, seed: int, offset: int):
-    """The 16 random bits of mask element(s) (b, h, i, j); i and j may be
+def random8(b, h, H, i, j, seed: int, offset: int):
+    """The 8 random bits of mask element(s) (b, h, i, j); i and j may be
     broadcastable integer arrays."""
     i = np.asarray(i, dtype=np.uint64)
     j = np.asarray(j, dtype=np.uint64)
     i, j = np.broadcast_arrays(i, j)
-    ctr = np.stack([j >> np.uint64(3), i,
+    ctr = np.stack([j >> np.uint64(4), i,
                     np.full(i.shape, b * H + h, dtype=np.uint64),
                     np.full(i.shape, offset & MASK32, dtype=np.uint64)], axis=-1)
     out = philox4x32_10(ctr, (seed & MASK32, (seed >> 32) & MASK32))
-    word = np.take_along_axis(out, ((j & np.uint64(7)) >> np.uint64(1)).astype(np.int64)[..., None],
+    word = np.take_along_axis(out, ((j & np.uint64(15)) >> np.uint64(2)).astype(np.int64)[..., None],
                               axis=-1)[..., 0]
-    return (word >> (np.uint64(16) * (j & np.uint64(1)))) & np.uint64(0xFFFF)
+    return (word >> (np.uint64(8) * (j & np.uint64(3)))) & np.uint64(0xFF)
 
 
 def keep_mask_head(b, h, H, T, p: float, seed: int, offset: int):
     """Boolean (T, T) keep mask of head (b, h): True where kept (the future
     half is returned too, though it never matters)."""
-    r = random16(b, h, H, np.arange(T)[:, None], np.arange(T)[None, :], seed, offset)
+    r = random8(b, h, H, np.arange(T)[:, None], np.arange(T)[None, :], seed, offset)
     return r >= np.uint64(drop_threshold(p))
 
 

@@ -4,10 +4,11 @@
   vectors (tests/golden/philox4x32_10_kat.txt).
 * The mask: drop rate and pair statistics at the requested probability,
   determinism, dependence on seed and offset, and the documented placement
-  of each element's 16 bits in the Philox blocks.
+  of each element's 8 bits in the Philox blocks.
 * The arithmetic: p = 0 reduces exactly to the dropout-free oracle; the
   dropout output is unbiased (its mean over many masks is the dropout-free
-  output, which pins the keep scale); central finite differences of
+  output) and the keep scale is exactly 1 / the keep probability of the
+  8-bit draw; central finite differences of
   L = <O, dO> with the mask held fixed match the backward.
 * Planted mistakes in a copy of the module are each caught by some pin.
 """
@@ -33,7 +34,7 @@ def _rand(seed, B, H, T, D, std=1.0):
 
 def _impl(mod=drop_mod):
     return types.SimpleNamespace(
-        philox=mod.philox4x32_10, mask=mod.keep_mask_head, r16=mod.random16,
+        philox=mod.philox4x32_10, mask=mod.keep_mask_head, r8=mod.random8,
         fwd=mod.attention_forward_dropout, bwd=mod.attention_backward_dropout,
         ks=mod.keep_scale)
 
@@ -52,10 +53,10 @@ def pin_kat(impl):
 
 def pin_drop_rate(impl):
     T = 1024
-    for p in (0.2, 0.5):
+    for p in (0.1, 0.2, 0.5):  # 0.1 is 25.6 / 256: rounded, not truncated
         m = impl.mask(1, 2, 3, T, p, 0x1234_5678_9ABC_DEF0, 7)
         n = T * T
-        t = round(p * 65536) / 65536
+        t = round(p * 256) / 256
         drop = 1.0 - m.mean()
         sigma = np.sqrt(t * (1 - t) / n)
         assert abs(drop - t) < 5 * sigma, (p, drop)
@@ -65,13 +66,14 @@ def pin_drop_rate(impl):
 
 
 def pin_uniform_bits(impl):
-    """the 16-bit values are uniform: chi-square over the 256 values of
-    the high byte and of the low byte."""
+    """the 8-bit values are uniform: chi-square over their 256 values, for
+    all keys and for each of the four byte positions j & 3 alone."""
     T = 512
-    r = impl.r16(0, 0, 1, np.arange(T)[:, None], np.arange(T)[None, :], 99, 3).ravel()
-    for byte in (r >> np.uint64(8), r & np.uint64(255)):
-        counts = np.bincount(byte.astype(np.int64), minlength=256)
-        e = r.size / 256
+    r = impl.r8(0, 0, 1, np.arange(T)[:, None], np.arange(T)[None, :], 99, 3)
+    for sel in (r.ravel(), r[:, 0::4].ravel(), r[:, 1::4].ravel(), r[:, 2::4].ravel(),
+                r[:, 3::4].ravel()):
+        counts = np.bincount(sel.astype(np.int64), minlength=256)
+        e = sel.size / 256
         chi2 = ((counts - e) ** 2 / e).sum()
         assert 160 < chi2 < 370, chi2     # 255 degrees of freedom, beyond 4.5 sigma
 
@@ -88,18 +90,18 @@ def pin_stream_separation(impl):
 
 
 def pin_bit_placement(impl):
-    """element (b, h, i, j): word (j & 7) >> 1, half j & 1 of the block with
-    counter (j >> 3, i, b*H + h, offset) and key (seed low, seed high)."""
+    """element (b, h, i, j): word (j & 15) >> 2, byte j & 3 of the block
+    with counter (j >> 4, i, b*H + h, offset) and key (seed low, seed high)."""
     seed, offset, H = 0xDEADBEEF_01234567, 11, 5
     for b, h, i, j in ((0, 0, 0, 0), (1, 2, 5, 13), (3, 4, 1000, 999), (0, 3, 77, 64)):
-        blk = impl.philox(np.array([j >> 3, i, b * H + h, offset]),
+        blk = impl.philox(np.array([j >> 4, i, b * H + h, offset]),
                           (seed & 0xFFFFFFFF, seed >> 32))
-        want = (int(blk[(j & 7) >> 1]) >> (16 * (j & 1))) & 0xFFFF
-        assert int(impl.r16(b, h, H, i, j, seed, offset)) == want
-        # dropped iff the 16 bits are below round(p * 65536)
+        want = (int(blk[(j & 15) >> 2]) >> (8 * (j & 3))) & 0xFF
+        assert int(impl.r8(b, h, H, i, j, seed, offset)) == want
+        # dropped iff the 8 bits are below round(p * 256)
         for pr in (0.1, 0.5, 0.9):
             m = impl.mask(b, h, H, max(i, j) + 1, pr, seed, offset)
-            assert bool(m[i, j]) == (want >= round(pr * 65536)), (b, h, i, j, pr)
+            assert bool(m[i, j]) == (want >= round(pr * 256)), (b, h, i, j, pr)
 
 
 def pin_p_zero(impl):
@@ -122,6 +124,20 @@ def pin_unbiased(impl):
     mean, sd = outs.mean(0), outs.std(0)
     z = np.abs(mean - ref) / (sd / np.sqrt(n) + 1e-12)
     assert z.max() < 6.0, z.max()
+
+
+def pin_exact_keep_scale(impl):
+    """the keep scale times the exact keep probability is 1: the byte is
+    uniform over 256 values, so with the threshold t read off the mask
+    (the smallest kept byte, the largest dropped one plus 1) the keep
+    probability is (256 - t) / 256."""
+    T = 256
+    r = impl.r8(0, 1, 2, np.arange(T)[:, None], np.arange(T)[None, :], 5, 6)
+    for p in (0.1, 0.3, 0.77):
+        m = impl.mask(0, 1, 2, T, p, 5, 6)
+        t = int(r[m].min())
+        assert t == int(r[~m].max()) + 1, p
+        assert abs(impl.ks(p) * (256 - t) / 256 - 1.0) < 1e-12, (p, t, impl.ks(p))
 
 
 def pin_finite_differences(impl):
@@ -155,8 +171,8 @@ def pin_lse_unchanged(impl):
 
 
 ALL_PINS = [pin_kat, pin_drop_rate, pin_uniform_bits, pin_stream_separation,
-            pin_bit_placement, pin_p_zero, pin_unbiased, pin_finite_differences,
-            pin_lse_unchanged]
+            pin_bit_placement, pin_p_zero, pin_unbiased, pin_exact_keep_scale,
+            pin_finite_differences, pin_lse_unchanged]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
@@ -165,9 +181,12 @@ def test_pin_holds(pin):
 
 
 def test_threshold_and_scale():
-    assert drop_mod.drop_threshold(0.2) == 13107
+    assert drop_mod.drop_threshold(0.2) == 51
+    assert drop_mod.drop_threshold(0.1) == 26
     assert drop_mod.drop_threshold(0.0) == 0
-    assert drop_mod.drop_threshold(0.99999999) == 65535
+    assert drop_mod.drop_threshold(0.001) == 0
+    assert drop_mod.drop_threshold(0.99999999) == 255
+    assert drop_mod.keep_scale(0.2) == 256.0 / 205.0
     assert drop_mod.keep_scale(0.5) == 2.0
     with pytest.raises(ValueError):
         drop_mod.drop_threshold(1.0)
@@ -181,14 +200,19 @@ MUTANTS = [
     ("key not bumped", "k1 = (k1 + PHILOX_W1) & MASK32", "k1 = k1"),
     ("nine rounds", "for rnd in range(10):", "for rnd in range(9):"),
     ("output words swapped", "hi0 ^ c3 ^ np.uint64(k1), lo0)", "lo0, hi0 ^ c3 ^ np.uint64(k1))"),
-    ("word chosen by j & 3", "((j & np.uint64(7)) >> np.uint64(1))", "(j & np.uint64(3))"),
-    ("high half for even keys", "(np.uint64(16) * (j & np.uint64(1)))",
-     "(np.uint64(16) * (np.uint64(1) - (j & np.uint64(1))))"),
-    ("counter words i and j swapped", "ctr = np.stack([j >> np.uint64(3), i,",
-     "ctr = np.stack([i >> np.uint64(3), j,"),
+    ("word chosen by j & 3", "((j & np.uint64(15)) >> np.uint64(2))", "(j & np.uint64(3))"),
+    ("bytes taken high first", "(np.uint64(8) * (j & np.uint64(3)))",
+     "(np.uint64(8) * (np.uint64(3) - (j & np.uint64(3))))"),
+    ("16 keys per block, counter j >> 3", "ctr = np.stack([j >> np.uint64(4), i,",
+     "ctr = np.stack([j >> np.uint64(3), i,"),
+    ("counter words i and j swapped", "ctr = np.stack([j >> np.uint64(4), i,",
+     "ctr = np.stack([i >> np.uint64(4), j,"),
+    ("seven bits drawn", "& np.uint64(0xFF)", "& np.uint64(0x7F)"),
     ("keep where below the threshold", "return r >= np.uint64(drop_threshold(p))",
-     "return r < np.uint64(65536 - drop_threshold(p))"),
-    ("keep scale 1/p", "return 65536.0 / (65536.0 - t)", "return 65536.0 / max(t, 1)"),
+     "return r < np.uint64(256 - drop_threshold(p))"),
+    ("threshold truncated", "min(int(np.rint(p * 256.0)), 255)", "min(int(p * 256.0), 255)"),
+    ("keep scale 1/p", "return 256.0 / (256.0 - t)", "return 256.0 / max(t, 1)"),
+    ("keep scale from the unrounded p", "return 256.0 / (256.0 - t)", "return 1.0 / (1.0 - p)"),
     ("no rescale in the forward", "o[b, h] = (pr * m * ks) @ v[b, h]", "o[b, h] = (pr * m) @ v[b, h]"),
     ("dP without the mask", "dp = dpd * m * ks", "dp = dpd * ks"),
     ("dP without the keep scale", "dp = dpd * m * ks", "dp = dpd * m"),
