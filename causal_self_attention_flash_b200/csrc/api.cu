@@ -526,7 +526,7 @@ cattn_status bwd_dispatch(bool slo, int dev, const void* q, const void* k, const
   const bool flat = collapses(ly.q, H) && collapses(ly.k, H) && collapses(ly.v, H) &&
                     collapses(ly.dout, H) && collapses(ly.dk, H) && collapses(ly.dv, H);
   // one instance per (SLO, DROP, FLAT); each line picks exactly one
-  const bool drop = dp.t16x != 0;
+  const bool drop = dp.t != 0;
 #define CATTN_BWD(SS, DR, FL) \
   bwd_impl<D, SS, DR, FL>(dev, q, k, v, o, o_lo, lse, dout, scale, B, H, T, dq, dk, dv, ly, f32, ws, dp, s)
   if (slo && drop) return flat ? CATTN_BWD(true, true, true) : CATTN_BWD(true, true, false);
@@ -536,23 +536,25 @@ cattn_status bwd_dispatch(bool slo, int dev, const void* q, const void* k, const
 #undef CATTN_BWD
 }
 
-// Dropout parameters of a call: t = round(p * 65536) (the drop threshold on
-// 16 random bits), 1 / (1 - t / 65536) as the keep scale; false for a
-// probability outside [0, 1).  t = 0 (no dropout, p < 2^-17) selects the
+// Dropout parameters of a call: t = round(p * 256) (the drop threshold on
+// 8 random bits), 1 / (1 - t / 256) as the keep scale; false for a
+// probability outside [0, 1).  t = 0 (no dropout, p < 2^-9) selects the
 // kernels without the mask, whose result is then the same.
 bool drop_params(const cattn_dropout* d, DropParams* out) {
-  *out = DropParams{0u, 0u, 0u, 0u, 1.f, nullptr};
+  *out = DropParams{};
   if (d == nullptr) return true;
   if (!(d->p >= 0.f) || !(d->p < 1.f)) return false;
   if (!aligned(d->mask, 16)) return false;
   out->mask = static_cast<uint32_t*>(d->mask);
-  long t = lrint(static_cast<double>(d->p) * 65536.0);
-  if (t > 65535) t = 65535;
-  out->t16x = static_cast<uint32_t>(t) << 16;
-  out->k0 = static_cast<uint32_t>(d->seed & 0xffffffffull);
-  out->k1 = static_cast<uint32_t>(d->seed >> 32);
+  long t = lrint(static_cast<double>(d->p) * 256.0);
+  if (t > 255) t = 255;
+  out->t = static_cast<uint32_t>(t);
+  out->t_lo = (out->t & 0x7Fu) * 0x01010101u;
+  out->t_maj = out->t < 128u ? 0xFFFFFFFFu : 0u;
+  philox_round_keys(static_cast<uint32_t>(d->seed & 0xffffffffull),
+                    static_cast<uint32_t>(d->seed >> 32), out->rk);
   out->offset = d->offset;
-  out->inv_keep = static_cast<float>(65536.0 / (65536.0 - static_cast<double>(t)));
+  out->inv_keep = static_cast<float>(256.0 / (256.0 - static_cast<double>(t)));
   return true;
 }
 
@@ -635,7 +637,7 @@ cattn_status attn_fwd_dropout(const void* q, cattn_layout lq, const void* k, cat
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // FLAT: q, k, v and o all collapse to one b*H + h axis (see bwd_dispatch)
   const bool flat = collapses(lq, H) && collapses(lk, H) && collapses(lv, H) && collapses(lo, H);
-  const bool plo = o_lo != nullptr, drop = dp.t16x != 0;
+  const bool plo = o_lo != nullptr, drop = dp.t != 0;
   switch (D) {
     case 16: return fwd_dispatch<16>(plo, drop, flat, dev, q, lq, k, lk, v, lv, scale, B, H, T, o, lo, lse, o_lo, dp, s);
     case 32: return fwd_dispatch<32>(plo, drop, flat, dev, q, lq, k, lk, v, lv, scale, B, H, T, o, lo, lse, o_lo, dp, s);
@@ -863,7 +865,7 @@ cattn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const
   // the backward clears what must start at zero (the dQ accumulator) and
   // overwrites the rest on every call
   const BwdLayouts ly = contiguous_bwd_layouts(H, T, D);
-  const DropParams no_drop{0u, 0u, 0u, 0u, 1.f};
+  const DropParams no_drop{};
   switch (D) {
     case 16:
       return bwd_impl<16, false, false, true>(dev, q, k, v, o, nullptr, lse, dout, scale, B, H, T, dq, dk,

@@ -934,26 +934,20 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       const int n_iter = p.n_tiles - kt;
       for (int i = 0; i < n_iter; ++i, ++t) {
         const int qs = t % C::QST;
-        // ---- dropout keep bits (DROP), while S is on its way: bit c of
-        // keepm is this key row's bit for query column 32g + c.  Lane l
-        // draws the bits of keys 8*(l/8) .. +7 of its warp for query
-        // 8s + l%8 (one generator block each); a shuffle per query hands
-        // every lane the bit of its own key.
+        // ---- dropout keep bits (DROP), while S is on its way: bit
+        // il_pos(c) of keepm is this key row's bit for query column 32g + c.
+        // Lane l draws query 32g + il_key(l)'s bits for the warp's 32 keys
+        // (two generator blocks), and a 32 x 32 warp transpose hands every
+        // lane its own key's bits for the 32 queries.
         [[maybe_unused]] uint32_t keepm = 0u;
         if (DROP && p.drop.mask != nullptr) {  // the forward's copy: one word
           keepm = p.drop.mask[keep_cache_block(bh, p.n_tiles, kt + i, kt) + r * 4 + grp];
         } else if constexpr (DROP) {
-          const uint32_t jg = static_cast<uint32_t>((kt * 128 + quarter * 32) / 8 + (lane >> 3));
-          const uint32_t qb = static_cast<uint32_t>((kt + i) * 128 + grp * 32 + (lane & 7));
-#pragma unroll
-          for (int s8 = 0; s8 < 4; ++s8) {
-            const uint32_t byte = keep_byte(jg, qb + 8 * s8, static_cast<uint32_t>(bh), p.drop);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const uint32_t v8 = __shfl_sync(0xffffffffu, byte, (lane & ~7) | q);
-              keepm |= ((v8 >> (lane & 7)) & 1u) << (8 * s8 + q);
-            }
-          }
+          const uint32_t jg = static_cast<uint32_t>((kt * 128 + quarter * 32) / 16);
+          const uint32_t qi = static_cast<uint32_t>((kt + i) * 128 + grp * 32 + il_key(lane));
+          const uint32_t bhu = static_cast<uint32_t>(bh);
+          keepm = warp_transpose32(keep16(jg, qi, bhu, p.drop) | keep16(jg + 1, qi, bhu, p.drop) << 16,
+                                   lane);
         }
         // ---- P phase
         wait_warp(w, bar(BB_SFULL), t & 1, 15);
@@ -990,17 +984,15 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
               if (c < lim) pv[c] = 0.f;
           }
           uint32_t hi[8], lo[8];
-          if constexpr (DROP) {  // dV takes the dropped P (scaled in the epilogue)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float a0 = ((keepm >> (16 * h + 2 * e)) & 1u) ? pv[16 * h + 2 * e] : 0.f;
-              const float a1 = ((keepm >> (16 * h + 2 * e + 1)) & 1u) ? pv[16 * h + 2 * e + 1] : 0.f;
-              split_bf16x2_p(f2(a0, a1), hi[e], lo[e]);
+          for (int e = 0; e < 8; ++e) {
+            split_bf16x2_p(f2(pv[16 * h + 2 * e], pv[16 * h + 2 * e + 1]), hi[e], lo[e]);
+            if constexpr (DROP) {  // dV takes the dropped P (scaled in the epilogue)
+              const uint32_t m =
+                  prmt_sign(keepm << (7 - 4 * h - (e >> 1)), (e & 1) ? 0xBBAAu : 0x9988u);
+              hi[e] &= m;
+              lo[e] &= m;
             }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              split_bf16x2_p(f2(pv[16 * h + 2 * e], pv[16 * h + 2 * e + 1]), hi[e], lo[e]);
           }
           tmem_st8(tbase + lane_base + C::COL_S + grp * 32 + 8 * h, hi);
           tmem_st8(tbase + lane_base + C::COL_S + grp * 32 + 16 + 8 * h, lo);
@@ -1030,26 +1022,23 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             float d0, d1, d2, d3;
             ld_shared_v4f(sD + e * 4, d0, d1, d2, d3);
             float s0, s1, s2, s3;
+            float g0 = __uint_as_float(v[e]), g1 = __uint_as_float(v[e + 1]);
+            float g2 = __uint_as_float(v[e + 2]), g3 = __uint_as_float(v[e + 3]);
             if constexpr (DROP) {  // dP = dP~ * mask / (1 - p)
               const float kp = p.drop.inv_keep;
-              const float g0 = ((keepm >> e) & 1u) ? __uint_as_float(v[e]) * kp : 0.f;
-              const float g1 = ((keepm >> (e + 1)) & 1u) ? __uint_as_float(v[e + 1]) * kp : 0.f;
-              const float g2 = ((keepm >> (e + 2)) & 1u) ? __uint_as_float(v[e + 2]) * kp : 0.f;
-              const float g3 = ((keepm >> (e + 3)) & 1u) ? __uint_as_float(v[e + 3]) * kp : 0.f;
-              s0 = pv[e] * (g0 - d0);
-              s1 = pv[e + 1] * (g1 - d1);
-              s2 = pv[e + 2] * (g2 - d2);
-              s3 = pv[e + 3] * (g3 - d3);
-            } else {
-              const uint64_t a01 = mul2(f2(pv[e], pv[e + 1]),
-                                        sub2(f2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])),
-                                             f2(d0, d1)));
-              const uint64_t a23 = mul2(f2(pv[e + 2], pv[e + 3]),
-                                        sub2(f2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])),
-                                             f2(d2, d3)));
-              f2_split(a01, s0, s1);
-              f2_split(a23, s2, s3);
+              f2_split(mul2(f2(g0, g1), f2(kp, kp)), g0, g1);
+              f2_split(mul2(f2(g2, g3), f2(kp, kp)), g2, g3);
+              // queries 32g + e .. + 3 are at the byte tops of y
+              const uint32_t y = keepm << (7 - 4 * (e >> 4) - ((e >> 2) & 3));
+              g0 = __uint_as_float(__float_as_uint(g0) & prmt_sign(y, 0x8888u));
+              g1 = __uint_as_float(__float_as_uint(g1) & prmt_sign(y, 0x9999u));
+              g2 = __uint_as_float(__float_as_uint(g2) & prmt_sign(y, 0xAAAAu));
+              g3 = __uint_as_float(__float_as_uint(g3) & prmt_sign(y, 0xBBBBu));
             }
+            const uint64_t a01 = mul2(f2(pv[e], pv[e + 1]), sub2(f2(g0, g1), f2(d0, d1)));
+            const uint64_t a23 = mul2(f2(pv[e + 2], pv[e + 3]), sub2(f2(g2, g3), f2(d2, d3)));
+            f2_split(a01, s0, s1);
+            f2_split(a23, s2, s3);
             if (SLO) {
               split_bf16x2_p(f2(s0, s1), hi[e / 2], lo[e / 2]);
               split_bf16x2_p(f2(s2, s3), hi[e / 2 + 1], lo[e / 2 + 1]);

@@ -57,14 +57,10 @@
 // unchanged: it is still exactly the softmax, as the online rewrite is.
 //
 // Instances fwd_kernel<D, PLO, DROP, FLAT>:
-//   DROP   attention dropout (philox.cuh): the softmax writes the dropped
-//          P entries as 0 (the row sum l still takes every entry) and folds
-//          the keep scale 1 / (1 - p) into 1 / l.  With D <= 64 a fourth
-//          warpgroup draws the keep bits (one thread per query row, a key
-//          tile ahead of the softmax) into a shared-memory ring, so the
-//          generator's integer work runs beside the softmax instead of in
-//          it; with D = 128 each softmax thread draws its own row's bits
-//          before the tile's scores arrive.
+//   DROP   attention dropout (philox.cuh): each softmax thread draws its
+//          row's keep bits for a key tile before that tile's scores arrive,
+//          writes the dropped P entries as 0 (the row sum l still takes
+//          every entry) and folds the keep scale 1 / (1 - p) into 1 / l.
 //   FLAT   Q, K, V and O address (b, h) as one b*H + h index (3-D tensor
 //          maps); otherwise 4-D maps {d, t, h, b} take any element strides,
 //          e.g. q, k, v as views into one fused (B, T, 3C) projection.
@@ -105,13 +101,8 @@ struct FwdCfg {
   static constexpr int OFF_Q = 0;                              // [2] query tiles
   static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
-  // MASKW: dropout keep bits drawn by their own warpgroup into
-  // [2 groups][2 slots][128 rows] x 16 bytes (128 bits per row and key tile)
-  static constexpr bool MASKW = DROP && D <= 64;
-  static constexpr int OFF_MASK = OFF_V + STAGES * TILE_BYTES;
-  static constexpr int MASK_BYTES = MASKW ? 2 * 2 * 128 * 16 : 0;
-  static constexpr int OFF_BAR = OFF_MASK + MASK_BYTES;
-  static constexpr int NUM_BARS = 55;
+  static constexpr int OFF_BAR = OFF_V + STAGES * TILE_BYTES;
+  static constexpr int NUM_BARS = 47;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_USED = OFF_MISC + 64;
   // at least 116 KB so that one CTA holds an SM (it takes all 512 TMEM columns)
@@ -132,7 +123,7 @@ struct FwdCfg {
   static constexpr uint32_t COL_OL1 = SPLIT ? 256 + 3 * D : COL_O1;
   static constexpr uint32_t TMEM_COLS = 512;
   // Two softmax warpgroups, then the producer and two MMA issuers.  With
-  // D = 128 (REBALANCE) a twelfth, idle warp completes the third warpgroup
+  // D >= 64 (REBALANCE) a twelfth, idle warp completes the third warpgroup
   // so that its registers can be handed to the softmax warps (setmaxnreg
   // acts on whole warpgroups): at launch every thread holds LAUNCH_REGS
   // (65536 / 384, rounded down to 8); the third warpgroup then drops to
@@ -141,13 +132,15 @@ struct FwdCfg {
   // on the long-context workload, at 216 and 64; 208 and 80 measured 2-4 %
   // faster still, 224 and 48 between them).  D = 64 takes 200 and 88 (1 %
   // faster than 168 throughout; 208 and 72 the same; 216 and 64 measured
-  // 4 % slower); D <= 32 keeps 11 warps and 168 registers.  MASKW adds the keep-bit warpgroup (16
-  // warps): 128 registers at launch, 184 for the softmax, 72 for the rest.
-  static constexpr bool REBALANCE = D >= 64 || MASKW;
-  static constexpr int THREADS = MASKW ? 512 : REBALANCE ? 384 : 352;
-  static constexpr int LAUNCH_REGS = MASKW ? 128 : 168;
-  static constexpr int REGS_SOFTMAX = MASKW ? 184 : D == 128 ? 208 : 200;
-  static constexpr int REGS_OTHER = MASKW ? 72 : D == 128 ? 80 : 88;
+  // 4 % slower); D <= 32 keeps 11 warps and 168 registers.  With dropout
+  // the softmax threads draw the keep bits themselves: at 200 registers
+  // that measured faster than a fourth warpgroup drawing them into a
+  // shared-memory ring (145 against 167 us on the GPT-2 layer).
+  static constexpr bool REBALANCE = D >= 64;
+  static constexpr int THREADS = REBALANCE ? 384 : 352;
+  static constexpr int LAUNCH_REGS = 168;
+  static constexpr int REGS_SOFTMAX = D == 128 ? 208 : 200;
+  static constexpr int REGS_OTHER = D == 128 ? 80 : 88;
   static_assert(!REBALANCE ||
                     256 * REGS_SOFTMAX + (THREADS - 256) * REGS_OTHER <= THREADS * LAUNCH_REGS,
                 "register split exceeds the launch allocation");
@@ -162,9 +155,7 @@ enum : int {
   FB_QFREE = FB_QFULL + 2, FB_SFULL = FB_QFULL + 4, FB_ODONE = FB_QFULL + 6,
   FB_OFREE = FB_QFULL + 8, FB_SFREE = FB_QFULL + 10, FB_DRAIN = FB_QFULL + 12,
   FB_PFULL = FB_QFULL + 14,  // FB_PFULL + 4 * g + part
-  FB_OFFSET = FB_PFULL + 8,  // the one-time start offset of the two groups
-  FB_MFULL = FB_OFFSET + 1,  // keep bits of group g, slot s: FB_MFULL + 2 * g + s
-  FB_MEMPTY = FB_MFULL + 4   // the slot read by all 128 softmax threads
+  FB_OFFSET = FB_PFULL + 8   // the one-time start offset of the two groups
 };
 
 // Pairs of score columns whose exponential is taken by exp2_poly2 on the FMA
@@ -198,8 +189,9 @@ constexpr int kPvParts = 2;
 
 // P = 2^(s * scale_log2 - m) for one row of a 128-column tile: written to
 // TMEM as bf16 (or bf16 hi/lo), the row sum accumulated in sum2.
-// DROP: P entries whose bit in keep (bit c of keep[c / 32] for column c) is
-// clear are written as 0; the row sum still takes every entry.
+// DROP: P entries whose bit in keep (column c at bit il_pos(c % 32) of
+// keep[c / 32]) is clear are written as 0; the row sum still takes every
+// entry.  A pair's two bits become a bf16x2 AND mask with one prmt.
 template <int D, bool POLY, bool PLO, bool DROP>
 __device__ __forceinline__ void fwd_exp_row(const float (&s)[128], uint64_t sl2x2, uint64_t negm2,
                                             uint32_t scol, uint64_t (&sum2)[2], uint32_t pfull0,
@@ -221,20 +213,21 @@ __device__ __forceinline__ void fwd_exp_row(const float (&s)[128], uint64_t sl2x
         p2 = f2(ex2(x0), ex2(x1));
       }
       sum2[e & 1] = add2(sum2[e & 1], p2);
-      if constexpr (DROP) {
-        const int c = ch * 16 + 2 * e;
-        float p0, p1;
-        f2_split(p2, p0, p1);
-        p0 = ((keep[c >> 5] >> (c & 31)) & 1u) ? p0 : 0.f;
-        p1 = ((keep[c >> 5] >> ((c + 1) & 31)) & 1u) ? p1 : 0.f;
-        p2 = f2(p0, p1);
-      }
       if (PLO) {
         split_bf16x2_p(p2, hi[e], lo[e]);
       } else {
         float p0, p1;
         f2_split(p2, p0, p1);
         hi[e] = pack_bf16(p0, p1);
+      }
+      if constexpr (DROP) {
+        // columns 16 ch + 2 e, + 1: keys 16 h + 4 v + k, k = 2 (e & 1) and
+        // 2 (e & 1) + 1, of word ch / 2; the shift moves their flags to the
+        // top of bytes k
+        const uint32_t y = keep[ch >> 1] << (7 - 4 * (ch & 1) - (e >> 1));
+        const uint32_t m = prmt_sign(y, (e & 1) ? 0xBBAAu : 0x9988u);
+        hi[e] &= m;
+        if (PLO) lo[e] &= m;
       }
     }
     tmem_st8(scol + ch * 8, hi);
@@ -292,7 +285,7 @@ __global__ void __launch_bounds__(FwdCfg<D, PLO, DROP>::THREADS, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = FwdCfg<D, PLO, DROP>;
-  static_assert(FB_MEMPTY + 4 <= C::NUM_BARS, "barrier count");
+  static_assert(FB_OFFSET + 1 <= C::NUM_BARS, "barrier count");
   static_assert(C::STAGES <= kMaxStages, "barrier map");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = aligned_smem(smem_raw, C::SMEM_USED, nullptr);
@@ -331,10 +324,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       mbar_init(bar(FB_DRAIN + g), 1);
     }
     mbar_init(bar(FB_OFFSET), 128);
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(bar(FB_MFULL + i), 128);
-      mbar_init(bar(FB_MEMPTY + i), 128);
-    }
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -348,55 +337,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 
   if (warp >= 8) {
   // third warpgroup: producer, MMA issuers (and with REBALANCE an idle
-  // warp); with MASKW the fourth, keep-bit warpgroup too
+  // warp)
   if constexpr (C::REBALANCE) regs_dec<C::REGS_OTHER>();
-  if (warp >= 12) {
-    // ------------------------------------------------ keep bits (MASKW only)
-    // Thread t draws row t's keep bits for every key tile the softmax
-    // groups visit, in their order (tile j of group 0, then of group 1),
-    // into slot (tile count) % 2 of the group's ring, at most two tiles
-    // ahead of the group's softmax.
-    if constexpr (C::MASKW) {
-      const int t = threadIdx.x - 384;  // query row within the tile
-      uint4* mask = reinterpret_cast<uint4*>(smem + C::OFF_MASK);
-      int mg[2] = {0, 0};  // tiles drawn per group
-      bool ok = true;
-      for (int k = 0; ok; ++k) {
-        const int u = fwd_item(k, b, G, n_items);
-        if (u < 0) break;
-        const FwdItem it = fwd_item_info(u, k, p.BH, n_pairs, p.n_qtiles);
-        const int jmax = it.n[0] > it.n[1] ? it.n[0] : it.n[1];
-        for (int j = 0; j < jmax && ok; ++j) {
-          for (int g = 0; g < 2; ++g) {
-            if (j >= it.n[g]) continue;
-            const int slot = mg[g] & 1;
-            if (mg[g] >= 2) {
-              const uint32_t ph = ((mg[g] >> 1) - 1) & 1;
-              if (!wait_warp(w, bar(FB_MEMPTY + 2 * g + slot), ph, 15)) {
-                ok = false;
-                break;
-              }
-              (void)mbar_try_wait(bar(FB_MEMPTY + 2 * g + slot), ph);  // acquire, every lane
-            }
-            const uint32_t qi = static_cast<uint32_t>(it.tile[g] * C::BM + t);
-            uint32_t kw[4] = {0u, 0u, 0u, 0u};
-#pragma unroll 2  // fully unrolled, the 16 generator blocks spill at 72 registers
-            for (int c4 = 0; c4 < 4; ++c4)
-#pragma unroll
-              for (int x = 0; x < 4; ++x)
-                kw[c4] |= keep_byte(static_cast<uint32_t>(j * 16 + c4 * 4 + x), qi,
-                                    static_cast<uint32_t>(it.bh), p.drop) << (8 * x);
-            mask[(2 * g + slot) * 128 + t] = make_uint4(kw[0], kw[1], kw[2], kw[3]);
-            mbar_arrive(bar(FB_MFULL + 2 * g + slot));
-            if (p.drop.mask != nullptr)  // the backward's copy
-              store_keep_block(kw, p.drop.mask + keep_cache_block(it.bh, p.n_qtiles, it.tile[g], j),
-                               t >> 5, lane);
-            ++mg[g];
-          }
-        }
-      }
-    }
-  } else if (warp == 8) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     // Per item: Q_g once the previous item no longer needs the Q_g buffer,
     // then K_j, V_j through a ring that runs on across items (tk counts the
@@ -602,14 +545,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // dropout keep bits of this row's 128 keys of tile j, computed while
         // the scores are still on their way
         [[maybe_unused]] uint32_t keep[4] = {0u, 0u, 0u, 0u};
-        if constexpr (DROP && !C::MASKW) {
+        if constexpr (DROP) {
           const uint32_t qi = static_cast<uint32_t>(it.tile[g] * C::BM + row);
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4)
-#pragma unroll
-            for (int x = 0; x < 4; ++x)
-              keep[c4] |= keep_byte(static_cast<uint32_t>(j * 16 + c4 * 4 + x), qi,
-                                    static_cast<uint32_t>(it.bh), p.drop) << (8 * x);
+            keep[c4] = keep32_il(static_cast<uint32_t>(j * 4 + c4), qi, static_cast<uint32_t>(it.bh),
+                                 p.drop);
           if (p.drop.mask != nullptr)  // the backward's copy
             store_keep_block(keep, p.drop.mask + keep_cache_block(it.bh, p.n_qtiles, it.tile[g], j),
                              quarter, lane);
@@ -685,17 +626,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const uint64_t sl2x2 = f2(sl2, sl2);
         const uint64_t negm2 = f2(-m_used, -m_used);
         uint64_t sum2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
-        if constexpr (C::MASKW) {  // this row's keep bits of tile j, from the ring
-          const int slot = tgj & 1;
-          wait_warp(w, bar(FB_MFULL + 2 * g + slot), (tgj >> 1) & 1, 16);
-          (void)mbar_try_wait(bar(FB_MFULL + 2 * g + slot), (tgj >> 1) & 1);  // acquire, every lane
-          const uint4 kw = reinterpret_cast<const uint4*>(smem + C::OFF_MASK)[(2 * g + slot) * 128 + row];
-          keep[0] = kw.x;
-          keep[1] = kw.y;
-          keep[2] = kw.z;
-          keep[3] = kw.w;
-          mbar_arrive(bar(FB_MEMPTY + 2 * g + slot));
-        }
         // Group 0's side of the one-time offset (see before the item loop).
         const bool offset = k == 0 && j == 0 && it.n[0] > 0 && it.n[1] > 0;
         if constexpr (fwd_exp_turns(D)) {

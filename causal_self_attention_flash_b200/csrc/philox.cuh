@@ -14,14 +14,14 @@
 // the 64-bit products and mixes the high halves with the other two words
 // and the key; the key advances by two Weyl constants between rounds.
 //
-// Mask element (b, h, i, j), query i and key j, takes 16 bits of the block
-// with counter (j >> 3, i, b*H + h, offset) and key (seed low, seed high):
-// word (j & 7) >> 1, low half for even j and high half for odd j.  It is
-// dropped iff those bits are below t = round(p * 65536), so the keep scale is
-// 65536 / (65536 - t) (the drop probability is t / 65536, p to within 2^-17).
-// The mask therefore does not depend on how the kernels tile the work: the
-// forward (thread = query row) and the backward (thread = key row) derive
-// the same bits.
+// Mask element (b, h, i, j), query i and key j, takes 8 bits of the block
+// with counter (j >> 4, i, b*H + h, offset) and key (seed low, seed high):
+// byte j & 3 of word (j & 15) >> 2.  It is dropped iff that byte is below
+// t = round(p * 256), so the keep scale is 256 / (256 - t) (the drop
+// probability is t / 256, p to within 2^-9).  One block serves 16 keys of
+// one query.  The mask does not depend on how the kernels tile the work:
+// the forward (thread = query row) and the backward (thread = key row)
+// derive the same bits.
 #pragma once
 
 #include <cstdint>
@@ -33,82 +33,149 @@ constexpr uint32_t kPhiloxM1 = 0xCD9E8D57u;
 constexpr uint32_t kPhiloxW0 = 0x9E3779B9u;
 constexpr uint32_t kPhiloxW1 = 0xBB67AE85u;
 
+constexpr int kPhiloxRounds = 10;
+
+// DropParams{} is "no dropout".
 struct DropParams {
-  uint32_t t16x;    // drop threshold t shifted left by 16 (t = round(p * 65536))
-  uint32_t k0, k1;  // seed, low and high word
-  uint32_t offset;  // counter word 3
-  float inv_keep;   // 65536 / (65536 - t)
-  uint32_t* mask;   // the keep bits kept between forward and backward, or null
+  uint32_t t = 0;              // drop threshold round(p * 256); 0 = no dropout
+  uint32_t t_lo = 0;           // (t & 0x7F) in every byte
+  uint32_t t_maj = 0;          // all ones when t < 128, else 0 (see keep_nibble)
+  uint32_t offset = 0;         // counter word 3
+  // the key of every round: rk[2r] = seed low + r * W0, rk[2r + 1] =
+  // seed high + r * W1 (mod 2^32), set on the host so that the rounds read
+  // them as kernel parameters
+  uint32_t rk[2 * kPhiloxRounds] = {};
+  float inv_keep = 1.f;        // 256 / (256 - t)
+  uint32_t* mask = nullptr;    // the keep bits kept between forward and backward, or null
 };
+
+// The round keys of seed (k0 low, k1 high word).
+__host__ __device__ inline void philox_round_keys(uint32_t k0, uint32_t k1, uint32_t* rk) {
+  for (int r = 0; r < kPhiloxRounds; ++r) {
+    rk[2 * r] = k0;
+    rk[2 * r + 1] = k1;
+    k0 += kPhiloxW0;
+    k1 += kPhiloxW1;
+  }
+}
 
 // Keep-bit cache: one block of 128 x 4 words per (head bh, query tile qt,
 // key tile kt <= qt) of 128 x 128, at block bh * n_pairs + qt (qt + 1) / 2
 // + kt (n_pairs = n_tiles (n_tiles + 1) / 2); word [kr][w] of a block holds
-// bit c = keep bit of query 128 qt + 32 w + c, key 128 kt + kr.  Keys and
-// queries past T hold generator bits too; nothing reads them.  The forward
-// (thread = query row) writes it, the backward (thread = key row) reads one
-// word per 32 queries.
+// the keep bit of query 128 qt + 32 w + c, key 128 kt + kr, at bit
+// il_pos(c) (the interleaved order below).  Keys and queries past T hold
+// generator bits too; nothing reads them.  The forward (thread = query
+// row) writes it, the backward (thread = key row) reads one word per 32
+// queries.
 __host__ __device__ constexpr size_t keep_cache_block(long long bh, int n_tiles, int qt, int kt) {
   return (static_cast<size_t>(bh) * (static_cast<size_t>(n_tiles) * (n_tiles + 1) / 2) +
           static_cast<size_t>(qt) * (qt + 1) / 2 + kt) * 512;
 }
 
+// 32 x 32 bit transpose across a warp: on entry lane l holds row l (bit c
+// = element (l, c)), on return column l (bit c = element (c, l)).  Five
+// exchange rounds: at round j the off-diagonal j x j sub-blocks of every
+// 2j x 2j block swap between lanes l and l ^ j.
+__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane) {
+#pragma unroll
+  for (int j = 16, i = 0; j > 0; j >>= 1, ++i) {
+    const uint32_t m = i == 0 ? 0x0000FFFFu : i == 1 ? 0x00FF00FFu : i == 2 ? 0x0F0F0F0Fu
+                                              : i == 3 ? 0x33333333u : 0x55555555u;
+    const uint32_t y = __shfl_xor_sync(0xffffffffu, x, j);
+    x = (lane & j) ? ((x & ~m) | ((y >> j) & m)) : ((x & m) | ((y & m) << j));
+  }
+  return x;
+}
+
+// Interleaved order of a 32-element keep word (keys in the forward's
+// keep32_il, queries in the cache and the backward): element 16 h + 4 v + k
+// sits at bit 8 k + 4 h + v, so that shifting the word left by 7 - 4 h - v
+// puts the flags of elements 16 h + 4 v .. + 3 on the top bits of bytes
+// 0 .. 3 (for prmt_sign).  il_key(position) inverts it.
+__host__ __device__ constexpr int il_pos(int key) {
+  return 8 * (key & 3) + 4 * ((key >> 4) & 1) + ((key >> 2) & 3);
+}
+__host__ __device__ constexpr int il_key(int pos) {
+  return 16 * ((pos >> 2) & 1) + 4 * (pos & 3) + (pos >> 3);
+}
+
 // The calling warp holds 32 consecutive query rows (32 w .. 32 w + 31 of a
-// tile), each lane its row's keep bits for 128 keys (bit c of kw[c / 32]);
-// stores them transposed into cache block `blk`: word [kr][w] gets bit
-// `lane` from lane's key kr.  Each 32 x 32 bit block is transposed across
-// the warp in five exchange rounds: at round j the off-diagonal j x j
-// sub-blocks of every 2j x 2j block swap between lanes l and l ^ j.
+// tile), each lane its row's keep bits for 128 keys, key 32 kb + c at bit
+// il_pos(c) of kw[kb]; stores them transposed into cache block `blk`: word
+// [kr][w] gets query 32 w + c's bit for key kr at bit il_pos(c).  Lane p
+// first takes the row of query il_key(p), so that the transpose puts the
+// queries in the interleaved order; lane p then holds key il_key(p).
 __device__ __forceinline__ void store_keep_block(const uint32_t (&kw)[4], uint32_t* blk, int w,
                                                  int lane) {
+  const int kr = il_key(lane);
 #pragma unroll
-  for (int kb = 0; kb < 4; ++kb) {
-    uint32_t x = kw[kb];
-#pragma unroll
-    for (int j = 16, i = 0; j > 0; j >>= 1, ++i) {
-      const uint32_t m = i == 0 ? 0x0000FFFFu : i == 1 ? 0x00FF00FFu : i == 2 ? 0x0F0F0F0Fu
-                                                : i == 3 ? 0x33333333u : 0x55555555u;
-      const uint32_t y = __shfl_xor_sync(0xffffffffu, x, j);
-      x = (lane & j) ? ((x & ~m) | ((y >> j) & m)) : ((x & m) | ((y & m) << j));
-    }
-    blk[(32 * kb + lane) * 4 + w] = x;
-  }
+  for (int kb = 0; kb < 4; ++kb)
+    blk[(32 * kb + kr) * 4 + w] = warp_transpose32(__shfl_sync(0xffffffffu, kw[kb], kr), lane);
 }
 
+// One round: both 32 x 32 -> 64-bit products as single widening multiplies.
 __device__ __forceinline__ void philox4x32_10(uint32_t& c0, uint32_t& c1, uint32_t& c2,
-                                              uint32_t& c3, uint32_t k0, uint32_t k1) {
+                                              uint32_t& c3, const uint32_t (&rk)[2 * kPhiloxRounds]) {
 #pragma unroll
-  for (int r = 0; r < 10; ++r) {
-    if (r > 0) {
-      k0 += kPhiloxW0;
-      k1 += kPhiloxW1;
-    }
-    const uint32_t lo0 = c0 * kPhiloxM0, hi0 = __umulhi(c0, kPhiloxM0);
-    const uint32_t lo1 = c2 * kPhiloxM1, hi1 = __umulhi(c2, kPhiloxM1);
-    const uint32_t n0 = hi1 ^ c1 ^ k0;
-    const uint32_t n2 = hi0 ^ c3 ^ k1;
+  for (int r = 0; r < kPhiloxRounds; ++r) {
+    const uint64_t p0 = static_cast<uint64_t>(c0) * kPhiloxM0;
+    const uint64_t p1 = static_cast<uint64_t>(c2) * kPhiloxM1;
+    const uint32_t n0 = static_cast<uint32_t>(p1 >> 32) ^ c1 ^ rk[2 * r];
+    const uint32_t n2 = static_cast<uint32_t>(p0 >> 32) ^ c3 ^ rk[2 * r + 1];
     c0 = n0;
-    c1 = lo1;
+    c1 = static_cast<uint32_t>(p1);
     c2 = n2;
-    c3 = lo0;
+    c3 = static_cast<uint32_t>(p0);
   }
 }
 
-// Keep bits of keys 8*jg .. 8*jg + 7 for query i of head bh: bit e set iff
-// key 8*jg + e is kept.  A 16-bit half h of word w is >= t exactly when
-// (w << 16) (low half) or w (high half) is >= t << 16.
-__device__ __forceinline__ uint32_t keep_byte(uint32_t jg, uint32_t i, uint32_t bh,
-                                              const DropParams& d) {
+// Bit k (k < 4) set iff byte k of w is >= t, all four bytes at once.
+// r = (w | 0x80 in every byte) - (t & 0x7F in every byte) borrows across
+// no byte boundary, and its top bit in byte k says whether the byte's low
+// seven bits reach t's.  byte >= t iff its top bit beats t's, or the top
+// bits are equal and the low seven bits reach t's: the majority of the
+// byte's top bit, r's top bit and (t < 128).  The four top bits are then
+// gathered by one multiplication (the partial products land on distinct
+// bits, so nothing carries into bits 28..31).
+__device__ __forceinline__ uint32_t keep_flags(uint32_t w, const DropParams& d) {
+  const uint32_t r = (w | 0x80808080u) - d.t_lo;
+  return ((w & r) | (d.t_maj & (w | r))) & 0x80808080u;
+}
+__device__ __forceinline__ uint32_t keep_nibble(uint32_t w, const DropParams& d) {
+  return (keep_flags(w, d) * 0x00204081u) >> 28;
+}
+
+// Keep bits of keys 16*jg .. 16*jg + 15 for query i of head bh: bit e set
+// iff key 16*jg + e is kept.
+__device__ __forceinline__ uint32_t keep16(uint32_t jg, uint32_t i, uint32_t bh,
+                                           const DropParams& d) {
   uint32_t c0 = jg, c1 = i, c2 = bh, c3 = d.offset;
-  philox4x32_10(c0, c1, c2, c3, d.k0, d.k1);
-  const uint32_t w[4] = {c0, c1, c2, c3};
-  uint32_t b = 0;
+  philox4x32_10(c0, c1, c2, c3, d.rk);
+  return keep_nibble(c0, d) | keep_nibble(c1, d) << 4 | keep_nibble(c2, d) << 8 |
+         keep_nibble(c3, d) << 12;
+}
+
+// Keep bits of keys 32*jp .. 32*jp + 31 for query i in the interleaved
+// order (il_pos): the four flag words of a block need only a shift each.
+__device__ __forceinline__ uint32_t keep32_il(uint32_t jp, uint32_t i, uint32_t bh,
+                                              const DropParams& d) {
+  uint32_t x = 0;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    b |= static_cast<uint32_t>((w[k] << 16) >= d.t16x) << (2 * k);
-    b |= static_cast<uint32_t>(w[k] >= d.t16x) << (2 * k + 1);
+  for (int h = 0; h < 2; ++h) {
+    uint32_t c0 = 2 * jp + h, c1 = i, c2 = bh, c3 = d.offset;
+    philox4x32_10(c0, c1, c2, c3, d.rk);
+    x |= keep_flags(c0, d) >> (7 - 4 * h) | keep_flags(c1, d) >> (6 - 4 * h) |
+         keep_flags(c2, d) >> (5 - 4 * h) | keep_flags(c3, d) >> (4 - 4 * h);
   }
-  return b;
+  return x;
+}
+
+// Byte-wise sign replication: byte n of the result is 0xFF iff the top
+// bit of the byte of x chosen by selector nibble n (its low 3 bits) is set.
+__device__ __forceinline__ uint32_t prmt_sign(uint32_t x, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(x), "r"(sel));
+  return r;
 }
 
 }  // namespace cattn

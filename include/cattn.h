@@ -227,11 +227,11 @@ CATTN_API cattn_status attn_bwd_strided(const void* q, cattn_layout lq, const vo
  * M comes from Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random
  * numbers: as easy as 1, 2, 3", SC 2011), key = (seed low 32 bits, seed
  * high 32 bits).  Element (b, h, i, j) (query i, key j) uses the block with
- * counter (j >> 3, i, b*H + h, offset), word (j & 7) >> 1, low 16 bits for
- * even j and high 16 bits for odd j; it is dropped iff those 16 bits are
- * below t = round(p * 65536) (t at most 65535), and kept entries are scaled
- * by 65536 / (65536 - t).  So the drop probability is t / 65536 (p to within
- * 2^-17) and E[P~] = P exactly.  The mask depends only on (seed, offset,
+ * counter (j >> 4, i, b*H + h, offset), byte j & 3 (bits 8 (j & 3) ..
+ * 8 (j & 3) + 7) of word (j & 15) >> 2; it is dropped iff that byte is
+ * below t = round(p * 256) (t at most 255), and kept entries are scaled by
+ * 256 / (256 - t).  So the drop probability is t / 256 (p to within 2^-9)
+ * and E[P~] = P exactly.  The mask depends only on (seed, offset,
  * b*H + h, i, j): the forward and backward of one step must get the same
  * seed and offset; use another offset (or seed) for every call that wants a
  * fresh mask (each layer, each step).

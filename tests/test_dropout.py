@@ -168,14 +168,22 @@ def test_autograd_qkv_with_dropout(lib):
     check_bf16("dv", as_f64(view(g[..., 2 * C:])), rv)
 
 
+def _il_pos(c):
+    """Bit position of element c (0..31) of a keep word in the interleaved
+    order: c = 16 h + 4 v + k sits at bit 8 k + 4 h + v."""
+    return 8 * (c & 3) + 4 * ((c >> 4) & 1) + ((c >> 2) & 3)
+
+
 def _unpack_mask(buf, B, H, T):
     """The keep-bit cache as a (B, H, T, T) bool array [query, key]: block
-    bh * n_pairs + qt (qt + 1) / 2 + kt holds words [kr][w], bit c = query
-    128 qt + 32 w + c, key 128 kt + kr (tiles on or below the diagonal)."""
+    bh * n_pairs + qt (qt + 1) / 2 + kt holds words [kr][w], bit il_pos(c) =
+    query 128 qt + 32 w + c, key 128 kt + kr (tiles on or below the
+    diagonal)."""
     n = (T + 127) // 128
     n_pairs = n * (n + 1) // 2
     words = buf.view(torch.int32).cpu().numpy().view(np.uint32).reshape(B * H, n_pairs, 128, 4)
-    bits = (words[..., None] >> np.arange(32, dtype=np.uint32)) & 1  # [bh, blk, kr, w, c]
+    pos = np.array([_il_pos(c) for c in range(32)], dtype=np.uint32)
+    bits = (words[..., None] >> pos) & 1  # [bh, blk, kr, w, c]
     full = np.zeros((B * H, n * 128, n * 128), dtype=bool)
     for qt in range(n):
         for kt in range(qt + 1):
