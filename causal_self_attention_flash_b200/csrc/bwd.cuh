@@ -71,6 +71,8 @@ struct PreParams {
 // CONTIG: O and dO are contiguous (B, H, T, D), addressed as rows of D.
 template <int D, bool CONTIG>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
+  grid_dep_wait();    // the previous kernel's O, dO, LSE
+  grid_dep_launch();  // the main kernel may take SMs as this grid drains
   constexpr int TPR = D / 8;
   constexpr int RPW = 32 / TPR;  // rows per warp per step
   const int lane = threadIdx.x & 31;
@@ -165,6 +167,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
 __global__ void __launch_bounds__(256) dq_convert_f32_kernel(const float4* __restrict__ acc,
                                                              float4* __restrict__ dq, size_t n4,
                                                              float scale) {
+  grid_dep_wait();  // the main kernel's accumulator
   const size_t tid = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const size_t nth = static_cast<size_t>(gridDim.x) * blockDim.x;
   for (size_t i = tid; i < n4; i += nth) {
@@ -176,6 +179,7 @@ __global__ void __launch_bounds__(256) dq_convert_f32_kernel(const float4* __res
 __global__ void __launch_bounds__(256) dq_convert_kernel(const float4* __restrict__ acc,
                                                          uint4* __restrict__ dq, size_t n8,
                                                          float scale) {
+  grid_dep_wait();  // the main kernel's accumulator
   const size_t tid = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const size_t nth = static_cast<size_t>(gridDim.x) * blockDim.x;
   for (size_t i = tid; i < n8; i += nth) {
@@ -198,6 +202,7 @@ __global__ void __launch_bounds__(256) dq_convert_strided_kernel(const float4* _
                                                                  int T, long long n8,
                                                                  long long sb, long long sh,
                                                                  long long st, float scale) {
+  grid_dep_wait();  // the main kernel's accumulator
   constexpr int C8 = D / 8;  // 8-element chunks per row
   const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long nth = static_cast<long long>(gridDim.x) * blockDim.x;
@@ -397,6 +402,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   using C = BwdCfg<D, SLO>;
   static_assert(BB_PFULL2 + 1 <= C::NUM_BARS, "barrier count");
   static_assert(C::QST <= 4 && C::DOST <= 4, "barrier map");
+  // launched behind the preprocess, which writes Delta, LSE, the cleared
+  // accumulator and status words: nothing before this line touches memory
+  grid_dep_wait();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = aligned_smem(smem_raw, C::SMEM_USED, p.status);
   if (smem == nullptr) return;  // uniform over the CTA: nothing touched yet

@@ -126,6 +126,11 @@ __global__ void __launch_bounds__(kDecodeThreads, decode_ctas_per_sm(D))
   static_assert(NS % 2 == 0 && D % 16 == 0, "tiles");
   static_assert((2 * NW * 8 + NW * 8 * D + 16 + 8 * D) * 4 <= decode_smem_bytes(D), "merge area");
 
+  // launched as a programmatic dependent: the previous kernel (say, the one
+  // that appends to the cache) has finished and its writes are visible
+  // after this; the next call may then take SMs as this grid drains
+  dec_grid_dep_wait();
+  dec_grid_dep_launch();
   uint8_t* smem = dec_dynamic_smem();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t4 = lane & 3;  // fragment row, column pair

@@ -36,6 +36,15 @@ __device__ __forceinline__ void dec_cp_async16(void* dst, const void* src, bool 
                "l"(src), "r"(valid ? 16 : 0)
                : "memory");
 }
+// Programmatic dependent launch (as grid_dep_wait / grid_dep_launch of the
+// main kernels): wait for the grid launched before this one to complete
+// and its writes to be visible; let the next grid be scheduled.
+__device__ __forceinline__ void dec_grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void dec_grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 __device__ __forceinline__ void dec_cp_async_commit() {
   asm volatile("cp.async.commit_group;\n" ::: "memory");
 }

@@ -122,6 +122,10 @@ inline uint32_t dec_pack_bf16(float lo, float hi) {
 
 inline void dec_cluster_sync() { emu::t_cta->cluster->bar->arrive_and_wait(); }
 
+// One grid at a time: nothing to wait for, nothing to release.
+inline void dec_grid_dep_wait() {}
+inline void dec_grid_dep_launch() {}
+
 inline float dec_cluster_ld(const float* local, unsigned rank) {
   emu::check_smem(local, 4, 4);
   const emu::Cta* c = emu::t_cta;
