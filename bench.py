@@ -377,7 +377,52 @@ def measure_detail(args, w, sets, olos, step, stream, cattn):
         detail["decode"] = measure_decode(w, sets, stream, cattn, n)
     except Exception as e:  # noqa: BLE001  (a side measurement; the step stands)
         detail["decode"] = {"unavailable": str(e)[:120]}
+    try:
+        detail["dropout"] = measure_dropout(w, sets, stream, cattn, timed, pct,
+                                            pct(fwd_ms, 0.5), pct(bwd_ms, 0.5))
+    except Exception as e:  # noqa: BLE001  (a side measurement; the step stands)
+        detail["dropout"] = {"unavailable": str(e)[:120]}
     return detail
+
+
+DROPOUT_P = 0.2  # the pages' Shakespeare model (nanoGPT page, section 3)
+
+
+def measure_dropout(w, sets, stream, cattn, timed, pct, fwd_plain_ms, bwd_plain_ms):
+    """The workload's forward and backward calls with attention dropout
+    p = 0.2 (the _strided calls with a Dropout), keep bits drawn in both
+    calls or kept by the forward for the backward (the keep-bit cache);
+    median ms per call over the rotating input sets, and the ratio to the
+    plain calls."""
+    n = 20
+    B, H, T = w.B, w.H, w.T
+    masks = [cattn.attn_dropout_mask(B, H, T, sets[0][0].device) for _ in range(N_SETS)]
+    out = {"p": DROPOUT_P, "calls": n}
+    for kind in ("drawn", "cached"):
+        def params(i):
+            return cattn.dropout_params(DROPOUT_P, seed=1234, offset=i % N_SETS,
+                                        mask=masks[i % N_SETS] if kind == "cached" else None)
+
+        def fwd(i):
+            qd, kd, vd, dod, o, lse, dq, dk, dv, ws = sets[i % N_SETS]
+            cattn.attn_fwd_strided(qd, kd, vd, w.scale, o=o, lse=lse, stream=stream,
+                                   dropout=params(i))
+
+        def bwd(i):
+            qd, kd, vd, dod, o, lse, dq, dk, dv, ws = sets[i % N_SETS]
+            cattn.attn_bwd_strided(qd, kd, vd, o, lse, dod, w.scale, dq=dq, dk=dk, dv=dv,
+                                   workspace=ws, stream=stream, dropout=params(i))
+
+        for i in range(N_SETS):
+            fwd(i)
+        f = pct(timed(fwd, n), 0.5)
+        # input set s's backward then holds its forward's mask (offset s)
+        for i in range(N_SETS):
+            fwd(i)
+        b = pct(timed(bwd, n), 0.5)
+        out[kind] = {"fwd_ms": f, "bwd_ms": b, "fwd_vs_plain": f / fwd_plain_ms,
+                     "bwd_vs_plain": b / bwd_plain_ms}
+    return out
 
 
 def decode_bytes(B, H, L, D, Tq=1) -> int:
