@@ -75,6 +75,7 @@ SIGNATURES = {
     "cattn_timing_read": (_i, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int), _i]),
     "cattn_status_string": (ctypes.c_char_p, [_i]),
     "cattn_version": (_i, []),
+    "cattn_plan_passes": (_i, [_i, _i, _i, _i, ctypes.POINTER(ctypes.c_uint16), _i]),
     "cattn_last_cuda_error": (_i, []),
 }
 

@@ -7,6 +7,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <array>
+#include <map>
 #include <mutex>
 #include <utility>
 #include <vector>
@@ -113,6 +115,85 @@ cattn_status ensure_smem(int dev, unsigned bit, K kernel, int bytes, int launch_
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Pass codes for items of the given costs (numbered longest first) on G
+// CTAs, planned greedily pass by pass (sched.cuh): each pass takes the
+// direction and rotation that leave the lowest maximum CTA load, then the
+// lowest sum of squared loads.  More than kMaxPassCodes passes: none
+// (every pass alternates).
+void plan_passes(const std::vector<int>& cost, int G, PassCodes* pc) {
+  pc->n = 0;
+  const long long n = static_cast<long long>(cost.size());
+  if (G < 2 || n == 0) return;
+  const long long passes = (n + G - 1) / G;
+  if (passes > kMaxPassCodes) return;
+  std::vector<long long> load(G, 0), trial(G);
+  for (int k = 0; k < passes; ++k) {
+    const long long first = static_cast<long long>(k) * G;
+    const int m = static_cast<int>(n - first < G ? n - first : G);
+    long long best_mx = -1, best_sq = 0;
+    int best = 0;
+    for (int d = 0; d < 2; ++d)
+      for (int r = 0; r < G; ++r) {
+        trial = load;
+        for (int j = 0; j < m; ++j) {
+          int b = (d ? r - j : r + j) % G;
+          if (b < 0) b += G;
+          trial[b] += cost[first + j];
+        }
+        long long mx = 0, sq = 0;
+        for (long long x : trial) {
+          mx = x > mx ? x : mx;
+          sq += x * x;
+        }
+        if (best_mx < 0 || mx < best_mx || (mx == best_mx && sq < best_sq)) {
+          best_mx = mx;
+          best_sq = sq;
+          best = (d << 15) | r;
+        }
+      }
+    for (int j = 0; j < m; ++j) {
+      const int r = best & 0x7fff;
+      int b = ((best >> 15) ? r - j : r + j) % G;
+      if (b < 0) b += G;
+      load[b] += cost[first + j];
+    }
+    pc->code[k] = static_cast<uint16_t>(best);
+  }
+  pc->n = static_cast<int>(passes);
+}
+
+// The pass codes of a persistent launch, planned once per (kernel kind,
+// B*H, tiles, grid size): kind 0 deals the forward's items (query-tile
+// pairs, an item's load its two groups' key tiles).  The backward (kind 1)
+// keeps alternating passes: every variant of it that looked its items up
+// through pass codes measured slower (GPT-2 layer backward call 180-187
+// against 170 us), even with all passes alternating.
+PassCodes pass_plan(int kind, int BH, int n_tiles, int G) {
+  static std::map<std::array<int, 4>, PassCodes> cache;
+  const std::array<int, 4> key{kind, BH, n_tiles, G};
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  PassCodes pc;
+  pc.n = 0;
+  const long long items = kind == 0 ? static_cast<long long>(BH) * ((n_tiles + 1) / 2)
+                                    : static_cast<long long>(BH) * n_tiles;
+  if (kind != 0 || G < 2 || (items + G - 1) / G > kMaxPassCodes) {  // every pass alternates
+    cache.emplace(key, pc);
+    return pc;
+  }
+  const int n_pairs = (n_tiles + 1) / 2;
+  std::vector<int> cost(static_cast<size_t>(BH) * n_pairs);
+  for (size_t u = 0; u < cost.size(); ++u) {
+    const int c = n_pairs - 1 - static_cast<int>(u / BH);
+    const int nlo = 2 * c + 1, nhi = 2 * c + 1 < n_tiles ? 2 * c + 2 : 0;
+    cost[u] = nlo + nhi;
+  }
+  plan_passes(cost, G, &pc);
+  cache.emplace(key, pc);
+  return pc;
+}
 
 // Launch `kernel` on stream s; with `dependent`, behind the previous kernel
 // as a programmatic dependent: its CTAs may be scheduled while that kernel
@@ -354,6 +435,7 @@ cattn_status fwd_impl(int dev, const void* q, cattn_layout lq, const void* k, ca
   const long long n_items = static_cast<long long>(BH) * ((p.n_qtiles + 1) / 2);
   if (n_items > 0x7fffffffLL) return CATTN_ERR_INVALID_ARG;
   dim3 grid(static_cast<unsigned>(n_items < g_sm_count[dev] ? n_items : g_sm_count[dev]));
+  p.passes = pass_plan(0, BH, p.n_qtiles, static_cast<int>(grid.x));
   cudaError_t e;
   {
     LaunchTimer t(K_FWD, s);
@@ -1024,6 +1106,13 @@ const char* cattn_status_string(cattn_status s) {
 }
 
 int cattn_version(void) { return 100; }
+
+int cattn_plan_passes(int kind, int BH, int n_tiles, int G, uint16_t* codes, int max_codes) {
+  if ((kind != 0 && kind != 1) || BH < 1 || n_tiles < 1 || G < 1) return -1;
+  const PassCodes pc = pass_plan(kind, BH, n_tiles, G);
+  for (int k = 0; k < pc.n && k < max_codes; ++k) codes[k] = pc.code[k];
+  return pc.n;
+}
 
 int cattn_last_cuda_error(void) { return g_last_cuda_error; }
 

@@ -67,6 +67,7 @@
 #pragma once
 
 #include "philox.cuh"
+#include "sched.cuh"
 #include "sm100.cuh"
 
 namespace cattn {
@@ -83,6 +84,7 @@ struct FwdParams {
   float scale_log2;    // scale * log2(e)
   uint64_t timeout_ns;
   DropParams drop;     // attention dropout (kernels instantiated with DROP only)
+  PassCodes passes;    // how the work items are dealt to the CTAs (sched.cuh)
 };
 
 template <int D, bool PLO, bool DROP = false>
@@ -104,7 +106,8 @@ struct FwdCfg {
   static constexpr int OFF_BAR = OFF_V + STAGES * TILE_BYTES;
   static constexpr int NUM_BARS = 47;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM_USED = OFF_MISC + 64;
+  static constexpr int OFF_PASS = OFF_MISC + 64;  // the pass codes (sched.cuh)
+  static constexpr int SMEM_USED = OFF_PASS + kPassSmemBytes;
   // at least 116 KB so that one CTA holds an SM (it takes all 512 TMEM columns)
   static constexpr int SMEM_WANT = SMEM_USED + 1024 < 116 * 1024 ? 116 * 1024 : SMEM_USED + 1024;
   static constexpr int SMEM_BYTES = SMEM_WANT <= kMaxDynSmem ? SMEM_WANT : SMEM_USED;
@@ -243,12 +246,12 @@ __device__ __forceinline__ void fwd_exp_row(const float (&s)[128], uint64_t sl2x
 // Work items: pairs (c, bh) of query tiles 2c, 2c+1 of head bh, numbered
 // longest first (u = 0 .. BH*n_pairs-1: c = n_pairs-1 - u / BH, bh = u % BH).
 // The grid is persistent (at most one CTA per SM); CTA b takes items in
-// passes over the grid, alternating direction, so that every CTA gets a
-// similar mix of long and short items: pass k takes item k*G + b (k even)
-// or k*G + G-1-b (k odd).  Returns -1 past the last item.
-__device__ __forceinline__ int fwd_item(int k, int b, int G, int n_items) {
-  const int u = k * G + ((k & 1) ? G - 1 - b : b);
-  return u < n_items ? u : -1;
+// passes over the grid, one item per pass, dealt by the call's pass codes
+// (sched.cuh) so that every CTA gets a similar total.  Returns -1 past the
+// last item.
+__device__ __forceinline__ int fwd_item(int k, int b, int G, int n_items, int n_codes,
+                                         const uint16_t* codes_s) {
+  return pass_item_smem(k, b, G, n_items, n_codes, codes_s);
 }
 
 // An item's two query tiles go to the two softmax groups, the longer one
@@ -333,6 +336,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     tmem_alloc(sbase + C::OFF_MISC, C::TMEM_COLS);
     tmem_relinquish();
   }
+  uint16_t* const pass_s = reinterpret_cast<uint16_t*>(smem + C::OFF_PASS);
+  pass_codes_to_smem(p.passes, pass_s);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -363,7 +368,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           tma_load_4d(dst, m, mbar, x, y, bh % p.H, bh / p.H);
       };
       for (int k = 0;; ++k) {
-        const int u = fwd_item(k, b, G, n_items);
+        const int u = fwd_item(k, b, G, n_items, p.passes.n, pass_s);
         if (u < 0 || *abort_flag) break;
         const FwdItem it = fwd_item_info(u, k, p.BH, n_pairs, p.n_qtiles);
         for (int g = 0; g < 2; ++g) {
@@ -457,7 +462,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         mma_commit(bar(FB_ODONE + g));
       };
       for (int k = 0;; ++k) {
-        const int u = fwd_item(k, b, G, n_items);
+        const int u = fwd_item(k, b, G, n_items, p.passes.n, pass_s);
         if (u < 0) break;
         const FwdItem it = fwd_item_info(u, k, p.BH, n_pairs, p.n_qtiles);
         const int ng = it.n[g];
@@ -529,14 +534,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     // groups have a tile in the first item.  Waiting before the loop keeps
     // the wait out of the loop body.
     {
-      const int u0 = fwd_item(0, b, G, n_items);
+      const int u0 = fwd_item(0, b, G, n_items, p.passes.n, pass_s);
       if (u0 >= 0 && g == 1) {
         const FwdItem it0 = fwd_item_info(u0, 0, p.BH, n_pairs, p.n_qtiles);
         if (it0.n[0] > 0 && it0.n[1] > 0) wait_warp(w, bar(FB_OFFSET), 0, 11);
       }
     }
     for (int k = 0;; ++k) {
-      const int u = fwd_item(k, b, G, n_items);
+      const int u = fwd_item(k, b, G, n_items, p.passes.n, pass_s);
       if (u < 0) break;
       const FwdItem it = fwd_item_info(u, k, p.BH, n_pairs, p.n_qtiles);
       const int ng = it.n[g];

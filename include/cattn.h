@@ -420,6 +420,24 @@ CATTN_API int cattn_last_cuda_error(void);
 /* Library version, major*10000 + minor*100 + patch. */
 CATTN_API int cattn_version(void);
 
+/* How the persistent forward (kind 0) or backward (kind 1) grid of G CTAs
+ * deals its work items for B*H = BH heads of n_tiles 128-row tiles
+ * (diagnostic; host only, no device access).  The items are numbered
+ * longest first: the forward's item u is the query-tile pair
+ * c = n_pairs - 1 - u / BH (n_pairs = (n_tiles + 1) / 2), the backward's the
+ * key tile u / BH, both of head u % BH.  CTA b takes one item per pass;
+ * pass k deals items k*G .. k*G + G-1.  For k < the returned count,
+ * codes[k] gives the pass's direction (bit 15) and rotation r (bits 0..14):
+ * item k*G + j goes to CTA (r + j) mod G, or (r - j) mod G with the
+ * direction bit set.  Later passes alternate: item k*G + b (k even) or
+ * k*G + G-1-b (k odd) to CTA b.  The library plans the forward's codes
+ * once per shape so that the CTAs' loads (an item's key tiles) stay close
+ * to even; the backward's passes always alternate (count 0).  Writes at
+ * most max_codes codes; returns their count, or -1 for kind not 0 or 1,
+ * BH < 1, n_tiles < 1 or G < 1. */
+CATTN_API int cattn_plan_passes(int kind, int BH, int n_tiles, int G, uint16_t* codes,
+                                int max_codes);
+
 #ifdef __cplusplus
 }
 #endif
