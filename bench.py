@@ -76,7 +76,7 @@ def load_peaks():
 
 
 KERNEL_SOURCES = {
-    "fwd_kernel": ("fwd.cuh", "philox.cuh", "sm100.cuh"),
+    "fwd_kernel": ("fwd.cuh", "philox.cuh", "sched.cuh", "sm100.cuh"),
     "bwd_kernel": ("bwd.cuh", "philox.cuh", "sm100.cuh"),
     "bwd_pre_kernel": ("bwd.cuh", "philox.cuh", "sm100.cuh"),
     "dq_convert_kernel": ("bwd.cuh", "philox.cuh", "sm100.cuh"),
