@@ -123,6 +123,7 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 // (every pass alternates).
 void plan_passes(const std::vector<int>& cost, int G, PassCodes* pc) {
   pc->n = 0;
+  for (uint32_t& w : pc->code2) w = 0u;
   const long long n = static_cast<long long>(cost.size());
   if (G < 2 || n == 0) return;
   const long long passes = (n + G - 1) / G;
@@ -158,7 +159,8 @@ void plan_passes(const std::vector<int>& cost, int G, PassCodes* pc) {
       if (b < 0) b += G;
       load[b] += cost[first + j];
     }
-    pc->code[k] = static_cast<uint16_t>(best);
+    pc->code2[k >> 1] = (pc->code2[k >> 1] & (0xffffu << (16 * (1 - (k & 1))))) |
+                        (static_cast<uint32_t>(best) << (16 * (k & 1)));
   }
   pc->n = static_cast<int>(passes);
 }
@@ -167,16 +169,16 @@ void plan_passes(const std::vector<int>& cost, int G, PassCodes* pc) {
 // B*H, tiles, grid size): kind 0 deals the forward's items (query-tile
 // pairs, an item's load its two groups' key tiles).  The backward (kind 1)
 // keeps alternating passes: every variant of it that looked its items up
-// through pass codes measured slower (GPT-2 layer backward call 180-187
-// against 170 us), even with all passes alternating.
+// through pass codes (from the parameters or from shared memory) measured
+// slower (GPT-2 layer backward call 180-187 against 170 us), even with all
+// passes alternating.
 PassCodes pass_plan(int kind, int BH, int n_tiles, int G) {
   static std::map<std::array<int, 4>, PassCodes> cache;
   const std::array<int, 4> key{kind, BH, n_tiles, G};
   std::lock_guard<std::mutex> lk(g_mu);
   auto it = cache.find(key);
   if (it != cache.end()) return it->second;
-  PassCodes pc;
-  pc.n = 0;
+  PassCodes pc{};
   const long long items = kind == 0 ? static_cast<long long>(BH) * ((n_tiles + 1) / 2)
                                     : static_cast<long long>(BH) * n_tiles;
   if (kind != 0 || G < 2 || (items + G - 1) / G > kMaxPassCodes) {  // every pass alternates
@@ -1110,7 +1112,7 @@ int cattn_version(void) { return 100; }
 int cattn_plan_passes(int kind, int BH, int n_tiles, int G, uint16_t* codes, int max_codes) {
   if ((kind != 0 && kind != 1) || BH < 1 || n_tiles < 1 || G < 1) return -1;
   const PassCodes pc = pass_plan(kind, BH, n_tiles, G);
-  for (int k = 0; k < pc.n && k < max_codes; ++k) codes[k] = pc.code[k];
+  for (int k = 0; k < pc.n && k < max_codes; ++k) codes[k] = static_cast<uint16_t>(pass_code(pc, k));
   return pc.n;
 }
 

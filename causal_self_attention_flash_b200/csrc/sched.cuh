@@ -25,13 +25,17 @@ namespace cattn {
 constexpr int kMaxPassCodes = 64;
 
 struct PassCodes {
-  uint16_t code[kMaxPassCodes];
-  int n;  // passes with a code (0: all alternate)
+  uint32_t code2[kMaxPassCodes / 2];  // pass k's code in bits 16 (k & 1) .. + 15 of code2[k / 2]
+  int n;                              // passes with a code (0: all alternate)
 };
 
+__host__ __device__ inline uint32_t pass_code(const PassCodes& pc, int k) {
+  return (pc.code2[k >> 1] >> (16 * (k & 1))) & 0xffffu;
+}
+
 // The forward copies the codes into shared memory once (kPassSmemBytes at
-// a 4-byte aligned address, by the first kMaxPassCodes / 2 threads, before
-// its start-up barrier) and looks them up there.
+// a 4-byte aligned address, before its start-up barrier) and looks them up
+// there; the copy reads the kernel parameter at compile-time indices only.
 constexpr int kPassSmemBytes = 2 * kMaxPassCodes;
 
 // The item of pass k for CTA b, or -1 past the last item; `code` is pass
@@ -51,15 +55,18 @@ __host__ __device__ inline int pass_item_coded(int k, int b, int G, int n_items,
 }
 
 __host__ __device__ inline int pass_item(int k, int b, int G, int n_items, const PassCodes& pc) {
-  return pass_item_coded(k, b, G, n_items, pc.n, k < pc.n ? pc.code[k] : 0u);
+  return pass_item_coded(k, b, G, n_items, pc.n, k < pc.n ? pass_code(pc, k) : 0u);
 }
 
 #ifdef __CUDACC__
-// The copy into shared memory, and the lookup from there.
+// The copy into shared memory (thread 0, fully unrolled), and the lookup
+// from there.
 __device__ __forceinline__ void pass_codes_to_smem(const PassCodes& pc, uint16_t* codes_s) {
-  if (threadIdx.x < kMaxPassCodes / 2)
-    reinterpret_cast<uint32_t*>(codes_s)[threadIdx.x] =
-        reinterpret_cast<const uint32_t*>(pc.code)[threadIdx.x];
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int i = 0; i < kMaxPassCodes / 2; ++i)
+      reinterpret_cast<uint32_t*>(codes_s)[i] = pc.code2[i];
+  }
 }
 __device__ __forceinline__ int pass_item_smem(int k, int b, int G, int n_items, int n_codes,
                                               const uint16_t* codes_s) {
