@@ -71,8 +71,10 @@ struct PreParams {
 // CONTIG: O and dO are contiguous (B, H, T, D), addressed as rows of D.
 template <int D, bool CONTIG>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
-  grid_dep_wait();    // the previous kernel's O, dO, LSE
-  grid_dep_launch();  // the main kernel may take SMs as this grid drains
+  // the previous kernel's O, dO, LSE.  (The main kernel is not released
+  // early: its CTAs, resident while this grid drained, made the GPT-2
+  // layer's backward call 168.6 against 165.9 us.)
+  grid_dep_wait();
   constexpr int TPR = D / 8;
   constexpr int RPW = 32 / TPR;  // rows per warp per step
   const int lane = threadIdx.x & 31;

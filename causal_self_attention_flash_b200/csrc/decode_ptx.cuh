@@ -36,9 +36,10 @@ __device__ __forceinline__ void dec_cp_async16(void* dst, const void* src, bool 
                "l"(src), "r"(valid ? 16 : 0)
                : "memory");
 }
-// Programmatic dependent launch (as grid_dep_wait / grid_dep_launch of the
-// main kernels): wait for the grid launched before this one to complete
-// and its writes to be visible; let the next grid be scheduled.
+// Programmatic dependent launch (as grid_dep_wait of the main kernels):
+// wait for the grid launched before this one to complete and its writes to
+// be visible; let the next grid be scheduled once every CTA of this one
+// has executed dec_grid_dep_launch (or exited).
 __device__ __forceinline__ void dec_grid_dep_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }

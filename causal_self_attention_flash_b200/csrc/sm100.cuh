@@ -73,15 +73,10 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
 }
 
-// Programmatic dependent launch.  grid_dep_wait: wait until the grid this
-// one was launched behind has completed and its memory writes are visible
-// (returns at once for a launch without that dependency).
-// grid_dep_launch: the grid launched behind this one may be scheduled once
-// every CTA of this grid has executed it (or exited).
+// Programmatic dependent launch: wait until the grid this one was launched
+// behind has completed and its memory writes are visible (returns at once
+// for a launch without that dependency).
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void grid_dep_launch() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
 
 // Make barrier initialisation visible to the async proxy (TMA, tcgen05).
 __device__ __forceinline__ void fence_mbar_init() {
