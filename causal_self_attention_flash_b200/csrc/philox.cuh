@@ -39,7 +39,7 @@ constexpr int kPhiloxRounds = 10;
 struct DropParams {
   uint32_t t = 0;              // drop threshold round(p * 256); 0 = no dropout
   uint32_t t_lo = 0;           // (t & 0x7F) in every byte
-  uint32_t t_maj = 0;          // all ones when t < 128, else 0 (see keep_nibble)
+  uint32_t t_maj = 0;          // all ones when t < 128, else 0 (see keep_flags)
   uint32_t offset = 0;         // counter word 3
   // the key of every round: rk[2r] = seed low + r * W0, rk[2r + 1] =
   // seed high + r * W1 (mod 2^32), set on the host so that the rounds read
