@@ -201,10 +201,10 @@ PassCodes pass_plan(int kind, int BH, int n_tiles, int G) {
 // as a programmatic dependent: its CTAs may be scheduled while that kernel
 // drains.  Every kernel launched so starts with grid_dep_wait, before its
 // first access to global memory, so whatever kernel precedes it on the
-// stream has completed and its writes are visible.  (Without dropout: 55
-// against 60 us for the 64x6x256x64 backward, 172 against 173 us on the
-// GPT-2 layer; with dropout the GPT-2 layer's backward measured 218
-// against 211 us, so the dropout calls launch plainly.)
+// stream has completed and its writes are visible.  (55 against 60 us for
+// the 64x6x256x64 backward, 172 against 173 us on the GPT-2 layer; with
+// dropout, 206 against 212 us for the GPT-2 layer's backward and 59
+// against 67 us for the 64x6x256x64 one.)
 template <typename... KArgs, typename... Args>
 cudaError_t launch_dependent(bool dependent, void (*kernel)(KArgs...), dim3 grid, dim3 block,
                              size_t smem, cudaStream_t s, Args&&... args) {
@@ -441,7 +441,7 @@ cattn_status fwd_impl(int dev, const void* q, cattn_layout lq, const void* k, ca
   cudaError_t e;
   {
     LaunchTimer t(K_FWD, s);
-    e = launch_dependent(!DROP, fwd_kernel<D, PLO, DROP, FLAT>, grid, dim3(C::THREADS),
+    e = launch_dependent(true, fwd_kernel<D, PLO, DROP, FLAT>, grid, dim3(C::THREADS),
                          C::SMEM_BYTES, s, mq, mk, mv, p);
   }
   return e == cudaSuccess ? CATTN_OK : cuda_fail(e);
@@ -568,8 +568,7 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
     return st;
 
   st = pre_impl<D>(o, ly.o, o_lo, dout, ly.dout, lse, delta, lse2,
-                   reinterpret_cast<float4*>(dq_acc), n_dq / 4, B, H, T, L.T_pad, status, s,
-                   !DROP);
+                   reinterpret_cast<float4*>(dq_acc), n_dq / 4, B, H, T, L.T_pad, status, s);
   if (st != CATTN_OK) return st;
 
   BwdParams p;
@@ -600,7 +599,7 @@ cattn_status bwd_impl(int dev, const void* q, const void* k, const void* v, cons
   if (n_items > 0x7fffffffLL) return CATTN_ERR_INVALID_ARG;
   dim3 grid(static_cast<unsigned>(n_items < g_sm_count[dev] ? n_items : g_sm_count[dev]));
   cudaError_t e;
-  constexpr bool dep = !DROP;  // programmatic dependents (see launch_dependent)
+  constexpr bool dep = true;  // programmatic dependents (see launch_dependent)
   {
     LaunchTimer t(K_BWD_MAIN, s);
     e = launch_dependent(dep, bwd_kernel<D, SLO, DROP, FLAT>, grid, dim3(C::THREADS),

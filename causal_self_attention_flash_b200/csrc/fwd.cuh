@@ -290,8 +290,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   using C = FwdCfg<D, PLO, DROP>;
   static_assert(FB_OFFSET + 1 <= C::NUM_BARS, "barrier count");
   static_assert(C::STAGES <= kMaxStages, "barrier map");
-  // launched as a programmatic dependent of the previous kernel (without
-  // dropout): its writes (Q, K, V) are visible after this
+  // launched as a programmatic dependent of the previous kernel: its
+  // writes (Q, K, V) are visible after this
   grid_dep_wait();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = aligned_smem(smem_raw, C::SMEM_USED, nullptr);
